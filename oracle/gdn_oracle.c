@@ -1,0 +1,427 @@
+/*
+ * gdn_oracle.c -- plain fp64 CPU oracle for the gated delta rule.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path (the CUDA library
+ * and its Python binding) may include, link, load or call this file.  Only
+ * the tests, the smoke check and the CPU-baseline leg of the benchmark use
+ * it.  It shares no code, header, helper or constant with the CUDA path.
+ *
+ * What it computes (the sources are the web pages this project is built
+ * from):
+ *
+ *   "Architecture Thread I: Gated Attention, DeltaNet, and Hybrid Models",
+ *   section "Gated DeltaNet":  S_t = S_{t-1} (alpha_t (I - beta_t k_t k_t^T))
+ *   + beta_t v_t k_t^T, and the read-out o_t = S_t q_t used with the same
+ *   state orientation in the linear-attention recurrences of
+ *   "Gated Attention Architectures", section 1 (GLA) and section 3
+ *   (Gated DeltaNet, "Mathematical Formulation").
+ *
+ * Conventions (the readings of the pages this oracle takes):
+ *   - S is d_v x d_k (row = value index, key index fastest), o_t = S_t q_t.
+ *   - alpha_t = exp(g_t); g and beta are given per token per VALUE head.
+ *   - value head h reads query/key head h / (Hv / Hk) (contiguous groups).
+ *   - q and k are used exactly as given (no renormalisation, no scale).
+ *   - sequences are independent; each has its own initial / final state;
+ *     a NULL initial state means zeros.
+ *   - the output at t reads the state AFTER the update at t.
+ *
+ * Three independent formulations live here:
+ *   gdn_oracle_recurrent   -- the token recurrence (the oracle proper).
+ *   gdn_oracle_chunkwise   -- the chunked form with a per-chunk cumulative
+ *                             decay and the WY/UT triangular factor, derived
+ *                             from the recurrence ("Gated Attention
+ *                             Architectures", sections 2 and 3: the WY
+ *                             representation and the per-chunk cumulative
+ *                             decay products; the output follows the GLA
+ *                             chunkwise form of section 1 with a
+ *                             decay-aware causal mask).
+ *   gdn_oracle_delta_error_form -- DeltaNet written as the error-correcting
+ *                             write S <- S - beta (S k - v) k^T
+ *                             ("Architecture Thread I", the delta-rule
+ *                             update), with no gate.
+ *
+ * Layouts (all row-major, token-major, fp64):
+ *   q, k          [T_total, Hk, d_k]
+ *   v, o          [T_total, Hv, d_v]
+ *   g, beta       [T_total, Hv]
+ *   s0, s_final   [N, Hv, d_v, d_k]
+ *   cu_seqlens    int64 [N + 1]; sequence n holds tokens [cu[n], cu[n+1])
+ * A "unit" is one (sequence n, value head h) pair, numbered n * Hv + h.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct {
+    int64_t num_seqs;
+    const int64_t *cu_seqlens;
+    int32_t hk, hv, dk, dv;
+    const double *q, *k, *v, *g, *beta;
+    const double *s0;   /* may be NULL: zero initial state */
+    double *o;          /* may be NULL: outputs not wanted */
+    double *s_final;    /* may be NULL */
+} gdn_oracle_problem;
+
+/* Optional per-chunk intermediates of the chunkwise form, indexed by the
+ * global chunk number (sequences in order, chunks in order inside each
+ * sequence; a tail chunk keeps its C-row slot with the unused rows left
+ * untouched).  Any pointer may be NULL.
+ *   gcum  [chunks, Hv, C]          cumulative log-decay G inside the chunk
+ *   tmat  [chunks, Hv, C, C]       T = (I + A)^-1
+ *   w     [chunks, Hv, C, d_k]     W = T diag(beta * gamma) K
+ *   ut    [chunks, Hv, C, d_v]     U~ = T diag(beta) V
+ *   u     [chunks, Hv, C, d_v]     U = U~ - W S0^T
+ *   sc    [chunks, Hv, d_v, d_k]   state at the start of the chunk      */
+typedef struct {
+    int32_t chunk;
+    double *gcum, *tmat, *w, *ut, *u, *sc;
+} gdn_oracle_chunk_out;
+
+static int64_t seq_len_of(const gdn_oracle_problem *p, int64_t n) {
+    return p->cu_seqlens[n + 1] - p->cu_seqlens[n];
+}
+
+/* ------------------------------------------------------------------ */
+/* 1. Token recurrence.                                                 */
+/* ------------------------------------------------------------------ */
+static void recurrent_unit(const gdn_oracle_problem *p, int64_t unit, double *S, double *pk) {
+    const int64_t n = unit / p->hv;
+    const int h = (int)(unit % p->hv);
+    const int hq = h / (p->hv / p->hk);
+    const int dk = p->dk, dv = p->dv;
+
+    if (p->s0) memcpy(S, p->s0 + unit * (int64_t)dv * dk, sizeof(double) * dv * dk);
+    else memset(S, 0, sizeof(double) * dv * dk);
+
+    for (int64_t t = p->cu_seqlens[n]; t < p->cu_seqlens[n + 1]; ++t) {
+        const double *kt = p->k + (t * p->hk + hq) * dk;
+        const double *qt = p->q + (t * p->hk + hq) * dk;
+        const double *vt = p->v + (t * p->hv + h) * dv;
+        const double alpha = exp(p->g[t * p->hv + h]);
+        const double beta = p->beta[t * p->hv + h];
+
+        /* prediction of the old memory for key k_t: S_{t-1} k_t */
+        for (int i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) acc += S[i * dk + j] * kt[j];
+            pk[i] = acc;
+        }
+        /* S_t = alpha S_{t-1} (I - beta k k^T) + beta v k^T
+         *     = alpha S_{t-1} + beta (v - alpha S_{t-1} k) k^T            */
+        for (int i = 0; i < dv; ++i) {
+            const double ui = beta * (vt[i] - alpha * pk[i]);
+            for (int j = 0; j < dk; ++j) S[i * dk + j] = alpha * S[i * dk + j] + ui * kt[j];
+        }
+        /* o_t = S_t q_t */
+        if (p->o) {
+            double *ot = p->o + (t * p->hv + h) * dv;
+            for (int i = 0; i < dv; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < dk; ++j) acc += S[i * dk + j] * qt[j];
+                ot[i] = acc;
+            }
+        }
+    }
+    if (p->s_final) memcpy(p->s_final + unit * (int64_t)dv * dk, S, sizeof(double) * dv * dk);
+}
+
+/* ------------------------------------------------------------------ */
+/* 2. DeltaNet in its error-correcting form (no decay gate).            */
+/* ------------------------------------------------------------------ */
+static void delta_error_unit(const gdn_oracle_problem *p, int64_t unit, double *S, double *err) {
+    const int64_t n = unit / p->hv;
+    const int h = (int)(unit % p->hv);
+    const int hq = h / (p->hv / p->hk);
+    const int dk = p->dk, dv = p->dv;
+
+    if (p->s0) memcpy(S, p->s0 + unit * (int64_t)dv * dk, sizeof(double) * dv * dk);
+    else memset(S, 0, sizeof(double) * dv * dk);
+
+    for (int64_t t = p->cu_seqlens[n]; t < p->cu_seqlens[n + 1]; ++t) {
+        const double *kt = p->k + (t * p->hk + hq) * dk;
+        const double *qt = p->q + (t * p->hk + hq) * dk;
+        const double *vt = p->v + (t * p->hv + h) * dv;
+        const double beta = p->beta[t * p->hv + h];
+        /* error = S k - v */
+        for (int i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) acc += S[i * dk + j] * kt[j];
+            err[i] = acc - vt[i];
+        }
+        /* S <- S - beta * error * k^T */
+        for (int i = 0; i < dv; ++i)
+            for (int j = 0; j < dk; ++j) S[i * dk + j] -= beta * err[i] * kt[j];
+        if (p->o) {
+            double *ot = p->o + (t * p->hv + h) * dv;
+            for (int i = 0; i < dv; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < dk; ++j) acc += S[i * dk + j] * qt[j];
+                ot[i] = acc;
+            }
+        }
+    }
+    if (p->s_final) memcpy(p->s_final + unit * (int64_t)dv * dk, S, sizeof(double) * dv * dk);
+}
+
+/* ------------------------------------------------------------------ */
+/* 3. Chunkwise form.                                                   */
+/*                                                                      */
+/* Inside a chunk of L <= C tokens r = 0..L-1 with start state S0:      */
+/*   G_r   = g_0 + ... + g_r          (cumulative log-decay)             */
+/*   gamma_r = exp(G_r),  Gamma_rj = exp(G_r - G_j) for j <= r          */
+/*   unrolling S_r = alpha_r S_{r-1} + u_r k_r^T with                   */
+/*   u_r = beta_r (v_r - alpha_r S_{r-1} k_r) gives                     */
+/*   (I + A) U = diag(beta) V - diag(beta gamma) K S0^T,                */
+/*   A_rj = beta_r Gamma_rj (k_r . k_j) for j < r (strictly lower), so  */
+/*   U = T diag(beta) V - T diag(beta gamma) K S0^T = U~ - W S0^T,       */
+/*   T = (I + A)^-1;  then                                              */
+/*   O = diag(gamma) Q S0^T + (Q K^T (.) Gamma) U                        */
+/*   S_L = gamma_{L-1} S0 + U^T diag(exp(G_{L-1} - G)) K.                */
+/* ------------------------------------------------------------------ */
+typedef struct {
+    double *S, *G, *A, *T, *W, *Ut, *U, *Kc, *Qc, *Vc;
+} chunk_scratch;
+
+static void chunkwise_unit(const gdn_oracle_problem *p, const gdn_oracle_chunk_out *co,
+                           int64_t unit, chunk_scratch *sc, int64_t chunk_base) {
+    const int64_t n = unit / p->hv;
+    const int h = (int)(unit % p->hv);
+    const int hq = h / (p->hv / p->hk);
+    const int dk = p->dk, dv = p->dv, C = co->chunk;
+    double *S = sc->S, *G = sc->G, *A = sc->A, *T = sc->T, *W = sc->W, *Ut = sc->Ut, *U = sc->U;
+    double *K = sc->Kc, *Q = sc->Qc, *V = sc->Vc;
+
+    if (p->s0) memcpy(S, p->s0 + unit * (int64_t)dv * dk, sizeof(double) * dv * dk);
+    else memset(S, 0, sizeof(double) * dv * dk);
+
+    const int64_t t_begin = p->cu_seqlens[n], t_end = p->cu_seqlens[n + 1];
+    int64_t chunk_idx = chunk_base;
+    for (int64_t c0 = t_begin; c0 < t_end; c0 += C, ++chunk_idx) {
+        const int L = (int)((t_end - c0) < C ? (t_end - c0) : C);
+        const int64_t slot = chunk_idx * p->hv + h;
+        if (co->sc) memcpy(co->sc + slot * (int64_t)dv * dk, S, sizeof(double) * dv * dk);
+
+        /* gather this chunk's rows */
+        for (int r = 0; r < L; ++r) {
+            const int64_t t = c0 + r;
+            memcpy(K + r * dk, p->k + (t * p->hk + hq) * dk, sizeof(double) * dk);
+            memcpy(Q + r * dk, p->q + (t * p->hk + hq) * dk, sizeof(double) * dk);
+            memcpy(V + r * dv, p->v + (t * p->hv + h) * dv, sizeof(double) * dv);
+        }
+        /* cumulative log-decay */
+        double run = 0.0;
+        for (int r = 0; r < L; ++r) {
+            run += p->g[(c0 + r) * p->hv + h];
+            G[r] = run;
+        }
+        /* A (strictly lower) */
+        for (int r = 0; r < L; ++r)
+            for (int j = 0; j < L; ++j) {
+                double a = 0.0;
+                if (j < r) {
+                    double kk = 0.0;
+                    for (int x = 0; x < dk; ++x) kk += K[r * dk + x] * K[j * dk + x];
+                    a = p->beta[(c0 + r) * p->hv + h] * exp(G[r] - G[j]) * kk;
+                }
+                A[r * L + j] = a;
+            }
+        /* T = (I + A)^-1 by forward substitution: row r of (I + A) T = I
+         * gives T_r = e_r - sum_{j<r} A_rj T_j.                          */
+        for (int r = 0; r < L; ++r)
+            for (int c = 0; c < L; ++c) {
+                double x = (r == c) ? 1.0 : 0.0;
+                for (int j = 0; j < r; ++j) x -= A[r * L + j] * T[j * L + c];
+                T[r * L + c] = x;
+            }
+        /* W = T diag(beta gamma) K ;  U~ = T diag(beta) V */
+        for (int r = 0; r < L; ++r) {
+            for (int x = 0; x < dk; ++x) {
+                double acc = 0.0;
+                for (int j = 0; j < L; ++j)
+                    acc += T[r * L + j] * p->beta[(c0 + j) * p->hv + h] * exp(G[j]) * K[j * dk + x];
+                W[r * dk + x] = acc;
+            }
+            for (int i = 0; i < dv; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < L; ++j)
+                    acc += T[r * L + j] * p->beta[(c0 + j) * p->hv + h] * V[j * dv + i];
+                Ut[r * dv + i] = acc;
+            }
+        }
+        /* U = U~ - W S0^T */
+        for (int r = 0; r < L; ++r)
+            for (int i = 0; i < dv; ++i) {
+                double acc = 0.0;
+                for (int x = 0; x < dk; ++x) acc += W[r * dk + x] * S[i * dk + x];
+                U[r * dv + i] = Ut[r * dv + i] - acc;
+            }
+        /* O = diag(gamma) Q S0^T + (Q K^T (.) Gamma) U */
+        if (p->o) {
+            for (int r = 0; r < L; ++r) {
+                double *ot = p->o + ((c0 + r) * p->hv + h) * dv;
+                for (int i = 0; i < dv; ++i) {
+                    double inter = 0.0;
+                    for (int x = 0; x < dk; ++x) inter += Q[r * dk + x] * S[i * dk + x];
+                    double intra = 0.0;
+                    for (int j = 0; j <= r; ++j) {
+                        double qk = 0.0;
+                        for (int x = 0; x < dk; ++x) qk += Q[r * dk + x] * K[j * dk + x];
+                        intra += qk * exp(G[r] - G[j]) * U[j * dv + i];
+                    }
+                    ot[i] = exp(G[r]) * inter + intra;
+                }
+            }
+        }
+        /* S_L = gamma_{L-1} S0 + U^T diag(exp(G_{L-1} - G)) K */
+        const double gl = G[L - 1];
+        for (int i = 0; i < dv; ++i)
+            for (int x = 0; x < dk; ++x) {
+                double acc = 0.0;
+                for (int j = 0; j < L; ++j) acc += U[j * dv + i] * exp(gl - G[j]) * K[j * dk + x];
+                S[i * dk + x] = exp(gl) * S[i * dk + x] + acc;
+            }
+
+        if (co->gcum) memcpy(co->gcum + slot * C, G, sizeof(double) * L);
+        if (co->tmat)
+            for (int r = 0; r < L; ++r) memcpy(co->tmat + (slot * C + r) * C, T + r * L, sizeof(double) * L);
+        if (co->w) memcpy(co->w + slot * (int64_t)C * dk, W, sizeof(double) * L * dk);
+        if (co->ut) memcpy(co->ut + slot * (int64_t)C * dv, Ut, sizeof(double) * L * dv);
+        if (co->u) memcpy(co->u + slot * (int64_t)C * dv, U, sizeof(double) * L * dv);
+    }
+    if (p->s_final) memcpy(p->s_final + unit * (int64_t)dv * dk, S, sizeof(double) * dv * dk);
+}
+
+/* ------------------------------------------------------------------ */
+/* Threading: units are independent, so threads take units round-robin. */
+/* ------------------------------------------------------------------ */
+enum { KIND_RECURRENT = 0, KIND_DELTA = 1, KIND_CHUNK = 2 };
+
+typedef struct {
+    int kind;
+    const gdn_oracle_problem *p;
+    const gdn_oracle_chunk_out *co;
+    const int64_t *units;  /* NULL = all */
+    int64_t n_units;
+    const int64_t *chunk_base; /* per sequence, for KIND_CHUNK */
+    int tid, nthreads;
+    int failed;
+} worker_arg;
+
+static void *worker(void *vp) {
+    worker_arg *a = (worker_arg *)vp;
+    const gdn_oracle_problem *p = a->p;
+    const int dk = p->dk, dv = p->dv;
+    const int C = a->co ? a->co->chunk : 1;
+    const int dm = dk > dv ? dk : dv;
+    double *S = malloc(sizeof(double) * dv * dk);
+    double *buf = malloc(sizeof(double) * (size_t)(dm + 8));
+    chunk_scratch sc = {0};
+    if (a->kind == KIND_CHUNK) {
+        sc.S = S;
+        sc.G = malloc(sizeof(double) * C);
+        sc.A = malloc(sizeof(double) * C * C);
+        sc.T = malloc(sizeof(double) * C * C);
+        sc.W = malloc(sizeof(double) * C * dk);
+        sc.Ut = malloc(sizeof(double) * C * dv);
+        sc.U = malloc(sizeof(double) * C * dv);
+        sc.Kc = malloc(sizeof(double) * C * dk);
+        sc.Qc = malloc(sizeof(double) * C * dk);
+        sc.Vc = malloc(sizeof(double) * C * dv);
+        if (!sc.G || !sc.A || !sc.T || !sc.W || !sc.Ut || !sc.U || !sc.Kc || !sc.Qc || !sc.Vc) a->failed = 1;
+    }
+    if (!S || !buf) a->failed = 1;
+    if (!a->failed) {
+        for (int64_t i = a->tid; i < a->n_units; i += a->nthreads) {
+            const int64_t unit = a->units ? a->units[i] : i;
+            if (a->kind == KIND_RECURRENT) recurrent_unit(p, unit, S, buf);
+            else if (a->kind == KIND_DELTA) delta_error_unit(p, unit, S, buf);
+            else chunkwise_unit(p, a->co, unit, &sc, a->chunk_base[unit / p->hv]);
+        }
+    }
+    free(S);
+    free(buf);
+    if (a->kind == KIND_CHUNK) {
+        free(sc.G); free(sc.A); free(sc.T); free(sc.W); free(sc.Ut); free(sc.U);
+        free(sc.Kc); free(sc.Qc); free(sc.Vc);
+    }
+    return NULL;
+}
+
+static int validate(const gdn_oracle_problem *p) {
+    if (!p || !p->cu_seqlens || p->num_seqs < 0) return -1;
+    if (p->hk <= 0 || p->hv <= 0 || p->dk <= 0 || p->dv <= 0) return -1;
+    if (p->hv % p->hk != 0) return -1;
+    if (!p->q || !p->k || !p->v || !p->g || !p->beta) return -1;
+    if (p->cu_seqlens[0] != 0) return -1;
+    for (int64_t n = 0; n < p->num_seqs; ++n)
+        if (seq_len_of(p, n) < 0) return -1;
+    return 0;
+}
+
+static int run(int kind, const gdn_oracle_problem *p, const gdn_oracle_chunk_out *co,
+               const int64_t *units, int64_t n_units, int n_threads) {
+    if (validate(p) != 0) return -1;
+    const int64_t total_units = p->num_seqs * p->hv;
+    if (!units) n_units = total_units;
+    for (int64_t i = 0; units && i < n_units; ++i)
+        if (units[i] < 0 || units[i] >= total_units) return -1;
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > 256) n_threads = 256;
+    if (n_threads > n_units && n_units > 0) n_threads = (int)n_units;
+
+    int64_t *chunk_base = NULL;
+    if (kind == KIND_CHUNK) {
+        if (!co || co->chunk <= 0) return -1;
+        chunk_base = malloc(sizeof(int64_t) * (size_t)(p->num_seqs + 1));
+        if (!chunk_base) return -1;
+        int64_t acc = 0;
+        for (int64_t n = 0; n < p->num_seqs; ++n) {
+            chunk_base[n] = acc;
+            acc += (seq_len_of(p, n) + co->chunk - 1) / co->chunk;
+        }
+        chunk_base[p->num_seqs] = acc;
+    }
+
+    pthread_t th[256];
+    worker_arg args[256];
+    int failed = 0;
+    for (int i = 0; i < n_threads; ++i) {
+        args[i] = (worker_arg){kind, p, co, units, n_units, chunk_base, i, n_threads, 0};
+        if (pthread_create(&th[i], NULL, worker, &args[i]) != 0) {
+            args[i].failed = 1;
+            worker(&args[i]); /* run inline: correctness over speed */
+            args[i].failed = 0;
+            th[i] = 0;
+        }
+    }
+    for (int i = 0; i < n_threads; ++i) {
+        if (th[i]) pthread_join(th[i], NULL);
+        failed |= args[i].failed;
+    }
+    free(chunk_base);
+    return failed ? -2 : 0;
+}
+
+/* Public entry points (called through ctypes by the tests). */
+int gdn_oracle_recurrent(const gdn_oracle_problem *p, const int64_t *units, int64_t n_units, int n_threads) {
+    return run(KIND_RECURRENT, p, NULL, units, n_units, n_threads);
+}
+
+int gdn_oracle_delta_error_form(const gdn_oracle_problem *p, const int64_t *units, int64_t n_units,
+                                int n_threads) {
+    return run(KIND_DELTA, p, NULL, units, n_units, n_threads);
+}
+
+int gdn_oracle_chunkwise(const gdn_oracle_problem *p, const gdn_oracle_chunk_out *co, const int64_t *units,
+                         int64_t n_units, int n_threads) {
+    return run(KIND_CHUNK, p, co, units, n_units, n_threads);
+}
+
+/* Number of chunks the chunkwise form uses (size of its intermediates). */
+int64_t gdn_oracle_num_chunks(const int64_t *cu_seqlens, int64_t num_seqs, int32_t chunk) {
+    int64_t acc = 0;
+    for (int64_t n = 0; n < num_seqs; ++n) acc += (cu_seqlens[n + 1] - cu_seqlens[n] + chunk - 1) / chunk;
+    return acc;
+}

@@ -1,0 +1,231 @@
+"""ctypes front end of the fp64 CPU oracle for the gated delta rule.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module; the product path
+(``linear_attention_sequence_sm_b200``) never does.  The arithmetic lives in
+``gdn_oracle.c``; this file only builds that file with gcc, marshals numpy
+arrays, and hands back numpy arrays.
+
+Readings of the pages (see ``gdn_oracle.c`` for the formulas):
+state S is d_v x d_k, o_t = S_t q_t after the update at t, alpha = exp(g),
+g and beta per token per value head, value head h reads q/k head
+h // (Hv // Hk), NULL initial state = zeros.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libgdn_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:
+    """Compile the oracle (plain C11, fp64, no fast-math) into a shared library."""
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
+        return out
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", "-fno-fast-math",
+           "-ffp-contract=off", "-o", out, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+class _Problem(ctypes.Structure):
+    _fields_ = [
+        ("num_seqs", ctypes.c_int64),
+        ("cu_seqlens", ctypes.POINTER(ctypes.c_int64)),
+        ("hk", ctypes.c_int32), ("hv", ctypes.c_int32),
+        ("dk", ctypes.c_int32), ("dv", ctypes.c_int32),
+        ("q", ctypes.POINTER(ctypes.c_double)), ("k", ctypes.POINTER(ctypes.c_double)),
+        ("v", ctypes.POINTER(ctypes.c_double)), ("g", ctypes.POINTER(ctypes.c_double)),
+        ("beta", ctypes.POINTER(ctypes.c_double)),
+        ("s0", ctypes.POINTER(ctypes.c_double)),
+        ("o", ctypes.POINTER(ctypes.c_double)),
+        ("s_final", ctypes.POINTER(ctypes.c_double)),
+    ]
+
+
+class _ChunkOut(ctypes.Structure):
+    _fields_ = [
+        ("chunk", ctypes.c_int32),
+        ("gcum", ctypes.POINTER(ctypes.c_double)), ("tmat", ctypes.POINTER(ctypes.c_double)),
+        ("w", ctypes.POINTER(ctypes.c_double)), ("ut", ctypes.POINTER(ctypes.c_double)),
+        ("u", ctypes.POINTER(ctypes.c_double)), ("sc", ctypes.POINTER(ctypes.c_double)),
+    ]
+
+
+def load(path: str | None = None):
+    """Load (building first if needed) the oracle library; cached per process."""
+    global _lib
+    with _lock:
+        if path is not None:
+            lib = ctypes.CDLL(path)
+        else:
+            if _lib is not None:
+                return _lib
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.POINTER(_Problem)
+        U = ctypes.POINTER(ctypes.c_int64)
+        for name in ("gdn_oracle_recurrent", "gdn_oracle_delta_error_form"):
+            fn = getattr(lib, name)
+            fn.argtypes = [P, U, ctypes.c_int64, ctypes.c_int]
+            fn.restype = ctypes.c_int
+        lib.gdn_oracle_chunkwise.argtypes = [P, ctypes.POINTER(_ChunkOut), U, ctypes.c_int64, ctypes.c_int]
+        lib.gdn_oracle_chunkwise.restype = ctypes.c_int
+        lib.gdn_oracle_num_chunks.argtypes = [U, ctypes.c_int64, ctypes.c_int32]
+        lib.gdn_oracle_num_chunks.restype = ctypes.c_int64
+        if path is None:
+            _lib = lib
+        return lib
+
+
+def _dptr(a):
+    if a is None:
+        return ctypes.POINTER(ctypes.c_double)()
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _f64(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count() or 1)
+
+
+def _prepare(q, k, v, g, beta, initial_state, cu_seqlens):
+    """Accept [B,T,H,d] batched or [T_total,H,d] packed (with cu_seqlens)."""
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    if cu_seqlens is None:
+        if q.ndim != 4:
+            raise ValueError("batched inputs must be [B, T, H, d]")
+        B, T = q.shape[:2]
+        cu = np.arange(B + 1, dtype=np.int64) * T
+        q, k, v = (x.reshape(B * T, x.shape[2], x.shape[3]) for x in (q, k, v))
+        g, beta = (x.reshape(B * T, x.shape[2]) for x in (g, beta))
+        batched = (B, T)
+    else:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+        if q.ndim == 4:
+            if q.shape[0] != 1:
+                raise ValueError("packed inputs need batch 1")
+            q, k, v = (x[0] for x in (q, k, v))
+            g, beta = (x[0] for x in (g, beta))
+            q, k, v, g, beta = (np.ascontiguousarray(x) for x in (q, k, v, g, beta))
+            batched = (1, q.shape[0])
+        else:
+            batched = None
+    N = cu.shape[0] - 1
+    Ttot, hk, dk = q.shape
+    hv, dv = v.shape[1], v.shape[2]
+    if k.shape != q.shape or v.shape[0] != Ttot or g.shape != (Ttot, hv) or beta.shape != (Ttot, hv):
+        raise ValueError("shape mismatch")
+    if int(cu[-1]) != Ttot:
+        raise ValueError("cu_seqlens[-1] must equal the token count")
+    s0 = None if initial_state is None else _f64(initial_state).reshape(N, hv, dv, dk)
+    return q, k, v, g, beta, s0, cu, batched, (N, Ttot, hk, hv, dk, dv)
+
+
+def _problem(q, k, v, g, beta, s0, cu, o, sf, dims):
+    N, Ttot, hk, hv, dk, dv = dims
+    return _Problem(N, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), hk, hv, dk, dv,
+                    _dptr(q), _dptr(k), _dptr(v), _dptr(g), _dptr(beta), _dptr(s0), _dptr(o), _dptr(sf))
+
+
+def _units_arg(units):
+    if units is None:
+        return None, ctypes.POINTER(ctypes.c_int64)(), 0
+    u = np.ascontiguousarray(np.asarray(units, dtype=np.int64))
+    return u, u.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), u.shape[0]
+
+
+def _finish(o, sf, batched, dims):
+    N, Ttot, hk, hv, dk, dv = dims
+    if batched is not None:
+        B, T = batched
+        o = o.reshape(B, T, hv, dv)
+    return o, sf
+
+
+def recurrent(q, k, v, g, beta, initial_state=None, cu_seqlens=None, units=None, threads=None, lib=None):
+    """Token recurrence (the oracle proper).  Returns (o, final_state) in fp64.
+
+    ``units`` restricts the work to the listed (sequence * Hv + head) pairs;
+    entries of other units are left as NaN so a caller cannot mistake them
+    for computed values.
+    """
+    q, k, v, g, beta, s0, cu, batched, dims = _prepare(q, k, v, g, beta, initial_state, cu_seqlens)
+    N, Ttot, hk, hv, dk, dv = dims
+    o = np.full((Ttot, hv, dv), np.nan)
+    sf = np.full((N, hv, dv, dk), np.nan)
+    prob = _problem(q, k, v, g, beta, s0, cu, o, sf, dims)
+    keep, uptr, nu = _units_arg(units)
+    rc = (lib or load()).gdn_oracle_recurrent(ctypes.byref(prob), uptr, nu, threads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"oracle recurrent failed ({rc})")
+    return _finish(o, sf, batched, dims)
+
+
+def delta_error_form(q, k, v, beta, initial_state=None, cu_seqlens=None, threads=None, lib=None):
+    """DeltaNet as S <- S - beta (S k - v) k^T, o = S q (no decay gate)."""
+    q = _f64(q)
+    g = np.zeros(q.shape[:-2] + (np.asarray(v).shape[-2],))
+    q, k, v, g, beta, s0, cu, batched, dims = _prepare(q, k, v, g, beta, initial_state, cu_seqlens)
+    N, Ttot, hk, hv, dk, dv = dims
+    o = np.full((Ttot, hv, dv), np.nan)
+    sf = np.full((N, hv, dv, dk), np.nan)
+    prob = _problem(q, k, v, g, beta, s0, cu, o, sf, dims)
+    rc = (lib or load()).gdn_oracle_delta_error_form(ctypes.byref(prob), None, 0, threads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"oracle delta form failed ({rc})")
+    return _finish(o, sf, batched, dims)
+
+
+def chunkwise(q, k, v, g, beta, chunk, initial_state=None, cu_seqlens=None, intermediates=False,
+              units=None, threads=None, lib=None):
+    """Chunkwise (WY/UT) form in fp64.  Returns (o, final_state[, inter]).
+
+    ``inter`` holds per-chunk arrays indexed [chunk, Hv, ...] (see the C file).
+    """
+    q, k, v, g, beta, s0, cu, batched, dims = _prepare(q, k, v, g, beta, initial_state, cu_seqlens)
+    N, Ttot, hk, hv, dk, dv = dims
+    lib = lib or load()
+    nch = lib.gdn_oracle_num_chunks(cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), N, chunk)
+    o = np.full((Ttot, hv, dv), np.nan)
+    sf = np.full((N, hv, dv, dk), np.nan)
+    inter = None
+    if intermediates:
+        inter = {
+            "gcum": np.full((nch, hv, chunk), np.nan),
+            "tmat": np.full((nch, hv, chunk, chunk), np.nan),
+            "w": np.full((nch, hv, chunk, dk), np.nan),
+            "ut": np.full((nch, hv, chunk, dv), np.nan),
+            "u": np.full((nch, hv, chunk, dv), np.nan),
+            "sc": np.full((nch, hv, dv, dk), np.nan),
+        }
+    co = _ChunkOut(chunk, *(_dptr(inter[n]) if inter else _dptr(None)
+                            for n in ("gcum", "tmat", "w", "ut", "u", "sc")))
+    prob = _problem(q, k, v, g, beta, s0, cu, o, sf, dims)
+    keep, uptr, nu = _units_arg(units)
+    rc = lib.gdn_oracle_chunkwise(ctypes.byref(prob), ctypes.byref(co), uptr, nu, threads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"oracle chunkwise failed ({rc})")
+    o, sf = _finish(o, sf, batched, dims)
+    return (o, sf, inter) if intermediates else (o, sf)
+
+
+def decode_step(q, k, v, g, beta, state, threads=None, lib=None):
+    """One decode token per sequence: q,k [N,Hk,dk], v [N,Hv,dv], g,beta [N,Hv],
+    state [N,Hv,dv,dk].  Returns (o [N,Hv,dv], new_state).  This is the token
+    recurrence applied to N one-token sequences."""
+    N = np.asarray(q).shape[0]
+    cu = np.arange(N + 1, dtype=np.int64)
+    return recurrent(q, k, v, g, beta, initial_state=state, cu_seqlens=cu, threads=threads, lib=lib)

@@ -1,0 +1,117 @@
+"""Plant mistakes in a copy of the oracle and check that the pins catch each.
+
+Every mutant is a plausible slip (a dropped term, a wrong sign, a wrong
+index or head mapping, an ignored state, a misplaced decay).  The mutated
+copy is compiled into a temporary library; the pins of
+``test_oracle_pins.py`` run against it; at least one must fail.  The real
+oracle source is never modified.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import test_oracle_pins as pins
+from oracle import oracle
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "gdn_oracle.c")
+
+# (name, text to find, replacement); only the first occurrence is replaced,
+# which for the shared idioms is the one inside the token recurrence.
+MUTANTS = [
+    ("erase term without alpha",
+     "const double ui = beta * (vt[i] - alpha * pk[i]);", "const double ui = beta * (vt[i] - pk[i]);"),
+    ("beta dropped",
+     "const double ui = beta * (vt[i] - alpha * pk[i]);", "const double ui = (vt[i] - alpha * pk[i]);"),
+    ("write with wrong sign",
+     "S[i * dk + j] = alpha * S[i * dk + j] + ui * kt[j];", "S[i * dk + j] = alpha * S[i * dk + j] - ui * kt[j];"),
+    ("decay applied to the write too",
+     "S[i * dk + j] = alpha * S[i * dk + j] + ui * kt[j];",
+     "S[i * dk + j] = alpha * (S[i * dk + j] + ui * kt[j]);"),
+    ("read-out with k instead of q",
+     "for (int j = 0; j < dk; ++j) acc += S[i * dk + j] * qt[j];",
+     "for (int j = 0; j < dk; ++j) acc += S[i * dk + j] * kt[j];"),
+    ("modulo head mapping",
+     "const int hq = h / (p->hv / p->hk);", "const int hq = h % p->hk;"),
+    ("initial state ignored",
+     "if (p->s0) memcpy(S, p->s0 + unit", "if (0) memcpy(S, p->s0 + unit"),
+    ("gate sign flipped",
+     "const double alpha = exp(p->g[t * p->hv + h]);", "const double alpha = exp(-p->g[t * p->hv + h]);"),
+    ("chunk mask without its diagonal",
+     "for (int j = 0; j <= r; ++j) {", "for (int j = 0; j < r; ++j) {"),
+    ("triangular solve with wrong sign",
+     "x -= A[r * L + j] * T[j * L + c];", "x += A[r * L + j] * T[j * L + c];"),
+    ("W without the cumulative decay",
+     "acc += T[r * L + j] * p->beta[(c0 + j) * p->hv + h] * exp(G[j]) * K[j * dk + x];",
+     "acc += T[r * L + j] * p->beta[(c0 + j) * p->hv + h] * K[j * dk + x];"),
+    ("carried state not decayed",
+     "S[i * dk + x] = exp(gl) * S[i * dk + x] + acc;", "S[i * dk + x] = S[i * dk + x] + acc;"),
+    ("inter-chunk output term without gamma",
+     "ot[i] = exp(G[r]) * inter + intra;", "ot[i] = inter + intra;"),
+    ("A built with Gamma transposed",
+     "a = p->beta[(c0 + r) * p->hv + h] * exp(G[r] - G[j]) * kk;",
+     "a = p->beta[(c0 + r) * p->hv + h] * exp(G[j] - G[r]) * kk;"),
+]
+
+
+class _Bound:
+    """The oracle module's API bound to a given (mutant) library."""
+
+    def __init__(self, lib):
+        self.lib = lib
+
+    def recurrent(self, *a, **kw):
+        return oracle.recurrent(*a, lib=self.lib, **kw)
+
+    def chunkwise(self, *a, **kw):
+        return oracle.chunkwise(*a, lib=self.lib, **kw)
+
+    def delta_error_form(self, *a, **kw):
+        return oracle.delta_error_form(*a, lib=self.lib, **kw)
+
+    def decode_step(self, *a, **kw):
+        return oracle.decode_step(*a, lib=self.lib, **kw)
+
+
+def _pin_calls(m):
+    return [
+        lambda: pins.test_handworked_example(m),
+        lambda: pins.test_one_token_and_head_mapping(m),
+        lambda: pins.test_g_zero_is_delta_rule(m, True),
+        lambda: pins.test_beta_zero_decay_only(m),
+        lambda: pins.test_exact_recall_orthonormal_keys(m),
+        lambda: pins.test_alpha_zero_clears_state(m),
+        lambda: pins.test_brute_force_explicit_matrices(m),
+        lambda: pins.test_chunkwise_equals_recurrent(m, 4, True),
+        lambda: pins.test_chunkwise_equals_recurrent(m, 16, False),
+        lambda: pins.test_continuation(m, 13),
+    ]
+
+
+def _caught(m):
+    failures = 0
+    for call in _pin_calls(m):
+        try:
+            with np.errstate(all="ignore"):
+                call()
+        except AssertionError:
+            failures += 1
+    return failures
+
+
+def test_unmutated_copy_passes(tmp_path):
+    src = open(SRC).read()
+    p = tmp_path / "copy.c"
+    p.write_text(src)
+    lib = oracle.load(oracle.build(force=True, src=str(p), out=str(tmp_path / "libcopy.so")))
+    assert _caught(_Bound(lib)) == 0
+
+
+@pytest.mark.parametrize("name,find,repl", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(tmp_path, name, find, repl):
+    src = open(SRC).read()
+    assert find in src, f"mutation anchor missing: {find}"
+    p = tmp_path / "mutant.c"
+    p.write_text(src.replace(find, repl, 1))
+    lib = oracle.load(oracle.build(force=True, src=str(p), out=str(tmp_path / "libmutant.so")))
+    assert _caught(_Bound(lib)) > 0, f"no pin caught the mutant: {name}"

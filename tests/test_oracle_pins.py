@@ -1,0 +1,327 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: a
+hand-worked example, a closed form, an invariant, a limiting case the pages
+state, an independently written formulation, or brute force with explicit
+matrices.  ``test_oracle_mutants.py`` plants mistakes in a copy of the oracle
+and checks that these pins catch every one.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from conftest import rel_l2_per_slice
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def _rand_problem(rng, T, hk, hv, dk, dv, s0=True, unit_keys=True, g_scale=1.0):
+    q = rng.standard_normal((1, T, hk, dk))
+    k = rng.standard_normal((1, T, hk, dk))
+    if unit_keys:
+        q /= np.linalg.norm(q, axis=-1, keepdims=True)
+        k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((1, T, hv, dv))
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal((1, T, hv))))
+    g = -g_scale * np.logaddexp(0.0, rng.standard_normal((1, T, hv)))
+    S0 = 0.3 * rng.standard_normal((1, hv, dv, dk)) if s0 else None
+    return q, k, v, g, beta, S0
+
+
+# ---------------------------------------------------------------------------
+# Hand-worked example (pencil and paper; tests/golden/handworked_d2.json)
+# ---------------------------------------------------------------------------
+def test_handworked_example(oracle_mod):
+    with open(os.path.join(HERE, "golden", "handworked_d2.json")) as f:
+        gold = json.load(f)
+    q = np.array(gold["q"])[None, :, None, :]
+    k = np.array(gold["k"])[None, :, None, :]
+    v = np.array(gold["v"])[None, :, None, :]
+    beta = np.array(gold["beta"])[None, :, None]
+    g = np.array(gold["g"])[None, :, None]
+    o, sf = oracle_mod.recurrent(q, k, v, g, beta)
+    np.testing.assert_allclose(o[0, :, 0, :], np.array(gold["o"]), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(sf[0, 0], np.array(gold["s_final"]), rtol=0, atol=1e-12)
+    for C in (1, 2, 3):
+        oc, sc = oracle_mod.chunkwise(q, k, v, g, beta, C)
+        np.testing.assert_allclose(oc[0, :, 0, :], np.array(gold["o"]), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(sc[0, 0], np.array(gold["s_final"]), rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# P-6: one token from a zero state: o = beta v (k.q), S = beta v k^T, and the
+# grouped-head mapping (value head h reads q/k head h // (Hv/Hk)).
+# ---------------------------------------------------------------------------
+def test_one_token_and_head_mapping(oracle_mod):
+    rng = np.random.default_rng(6)
+    hk, hv, dk, dv = 2, 6, 5, 3
+    q, k, v, g, beta, _ = _rand_problem(rng, 1, hk, hv, dk, dv, s0=False)
+    o, sf = oracle_mod.recurrent(q, k, v, g, beta)
+    for h in range(hv):
+        hq = h // (hv // hk)
+        kq = k[0, 0, hq] @ q[0, 0, hq]
+        np.testing.assert_allclose(o[0, 0, h], beta[0, 0, h] * v[0, 0, h] * kq, rtol=1e-13, atol=1e-15)
+        np.testing.assert_allclose(sf[0, h], beta[0, 0, h] * np.outer(v[0, 0, h], k[0, 0, hq]), rtol=1e-13,
+                                   atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# P-2: g = 0 (alpha = 1) is DeltaNet; compare with the error-correcting form
+# S <- S - beta (S k - v) k^T, written separately.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("s0", [False, True])
+def test_g_zero_is_delta_rule(oracle_mod, s0):
+    rng = np.random.default_rng(2)
+    q, k, v, g, beta, S0 = _rand_problem(rng, 40, 2, 4, 8, 6, s0=s0)
+    g = np.zeros_like(g)
+    o, sf = oracle_mod.recurrent(q, k, v, g, beta, initial_state=S0)
+    od, sd = oracle_mod.delta_error_form(q, k, v, beta, initial_state=S0)
+    assert rel_l2_per_slice(o[0], od[0], axes=(0, 2)) < 1e-13
+    assert rel_l2_per_slice(sf, sd, axes=(2, 3)) < 1e-13
+
+
+# ---------------------------------------------------------------------------
+# P-3: beta = 0 leaves only the decay: S_t = exp(g_1 + ... + g_t) S0 and
+# o_t = exp(G_t) S0 q_t.  With g = 0 as well, S is unchanged.
+# ---------------------------------------------------------------------------
+def test_beta_zero_decay_only(oracle_mod):
+    rng = np.random.default_rng(3)
+    hk, hv, dk, dv, T = 1, 2, 6, 4, 17
+    q, k, v, g, beta, S0 = _rand_problem(rng, T, hk, hv, dk, dv)
+    beta = np.zeros_like(beta)
+    o, sf = oracle_mod.recurrent(q, k, v, g, beta, initial_state=S0)
+    G = np.cumsum(g[0], axis=0)  # [T, hv]
+    for h in range(hv):
+        np.testing.assert_allclose(sf[0, h], np.exp(G[-1, h]) * S0[0, h], rtol=1e-13)
+        for t in range(T):
+            np.testing.assert_allclose(o[0, t, h], np.exp(G[t, h]) * S0[0, h] @ q[0, t, 0], rtol=1e-12,
+                                       atol=1e-300)
+    o2, sf2 = oracle_mod.recurrent(q, k, v, np.zeros_like(g), beta, initial_state=S0)
+    np.testing.assert_array_equal(sf2, S0)
+    for t in range(T):
+        np.testing.assert_allclose(o2[0, t, 0], S0[0, 0] @ q[0, t, 0], rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# P-4: exact recall.  alpha = 1, beta = 1, orthonormal keys written in order:
+# S k_i = v_i for every written pair, S = S0 (I - sum k k^T) + sum v k^T.
+# ---------------------------------------------------------------------------
+def test_exact_recall_orthonormal_keys(oracle_mod):
+    rng = np.random.default_rng(4)
+    d, m, dv = 8, 6, 5
+    Qm, _ = np.linalg.qr(rng.standard_normal((d, d)))
+    keys = Qm[:, :m].T  # m orthonormal rows
+    k = keys[None, :, None, :]
+    q = rng.standard_normal((1, m, 1, d))
+    v = rng.standard_normal((1, m, 1, dv))
+    beta = np.ones((1, m, 1))
+    g = np.zeros((1, m, 1))
+    S0 = rng.standard_normal((1, 1, dv, d))
+    _, sf = oracle_mod.recurrent(q, k, v, g, beta, initial_state=S0)
+    S = sf[0, 0]
+    for i in range(m):
+        np.testing.assert_allclose(S @ keys[i], v[0, i, 0], rtol=1e-12, atol=1e-12)
+    P = keys.T @ keys
+    np.testing.assert_allclose(S, S0[0, 0] @ (np.eye(d) - P) + v[0, :, 0].T @ keys, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# P-5: alpha -> 0 (g = -inf) clears the state: S_t = beta v k^T and
+# o_t = beta v (k.q), whatever came before.
+# ---------------------------------------------------------------------------
+def test_alpha_zero_clears_state(oracle_mod):
+    rng = np.random.default_rng(5)
+    q, k, v, g, beta, S0 = _rand_problem(rng, 9, 1, 2, 4, 3)
+    g[:] = -np.inf
+    o, sf = oracle_mod.recurrent(q, k, v, g, beta, initial_state=S0)
+    for h in range(2):
+        for t in range(9):
+            np.testing.assert_allclose(o[0, t, h], beta[0, t, h] * v[0, t, h] * (k[0, t, 0] @ q[0, t, 0]),
+                                       rtol=1e-13, atol=1e-15)
+        np.testing.assert_allclose(sf[0, h], beta[0, -1, h] * np.outer(v[0, -1, h], k[0, -1, 0]), rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# P-7: the norm bound that unit keys and beta in (0,1) give:
+# ||S_t||_2 <= alpha_t ||S_{t-1}||_2 + beta_t ||v_t|| ||k_t||.
+# ---------------------------------------------------------------------------
+def test_norm_bound(oracle_mod):
+    rng = np.random.default_rng(7)
+    T, dk, dv = 60, 6, 5
+    q, k, v, g, beta, S0 = _rand_problem(rng, T, 1, 1, dk, dv, g_scale=0.05)
+    S = S0[0, 0]
+    for t in range(T):
+        sl = slice(t, t + 1)
+        _, sf = oracle_mod.recurrent(q[:, sl], k[:, sl], v[:, sl], g[:, sl], beta[:, sl],
+                                     initial_state=S[None, None])
+        Sn = sf[0, 0]
+        bound = np.exp(g[0, t, 0]) * np.linalg.norm(S, 2) + beta[0, t, 0] * np.linalg.norm(v[0, t, 0]) * \
+            np.linalg.norm(k[0, t, 0])
+        assert np.linalg.norm(Sn, 2) <= bound * (1 + 1e-12)
+        # the transition alone is a contraction along k: ||S(I - beta k k^T)|| <= ||S||
+        M = np.eye(dk) - beta[0, t, 0] * np.outer(k[0, t, 0], k[0, t, 0])
+        assert np.linalg.norm(M, 2) <= 1 + 1e-12
+        S = Sn
+
+
+# ---------------------------------------------------------------------------
+# P-9: brute force with explicit d x d matrices of the pages' product form:
+# S_T = S0 prod_t M_t + sum_s beta_s v_s k_s^T prod_{t>s} M_t,
+# M_t = alpha_t (I - beta_t k_t k_t^T);  o_t = S_t q_t.
+# ---------------------------------------------------------------------------
+def test_brute_force_explicit_matrices(oracle_mod):
+    rng = np.random.default_rng(9)
+    T, hk, hv, dk, dv = 7, 1, 2, 5, 3
+    q, k, v, g, beta, S0 = _rand_problem(rng, T, hk, hv, dk, dv, unit_keys=False)
+    o, sf = oracle_mod.recurrent(q, k, v, g, beta, initial_state=S0)
+    for h in range(hv):
+        Ms = [np.exp(g[0, t, h]) * (np.eye(dk) - beta[0, t, h] * np.outer(k[0, t, 0], k[0, t, 0])) for t in range(T)]
+        for tt in range(T):
+            P = np.eye(dk)
+            for t in range(tt + 1):
+                P = P @ Ms[t]
+            St = S0[0, h] @ P
+            for s in range(tt + 1):
+                R = np.eye(dk)
+                for t in range(s + 1, tt + 1):
+                    R = R @ Ms[t]
+                St = St + beta[0, s, h] * np.outer(v[0, s, h], k[0, s, 0]) @ R
+            np.testing.assert_allclose(o[0, tt, h], St @ q[0, tt, 0], rtol=1e-11, atol=1e-13)
+            if tt == T - 1:
+                np.testing.assert_allclose(sf[0, h], St, rtol=1e-11, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# P-1: the chunkwise (WY/UT) form equals the recurrence to 1e-12 -- several
+# chunk sizes, grouped heads, d_k != d_v, varlen with ragged tails.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("C", [1, 4, 16])
+@pytest.mark.parametrize("s0", [False, True])
+def test_chunkwise_equals_recurrent(oracle_mod, C, s0):
+    rng = np.random.default_rng(11 + C)
+    lens = [37, 1, 16, 64, 5]
+    T = sum(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    q, k, v, g, beta, _ = _rand_problem(rng, T, 2, 4, 12, 10)
+    S0 = 0.3 * rng.standard_normal((len(lens), 4, 10, 12)) if s0 else None
+    o, sf = oracle_mod.recurrent(q, k, v, g, beta, initial_state=S0, cu_seqlens=cu)
+    oc, sc = oracle_mod.chunkwise(q, k, v, g, beta, C, initial_state=S0, cu_seqlens=cu)
+    assert rel_l2_per_slice(oc, o, axes=(0, 2)) < 1e-12
+    assert rel_l2_per_slice(sc, sf, axes=(2, 3)) < 1e-12
+
+
+def test_chunkwise_strong_decay_and_clearing(oracle_mod):
+    """Very negative g (exp(g) underflows to exactly 0 in fp64) keeps the chunk
+    form finite: Gamma is built as exp(G_r - G_j), never as a ratio of
+    underflowed products.  (g = -inf itself is a limit of the recurrence,
+    pinned by test_alpha_zero_clears_state; prefix sums of -inf are not
+    defined, so the chunk form takes finite g.)"""
+    rng = np.random.default_rng(12)
+    q, k, v, g, beta, S0 = _rand_problem(rng, 48, 1, 1, 6, 6)
+    g[0, ::7, 0] = -200.0
+    g[0, 5, 0] = -1000.0
+    o, sf = oracle_mod.recurrent(q, k, v, g, beta, initial_state=S0)
+    oc, sc = oracle_mod.chunkwise(q, k, v, g, beta, 16, initial_state=S0)
+    assert np.all(np.isfinite(oc)) and np.all(np.isfinite(sc))
+    assert rel_l2_per_slice(oc, o, axes=(1, 3)) < 1e-12
+    assert rel_l2_per_slice(sc, sf, axes=(2, 3)) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# Chunk intermediates pinned to per-token quantities.  The state at each
+# chunk start must equal the recurrence run up to that token; the rows of
+# U are u_r = beta_r (v_r - alpha_r S_{r-1} k_r); U is affine in S0 with
+# U(S0=0) = U~ and U(0) - U(S0) = W S0^T.
+# ---------------------------------------------------------------------------
+def test_chunk_intermediates_pinned_by_recurrence(oracle_mod):
+    rng = np.random.default_rng(13)
+    C, T, dk, dv = 8, 29, 6, 5
+    q, k, v, g, beta, S0 = _rand_problem(rng, T, 1, 1, dk, dv)
+    _, _, inter = oracle_mod.chunkwise(q, k, v, g, beta, C, initial_state=S0, intermediates=True)
+    _, _, inter0 = oracle_mod.chunkwise(q, k, v, g, beta, C, initial_state=None, intermediates=True)
+    # per-token states by running the recurrence on every prefix
+    states = [S0[0, 0]]
+    for t in range(T):
+        _, sf = oracle_mod.recurrent(q[:, :t + 1], k[:, :t + 1], v[:, :t + 1], g[:, :t + 1], beta[:, :t + 1],
+                                     initial_state=S0)
+        states.append(sf[0, 0])
+    for c, c0 in enumerate(range(0, T, C)):
+        np.testing.assert_allclose(inter["sc"][c, 0], states[c0], rtol=1e-12, atol=1e-13)
+        L = min(C, T - c0)
+        for r in range(L):
+            t = c0 + r
+            u_ref = beta[0, t, 0] * (v[0, t, 0] - np.exp(g[0, t, 0]) * states[t] @ k[0, t, 0])
+            np.testing.assert_allclose(inter["u"][c, 0, r], u_ref, rtol=1e-11, atol=1e-13)
+            np.testing.assert_allclose(inter["gcum"][c, 0, r], g[0, c0:t + 1, 0].sum(), rtol=1e-13)
+        # U~ is U with a zero start state only for the first chunk (later
+        # chunks start from the carried state), so compare affine parts
+        if c == 0:
+            np.testing.assert_allclose(inter0["u"][c, 0, :L], inter["ut"][c, 0, :L], rtol=1e-12, atol=1e-13)
+            np.testing.assert_allclose(inter0["u"][c, 0, :L] - inter["u"][c, 0, :L],
+                                       inter["w"][c, 0, :L] @ S0[0, 0].T, rtol=1e-11, atol=1e-13)
+        # T is unit lower-triangular
+        Tm = inter["tmat"][c, 0, :L, :L]
+        np.testing.assert_array_equal(np.diag(Tm), np.ones(L))
+        assert np.all(np.triu(Tm, 1) == 0)
+
+
+# ---------------------------------------------------------------------------
+# P-8: continuation.  run(x[:T1]) -> S; run(x[T1:], S) equals run(x); and
+# one-token decode steps after a prefill equal a longer prefill.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("T1", [1, 13, 31])
+def test_continuation(oracle_mod, T1):
+    rng = np.random.default_rng(8)
+    T = 32
+    q, k, v, g, beta, S0 = _rand_problem(rng, T, 2, 4, 7, 5)
+    o, sf = oracle_mod.recurrent(q, k, v, g, beta, initial_state=S0)
+    a = slice(0, T1)
+    b = slice(T1, T)
+    oa, sa = oracle_mod.recurrent(q[:, a], k[:, a], v[:, a], g[:, a], beta[:, a], initial_state=S0)
+    ob, sb = oracle_mod.recurrent(q[:, b], k[:, b], v[:, b], g[:, b], beta[:, b], initial_state=sa)
+    np.testing.assert_allclose(np.concatenate([oa, ob], axis=1), o, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(sb, sf, rtol=1e-12, atol=1e-14)
+    # decode steps after the prefix
+    S = sa
+    for t in range(T1, T):
+        od, S = oracle_mod.decode_step(q[:, t], k[:, t], v[:, t], g[:, t], beta[:, t], S)
+        np.testing.assert_allclose(od[0], o[0, t], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(S, sf, rtol=1e-12, atol=1e-14)
+
+
+def test_varlen_equals_per_sequence(oracle_mod):
+    rng = np.random.default_rng(10)
+    lens = [3, 0, 11, 1]
+    T = sum(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    q, k, v, g, beta, _ = _rand_problem(rng, T, 1, 2, 4, 4)
+    S0 = rng.standard_normal((len(lens), 2, 4, 4))
+    o, sf = oracle_mod.recurrent(q, k, v, g, beta, initial_state=S0, cu_seqlens=cu)
+    for n, L in enumerate(lens):
+        sl = slice(cu[n], cu[n + 1])
+        if L == 0:
+            np.testing.assert_array_equal(sf[n], S0[n])  # empty sequence: final = initial
+            continue
+        on, sn = oracle_mod.recurrent(q[:, sl], k[:, sl], v[:, sl], g[:, sl], beta[:, sl], initial_state=S0[n:n + 1])
+        np.testing.assert_array_equal(o[0, cu[n]:cu[n + 1]], on[0])
+        np.testing.assert_array_equal(sf[n], sn[0])
+
+
+def test_unit_subset_matches_full(oracle_mod):
+    rng = np.random.default_rng(14)
+    q, k, v, g, beta, _ = _rand_problem(rng, 20, 2, 4, 5, 5)
+    q = np.concatenate([q, q[:, ::-1]], axis=0)
+    k = np.concatenate([k, k], axis=0)
+    v = np.concatenate([v, v], axis=0)
+    g = np.concatenate([g, g], axis=0)
+    beta = np.concatenate([beta, beta], axis=0)
+    o, sf = oracle_mod.recurrent(q, k, v, g, beta)
+    units = [1, 6]
+    os_, ss = oracle_mod.recurrent(q, k, v, g, beta, units=units)
+    for u in units:
+        n, h = divmod(u, 4)
+        np.testing.assert_array_equal(os_[n, :, h], o[n, :, h])
+        np.testing.assert_array_equal(ss[n, h], sf[n, h])
+    assert np.isnan(os_[0, :, 0]).all()
