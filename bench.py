@@ -1,0 +1,397 @@
+#!/usr/bin/env python
+"""Benchmark of the gated delta rule on B200: prefill tokens/s (with its
+fraction of the bf16 tensor-core roofline) and decode state-update HBM GB/s.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one chunkwise prefill of the 4 x 4096-token, 16 q/k-head,
+32 v-head, d = 128, C = 64 bf16 workload (zero initial state), inputs
+resident in HBM.  The decode step of the 256-sequence, 16/32-head, d = 128
+workload (fp32 state of 512 MiB updated in place) is timed in the same run
+and reported under "decode".  With N > 1 (torchrun) every rank runs an
+independent replica on its own GPU (the problems are independent; there is
+no data-path collective): "scaling" is "weak" and the value is the tokens
+of all ranks over the slowest rank's device time.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (on
+rank 0 only), each step a bounded sample of (sequence, head) units of the
+same workload, extrapolated to the workload's tokens/s.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN prefill tokens/s (% of bf16 TC peak); decode state-update HBM GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Useful chunk FLOPs per (token, v-head) at d = 128, C = 64 with 2 v-heads per
+# q/k head: inter-chunk 6 d^2 + triangular intra-chunk 3 C d + shared Gram 2 C d / G.
+USEFUL_FLOPS_PER_VHEAD_TOKEN = 6 * 128 * 128 + 3 * 64 * 128 + 2 * 64 * 128 // 2
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--decode-steps", type=int, default=512)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
+    return p.parse_args(argv)
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_traffic(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, only if the kernel's
+    source has not changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        entries = json.load(f)
+    e = entries.get(kernel)
+    if not e:
+        return None
+    src = os.path.join(ROOT, e["source"])
+    if not os.path.exists(src):
+        return None
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    return e["bytes_per_launch"] if sha == e["source_sha256"] else None
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80, "sync_boost": 0x10}
+
+    def __init__(self, index: int, interval: float = 0.01):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.interval = interval
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML unavailable: report no clocks rather than fail the bench
+            self.nv = None
+
+    def _sample(self):
+        if self.nv is None:
+            return
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            bits = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for name, mask in self.REASONS.items():
+                if bits & mask:
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.interval)
+
+    def __enter__(self):
+        self._sample()
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._sample()
+        self._stop.set()
+        self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def max_over_ranks(x: float, device, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def timed(fn, steps, stream):
+    """Device time per call (ms) over ``steps`` calls, CUDA events on ``stream``."""
+    import torch
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / steps
+
+
+def cpu_oracle_sample(w, inp, target_s: float):
+    """Time the fp64 oracle on whole (sequence, head) units of the workload and
+    extrapolate to the full workload's tokens/s."""
+    import numpy as np
+    from oracle import oracle
+    f64 = lambda t: None if t is None else t.to(dtype=__import__("torch").float64).numpy()
+    q, k, v, g, b = (f64(inp[n]) for n in ("q", "k", "v", "g", "beta"))
+    s0 = f64(inp["initial_state"])
+    threads = oracle.default_threads()
+    total_units = w.num_seqs * w.hv
+    # calibrate with one round of `threads` units, then run a sample of about target_s
+    cal = list(range(min(threads, total_units)))
+    t0 = time.perf_counter()
+    oracle.recurrent(q, k, v, g, b, initial_state=s0, units=cal, threads=threads)
+    t_cal = time.perf_counter() - t0
+    rounds = max(1, int(target_s / max(t_cal, 1e-3)))
+    n_units = min(total_units, rounds * len(cal))
+    units = list(range(n_units))
+    t0 = time.perf_counter()
+    oracle.recurrent(q, k, v, g, b, initial_state=s0, units=units, threads=threads)
+    t = time.perf_counter() - t0
+    full = t * total_units / n_units
+    return {"value": w.total_tokens / full, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n_units} of {total_units} (sequence, v-head) units of {w.name} (whole sequences, "
+                      f"{t:.1f} s wall), extrapolated to the full workload"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from linear_attention_sequence_sm_b200 import inputs as I
+    from oracle import oracle
+    import numpy as np
+    w = I.prefill_bf16()
+    inp = I.make_prefill_inputs(w)
+    f64 = lambda t: None if t is None else t.to(dtype=__import__("torch").float64).numpy()
+    q, k, v, g, b = (f64(inp[n]) for n in ("q", "k", "v", "g", "beta"))
+    threads = oracle.default_threads()
+    total_units = w.num_seqs * w.hv
+    per_step = min(total_units, threads)  # one unit per host thread per step
+    times = []
+    for i in range(args.warmup + args.steps):
+        units = [(i * per_step + j) % total_units for j in range(per_step)]
+        t0 = time.perf_counter()
+        oracle.recurrent(q, k, v, g, b, units=units, threads=threads)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    step_s = statistics.mean(times) * total_units / per_step  # extrapolated full-workload step
+    value = w.total_tokens / step_s
+    sample = f"{per_step} of {total_units} (sequence, v-head) units per step of {w.name}, extrapolated"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded splitmix64)",
+        "config": {"workload": w.name, "global_batch": w.batch, "seq_len": w.seq_len, "parallelism": "none (host cores)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    rank, world, local_rank = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    from linear_attention_sequence_sm_b200 import gdn
+    from linear_attention_sequence_sm_b200 import inputs as I
+
+    peaks, peak_src = load_peaks()
+    w = I.prefill_bf16(seed=1002 + rank)
+    host = I.make_prefill_inputs(w)
+    dev = {k: (v.to(device) if v is not None else None) for k, v in host.items()}
+    o = torch.empty_like(dev["v"])
+    sf = torch.empty((w.num_seqs, w.hv, w.d, w.d), dtype=torch.float32, device=device)
+    shape = gdn.make_shape(dev["q"], dev["v"], None, w.chunk)
+    ws = torch.empty(gdn.workspace_size(shape), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        gdn.chunk_forward(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], initial_state=None, out=o,
+                          final_state=sf, workspace=ws, chunk_size=w.chunk)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    n0 = gdn.launch_count()
+    with ClockSampler(device.index) as clocks:
+        ms = timed(step, args.steps, stream)
+        torch.cuda.synchronize(device)
+    launches = gdn.launch_count() - n0
+    barrier(world, device)
+    ms_max = max_over_ranks(ms, device, world)
+    tokens = w.total_tokens
+    value = world * tokens / (ms_max / 1e3)
+    flops = USEFUL_FLOPS_PER_VHEAD_TOKEN * tokens * w.hv
+    achieved_tflops = flops / (ms / 1e3) / 1e12
+    kernel_name = "gdn_chunk_tc" if gdn_tc_active(gdn, dev, w) else "gdn_chunk_simt"
+    roofline = {"bound": "tensor", "achieved": achieved_tflops, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved_tflops / peaks["bf16_tflops"],
+                "traffic": kernel_traffic(kernel_name), "kernel": kernel_name,
+                "peak_source": f"{peak_src} bf16 dense (burst)",
+                "flops_per_launch": flops, "algorithmic_bytes_per_launch": prefill_bytes(w)}
+
+    # ---- decode: 256 sequences, fp32 state 512 MiB, in place ----
+    dw = I.decode_bf16()
+    gen = torch.Generator(device=device)
+    gen.manual_seed(dw.seed + rank)
+    state = torch.randn((dw.num_seqs, dw.hv, dw.d, dw.d), generator=gen, device=device) * dw.s0_std
+    ring = [{k: v.to(device) for k, v in I.make_decode_inputs(dw, s).items()} for s in range(8)]
+    od = torch.empty((dw.num_seqs, dw.hv, dw.d), dtype=torch.bfloat16, device=device)
+    it = [0]
+
+    def dstep():
+        x = ring[it[0] % len(ring)]
+        it[0] += 1
+        gdn.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state, out=od)
+
+    for _ in range(max(3, args.warmup)):
+        dstep()
+    torch.cuda.synchronize(device)
+    with ClockSampler(device.index) as dclocks:
+        dms = timed(dstep, args.decode_steps, stream)
+    dms = max_over_ranks(dms, device, world)
+    dbytes = decode_bytes(dw)
+    dgbs = dbytes / (dms / 1e3) / 1e9
+    decode = {"value": world * dgbs, "unit": "GB/s", "ms_per_step": dms, "steps": args.decode_steps,
+              "tokens_per_s": world * dw.num_seqs / (dms / 1e3), "workload": dw.name,
+              "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                           "frac": dgbs / peaks["hbm_gbs"], "traffic": kernel_traffic("gdn_decode"),
+                           "kernel": "gdn_decode", "peak_source": f"{peak_src} HBM copy",
+                           "bytes_per_launch": dbytes},
+              "clocks": dclocks.summary()}
+    del state
+
+    # ---- end to end through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        pin = {k: v.pin_memory() for k, v in host.items() if v is not None}
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        sf_host = torch.empty(sf.shape, dtype=sf.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in pin.values())
+        d2h = o_host.numel() * o_host.element_size() + sf_host.numel() * sf_host.element_size()
+
+        def e2e_step():
+            x = {k: v.to(device, non_blocking=True) for k, v in pin.items()}
+            oo, ss = gdn.chunk_forward(x["q"], x["k"], x["v"], x["g"], x["beta"], chunk_size=w.chunk, workspace=ws)
+            o_host.copy_(oo, non_blocking=True)
+            sf_host.copy_(ss, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(device)
+        barrier(world, device)
+        e_ms = timed(e2e_step, max(3, min(args.steps, 20)), stream)
+        e_ms = max_over_ranks(e_ms, device, world)
+        e2e = {"value": world * tokens / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample(w, host, args.cpu_seconds)
+
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded splitmix64 / Box-Muller)",
+            "config": {"workload": w.name, "global_batch": w.batch * world, "seq_len": w.seq_len,
+                       "heads_qk_v": [w.hk, w.hv], "head_dim": w.d, "chunk": w.chunk,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (about 410 MB of mandatory traffic per step)"},
+            "roofline": roofline, "decode": decode, "e2e": e2e, "cpu_baseline": cpu,
+            "gpu_launches": launches, "clocks": clocks.summary(),
+        }), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def gdn_tc_active(gdn, dev, w) -> bool:
+    import torch
+    major, _ = torch.cuda.get_device_capability()
+    return major == 10 and w.dtype == "bf16" and w.d == 128 and w.chunk == 64 and tc_built(gdn)
+
+
+def tc_built(gdn) -> bool:
+    src = open(os.path.join(ROOT, "linear_attention_sequence_sm_b200", "csrc", "gdn_chunk_tc.cu")).read()
+    return "tcgen05.mma" in src
+
+
+def prefill_bytes(w) -> int:
+    """Mandatory HBM bytes of one prefill: q, k, v, o once, g and beta, the
+    initial state (if any) and the final state."""
+    esz = 2 if w.dtype == "bf16" else 4
+    t = w.total_tokens
+    b = t * w.hk * w.d * esz * 2 + t * w.hv * w.d * esz * 2 + t * w.hv * 8
+    b += w.num_seqs * w.hv * w.d * w.d * 4 * (2 if w.s0_std > 0 else 1)
+    return b
+
+
+def decode_bytes(dw) -> int:
+    """Bytes one decode step must move: the fp32 state read and written once,
+    plus q, k, v, o (bf16) and g, beta (fp32)."""
+    s = dw.num_seqs * dw.hv * dw.d * dw.d * 4
+    return 2 * s + dw.num_seqs * (2 * dw.hk * dw.d * 2 + 2 * dw.hv * dw.d * 2 + 2 * dw.hv * 4)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,168 @@
+/*
+ * gdn.h -- C ABI of libgdn.so: the gated delta rule (Gated DeltaNet sequence
+ * mixer) on NVIDIA B200 (sm_100a).
+ *
+ * The operation.  For every sequence and every value head, a d_v x d_k
+ * matrix state S evolves token by token as
+ *
+ *     S_t = S_{t-1} (alpha_t (I - beta_t k_t k_t^T)) + beta_t v_t k_t^T,
+ *     o_t = S_t q_t,                     alpha_t = exp(g_t),
+ *
+ * the gated delta rule of "Architecture Thread I: Gated Attention, DeltaNet,
+ * and Hybrid Models" (section "Gated DeltaNet") and of "Gated Attention
+ * Architectures" (section 3, Gated DeltaNet, "Mathematical Formulation"),
+ * with the read-out o_t = S_t q_t of the same page's section 1.  The state
+ * does not grow with the sequence ("The Transformer Isn't Alone Anymore",
+ * the long-context section), so prefill returns it and decode updates it.
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are dense, row-major and token-major; every pointer is device
+ *     memory owned by the caller.  The library allocates nothing, keeps no
+ *     state between calls, never synchronises, and is stream-ordered: work
+ *     is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream) and runs asynchronously.
+ *   - q, k: [tokens, Hk, d_k]; v, o: [tokens, Hv, d_v], all of `dtype`.
+ *     g, beta: [tokens, Hv] fp32.  States: [N, Hv, d_v, d_k] fp32, row =
+ *     value index, key index fastest.
+ *   - Value head h reads query/key head h / (Hv / Hk) (grouped heads share
+ *     their q/k head in contiguous groups); Hv % Hk must be 0.
+ *   - Unchecked preconditions (documented, not verified): q and k are
+ *     L2-normalised by the caller; beta in (0, 1); g <= 0.  The kernels
+ *     read g as max(g, -20): exp(-20) is about 2e-9, below fp32 resolution
+ *     relative to the state, and the floor keeps the chunk-local prefix
+ *     sums of g finite and accurate (g = -inf would make them undefined).
+ *   - The output reads the state after the update at the same token.
+ *   - Base pointers must be 16-byte aligned (tensor-memory-accelerator
+ *     loads); violations return GDN_ERR_MISALIGNED before any launch.
+ *   - Errors are returned as a status; nothing aborts or prints.  A status
+ *     other than GDN_OK means nothing was enqueued, except GDN_ERR_CUDA
+ *     raised by a launch, which reports the CUDA error of that launch.
+ *   - The last error's detail text is kept per host thread
+ *     (gdn_last_error_message).
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARGUMENT = 1,   /* null pointer, bad shape, Hv % Hk != 0 */
+    GDN_ERR_UNSUPPORTED = 2,        /* valid but not implemented (sizes)     */
+    GDN_ERR_MISALIGNED = 3,         /* a base pointer not 16-byte aligned    */
+    GDN_ERR_WORKSPACE_TOO_SMALL = 4,
+    GDN_ERR_CUDA = 5,               /* a CUDA runtime call or launch failed  */
+    GDN_ERR_DEVICE_CHECK = 6        /* a kernel rejected its inputs (see
+                                       gdn_read_device_status)               */
+} gdn_status_t;
+
+typedef enum { GDN_DTYPE_F32 = 0, GDN_DTYPE_BF16 = 1 } gdn_dtype_t;
+
+/* Flags for gdn_shape_t.flags. */
+#define GDN_FLAG_FORCE_SIMT 1u  /* run the fp32 CUDA-core kernel even where the
+                                   tensor-core kernel applies (cross-checks) */
+
+/* Shape of a prefill problem.
+ *   batch, seq_len  without cu_seqlens: B sequences of T tokens each
+ *                   (tokens = B * T).  With cu_seqlens: batch must be 1 and
+ *                   seq_len is the total packed token count.
+ *   num_seqs        N = batch, or the number of packed sequences.
+ *   chunk_size      C, the chunk length of the chunkwise algorithm: 16, 32
+ *                   or 64.  It changes rounding only, never the result.
+ *   dtype           gdn_dtype_t of q, k, v, o.                             */
+typedef struct {
+    int32_t batch;
+    int32_t seq_len;
+    int32_t num_seqs;
+    int32_t num_qk_heads;
+    int32_t num_v_heads;
+    int32_t head_dim_k;
+    int32_t head_dim_v;
+    int32_t chunk_size;
+    int32_t dtype;
+    uint32_t flags;
+} gdn_shape_t;
+
+/* Bytes of device workspace gdn_chunk_forward needs for `shape` (a pure
+ * function of the shape; the caller allocates it, 256-byte aligned). */
+GDN_API gdn_status_t gdn_chunk_forward_workspace_size(const gdn_shape_t *shape, size_t *bytes);
+
+/* Chunkwise prefill ("Gated Attention Architectures", sections 2 and 3: the
+ * WY representation of the generalised Householder transitions, extended
+ * with per-chunk cumulative decay products, and the decay-masked chunk
+ * output of section 1).  Computes o for every token and, if final_state is
+ * not NULL, the state after each sequence's last token.
+ *   q, k            [tokens, Hk, d_k] dtype
+ *   v               [tokens, Hv, d_v] dtype
+ *   g, beta         [tokens, Hv] fp32 (log-decay, write strength)
+ *   initial_state   [N, Hv, d_v, d_k] fp32, or NULL for zeros
+ *   cu_seqlens      [N + 1] int32 device array of sequence starts
+ *                   (cu[0] = 0, non-decreasing, cu[N] = tokens), or NULL
+ *                   for the batched layout.  Chunks never cross a sequence
+ *                   boundary; empty sequences are allowed (final = initial).
+ *                   Its contents are checked on the device: a violation
+ *                   makes every kernel skip its work and records
+ *                   GDN_ERR_DEVICE_CHECK in the workspace status word.
+ *   o               [tokens, Hv, d_v] dtype (written)
+ *   final_state     [N, Hv, d_v, d_k] fp32 or NULL; may alias initial_state.
+ *   workspace       device scratch of at least the queried size.
+ * Paths: bf16 with d_k = d_v = 128 and C = 64 runs the tensor-core
+ * (tcgen05/TMEM, TMA-fed) kernel; every other supported shape (d_k, d_v <=
+ * 128, C in {16, 32, 64}) runs the fp32 CUDA-core kernel. */
+GDN_API gdn_status_t gdn_chunk_forward(const gdn_shape_t *shape,
+                               const void *q, const void *k, const void *v,
+                               const float *g, const float *beta,
+                               const float *initial_state,
+                               const int32_t *cu_seqlens,
+                               void *o, float *final_state,
+                               void *workspace, size_t workspace_bytes,
+                               void *stream);
+
+/* Reads the device status word that gdn_chunk_forward left in `workspace`
+ * (GDN_OK or GDN_ERR_DEVICE_CHECK) into *device_status.  Synchronises
+ * `stream`.  This is the only entry point that waits for the GPU. */
+GDN_API gdn_status_t gdn_read_device_status(const void *workspace, int32_t *device_status, void *stream);
+
+/* One decode token for each of N sequences, state updated in place
+ * ("The Transformer Isn't Alone Anymore": the recurrent state is read and
+ * updated every step, which makes decoding memory-bound).  Per value head
+ * and per state row i: p_i = s_i . k, r_i = s_i . q,
+ * u_i = beta (v_i - alpha p_i), s_i <- alpha s_i + u_i k^T,
+ * o_i = alpha r_i + u_i (k . q)  (= s_i,new . q): one read and one write
+ * of S.
+ *   q, k   [N, Hk, d_k] dtype;  v, o [N, Hv, d_v] dtype
+ *   g, beta [N, Hv] fp32
+ *   state  [N, Hv, d_v, d_k] fp32, read and written in place.
+ * d_k = 128 takes the vectorised kernel; other d_k <= 256 a generic one. */
+GDN_API gdn_status_t gdn_decode_step(int32_t num_seqs, int32_t num_qk_heads, int32_t num_v_heads,
+                             int32_t head_dim_k, int32_t head_dim_v, int32_t dtype,
+                             const void *q, const void *k, const void *v,
+                             const float *g, const float *beta,
+                             float *state, void *o, void *stream);
+
+/* Static text for a status code. */
+GDN_API const char *gdn_status_string(gdn_status_t status);
+
+/* Detail of the last error returned on the calling host thread ("" if none). */
+GDN_API const char *gdn_last_error_message(void);
+
+/* Number of kernels this library has launched in this process (all host
+ * threads), for accounting of launches inside a timed region. */
+GDN_API uint64_t gdn_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

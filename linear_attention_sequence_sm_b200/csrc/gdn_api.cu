@@ -1,0 +1,191 @@
+// gdn_api.cu -- the extern "C" entry points of libgdn.so: argument checks,
+// path selection and stream-ordered launches.  No allocation, no sync
+// (except gdn_read_device_status, documented as synchronising).
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "gdn_internal.cuh"
+
+namespace gdn {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+static thread_local char g_msg[512] = "";
+
+static gdn_status_t fail(gdn_status_t st, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+static gdn_status_t cuda_fail(cudaError_t e, const char *what) {
+    return fail(GDN_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int device_sm_count(int *major) {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    if (major && cudaDeviceGetAttribute(major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return -1;
+    return sms;
+}
+
+static gdn_status_t check_shape(const gdn_shape_t *s) {
+    if (!s) return fail(GDN_ERR_INVALID_ARGUMENT, "shape is NULL");
+    if (s->batch < 0 || s->seq_len < 0 || s->num_seqs < 0)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "negative batch/seq_len/num_seqs");
+    if (s->num_qk_heads <= 0 || s->num_v_heads <= 0 || s->head_dim_k <= 0 || s->head_dim_v <= 0)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "heads and head dims must be positive");
+    if (s->num_v_heads % s->num_qk_heads != 0)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "num_v_heads (%d) must be a multiple of num_qk_heads (%d)",
+                    s->num_v_heads, s->num_qk_heads);
+    if (s->dtype != GDN_DTYPE_F32 && s->dtype != GDN_DTYPE_BF16)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "dtype %d is not GDN_DTYPE_F32 or GDN_DTYPE_BF16", s->dtype);
+    if (s->chunk_size != 16 && s->chunk_size != 32 && s->chunk_size != 64)
+        return fail(GDN_ERR_UNSUPPORTED, "chunk_size %d not in {16, 32, 64}", s->chunk_size);
+    if (s->head_dim_k > 128 || s->head_dim_v > 128)
+        return fail(GDN_ERR_UNSUPPORTED, "head dims above 128 are not supported (d_k=%d, d_v=%d)",
+                    s->head_dim_k, s->head_dim_v);
+    int64_t tokens = int64_t(s->batch) * s->seq_len;
+    if (tokens > INT32_MAX) return fail(GDN_ERR_UNSUPPORTED, "more than 2^31-1 tokens");
+    if (int64_t(tokens) * s->num_v_heads * s->head_dim_v > (int64_t(1) << 40))
+        return fail(GDN_ERR_UNSUPPORTED, "problem too large");
+    return GDN_OK;
+}
+
+}  // namespace gdn
+
+using namespace gdn;
+
+extern "C" {
+
+const char *gdn_status_string(gdn_status_t st) {
+    switch (st) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARGUMENT: return "GDN_ERR_INVALID_ARGUMENT";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+        case GDN_ERR_MISALIGNED: return "GDN_ERR_MISALIGNED";
+        case GDN_ERR_WORKSPACE_TOO_SMALL: return "GDN_ERR_WORKSPACE_TOO_SMALL";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+        case GDN_ERR_DEVICE_CHECK: return "GDN_ERR_DEVICE_CHECK";
+    }
+    return "GDN_ERR_UNKNOWN";
+}
+
+const char *gdn_last_error_message(void) { return g_msg; }
+
+uint64_t gdn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+gdn_status_t gdn_chunk_forward_workspace_size(const gdn_shape_t *s, size_t *bytes) {
+    g_msg[0] = 0;
+    if (!bytes) return fail(GDN_ERR_INVALID_ARGUMENT, "bytes is NULL");
+    gdn_status_t st = check_shape(s);
+    if (st != GDN_OK) return st;
+    *bytes = ws_layout(s->num_seqs).total;
+    return GDN_OK;
+}
+
+gdn_status_t gdn_chunk_forward(const gdn_shape_t *s, const void *q, const void *k, const void *v,
+                               const float *g, const float *beta, const float *initial_state,
+                               const int32_t *cu_seqlens, void *o, float *final_state, void *workspace,
+                               size_t workspace_bytes, void *stream_) {
+    g_msg[0] = 0;
+    gdn_status_t st = check_shape(s);
+    if (st != GDN_OK) return st;
+    const int64_t tokens = int64_t(s->batch) * s->seq_len;
+    if (cu_seqlens) {
+        if (s->batch != 1) return fail(GDN_ERR_INVALID_ARGUMENT, "batch must be 1 with cu_seqlens");
+    } else if (s->num_seqs != s->batch) {
+        return fail(GDN_ERR_INVALID_ARGUMENT, "num_seqs (%d) must equal batch (%d) without cu_seqlens",
+                    s->num_seqs, s->batch);
+    }
+    if (tokens > 0 && (!q || !k || !v || !g || !beta || !o))
+        return fail(GDN_ERR_INVALID_ARGUMENT, "q, k, v, g, beta and o must be non-NULL");
+    if (!workspace) return fail(GDN_ERR_INVALID_ARGUMENT, "workspace is NULL");
+    const WsLayout L = ws_layout(s->num_seqs);
+    if (workspace_bytes < L.total)
+        return fail(GDN_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", workspace_bytes, L.total);
+    const void *ptrs[] = {q, k, v, g, beta, initial_state, cu_seqlens, o, final_state};
+    const char *names[] = {"q", "k", "v", "g", "beta", "initial_state", "cu_seqlens", "o", "final_state"};
+    for (int i = 0; i < 9; ++i)
+        if (ptrs[i] && !aligned16(ptrs[i]))
+            return fail(GDN_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(GDN_ERR_MISALIGNED, "workspace is not 256-byte aligned");
+
+    int major = 0;
+    const int sms = device_sm_count(&major);
+    if (sms <= 0) return fail(GDN_ERR_CUDA, "no usable CUDA device");
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+
+    cudaError_t e = launch_schedule(*s, cu_seqlens, workspace, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "schedule kernel launch");
+
+    PrefillArgs a;
+    a.num_seqs = s->num_seqs;
+    a.hk = s->num_qk_heads;
+    a.hv = s->num_v_heads;
+    a.dk = s->head_dim_k;
+    a.dv = s->head_dim_v;
+    a.chunk = s->chunk_size;
+    a.dtype = s->dtype;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.s0 = initial_state; a.o = o; a.s_final = final_state;
+    char *ws = static_cast<char *>(workspace);
+    a.sched.hdr = reinterpret_cast<WsHeader *>(ws);
+    a.sched.order = reinterpret_cast<const int32_t *>(ws + L.order_off);
+    a.sched.start = reinterpret_cast<const int32_t *>(ws + L.start_off);
+    a.sched.len = reinterpret_cast<const int32_t *>(ws + L.len_off);
+    if (s->num_seqs == 0) return GDN_OK;
+
+    const bool use_tc = major == 10 && !(s->flags & GDN_FLAG_FORCE_SIMT) && chunk_tc_supported(*s);
+    e = use_tc ? launch_chunk_tc(a, stream, sms) : launch_chunk_simt(a, stream, sms);
+    if (e != cudaSuccess) return cuda_fail(e, use_tc ? "tensor-core prefill launch" : "prefill launch");
+    return GDN_OK;
+}
+
+gdn_status_t gdn_read_device_status(const void *workspace, int32_t *device_status, void *stream_) {
+    g_msg[0] = 0;
+    if (!workspace || !device_status) return fail(GDN_ERR_INVALID_ARGUMENT, "NULL argument");
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    WsHeader h;
+    cudaError_t e = cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status");
+    *device_status = h.status;
+    if (h.status != GDN_OK)
+        fail(GDN_ERR_DEVICE_CHECK, "cu_seqlens rejected on the device at index %d", h.bad_index);
+    return GDN_OK;
+}
+
+gdn_status_t gdn_decode_step(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
+                             const void *q, const void *k, const void *v, const float *g, const float *beta,
+                             float *state, void *o, void *stream_) {
+    g_msg[0] = 0;
+    if (n < 0 || hk <= 0 || hv <= 0 || dk <= 0 || dv <= 0)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "bad decode shape");
+    if (hv % hk != 0) return fail(GDN_ERR_INVALID_ARGUMENT, "num_v_heads must be a multiple of num_qk_heads");
+    if (dtype != GDN_DTYPE_F32 && dtype != GDN_DTYPE_BF16)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "dtype %d is not GDN_DTYPE_F32 or GDN_DTYPE_BF16", dtype);
+    if (dk > 256) return fail(GDN_ERR_UNSUPPORTED, "decode supports d_k <= 256 (got %d)", dk);
+    if (n == 0) return GDN_OK;
+    if (!q || !k || !v || !g || !beta || !state || !o)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "decode pointers must be non-NULL");
+    const void *ptrs[] = {q, k, v, g, beta, state, o};
+    const char *names[] = {"q", "k", "v", "g", "beta", "state", "o"};
+    for (int i = 0; i < 7; ++i)
+        if (!aligned16(ptrs[i])) return fail(GDN_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+    if (int64_t(n) * hv * dv * dk > (int64_t(1) << 40)) return fail(GDN_ERR_UNSUPPORTED, "state too large");
+    cudaError_t e = launch_decode(n, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o,
+                                  static_cast<cudaStream_t>(stream_));
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    return GDN_OK;
+}
+
+}  // extern "C"

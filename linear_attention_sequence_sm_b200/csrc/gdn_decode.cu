@@ -1,0 +1,184 @@
+// gdn_decode.cu -- one decode token per sequence, state updated in place.
+//
+// Per value head and per state row i (s_i = row i of S, length d_k):
+//   p_i = s_i . k,  r_i = s_i . q                 (the two dot products)
+//   u_i = beta (v_i - alpha p_i)                  (error-corrected write)
+//   s_i <- alpha s_i + u_i k^T
+//   o_i = alpha r_i + u_i (k . q)                 (= s_i,new . q)
+// which is the gated delta rule S_t = S_{t-1}(alpha(I - beta k k^T)) +
+// beta v k^T, o = S_t q ("Architecture Thread I", section "Gated DeltaNet";
+// "Gated Attention Architectures", section 3) written so that S is read once
+// and written once.  Decode is bound by that traffic ("The Transformer Isn't
+// Alone Anymore": the recurrent state is read and updated every step).
+//
+// d_k = 128: a warp owns whole rows; lane l holds s_i[4l .. 4l+3] as one
+// float4 (a row is one coalesced 512-byte segment).  Each warp keeps
+// kRowBatch rows of loads in flight before reducing, for memory-level
+// parallelism.  Other d_k (<= 256): a generic warp-per-row kernel.
+#include "gdn_internal.cuh"
+
+namespace gdn {
+
+constexpr int kDecodeWarps = 4;     // warps per block; a block owns one (sequence, head)
+constexpr int kRowBatch = 8;        // rows in flight per warp
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+    return x;
+}
+
+__device__ __forceinline__ float4 load4(const float *p) { return __ldcs(reinterpret_cast<const float4 *>(p)); }
+__device__ __forceinline__ void store4(float *p, float4 x) { __stcs(reinterpret_cast<float4 *>(p), x); }
+
+__device__ __forceinline__ void load_vec4(const float *p, float out[4]) {
+    const float4 x = *reinterpret_cast<const float4 *>(p);
+    out[0] = x.x; out[1] = x.y; out[2] = x.z; out[3] = x.w;
+}
+__device__ __forceinline__ void load_vec4(const __nv_bfloat16 *p, float out[4]) {
+    const uint2 x = *reinterpret_cast<const uint2 *>(p);
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(&x.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&x.y);
+    const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    out[0] = fa.x; out[1] = fa.y; out[2] = fb.x; out[3] = fb.y;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kDecodeWarps * 32)
+decode_d128_kernel(int32_t hk, int32_t hv, int32_t dv, const T *__restrict__ q, const T *__restrict__ k,
+                   const T *__restrict__ v, const float *__restrict__ g, const float *__restrict__ beta,
+                   float *__restrict__ state, T *__restrict__ o) {
+    constexpr int dk = 128;
+    const int unit = blockIdx.x;            // sequence * hv + head
+    const int n = unit / hv, h = unit % hv;
+    const int hq = h / (hv / hk);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    float kf[4], qf[4];
+    load_vec4(k + (size_t(n) * hk + hq) * dk + 4 * lane, kf);
+    load_vec4(q + (size_t(n) * hk + hq) * dk + 4 * lane, qf);
+    const float kq = warp_sum(kf[0] * qf[0] + kf[1] * qf[1] + kf[2] * qf[2] + kf[3] * qf[3]);
+    const float alpha = __expf(fmaxf(g[unit], kGFloor));
+    const float b = beta[unit];
+
+    float *S = state + size_t(unit) * dv * dk;
+    const T *vrow = v + size_t(unit) * dv;
+    T *orow = o + size_t(unit) * dv;
+
+    for (int i0 = warp * kRowBatch; i0 < dv; i0 += kDecodeWarps * kRowBatch) {
+        float4 s[kRowBatch];
+#pragma unroll
+        for (int r = 0; r < kRowBatch; ++r)
+            if (i0 + r < dv) s[r] = load4(S + size_t(i0 + r) * dk + 4 * lane);
+        float vr[kRowBatch];
+#pragma unroll
+        for (int r = 0; r < kRowBatch; ++r) vr[r] = (i0 + r < dv) ? to_f32(vrow[i0 + r]) : 0.f;
+        float p[kRowBatch], rq[kRowBatch];
+#pragma unroll
+        for (int r = 0; r < kRowBatch; ++r) {
+            if (i0 + r < dv) {
+                p[r] = s[r].x * kf[0] + s[r].y * kf[1] + s[r].z * kf[2] + s[r].w * kf[3];
+                rq[r] = s[r].x * qf[0] + s[r].y * qf[1] + s[r].z * qf[2] + s[r].w * qf[3];
+            } else {
+                p[r] = rq[r] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) {
+#pragma unroll
+            for (int r = 0; r < kRowBatch; ++r) {
+                p[r] += __shfl_xor_sync(0xffffffffu, p[r], m);
+                rq[r] += __shfl_xor_sync(0xffffffffu, rq[r], m);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < kRowBatch; ++r) {
+            if (i0 + r >= dv) continue;
+            const float u = b * (vr[r] - alpha * p[r]);
+            float4 sn;
+            sn.x = fmaf(alpha, s[r].x, u * kf[0]);
+            sn.y = fmaf(alpha, s[r].y, u * kf[1]);
+            sn.z = fmaf(alpha, s[r].z, u * kf[2]);
+            sn.w = fmaf(alpha, s[r].w, u * kf[3]);
+            store4(S + size_t(i0 + r) * dk + 4 * lane, sn);
+            if (lane == r) orow[i0 + r] = from_f32<T>(fmaf(alpha, rq[r], u * kq));
+        }
+    }
+}
+
+// Generic d_k <= 256: warp per row, lane l holds elements l, l+32, ...
+template <typename T>
+__global__ void __launch_bounds__(kDecodeWarps * 32)
+decode_generic_kernel(int32_t hk, int32_t hv, int32_t dk, int32_t dv, const T *__restrict__ q,
+                      const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ g,
+                      const float *__restrict__ beta, float *__restrict__ state, T *__restrict__ o) {
+    constexpr int kMaxPer = 8;  // 8 * 32 = 256 elements
+    const int unit = blockIdx.x;
+    const int n = unit / hv, h = unit % hv;
+    const int hq = h / (hv / hk);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float kf[kMaxPer], qf[kMaxPer];
+    float kq = 0.f;
+#pragma unroll
+    for (int e = 0; e < kMaxPer; ++e) {
+        const int j = lane + 32 * e;
+        kf[e] = j < dk ? to_f32(k[(size_t(n) * hk + hq) * dk + j]) : 0.f;
+        qf[e] = j < dk ? to_f32(q[(size_t(n) * hk + hq) * dk + j]) : 0.f;
+        kq += kf[e] * qf[e];
+    }
+    kq = warp_sum(kq);
+    const float alpha = __expf(fmaxf(g[unit], kGFloor));
+    const float b = beta[unit];
+    float *S = state + size_t(unit) * dv * dk;
+    for (int i = warp; i < dv; i += kDecodeWarps) {
+        float s[kMaxPer];
+        float p = 0.f, rq = 0.f;
+#pragma unroll
+        for (int e = 0; e < kMaxPer; ++e) {
+            const int j = lane + 32 * e;
+            s[e] = j < dk ? S[size_t(i) * dk + j] : 0.f;
+            p += s[e] * kf[e];
+            rq += s[e] * qf[e];
+        }
+        p = warp_sum(p);
+        rq = warp_sum(rq);
+        const float u = b * (to_f32(v[size_t(unit) * dv + i]) - alpha * p);
+#pragma unroll
+        for (int e = 0; e < kMaxPer; ++e) {
+            const int j = lane + 32 * e;
+            if (j < dk) S[size_t(i) * dk + j] = fmaf(alpha, s[e], u * kf[e]);
+        }
+        if (lane == 0) o[size_t(unit) * dv + i] = from_f32<T>(fmaf(alpha, rq, u * kq));
+    }
+}
+
+cudaError_t launch_decode(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
+                          const void *q, const void *k, const void *v, const float *g, const float *beta,
+                          float *state, void *o, cudaStream_t stream) {
+    const int64_t units = int64_t(n) * hv;
+    if (units > INT32_MAX) return cudaErrorInvalidValue;
+    const dim3 grid(static_cast<unsigned>(units)), block(kDecodeWarps * 32);
+    if (dk == 128) {
+        if (dtype == GDN_DTYPE_BF16)
+            decode_d128_kernel<__nv_bfloat16><<<grid, block, 0, stream>>>(
+                hk, hv, dv, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+                static_cast<const __nv_bfloat16 *>(v), g, beta, state, static_cast<__nv_bfloat16 *>(o));
+        else
+            decode_d128_kernel<float><<<grid, block, 0, stream>>>(
+                hk, hv, dv, static_cast<const float *>(q), static_cast<const float *>(k),
+                static_cast<const float *>(v), g, beta, state, static_cast<float *>(o));
+    } else {
+        if (dtype == GDN_DTYPE_BF16)
+            decode_generic_kernel<__nv_bfloat16><<<grid, block, 0, stream>>>(
+                hk, hv, dk, dv, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+                static_cast<const __nv_bfloat16 *>(v), g, beta, state, static_cast<__nv_bfloat16 *>(o));
+        else
+            decode_generic_kernel<float><<<grid, block, 0, stream>>>(
+                hk, hv, dk, dv, static_cast<const float *>(q), static_cast<const float *>(k),
+                static_cast<const float *>(v), g, beta, state, static_cast<float *>(o));
+    }
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

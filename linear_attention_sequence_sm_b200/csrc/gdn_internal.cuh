@@ -1,0 +1,96 @@
+// gdn_internal.cuh -- declarations shared by the translation units of
+// libgdn.so (host launch layer and kernels).  Not part of the public ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gdn.h"
+
+namespace gdn {
+
+// Floor applied to the log-decay g inside the kernels: exp(-20) ~ 2.1e-9 is
+// below fp32 resolution relative to the state, and the floor keeps the
+// chunk-local prefix sums of g finite (g = -inf would give -inf - -inf).
+constexpr float kGFloor = -20.0f;
+
+// ---------------------------------------------------------------------------
+// Workspace layout of gdn_chunk_forward (all offsets 256-byte aligned).
+//   [0, 256)              WsHeader
+//   seq_order [N]         sequences, longest first (ties by index)
+//   seq_start [N]         first token of each sequence
+//   seq_len   [N]         tokens of each sequence
+// ---------------------------------------------------------------------------
+struct WsHeader {
+    int32_t status;        // GDN_OK or GDN_ERR_DEVICE_CHECK
+    int32_t bad_index;     // first offending cu_seqlens index (diagnostics)
+    uint32_t next_unit;    // work counter of the persistent prefill kernels
+    int32_t num_seqs;
+    int32_t pad[60];
+};
+static_assert(sizeof(WsHeader) == 256, "header must be 256 bytes");
+
+struct WsLayout {
+    size_t order_off, start_off, len_off, total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline WsLayout ws_layout(int32_t num_seqs) {
+    WsLayout L;
+    size_t off = 256;
+    L.order_off = off; off = align256(off + 4 * size_t(num_seqs));
+    L.start_off = off; off = align256(off + 4 * size_t(num_seqs));
+    L.len_off = off;   off = align256(off + 4 * size_t(num_seqs));
+    L.total = off;
+    return L;
+}
+
+// Pointers into the workspace, as the kernels see them.
+struct Sched {
+    WsHeader *hdr;
+    const int32_t *order;
+    const int32_t *start;
+    const int32_t *len;
+};
+
+// Element access for the two storage types.
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Launch counter (defined in gdn_api.cu).
+void count_launch();
+
+// Prefill schedule: validates cu_seqlens (or synthesises the batched layout)
+// and fills the workspace tables.  One block.
+cudaError_t launch_schedule(const gdn_shape_t &s, const int32_t *cu_seqlens, void *workspace,
+                            cudaStream_t stream);
+
+struct PrefillArgs {
+    int32_t num_seqs, hk, hv, dk, dv, chunk, dtype;
+    const void *q, *k, *v;
+    const float *g, *beta, *s0;
+    void *o;
+    float *s_final;
+    Sched sched;
+};
+
+// fp32 CUDA-core chunkwise kernel (any dtype, d_k, d_v <= 128, C in {16,32,64}).
+cudaError_t launch_chunk_simt(const PrefillArgs &a, cudaStream_t stream, int num_sms);
+
+// Tensor-core chunkwise kernel (bf16, d = 128, C = 64).
+cudaError_t launch_chunk_tc(const PrefillArgs &a, cudaStream_t stream, int num_sms);
+bool chunk_tc_supported(const gdn_shape_t &s);
+
+// Decode step.
+cudaError_t launch_decode(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
+                          const void *q, const void *k, const void *v, const float *g, const float *beta,
+                          float *state, void *o, cudaStream_t stream);
+
+}  // namespace gdn

@@ -1,0 +1,193 @@
+"""Python binding of libgdn.so (the gated delta rule on B200).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in ``include/gdn.h``.  PyTorch provides
+device memory and streams.  There is no CPU fallback: if the library is
+missing, importing this module raises.
+
+Layouts (row-major, token-major):
+  q, k  [B, T, Hk, d_k] (or [T, Hk, d_k] packed with cu_seqlens)
+  v, o  [B, T, Hv, d_v]
+  g, beta [B, T, Hv] fp32;  states [N, Hv, d_v, d_k] fp32
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn.so")
+
+GDN_OK = 0
+GDN_ERR_INVALID_ARGUMENT = 1
+GDN_ERR_UNSUPPORTED = 2
+GDN_ERR_MISALIGNED = 3
+GDN_ERR_WORKSPACE_TOO_SMALL = 4
+GDN_ERR_CUDA = 5
+GDN_ERR_DEVICE_CHECK = 6
+GDN_DTYPE_F32 = 0
+GDN_DTYPE_BF16 = 1
+GDN_FLAG_FORCE_SIMT = 1
+
+EXPORTED = ("gdn_chunk_forward_workspace_size", "gdn_chunk_forward", "gdn_read_device_status",
+            "gdn_decode_step", "gdn_status_string", "gdn_last_error_message", "gdn_launch_count")
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{message} [status {status}]")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("seq_len", ctypes.c_int32), ("num_seqs", ctypes.c_int32),
+                ("num_qk_heads", ctypes.c_int32), ("num_v_heads", ctypes.c_int32),
+                ("head_dim_k", ctypes.c_int32), ("head_dim_v", ctypes.c_int32),
+                ("chunk_size", ctypes.c_int32), ("dtype", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+
+
+def _load(path: str = LIB_PATH):
+    if not os.path.exists(path):
+        raise ImportError(f"libgdn.so not found at {path}; build it with "
+                          "`python -m linear_attention_sequence_sm_b200.build` (no CPU fallback exists)")
+    lib = ctypes.CDLL(path)
+    vp, i32, st = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int
+    lib.gdn_chunk_forward_workspace_size.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(ctypes.c_size_t)]
+    lib.gdn_chunk_forward_workspace_size.restype = st
+    lib.gdn_chunk_forward.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                      ctypes.c_size_t, vp]
+    lib.gdn_chunk_forward.restype = st
+    lib.gdn_read_device_status.argtypes = [vp, ctypes.POINTER(i32), vp]
+    lib.gdn_read_device_status.restype = st
+    lib.gdn_decode_step.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.gdn_decode_step.restype = st
+    lib.gdn_status_string.argtypes = [st]
+    lib.gdn_status_string.restype = ctypes.c_char_p
+    lib.gdn_last_error_message.argtypes = []
+    lib.gdn_last_error_message.restype = ctypes.c_char_p
+    lib.gdn_launch_count.argtypes = []
+    lib.gdn_launch_count.restype = ctypes.c_uint64
+    return lib
+
+
+LIB = _load()
+
+
+def _check(status: int):
+    if status != GDN_OK:
+        name = LIB.gdn_status_string(status).decode()
+        raise GdnError(status, f"{name}: {LIB.gdn_last_error_message().decode()}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return GDN_DTYPE_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _stream_handle(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, dtype=None, device=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def make_shape(q, v, cu_seqlens=None, chunk_size=64, force_simt=False) -> Shape:
+    if cu_seqlens is not None:
+        T = q.shape[-3]
+        B, N = 1, cu_seqlens.shape[0] - 1
+    else:
+        if q.dim() != 4:
+            raise ValueError("batched q must be [B, T, Hk, d_k]")
+        B, T = q.shape[0], q.shape[1]
+        N = B
+    return Shape(B, T, N, q.shape[-2], v.shape[-2], q.shape[-1], v.shape[-1], chunk_size, _dtype_code(q),
+                 GDN_FLAG_FORCE_SIMT if force_simt else 0)
+
+
+def workspace_size(shape: Shape) -> int:
+    n = ctypes.c_size_t(0)
+    _check(LIB.gdn_chunk_forward_workspace_size(ctypes.byref(shape), ctypes.byref(n)))
+    return n.value
+
+
+def chunk_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_size=64,
+                  output_final_state=True, out=None, final_state=None, workspace=None, force_simt=False,
+                  stream=None):
+    """Chunkwise prefill.  Returns (o, final_state or None).  Asynchronous on
+    ``stream`` (default: the current stream)."""
+    dev = q.device
+    dt = q.dtype
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, dt, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(initial_state, "initial_state", torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    if k.shape != q.shape:
+        raise ValueError("k must have the shape of q")
+    shape = make_shape(q, v, cu_seqlens, chunk_size, force_simt)
+    if out is None:
+        out = torch.empty(v.shape, dtype=dt, device=dev)
+    _need(out, "out", dt, dev)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((shape.num_seqs, shape.num_v_heads, shape.head_dim_v, shape.head_dim_k),
+                                  dtype=torch.float32, device=dev)
+    _need(final_state, "final_state", torch.float32, dev)
+    nbytes = workspace_size(shape)
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _check(LIB.gdn_chunk_forward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                 _ptr(initial_state), _ptr(cu_seqlens), _ptr(out), _ptr(final_state),
+                                 _ptr(workspace), workspace.numel(), _stream_handle(stream)))
+    return out, final_state
+
+
+def read_device_status(workspace, stream=None) -> int:
+    """Synchronise the stream and return the device status word of the last
+    gdn_chunk_forward that used ``workspace``."""
+    st = ctypes.c_int32(-1)
+    _check(LIB.gdn_read_device_status(_ptr(workspace), ctypes.byref(st), _stream_handle(stream)))
+    return st.value
+
+
+def decode_step(q, k, v, g, beta, state, out=None, stream=None):
+    """One token per sequence; ``state`` [N, Hv, d_v, d_k] fp32 is updated in
+    place.  Returns o [N, Hv, d_v]."""
+    dev, dt = q.device, q.dtype
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, dt, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(state, "state", torch.float32, dev)
+    if out is None:
+        out = torch.empty(v.shape, dtype=dt, device=dev)
+    _need(out, "out", dt, dev)
+    N, hk, dk = q.shape
+    hv, dv = v.shape[1], v.shape[2]
+    _check(LIB.gdn_decode_step(N, hk, hv, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                               _ptr(beta), _ptr(state), _ptr(out), _stream_handle(stream)))
+    return out
+
+
+def launch_count() -> int:
+    return int(LIB.gdn_launch_count())

@@ -1,0 +1,133 @@
+"""The C-ABI library loads and exports every declared symbol; host-side
+argument checks reject bad calls before any CUDA work (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+@pytest.fixture(scope="module")
+def gdn():
+    from linear_attention_sequence_sm_b200 import build
+    build.build()
+    from linear_attention_sequence_sm_b200 import gdn as mod
+    return mod
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    assert "gdn_chunk_forward" in names and "gdn_decode_step" in names
+    assert len(names) >= 7
+
+
+def test_library_exports_every_declared_symbol(gdn):
+    lib = ctypes.CDLL(gdn.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(gdn.EXPORTED) == set(declared_functions())
+
+
+def test_status_strings(gdn):
+    for code in range(7):
+        s = gdn.LIB.gdn_status_string(code).decode()
+        assert s.startswith("GDN_")
+    assert gdn.LIB.gdn_status_string(99).decode() == "GDN_ERR_UNKNOWN"
+
+
+def _shape(gdn, **kw):
+    base = dict(batch=2, seq_len=64, num_seqs=2, num_qk_heads=2, num_v_heads=4, head_dim_k=128,
+                head_dim_v=128, chunk_size=64, dtype=gdn.GDN_DTYPE_BF16, flags=0)
+    base.update(kw)
+    return gdn.Shape(**base)
+
+
+def test_workspace_size(gdn):
+    n = gdn.workspace_size(_shape(gdn))
+    assert n >= 256 and n % 256 == 0
+    big = gdn.workspace_size(_shape(gdn, batch=1, num_seqs=10000, seq_len=100000))
+    assert big > n
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(num_v_heads=3), 1),          # Hv % Hk != 0
+    (dict(dtype=7), 1),                # unknown dtype
+    (dict(chunk_size=48), 2),          # unsupported chunk
+    (dict(head_dim_k=256), 2),         # d_k > 128
+    (dict(num_qk_heads=0), 1),
+    (dict(seq_len=-1), 1),
+])
+def test_shape_rejected(gdn, kw, code):
+    n = ctypes.c_size_t(0)
+    st = gdn.LIB.gdn_chunk_forward_workspace_size(ctypes.byref(_shape(gdn, **kw)), ctypes.byref(n))
+    assert st == code
+    assert gdn.LIB.gdn_last_error_message().decode() != ""
+
+
+FAKE = 0x10000000  # a 256-byte aligned address; never dereferenced: every call below fails validation first
+
+
+def _call(gdn, shape, **over):
+    p = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, s0=None, cu=None, o=FAKE, sf=None, ws=FAKE,
+             wsb=1 << 20)
+    p.update(over)
+    vp = ctypes.c_void_p
+    return gdn.LIB.gdn_chunk_forward(ctypes.byref(shape), vp(p["q"]), vp(p["k"]), vp(p["v"]), vp(p["g"]),
+                                     vp(p["beta"]), vp(p["s0"]), vp(p["cu"]), vp(p["o"]), vp(p["sf"]),
+                                     vp(p["ws"]), p["wsb"], None)
+
+
+def test_null_and_misaligned_pointers(gdn):
+    s = _shape(gdn)
+    assert _call(gdn, s, q=None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert _call(gdn, s, ws=None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert _call(gdn, s, v=FAKE + 8) == gdn.GDN_ERR_MISALIGNED
+    assert "v is not 16-byte aligned" in gdn.LIB.gdn_last_error_message().decode()
+    assert _call(gdn, s, ws=FAKE + 16) == gdn.GDN_ERR_MISALIGNED
+    assert _call(gdn, s, wsb=16) == gdn.GDN_ERR_WORKSPACE_TOO_SMALL
+    # varlen needs batch 1; batched needs num_seqs == batch
+    assert _call(gdn, _shape(gdn, batch=2), cu=FAKE) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert _call(gdn, _shape(gdn, num_seqs=3)) == gdn.GDN_ERR_INVALID_ARGUMENT
+
+
+def test_decode_argument_checks(gdn):
+    vp = ctypes.c_void_p
+    f = gdn.LIB.gdn_decode_step
+    args = [vp(FAKE)] * 7 + [None]
+    assert f(4, 2, 3, 128, 128, 1, *args) == gdn.GDN_ERR_INVALID_ARGUMENT   # Hv % Hk
+    assert f(4, 2, 4, 512, 128, 1, *args) == gdn.GDN_ERR_UNSUPPORTED        # d_k > 256
+    assert f(4, 2, 4, 128, 128, 5, *args) == gdn.GDN_ERR_INVALID_ARGUMENT   # dtype
+    bad = [vp(FAKE)] * 5 + [vp(FAKE + 4), vp(FAKE), None]
+    assert f(4, 2, 4, 128, 128, 1, *bad) == gdn.GDN_ERR_MISALIGNED
+    assert f(0, 2, 4, 128, 128, 1, *args) == gdn.GDN_OK                     # nothing to do
+
+
+def test_no_device_reports_cuda_error(gdn):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("only meaningful without a GPU")
+    assert _call(gdn, _shape(gdn)) == gdn.GDN_ERR_CUDA
+
+
+def test_launch_counter_is_monotonic(gdn):
+    a = gdn.launch_count()
+    assert gdn.launch_count() >= a
+
+
+def test_product_path_has_no_oracle_or_cpu_fallback():
+    """The package and its CUDA sources never import, load or include the oracle."""
+    pkg = os.path.join(ROOT, "linear_attention_sequence_sm_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, fn)).read()
+                assert not re.search(r"(from|import)\s+oracle|gdn_oracle|libgdn_oracle", text), fn
