@@ -45,6 +45,8 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--decode-steps", type=int, default=512)
+    p.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+                   help="time only one of the two paths (used by profiling commands)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
@@ -258,18 +260,22 @@ def run_ours(args):
         gdn.chunk_forward(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], initial_state=None, out=o,
                           final_state=sf, workspace=ws, chunk_size=w.chunk)
 
-    for _ in range(max(3, args.warmup)):
-        step()
-    torch.cuda.synchronize(device)
-    barrier(world, device)
-    torch.cuda.synchronize(device)
-    n0 = gdn.launch_count()
-    with ClockSampler(device.index) as clocks:
-        ms = timed(step, args.steps, stream)
+    ms = ms_max = float("nan")
+    launches = 0
+    clocks = ClockSampler(device.index)
+    if args.only in ("all", "prefill"):
+        for _ in range(max(3, args.warmup)):
+            step()
         torch.cuda.synchronize(device)
-    launches = gdn.launch_count() - n0
-    barrier(world, device)
-    ms_max = max_over_ranks(ms, device, world)
+        barrier(world, device)
+        torch.cuda.synchronize(device)
+        n0 = gdn.launch_count()
+        with clocks:
+            ms = timed(step, args.steps, stream)
+            torch.cuda.synchronize(device)
+        launches = gdn.launch_count() - n0
+        barrier(world, device)
+        ms_max = max_over_ranks(ms, device, world)
     tokens = w.total_tokens
     value = world * tokens / (ms_max / 1e3)
     flops = USEFUL_FLOPS_PER_VHEAD_TOKEN * tokens * w.hv
@@ -282,39 +288,43 @@ def run_ours(args):
                 "flops_per_launch": flops, "algorithmic_bytes_per_launch": prefill_bytes(w)}
 
     # ---- decode: 256 sequences, fp32 state 512 MiB, in place ----
+    decode = None
     dw = I.decode_bf16()
-    gen = torch.Generator(device=device)
-    gen.manual_seed(dw.seed + rank)
-    state = torch.randn((dw.num_seqs, dw.hv, dw.d, dw.d), generator=gen, device=device) * dw.s0_std
-    ring = [{k: v.to(device) for k, v in I.make_decode_inputs(dw, s).items()} for s in range(8)]
-    od = torch.empty((dw.num_seqs, dw.hv, dw.d), dtype=torch.bfloat16, device=device)
-    it = [0]
+    if args.only == "prefill":
+        args.decode_steps = 0
+    if args.decode_steps > 0:
+        gen = torch.Generator(device=device)
+        gen.manual_seed(dw.seed + rank)
+        state = torch.randn((dw.num_seqs, dw.hv, dw.d, dw.d), generator=gen, device=device) * dw.s0_std
+        ring = [{k: v.to(device) for k, v in I.make_decode_inputs(dw, s).items()} for s in range(8)]
+        od = torch.empty((dw.num_seqs, dw.hv, dw.d), dtype=torch.bfloat16, device=device)
+        it = [0]
 
-    def dstep():
-        x = ring[it[0] % len(ring)]
-        it[0] += 1
-        gdn.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state, out=od)
+        def dstep():
+            x = ring[it[0] % len(ring)]
+            it[0] += 1
+            gdn.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state, out=od)
 
-    for _ in range(max(3, args.warmup)):
-        dstep()
-    torch.cuda.synchronize(device)
-    with ClockSampler(device.index) as dclocks:
-        dms = timed(dstep, args.decode_steps, stream)
-    dms = max_over_ranks(dms, device, world)
-    dbytes = decode_bytes(dw)
-    dgbs = dbytes / (dms / 1e3) / 1e9
-    decode = {"value": world * dgbs, "unit": "GB/s", "ms_per_step": dms, "steps": args.decode_steps,
-              "tokens_per_s": world * dw.num_seqs / (dms / 1e3), "workload": dw.name,
-              "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                           "frac": dgbs / peaks["hbm_gbs"], "traffic": kernel_traffic("gdn_decode"),
-                           "kernel": "gdn_decode", "peak_source": f"{peak_src} HBM copy",
-                           "bytes_per_launch": dbytes},
-              "clocks": dclocks.summary()}
-    del state
+        for _ in range(max(3, args.warmup)):
+            dstep()
+        torch.cuda.synchronize(device)
+        with ClockSampler(device.index) as dclocks:
+            dms = timed(dstep, args.decode_steps, stream)
+        dms = max_over_ranks(dms, device, world)
+        dbytes = decode_bytes(dw)
+        dgbs = dbytes / (dms / 1e3) / 1e9
+        decode = {"value": world * dgbs, "unit": "GB/s", "ms_per_step": dms, "steps": args.decode_steps,
+                  "tokens_per_s": world * dw.num_seqs / (dms / 1e3), "workload": dw.name,
+                  "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                               "frac": dgbs / peaks["hbm_gbs"], "traffic": kernel_traffic("gdn_decode"),
+                               "kernel": "gdn_decode", "peak_source": f"{peak_src} HBM copy",
+                               "bytes_per_launch": dbytes},
+                  "clocks": dclocks.summary()}
+        del state
 
     # ---- end to end through the public API with host buffers ----
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.only != "decode":
         pin = {k: v.pin_memory() for k, v in host.items() if v is not None}
         o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
         sf_host = torch.empty(sf.shape, dtype=sf.dtype).pin_memory()
@@ -337,7 +347,7 @@ def run_ours(args):
                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only != "decode":
         cpu = cpu_oracle_sample(w, host, args.cpu_seconds)
 
     if rank == 0:
