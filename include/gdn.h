@@ -129,6 +129,32 @@ GDN_API gdn_status_t gdn_chunk_forward(const gdn_shape_t *shape,
                                void *workspace, size_t workspace_bytes,
                                void *stream);
 
+/* gdn_chunk_forward without a caller-provided workspace.  The source pages
+ * have no counterpart for this entry point: it exists for callers that
+ * cannot allocate device memory, such as a plugin that a host runtime hands
+ * only tensor pointers and no allocator, or a serving loop that must not
+ * call cudaMalloc on the request path (cudaMalloc may synchronise the whole
+ * device).  The scratch the prefill needs (schedule tables and status word)
+ * lives instead in a device array built into the library: 196,864 bytes on
+ * every GPU that loads the library, held until the process exits, enough
+ * for at most 16,384 sequences per call (more returns GDN_ERR_UNSUPPORTED
+ * with a message; nothing is launched).  Arguments and results are those of
+ * gdn_chunk_forward.  The first call on a device looks up the array's device
+ * address once (cudaGetSymbolAddress, with that device current); make that
+ * first call before any stream capture.  No call allocates or frees memory.
+ * All calls on a device share the one array: calls that overlap on the GPU
+ * (two streams, or two host threads) race on it and give wrong results, so
+ * serialise them.  Each call re-initialises the scratch before use, so what
+ * an earlier call left there is harmless.  The device status word of a
+ * cu_seqlens check cannot be read back through this entry point. */
+GDN_API gdn_status_t gdn_chunk_forward_noalloc(const gdn_shape_t *shape,
+                                       const void *q, const void *k, const void *v,
+                                       const float *g, const float *beta,
+                                       const float *initial_state,
+                                       const int32_t *cu_seqlens,
+                                       void *o, float *final_state,
+                                       void *stream);
+
 /* Reads the device status word that gdn_chunk_forward left in `workspace`
  * (GDN_OK or GDN_ERR_DEVICE_CHECK) into *device_status.  Synchronises
  * `stream`.  This is the only entry point that waits for the GPU. */

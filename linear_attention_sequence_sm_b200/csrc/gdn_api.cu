@@ -23,6 +23,12 @@ static gdn_status_t fail(gdn_status_t st, const char *fmt, ...) {
     return st;
 }
 
+// Records the per-thread error text for entry points defined in other files.
+gdn_status_t set_error(gdn_status_t st, const char *text) {
+    snprintf(g_msg, sizeof(g_msg), "%s", text);
+    return st;
+}
+
 static gdn_status_t cuda_fail(cudaError_t e, const char *what) {
     return fail(GDN_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }

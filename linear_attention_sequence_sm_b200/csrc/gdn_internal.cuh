@@ -64,6 +64,10 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
+// Sets the per-thread error text returned by gdn_last_error_message
+// (defined in gdn_api.cu) and returns `st`.
+gdn_status_t set_error(gdn_status_t st, const char *text);
+
 // Launch counter (defined in gdn_api.cu).
 void count_launch();
 

@@ -1,0 +1,82 @@
+// gdn_noalloc.cu -- gdn_chunk_forward for callers that cannot allocate.
+//
+// Some callers have no way to obtain device memory for a workspace: a
+// plugin inside a host runtime that hands it only the tensors' pointers and
+// no allocator, or serving code whose memory is fixed up front and which
+// must not call cudaMalloc on the request path (cudaMalloc can synchronise
+// the device and stall every stream).  For them this file keeps the
+// prefill's scratch (the schedule tables and the status word) in a fixed
+// device array that the library owns, so the call needs only inputs and
+// outputs.
+//
+// The array lives in every GPU that loads the library, for the life of the
+// process, and is shared by all calls on that device: calls that overlap on
+// the GPU (different streams, or host threads racing) overwrite each
+// other's scratch and give wrong results.  Each call re-initialises what it
+// needs (the schedule kernel rewrites the tables, the status word and the
+// work counter before the prefill kernel reads them), so stale contents from
+// an earlier call do no harm.
+#include <cstdio>
+#include <mutex>
+
+#include "gdn_internal.cuh"
+
+namespace gdn {
+
+// Scratch of the prefill schedule for up to kNoAllocMaxSeqs sequences:
+// a 256-byte header plus three int32 tables of that length.
+constexpr int32_t kNoAllocMaxSeqs = 16384;
+constexpr size_t kNoAllocScratchBytes = 256 + 3 * 4 * size_t(kNoAllocMaxSeqs);
+static_assert(kNoAllocScratchBytes % 256 == 0, "scratch size must keep 256-byte alignment");
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch per device ordinal, resolved once per
+// device with that device current (the host-side symbol is only a stand-in
+// and must never be passed to a kernel).
+constexpr int kMaxDevices = 64;
+static void *g_scratch_ptr[kMaxDevices];
+static std::mutex g_scratch_mu;
+
+static cudaError_t scratch_address(void **out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace gdn
+
+extern "C" GDN_API gdn_status_t gdn_chunk_forward_noalloc(const gdn_shape_t *shape, const void *q, const void *k,
+                                                          const void *v, const float *g, const float *beta,
+                                                          const float *initial_state, const int32_t *cu_seqlens,
+                                                          void *o, float *final_state, void *stream) {
+    using namespace gdn;
+    if (shape && shape->num_seqs > kNoAllocMaxSeqs) {
+        char msg[160];
+        snprintf(msg, sizeof(msg),
+                 "gdn_chunk_forward_noalloc handles at most %d sequences per call (got %d); "
+                 "use gdn_chunk_forward with a caller-allocated workspace",
+                 int(kNoAllocMaxSeqs), int(shape->num_seqs));
+        return set_error(GDN_ERR_UNSUPPORTED, msg);
+    }
+    void *scratch = nullptr;
+    const cudaError_t e = scratch_address(&scratch);
+    if (e != cudaSuccess) {
+        char msg[200];
+        snprintf(msg, sizeof(msg), "resolving the device address of the built-in scratch array failed: %s",
+                 cudaGetErrorString(e));
+        return set_error(GDN_ERR_CUDA, msg);
+    }
+    return gdn_chunk_forward(shape, q, k, v, g, beta, initial_state, cu_seqlens, o, final_state, scratch,
+                             kNoAllocScratchBytes, stream);
+}

@@ -32,7 +32,8 @@ GDN_DTYPE_BF16 = 1
 GDN_FLAG_FORCE_SIMT = 1
 
 EXPORTED = ("gdn_chunk_forward_workspace_size", "gdn_chunk_forward", "gdn_read_device_status",
-            "gdn_decode_step", "gdn_status_string", "gdn_last_error_message", "gdn_launch_count")
+            "gdn_decode_step", "gdn_status_string", "gdn_last_error_message", "gdn_launch_count",
+            "gdn_chunk_forward_noalloc")
 
 
 class GdnError(RuntimeError):
@@ -59,6 +60,8 @@ def _load(path: str = LIB_PATH):
     lib.gdn_chunk_forward.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                       ctypes.c_size_t, vp]
     lib.gdn_chunk_forward.restype = st
+    lib.gdn_chunk_forward_noalloc.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.gdn_chunk_forward_noalloc.restype = st
     lib.gdn_read_device_status.argtypes = [vp, ctypes.POINTER(i32), vp]
     lib.gdn_read_device_status.restype = st
     lib.gdn_decode_step.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]
@@ -159,6 +162,35 @@ def chunk_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_s
     _check(LIB.gdn_chunk_forward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
                                  _ptr(initial_state), _ptr(cu_seqlens), _ptr(out), _ptr(final_state),
                                  _ptr(workspace), workspace.numel(), _stream_handle(stream)))
+    return out, final_state
+
+
+def chunk_forward_noalloc(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_size=64,
+                          output_final_state=True, out=None, final_state=None, force_simt=False, stream=None):
+    """chunk_forward for callers that cannot allocate device scratch: the
+    library's built-in scratch array stands in for the workspace (at most
+    16,384 sequences; calls that overlap on the GPU race on that array).
+    Output tensors are still the caller's (allocated here only when not
+    given)."""
+    dev = q.device
+    dt = q.dtype
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, dt, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(initial_state, "initial_state", torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    shape = make_shape(q, v, cu_seqlens, chunk_size, force_simt)
+    if out is None:
+        out = torch.empty(v.shape, dtype=dt, device=dev)
+    _need(out, "out", dt, dev)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((shape.num_seqs, shape.num_v_heads, shape.head_dim_v, shape.head_dim_k),
+                                  dtype=torch.float32, device=dev)
+    _need(final_state, "final_state", torch.float32, dev)
+    _check(LIB.gdn_chunk_forward_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                         _ptr(initial_state), _ptr(cu_seqlens), _ptr(out), _ptr(final_state),
+                                         _stream_handle(stream)))
     return out, final_state
 
 
