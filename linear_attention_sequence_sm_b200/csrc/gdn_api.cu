@@ -142,6 +142,7 @@ gdn_status_t gdn_chunk_forward(const gdn_shape_t *s, const void *q, const void *
     a.dv = s->head_dim_v;
     a.chunk = s->chunk_size;
     a.dtype = s->dtype;
+    a.tokens = int32_t(tokens);
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.s0 = initial_state; a.o = o; a.s_final = final_state;
     char *ws = static_cast<char *>(workspace);
     a.sched.hdr = reinterpret_cast<WsHeader *>(ws);

@@ -1,7 +1,525 @@
-// gdn_chunk_tc.cu -- tensor-core (tcgen05/TMEM) chunkwise kernel: not yet built.
+// gdn_chunk_tc.cu -- chunkwise gated delta rule on the 5th-generation tensor
+// cores (tcgen05.mma, fp32 accumulators in tensor memory), bf16 inputs,
+// d_k = d_v = 128, chunk C = 64.
+//
+// Chunk algebra (per chunk of L <= 64 tokens r, j with start state S, as in
+// the fp32 kernel): G = prefix sums of g, gamma = e^G,
+// Gamma_rj = e^(G_r - G_j); A_rj = beta_r Gamma_rj (k_r.k_j) (j < r);
+// T = (I + A)^-1; W = T diag(beta gamma) K; U~ = T diag(beta) V;
+// U = U~ - W S^T; O = diag(gamma) Q S^T + (Q K^T (.) Gamma) U;
+// S <- gamma_C S + U^T diag(e^(G_C - G)) K.  This is the WY representation of
+// the DeltaNet transitions with per-chunk cumulative decay ("Gated Attention
+// Architectures", sections 2 and 3) and the decay-masked chunk output of its
+// section 1, applied to the corrected values U.
+//
+// Mapping to the tensor cores.  Every contraction is issued with M = 128 so
+// that the accumulator row is the tensor-memory lane:
+//   (1) [K;Q] K^T      -> Gram (lanes 0-63: K K^T, 64-127: Q K^T)   128x64x128
+//   (2) W^T = K^T T'^T  (T' = T diag(beta gamma))                   128x64x64
+//   (3) U~^T = V^T T''^T (T'' = T diag(beta))                       128x64x64
+//   (4) U^T = U~^T - S W^T   (accumulates into (3), A negated)      128x64x128
+//   (5) X1 = S Q^T                                                   128x64x128
+//   (6) X2 = U^T P^T,  P = Q K^T (.) Gamma                           128x64x64
+//   (7) dS = (U^T diag(lambda)) K,  lambda_j = e^(G_C - G_j)         128x128x64
+// O[r][i] = gamma_r X1[i][r] + X2[i][r];  S <- gamma_C S + dS.
+// Operands are bf16 in 128-byte-swizzled shared memory; q, k, v tiles arrive
+// by TMA (no multicast); the fp32 state S lives in registers (thread = state
+// row, half of the key columns) and is re-staged as a bf16 operand each
+// chunk.  The triangular inverse runs on the CUDA cores in fp32 (16 x 16
+// diagonal blocks by forward substitution, then the off-diagonal blocks).
+//
+// One CTA per SM (the shared-memory footprint forces it) owns a unit
+// (sequence, value head) at a time, taking units longest sequence first from
+// an atomic counter, and walks the unit's chunks in order.  Every wait on an
+// mbarrier is bounded; a timeout records GDN_ERR_DEVICE_CHECK (bad_index -2)
+// in the workspace status word and the CTA frees its tensor memory and exits.
+#include <cuda.h>
+
+#include <mutex>
+
 #include "gdn_internal.cuh"
+#include "gdn_sm100.cuh"
 
 namespace gdn {
-bool chunk_tc_supported(const gdn_shape_t &) { return false; }
-cudaError_t launch_chunk_tc(const PrefillArgs &, cudaStream_t, int) { return cudaErrorNotSupported; }
+using namespace sm100;
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kLdA = 65;  // fp32 row stride of the A and T scratch matrices
+
+// Shared-memory map (bytes from a 1024-byte-aligned base).  Tiles are
+// 128-byte-swizzled: "atom columns" of 64 bf16 (128 bytes) per row.
+constexpr uint32_t kOffKQ0 = 0;       // [K;Q] chunk buffer 0: 2 atom columns x 128 rows (K 0-63, Q 64-127)
+constexpr uint32_t kOffKQ1 = 32768;   // [K;Q] chunk buffer 1
+constexpr uint32_t kOffV = 65536;     // V: 2 atom columns x 64 rows
+constexpr uint32_t kOffS = 81920;     // S operand (bf16): 2 atom columns x 128 rows (d_v)
+constexpr uint32_t kOffTp = 114688;   // T diag(beta gamma): 64 x 64
+constexpr uint32_t kOffTpp = 122880;  // T diag(beta): 64 x 64
+constexpr uint32_t kOffWT = 131072;   // W^T: 128 rows (d_k) x 64 tokens
+constexpr uint32_t kOffP = 147456;    // P: 64 x 64
+constexpr uint32_t kOffUT = 155648;   // U^T: 128 rows (d_v) x 64 tokens
+constexpr uint32_t kOffUTl = 172032;  // U^T diag(lambda)
+constexpr uint32_t kOffAf = 188416;   // A, fp32 64 x kLdA
+constexpr uint32_t kOffTf = kOffAf + 64 * kLdA * 4;  // T, fp32 64 x kLdA
+constexpr uint32_t kOffY = kOffTf + 64 * kLdA * 4;   // blocked-inverse scratch, 3 x 16 x 16 fp32
+constexpr uint32_t kOffVec = kOffY + 3 * 256 * 4;    // per-token vectors, 8 x 64 fp32
+constexpr uint32_t kOffBar = kOffVec + 8 * 64 * 4;   // 4 mbarriers + tensor-memory slot
+constexpr uint32_t kSmemBytes = kOffBar + 64 + 1024; // + alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 per-block limit");
+
+// Tensor-memory columns (fp32 accumulators, 128 lanes each).
+constexpr uint32_t kColGram = 0, kColW = 64, kColU = 128, kColX1 = 192, kColX2 = 256, kColDS = 320;
+constexpr uint32_t kTmemCols = 512;
+
+constexpr uint32_t kBytesKQ = 4 * 8192;  // four 64 x 64 bf16 boxes
+constexpr uint32_t kBytesV = 2 * 8192;
+
+__device__ __forceinline__ void store_row_bf16(uint32_t tile, int row, int chunk0, const float *x, int nchunks) {
+#pragma unroll
+    for (int c = 0; c < nchunks; ++c) st_shared_v4(tile + sw128_offset(row, chunk0 + c), pack_bf16x8(x + 8 * c));
+}
+
+// T = (I + A)^-1 for the 64 x 64 unit-lower-triangular system, fp32, in
+// shared memory.  Diagonal 16 x 16 blocks B_I = (I + A_II)^-1 by forward
+// substitution (one thread per column), then block rows I = 1..3:
+// T_IJ = -B_I sum_{K=J}^{I-1} A_IK T_KJ.  All threads must call it.
+__device__ void invert_unit_lower(const float *Af, float *Tf, float *Y, int tid) {
+    if (tid < 64) {
+        const int b = tid >> 4, c = tid & 15;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) x[r] = (r == c) ? 1.f : 0.f;
+#pragma unroll
+        for (int j = 0; j < 15; ++j) {
+#pragma unroll
+            for (int r = j + 1; r < 16; ++r) x[r] = fmaf(-Af[(16 * b + r) * kLdA + 16 * b + j], x[j], x[r]);
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Tf[(16 * b + r) * kLdA + 16 * b + c] = x[r];
+    }
+    __syncthreads();
+    for (int I = 1; I < 4; ++I) {
+        for (int e = tid; e < I * 256; e += kThreads) {
+            const int J = e >> 8, r = (e >> 4) & 15, c = e & 15;
+            float acc = 0.f;
+            for (int K = J; K < I; ++K) {
+#pragma unroll
+                for (int m = 0; m < 16; ++m)
+                    acc = fmaf(Af[(16 * I + r) * kLdA + 16 * K + m], Tf[(16 * K + m) * kLdA + 16 * J + c], acc);
+            }
+            Y[e] = acc;
+        }
+        __syncthreads();
+        for (int e = tid; e < I * 256; e += kThreads) {
+            const int J = e >> 8, r = (e >> 4) & 15, c = e & 15;
+            float acc = 0.f;
+            for (int m = 0; m <= r; ++m) acc = fmaf(Tf[(16 * I + r) * kLdA + 16 * I + m], Y[J * 256 + m * 16 + c], acc);
+            Tf[(16 * I + r) * kLdA + 16 * J + c] = -acc;
+        }
+        __syncthreads();
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                            ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(smem);
+    float *Af = reinterpret_cast<float *>(smem + kOffAf);
+    float *Tf = reinterpret_cast<float *>(smem + kOffTf);
+    float *Yb = reinterpret_cast<float *>(smem + kOffY);
+    float *gs = reinterpret_cast<float *>(smem + kOffVec);  // g, then its prefix sums G
+    float *bs = gs + 64;                                   // beta
+    float *gam = gs + 128;                                 // gamma = e^G
+    float *bg = gs + 192;                                  // beta gamma
+    float *lam = gs + 256;                                 // e^(G_C - G), 0 past the sequence end
+    const uint32_t bar_kq0 = sb + kOffBar, bar_kq1 = sb + kOffBar + 8, bar_v = sb + kOffBar + 16,
+                   bar_mma = sb + kOffBar + 24;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + kOffBar + 32);
+    int *s_unit = reinterpret_cast<int *>(smem + kOffBar + 40);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;  // tensor-memory lane = accumulator row of this thread
+    const uint32_t lane_bits = uint32_t(quarter * 32) << 16;
+    WsHeader *hdr = a.sched.hdr;
+    if (hdr->status != GDN_OK) return;
+
+    if (tid == 0) {
+        mbar_init(bar_kq0, 1);
+        mbar_init(bar_kq1, 1);
+        mbar_init(bar_v, 1);
+        mbar_init(bar_mma, 1);
+        fence_mbarrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tslot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+
+    const int hv = a.hv, hk = a.hk, group = hv / hk;
+    const int total_units = a.num_seqs * hv;
+    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(a.o);
+    uint32_t ph_kq0 = 0, ph_kq1 = 0, ph_v = 0, ph_mma = 0;
+    uint32_t pending = 0;  // (tid 0) bit 0/1: KQ buffer load in flight, bit 2: V load in flight
+    bool aborted = false;
+
+    const uint32_t id_gram = idesc_bf16(128, 64, false, false);
+    const uint32_t id_w = idesc_bf16(128, 64, true, false);
+    const uint32_t id_u = idesc_bf16(128, 64, false, true, true);
+    const uint32_t id_x = idesc_bf16(128, 64, false, false);
+    const uint32_t id_ds = idesc_bf16(128, 128, false, true);
+
+    for (;;) {
+        if (tid == 0) *s_unit = int(atomicAdd(&hdr->next_unit, 1u));
+        __syncthreads();
+        const int unit = *s_unit;
+        __syncthreads();
+        if (unit >= total_units) break;
+        const int seq = a.sched.order[unit / hv];
+        const int h = unit % hv, hq = h / group;
+        const int t0 = a.sched.start[seq], len = a.sched.len[seq];
+        const int nchunks = (len + 63) / 64;
+        const size_t sbase = (size_t(seq) * hv + h) * 128 * 128;
+
+        if (tid == 0 && nchunks > 0) {
+            mbar_arrive_expect_tx(bar_kq0, kBytesKQ);
+            tma_load_3d(sb + kOffKQ0, &tm_k, 0, hq, t0, bar_kq0);
+            tma_load_3d(sb + kOffKQ0 + 8192, &tm_q, 0, hq, t0, bar_kq0);
+            tma_load_3d(sb + kOffKQ0 + 16384, &tm_k, 64, hq, t0, bar_kq0);
+            tma_load_3d(sb + kOffKQ0 + 24576, &tm_q, 64, hq, t0, bar_kq0);
+            mbar_arrive_expect_tx(bar_v, kBytesV);
+            tma_load_3d(sb + kOffV, &tm_v, 0, h, t0, bar_v);
+            tma_load_3d(sb + kOffV + 8192, &tm_v, 64, h, t0, bar_v);
+            pending |= 1u | 4u;
+        }
+        // initial state: fp32 in registers, bf16 copy as the MMA operand
+        float S[64];
+        if (a.s0) {
+            const float4 *src = reinterpret_cast<const float4 *>(a.s0 + sbase + size_t(row) * 128 + 64 * half);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const float4 x = src[c];
+                S[4 * c] = x.x; S[4 * c + 1] = x.y; S[4 * c + 2] = x.z; S[4 * c + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) S[c] = 0.f;
+        }
+        store_row_bf16(sb + kOffS + half * 16384, row, 0, S, 8);
+        fence_proxy_async_shared();
+        __syncthreads();
+
+        for (int n = 0; n < nchunks; ++n) {
+            const int c0 = t0 + n * 64;
+            const int L = min(64, len - n * 64);
+            const int buf = n & 1;
+            const uint32_t kq = sb + (buf ? kOffKQ1 : kOffKQ0);
+            if (tid < 64) {
+                const size_t off = size_t(c0 + tid) * hv + h;
+                gs[tid] = tid < L ? fmaxf(a.g[off], kGFloor) : 0.f;
+                bs[tid] = tid < L ? a.beta[off] : 0.f;
+            }
+            // (1) Gram, once this chunk's K and Q are in
+            {
+                const bool ok = mbar_wait(buf ? bar_kq1 : bar_kq0, buf ? ph_kq1 : ph_kq0);
+                if (buf) ph_kq1 ^= 1; else ph_kq0 ^= 1;
+                if (__syncthreads_or(!ok)) { aborted = true; break; }
+            }
+            if (tid == 0) {
+                pending &= ~(1u << buf);
+                if (n + 1 < nchunks) {
+                    const uint32_t nb = buf ? kOffKQ0 : kOffKQ1, nbar = buf ? bar_kq0 : bar_kq1;
+                    mbar_arrive_expect_tx(nbar, kBytesKQ);
+                    tma_load_3d(sb + nb, &tm_k, 0, hq, c0 + 64, nbar);
+                    tma_load_3d(sb + nb + 8192, &tm_q, 0, hq, c0 + 64, nbar);
+                    tma_load_3d(sb + nb + 16384, &tm_k, 64, hq, c0 + 64, nbar);
+                    tma_load_3d(sb + nb + 24576, &tm_q, 64, hq, c0 + 64, nbar);
+                    pending |= 1u << (buf ^ 1);
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+                    mma_bf16(tmem + kColGram, smem_desc(kq + off, 16, 1024), smem_desc(kq + off, 16, 1024), id_gram,
+                             s > 0);
+                }
+                mma_commit(bar_mma);
+            }
+            // chunk-local prefix sums of g (warp 0) while the Gram runs
+            if (warp == 0) {
+                const float g0 = gs[2 * lane], g1 = gs[2 * lane + 1];
+                float incl = g0 + g1;
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    const float t = __shfl_up_sync(0xffffffffu, incl, d);
+                    if (lane >= d) incl += t;
+                }
+                const float excl = incl - (g0 + g1);
+                gs[2 * lane] = excl + g0;
+                gs[2 * lane + 1] = excl + g0 + g1;
+            }
+            __syncthreads();
+            if (tid < 64) {
+                const float G = gs[tid];
+                gam[tid] = __expf(G);
+                bg[tid] = bs[tid] * __expf(G);
+                lam[tid] = tid < L ? __expf(gs[L - 1] - G) : 0.f;
+            }
+            {
+                const bool ok = mbar_wait(bar_mma, ph_mma);
+                ph_mma ^= 1;
+                if (__syncthreads_or(!ok)) { aborted = true; break; }
+            }
+            tc_fence_after();
+            // A (fp32, for the inverse) and P (bf16 operand) from the Gram
+            {
+                float v[32];
+                tmem_ld32(tmem + lane_bits + kColGram + 32 * half, v);
+                tmem_wait_ld();
+                if (row < 64) {
+                    const int r = row;
+                    const float br = bs[r], Gr = gs[r];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int jj = 32 * half + j;
+                        Af[r * kLdA + jj] = jj < r ? br * __expf(Gr - gs[jj]) * v[j] : 0.f;
+                    }
+                } else {
+                    const int r = row - 64;
+                    const float Gr = gs[r];
+                    float p[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int jj = 32 * half + j;
+                        p[j] = jj <= r ? __expf(Gr - gs[jj]) * v[j] : 0.f;
+                    }
+                    store_row_bf16(sb + kOffP, r, 4 * half, p, 4);
+                }
+            }
+            fence_proxy_async_shared();
+            tc_fence_before();
+            __syncthreads();
+            invert_unit_lower(Af, Tf, Yb, tid);
+            for (int e = tid; e < 64 * 8; e += kThreads) {
+                const int r = e >> 3, c8 = e & 7;
+                float x1[8], x2[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int j = 8 * c8 + u;
+                    const float t = j <= r ? Tf[r * kLdA + j] : 0.f;
+                    x1[u] = t * bg[j];
+                    x2[u] = t * bs[j];
+                }
+                st_shared_v4(sb + kOffTp + sw128_offset(r, c8), pack_bf16x8(x1));
+                st_shared_v4(sb + kOffTpp + sw128_offset(r, c8), pack_bf16x8(x2));
+            }
+            fence_proxy_async_shared();
+            {
+                const bool ok = mbar_wait(bar_v, ph_v);
+                ph_v ^= 1;
+                if (__syncthreads_or(!ok)) { aborted = true; break; }
+            }
+            // (2) W^T, (3) U~^T, (5) X1 = S Q^T
+            if (tid == 0) {
+                pending &= ~4u;
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tmem + kColW, smem_desc(kq + s * 2048, 16384, 1024),
+                             smem_desc(sb + kOffTp + s * 32, 16, 1024), id_w, s > 0);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tmem + kColU, smem_desc(sb + kOffV + s * 2048, 8192, 1024),
+                             smem_desc(sb + kOffTpp + s * 32, 16, 1024), id_w, s > 0);
+#pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+                    mma_bf16(tmem + kColX1, smem_desc(sb + kOffS + off, 16, 1024),
+                             smem_desc(kq + 8192 + off, 16, 1024), id_x, s > 0);
+                }
+                mma_commit(bar_mma);
+            }
+            {
+                const bool ok = mbar_wait(bar_mma, ph_mma);
+                ph_mma ^= 1;
+                if (__syncthreads_or(!ok)) { aborted = true; break; }
+            }
+            tc_fence_after();
+            if (tid == 0 && n + 1 < nchunks) {
+                mbar_arrive_expect_tx(bar_v, kBytesV);
+                tma_load_3d(sb + kOffV, &tm_v, 0, h, c0 + 64, bar_v);
+                tma_load_3d(sb + kOffV + 8192, &tm_v, 64, h, c0 + 64, bar_v);
+                pending |= 4u;
+            }
+            {
+                float v[32];
+                tmem_ld32(tmem + lane_bits + kColW + 32 * half, v);
+                tmem_wait_ld();
+                store_row_bf16(sb + kOffWT, row, 4 * half, v, 4);
+            }
+            fence_proxy_async_shared();
+            tc_fence_before();
+            __syncthreads();
+            // (4) U^T = U~^T - S W^T
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+                    mma_bf16(tmem + kColU, smem_desc(sb + kOffS + off, 16, 1024),
+                             smem_desc(sb + kOffWT + s * 2048, 16384, 1024), id_u, 1);
+                }
+                mma_commit(bar_mma);
+            }
+            {
+                const bool ok = mbar_wait(bar_mma, ph_mma);
+                ph_mma ^= 1;
+                if (__syncthreads_or(!ok)) { aborted = true; break; }
+            }
+            tc_fence_after();
+            {
+                float v[32], w[32];
+                tmem_ld32(tmem + lane_bits + kColU + 32 * half, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) w[j] = v[j] * lam[32 * half + j];
+                store_row_bf16(sb + kOffUT, row, 4 * half, v, 4);
+                store_row_bf16(sb + kOffUTl, row, 4 * half, w, 4);
+            }
+            fence_proxy_async_shared();
+            tc_fence_before();
+            __syncthreads();
+            // (6) X2 = U^T P^T, (7) dS = U^T diag(lambda) K
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tmem + kColX2, smem_desc(sb + kOffUT + s * 32, 16, 1024),
+                             smem_desc(sb + kOffP + s * 32, 16, 1024), id_x, s > 0);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tmem + kColDS, smem_desc(sb + kOffUTl + s * 32, 16, 1024),
+                             smem_desc(kq + s * 2048, 16384, 1024), id_ds, s > 0);
+                mma_commit(bar_mma);
+            }
+            {
+                const bool ok = mbar_wait(bar_mma, ph_mma);
+                ph_mma ^= 1;
+                if (__syncthreads_or(!ok)) { aborted = true; break; }
+            }
+            tc_fence_after();
+            {
+                const float gC = gam[63];  // padded rows carry g = 0, so G_63 = G_{L-1}
+                float v[32];
+                tmem_ld32(tmem + lane_bits + kColDS + 64 * half, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) S[j] = fmaf(gC, S[j], v[j]);
+                tmem_ld32(tmem + lane_bits + kColDS + 64 * half + 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) S[32 + j] = fmaf(gC, S[32 + j], v[j]);
+                store_row_bf16(sb + kOffS + half * 16384, row, 0, S, 8);
+                float x1[32], x2[32];
+                tmem_ld32(tmem + lane_bits + kColX1 + 32 * half, x1);
+                tmem_ld32(tmem + lane_bits + kColX2 + 32 * half, x2);
+                tmem_wait_ld();
+                __nv_bfloat16 *orow = o + (size_t(c0) * hv + h) * 128 + row;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int r = 32 * half + j;
+                    if (r < L) orow[size_t(r) * hv * 128] = __float2bfloat16_rn(fmaf(gam[r], x1[j], x2[j]));
+                }
+            }
+            fence_proxy_async_shared();
+            tc_fence_before();
+            __syncthreads();
+        }
+        if (aborted) break;
+        if (a.s_final) {
+            float4 *dst = reinterpret_cast<float4 *>(a.s_final + sbase + size_t(row) * 128 + 64 * half);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
+        }
+    }
+
+    if (aborted && tid == 0) {
+        // let this CTA's own asynchronous work drain (bounded) before freeing tensor memory
+        mma_commit(bar_mma);
+        (void)mbar_wait(bar_mma, ph_mma);
+        if (pending & 1u) (void)mbar_wait(bar_kq0, ph_kq0);
+        if (pending & 2u) (void)mbar_wait(bar_kq1, ph_kq1);
+        if (pending & 4u) (void)mbar_wait(bar_v, ph_v);
+        hdr->bad_index = -2;
+        atomicExch(&hdr->status, int(GDN_ERR_DEVICE_CHECK));
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [tokens, heads, 128] bf16 viewed as a 3-D tensor (d fastest), boxes of
+// 64 (d) x 1 (head) x 64 (tokens), 128-byte swizzle; rows past the last token
+// read as zeros.
+bool make_map(CUtensorMap *map, const void *base, int heads, int tokens) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {128, cuuint64_t(heads), cuuint64_t(tokens)};
+    const cuuint64_t strides[2] = {128 * 2, cuuint64_t(heads) * 128 * 2};
+    const cuuint32_t box[3] = {64, 1, 64};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool chunk_tc_supported(const gdn_shape_t &s) {
+    return s.dtype == GDN_DTYPE_BF16 && s.head_dim_k == 128 && s.head_dim_v == 128 && s.chunk_size == 64;
+}
+
+cudaError_t launch_chunk_tc(const PrefillArgs &a, cudaStream_t stream, int num_sms) {
+    // With no tokens at all there is nothing to load; the fp32 kernel writes
+    // the final states (= initial states) of the empty sequences.
+    if (a.tokens <= 0) return launch_chunk_simt(a, stream, num_sms);
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, a.q, a.hk, a.tokens) || !make_map(&mk, a.k, a.hk, a.tokens) ||
+        !make_map(&mv, a.v, a.hv, a.tokens))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+    if (e != cudaSuccess) return e;
+    const int64_t units = int64_t(a.num_seqs) * a.hv;
+    const int grid = int(units < num_sms ? units : num_sms);
+    if (grid <= 0) return cudaSuccess;
+    chunk_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, a);
+    count_launch();
+    return cudaGetLastError();
+}
+
 }  // namespace gdn

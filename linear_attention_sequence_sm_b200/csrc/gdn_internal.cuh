@@ -78,6 +78,7 @@ cudaError_t launch_schedule(const gdn_shape_t &s, const int32_t *cu_seqlens, voi
 
 struct PrefillArgs {
     int32_t num_seqs, hk, hv, dk, dv, chunk, dtype;
+    int32_t tokens;  // rows of q, k, v, o (B * T, or the packed total)
     const void *q, *k, *v;
     const float *g, *beta, *s0;
     void *o;
