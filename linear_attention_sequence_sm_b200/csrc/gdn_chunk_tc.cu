@@ -46,7 +46,8 @@ using namespace sm100;
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kLdA = 65;  // fp32 row stride of the A and T scratch matrices
+constexpr int kLdA = 68;  // fp32 row stride of the A and T scratch matrices (16-byte aligned rows)
+constexpr int kLdY = 36;  // fp32 row stride of the inverse's 32 x 32 scratch
 
 // Shared-memory map (bytes from a 1024-byte-aligned base).  Tiles are
 // 128-byte-swizzled: "atom columns" of 64 bf16 (128 bytes) per row.
@@ -62,14 +63,16 @@ constexpr uint32_t kOffUT = 155648;   // U^T: 128 rows (d_v) x 64 tokens
 constexpr uint32_t kOffUTl = 172032;  // U^T diag(lambda)
 constexpr uint32_t kOffAf = 188416;   // A, fp32 64 x kLdA
 constexpr uint32_t kOffTf = kOffAf + 64 * kLdA * 4;  // T, fp32 64 x kLdA
-constexpr uint32_t kOffY = kOffTf + 64 * kLdA * 4;   // blocked-inverse scratch, 3 x 16 x 16 fp32
-constexpr uint32_t kOffVec = kOffY + 3 * 256 * 4;    // per-token vectors, 8 x 64 fp32
+constexpr uint32_t kOffY = kOffTf + 64 * kLdA * 4;   // inverse scratch, 32 x kLdY fp32
+constexpr uint32_t kOffVec = kOffY + 32 * kLdY * 4;  // per-token vectors, 8 x 64 fp32
 constexpr uint32_t kOffBar = kOffVec + 8 * 64 * 4;   // 4 mbarriers + tensor-memory slot
 constexpr uint32_t kSmemBytes = kOffBar + 64 + 1024; // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 per-block limit");
 
-// Tensor-memory columns (fp32 accumulators, 128 lanes each).
-constexpr uint32_t kColGram = 0, kColW = 64, kColU = 128, kColX1 = 192, kColX2 = 256, kColDS = 320;
+// Tensor-memory columns (fp32, 128 lanes each).  The state S (d_v lanes x
+// d_k columns) lives at kColS for the whole unit and is the accumulator of
+// the state-update product.
+constexpr uint32_t kColGram = 0, kColW = 64, kColU = 128, kColX1 = 192, kColX2 = 256, kColS = 320;
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t kBytesKQ = 4 * 8192;  // four 64 x 64 bf16 boxes
@@ -81,52 +84,118 @@ __device__ __forceinline__ void store_row_bf16(uint32_t tile, int row, int chunk
 }
 
 // T = (I + A)^-1 for the 64 x 64 unit-lower-triangular system, fp32, in
-// shared memory.  Diagonal 16 x 16 blocks B_I = (I + A_II)^-1 by forward
-// substitution (one thread per column), then block rows I = 1..3:
-// T_IJ = -B_I sum_{K=J}^{I-1} A_IK T_KJ.  All threads must call it.
+// shared memory, by divide and conquer on the block structure
+//   [[X, 0], [C, Z]]^-1 = [[X^-1, 0], [-Z^-1 C X^-1, Z^-1]]:
+// the four 16 x 16 diagonal blocks by row-wise forward substitution (one
+// thread per column), then the two 32 x 32 halves (two 16 x 16 products each),
+// then the 64 x 64 matrix (two 32 x 32 products, 2 x 2 outputs per thread).
+// The strictly-upper 16 x 16 blocks inside each 32 x 32 half must be zero in
+// Tf on entry (they are zeroed once and never written).  All threads call it.
 __device__ void invert_unit_lower(const float *Af, float *Tf, float *Y, int tid) {
     if (tid < 64) {
         const int b = tid >> 4, c = tid & 15;
+        const float *Ab = Af + (16 * b) * kLdA + 16 * b;
         float x[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) x[r] = (r == c) ? 1.f : 0.f;
+        for (int r = 0; r < 16; ++r) {
+            float a[16];
 #pragma unroll
-        for (int j = 0; j < 15; ++j) {
+            for (int q = 0; q < 4; ++q) {
+                const float4 t = *reinterpret_cast<const float4 *>(Ab + r * kLdA + 4 * q);
+                a[4 * q] = t.x; a[4 * q + 1] = t.y; a[4 * q + 2] = t.z; a[4 * q + 3] = t.w;
+            }
+            float acc0 = (r == c) ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
-            for (int r = j + 1; r < 16; ++r) x[r] = fmaf(-Af[(16 * b + r) * kLdA + 16 * b + j], x[j], x[r]);
+            for (int jj = 0; jj < r; ++jj) {
+                if (jj & 1) acc1 = fmaf(-a[jj], x[jj], acc1);
+                else acc0 = fmaf(-a[jj], x[jj], acc0);
+            }
+            x[r] = acc0 + acc1;
         }
+        float *Tb = Tf + (16 * b) * kLdA + 16 * b;
 #pragma unroll
-        for (int r = 0; r < 16; ++r) Tf[(16 * b + r) * kLdA + 16 * b + c] = x[r];
+        for (int r = 0; r < 16; ++r) Tb[r * kLdA + c] = x[r];
     }
     __syncthreads();
-    for (int I = 1; I < 4; ++I) {
-        for (int e = tid; e < I * 256; e += kThreads) {
-            const int J = e >> 8, r = (e >> 4) & 15, c = e & 15;
-            float acc = 0.f;
-            for (int K = J; K < I; ++K) {
+    // 32 x 32 halves p = 0, 1: Y_p = A[32p+16.., 32p..] B_{2p}, T[32p+16.., 32p..] = -B_{2p+1} Y_p
+    const int p = tid >> 7, e = tid & 127, r1 = e >> 3, c1 = (e & 7) * 2;
+    {
+        const float *Arow = Af + (32 * p + 16 + r1) * kLdA + 32 * p;
+        const float *Bm = Tf + (32 * p) * kLdA + 32 * p;
+        float z0 = 0.f, z1 = 0.f;
 #pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    acc = fmaf(Af[(16 * I + r) * kLdA + 16 * K + m], Tf[(16 * K + m) * kLdA + 16 * J + c], acc);
-            }
-            Y[e] = acc;
+        for (int m = 0; m < 16; ++m) {
+            const float a = Arow[m];
+            const float2 t = *reinterpret_cast<const float2 *>(Bm + m * kLdA + c1);
+            z0 = fmaf(a, t.x, z0);
+            z1 = fmaf(a, t.y, z1);
         }
-        __syncthreads();
-        for (int e = tid; e < I * 256; e += kThreads) {
-            const int J = e >> 8, r = (e >> 4) & 15, c = e & 15;
-            float acc = 0.f;
-            for (int m = 0; m <= r; ++m) acc = fmaf(Tf[(16 * I + r) * kLdA + 16 * I + m], Y[J * 256 + m * 16 + c], acc);
-            Tf[(16 * I + r) * kLdA + 16 * J + c] = -acc;
-        }
-        __syncthreads();
+        *reinterpret_cast<float2 *>(Y + (16 * p + r1) * kLdY + c1) = make_float2(z0, z1);
     }
+    __syncthreads();
+    {
+        const float *Brow = Tf + (32 * p + 16 + r1) * kLdA + 32 * p + 16;
+        float z0 = 0.f, z1 = 0.f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            const float bm = Brow[m];  // zero above the diagonal
+            const float2 t = *reinterpret_cast<const float2 *>(Y + (16 * p + m) * kLdY + c1);
+            z0 = fmaf(bm, t.x, z0);
+            z1 = fmaf(bm, t.y, z1);
+        }
+        *reinterpret_cast<float2 *>(Tf + (32 * p + 16 + r1) * kLdA + 32 * p + c1) = make_float2(-z0, -z1);
+    }
+    __syncthreads();
+    // 64 x 64: Y = A[32.., 0..32] T_a, T[32.., 0..32] = -T_b Y
+    const int r0 = (tid >> 4) * 2, c0 = (tid & 15) * 2;
+    {
+        const float *A0 = Af + (32 + r0) * kLdA, *A1 = A0 + kLdA;
+        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+#pragma unroll
+        for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 a0 = *reinterpret_cast<const float4 *>(A0 + 4 * k4);
+            const float4 a1 = *reinterpret_cast<const float4 *>(A1 + 4 * k4);
+            const float a0v[4] = {a0.x, a0.y, a0.z, a0.w}, a1v[4] = {a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float2 t = *reinterpret_cast<const float2 *>(Tf + (4 * k4 + u) * kLdA + c0);
+                y00 = fmaf(a0v[u], t.x, y00); y01 = fmaf(a0v[u], t.y, y01);
+                y10 = fmaf(a1v[u], t.x, y10); y11 = fmaf(a1v[u], t.y, y11);
+            }
+        }
+        *reinterpret_cast<float2 *>(Y + r0 * kLdY + c0) = make_float2(y00, y01);
+        *reinterpret_cast<float2 *>(Y + (r0 + 1) * kLdY + c0) = make_float2(y10, y11);
+    }
+    __syncthreads();
+    {
+        const float *B0 = Tf + (32 + r0) * kLdA + 32, *B1 = B0 + kLdA;
+        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+#pragma unroll
+        for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 b0 = *reinterpret_cast<const float4 *>(B0 + 4 * k4);
+            const float4 b1 = *reinterpret_cast<const float4 *>(B1 + 4 * k4);
+            const float b0v[4] = {b0.x, b0.y, b0.z, b0.w}, b1v[4] = {b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float2 t = *reinterpret_cast<const float2 *>(Y + (4 * k4 + u) * kLdY + c0);
+                y00 = fmaf(b0v[u], t.x, y00); y01 = fmaf(b0v[u], t.y, y01);
+                y10 = fmaf(b1v[u], t.x, y10); y11 = fmaf(b1v[u], t.y, y11);
+            }
+        }
+        *reinterpret_cast<float2 *>(Tf + (32 + r0) * kLdA + c0) = make_float2(-y00, -y01);
+        *reinterpret_cast<float2 *>(Tf + (32 + r0 + 1) * kLdA + c0) = make_float2(-y10, -y11);
+    }
+    __syncthreads();
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
     extern __shared__ unsigned char smem_raw[];
-    unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                            ~uintptr_t(1023));
+    // Align to 1024 bytes with a byte offset on the shared array itself (not
+    // through an integer cast), so that the compiler keeps every access below in
+    // the shared address space (ld.shared / st.shared, not generic loads).
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sb = smem_u32(smem);
     float *Af = reinterpret_cast<float *>(smem + kOffAf);
     float *Tf = reinterpret_cast<float *>(smem + kOffTf);
@@ -163,6 +232,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
+    // T starts all zero: the inverse writes only the lower-triangular blocks
+    // (and zeros above the diagonal inside the diagonal blocks), so everything
+    // above the diagonal reads as zero for the rest of the kernel.
+    for (int e = tid; e < 64 * kLdA; e += kThreads) Tf[e] = 0.f;
+    __syncthreads();
 
     const int hv = a.hv, hk = a.hk, group = hv / hk;
     const int total_units = a.num_seqs * hv;
@@ -175,7 +249,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t id_w = idesc_bf16(128, 64, true, false);
     const uint32_t id_u = idesc_bf16(128, 64, false, true, true);
     const uint32_t id_x = idesc_bf16(128, 64, false, false);
-    const uint32_t id_ds = idesc_bf16(128, 128, false, true);
+    const uint32_t id_ds = idesc_bf16(128, 128, false, true);  // state update, accumulates into S
 
     for (;;) {
         if (tid == 0) *s_unit = int(atomicAdd(&hdr->next_unit, 1u));
@@ -200,22 +274,31 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tma_load_3d(sb + kOffV + 8192, &tm_v, 64, h, t0, bar_v);
             pending |= 1u | 4u;
         }
-        // initial state: fp32 in registers, bf16 copy as the MMA operand
-        float S[64];
-        if (a.s0) {
-            const float4 *src = reinterpret_cast<const float4 *>(a.s0 + sbase + size_t(row) * 128 + 64 * half);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const float4 x = src[c];
-                S[4 * c] = x.x; S[4 * c + 1] = x.y; S[4 * c + 2] = x.z; S[4 * c + 3] = x.w;
-            }
-        } else {
-#pragma unroll
-            for (int c = 0; c < 64; ++c) S[c] = 0.f;
+        // gates of the first chunk (threads 0-63 keep one chunk of g, beta in flight)
+        float g_next = 0.f, b_next = 0.f;
+        if (tid < 64 && tid < len) {
+            g_next = a.g[size_t(t0 + tid) * hv + h];
+            b_next = a.beta[size_t(t0 + tid) * hv + h];
         }
-        store_row_bf16(sb + kOffS + half * 16384, row, 0, S, 8);
-        fence_proxy_async_shared();
-        __syncthreads();
+        // initial state into tensor memory (this thread: lane `row`, 64 key columns)
+#pragma unroll
+        for (int p2 = 0; p2 < 2; ++p2) {
+            float v[32];
+            if (a.s0) {
+                const float4 *src =
+                    reinterpret_cast<const float4 *>(a.s0 + sbase + size_t(row) * 128 + 64 * half + 32 * p2);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const float4 x = src[c];
+                    v[4 * c] = x.x; v[4 * c + 1] = x.y; v[4 * c + 2] = x.z; v[4 * c + 3] = x.w;
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 32; ++c) v[c] = 0.f;
+            }
+            tmem_st32(tmem + lane_bits + kColS + 64 * half + 32 * p2, v);
+        }
+        tmem_wait_st();
 
         for (int n = 0; n < nchunks; ++n) {
             const int c0 = t0 + n * 64;
@@ -223,9 +306,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int buf = n & 1;
             const uint32_t kq = sb + (buf ? kOffKQ1 : kOffKQ0);
             if (tid < 64) {
-                const size_t off = size_t(c0 + tid) * hv + h;
-                gs[tid] = tid < L ? fmaxf(a.g[off], kGFloor) : 0.f;
-                bs[tid] = tid < L ? a.beta[off] : 0.f;
+                gs[tid] = tid < L ? fmaxf(g_next, kGFloor) : 0.f;
+                bs[tid] = tid < L ? b_next : 0.f;
+                // prefetch the next chunk's gates; they are consumed one chunk later
+                if (n + 1 < nchunks && tid < min(64, len - (n + 1) * 64)) {
+                    const size_t off = size_t(c0 + 64 + tid) * hv + h;
+                    g_next = a.g[off];
+                    b_next = a.beta[off];
+                }
             }
             // (1) Gram, once this chunk's K and Q are in
             {
@@ -273,6 +361,25 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 bg[tid] = bs[tid] * __expf(G);
                 lam[tid] = tid < L ? __expf(gs[L - 1] - G) : 0.f;
             }
+            // S pass: the chunk-start state S_n becomes the bf16 operand, and the
+            // fp32 state in tensor memory is decayed to gamma_C S_n so that the
+            // state-update product can accumulate onto it.  Padded rows carry
+            // g = 0, so G_63 = G_{L-1}.
+            {
+                const float gC = __expf(gs[63]);
+#pragma unroll
+                for (int p2 = 0; p2 < 2; ++p2) {
+                    float v[32];
+                    tmem_ld32(tmem + lane_bits + kColS + 64 * half + 32 * p2, v);
+                    tmem_wait_ld();
+                    store_row_bf16(sb + kOffS + half * 16384, row, 4 * p2, v, 4);
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) v[jj] *= gC;
+                    tmem_st32(tmem + lane_bits + kColS + 64 * half + 32 * p2, v);
+                }
+                tmem_wait_st();
+            }
+            fence_proxy_async_shared();
             {
                 const bool ok = mbar_wait(bar_mma, ph_mma);
                 ph_mma ^= 1;
@@ -281,27 +388,33 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_after();
             // A (fp32, for the inverse) and P (bf16 operand) from the Gram
             {
-                float v[32];
+                float v[32], gj[32];
                 tmem_ld32(tmem + lane_bits + kColGram + 32 * half, v);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 t = *reinterpret_cast<const float4 *>(gs + 32 * half + 4 * q);
+                    gj[4 * q] = t.x; gj[4 * q + 1] = t.y; gj[4 * q + 2] = t.z; gj[4 * q + 3] = t.w;
+                }
+                const int r = row & 63;
+                const float Gr = gs[r];
+                const bool is_a = row < 64;
+                const float scale = is_a ? bs[r] : 1.f;
+                const int lim = is_a ? r : r + 1;  // A: j < r;  P: j <= r
                 tmem_wait_ld();
-                if (row < 64) {
-                    const int r = row;
-                    const float br = bs[r], Gr = gs[r];
+                float x[32];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int jj = 32 * half + j;
-                        Af[r * kLdA + jj] = jj < r ? br * __expf(Gr - gs[jj]) * v[j] : 0.f;
-                    }
+                for (int jj = 0; jj < 32; ++jj) {
+                    // branch-free: every lane evaluates the exponential, a 0/1 factor masks it
+                    const float keep = (32 * half + jj < lim) ? 1.f : 0.f;
+                    x[jj] = keep * scale * __expf(fminf(Gr - gj[jj], 0.f)) * v[jj];
+                }
+                if (is_a) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        *reinterpret_cast<float4 *>(Af + r * kLdA + 32 * half + 4 * q) =
+                            make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
                 } else {
-                    const int r = row - 64;
-                    const float Gr = gs[r];
-                    float p[32];
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int jj = 32 * half + j;
-                        p[j] = jj <= r ? __expf(Gr - gs[jj]) * v[j] : 0.f;
-                    }
-                    store_row_bf16(sb + kOffP, r, 4 * half, p, 4);
+                    store_row_bf16(sb + kOffP, r, 4 * half, x, 4);
                 }
             }
             fence_proxy_async_shared();
@@ -313,10 +426,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 float x1[8], x2[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    const int j = 8 * c8 + u;
-                    const float t = j <= r ? Tf[r * kLdA + j] : 0.f;
-                    x1[u] = t * bg[j];
-                    x2[u] = t * bs[j];
+                    const int jj = 8 * c8 + u;
+                    const float t = Tf[r * kLdA + jj];  // zero above the diagonal
+                    x1[u] = t * bg[jj];
+                    x2[u] = t * bs[jj];
                 }
                 st_shared_v4(sb + kOffTp + sw128_offset(r, c8), pack_bf16x8(x1));
                 st_shared_v4(sb + kOffTpp + sw128_offset(r, c8), pack_bf16x8(x2));
@@ -390,14 +503,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tmem_ld32(tmem + lane_bits + kColU + 32 * half, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) w[j] = v[j] * lam[32 * half + j];
+                for (int jj = 0; jj < 32; ++jj) w[jj] = v[jj] * lam[32 * half + jj];
                 store_row_bf16(sb + kOffUT, row, 4 * half, v, 4);
                 store_row_bf16(sb + kOffUTl, row, 4 * half, w, 4);
             }
             fence_proxy_async_shared();
             tc_fence_before();
             __syncthreads();
-            // (6) X2 = U^T P^T, (7) dS = U^T diag(lambda) K
+            // (6) X2 = U^T P^T, (7) S += U^T diag(lambda) K
             if (tid == 0) {
                 tc_fence_after();
 #pragma unroll
@@ -406,8 +519,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                              smem_desc(sb + kOffP + s * 32, 16, 1024), id_x, s > 0);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + kColDS, smem_desc(sb + kOffUTl + s * 32, 16, 1024),
-                             smem_desc(kq + s * 2048, 16384, 1024), id_ds, s > 0);
+                    mma_bf16(tmem + kColS, smem_desc(sb + kOffUTl + s * 32, 16, 1024),
+                             smem_desc(kq + s * 2048, 16384, 1024), id_ds, 1);
                 mma_commit(bar_mma);
             }
             {
@@ -416,39 +529,46 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (__syncthreads_or(!ok)) { aborted = true; break; }
             }
             tc_fence_after();
+            // O[r][i] = gamma_r X1[i][r] + X2[i][r], staged through shared memory
+            // (over the inverse's scratch) so that each token row leaves as
+            // contiguous 16-byte stores
             {
-                const float gC = gam[63];  // padded rows carry g = 0, so G_63 = G_{L-1}
-                float v[32];
-                tmem_ld32(tmem + lane_bits + kColDS + 64 * half, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) S[j] = fmaf(gC, S[j], v[j]);
-                tmem_ld32(tmem + lane_bits + kColDS + 64 * half + 32, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) S[32 + j] = fmaf(gC, S[32 + j], v[j]);
-                store_row_bf16(sb + kOffS + half * 16384, row, 0, S, 8);
                 float x1[32], x2[32];
                 tmem_ld32(tmem + lane_bits + kColX1 + 32 * half, x1);
                 tmem_ld32(tmem + lane_bits + kColX2 + 32 * half, x2);
                 tmem_wait_ld();
-                __nv_bfloat16 *orow = o + (size_t(c0) * hv + h) * 128 + row;
+                __nv_bfloat16 *Ot = reinterpret_cast<__nv_bfloat16 *>(smem + kOffAf);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int r = 32 * half + j;
-                    if (r < L) orow[size_t(r) * hv * 128] = __float2bfloat16_rn(fmaf(gam[r], x1[j], x2[j]));
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int r = 32 * half + jj;
+                    Ot[r * 128 + row] = __float2bfloat16_rn(fmaf(gam[r], x1[jj], x2[jj]));
                 }
             }
-            fence_proxy_async_shared();
             tc_fence_before();
+            __syncthreads();
+            for (int e = tid; e < 64 * 16; e += kThreads) {
+                const int r = e >> 4, c = e & 15;
+                if (r < L) {
+                    const uint4 val = *reinterpret_cast<const uint4 *>(smem + kOffAf + r * 256 + c * 16);
+                    *reinterpret_cast<uint4 *>(o + (size_t(c0 + r) * hv + h) * 128 + c * 8) = val;
+                }
+            }
             __syncthreads();
         }
         if (aborted) break;
-        if (a.s_final) {
-            float4 *dst = reinterpret_cast<float4 *>(a.s_final + sbase + size_t(row) * 128 + 64 * half);
+        // final state out of tensor memory
 #pragma unroll
-            for (int c = 0; c < 16; ++c) dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
+        for (int p2 = 0; p2 < 2; ++p2) {
+            float v[32];
+            tmem_ld32(tmem + lane_bits + kColS + 64 * half + 32 * p2, v);
+            tmem_wait_ld();
+            if (a.s_final) {
+                float4 *dst = reinterpret_cast<float4 *>(a.s_final + sbase + size_t(row) * 128 + 64 * half + 32 * p2);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) dst[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            }
         }
+        tc_fence_before();
     }
 
     if (aborted && tid == 0) {
