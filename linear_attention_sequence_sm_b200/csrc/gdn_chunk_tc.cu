@@ -205,6 +205,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float *gam = gs + 128;                                 // gamma = e^G
     float *bg = gs + 192;                                  // beta gamma
     float *lam = gs + 256;                                 // e^(G_C - G), 0 past the sequence end
+    float *igam = gs + 320;                                // e^(-G), used when the chunk's decay is mild
     const uint32_t bar_kq0 = sb + kOffBar, bar_kq1 = sb + kOffBar + 8, bar_v = sb + kOffBar + 16,
                    bar_mma = sb + kOffBar + 24;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + kOffBar + 32);
@@ -360,6 +361,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 gam[tid] = __expf(G);
                 bg[tid] = bs[tid] * __expf(G);
                 lam[tid] = tid < L ? __expf(gs[L - 1] - G) : 0.f;
+                igam[tid] = __expf(-G);
             }
             // S pass: the chunk-start state S_n becomes the bf16 operand, and the
             // fp32 state in tensor memory is decayed to gamma_C S_n so that the
@@ -367,16 +369,19 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // g = 0, so G_63 = G_{L-1}.
             {
                 const float gC = __expf(gs[63]);
+                float v0[32], v1[32];
+                tmem_ld32(tmem + lane_bits + kColS + 64 * half, v0);
+                tmem_ld32(tmem + lane_bits + kColS + 64 * half + 32, v1);
+                tmem_wait_ld();
+                store_row_bf16(sb + kOffS + half * 16384, row, 0, v0, 4);
+                store_row_bf16(sb + kOffS + half * 16384, row, 4, v1, 4);
 #pragma unroll
-                for (int p2 = 0; p2 < 2; ++p2) {
-                    float v[32];
-                    tmem_ld32(tmem + lane_bits + kColS + 64 * half + 32 * p2, v);
-                    tmem_wait_ld();
-                    store_row_bf16(sb + kOffS + half * 16384, row, 4 * p2, v, 4);
-#pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) v[jj] *= gC;
-                    tmem_st32(tmem + lane_bits + kColS + 64 * half + 32 * p2, v);
+                for (int jj = 0; jj < 32; ++jj) {
+                    v0[jj] *= gC;
+                    v1[jj] *= gC;
                 }
+                tmem_st32(tmem + lane_bits + kColS + 64 * half, v0);
+                tmem_st32(tmem + lane_bits + kColS + 64 * half + 32, v1);
                 tmem_wait_st();
             }
             fence_proxy_async_shared();
@@ -400,13 +405,32 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const bool is_a = row < 64;
                 const float scale = is_a ? bs[r] : 1.f;
                 const int lim = is_a ? r : r + 1;  // A: j < r;  P: j <= r
-                tmem_wait_ld();
                 float x[32];
+                // Gamma_rj = e^(G_r - G_j).  While the chunk's total log-decay is
+                // at least -80, e^(-G_j) stays finite in fp32 and Gamma is the
+                // rank-1 product e^(G_r) e^(-G_j) (64 exponentials, not 4096).
+                if (gs[63] >= -80.f) {
+                    float ig[32];
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    // branch-free: every lane evaluates the exponential, a 0/1 factor masks it
-                    const float keep = (32 * half + jj < lim) ? 1.f : 0.f;
-                    x[jj] = keep * scale * __expf(fminf(Gr - gj[jj], 0.f)) * v[jj];
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 t = *reinterpret_cast<const float4 *>(igam + 32 * half + 4 * q);
+                        ig[4 * q] = t.x; ig[4 * q + 1] = t.y; ig[4 * q + 2] = t.z; ig[4 * q + 3] = t.w;
+                    }
+                    const float sg = scale * gam[r];
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const float keep = (32 * half + jj < lim) ? 1.f : 0.f;
+                        x[jj] = keep * sg * ig[jj] * v[jj];
+                    }
+                } else {
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        // branch-free: every lane evaluates the exponential, a 0/1 factor masks it
+                        const float keep = (32 * half + jj < lim) ? 1.f : 0.f;
+                        x[jj] = keep * scale * __expf(fminf(Gr - gj[jj], 0.f)) * v[jj];
+                    }
                 }
                 if (is_a) {
 #pragma unroll
@@ -423,13 +447,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             invert_unit_lower(Af, Tf, Yb, tid);
             for (int e = tid; e < 64 * 8; e += kThreads) {
                 const int r = e >> 3, c8 = e & 7;
-                float x1[8], x2[8];
+                float t[8], b1[8], b2[8], x1[8], x2[8];
+#pragma unroll
+                for (int hq4 = 0; hq4 < 2; ++hq4) {
+                    const float4 tv = *reinterpret_cast<const float4 *>(Tf + r * kLdA + 8 * c8 + 4 * hq4);  // zero above the diagonal
+                    const float4 bv = *reinterpret_cast<const float4 *>(bg + 8 * c8 + 4 * hq4);
+                    const float4 sv = *reinterpret_cast<const float4 *>(bs + 8 * c8 + 4 * hq4);
+                    t[4 * hq4] = tv.x; t[4 * hq4 + 1] = tv.y; t[4 * hq4 + 2] = tv.z; t[4 * hq4 + 3] = tv.w;
+                    b1[4 * hq4] = bv.x; b1[4 * hq4 + 1] = bv.y; b1[4 * hq4 + 2] = bv.z; b1[4 * hq4 + 3] = bv.w;
+                    b2[4 * hq4] = sv.x; b2[4 * hq4 + 1] = sv.y; b2[4 * hq4 + 2] = sv.z; b2[4 * hq4 + 3] = sv.w;
+                }
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    const int jj = 8 * c8 + u;
-                    const float t = Tf[r * kLdA + jj];  // zero above the diagonal
-                    x1[u] = t * bg[jj];
-                    x2[u] = t * bs[jj];
+                    x1[u] = t[u] * b1[u];
+                    x2[u] = t[u] * b2[u];
                 }
                 st_shared_v4(sb + kOffTp + sw128_offset(r, c8), pack_bf16x8(x1));
                 st_shared_v4(sb + kOffTpp + sw128_offset(r, c8), pack_bf16x8(x2));
