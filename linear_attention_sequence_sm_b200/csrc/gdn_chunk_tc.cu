@@ -20,19 +20,31 @@
 //   (4) U^T = U~^T - S W^T   (accumulates into (3), A negated)      128x64x128
 //   (5) X1 = S Q^T                                                   128x64x128
 //   (6) X2 = U^T P^T,  P = Q K^T (.) Gamma                           128x64x64
-//   (7) dS = (U^T diag(lambda)) K,  lambda_j = e^(G_C - G_j)         128x128x64
-// O[r][i] = gamma_r X1[i][r] + X2[i][r];  S <- gamma_C S + dS.
-// Operands are bf16 in 128-byte-swizzled shared memory; q, k, v tiles arrive
-// by TMA (no multicast); the fp32 state S lives in registers (thread = state
-// row, half of the key columns) and is re-staged as a bf16 operand each
-// chunk.  The triangular inverse runs on the CUDA cores in fp32 (16 x 16
-// diagonal blocks by forward substitution, then the off-diagonal blocks).
+//   (7) S += (U^T diag(lambda)) K,  lambda_j = e^(G_C - G_j)         128x128x64
+// O[r][i] = gamma_r X1[i][r] + X2[i][r].  Operands are bf16 in
+// 128-byte-swizzled shared memory; q, k, v tiles arrive by TMA (no
+// multicast).  The fp32 state S lives in tensor memory as the accumulator of
+// (7); once per chunk it is read, staged as the bf16 operand of (4) and (5),
+// and rescaled by gamma_C in place.
 //
-// One CTA per SM (the shared-memory footprint forces it) owns a unit
-// (sequence, value head) at a time, taking units longest sequence first from
-// an atomic counter, and walks the unit's chunks in order.  Every wait on an
-// mbarrier is bounded; a timeout records GDN_ERR_DEVICE_CHECK (bad_index -2)
-// in the workspace status word and the CTA frees its tensor memory and exits.
+// Warp specialisation.  Only (4), (7) and the state pass depend on the state
+// carried from the previous chunk; everything else in a chunk does not.  So a
+// CTA runs two warp groups on one (sequence, value head) unit:
+//   chain  (warps 0-3):  state pass, (4)+(5), U epilogue, (6)+(7), output
+//   intra  (warps 4-11): gates and their prefix sums, (1), decay masks A and
+//                        P, the triangular inverse (CUDA cores, fp32), T'
+//                        and T'', (2)+(3), W^T epilogue -- one chunk ahead.
+// They hand chunks over through mbarriers: "full[b]" (intra -> chain: W^T,
+// P, U~ in tensor memory and the per-token vectors of buffer b are ready),
+// "empty[b]" (chain -> intra: buffer b may be refilled), "wt_free" (the
+// single W^T tile has been consumed).  q/k tiles are double-buffered; the
+// chain refills a buffer two chunks ahead as soon as its last reader (7)
+// completes.  Each group synchronises internally with its own named barrier.
+//
+// One CTA per SM (shared memory and the 512 tensor-memory columns force it)
+// takes units longest sequence first from an atomic counter.  Every wait is
+// bounded; a timeout records GDN_ERR_DEVICE_CHECK (bad_index -2) in the
+// workspace status word, and the CTA frees its tensor memory and exits.
 #include <cuda.h>
 
 #include <mutex>
@@ -45,42 +57,75 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;      // warps 0-3: chain group; warps 4-11: intra group
+constexpr int kChain = 128, kIntra = 256;
+constexpr int kBarChain = 1, kBarIntra = 2;  // named barrier ids (0 is __syncthreads)
 constexpr int kLdA = 68;  // fp32 row stride of the A and T scratch matrices (16-byte aligned rows)
 constexpr int kLdY = 36;  // fp32 row stride of the inverse's 32 x 32 scratch
 
 // Shared-memory map (bytes from a 1024-byte-aligned base).  Tiles are
 // 128-byte-swizzled: "atom columns" of 64 bf16 (128 bytes) per row.
-constexpr uint32_t kOffKQ0 = 0;       // [K;Q] chunk buffer 0: 2 atom columns x 128 rows (K 0-63, Q 64-127)
-constexpr uint32_t kOffKQ1 = 32768;   // [K;Q] chunk buffer 1
-constexpr uint32_t kOffV = 65536;     // V: 2 atom columns x 64 rows
-constexpr uint32_t kOffS = 81920;     // S operand (bf16): 2 atom columns x 128 rows (d_v)
-constexpr uint32_t kOffTp = 114688;   // T diag(beta gamma): 64 x 64
-constexpr uint32_t kOffTpp = 122880;  // T diag(beta): 64 x 64
-constexpr uint32_t kOffWT = 131072;   // W^T: 128 rows (d_k) x 64 tokens
-constexpr uint32_t kOffP = 147456;    // P: 64 x 64
-constexpr uint32_t kOffUT = 155648;   // U^T: 128 rows (d_v) x 64 tokens
-constexpr uint32_t kOffUTl = 172032;  // U^T diag(lambda)
-constexpr uint32_t kOffAf = 188416;   // A, fp32 64 x kLdA
+constexpr uint32_t kOffKQ0 = 0;       // [K;Q] buffer 0: 2 atom columns x 128 rows (K 0-63, Q 64-127)
+constexpr uint32_t kOffKQ1 = 32768;   // [K;Q] buffer 1
+constexpr uint32_t kOffV = 65536;     // V: 2 atom columns x 64 rows (intra only)
+constexpr uint32_t kOffWT = 81920;    // W^T: 128 rows (d_k) x 64 tokens
+constexpr uint32_t kOffP0 = 98304;    // P = Q K^T (.) Gamma, buffer 0: 64 x 64
+constexpr uint32_t kOffP1 = 106496;   // P, buffer 1
+constexpr uint32_t kOffS = 114688;    // S operand (bf16): 2 atom columns x 128 rows (chain only)
+constexpr uint32_t kOffUT = 147456;   // U^T: 128 rows (d_v) x 64 tokens; then the output staging tile
+constexpr uint32_t kOffUTl = 163840;  // U^T diag(lambda)
+constexpr uint32_t kOffAf = 180224;   // A, fp32 64 x kLdA; after the inverse: T' (8 KB) and T'' (8 KB)
+constexpr uint32_t kOffTp = kOffAf, kOffTpp = kOffAf + 8192;
 constexpr uint32_t kOffTf = kOffAf + 64 * kLdA * 4;  // T, fp32 64 x kLdA
 constexpr uint32_t kOffY = kOffTf + 64 * kLdA * 4;   // inverse scratch, 32 x kLdY fp32
-constexpr uint32_t kOffVec = kOffY + 32 * kLdY * 4;  // per-token vectors, 8 x 64 fp32
-constexpr uint32_t kOffBar = kOffVec + 8 * 64 * 4;   // 4 mbarriers + tensor-memory slot
-constexpr uint32_t kSmemBytes = kOffBar + 64 + 1024; // + alignment slack
+constexpr uint32_t kOffVec0 = kOffY + 32 * kLdY * 4;  // per-token vectors of buffer 0 (6 x 64 fp32)
+constexpr uint32_t kOffVec1 = kOffVec0 + 6 * 64 * 4;  // buffer 1
+constexpr uint32_t kOffBar = kOffVec1 + 6 * 64 * 4;   // mbarriers, tensor-memory slot, unit slot
+constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024; // + alignment slack
+static_assert(kOffTpp + 8192 <= kOffTf, "T' and T'' must fit in the A scratch");
 static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 per-block limit");
+// per-token vectors inside a buffer (floats)
+constexpr int kVecG = 0, kVecB = 64, kVecGam = 128, kVecBG = 192, kVecLam = 256, kVecIGam = 320;
+// mbarrier slots
+constexpr int kBarTKQ = 0, kBarTV = 2, kBarI = 3, kBarC = 4, kBarFull = 5, kBarEmpty = 7, kBarWT = 9, kNumBars = 10;
 
-// Tensor-memory columns (fp32, 128 lanes each).  The state S (d_v lanes x
-// d_k columns) lives at kColS for the whole unit and is the accumulator of
-// the state-update product.
-constexpr uint32_t kColGram = 0, kColW = 64, kColU = 128, kColX1 = 192, kColX2 = 256, kColS = 320;
+// Tensor-memory columns (fp32, 128 lanes each).
+constexpr uint32_t kColGram = 0, kColW = 64, kColU0 = 128, kColU1 = 192, kColX1 = 256, kColX2 = 320, kColS = 384;
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t kBytesKQ = 4 * 8192;  // four 64 x 64 bf16 boxes
 constexpr uint32_t kBytesV = 2 * 8192;
 
+__device__ __forceinline__ void named_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Barrier over one warp group that also ORs a predicate across it.
+__device__ __forceinline__ bool named_sync_or(int id, int count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(uint32_t(pred)), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void store_row_bf16(uint32_t tile, int row, int chunk0, const float *x, int nchunks) {
 #pragma unroll
     for (int c = 0; c < nchunks; ++c) st_shared_v4(tile + sw128_offset(row, chunk0 + c), pack_bf16x8(x + 8 * c));
+}
+
+__device__ __forceinline__ void load4(const float *p, float *x) {
+    const float4 t = *reinterpret_cast<const float4 *>(p);
+    x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
 }
 
 // T = (I + A)^-1 for the 64 x 64 unit-lower-triangular system, fp32, in
@@ -89,21 +134,18 @@ __device__ __forceinline__ void store_row_bf16(uint32_t tile, int row, int chunk
 // the four 16 x 16 diagonal blocks by row-wise forward substitution (one
 // thread per column), then the two 32 x 32 halves (two 16 x 16 products each),
 // then the 64 x 64 matrix (two 32 x 32 products, 2 x 2 outputs per thread).
-// The strictly-upper 16 x 16 blocks inside each 32 x 32 half must be zero in
-// Tf on entry (they are zeroed once and never written).  All threads call it.
-__device__ void invert_unit_lower(const float *Af, float *Tf, float *Y, int tid) {
-    if (tid < 64) {
-        const int b = tid >> 4, c = tid & 15;
+// Everything of Tf above the diagonal must be zero on entry (it is zeroed once
+// and never written).  Called by the 256 threads of the intra group (t = 0..255).
+__device__ void invert_unit_lower(const float *Af, float *Tf, float *Y, int t) {
+    if (t < 64) {
+        const int b = t >> 4, c = t & 15;
         const float *Ab = Af + (16 * b) * kLdA + 16 * b;
         float x[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
             float a[16];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 t = *reinterpret_cast<const float4 *>(Ab + r * kLdA + 4 * q);
-                a[4 * q] = t.x; a[4 * q + 1] = t.y; a[4 * q + 2] = t.z; a[4 * q + 3] = t.w;
-            }
+            for (int q = 0; q < 4; ++q) load4(Ab + r * kLdA + 4 * q, a + 4 * q);
             float acc0 = (r == c) ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
             for (int jj = 0; jj < r; ++jj) {
@@ -116,76 +158,92 @@ __device__ void invert_unit_lower(const float *Af, float *Tf, float *Y, int tid)
 #pragma unroll
         for (int r = 0; r < 16; ++r) Tb[r * kLdA + c] = x[r];
     }
-    __syncthreads();
+    named_sync(kBarIntra, kIntra);
     // 32 x 32 halves p = 0, 1: Y_p = A[32p+16.., 32p..] B_{2p}, T[32p+16.., 32p..] = -B_{2p+1} Y_p
-    const int p = tid >> 7, e = tid & 127, r1 = e >> 3, c1 = (e & 7) * 2;
+    const int p = t >> 7, e = t & 127, r1 = e >> 3, c1 = (e & 7) * 2;
     {
         const float *Arow = Af + (32 * p + 16 + r1) * kLdA + 32 * p;
         const float *Bm = Tf + (32 * p) * kLdA + 32 * p;
         float z0 = 0.f, z1 = 0.f;
 #pragma unroll
         for (int m = 0; m < 16; ++m) {
-            const float a = Arow[m];
-            const float2 t = *reinterpret_cast<const float2 *>(Bm + m * kLdA + c1);
-            z0 = fmaf(a, t.x, z0);
-            z1 = fmaf(a, t.y, z1);
+            const float av = Arow[m];
+            const float2 tv = *reinterpret_cast<const float2 *>(Bm + m * kLdA + c1);
+            z0 = fmaf(av, tv.x, z0);
+            z1 = fmaf(av, tv.y, z1);
         }
         *reinterpret_cast<float2 *>(Y + (16 * p + r1) * kLdY + c1) = make_float2(z0, z1);
     }
-    __syncthreads();
+    named_sync(kBarIntra, kIntra);
     {
         const float *Brow = Tf + (32 * p + 16 + r1) * kLdA + 32 * p + 16;
         float z0 = 0.f, z1 = 0.f;
 #pragma unroll
         for (int m = 0; m < 16; ++m) {
             const float bm = Brow[m];  // zero above the diagonal
-            const float2 t = *reinterpret_cast<const float2 *>(Y + (16 * p + m) * kLdY + c1);
-            z0 = fmaf(bm, t.x, z0);
-            z1 = fmaf(bm, t.y, z1);
+            const float2 tv = *reinterpret_cast<const float2 *>(Y + (16 * p + m) * kLdY + c1);
+            z0 = fmaf(bm, tv.x, z0);
+            z1 = fmaf(bm, tv.y, z1);
         }
         *reinterpret_cast<float2 *>(Tf + (32 * p + 16 + r1) * kLdA + 32 * p + c1) = make_float2(-z0, -z1);
     }
-    __syncthreads();
+    named_sync(kBarIntra, kIntra);
     // 64 x 64: Y = A[32.., 0..32] T_a, T[32.., 0..32] = -T_b Y
-    const int r0 = (tid >> 4) * 2, c0 = (tid & 15) * 2;
+    const int r0 = (t >> 4) * 2, c0 = (t & 15) * 2;
     {
         const float *A0 = Af + (32 + r0) * kLdA, *A1 = A0 + kLdA;
         float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 a0 = *reinterpret_cast<const float4 *>(A0 + 4 * k4);
-            const float4 a1 = *reinterpret_cast<const float4 *>(A1 + 4 * k4);
-            const float a0v[4] = {a0.x, a0.y, a0.z, a0.w}, a1v[4] = {a1.x, a1.y, a1.z, a1.w};
+            float a0v[4], a1v[4];
+            load4(A0 + 4 * k4, a0v);
+            load4(A1 + 4 * k4, a1v);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const float2 t = *reinterpret_cast<const float2 *>(Tf + (4 * k4 + u) * kLdA + c0);
-                y00 = fmaf(a0v[u], t.x, y00); y01 = fmaf(a0v[u], t.y, y01);
-                y10 = fmaf(a1v[u], t.x, y10); y11 = fmaf(a1v[u], t.y, y11);
+                const float2 tv = *reinterpret_cast<const float2 *>(Tf + (4 * k4 + u) * kLdA + c0);
+                y00 = fmaf(a0v[u], tv.x, y00); y01 = fmaf(a0v[u], tv.y, y01);
+                y10 = fmaf(a1v[u], tv.x, y10); y11 = fmaf(a1v[u], tv.y, y11);
             }
         }
         *reinterpret_cast<float2 *>(Y + r0 * kLdY + c0) = make_float2(y00, y01);
         *reinterpret_cast<float2 *>(Y + (r0 + 1) * kLdY + c0) = make_float2(y10, y11);
     }
-    __syncthreads();
+    named_sync(kBarIntra, kIntra);
     {
         const float *B0 = Tf + (32 + r0) * kLdA + 32, *B1 = B0 + kLdA;
         float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 b0 = *reinterpret_cast<const float4 *>(B0 + 4 * k4);
-            const float4 b1 = *reinterpret_cast<const float4 *>(B1 + 4 * k4);
-            const float b0v[4] = {b0.x, b0.y, b0.z, b0.w}, b1v[4] = {b1.x, b1.y, b1.z, b1.w};
+            float b0v[4], b1v[4];
+            load4(B0 + 4 * k4, b0v);
+            load4(B1 + 4 * k4, b1v);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const float2 t = *reinterpret_cast<const float2 *>(Y + (4 * k4 + u) * kLdY + c0);
-                y00 = fmaf(b0v[u], t.x, y00); y01 = fmaf(b0v[u], t.y, y01);
-                y10 = fmaf(b1v[u], t.x, y10); y11 = fmaf(b1v[u], t.y, y11);
+                const float2 tv = *reinterpret_cast<const float2 *>(Y + (4 * k4 + u) * kLdY + c0);
+                y00 = fmaf(b0v[u], tv.x, y00); y01 = fmaf(b0v[u], tv.y, y01);
+                y10 = fmaf(b1v[u], tv.x, y10); y11 = fmaf(b1v[u], tv.y, y11);
             }
         }
         *reinterpret_cast<float2 *>(Tf + (32 + r0) * kLdA + c0) = make_float2(-y00, -y01);
         *reinterpret_cast<float2 *>(Tf + (32 + r0 + 1) * kLdA + c0) = make_float2(-y10, -y11);
     }
-    __syncthreads();
+    named_sync(kBarIntra, kIntra);
+}
+
+// Loads chunk `c0` of q and k for q/k head `hq` into a [K;Q] buffer.
+__device__ __forceinline__ void load_kq(uint32_t dst, uint32_t bar, const CUtensorMap *tk, const CUtensorMap *tq,
+                                        int hq, int c0) {
+    mbar_arrive_expect_tx(bar, kBytesKQ);
+    tma_load_3d(dst, tk, 0, hq, c0, bar);
+    tma_load_3d(dst + 8192, tq, 0, hq, c0, bar);
+    tma_load_3d(dst + 16384, tk, 64, hq, c0, bar);
+    tma_load_3d(dst + 24576, tq, 64, hq, c0, bar);
+}
+
+__device__ __forceinline__ void load_v(uint32_t dst, uint32_t bar, const CUtensorMap *tv, int h, int c0) {
+    mbar_arrive_expect_tx(bar, kBytesV);
+    tma_load_3d(dst, tv, 0, h, c0, bar);
+    tma_load_3d(dst + 8192, tv, 64, h, c0, bar);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -200,50 +258,39 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float *Af = reinterpret_cast<float *>(smem + kOffAf);
     float *Tf = reinterpret_cast<float *>(smem + kOffTf);
     float *Yb = reinterpret_cast<float *>(smem + kOffY);
-    float *gs = reinterpret_cast<float *>(smem + kOffVec);  // g, then its prefix sums G
-    float *bs = gs + 64;                                   // beta
-    float *gam = gs + 128;                                 // gamma = e^G
-    float *bg = gs + 192;                                  // beta gamma
-    float *lam = gs + 256;                                 // e^(G_C - G), 0 past the sequence end
-    float *igam = gs + 320;                                // e^(-G), used when the chunk's decay is mild
-    const uint32_t bar_kq0 = sb + kOffBar, bar_kq1 = sb + kOffBar + 8, bar_v = sb + kOffBar + 16,
-                   bar_mma = sb + kOffBar + 24;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + kOffBar + 32);
-    int *s_unit = reinterpret_cast<int *>(smem + kOffBar + 40);
+    const uint32_t bars = sb + kOffBar;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + kOffBar + 8 * kNumBars);
+    int *s_unit = reinterpret_cast<int *>(smem + kOffBar + 8 * kNumBars + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quarter = warp & 3, half = warp >> 2;
-    const int row = quarter * 32 + lane;  // tensor-memory lane = accumulator row of this thread
-    const uint32_t lane_bits = uint32_t(quarter * 32) << 16;
+    const bool is_chain = warp < 4;
+    const uint32_t lane_bits = uint32_t((warp & 3) * 32) << 16;  // this warp's tensor-memory lane quarter
     WsHeader *hdr = a.sched.hdr;
     if (hdr->status != GDN_OK) return;
 
     if (tid == 0) {
-        mbar_init(bar_kq0, 1);
-        mbar_init(bar_kq1, 1);
-        mbar_init(bar_v, 1);
-        mbar_init(bar_mma, 1);
+        for (int i = 0; i < kNumBars; ++i) mbar_init(bars + 8 * i, 1);
         fence_mbarrier_init();
     }
     if (warp == 0) {
         tmem_alloc(smem_u32(tslot), kTmemCols);
         tmem_relinquish();
     }
+    // T starts all zero: the inverse writes only the lower-triangular blocks
+    // (and zeros above the diagonal inside the diagonal blocks), so everything
+    // above the diagonal reads as zero for the rest of the kernel.
+    if (!is_chain)
+        for (int e = tid - kChain; e < 64 * kLdA; e += kIntra) Tf[e] = 0.f;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    // T starts all zero: the inverse writes only the lower-triangular blocks
-    // (and zeros above the diagonal inside the diagonal blocks), so everything
-    // above the diagonal reads as zero for the rest of the kernel.
-    for (int e = tid; e < 64 * kLdA; e += kThreads) Tf[e] = 0.f;
-    __syncthreads();
 
     const int hv = a.hv, hk = a.hk, group = hv / hk;
     const int total_units = a.num_seqs * hv;
     __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(a.o);
-    uint32_t ph_kq0 = 0, ph_kq1 = 0, ph_v = 0, ph_mma = 0;
-    uint32_t pending = 0;  // (tid 0) bit 0/1: KQ buffer load in flight, bit 2: V load in flight
+    uint32_t gn = 0;  // chunks this CTA has processed so far (selects buffers and barrier phases)
+    uint32_t ph_full = 0, ph_empty = 0, ph_tkq = 0, ph_v = 0, ph_i = 0, ph_c = 0, ph_wt = 0;
     bool aborted = false;
 
     const uint32_t id_gram = idesc_bf16(128, 64, false, false);
@@ -253,364 +300,391 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t id_ds = idesc_bf16(128, 128, false, true);  // state update, accumulates into S
 
     for (;;) {
+        if (__syncthreads_or(aborted)) break;
         if (tid == 0) *s_unit = int(atomicAdd(&hdr->next_unit, 1u));
         __syncthreads();
         const int unit = *s_unit;
-        __syncthreads();
         if (unit >= total_units) break;
         const int seq = a.sched.order[unit / hv];
         const int h = unit % hv, hq = h / group;
         const int t0 = a.sched.start[seq], len = a.sched.len[seq];
         const int nchunks = (len + 63) / 64;
         const size_t sbase = (size_t(seq) * hv + h) * 128 * 128;
-
         if (tid == 0 && nchunks > 0) {
-            mbar_arrive_expect_tx(bar_kq0, kBytesKQ);
-            tma_load_3d(sb + kOffKQ0, &tm_k, 0, hq, t0, bar_kq0);
-            tma_load_3d(sb + kOffKQ0 + 8192, &tm_q, 0, hq, t0, bar_kq0);
-            tma_load_3d(sb + kOffKQ0 + 16384, &tm_k, 64, hq, t0, bar_kq0);
-            tma_load_3d(sb + kOffKQ0 + 24576, &tm_q, 64, hq, t0, bar_kq0);
-            mbar_arrive_expect_tx(bar_v, kBytesV);
-            tma_load_3d(sb + kOffV, &tm_v, 0, h, t0, bar_v);
-            tma_load_3d(sb + kOffV + 8192, &tm_v, 64, h, t0, bar_v);
-            pending |= 1u | 4u;
+            load_kq(sb + ((gn & 1) ? kOffKQ1 : kOffKQ0), bars + 8 * (kBarTKQ + (gn & 1)), &tm_k, &tm_q, hq, t0);
+            if (nchunks > 1)
+                load_kq(sb + (((gn + 1) & 1) ? kOffKQ1 : kOffKQ0), bars + 8 * (kBarTKQ + ((gn + 1) & 1)), &tm_k,
+                        &tm_q, hq, t0 + 64);
+            load_v(sb + kOffV, bars + 8 * kBarTV, &tm_v, h, t0);
         }
-        // gates of the first chunk (threads 0-63 keep one chunk of g, beta in flight)
-        float g_next = 0.f, b_next = 0.f;
-        if (tid < 64 && tid < len) {
-            g_next = a.g[size_t(t0 + tid) * hv + h];
-            b_next = a.beta[size_t(t0 + tid) * hv + h];
-        }
-        // initial state into tensor memory (this thread: lane `row`, 64 key columns)
-#pragma unroll
-        for (int p2 = 0; p2 < 2; ++p2) {
-            float v[32];
-            if (a.s0) {
-                const float4 *src =
-                    reinterpret_cast<const float4 *>(a.s0 + sbase + size_t(row) * 128 + 64 * half + 32 * p2);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const float4 x = src[c];
-                    v[4 * c] = x.x; v[4 * c + 1] = x.y; v[4 * c + 2] = x.z; v[4 * c + 3] = x.w;
-                }
-            } else {
-#pragma unroll
-                for (int c = 0; c < 32; ++c) v[c] = 0.f;
-            }
-            tmem_st32(tmem + lane_bits + kColS + 64 * half + 32 * p2, v);
-        }
-        tmem_wait_st();
 
-        for (int n = 0; n < nchunks; ++n) {
-            const int c0 = t0 + n * 64;
-            const int L = min(64, len - n * 64);
-            const int buf = n & 1;
-            const uint32_t kq = sb + (buf ? kOffKQ1 : kOffKQ0);
-            if (tid < 64) {
-                gs[tid] = tid < L ? fmaxf(g_next, kGFloor) : 0.f;
-                bs[tid] = tid < L ? b_next : 0.f;
-                // prefetch the next chunk's gates; they are consumed one chunk later
-                if (n + 1 < nchunks && tid < min(64, len - (n + 1) * 64)) {
-                    const size_t off = size_t(c0 + 64 + tid) * hv + h;
-                    g_next = a.g[off];
-                    b_next = a.beta[off];
+        if (is_chain) {
+            // ================= chain group: one thread per state row =================
+            const int row = tid;
+            // initial state into tensor memory
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                float v[32];
+                if (a.s0) {
+                    const float *src = a.s0 + sbase + size_t(row) * 128 + 32 * c4;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) load4(src + 4 * c, v + 4 * c);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) v[c] = 0.f;
                 }
+                tmem_st32(tmem + lane_bits + kColS + 32 * c4, v);
             }
-            // (1) Gram, once this chunk's K and Q are in
-            {
-                const bool ok = mbar_wait(buf ? bar_kq1 : bar_kq0, buf ? ph_kq1 : ph_kq0);
-                if (buf) ph_kq1 ^= 1; else ph_kq0 ^= 1;
-                if (__syncthreads_or(!ok)) { aborted = true; break; }
-            }
-            if (tid == 0) {
-                pending &= ~(1u << buf);
-                if (n + 1 < nchunks) {
-                    const uint32_t nb = buf ? kOffKQ0 : kOffKQ1, nbar = buf ? bar_kq0 : bar_kq1;
-                    mbar_arrive_expect_tx(nbar, kBytesKQ);
-                    tma_load_3d(sb + nb, &tm_k, 0, hq, c0 + 64, nbar);
-                    tma_load_3d(sb + nb + 8192, &tm_q, 0, hq, c0 + 64, nbar);
-                    tma_load_3d(sb + nb + 16384, &tm_k, 64, hq, c0 + 64, nbar);
-                    tma_load_3d(sb + nb + 24576, &tm_q, 64, hq, c0 + 64, nbar);
-                    pending |= 1u << (buf ^ 1);
+            tmem_wait_st();
+            for (int n = 0; n < nchunks; ++n) {
+                const uint32_t gcn = gn + n, b = gcn & 1;
+                const int c0 = t0 + n * 64, L = min(64, len - n * 64);
+                const float *vec = reinterpret_cast<const float *>(smem + (b ? kOffVec1 : kOffVec0));
+                const uint32_t kq = sb + (b ? kOffKQ1 : kOffKQ0);
+                const uint32_t pt = sb + (b ? kOffP1 : kOffP0);
+                const uint32_t colU = b ? kColU1 : kColU0;
+                {
+                    const bool ok = mbar_wait(bars + 8 * (kBarFull + b), (ph_full >> b) & 1u);
+                    ph_full ^= 1u << b;
+                    if (named_sync_or(kBarChain, kChain, !ok)) { aborted = true; break; }
                 }
                 tc_fence_after();
+                // state pass: S_n -> bf16 operand, S <- gamma_C S_n in place
+                {
+                    const float gC = vec[kVecGam + 63];  // padded rows carry g = 0, so G_63 = G_{L-1}
 #pragma unroll
-                for (int s = 0; s < 8; ++s) {
-                    const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
-                    mma_bf16(tmem + kColGram, smem_desc(kq + off, 16, 1024), smem_desc(kq + off, 16, 1024), id_gram,
-                             s > 0);
-                }
-                mma_commit(bar_mma);
-            }
-            // chunk-local prefix sums of g (warp 0) while the Gram runs
-            if (warp == 0) {
-                const float g0 = gs[2 * lane], g1 = gs[2 * lane + 1];
-                float incl = g0 + g1;
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float v0[32], v1[32];
+                        tmem_ld32(tmem + lane_bits + kColS + 64 * hh, v0);
+                        tmem_ld32(tmem + lane_bits + kColS + 64 * hh + 32, v1);
+                        tmem_wait_ld();
+                        store_row_bf16(sb + kOffS + hh * 16384, row, 0, v0, 4);
+                        store_row_bf16(sb + kOffS + hh * 16384, row, 4, v1, 4);
 #pragma unroll
-                for (int d = 1; d < 32; d <<= 1) {
-                    const float t = __shfl_up_sync(0xffffffffu, incl, d);
-                    if (lane >= d) incl += t;
+                        for (int j = 0; j < 32; ++j) {
+                            v0[j] *= gC;
+                            v1[j] *= gC;
+                        }
+                        tmem_st32(tmem + lane_bits + kColS + 64 * hh, v0);
+                        tmem_st32(tmem + lane_bits + kColS + 64 * hh + 32, v1);
+                    }
+                    tmem_wait_st();
                 }
-                const float excl = incl - (g0 + g1);
-                gs[2 * lane] = excl + g0;
-                gs[2 * lane + 1] = excl + g0 + g1;
-            }
-            __syncthreads();
-            if (tid < 64) {
-                const float G = gs[tid];
-                gam[tid] = __expf(G);
-                bg[tid] = bs[tid] * __expf(G);
-                lam[tid] = tid < L ? __expf(gs[L - 1] - G) : 0.f;
-                igam[tid] = __expf(-G);
-            }
-            // S pass: the chunk-start state S_n becomes the bf16 operand, and the
-            // fp32 state in tensor memory is decayed to gamma_C S_n so that the
-            // state-update product can accumulate onto it.  Padded rows carry
-            // g = 0, so G_63 = G_{L-1}.
-            {
-                const float gC = __expf(gs[63]);
-                float v0[32], v1[32];
-                tmem_ld32(tmem + lane_bits + kColS + 64 * half, v0);
-                tmem_ld32(tmem + lane_bits + kColS + 64 * half + 32, v1);
-                tmem_wait_ld();
-                store_row_bf16(sb + kOffS + half * 16384, row, 0, v0, 4);
-                store_row_bf16(sb + kOffS + half * 16384, row, 4, v1, 4);
+                fence_proxy_async_shared();
+                tc_fence_before();
+                named_sync(kBarChain, kChain);
+                // (4) U^T = U~^T - S W^T and (5) X1 = S Q^T
+                if (tid == 0) {
+                    tc_fence_after();
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    v0[jj] *= gC;
-                    v1[jj] *= gC;
-                }
-                tmem_st32(tmem + lane_bits + kColS + 64 * half, v0);
-                tmem_st32(tmem + lane_bits + kColS + 64 * half + 32, v1);
-                tmem_wait_st();
-            }
-            fence_proxy_async_shared();
-            {
-                const bool ok = mbar_wait(bar_mma, ph_mma);
-                ph_mma ^= 1;
-                if (__syncthreads_or(!ok)) { aborted = true; break; }
-            }
-            tc_fence_after();
-            // A (fp32, for the inverse) and P (bf16 operand) from the Gram
-            {
-                float v[32], gj[32];
-                tmem_ld32(tmem + lane_bits + kColGram + 32 * half, v);
+                    for (int s = 0; s < 8; ++s) {
+                        const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+                        mma_bf16(tmem + colU, smem_desc(sb + kOffS + off, 16, 1024),
+                                 smem_desc(sb + kOffWT + s * 2048, 16384, 1024), id_u, 1);
+                    }
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 t = *reinterpret_cast<const float4 *>(gs + 32 * half + 4 * q);
-                    gj[4 * q] = t.x; gj[4 * q + 1] = t.y; gj[4 * q + 2] = t.z; gj[4 * q + 3] = t.w;
+                    for (int s = 0; s < 8; ++s) {
+                        const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+                        mma_bf16(tmem + kColX1, smem_desc(sb + kOffS + off, 16, 1024),
+                                 smem_desc(kq + 8192 + off, 16, 1024), id_x, s > 0);
+                    }
+                    mma_commit(bars + 8 * kBarC);
                 }
-                const int r = row & 63;
-                const float Gr = gs[r];
-                const bool is_a = row < 64;
-                const float scale = is_a ? bs[r] : 1.f;
-                const int lim = is_a ? r : r + 1;  // A: j < r;  P: j <= r
-                float x[32];
-                // Gamma_rj = e^(G_r - G_j).  While the chunk's total log-decay is
-                // at least -80, e^(-G_j) stays finite in fp32 and Gamma is the
-                // rank-1 product e^(G_r) e^(-G_j) (64 exponentials, not 4096).
-                if (gs[63] >= -80.f) {
-                    float ig[32];
+                {
+                    const bool ok = mbar_wait(bars + 8 * kBarC, ph_c);
+                    ph_c ^= 1u;
+                    if (named_sync_or(kBarChain, kChain, !ok)) { aborted = true; break; }
+                }
+                tc_fence_after();
+                if (tid == 0) mbar_arrive(bars + 8 * kBarWT);  // W^T consumed
+                // U epilogue: U^T rows to bf16 operands (plain and lambda-scaled)
+                {
+                    float v0[32], v1[32];
+                    tmem_ld32(tmem + lane_bits + colU, v0);
+                    tmem_ld32(tmem + lane_bits + colU + 32, v1);
+                    float l0[32], l1[32];
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const float4 t = *reinterpret_cast<const float4 *>(igam + 32 * half + 4 * q);
-                        ig[4 * q] = t.x; ig[4 * q + 1] = t.y; ig[4 * q + 2] = t.z; ig[4 * q + 3] = t.w;
+                        load4(vec + kVecLam + 4 * q, l0 + 4 * q);
+                        load4(vec + kVecLam + 32 + 4 * q, l1 + 4 * q);
                     }
-                    const float sg = scale * gam[r];
                     tmem_wait_ld();
+                    store_row_bf16(sb + kOffUT, row, 0, v0, 4);
+                    store_row_bf16(sb + kOffUT, row, 4, v1, 4);
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const float keep = (32 * half + jj < lim) ? 1.f : 0.f;
-                        x[jj] = keep * sg * ig[jj] * v[jj];
+                    for (int j = 0; j < 32; ++j) {
+                        l0[j] *= v0[j];
+                        l1[j] *= v1[j];
                     }
-                } else {
+                    store_row_bf16(sb + kOffUTl, row, 0, l0, 4);
+                    store_row_bf16(sb + kOffUTl, row, 4, l1, 4);
+                }
+                fence_proxy_async_shared();
+                tc_fence_before();
+                named_sync(kBarChain, kChain);
+                // (6) X2 = U^T P^T and (7) S += U^T diag(lambda) K
+                if (tid == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        mma_bf16(tmem + kColX2, smem_desc(sb + kOffUT + s * 32, 16, 1024),
+                                 smem_desc(pt + s * 32, 16, 1024), id_x, s > 0);
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        mma_bf16(tmem + kColS, smem_desc(sb + kOffUTl + s * 32, 16, 1024),
+                                 smem_desc(kq + s * 2048, 16384, 1024), id_ds, 1);
+                    mma_commit(bars + 8 * kBarC);
+                }
+                {
+                    const bool ok = mbar_wait(bars + 8 * kBarC, ph_c);
+                    ph_c ^= 1u;
+                    if (named_sync_or(kBarChain, kChain, !ok)) { aborted = true; break; }
+                }
+                tc_fence_after();
+                // the [K;Q] buffer is free: refill it two chunks ahead
+                if (tid == 0 && n + 2 < nchunks) load_kq(kq, bars + 8 * (kBarTKQ + b), &tm_k, &tm_q, hq, c0 + 128);
+                // output O[r][i] = gamma_r X1[i][r] + X2[i][r], staged through the
+                // U^T tile so that each token row leaves as contiguous 16-byte stores
+                {
+                    __nv_bfloat16 *Ot = reinterpret_cast<__nv_bfloat16 *>(smem + kOffUT);
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float x1[32], x2[32];
+                        tmem_ld32(tmem + lane_bits + kColX1 + 32 * hh, x1);
+                        tmem_ld32(tmem + lane_bits + kColX2 + 32 * hh, x2);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int r = 32 * hh + j;
+                            Ot[r * 128 + row] = __float2bfloat16_rn(fmaf(vec[kVecGam + r], x1[j], x2[j]));
+                        }
+                    }
+                }
+                tc_fence_before();
+                named_sync(kBarChain, kChain);
+                for (int e = tid; e < 64 * 16; e += kChain) {
+                    const int r = e >> 4, c = e & 15;
+                    if (r < L) {
+                        const uint4 val = *reinterpret_cast<const uint4 *>(smem + kOffUT + r * 256 + c * 16);
+                        *reinterpret_cast<uint4 *>(o + (size_t(c0 + r) * hv + h) * 128 + c * 8) = val;
+                    }
+                }
+                named_sync(kBarChain, kChain);
+                if (tid == 0) mbar_arrive(bars + 8 * (kBarEmpty + b));  // buffers b may be refilled
+            }
+            if (!aborted) {
+                // final state out of tensor memory
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    float v[32];
+                    tmem_ld32(tmem + lane_bits + kColS + 32 * c4, v);
                     tmem_wait_ld();
+                    if (a.s_final) {
+                        float4 *dst = reinterpret_cast<float4 *>(a.s_final + sbase + size_t(row) * 128 + 32 * c4);
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        // branch-free: every lane evaluates the exponential, a 0/1 factor masks it
-                        const float keep = (32 * half + jj < lim) ? 1.f : 0.f;
-                        x[jj] = keep * scale * __expf(fminf(Gr - gj[jj], 0.f)) * v[jj];
+                        for (int c = 0; c < 8; ++c) dst[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
                     }
                 }
-                if (is_a) {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        *reinterpret_cast<float4 *>(Af + r * kLdA + 32 * half + 4 * q) =
-                            make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
-                } else {
-                    store_row_bf16(sb + kOffP, r, 4 * half, x, 4);
-                }
+                tc_fence_before();
             }
-            fence_proxy_async_shared();
-            tc_fence_before();
-            __syncthreads();
-            invert_unit_lower(Af, Tf, Yb, tid);
-            for (int e = tid; e < 64 * 8; e += kThreads) {
-                const int r = e >> 3, c8 = e & 7;
-                float t[8], b1[8], b2[8], x1[8], x2[8];
-#pragma unroll
-                for (int hq4 = 0; hq4 < 2; ++hq4) {
-                    const float4 tv = *reinterpret_cast<const float4 *>(Tf + r * kLdA + 8 * c8 + 4 * hq4);  // zero above the diagonal
-                    const float4 bv = *reinterpret_cast<const float4 *>(bg + 8 * c8 + 4 * hq4);
-                    const float4 sv = *reinterpret_cast<const float4 *>(bs + 8 * c8 + 4 * hq4);
-                    t[4 * hq4] = tv.x; t[4 * hq4 + 1] = tv.y; t[4 * hq4 + 2] = tv.z; t[4 * hq4 + 3] = tv.w;
-                    b1[4 * hq4] = bv.x; b1[4 * hq4 + 1] = bv.y; b1[4 * hq4 + 2] = bv.z; b1[4 * hq4 + 3] = bv.w;
-                    b2[4 * hq4] = sv.x; b2[4 * hq4 + 1] = sv.y; b2[4 * hq4 + 2] = sv.z; b2[4 * hq4 + 3] = sv.w;
-                }
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    x1[u] = t[u] * b1[u];
-                    x2[u] = t[u] * b2[u];
-                }
-                st_shared_v4(sb + kOffTp + sw128_offset(r, c8), pack_bf16x8(x1));
-                st_shared_v4(sb + kOffTpp + sw128_offset(r, c8), pack_bf16x8(x2));
+        } else {
+            // ================= intra group: next chunk's state-independent work =================
+            const int it = tid - kChain;                 // 0..255
+            const int irow = (warp & 3) * 32 + lane;     // tensor-memory lane of this thread
+            const int ih = (warp - 4) >> 2;              // which 32-column half of a 64-column tile
+            float g_next = 0.f, b_next = 0.f;            // gates kept one chunk in flight (it < 64)
+            if (it < 64 && it < len) {
+                g_next = a.g[size_t(t0 + it) * hv + h];
+                b_next = a.beta[size_t(t0 + it) * hv + h];
             }
-            fence_proxy_async_shared();
-            {
-                const bool ok = mbar_wait(bar_v, ph_v);
-                ph_v ^= 1;
-                if (__syncthreads_or(!ok)) { aborted = true; break; }
-            }
-            // (2) W^T, (3) U~^T, (5) X1 = S Q^T
-            if (tid == 0) {
-                pending &= ~4u;
+            for (int n = 0; n < nchunks; ++n) {
+                const uint32_t gcn = gn + n, b = gcn & 1;
+                const int c0 = t0 + n * 64, L = min(64, len - n * 64);
+                float *vec = reinterpret_cast<float *>(smem + (b ? kOffVec1 : kOffVec0));
+                float *gs = vec + kVecG, *bs = vec + kVecB;
+                const uint32_t kq = sb + (b ? kOffKQ1 : kOffKQ0);
+                const uint32_t pt = sb + (b ? kOffP1 : kOffP0);
+                const uint32_t colU = b ? kColU1 : kColU0;
+                if (gcn >= 2) {  // buffers b were last used by chunk gcn - 2
+                    const bool ok = mbar_wait(bars + 8 * (kBarEmpty + b), (ph_empty >> b) & 1u);
+                    ph_empty ^= 1u << b;
+                    if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
+                }
+                if (it < 64) {
+                    gs[it] = it < L ? fmaxf(g_next, kGFloor) : 0.f;
+                    bs[it] = it < L ? b_next : 0.f;
+                    if (n + 1 < nchunks && it < min(64, len - (n + 1) * 64)) {
+                        const size_t off = size_t(c0 + 64 + it) * hv + h;
+                        g_next = a.g[off];
+                        b_next = a.beta[off];
+                    }
+                }
+                {
+                    const bool ok = mbar_wait(bars + 8 * (kBarTKQ + b), (ph_tkq >> b) & 1u);
+                    ph_tkq ^= 1u << b;
+                    if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
+                }
+                // (1) Gram
+                if (it == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int s = 0; s < 8; ++s) {
+                        const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+                        mma_bf16(tmem + kColGram, smem_desc(kq + off, 16, 1024), smem_desc(kq + off, 16, 1024),
+                                 id_gram, s > 0);
+                    }
+                    mma_commit(bars + 8 * kBarI);
+                }
+                // chunk-local prefix sums of g (first intra warp) while the Gram runs
+                if (warp == 4) {
+                    const float g0 = gs[2 * lane], g1 = gs[2 * lane + 1];
+                    float incl = g0 + g1;
+#pragma unroll
+                    for (int d = 1; d < 32; d <<= 1) {
+                        const float tt = __shfl_up_sync(0xffffffffu, incl, d);
+                        if (lane >= d) incl += tt;
+                    }
+                    const float excl = incl - (g0 + g1);
+                    gs[2 * lane] = excl + g0;
+                    gs[2 * lane + 1] = excl + g0 + g1;
+                }
+                named_sync(kBarIntra, kIntra);
+                if (it < 64) {
+                    const float G = gs[it];
+                    vec[kVecGam + it] = __expf(G);
+                    vec[kVecBG + it] = bs[it] * __expf(G);
+                    vec[kVecLam + it] = it < L ? __expf(gs[L - 1] - G) : 0.f;
+                    vec[kVecIGam + it] = __expf(-G);
+                }
+                {
+                    const bool ok = mbar_wait(bars + 8 * kBarI, ph_i);
+                    ph_i ^= 1u;
+                    if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
+                }
                 tc_fence_after();
+                // A (fp32, for the inverse) and P (bf16 operand) from the Gram
+                {
+                    float v[32], x[32];
+                    tmem_ld32(tmem + lane_bits + kColGram + 32 * ih, v);
+                    const int r = irow & 63;
+                    const bool is_a = irow < 64;
+                    const float scale = is_a ? bs[r] : 1.f;
+                    const int lim = is_a ? r : r + 1;  // A: j < r;  P: j <= r
+                    // Gamma_rj = e^(G_r - G_j).  While the chunk's total log-decay is
+                    // at least -80, e^(-G_j) stays finite in fp32 and Gamma is the
+                    // rank-1 product e^(G_r) e^(-G_j) (64 exponentials, not 4096).
+                    if (gs[63] >= -80.f) {
+                        float ig[32];
 #pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + kColW, smem_desc(kq + s * 2048, 16384, 1024),
-                             smem_desc(sb + kOffTp + s * 32, 16, 1024), id_w, s > 0);
+                        for (int q = 0; q < 8; ++q) load4(vec + kVecIGam + 32 * ih + 4 * q, ig + 4 * q);
+                        const float sg = scale * vec[kVecGam + r];
+                        tmem_wait_ld();
 #pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + kColU, smem_desc(sb + kOffV + s * 2048, 8192, 1024),
-                             smem_desc(sb + kOffTpp + s * 32, 16, 1024), id_w, s > 0);
+                        for (int j = 0; j < 32; ++j) {
+                            const float keep = (32 * ih + j < lim) ? 1.f : 0.f;
+                            x[j] = keep * sg * ig[j] * v[j];
+                        }
+                    } else {
+                        float gj[32];
 #pragma unroll
-                for (int s = 0; s < 8; ++s) {
-                    const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
-                    mma_bf16(tmem + kColX1, smem_desc(sb + kOffS + off, 16, 1024),
-                             smem_desc(kq + 8192 + off, 16, 1024), id_x, s > 0);
+                        for (int q = 0; q < 8; ++q) load4(gs + 32 * ih + 4 * q, gj + 4 * q);
+                        const float Gr = gs[r];
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            // branch-free: every lane evaluates the exponential, a 0/1 factor masks it
+                            const float keep = (32 * ih + j < lim) ? 1.f : 0.f;
+                            x[j] = keep * scale * __expf(fminf(Gr - gj[j], 0.f)) * v[j];
+                        }
+                    }
+                    if (is_a) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            *reinterpret_cast<float4 *>(Af + r * kLdA + 32 * ih + 4 * q) =
+                                make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+                    } else {
+                        store_row_bf16(pt, r, 4 * ih, x, 4);
+                    }
                 }
-                mma_commit(bar_mma);
-            }
-            {
-                const bool ok = mbar_wait(bar_mma, ph_mma);
-                ph_mma ^= 1;
-                if (__syncthreads_or(!ok)) { aborted = true; break; }
-            }
-            tc_fence_after();
-            if (tid == 0 && n + 1 < nchunks) {
-                mbar_arrive_expect_tx(bar_v, kBytesV);
-                tma_load_3d(sb + kOffV, &tm_v, 0, h, c0 + 64, bar_v);
-                tma_load_3d(sb + kOffV + 8192, &tm_v, 64, h, c0 + 64, bar_v);
-                pending |= 4u;
-            }
-            {
-                float v[32];
-                tmem_ld32(tmem + lane_bits + kColW + 32 * half, v);
-                tmem_wait_ld();
-                store_row_bf16(sb + kOffWT, row, 4 * half, v, 4);
-            }
-            fence_proxy_async_shared();
-            tc_fence_before();
-            __syncthreads();
-            // (4) U^T = U~^T - S W^T
-            if (tid == 0) {
+                fence_proxy_async_shared();
+                tc_fence_before();
+                named_sync(kBarIntra, kIntra);
+                invert_unit_lower(Af, Tf, Yb, it);
+                // T' = T diag(beta gamma) and T'' = T diag(beta) as bf16 operands (over A)
+                for (int e = it; e < 64 * 8; e += kIntra) {
+                    const int r = e >> 3, c8 = e & 7;
+                    float tv[8], b1[8], b2[8], x1[8], x2[8];
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        load4(Tf + r * kLdA + 8 * c8 + 4 * q, tv + 4 * q);  // zero above the diagonal
+                        load4(vec + kVecBG + 8 * c8 + 4 * q, b1 + 4 * q);
+                        load4(bs + 8 * c8 + 4 * q, b2 + 4 * q);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        x1[u] = tv[u] * b1[u];
+                        x2[u] = tv[u] * b2[u];
+                    }
+                    st_shared_v4(sb + kOffTp + sw128_offset(r, c8), pack_bf16x8(x1));
+                    st_shared_v4(sb + kOffTpp + sw128_offset(r, c8), pack_bf16x8(x2));
+                }
+                fence_proxy_async_shared();
+                {
+                    const bool ok = mbar_wait(bars + 8 * kBarTV, ph_v);
+                    ph_v ^= 1u;
+                    if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
+                }
+                // (2) W^T and (3) U~^T
+                if (it == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        mma_bf16(tmem + kColW, smem_desc(kq + s * 2048, 16384, 1024),
+                                 smem_desc(sb + kOffTp + s * 32, 16, 1024), id_w, s > 0);
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        mma_bf16(tmem + colU, smem_desc(sb + kOffV + s * 2048, 8192, 1024),
+                                 smem_desc(sb + kOffTpp + s * 32, 16, 1024), id_w, s > 0);
+                    mma_commit(bars + 8 * kBarI);
+                }
+                {
+                    const bool ok = mbar_wait(bars + 8 * kBarI, ph_i);
+                    ph_i ^= 1u;
+                    if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
+                }
                 tc_fence_after();
-#pragma unroll
-                for (int s = 0; s < 8; ++s) {
-                    const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
-                    mma_bf16(tmem + kColU, smem_desc(sb + kOffS + off, 16, 1024),
-                             smem_desc(sb + kOffWT + s * 2048, 16384, 1024), id_u, 1);
+                if (it == 0 && n + 1 < nchunks) load_v(sb + kOffV, bars + 8 * kBarTV, &tm_v, h, c0 + 64);
+                if (gcn >= 1) {  // the chain has consumed the previous chunk's W^T
+                    const bool ok = mbar_wait(bars + 8 * kBarWT, ph_wt);
+                    ph_wt ^= 1u;
+                    if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
                 }
-                mma_commit(bar_mma);
-            }
-            {
-                const bool ok = mbar_wait(bar_mma, ph_mma);
-                ph_mma ^= 1;
-                if (__syncthreads_or(!ok)) { aborted = true; break; }
-            }
-            tc_fence_after();
-            {
-                float v[32], w[32];
-                tmem_ld32(tmem + lane_bits + kColU + 32 * half, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int jj = 0; jj < 32; ++jj) w[jj] = v[jj] * lam[32 * half + jj];
-                store_row_bf16(sb + kOffUT, row, 4 * half, v, 4);
-                store_row_bf16(sb + kOffUTl, row, 4 * half, w, 4);
-            }
-            fence_proxy_async_shared();
-            tc_fence_before();
-            __syncthreads();
-            // (6) X2 = U^T P^T, (7) S += U^T diag(lambda) K
-            if (tid == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + kColX2, smem_desc(sb + kOffUT + s * 32, 16, 1024),
-                             smem_desc(sb + kOffP + s * 32, 16, 1024), id_x, s > 0);
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + kColS, smem_desc(sb + kOffUTl + s * 32, 16, 1024),
-                             smem_desc(kq + s * 2048, 16384, 1024), id_ds, 1);
-                mma_commit(bar_mma);
-            }
-            {
-                const bool ok = mbar_wait(bar_mma, ph_mma);
-                ph_mma ^= 1;
-                if (__syncthreads_or(!ok)) { aborted = true; break; }
-            }
-            tc_fence_after();
-            // O[r][i] = gamma_r X1[i][r] + X2[i][r], staged through shared memory
-            // (over the inverse's scratch) so that each token row leaves as
-            // contiguous 16-byte stores
-            {
-                float x1[32], x2[32];
-                tmem_ld32(tmem + lane_bits + kColX1 + 32 * half, x1);
-                tmem_ld32(tmem + lane_bits + kColX2 + 32 * half, x2);
-                tmem_wait_ld();
-                __nv_bfloat16 *Ot = reinterpret_cast<__nv_bfloat16 *>(smem + kOffAf);
-#pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const int r = 32 * half + jj;
-                    Ot[r * 128 + row] = __float2bfloat16_rn(fmaf(gam[r], x1[jj], x2[jj]));
+                {
+                    float v[32];
+                    tmem_ld32(tmem + lane_bits + kColW + 32 * ih, v);
+                    tmem_wait_ld();
+                    store_row_bf16(sb + kOffWT, irow, 4 * ih, v, 4);
                 }
+                fence_proxy_async_shared();
+                tc_fence_before();
+                named_sync(kBarIntra, kIntra);
+                if (it == 0) mbar_arrive(bars + 8 * (kBarFull + b));  // chunk gcn ready for the chain
             }
-            tc_fence_before();
-            __syncthreads();
-            for (int e = tid; e < 64 * 16; e += kThreads) {
-                const int r = e >> 4, c = e & 15;
-                if (r < L) {
-                    const uint4 val = *reinterpret_cast<const uint4 *>(smem + kOffAf + r * 256 + c * 16);
-                    *reinterpret_cast<uint4 *>(o + (size_t(c0 + r) * hv + h) * 128 + c * 8) = val;
-                }
-            }
-            __syncthreads();
         }
-        if (aborted) break;
-        // final state out of tensor memory
-#pragma unroll
-        for (int p2 = 0; p2 < 2; ++p2) {
-            float v[32];
-            tmem_ld32(tmem + lane_bits + kColS + 64 * half + 32 * p2, v);
-            tmem_wait_ld();
-            if (a.s_final) {
-                float4 *dst = reinterpret_cast<float4 *>(a.s_final + sbase + size_t(row) * 128 + 64 * half + 32 * p2);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) dst[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-            }
-        }
-        tc_fence_before();
+        gn += uint32_t(nchunks);
     }
 
-    if (aborted && tid == 0) {
-        // let this CTA's own asynchronous work drain (bounded) before freeing tensor memory
-        mma_commit(bar_mma);
-        (void)mbar_wait(bar_mma, ph_mma);
-        if (pending & 1u) (void)mbar_wait(bar_kq0, ph_kq0);
-        if (pending & 2u) (void)mbar_wait(bar_kq1, ph_kq1);
-        if (pending & 4u) (void)mbar_wait(bar_v, ph_v);
-        hdr->bad_index = -2;
-        atomicExch(&hdr->status, int(GDN_ERR_DEVICE_CHECK));
+    if (aborted) {
+        // let this thread's own tensor-core work drain (bounded) before freeing tensor memory
+        if (tid == 0 || tid == kChain) {
+            const uint32_t bar = bars + 8 * (tid == 0 ? kBarC : kBarI);
+            mma_commit(bar);
+            (void)mbar_wait(bar, tid == 0 ? ph_c : ph_i);
+        }
+        if (tid == 0) {
+            hdr->bad_index = -2;
+            atomicExch(&hdr->status, int(GDN_ERR_DEVICE_CHECK));
+        }
     }
     tc_fence_before();
     __syncthreads();
