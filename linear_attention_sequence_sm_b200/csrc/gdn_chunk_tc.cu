@@ -30,8 +30,8 @@
 // Warp specialisation.  Only (4), (7) and the state pass depend on the state
 // carried from the previous chunk; everything else in a chunk does not.  So a
 // CTA runs two warp groups on one (sequence, value head) unit:
-//   chain  (warps 0-3):  state pass, (4)+(5), U epilogue, (6)+(7), output
-//   intra  (warps 4-11): gates and their prefix sums, (1), decay masks A and
+//   chain  (warps 0-7):  state pass, (4)+(5), U epilogue, (6)+(7), output
+//   intra  (warps 8-15): gates and their prefix sums, (1), decay masks A and
 //                        P, the triangular inverse (CUDA cores, fp32), T'
 //                        and T'', (2)+(3), W^T epilogue -- one chunk ahead.
 // They hand chunks over through mbarriers: "full[b]" (intra -> chain: W^T,
@@ -40,6 +40,7 @@
 // single W^T tile has been consumed).  q/k tiles are double-buffered; the
 // chain refills a buffer two chunks ahead as soon as its last reader (7)
 // completes.  Each group synchronises internally with its own named barrier.
+// A full chunk of output leaves through one TMA store of the staged tile.
 //
 // One CTA per SM (shared memory and the 512 tensor-memory columns force it)
 // takes units longest sequence first from an atomic counter.  Every wait is
@@ -57,8 +58,8 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kThreads = 384;      // warps 0-3: chain group; warps 4-11: intra group
-constexpr int kChain = 128, kIntra = 256;
+constexpr int kThreads = 512;      // warps 0-7: chain group; warps 8-15: intra group
+constexpr int kChain = 256, kIntra = 256;
 constexpr int kBarChain = 1, kBarIntra = 2;  // named barrier ids (0 is __syncthreads)
 constexpr int kLdA = 68;  // fp32 row stride of the A and T scratch matrices (16-byte aligned rows)
 constexpr int kLdY = 36;  // fp32 row stride of the inverse's 32 x 32 scratch
@@ -80,7 +81,8 @@ constexpr uint32_t kOffTf = kOffAf + 64 * kLdA * 4;  // T, fp32 64 x kLdA
 constexpr uint32_t kOffY = kOffTf + 64 * kLdA * 4;   // inverse scratch, 32 x kLdY fp32
 constexpr uint32_t kOffVec0 = kOffY + 32 * kLdY * 4;  // per-token vectors of buffer 0 (6 x 64 fp32)
 constexpr uint32_t kOffVec1 = kOffVec0 + 6 * 64 * 4;  // buffer 1
-constexpr uint32_t kOffBar = kOffVec1 + 6 * 64 * 4;   // mbarriers, tensor-memory slot, unit slot
+constexpr uint32_t kOffGst = kOffVec1 + 6 * 64 * 4;   // gates by TMA, per [K;Q] buffer: g, beta as 64 tokens x 4 heads
+constexpr uint32_t kOffBar = kOffGst + 2 * 2048;      // mbarriers, tensor-memory slot, unit slot
 constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024; // + alignment slack
 static_assert(kOffTpp + 8192 <= kOffTf, "T' and T'' must fit in the A scratch");
 static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 per-block limit");
@@ -93,7 +95,7 @@ constexpr int kBarTKQ = 0, kBarTV = 2, kBarI = 3, kBarC = 4, kBarFull = 5, kBarE
 constexpr uint32_t kColGram = 0, kColW = 64, kColU0 = 128, kColU1 = 192, kColX1 = 256, kColX2 = 320, kColS = 384;
 constexpr uint32_t kTmemCols = 512;
 
-constexpr uint32_t kBytesKQ = 4 * 8192;  // four 64 x 64 bf16 boxes
+constexpr uint32_t kBytesKQ = 4 * 8192 + 2 * 1024;  // four 64 x 64 bf16 boxes and two 64 x 4 fp32 gate boxes
 constexpr uint32_t kBytesV = 2 * 8192;
 
 __device__ __forceinline__ void named_sync(int id, int count) {
@@ -128,12 +130,38 @@ __device__ __forceinline__ void load4(const float *p, float *x) {
     x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
 }
 
+// c += X[0:16, 0:8nk] Z[0:8nk, n0:n0+8] for row-major fp32 blocks X (stride
+// ldx, rows from its first row) and Z (stride ldz), one warp, tf32 inputs.
+__device__ __forceinline__ void tile_mma(float (&c)[4], const float *X, int ldx, const float *Z, int ldz, int n0,
+                                         int nk, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+        if (s >= nk) break;
+        const int k = 8 * s;
+        const uint32_t av[4] = {to_tf32(X[g * ldx + k + t]), to_tf32(X[(g + 8) * ldx + k + t]),
+                                to_tf32(X[g * ldx + k + t + 4]), to_tf32(X[(g + 8) * ldx + k + t + 4])};
+        const uint32_t bv[2] = {to_tf32(Z[(k + t) * ldz + n0 + g]), to_tf32(Z[(k + t + 4) * ldz + n0 + g])};
+        mma_tf32_16x8x8(c, av, bv);
+    }
+}
+
+// D[m0.., n0..] (16 x 8 tile) = sgn * c.
+__device__ __forceinline__ void tile_store(float *D, int ldd, int m0, int n0, const float (&c)[4], float sgn,
+                                           int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    *reinterpret_cast<float2 *>(D + (m0 + g) * ldd + n0 + 2 * t) = make_float2(sgn * c[0], sgn * c[1]);
+    *reinterpret_cast<float2 *>(D + (m0 + g + 8) * ldd + n0 + 2 * t) = make_float2(sgn * c[2], sgn * c[3]);
+}
+
 // T = (I + A)^-1 for the 64 x 64 unit-lower-triangular system, fp32, in
 // shared memory, by divide and conquer on the block structure
 //   [[X, 0], [C, Z]]^-1 = [[X^-1, 0], [-Z^-1 C X^-1, Z^-1]]:
 // the four 16 x 16 diagonal blocks by row-wise forward substitution (one
-// thread per column), then the two 32 x 32 halves (two 16 x 16 products each),
-// then the 64 x 64 matrix (two 32 x 32 products, 2 x 2 outputs per thread).
+// thread per column, fp32), then the two 32 x 32 halves (two 16 x 16
+// products each) and the 64 x 64 matrix (two 32 x 32 products) as warp-level
+// tf32 products with fp32 accumulation (T is rounded to bf16 afterwards, so
+// the 10-bit tf32 mantissa is ample).
 // Everything of Tf above the diagonal must be zero on entry (it is zeroed once
 // and never written).  Called by the 256 threads of the intra group (t = 0..255).
 __device__ void invert_unit_lower(const float *Af, float *Tf, float *Y, int t) {
@@ -159,81 +187,49 @@ __device__ void invert_unit_lower(const float *Af, float *Tf, float *Y, int t) {
         for (int r = 0; r < 16; ++r) Tb[r * kLdA + c] = x[r];
     }
     named_sync(kBarIntra, kIntra);
-    // 32 x 32 halves p = 0, 1: Y_p = A[32p+16.., 32p..] B_{2p}, T[32p+16.., 32p..] = -B_{2p+1} Y_p
-    const int p = t >> 7, e = t & 127, r1 = e >> 3, c1 = (e & 7) * 2;
+    const int w = t >> 5, lane = t & 31;
+    // 32 x 32 halves p = 0, 1 (warps 0-3, one 16 x 8 tile each):
+    //   Y_p = A[32p+16.., 32p..] B_{2p};  T[32p+16.., 32p..] = -B_{2p+1} Y_p
+    if (w < 4) {
+        const int p = w >> 1, n0 = 8 * (w & 1);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        tile_mma(c, Af + (32 * p + 16) * kLdA + 32 * p, kLdA, Tf + (32 * p) * kLdA + 32 * p, kLdA, n0, 2, lane);
+        tile_store(Y + (16 * p) * kLdY, kLdY, 0, n0, c, 1.f, lane);
+    }
+    named_sync(kBarIntra, kIntra);
+    if (w < 4) {
+        const int p = w >> 1, n0 = 8 * (w & 1);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        tile_mma(c, Tf + (32 * p + 16) * kLdA + 32 * p + 16, kLdA, Y + (16 * p) * kLdY, kLdY, n0, 2, lane);
+        tile_store(Tf + (32 * p + 16) * kLdA + 32 * p, kLdA, 0, n0, c, -1.f, lane);
+    }
+    named_sync(kBarIntra, kIntra);
+    // 64 x 64 (8 warps, one 16 x 8 tile of the 32 x 32 block each):
+    //   Y = A[32.., 0..32] T_a;  T[32.., 0..32] = -T_b Y
     {
-        const float *Arow = Af + (32 * p + 16 + r1) * kLdA + 32 * p;
-        const float *Bm = Tf + (32 * p) * kLdA + 32 * p;
-        float z0 = 0.f, z1 = 0.f;
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            const float av = Arow[m];
-            const float2 tv = *reinterpret_cast<const float2 *>(Bm + m * kLdA + c1);
-            z0 = fmaf(av, tv.x, z0);
-            z1 = fmaf(av, tv.y, z1);
-        }
-        *reinterpret_cast<float2 *>(Y + (16 * p + r1) * kLdY + c1) = make_float2(z0, z1);
+        const int m0 = 16 * (w >> 2), n0 = 8 * (w & 3);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        tile_mma(c, Af + (32 + m0) * kLdA, kLdA, Tf, kLdA, n0, 4, lane);
+        tile_store(Y, kLdY, m0, n0, c, 1.f, lane);
     }
     named_sync(kBarIntra, kIntra);
     {
-        const float *Brow = Tf + (32 * p + 16 + r1) * kLdA + 32 * p + 16;
-        float z0 = 0.f, z1 = 0.f;
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            const float bm = Brow[m];  // zero above the diagonal
-            const float2 tv = *reinterpret_cast<const float2 *>(Y + (16 * p + m) * kLdY + c1);
-            z0 = fmaf(bm, tv.x, z0);
-            z1 = fmaf(bm, tv.y, z1);
-        }
-        *reinterpret_cast<float2 *>(Tf + (32 * p + 16 + r1) * kLdA + 32 * p + c1) = make_float2(-z0, -z1);
-    }
-    named_sync(kBarIntra, kIntra);
-    // 64 x 64: Y = A[32.., 0..32] T_a, T[32.., 0..32] = -T_b Y
-    const int r0 = (t >> 4) * 2, c0 = (t & 15) * 2;
-    {
-        const float *A0 = Af + (32 + r0) * kLdA, *A1 = A0 + kLdA;
-        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-#pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) {
-            float a0v[4], a1v[4];
-            load4(A0 + 4 * k4, a0v);
-            load4(A1 + 4 * k4, a1v);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float2 tv = *reinterpret_cast<const float2 *>(Tf + (4 * k4 + u) * kLdA + c0);
-                y00 = fmaf(a0v[u], tv.x, y00); y01 = fmaf(a0v[u], tv.y, y01);
-                y10 = fmaf(a1v[u], tv.x, y10); y11 = fmaf(a1v[u], tv.y, y11);
-            }
-        }
-        *reinterpret_cast<float2 *>(Y + r0 * kLdY + c0) = make_float2(y00, y01);
-        *reinterpret_cast<float2 *>(Y + (r0 + 1) * kLdY + c0) = make_float2(y10, y11);
-    }
-    named_sync(kBarIntra, kIntra);
-    {
-        const float *B0 = Tf + (32 + r0) * kLdA + 32, *B1 = B0 + kLdA;
-        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-#pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) {
-            float b0v[4], b1v[4];
-            load4(B0 + 4 * k4, b0v);
-            load4(B1 + 4 * k4, b1v);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float2 tv = *reinterpret_cast<const float2 *>(Y + (4 * k4 + u) * kLdY + c0);
-                y00 = fmaf(b0v[u], tv.x, y00); y01 = fmaf(b0v[u], tv.y, y01);
-                y10 = fmaf(b1v[u], tv.x, y10); y11 = fmaf(b1v[u], tv.y, y11);
-            }
-        }
-        *reinterpret_cast<float2 *>(Tf + (32 + r0) * kLdA + c0) = make_float2(-y00, -y01);
-        *reinterpret_cast<float2 *>(Tf + (32 + r0 + 1) * kLdA + c0) = make_float2(-y10, -y11);
+        const int m0 = 16 * (w >> 2), n0 = 8 * (w & 3);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        tile_mma(c, Tf + (32 + m0) * kLdA + 32, kLdA, Y, kLdY, n0, 4, lane);
+        tile_store(Tf + 32 * kLdA, kLdA, m0, n0, c, -1.f, lane);
     }
     named_sync(kBarIntra, kIntra);
 }
 
-// Loads chunk `c0` of q and k for q/k head `hq` into a [K;Q] buffer.
+// Loads chunk `c0` of q and k for q/k head `hq` into a [K;Q] buffer, and the
+// chunk's g and beta for the four value heads around `h` into `gst`.
 __device__ __forceinline__ void load_kq(uint32_t dst, uint32_t bar, const CUtensorMap *tk, const CUtensorMap *tq,
-                                        int hq, int c0) {
+                                        int hq, int c0, uint32_t gst, const CUtensorMap *tg, const CUtensorMap *tb,
+                                        int h) {
     mbar_arrive_expect_tx(bar, kBytesKQ);
+    tma_load_2d(gst, tg, h & ~3, c0, bar);
+    tma_load_2d(gst + 1024, tb, h & ~3, c0, bar);
     tma_load_3d(dst, tk, 0, hq, c0, bar);
     tma_load_3d(dst + 8192, tq, 0, hq, c0, bar);
     tma_load_3d(dst + 16384, tk, 64, hq, c0, bar);
@@ -248,7 +244,9 @@ __device__ __forceinline__ void load_v(uint32_t dst, uint32_t bar, const CUtenso
 
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_b,
+                const PrefillArgs a) {
     extern __shared__ unsigned char smem_raw[];
     // Align to 1024 bytes with a byte offset on the shared array itself (not
     // through an integer cast), so that the compiler keeps every access below in
@@ -263,7 +261,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     int *s_unit = reinterpret_cast<int *>(smem + kOffBar + 8 * kNumBars + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const bool is_chain = warp < 4;
+    const bool is_chain = warp < 8;
     const uint32_t lane_bits = uint32_t((warp & 3) * 32) << 16;  // this warp's tensor-memory lane quarter
     WsHeader *hdr = a.sched.hdr;
     if (hdr->status != GDN_OK) return;
@@ -311,19 +309,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int nchunks = (len + 63) / 64;
         const size_t sbase = (size_t(seq) * hv + h) * 128 * 128;
         if (tid == 0 && nchunks > 0) {
-            load_kq(sb + ((gn & 1) ? kOffKQ1 : kOffKQ0), bars + 8 * (kBarTKQ + (gn & 1)), &tm_k, &tm_q, hq, t0);
+            load_kq(sb + ((gn & 1) ? kOffKQ1 : kOffKQ0), bars + 8 * (kBarTKQ + (gn & 1)), &tm_k, &tm_q, hq, t0,
+                    sb + kOffGst + (gn & 1) * 2048, &tm_g, &tm_b, h);
             if (nchunks > 1)
                 load_kq(sb + (((gn + 1) & 1) ? kOffKQ1 : kOffKQ0), bars + 8 * (kBarTKQ + ((gn + 1) & 1)), &tm_k,
-                        &tm_q, hq, t0 + 64);
+                        &tm_q, hq, t0 + 64, sb + kOffGst + ((gn + 1) & 1) * 2048, &tm_g, &tm_b, h);
             load_v(sb + kOffV, bars + 8 * kBarTV, &tm_v, h, t0);
         }
 
         if (is_chain) {
-            // ================= chain group: one thread per state row =================
-            const int row = tid;
+            // ============ chain group: thread = (state row, half of the columns) ============
+            const int row = (warp & 3) * 32 + lane;
+            const int ch = warp >> 2;
             // initial state into tensor memory
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
+            for (int c4 = 2 * ch; c4 < 2 * ch + 2; ++c4) {
                 float v[32];
                 if (a.s0) {
                     const float *src = a.s0 + sbase + size_t(row) * 128 + 32 * c4;
@@ -353,20 +353,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 {
                     const float gC = vec[kVecGam + 63];  // padded rows carry g = 0, so G_63 = G_{L-1}
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        float v0[32], v1[32];
-                        tmem_ld32(tmem + lane_bits + kColS + 64 * hh, v0);
-                        tmem_ld32(tmem + lane_bits + kColS + 64 * hh + 32, v1);
+                    for (int p2 = 0; p2 < 2; ++p2) {
+                        float v0[32];
+                        tmem_ld32(tmem + lane_bits + kColS + 64 * ch + 32 * p2, v0);
                         tmem_wait_ld();
-                        store_row_bf16(sb + kOffS + hh * 16384, row, 0, v0, 4);
-                        store_row_bf16(sb + kOffS + hh * 16384, row, 4, v1, 4);
+                        store_row_bf16(sb + kOffS + ch * 16384, row, 4 * p2, v0, 4);
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            v0[j] *= gC;
-                            v1[j] *= gC;
-                        }
-                        tmem_st32(tmem + lane_bits + kColS + 64 * hh, v0);
-                        tmem_st32(tmem + lane_bits + kColS + 64 * hh + 32, v1);
+                        for (int j = 0; j < 32; ++j) v0[j] *= gC;
+                        tmem_st32(tmem + lane_bits + kColS + 64 * ch + 32 * p2, v0);
                     }
                     tmem_wait_st();
                 }
@@ -379,16 +373,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                     for (int s = 0; s < 8; ++s) {
                         const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
-                        mma_bf16(tmem + colU, smem_desc(sb + kOffS + off, 16, 1024),
-                                 smem_desc(sb + kOffWT + s * 2048, 16384, 1024), id_u, 1);
+                        mma_bf16(tmem + colU, (smem_desc(sb, 16, 1024) + uint64_t((kOffS + off) >> 4)),
+                                 (smem_desc(sb, 16384, 1024) + uint64_t((kOffWT + s * 2048) >> 4)), id_u, 1);
                     }
 #pragma unroll
                     for (int s = 0; s < 8; ++s) {
                         const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
-                        mma_bf16(tmem + kColX1, smem_desc(sb + kOffS + off, 16, 1024),
-                                 smem_desc(kq + 8192 + off, 16, 1024), id_x, s > 0);
+                        mma_bf16(tmem + kColX1, (smem_desc(sb, 16, 1024) + uint64_t((kOffS + off) >> 4)),
+                                 (smem_desc(kq, 16, 1024) + uint64_t((8192 + off) >> 4)), id_x, s > 0);
                     }
                     mma_commit(bars + 8 * kBarC);
+                    bulk_wait_read();  // the previous chunk's output store has read the staging tile
                 }
                 {
                     const bool ok = mbar_wait(bars + 8 * kBarC, ph_c);
@@ -399,25 +394,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (tid == 0) mbar_arrive(bars + 8 * kBarWT);  // W^T consumed
                 // U epilogue: U^T rows to bf16 operands (plain and lambda-scaled)
                 {
-                    float v0[32], v1[32];
-                    tmem_ld32(tmem + lane_bits + colU, v0);
-                    tmem_ld32(tmem + lane_bits + colU + 32, v1);
-                    float l0[32], l1[32];
+                    float v[32], l[32];
+                    tmem_ld32(tmem + lane_bits + colU + 32 * ch, v);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        load4(vec + kVecLam + 4 * q, l0 + 4 * q);
-                        load4(vec + kVecLam + 32 + 4 * q, l1 + 4 * q);
-                    }
+                    for (int q = 0; q < 8; ++q) load4(vec + kVecLam + 32 * ch + 4 * q, l + 4 * q);
                     tmem_wait_ld();
-                    store_row_bf16(sb + kOffUT, row, 0, v0, 4);
-                    store_row_bf16(sb + kOffUT, row, 4, v1, 4);
+                    store_row_bf16(sb + kOffUT, row, 4 * ch, v, 4);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        l0[j] *= v0[j];
-                        l1[j] *= v1[j];
-                    }
-                    store_row_bf16(sb + kOffUTl, row, 0, l0, 4);
-                    store_row_bf16(sb + kOffUTl, row, 4, l1, 4);
+                    for (int j = 0; j < 32; ++j) l[j] *= v[j];
+                    store_row_bf16(sb + kOffUTl, row, 4 * ch, l, 4);
                 }
                 fence_proxy_async_shared();
                 tc_fence_before();
@@ -427,12 +412,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tc_fence_after();
 #pragma unroll
                     for (int s = 0; s < 4; ++s)
-                        mma_bf16(tmem + kColX2, smem_desc(sb + kOffUT + s * 32, 16, 1024),
-                                 smem_desc(pt + s * 32, 16, 1024), id_x, s > 0);
+                        mma_bf16(tmem + kColX2, (smem_desc(sb, 16, 1024) + uint64_t((kOffUT + s * 32) >> 4)),
+                                 (smem_desc(pt, 16, 1024) + uint64_t((s * 32) >> 4)), id_x, s > 0);
 #pragma unroll
                     for (int s = 0; s < 4; ++s)
-                        mma_bf16(tmem + kColS, smem_desc(sb + kOffUTl + s * 32, 16, 1024),
-                                 smem_desc(kq + s * 2048, 16384, 1024), id_ds, 1);
+                        mma_bf16(tmem + kColS, (smem_desc(sb, 16, 1024) + uint64_t((kOffUTl + s * 32) >> 4)),
+                                 (smem_desc(kq, 16384, 1024) + uint64_t((s * 2048) >> 4)), id_ds, 1);
                     mma_commit(bars + 8 * kBarC);
                 }
                 {
@@ -442,40 +427,52 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 tc_fence_after();
                 // the [K;Q] buffer is free: refill it two chunks ahead
-                if (tid == 0 && n + 2 < nchunks) load_kq(kq, bars + 8 * (kBarTKQ + b), &tm_k, &tm_q, hq, c0 + 128);
+                if (tid == 0 && n + 2 < nchunks)
+                    load_kq(kq, bars + 8 * (kBarTKQ + b), &tm_k, &tm_q, hq, c0 + 128, sb + kOffGst + b * 2048, &tm_g,
+                            &tm_b, h);
                 // output O[r][i] = gamma_r X1[i][r] + X2[i][r], staged through the
-                // U^T tile so that each token row leaves as contiguous 16-byte stores
+                // U^T tile (token-major rows of 256 bytes); a full chunk leaves in
+                // one TMA store, a ragged last chunk row by row
                 {
                     __nv_bfloat16 *Ot = reinterpret_cast<__nv_bfloat16 *>(smem + kOffUT);
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        float x1[32], x2[32];
-                        tmem_ld32(tmem + lane_bits + kColX1 + 32 * hh, x1);
-                        tmem_ld32(tmem + lane_bits + kColX2 + 32 * hh, x2);
+                    for (int sl = 0; sl < 2; ++sl) {
+                        const int r0 = 32 * ch + 16 * sl;
+                        float x1[16], x2[16], gm[16];
+                        tmem_ld16(tmem + lane_bits + kColX1 + r0, x1);
+                        tmem_ld16(tmem + lane_bits + kColX2 + r0, x2);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) load4(vec + kVecGam + r0 + 4 * q, gm + 4 * q);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int r = 32 * hh + j;
-                            Ot[r * 128 + row] = __float2bfloat16_rn(fmaf(vec[kVecGam + r], x1[j], x2[j]));
-                        }
+                        for (int j = 0; j < 16; ++j)
+                            Ot[(r0 + j) * 128 + row] = __float2bfloat16_rn(fmaf(gm[j], x1[j], x2[j]));
                     }
                 }
+                fence_proxy_async_shared();
                 tc_fence_before();
                 named_sync(kBarChain, kChain);
-                for (int e = tid; e < 64 * 16; e += kChain) {
-                    const int r = e >> 4, c = e & 15;
-                    if (r < L) {
-                        const uint4 val = *reinterpret_cast<const uint4 *>(smem + kOffUT + r * 256 + c * 16);
-                        *reinterpret_cast<uint4 *>(o + (size_t(c0 + r) * hv + h) * 128 + c * 8) = val;
+                if (L == 64) {
+                    if (tid == 0) {
+                        tma_store_3d(&tm_o, sb + kOffUT, 0, h, c0);
+                        bulk_commit();
                     }
+                } else {
+                    for (int e = tid; e < 64 * 16; e += kChain) {
+                        const int r = e >> 4, c = e & 15;
+                        if (r < L) {
+                            const uint4 val = *reinterpret_cast<const uint4 *>(smem + kOffUT + r * 256 + c * 16);
+                            *reinterpret_cast<uint4 *>(o + (size_t(c0 + r) * hv + h) * 128 + c * 8) = val;
+                        }
+                    }
+                    named_sync(kBarChain, kChain);
                 }
-                named_sync(kBarChain, kChain);
                 if (tid == 0) mbar_arrive(bars + 8 * (kBarEmpty + b));  // buffers b may be refilled
             }
             if (!aborted) {
                 // final state out of tensor memory
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
+                for (int c4 = 2 * ch; c4 < 2 * ch + 2; ++c4) {
                     float v[32];
                     tmem_ld32(tmem + lane_bits + kColS + 32 * c4, v);
                     tmem_wait_ld();
@@ -491,12 +488,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // ================= intra group: next chunk's state-independent work =================
             const int it = tid - kChain;                 // 0..255
             const int irow = (warp & 3) * 32 + lane;     // tensor-memory lane of this thread
-            const int ih = (warp - 4) >> 2;              // which 32-column half of a 64-column tile
-            float g_next = 0.f, b_next = 0.f;            // gates kept one chunk in flight (it < 64)
-            if (it < 64 && it < len) {
-                g_next = a.g[size_t(t0 + it) * hv + h];
-                b_next = a.beta[size_t(t0 + it) * hv + h];
-            }
+            const int ih = (warp - 8) >> 2;              // which 32-column half of a 64-column tile
             for (int n = 0; n < nchunks; ++n) {
                 const uint32_t gcn = gn + n, b = gcn & 1;
                 const int c0 = t0 + n * 64, L = min(64, len - n * 64);
@@ -510,34 +502,33 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     ph_empty ^= 1u << b;
                     if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
                 }
-                if (it < 64) {
-                    gs[it] = it < L ? fmaxf(g_next, kGFloor) : 0.f;
-                    bs[it] = it < L ? b_next : 0.f;
-                    if (n + 1 < nchunks && it < min(64, len - (n + 1) * 64)) {
-                        const size_t off = size_t(c0 + 64 + it) * hv + h;
-                        g_next = a.g[off];
-                        b_next = a.beta[off];
-                    }
-                }
-                {
+                if (n == 0) {  // later chunks had q, k and their Gram started by the previous chunk
                     const bool ok = mbar_wait(bars + 8 * (kBarTKQ + b), (ph_tkq >> b) & 1u);
                     ph_tkq ^= 1u << b;
                     if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
                 }
                 // (1) Gram
-                if (it == 0) {
+                if (it == 0 && n == 0) {
                     tc_fence_after();
 #pragma unroll
                     for (int s = 0; s < 8; ++s) {
                         const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
-                        mma_bf16(tmem + kColGram, smem_desc(kq + off, 16, 1024), smem_desc(kq + off, 16, 1024),
+                        mma_bf16(tmem + kColGram, (smem_desc(kq, 16, 1024) + uint64_t((off) >> 4)), (smem_desc(kq, 16, 1024) + uint64_t((off) >> 4)),
                                  id_gram, s > 0);
                     }
                     mma_commit(bars + 8 * kBarI);
                 }
-                // chunk-local prefix sums of g (first intra warp) while the Gram runs
-                if (warp == 4) {
-                    const float g0 = gs[2 * lane], g1 = gs[2 * lane + 1];
+                // gates of this chunk (arrived with q and k) and their chunk-local
+                // prefix sums, by the first intra warp while the Gram runs; tokens
+                // past the sequence end get g = beta = 0 (the identity on S)
+                if (warp == 8) {
+                    const float *stg = reinterpret_cast<const float *>(smem + kOffGst + b * 2048);
+                    const int hc = h & 3;
+                    const bool ok0 = 2 * lane < L, ok1 = 2 * lane + 1 < L;
+                    const float g0 = ok0 ? fmaxf(stg[(2 * lane) * 4 + hc], kGFloor) : 0.f;
+                    const float g1 = ok1 ? fmaxf(stg[(2 * lane + 1) * 4 + hc], kGFloor) : 0.f;
+                    bs[2 * lane] = ok0 ? stg[256 + (2 * lane) * 4 + hc] : 0.f;
+                    bs[2 * lane + 1] = ok1 ? stg[256 + (2 * lane + 1) * 4 + hc] : 0.f;
                     float incl = g0 + g1;
 #pragma unroll
                     for (int d = 1; d < 32; d <<= 1) {
@@ -562,10 +553,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
                 }
                 tc_fence_after();
-                // A (fp32, for the inverse) and P (bf16 operand) from the Gram
+                // A (fp32, for the inverse) and P (bf16 operand) from the Gram, in
+                // slices of 16 columns
                 {
-                    float v[32], x[32];
-                    tmem_ld32(tmem + lane_bits + kColGram + 32 * ih, v);
                     const int r = irow & 63;
                     const bool is_a = irow < 64;
                     const float scale = is_a ? bs[r] : 1.f;
@@ -573,37 +563,31 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     // Gamma_rj = e^(G_r - G_j).  While the chunk's total log-decay is
                     // at least -80, e^(-G_j) stays finite in fp32 and Gamma is the
                     // rank-1 product e^(G_r) e^(-G_j) (64 exponentials, not 4096).
-                    if (gs[63] >= -80.f) {
-                        float ig[32];
+                    const bool rank1 = gs[63] >= -80.f;
+                    const float sg = scale * vec[kVecGam + r], Gr = gs[r];
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) load4(vec + kVecIGam + 32 * ih + 4 * q, ig + 4 * q);
-                        const float sg = scale * vec[kVecGam + r];
+                    for (int sl = 0; sl < 2; ++sl) {
+                        const int j0 = 32 * ih + 16 * sl;
+                        float v[16], e[16], x[16];
+                        tmem_ld16(tmem + lane_bits + kColGram + j0, v);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) load4((rank1 ? vec + kVecIGam : gs) + j0 + 4 * q, e + 4 * q);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float keep = (32 * ih + j < lim) ? 1.f : 0.f;
-                            x[j] = keep * sg * ig[j] * v[j];
+                        for (int jj = 0; jj < 16; ++jj) {
+                            // branch-free: a 0/1 factor masks the strictly upper part
+                            const float keep = (j0 + jj < lim) ? 1.f : 0.f;
+                            x[jj] = rank1 ? keep * sg * e[jj] * v[jj]
+                                          : keep * scale * __expf(fminf(Gr - e[jj], 0.f)) * v[jj];
                         }
-                    } else {
-                        float gj[32];
+                        if (is_a) {
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) load4(gs + 32 * ih + 4 * q, gj + 4 * q);
-                        const float Gr = gs[r];
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            // branch-free: every lane evaluates the exponential, a 0/1 factor masks it
-                            const float keep = (32 * ih + j < lim) ? 1.f : 0.f;
-                            x[j] = keep * scale * __expf(fminf(Gr - gj[j], 0.f)) * v[j];
+                            for (int q = 0; q < 4; ++q)
+                                *reinterpret_cast<float4 *>(Af + r * kLdA + j0 + 4 * q) =
+                                    make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+                        } else {
+                            store_row_bf16(pt, r, j0 / 8, x, 2);
                         }
-                    }
-                    if (is_a) {
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            *reinterpret_cast<float4 *>(Af + r * kLdA + 32 * ih + 4 * q) =
-                                make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
-                    } else {
-                        store_row_bf16(pt, r, 4 * ih, x, 4);
                     }
                 }
                 fence_proxy_async_shared();
@@ -639,12 +623,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tc_fence_after();
 #pragma unroll
                     for (int s = 0; s < 4; ++s)
-                        mma_bf16(tmem + kColW, smem_desc(kq + s * 2048, 16384, 1024),
-                                 smem_desc(sb + kOffTp + s * 32, 16, 1024), id_w, s > 0);
+                        mma_bf16(tmem + kColW, (smem_desc(kq, 16384, 1024) + uint64_t((s * 2048) >> 4)),
+                                 (smem_desc(sb, 16, 1024) + uint64_t((kOffTp + s * 32) >> 4)), id_w, s > 0);
 #pragma unroll
                     for (int s = 0; s < 4; ++s)
-                        mma_bf16(tmem + colU, smem_desc(sb + kOffV + s * 2048, 8192, 1024),
-                                 smem_desc(sb + kOffTpp + s * 32, 16, 1024), id_w, s > 0);
+                        mma_bf16(tmem + colU, (smem_desc(sb, 8192, 1024) + uint64_t((kOffV + s * 2048) >> 4)),
+                                 (smem_desc(sb, 16, 1024) + uint64_t((kOffTpp + s * 32) >> 4)), id_w, s > 0);
                     mma_commit(bars + 8 * kBarI);
                 }
                 {
@@ -669,11 +653,30 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc_fence_before();
                 named_sync(kBarIntra, kIntra);
                 if (it == 0) mbar_arrive(bars + 8 * (kBarFull + b));  // chunk gcn ready for the chain
+                // start the next chunk's Gram as soon as its q and k are in (the Gram
+                // accumulator was consumed by this chunk's decay-mask epilogue)
+                if (n + 1 < nchunks) {
+                    const uint32_t nb = b ^ 1u, nkq = sb + (nb ? kOffKQ1 : kOffKQ0);
+                    const bool ok = mbar_wait(bars + 8 * (kBarTKQ + nb), (ph_tkq >> nb) & 1u);
+                    ph_tkq ^= 1u << nb;
+                    if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
+                    if (it == 0) {
+                        tc_fence_after();
+                        const uint64_t dk = smem_desc(nkq, 16, 1024);
+#pragma unroll
+                        for (int s = 0; s < 8; ++s) {
+                            const uint64_t d = dk + uint64_t(((s >> 2) * 16384 + (s & 3) * 32) >> 4);
+                            mma_bf16(tmem + kColGram, d, d, id_gram, s > 0);
+                        }
+                        mma_commit(bars + 8 * kBarI);
+                    }
+                }
             }
         }
         gn += uint32_t(nchunks);
     }
 
+    if (tid == 0) bulk_wait_all();  // output stores complete before the CTA's shared memory goes away
     if (aborted) {
         // let this thread's own tensor-core work drain (bounded) before freeing tensor memory
         if (tid == 0 || tid == kChain) {
@@ -711,38 +714,57 @@ EncodeTiledFn encode_fn() {
 // [tokens, heads, 128] bf16 viewed as a 3-D tensor (d fastest), boxes of
 // 64 (d) x 1 (head) x 64 (tokens), 128-byte swizzle; rows past the last token
 // read as zeros.
-bool make_map(CUtensorMap *map, const void *base, int heads, int tokens) {
+// [tokens, heads] fp32 gates viewed as 2-D, boxes of 4 heads x 64 tokens (the
+// inner box must span at least 16 bytes; the kernel picks its head's column).
+bool make_gate_map(CUtensorMap *map, const float *base, int heads, int tokens) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cuuint64_t(heads), cuuint64_t(tokens)};
+    const cuuint64_t strides[1] = {cuuint64_t(heads) * 4};
+    const cuuint32_t box[2] = {4, 64};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// With `out` set: boxes of 128 (d) x 1 x 64 tokens, no swizzle -- the
+// token-major output tile staged in shared memory.
+bool make_map(CUtensorMap *map, const void *base, int heads, int tokens, bool out = false) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[3] = {128, cuuint64_t(heads), cuuint64_t(tokens)};
     const cuuint64_t strides[2] = {128 * 2, cuuint64_t(heads) * 128 * 2};
-    const cuuint32_t box[3] = {64, 1, 64};
+    const cuuint32_t box[3] = {out ? 128u : 64u, 1, 64};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+               CU_TENSOR_MAP_INTERLEAVE_NONE, out ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
 bool chunk_tc_supported(const gdn_shape_t &s) {
-    return s.dtype == GDN_DTYPE_BF16 && s.head_dim_k == 128 && s.head_dim_v == 128 && s.chunk_size == 64;
+    // value heads in multiples of 4: the gates arrive as boxes of 4 heads
+    return s.dtype == GDN_DTYPE_BF16 && s.head_dim_k == 128 && s.head_dim_v == 128 && s.chunk_size == 64 &&
+           s.num_v_heads % 4 == 0;
 }
 
 cudaError_t launch_chunk_tc(const PrefillArgs &a, cudaStream_t stream, int num_sms) {
     // With no tokens at all there is nothing to load; the fp32 kernel writes
     // the final states (= initial states) of the empty sequences.
     if (a.tokens <= 0) return launch_chunk_simt(a, stream, num_sms);
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo, mg, mb;
     if (!make_map(&mq, a.q, a.hk, a.tokens) || !make_map(&mk, a.k, a.hk, a.tokens) ||
-        !make_map(&mv, a.v, a.hv, a.tokens))
+        !make_map(&mv, a.v, a.hv, a.tokens) || !make_map(&mo, a.o, a.hv, a.tokens, true) ||
+        !make_gate_map(&mg, a.g, a.hv, a.tokens) || !make_gate_map(&mb, a.beta, a.hv, a.tokens))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
     if (e != cudaSuccess) return e;
     const int64_t units = int64_t(a.num_seqs) * a.hv;
     const int grid = int(units < num_sms ? units : num_sms);
     if (grid <= 0) return cudaSuccess;
-    chunk_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, a);
+    chunk_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mo, mg, mb, a);
     count_launch();
     return cudaGetLastError();
 }

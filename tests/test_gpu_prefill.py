@@ -39,7 +39,7 @@ def test_fp32_d128_ragged(C):
 
 
 @pytest.mark.parametrize("force_simt", PATHS)
-@pytest.mark.parametrize("hk,hv", [(2, 4), (1, 3), (2, 2)])
+@pytest.mark.parametrize("hk,hv", [(2, 4), (4, 12), (4, 4), (1, 3)])
 def test_bf16_d128_c64_batched(force_simt, hk, hv):
     w = I.custom(f"bf16_b2_T300_{hk}x{hv}", batch=2, seq_len=300, hk=hk, hv=hv, d=128, chunk=64, dtype="bf16",
                  seed=22 + hv, s0_std=0.02)
@@ -59,7 +59,7 @@ def test_bf16_varlen_edges(force_simt):
 def test_bf16_mild_decay_long(force_simt):
     """The milder decay of the 4 x 4096 workload (g = -0.1 softplus(N(0,1)+2)),
     where errors have the most room to grow, over 1024 tokens."""
-    w = I.custom("bf16_mild", batch=1, seq_len=1024, hk=1, hv=2, d=128, chunk=64, dtype="bf16", seed=24,
+    w = I.custom("bf16_mild", batch=1, seq_len=1024, hk=2, hv=4, d=128, chunk=64, dtype="bf16", seed=24,
                  g_shift=2.0, g_scale=0.1)
     _check(w, force_simt)
 
@@ -92,7 +92,7 @@ def test_degenerate_gates(force_simt):
     """beta = 0 on some tokens (pure decay), g far below the kernel floor and
     g = 0 (no decay) on others: the oracle uses them exactly (g = -inf gives
     alpha = 0); the kernels read max(g, -20), a relative change below 1e-8."""
-    w = I.custom("bf16_degenerate", batch=1, seq_len=260, hk=1, hv=2, d=128, chunk=64, dtype="bf16", seed=26,
+    w = I.custom("bf16_degenerate", batch=1, seq_len=260, hk=1, hv=4, d=128, chunk=64, dtype="bf16", seed=26,
                  s0_std=0.05)
     inp = I.make_prefill_inputs(w)
     inp["beta"][0, 10:40] = 0.0
@@ -110,7 +110,7 @@ def test_degenerate_gates(force_simt):
 def test_in_place_state_and_no_final(force_simt):
     """final_state may alias initial_state; output_final_state=False works."""
     from linear_attention_sequence_sm_b200 import gdn
-    w = I.custom("bf16_inplace", batch=2, seq_len=130, hk=1, hv=2, d=128, chunk=64, dtype="bf16", seed=27,
+    w = I.custom("bf16_inplace", batch=2, seq_len=130, hk=1, hv=4, d=128, chunk=64, dtype="bf16", seed=27,
                  s0_std=0.02)
     inp = I.make_prefill_inputs(w)
     o_ref, sf_ref = oracle_prefill(inp)
@@ -133,7 +133,7 @@ def test_bad_cu_seqlens_recorded_not_faulted():
     skip their work and the status word reads GDN_ERR_DEVICE_CHECK."""
     from linear_attention_sequence_sm_b200 import gdn
     dev = torch.device("cuda:0")
-    T, hk, hv, d = 100, 1, 2, 128
+    T, hk, hv, d = 100, 1, 4, 128
     q = torch.nn.functional.normalize(torch.randn(1, T, hk, d, device=dev), dim=-1).bfloat16()
     v = torch.randn(1, T, hv, d, device=dev).bfloat16()
     g = -torch.rand(1, T, hv, device=dev)
