@@ -30,14 +30,15 @@
 // Warp specialisation.  Only (4), (7) and the state pass depend on the state
 // carried from the previous chunk; everything else in a chunk does not.  So a
 // CTA runs two warp groups on one (sequence, value head) unit:
-//   chain  (warps 0-7):  state pass, (4)+(5), U epilogue, (6)+(7), output
+//   chain  (warps 0-7):  (2)+(3) under the state pass, W^T epilogue,
+//                        (4)+(5), U epilogue, (6)+(7), output
 //   intra  (warps 8-15): gates and their prefix sums, (1), decay masks A and
-//                        P, the triangular inverse (CUDA cores, fp32), T'
-//                        and T'', (2)+(3), W^T epilogue -- one chunk ahead.
-// They hand chunks over through mbarriers: "full[b]" (intra -> chain: W^T,
-// P, U~ in tensor memory and the per-token vectors of buffer b are ready),
-// "empty[b]" (chain -> intra: buffer b may be refilled), "wt_free" (the
-// single W^T tile has been consumed).  q/k tiles are double-buffered; the
+//                        P, the triangular inverse (fp32 diagonal blocks,
+//                        tf32 block products), T' and T'' -- one chunk ahead.
+// They hand chunks over through mbarriers: "full[b]" (intra -> chain: T',
+// T'', P and the per-token vectors of buffer b are ready), "empty[b]"
+// (chain -> intra: buffer b may be refilled), "t_free" (T' and T'', which
+// share space with the intra group's scratch, have been consumed).  q/k tiles are double-buffered; the
 // chain refills a buffer two chunks ahead as soon as its last reader (7)
 // completes.  Each group synchronises internally with its own named barrier.
 // A full chunk of output leaves through one TMA store of the staged tile.
@@ -90,6 +91,7 @@ static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 per-block lim
 constexpr int kVecG = 0, kVecB = 64, kVecGam = 128, kVecBG = 192, kVecLam = 256, kVecIGam = 320;
 // mbarrier slots
 constexpr int kBarTKQ = 0, kBarTV = 2, kBarI = 3, kBarC = 4, kBarFull = 5, kBarEmpty = 7, kBarWT = 9, kNumBars = 10;
+// (kBarWT: "T' and T'' consumed", chain -> intra)
 
 // Tensor-memory columns (fp32, 128 lanes each).
 constexpr uint32_t kColGram = 0, kColW = 64, kColU0 = 128, kColU1 = 192, kColX1 = 256, kColX2 = 320, kColS = 384;
@@ -344,11 +346,25 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const uint32_t pt = sb + (b ? kOffP1 : kOffP0);
                 const uint32_t colU = b ? kColU1 : kColU0;
                 {
-                    const bool ok = mbar_wait(bars + 8 * (kBarFull + b), (ph_full >> b) & 1u);
+                    const bool ok = mbar_wait(bars + 8 * (kBarFull + b), (ph_full >> b) & 1u) &&
+                                    mbar_wait(bars + 8 * kBarTV, ph_v);
                     ph_full ^= 1u << b;
+                    ph_v ^= 1u;
                     if (named_sync_or(kBarChain, kChain, !ok)) { aborted = true; break; }
                 }
                 tc_fence_after();
+                // (2) W^T = K^T T'^T and (3) U~^T = V^T T''^T, running under the state pass
+                if (tid == 0) {
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        mma_bf16(tmem + kColW, (smem_desc(kq, 16384, 1024) + uint64_t((s * 2048) >> 4)),
+                                 (smem_desc(sb, 16, 1024) + uint64_t((kOffTp + s * 32) >> 4)), id_w, s > 0);
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        mma_bf16(tmem + colU, (smem_desc(sb, 8192, 1024) + uint64_t((kOffV + s * 2048) >> 4)),
+                                 (smem_desc(sb, 16, 1024) + uint64_t((kOffTpp + s * 32) >> 4)), id_w, s > 0);
+                    mma_commit(bars + 8 * kBarC);
+                }
                 // state pass: S_n -> bf16 operand, S <- gamma_C S_n in place
                 {
                     const float gC = vec[kVecGam + 63];  // padded rows carry g = 0, so G_63 = G_{L-1}
@@ -363,6 +379,22 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         tmem_st32(tmem + lane_bits + kColS + 64 * ch + 32 * p2, v0);
                     }
                     tmem_wait_st();
+                }
+                {
+                    const bool ok = mbar_wait(bars + 8 * kBarC, ph_c);
+                    ph_c ^= 1u;
+                    if (named_sync_or(kBarChain, kChain, !ok)) { aborted = true; break; }
+                }
+                tc_fence_after();
+                if (tid == 0) {
+                    mbar_arrive(bars + 8 * kBarWT);  // T' and T'' consumed: the intra group may overwrite them
+                    if (n + 1 < nchunks) load_v(sb + kOffV, bars + 8 * kBarTV, &tm_v, h, c0 + 64);
+                }
+                {
+                    float v[32];
+                    tmem_ld32(tmem + lane_bits + kColW + 32 * ch, v);
+                    tmem_wait_ld();
+                    store_row_bf16(sb + kOffWT, row, 4 * ch, v, 4);
                 }
                 fence_proxy_async_shared();
                 tc_fence_before();
@@ -391,7 +423,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (named_sync_or(kBarChain, kChain, !ok)) { aborted = true; break; }
                 }
                 tc_fence_after();
-                if (tid == 0) mbar_arrive(bars + 8 * kBarWT);  // W^T consumed
                 // U epilogue: U^T rows to bf16 operands (plain and lambda-scaled)
                 {
                     float v[32], l[32];
@@ -553,6 +584,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
                 }
                 tc_fence_after();
+                if (gcn >= 1) {  // the chain has consumed the previous chunk's T' and T'' (over A)
+                    const bool ok = mbar_wait(bars + 8 * kBarWT, ph_wt);
+                    ph_wt ^= 1u;
+                    if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
+                }
                 // A (fp32, for the inverse) and P (bf16 operand) from the Gram, in
                 // slices of 16 columns
                 {
@@ -613,44 +649,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     st_shared_v4(sb + kOffTpp + sw128_offset(r, c8), pack_bf16x8(x2));
                 }
                 fence_proxy_async_shared();
-                {
-                    const bool ok = mbar_wait(bars + 8 * kBarTV, ph_v);
-                    ph_v ^= 1u;
-                    if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
-                }
-                // (2) W^T and (3) U~^T
-                if (it == 0) {
-                    tc_fence_after();
-#pragma unroll
-                    for (int s = 0; s < 4; ++s)
-                        mma_bf16(tmem + kColW, (smem_desc(kq, 16384, 1024) + uint64_t((s * 2048) >> 4)),
-                                 (smem_desc(sb, 16, 1024) + uint64_t((kOffTp + s * 32) >> 4)), id_w, s > 0);
-#pragma unroll
-                    for (int s = 0; s < 4; ++s)
-                        mma_bf16(tmem + colU, (smem_desc(sb, 8192, 1024) + uint64_t((kOffV + s * 2048) >> 4)),
-                                 (smem_desc(sb, 16, 1024) + uint64_t((kOffTpp + s * 32) >> 4)), id_w, s > 0);
-                    mma_commit(bars + 8 * kBarI);
-                }
-                {
-                    const bool ok = mbar_wait(bars + 8 * kBarI, ph_i);
-                    ph_i ^= 1u;
-                    if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
-                }
-                tc_fence_after();
-                if (it == 0 && n + 1 < nchunks) load_v(sb + kOffV, bars + 8 * kBarTV, &tm_v, h, c0 + 64);
-                if (gcn >= 1) {  // the chain has consumed the previous chunk's W^T
-                    const bool ok = mbar_wait(bars + 8 * kBarWT, ph_wt);
-                    ph_wt ^= 1u;
-                    if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
-                }
-                {
-                    float v[32];
-                    tmem_ld32(tmem + lane_bits + kColW + 32 * ih, v);
-                    tmem_wait_ld();
-                    store_row_bf16(sb + kOffWT, irow, 4 * ih, v, 4);
-                }
-                fence_proxy_async_shared();
-                tc_fence_before();
                 named_sync(kBarIntra, kIntra);
                 if (it == 0) mbar_arrive(bars + 8 * (kBarFull + b));  // chunk gcn ready for the chain
                 // start the next chunk's Gram as soon as its q and k are in (the Gram
