@@ -19,8 +19,14 @@
 
 namespace gdn {
 
+#ifndef GDN_DECODE_ROWS
+#define GDN_DECODE_ROWS 8
+#endif
+#ifndef GDN_DECODE_MINBLOCKS
+#define GDN_DECODE_MINBLOCKS 1
+#endif
 constexpr int kDecodeWarps = 4;     // warps per block; a block owns one (sequence, head)
-constexpr int kRowBatch = 8;        // rows in flight per warp
+constexpr int kRowBatch = GDN_DECODE_ROWS;  // rows in flight per warp
 
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
@@ -44,7 +50,7 @@ __device__ __forceinline__ void load_vec4(const __nv_bfloat16 *p, float out[4]) 
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kDecodeWarps * 32)
+__global__ void __launch_bounds__(kDecodeWarps * 32, GDN_DECODE_MINBLOCKS)
 decode_d128_kernel(int32_t hk, int32_t hv, int32_t dv, const T *__restrict__ q, const T *__restrict__ k,
                    const T *__restrict__ v, const float *__restrict__ g, const float *__restrict__ beta,
                    float *__restrict__ state, T *__restrict__ o) {

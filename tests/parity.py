@@ -66,3 +66,29 @@ def prefill_errors(inp, o_gpu, sf_gpu, o_ref, sf_ref, units=None):
                 err = np.linalg.norm(sg[n, h] - ref) / max(np.linalg.norm(ref), 1e-30)
                 worst_s = max(worst_s, err)
     return worst_o, worst_s
+
+
+def oracle_units_sliced(inp, units, hv, hk):
+    """Oracle outputs for the listed (sequence, head) units, each run on its own
+    head's slice of the inputs (keeps host memory bounded at full sizes).
+    Returns {unit: (o [T_n, d_v], final state [d_v, d_k])}."""
+    from oracle import oracle
+    G = hv // hk
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    res = {}
+    for u in units:
+        n, h = divmod(u, hv)
+        hq = h // G
+        if inp["cu_seqlens"] is None:
+            qs, ks = q[n, :, hq:hq + 1], k[n, :, hq:hq + 1]
+            vs, gs, bs = v[n, :, h:h + 1], inp["g"][n, :, h:h + 1], inp["beta"][n, :, h:h + 1]
+        else:
+            cu = inp["cu_seqlens"].tolist()
+            a, b = cu[n], cu[n + 1]
+            qs, ks = q[0, a:b, hq:hq + 1], k[0, a:b, hq:hq + 1]
+            vs, gs, bs = v[0, a:b, h:h + 1], inp["g"][0, a:b, h:h + 1], inp["beta"][0, a:b, h:h + 1]
+        s0 = None if inp["initial_state"] is None else to_f64(inp["initial_state"][n:n + 1, h:h + 1])
+        o, sf = oracle.recurrent(to_f64(qs)[None], to_f64(ks)[None], to_f64(vs)[None], to_f64(gs)[None],
+                                 to_f64(bs)[None], initial_state=s0)
+        res[u] = (o[0, :, 0], sf[0, 0])
+    return res

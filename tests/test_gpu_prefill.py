@@ -9,7 +9,7 @@ import pytest
 import torch
 
 from linear_attention_sequence_sm_b200 import inputs as I
-from parity import BAR, gpu_prefill, oracle_prefill, prefill_errors
+from parity import BAR, gpu_prefill, oracle_prefill, oracle_units_sliced, prefill_errors
 
 pytestmark = pytest.mark.gpu
 
@@ -202,3 +202,22 @@ def test_full_size_varlen_sampled():
     units.add(int(lens.argmax()) * w.hv + 5)
     units.add(int(lens.argmin()) * w.hv + 30)
     _check(w, force_simt=False, units=sorted(units))
+
+
+def test_full_size_long_context_sampled():
+    """The 65,536-token, 16/48-head (3 value heads per q/k head), d=128, C=64
+    bf16 workload with initial states, at full size; the oracle recomputes
+    4 sampled (sequence, head) units on their own head slices."""
+    w = I.long_bf16()
+    inp = I.make_prefill_inputs(w)
+    o, sf = gpu_prefill(inp, w.chunk)
+    units = [0, 17, 30, 47]
+    ref = oracle_units_sliced(inp, units, w.hv, w.hk)
+    og = o.float().cpu()
+    for u, (o_ref, s_ref) in ref.items():
+        h = u % w.hv
+        o_u = og[0, :, h].double().numpy()
+        s_u = sf[0, h].double().cpu().numpy()
+        eo = np.linalg.norm(o_u - o_ref) / np.linalg.norm(o_ref)
+        es = np.linalg.norm(s_u - s_ref) / np.linalg.norm(s_ref)
+        assert eo <= BAR["bf16"] and es <= BAR["bf16"], (u, eo, es)
