@@ -150,6 +150,12 @@ def max_over_ranks(x: float, device, world: int) -> float:
     return float(t.item())
 
 
+def aggregate_value(tokens_per_rank: int, ms_max: float, world: int) -> float:
+    """Whole-job tokens/s: every rank processes its own replica of the workload;
+    the slowest rank's device time bounds the job."""
+    return world * tokens_per_rank / (ms_max / 1e3)
+
+
 def barrier(world: int, device=None):
     if world > 1:
         import torch.distributed as dist
@@ -277,7 +283,7 @@ def run_ours(args):
         barrier(world, device)
         ms_max = max_over_ranks(ms, device, world)
     tokens = w.total_tokens
-    value = world * tokens / (ms_max / 1e3)
+    value = aggregate_value(tokens, ms_max, world)
     flops = USEFUL_FLOPS_PER_VHEAD_TOKEN * tokens * w.hv
     achieved_tflops = flops / (ms / 1e3) / 1e12
     kernel_name = "gdn_chunk_tc" if gdn_tc_active(gdn, dev, w) else "gdn_chunk_simt"

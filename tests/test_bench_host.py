@@ -1,0 +1,87 @@
+"""Host logic of bench.py, on CPU: the replica aggregation across ranks (two
+gloo processes), the reference arm on a non-zero rank, and the algorithmic
+byte/FLOP counts behind the roofline fields."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from conftest import ROOT
+
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, times, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        bench.barrier(world)
+        ms = bench.max_over_ranks(times[rank], torch.device("cpu"), world)
+        out[rank] = (ms, bench.aggregate_value(16384, ms, world))
+        bench.barrier(world)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_replicas_take_the_slowest_rank():
+    world, port = 2, _free_port()
+    times = [0.30, 0.45]
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_rank_main, args=(world, port, times, out), nprocs=world, join=True)
+    for r in range(world):
+        ms, value = out[r]
+        assert ms == pytest.approx(0.45)
+        assert value == pytest.approx(2 * 16384 / 0.45e-3)
+
+
+def test_single_rank_aggregate():
+    assert bench.max_over_ranks(0.3, torch.device("cpu"), 1) == 0.3
+    assert bench.aggregate_value(1000, 2.0, 1) == pytest.approx(5e5)
+
+
+def test_reference_arm_exits_quietly_on_other_ranks():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "0"], env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_roofline_counts():
+    from linear_attention_sequence_sm_b200 import inputs as I
+    # 6 d^2 + 3 C d + 2 C d / G at d = 128, C = 64, G = 2
+    assert bench.USEFUL_FLOPS_PER_VHEAD_TOKEN == 131072
+    w = I.prefill_bf16()
+    # q + k (16 heads) and v + o (32 heads) in bf16, g and beta fp32, the final state fp32
+    assert bench.prefill_bytes(w) == 16384 * (16 * 128 * 2 * 2 + 32 * 128 * 2 * 2 + 32 * 8) + 4 * 32 * 128 * 128 * 4
+    assert bench.decode_bytes(I.decode_bf16()) == 1080098816
+
+
+def test_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1")
+    import hashlib
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    entry = {"k": {"source": "k.cu", "source_sha256": hashlib.sha256(b"kernel v1").hexdigest(),
+                   "bytes_per_launch": 123}}
+    (prof / "traffic.json").write_text(json.dumps(entry))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.kernel_traffic("k") == 123
+    src.write_text("kernel v2")
+    assert bench.kernel_traffic("k") is None
+    assert bench.kernel_traffic("missing") is None
