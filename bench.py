@@ -45,6 +45,9 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--decode-steps", type=int, default=512)
+    p.add_argument("--workload", choices=["prefill", "long", "varlen"], default="prefill",
+                   help="prefill: 4 x 4096 tokens (the headline line); long: 65,536 tokens, 48 v heads, "
+                        "initial states; varlen: 32 packed sequences of 128..8192 tokens")
     p.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                    help="time only one of the two paths (used by profiling commands)")
     p.add_argument("--no-e2e", action="store_true")
@@ -68,8 +71,9 @@ def load_peaks():
 
 
 def kernel_traffic(kernel: str):
-    """DRAM bytes per launch from a committed ncu summary, only if the kernel's
-    source has not changed since the counters were taken."""
+    """DRAM bytes per launch from a committed ncu summary (keyed by
+    "kernel/workload"), only if the kernel's source has not changed since the
+    counters were taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -253,18 +257,19 @@ def run_ours(args):
     from linear_attention_sequence_sm_b200 import inputs as I
 
     peaks, peak_src = load_peaks()
-    w = I.prefill_bf16(seed=1002 + rank)
+    w = {"prefill": I.prefill_bf16, "long": I.long_bf16, "varlen": I.varlen_bf16}[args.workload](
+        seed={"prefill": 1002, "long": 1003, "varlen": 1005}[args.workload] + rank)
     host = I.make_prefill_inputs(w)
     dev = {k: (v.to(device) if v is not None else None) for k, v in host.items()}
     o = torch.empty_like(dev["v"])
     sf = torch.empty((w.num_seqs, w.hv, w.d, w.d), dtype=torch.float32, device=device)
-    shape = gdn.make_shape(dev["q"], dev["v"], None, w.chunk)
+    shape = gdn.make_shape(dev["q"], dev["v"], dev["cu_seqlens"], w.chunk)
     ws = torch.empty(gdn.workspace_size(shape), dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
 
     def step():
-        gdn.chunk_forward(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], initial_state=None, out=o,
-                          final_state=sf, workspace=ws, chunk_size=w.chunk)
+        gdn.chunk_forward(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], initial_state=dev["initial_state"],
+                          cu_seqlens=dev["cu_seqlens"], out=o, final_state=sf, workspace=ws, chunk_size=w.chunk)
 
     ms = ms_max = float("nan")
     launches = 0
@@ -284,12 +289,12 @@ def run_ours(args):
         ms_max = max_over_ranks(ms, device, world)
     tokens = w.total_tokens
     value = aggregate_value(tokens, ms_max, world)
-    flops = USEFUL_FLOPS_PER_VHEAD_TOKEN * tokens * w.hv
+    flops = useful_flops_per_vhead_token(w.hv // w.hk) * tokens * w.hv
     achieved_tflops = flops / (ms / 1e3) / 1e12
     kernel_name = "gdn_chunk_tc" if gdn_tc_active(gdn, dev, w) else "gdn_chunk_simt"
     roofline = {"bound": "tensor", "achieved": achieved_tflops, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved_tflops / peaks["bf16_tflops"],
-                "traffic": kernel_traffic(kernel_name), "kernel": kernel_name,
+                "traffic": kernel_traffic(f"{kernel_name}/{w.name}"), "kernel": kernel_name,
                 "peak_source": f"{peak_src} bf16 dense (burst)",
                 "flops_per_launch": flops, "algorithmic_bytes_per_launch": prefill_bytes(w)}
 
@@ -322,7 +327,7 @@ def run_ours(args):
         decode = {"value": world * dgbs, "unit": "GB/s", "ms_per_step": dms, "steps": args.decode_steps,
                   "tokens_per_s": world * dw.num_seqs / (dms / 1e3), "workload": dw.name,
                   "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                               "frac": dgbs / peaks["hbm_gbs"], "traffic": kernel_traffic("gdn_decode"),
+                               "frac": dgbs / peaks["hbm_gbs"], "traffic": kernel_traffic(f"gdn_decode/{dw.name}"),
                                "kernel": "gdn_decode", "peak_source": f"{peak_src} HBM copy",
                                "bytes_per_launch": dbytes},
                   "clocks": dclocks.summary()}
@@ -339,7 +344,8 @@ def run_ours(args):
 
         def e2e_step():
             x = {k: v.to(device, non_blocking=True) for k, v in pin.items()}
-            oo, ss = gdn.chunk_forward(x["q"], x["k"], x["v"], x["g"], x["beta"], chunk_size=w.chunk, workspace=ws)
+            oo, ss = gdn.chunk_forward(x["q"], x["k"], x["v"], x["g"], x["beta"], initial_state=x.get("initial_state"),
+                                       cu_seqlens=x.get("cu_seqlens"), chunk_size=w.chunk, workspace=ws)
             o_host.copy_(oo, non_blocking=True)
             sf_host.copy_(ss, non_blocking=True)
 
@@ -361,10 +367,10 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded splitmix64 / Box-Muller)",
-            "config": {"workload": w.name, "global_batch": w.batch * world, "seq_len": w.seq_len,
+            "config": {"workload": w.name, "global_batch": w.num_seqs * world, "seq_len": w.seq_len,
                        "heads_qk_v": [w.hk, w.hv], "head_dim": w.d, "chunk": w.chunk,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "inputs larger than L2 (about 410 MB of mandatory traffic per step)"},
+                       "l2": f"inputs larger than L2 ({prefill_bytes(w) / 1e6:.0f} MB of mandatory traffic per step)"},
             "roofline": roofline, "decode": decode, "e2e": e2e, "cpu_baseline": cpu,
             "gpu_launches": launches, "clocks": clocks.summary(),
         }), flush=True)
@@ -383,6 +389,12 @@ def gdn_tc_active(gdn, dev, w) -> bool:
 def tc_built(gdn) -> bool:
     src = open(os.path.join(ROOT, "linear_attention_sequence_sm_b200", "csrc", "gdn_chunk_tc.cu")).read()
     return "tcgen05.mma" in src
+
+
+def useful_flops_per_vhead_token(group: int, d: int = 128, chunk: int = 64) -> int:
+    """6 d^2 (inter-chunk) + 3 C d (triangular intra-chunk, counted at half)
+    + 2 C d / G (the Gram shared by the G value heads of a q/k head)."""
+    return 6 * d * d + 3 * chunk * d + 2 * chunk * d // group
 
 
 def prefill_bytes(w) -> int:
