@@ -62,6 +62,10 @@ namespace {
 constexpr int kThreads = 512;      // warps 0-7: chain group; warps 8-15: intra group
 constexpr int kChain = 256, kIntra = 256;
 constexpr int kBarChain = 1, kBarIntra = 2;  // named barrier ids (0 is __syncthreads)
+// The intra group's Gram MMAs are issued from its last warp, which does none of
+// the gate scan or the first inverse phase: an issue that stalls behind the
+// chain's tensor-core work then delays no other intra work.
+constexpr int kIntraIssuer = 224;
 constexpr int kLdA = 68;  // fp32 row stride of the A and T scratch matrices (16-byte aligned rows)
 constexpr int kLdY = 36;  // fp32 row stride of the inverse's 32 x 32 scratch
 
@@ -73,9 +77,9 @@ constexpr uint32_t kOffV = 65536;     // V: 2 atom columns x 64 rows (intra only
 constexpr uint32_t kOffWT = 81920;    // W^T: 128 rows (d_k) x 64 tokens
 constexpr uint32_t kOffP0 = 98304;    // P = Q K^T (.) Gamma, buffer 0: 64 x 64
 constexpr uint32_t kOffP1 = 106496;   // P, buffer 1
-constexpr uint32_t kOffS = 114688;    // S operand (bf16): 2 atom columns x 128 rows (chain only)
-constexpr uint32_t kOffUT = 147456;   // U^T: 128 rows (d_v) x 64 tokens; then the output staging tile
-constexpr uint32_t kOffUTl = 163840;  // U^T diag(lambda)
+constexpr uint32_t kOffFree = 114688; // 32 KB not used
+constexpr uint32_t kOffOst = 147456;  // output staging: 64 tokens x 128 bf16, token-major (one TMA store)
+constexpr uint32_t kOffFree2 = 163840; // 16 KB not used
 constexpr uint32_t kOffAf = 180224;   // A, fp32 64 x kLdA; after the inverse: T' (8 KB) and T'' (8 KB)
 constexpr uint32_t kOffTp = kOffAf, kOffTpp = kOffAf + 8192;
 constexpr uint32_t kOffTf = kOffAf + 64 * kLdA * 4;  // T, fp32 64 x kLdA
@@ -93,8 +97,12 @@ constexpr int kVecG = 0, kVecB = 64, kVecGam = 128, kVecBG = 192, kVecLam = 256,
 constexpr int kBarTKQ = 0, kBarTV = 2, kBarI = 3, kBarC = 4, kBarFull = 5, kBarEmpty = 7, kBarWT = 9, kNumBars = 10;
 // (kBarWT: "T' and T'' consumed", chain -> intra)
 
-// Tensor-memory columns (fp32, 128 lanes each).
-constexpr uint32_t kColGram = 0, kColW = 64, kColU0 = 128, kColU1 = 192, kColX1 = 256, kColX2 = 320, kColS = 384;
+// Tensor-memory columns (128 lanes each): fp32 accumulators, and bf16 A
+// operands packed two elements per column: the copy of S for (4) and (5), and
+// U^T and U^T diag(lambda) for (6) and (7), which reuse the W^T accumulator's
+// columns once its epilogue has read them.
+constexpr uint32_t kColGram = 0, kColW = 64, kColU = 128, kColSb = 192, kColX1 = 256, kColX2 = 320, kColS = 384;
+constexpr uint32_t kColUb = kColW, kColUlb = kColW + 32;
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t kBytesKQ = 4 * 8192 + 2 * 1024;  // four 64 x 64 bf16 boxes and two 64 x 4 fp32 gate boxes
@@ -264,6 +272,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool is_chain = warp < 8;
+    // One warp per group polls each mbarrier; the rest of the group blocks in the
+    // named barrier that follows every wait, so the spinning costs the shared-
+    // memory pipe one warp's requests instead of eight.
+    const bool chain_poll = warp == 0, intra_poll = warp == 8;
     const uint32_t lane_bits = uint32_t((warp & 3) * 32) << 16;  // this warp's tensor-memory lane quarter
     WsHeader *hdr = a.sched.hdr;
     if (hdr->status != GDN_OK) return;
@@ -344,10 +356,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const float *vec = reinterpret_cast<const float *>(smem + (b ? kOffVec1 : kOffVec0));
                 const uint32_t kq = sb + (b ? kOffKQ1 : kOffKQ0);
                 const uint32_t pt = sb + (b ? kOffP1 : kOffP0);
-                const uint32_t colU = b ? kColU1 : kColU0;
+                const uint32_t colU = kColU;
                 {
-                    const bool ok = mbar_wait(bars + 8 * (kBarFull + b), (ph_full >> b) & 1u) &&
-                                    mbar_wait(bars + 8 * kBarTV, ph_v);
+                    const bool ok = !chain_poll || (mbar_wait(bars + 8 * (kBarFull + b), (ph_full >> b) & 1u) &&
+                                    mbar_wait(bars + 8 * kBarTV, ph_v));
                     ph_full ^= 1u << b;
                     ph_v ^= 1u;
                     if (named_sync_or(kBarChain, kChain, !ok)) { aborted = true; break; }
@@ -373,7 +385,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         float v0[32];
                         tmem_ld32(tmem + lane_bits + kColS + 64 * ch + 32 * p2, v0);
                         tmem_wait_ld();
-                        store_row_bf16(sb + kOffS + ch * 16384, row, 4 * p2, v0, 4);
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(v0[2 * j], v0[2 * j + 1]);
+                        tmem_st16u(tmem + lane_bits + kColSb + 32 * ch + 16 * p2, pk);
 #pragma unroll
                         for (int j = 0; j < 32; ++j) v0[j] *= gC;
                         tmem_st32(tmem + lane_bits + kColS + 64 * ch + 32 * p2, v0);
@@ -381,7 +396,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tmem_wait_st();
                 }
                 {
-                    const bool ok = mbar_wait(bars + 8 * kBarC, ph_c);
+                    const bool ok = !chain_poll || mbar_wait(bars + 8 * kBarC, ph_c);
                     ph_c ^= 1u;
                     if (named_sync_or(kBarChain, kChain, !ok)) { aborted = true; break; }
                 }
@@ -403,39 +418,42 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (tid == 0) {
                     tc_fence_after();
 #pragma unroll
-                    for (int s = 0; s < 8; ++s) {
-                        const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
-                        mma_bf16(tmem + colU, (smem_desc(sb, 16, 1024) + uint64_t((kOffS + off) >> 4)),
-                                 (smem_desc(sb, 16384, 1024) + uint64_t((kOffWT + s * 2048) >> 4)), id_u, 1);
-                    }
+                    for (int s = 0; s < 8; ++s)
+                        mma_bf16_ts(tmem + colU, tmem + kColSb + 8 * s,
+                                    (smem_desc(sb, 16384, 1024) + uint64_t((kOffWT + s * 2048) >> 4)), id_u, 1);
 #pragma unroll
                     for (int s = 0; s < 8; ++s) {
                         const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
-                        mma_bf16(tmem + kColX1, (smem_desc(sb, 16, 1024) + uint64_t((kOffS + off) >> 4)),
+                        mma_bf16_ts(tmem + kColX1, tmem + kColSb + 8 * s,
                                  (smem_desc(kq, 16, 1024) + uint64_t((8192 + off) >> 4)), id_x, s > 0);
                     }
                     mma_commit(bars + 8 * kBarC);
                     bulk_wait_read();  // the previous chunk's output store has read the staging tile
                 }
                 {
-                    const bool ok = mbar_wait(bars + 8 * kBarC, ph_c);
+                    const bool ok = !chain_poll || mbar_wait(bars + 8 * kBarC, ph_c);
                     ph_c ^= 1u;
                     if (named_sync_or(kBarChain, kChain, !ok)) { aborted = true; break; }
                 }
                 tc_fence_after();
-                // U epilogue: U^T rows to bf16 operands (plain and lambda-scaled)
+                // U epilogue: U^T rows to bf16 A operands of (6) and (7), plain and
+                // lambda-scaled, in the W accumulator's columns (consumed above)
                 {
                     float v[32], l[32];
                     tmem_ld32(tmem + lane_bits + colU + 32 * ch, v);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) load4(vec + kVecLam + 32 * ch + 4 * q, l + 4 * q);
                     tmem_wait_ld();
-                    store_row_bf16(sb + kOffUT, row, 4 * ch, v, 4);
+                    uint32_t pu[16], pl[16];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) l[j] *= v[j];
-                    store_row_bf16(sb + kOffUTl, row, 4 * ch, l, 4);
+                    for (int j = 0; j < 16; ++j) {
+                        pu[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+                        pl[j] = pack_bf16x2(l[2 * j] * v[2 * j], l[2 * j + 1] * v[2 * j + 1]);
+                    }
+                    tmem_st16u(tmem + lane_bits + kColUb + 16 * ch, pu);
+                    tmem_st16u(tmem + lane_bits + kColUlb + 16 * ch, pl);
+                    tmem_wait_st();
                 }
-                fence_proxy_async_shared();
                 tc_fence_before();
                 named_sync(kBarChain, kChain);
                 // (6) X2 = U^T P^T and (7) S += U^T diag(lambda) K
@@ -443,16 +461,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tc_fence_after();
 #pragma unroll
                     for (int s = 0; s < 4; ++s)
-                        mma_bf16(tmem + kColX2, (smem_desc(sb, 16, 1024) + uint64_t((kOffUT + s * 32) >> 4)),
-                                 (smem_desc(pt, 16, 1024) + uint64_t((s * 32) >> 4)), id_x, s > 0);
+                        mma_bf16_ts(tmem + kColX2, tmem + kColUb + 8 * s,
+                                    (smem_desc(pt, 16, 1024) + uint64_t((s * 32) >> 4)), id_x, s > 0);
 #pragma unroll
                     for (int s = 0; s < 4; ++s)
-                        mma_bf16(tmem + kColS, (smem_desc(sb, 16, 1024) + uint64_t((kOffUTl + s * 32) >> 4)),
-                                 (smem_desc(kq, 16384, 1024) + uint64_t((s * 2048) >> 4)), id_ds, 1);
+                        mma_bf16_ts(tmem + kColS, tmem + kColUlb + 8 * s,
+                                    (smem_desc(kq, 16384, 1024) + uint64_t((s * 2048) >> 4)), id_ds, 1);
                     mma_commit(bars + 8 * kBarC);
                 }
                 {
-                    const bool ok = mbar_wait(bars + 8 * kBarC, ph_c);
+                    const bool ok = !chain_poll || mbar_wait(bars + 8 * kBarC, ph_c);
                     ph_c ^= 1u;
                     if (named_sync_or(kBarChain, kChain, !ok)) { aborted = true; break; }
                 }
@@ -461,11 +479,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (tid == 0 && n + 2 < nchunks)
                     load_kq(kq, bars + 8 * (kBarTKQ + b), &tm_k, &tm_q, hq, c0 + 128, sb + kOffGst + b * 2048, &tm_g,
                             &tm_b, h);
-                // output O[r][i] = gamma_r X1[i][r] + X2[i][r], staged through the
-                // U^T tile (token-major rows of 256 bytes); a full chunk leaves in
+                // output O[r][i] = gamma_r X1[i][r] + X2[i][r], staged token-major
+                // (rows of 256 bytes); a full chunk leaves in
                 // one TMA store, a ragged last chunk row by row
                 {
-                    __nv_bfloat16 *Ot = reinterpret_cast<__nv_bfloat16 *>(smem + kOffUT);
+                    __nv_bfloat16 *Ot = reinterpret_cast<__nv_bfloat16 *>(smem + kOffOst);
 #pragma unroll
                     for (int sl = 0; sl < 2; ++sl) {
                         const int r0 = 32 * ch + 16 * sl;
@@ -485,14 +503,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 named_sync(kBarChain, kChain);
                 if (L == 64) {
                     if (tid == 0) {
-                        tma_store_3d(&tm_o, sb + kOffUT, 0, h, c0);
+                        tma_store_3d(&tm_o, sb + kOffOst, 0, h, c0);
                         bulk_commit();
                     }
                 } else {
                     for (int e = tid; e < 64 * 16; e += kChain) {
                         const int r = e >> 4, c = e & 15;
                         if (r < L) {
-                            const uint4 val = *reinterpret_cast<const uint4 *>(smem + kOffUT + r * 256 + c * 16);
+                            const uint4 val = *reinterpret_cast<const uint4 *>(smem + kOffOst + r * 256 + c * 16);
                             *reinterpret_cast<uint4 *>(o + (size_t(c0 + r) * hv + h) * 128 + c * 8) = val;
                         }
                     }
@@ -527,19 +545,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 float *gs = vec + kVecG, *bs = vec + kVecB;
                 const uint32_t kq = sb + (b ? kOffKQ1 : kOffKQ0);
                 const uint32_t pt = sb + (b ? kOffP1 : kOffP0);
-                const uint32_t colU = b ? kColU1 : kColU0;
                 if (gcn >= 2) {  // buffers b were last used by chunk gcn - 2
-                    const bool ok = mbar_wait(bars + 8 * (kBarEmpty + b), (ph_empty >> b) & 1u);
+                    const bool ok = !intra_poll || mbar_wait(bars + 8 * (kBarEmpty + b), (ph_empty >> b) & 1u);
                     ph_empty ^= 1u << b;
                     if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
                 }
                 if (n == 0) {  // later chunks had q, k and their Gram started by the previous chunk
-                    const bool ok = mbar_wait(bars + 8 * (kBarTKQ + b), (ph_tkq >> b) & 1u);
+                    const bool ok = !intra_poll || mbar_wait(bars + 8 * (kBarTKQ + b), (ph_tkq >> b) & 1u);
                     ph_tkq ^= 1u << b;
                     if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
                 }
                 // (1) Gram
-                if (it == 0 && n == 0) {
+                if (it == kIntraIssuer && n == 0) {
                     tc_fence_after();
 #pragma unroll
                     for (int s = 0; s < 8; ++s) {
@@ -579,13 +596,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     vec[kVecIGam + it] = __expf(-G);
                 }
                 {
-                    const bool ok = mbar_wait(bars + 8 * kBarI, ph_i);
+                    const bool ok = !intra_poll || mbar_wait(bars + 8 * kBarI, ph_i);
                     ph_i ^= 1u;
                     if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
                 }
                 tc_fence_after();
                 if (gcn >= 1) {  // the chain has consumed the previous chunk's T' and T'' (over A)
-                    const bool ok = mbar_wait(bars + 8 * kBarWT, ph_wt);
+                    const bool ok = !intra_poll || mbar_wait(bars + 8 * kBarWT, ph_wt);
                     ph_wt ^= 1u;
                     if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
                 }
@@ -655,10 +672,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 // accumulator was consumed by this chunk's decay-mask epilogue)
                 if (n + 1 < nchunks) {
                     const uint32_t nb = b ^ 1u, nkq = sb + (nb ? kOffKQ1 : kOffKQ0);
-                    const bool ok = mbar_wait(bars + 8 * (kBarTKQ + nb), (ph_tkq >> nb) & 1u);
+                    const bool ok = !intra_poll || mbar_wait(bars + 8 * (kBarTKQ + nb), (ph_tkq >> nb) & 1u);
                     ph_tkq ^= 1u << nb;
                     if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
-                    if (it == 0) {
+                    if (it == kIntraIssuer) {
                         tc_fence_after();
                         const uint64_t dk = smem_desc(nkq, 16, 1024);
 #pragma unroll
@@ -677,7 +694,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (tid == 0) bulk_wait_all();  // output stores complete before the CTA's shared memory goes away
     if (aborted) {
         // let this thread's own tensor-core work drain (bounded) before freeing tensor memory
-        if (tid == 0 || tid == kChain) {
+        if (tid == 0 || tid == kChain + kIntraIssuer) {
             const uint32_t bar = bars + 8 * (tid == 0 ? kBarC : kBarI);
             mma_commit(bar);
             (void)mbar_wait(bar, tid == 0 ? ph_c : ph_i);
