@@ -17,31 +17,37 @@
 //   (1) [K;Q] K^T      -> Gram (lanes 0-63: K K^T, 64-127: Q K^T)   128x64x128
 //   (2) W^T = K^T T'^T  (T' = T diag(beta gamma))                   128x64x64
 //   (3) U~^T = V^T T''^T (T'' = T diag(beta))                       128x64x64
-//   (4) U^T = U~^T - S W^T   (accumulates into (3), A negated)      128x64x128
-//   (5) X1 = S Q^T                                                   128x64x128
+//   (4)+(5) [X1' | U^T] = [0 | U~^T] - S [Q; W]^T                   128x128x128
+//       (one product with A negated: X1' = -S Q^T, U^T = U~^T - S W^T)
 //   (6) X2 = U^T P^T,  P = Q K^T (.) Gamma                           128x64x64
 //   (7) S += (U^T diag(lambda)) K,  lambda_j = e^(G_C - G_j)         128x128x64
-// O[r][i] = gamma_r X1[i][r] + X2[i][r].  Operands are bf16 in
-// 128-byte-swizzled shared memory; q, k, v tiles arrive by TMA (no
-// multicast).  The fp32 state S lives in tensor memory as the accumulator of
-// (7); once per chunk it is read, staged as the bf16 operand of (4) and (5),
-// and rescaled by gamma_C in place.
+// O[r][i] = X2[i][r] - gamma_r X1'[i][r].  A tcgen05.mma of M = 128 costs
+// about the same whether N is 64 or 128, so (4) and (5), which share the
+// operand S, run as one instruction stream of N = 128.  B operands are bf16 in
+// 128-byte-swizzled shared memory (q, k, v tiles by TMA, no multicast; W is
+// written token-major next to Q); the A operands S, U^T and U^T diag(lambda)
+// are bf16 copies in tensor memory.  The fp32 state S lives in tensor memory
+// as the accumulator of (7); once per chunk it is read, copied to bf16 for
+// (4)+(5), and rescaled by gamma_C in place.
 //
 // Warp specialisation.  Only (4), (7) and the state pass depend on the state
 // carried from the previous chunk; everything else in a chunk does not.  So a
 // CTA runs two warp groups on one (sequence, value head) unit:
-//   chain  (warps 0-7):  (2)+(3) under the state pass, W^T epilogue,
-//                        (4)+(5), U epilogue, (6)+(7), output
+//   chain  (warps 0-7):  (2)+(3) under the state pass, W epilogue, (4)+(5),
+//                        U epilogue, (6)+(7), output
 //   intra  (warps 8-15): gates and their prefix sums, (1), decay masks A and
 //                        P, the triangular inverse (fp32 diagonal blocks,
-//                        tf32 block products), T' and T'' -- one chunk ahead.
+//                        tf32 block products) writing T' and T'' as its
+//                        blocks become final -- one chunk ahead.
 // They hand chunks over through mbarriers: "full[b]" (intra -> chain: T',
 // T'', P and the per-token vectors of buffer b are ready), "empty[b]"
-// (chain -> intra: buffer b may be refilled), "t_free" (T' and T'', which
-// share space with the intra group's scratch, have been consumed).  q/k tiles are double-buffered; the
-// chain refills a buffer two chunks ahead as soon as its last reader (7)
-// completes.  Each group synchronises internally with its own named barrier.
-// A full chunk of output leaves through one TMA store of the staged tile.
+// (chain -> intra: buffer b may be refilled), "t_free" (T' and T'' have been
+// consumed by (2) and (3); the intra group waits for it just before its
+// inverse).  q/k tiles are double-buffered; the chain refills a buffer two
+// chunks ahead as soon as its last reader (7) completes.  Each group
+// synchronises internally with its own named barrier, and one warp of each
+// group polls the mbarriers.  A full chunk of output leaves through one TMA
+// store of the staged tile.
 //
 // One CTA per SM (shared memory and the 512 tensor-memory columns force it)
 // takes units longest sequence first from an atomic counter.  Every wait is
@@ -71,25 +77,25 @@ constexpr int kLdY = 36;  // fp32 row stride of the inverse's 32 x 32 scratch
 
 // Shared-memory map (bytes from a 1024-byte-aligned base).  Tiles are
 // 128-byte-swizzled: "atom columns" of 64 bf16 (128 bytes) per row.
-constexpr uint32_t kOffKQ0 = 0;       // [K;Q] buffer 0: 2 atom columns x 128 rows (K 0-63, Q 64-127)
-constexpr uint32_t kOffKQ1 = 32768;   // [K;Q] buffer 1
-constexpr uint32_t kOffV = 65536;     // V: 2 atom columns x 64 rows (intra only)
-constexpr uint32_t kOffWT = 81920;    // W^T: 128 rows (d_k) x 64 tokens
-constexpr uint32_t kOffP0 = 98304;    // P = Q K^T (.) Gamma, buffer 0: 64 x 64
-constexpr uint32_t kOffP1 = 106496;   // P, buffer 1
-constexpr uint32_t kOffFree = 114688; // 32 KB not used
-constexpr uint32_t kOffOst = 147456;  // output staging: 64 tokens x 128 bf16, token-major (one TMA store)
-constexpr uint32_t kOffFree2 = 163840; // 16 KB not used
-constexpr uint32_t kOffAf = 180224;   // A, fp32 64 x kLdA; after the inverse: T' (8 KB) and T'' (8 KB)
-constexpr uint32_t kOffTp = kOffAf, kOffTpp = kOffAf + 8192;
+// A chunk buffer holds, per atom column, 64 rows each of K, Q and W (token-major):
+// [K;Q] is the Gram's A operand and [Q;W] the B operand of the merged (4)+(5).
+constexpr uint32_t kAtomKQ = 24576;   // one atom column of a chunk buffer: K, Q, W rows
+constexpr uint32_t kOffKQ0 = 0;       // chunk buffer 0: 2 atom columns
+constexpr uint32_t kOffKQ1 = 49152;   // chunk buffer 1
+constexpr uint32_t kOffV = 98304;     // V: 2 atom columns x 64 rows
+constexpr uint32_t kOffP0 = 114688;   // P = Q K^T (.) Gamma, buffer 0: 64 x 64
+constexpr uint32_t kOffP1 = 122880;   // P, buffer 1
+constexpr uint32_t kOffOst = 131072;  // output staging: 64 tokens x 128 bf16, token-major (one TMA store)
+constexpr uint32_t kOffAf = 147456;   // A, fp32 64 x kLdA (intra group)
 constexpr uint32_t kOffTf = kOffAf + 64 * kLdA * 4;  // T, fp32 64 x kLdA
 constexpr uint32_t kOffY = kOffTf + 64 * kLdA * 4;   // inverse scratch, 32 x kLdY fp32
 constexpr uint32_t kOffVec0 = kOffY + 32 * kLdY * 4;  // per-token vectors of buffer 0 (6 x 64 fp32)
 constexpr uint32_t kOffVec1 = kOffVec0 + 6 * 64 * 4;  // buffer 1
 constexpr uint32_t kOffGst = kOffVec1 + 6 * 64 * 4;   // gates by TMA, per [K;Q] buffer: g, beta as 64 tokens x 4 heads
-constexpr uint32_t kOffBar = kOffGst + 2 * 2048;      // mbarriers, tensor-memory slot, unit slot
+constexpr uint32_t kOffTp = (kOffGst + 2 * 2048 + 1023) / 1024 * 1024;  // T' = T diag(beta gamma), bf16 64 x 64
+constexpr uint32_t kOffTpp = kOffTp + 8192;                               // T'' = T diag(beta)
+constexpr uint32_t kOffBar = kOffTpp + 8192;          // mbarriers, tensor-memory slot, unit slot
 constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024; // + alignment slack
-static_assert(kOffTpp + 8192 <= kOffTf, "T' and T'' must fit in the A scratch");
 static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 per-block limit");
 // per-token vectors inside a buffer (floats)
 constexpr int kVecG = 0, kVecB = 64, kVecGam = 128, kVecBG = 192, kVecLam = 256, kVecIGam = 320;
@@ -101,7 +107,7 @@ constexpr int kBarTKQ = 0, kBarTV = 2, kBarI = 3, kBarC = 4, kBarFull = 5, kBarE
 // operands packed two elements per column: the copy of S for (4) and (5), and
 // U^T and U^T diag(lambda) for (6) and (7), which reuse the W^T accumulator's
 // columns once its epilogue has read them.
-constexpr uint32_t kColGram = 0, kColW = 64, kColU = 128, kColSb = 192, kColX1 = 256, kColX2 = 320, kColS = 384;
+constexpr uint32_t kColGram = 0, kColW = 64, kColX1 = 128, kColU = 192, kColSb = 256, kColX2 = 320, kColS = 384;
 constexpr uint32_t kColUb = kColW, kColUlb = kColW + 32;
 constexpr uint32_t kTmemCols = 512;
 
@@ -164,6 +170,15 @@ __device__ __forceinline__ void tile_store(float *D, int ldd, int m0, int n0, co
     *reinterpret_cast<float2 *>(D + (m0 + g + 8) * ldd + n0 + 2 * t) = make_float2(sgn * c[2], sgn * c[3]);
 }
 
+// T' = T diag(beta gamma) and T'' = T diag(beta) entries (R, C), (R, C + 1) as
+// bf16 pairs in the 128-byte-swizzled 64 x 64 operand tiles at tp and tpp.
+__device__ __forceinline__ void st_tt_pair(uint32_t tp, uint32_t tpp, int R, int C, float v0, float v1,
+                                           const float *bg, const float *bb) {
+    const uint32_t off = uint32_t(R) * 128 + ((uint32_t((C >> 3) ^ (R & 7))) << 4) + uint32_t(C & 7) * 2;
+    st_shared_u32(tp + off, pack_bf16x2(v0 * bg[C], v1 * bg[C + 1]));
+    st_shared_u32(tpp + off, pack_bf16x2(v0 * bb[C], v1 * bb[C + 1]));
+}
+
 // T = (I + A)^-1 for the 64 x 64 unit-lower-triangular system, fp32, in
 // shared memory, by divide and conquer on the block structure
 //   [[X, 0], [C, Z]]^-1 = [[X^-1, 0], [-Z^-1 C X^-1, Z^-1]]:
@@ -174,7 +189,16 @@ __device__ __forceinline__ void tile_store(float *D, int ldd, int m0, int n0, co
 // the 10-bit tf32 mantissa is ample).
 // Everything of Tf above the diagonal must be zero on entry (it is zeroed once
 // and never written).  Called by the 256 threads of the intra group (t = 0..255).
-__device__ void invert_unit_lower(const float *Af, float *Tf, float *Y, int t) {
+//
+// The bf16 operands T' and T'' (column scales bg = beta gamma, bb = beta) are
+// written as each block of T becomes final:
+// the diagonal 16 x 16 blocks from the forward substitution, the 16 x 16 and
+// 32 x 32 lower blocks from the tf32 products; the idle threads of the first
+// phase zero the blocks above the diagonal.  The fp32 copy of the last block
+// is not needed and not written.  Ends with every thread's operand writes
+// fenced for the tensor cores and a group barrier.
+__device__ void invert_to_operands(const float *Af, float *Tf, float *Y, int t, uint32_t tp, uint32_t tpp,
+                                   const float *bg, const float *bb) {
     if (t < 64) {
         const int b = t >> 4, c = t & 15;
         const float *Ab = Af + (16 * b) * kLdA + 16 * b;
@@ -193,13 +217,30 @@ __device__ void invert_unit_lower(const float *Af, float *Tf, float *Y, int t) {
             x[r] = acc0 + acc1;
         }
         float *Tb = Tf + (16 * b) * kLdA + 16 * b;
+        const int C = 16 * b + c;
+        const float sg = bg[C], sb = bb[C];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) Tb[r * kLdA + c] = x[r];
+        for (int r = 0; r < 16; ++r) {
+            Tb[r * kLdA + c] = x[r];
+            const int R = 16 * b + r;
+            const uint32_t off = uint32_t(R) * 128 + ((uint32_t((C >> 3) ^ (R & 7))) << 4) + uint32_t(C & 7) * 2;
+            st_shared_b16(tp + off, x[r] * sg);
+            st_shared_b16(tpp + off, x[r] * sb);
+        }
+    } else {
+        // zero the six 16 x 16 blocks above the diagonal of both tiles:
+        // 2 tiles x 6 blocks x 16 rows x 2 sixteen-byte chunks = 384 stores
+        for (int e = t - 64; e < 384; e += 192) {
+            const int tile = e / 192, w = e % 192, blk = w >> 5, rr = (w >> 1) & 15, half = w & 1;
+            const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+            const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+            const int R = 16 * bi + rr, ck = 2 * bj + half;
+            st_shared_v4((tile ? tpp : tp) + uint32_t(R) * 128 + (uint32_t(ck ^ (R & 7)) << 4), make_uint4(0, 0, 0, 0));
+        }
     }
     named_sync(kBarIntra, kIntra);
     const int w = t >> 5, lane = t & 31;
-    // 32 x 32 halves p = 0, 1 (warps 0-3, one 16 x 8 tile each):
-    //   Y_p = A[32p+16.., 32p..] B_{2p};  T[32p+16.., 32p..] = -B_{2p+1} Y_p
+    const int g = lane >> 2, tq = lane & 3;
     if (w < 4) {
         const int p = w >> 1, n0 = 8 * (w & 1);
         float c[4] = {0.f, 0.f, 0.f, 0.f};
@@ -212,10 +253,11 @@ __device__ void invert_unit_lower(const float *Af, float *Tf, float *Y, int t) {
         float c[4] = {0.f, 0.f, 0.f, 0.f};
         tile_mma(c, Tf + (32 * p + 16) * kLdA + 32 * p + 16, kLdA, Y + (16 * p) * kLdY, kLdY, n0, 2, lane);
         tile_store(Tf + (32 * p + 16) * kLdA + 32 * p, kLdA, 0, n0, c, -1.f, lane);
+        const int R = 32 * p + 16 + g, C = 32 * p + n0 + 2 * tq;
+        st_tt_pair(tp, tpp, R, C, -c[0], -c[1], bg, bb);
+        st_tt_pair(tp, tpp, R + 8, C, -c[2], -c[3], bg, bb);
     }
     named_sync(kBarIntra, kIntra);
-    // 64 x 64 (8 warps, one 16 x 8 tile of the 32 x 32 block each):
-    //   Y = A[32.., 0..32] T_a;  T[32.., 0..32] = -T_b Y
     {
         const int m0 = 16 * (w >> 2), n0 = 8 * (w & 3);
         float c[4] = {0.f, 0.f, 0.f, 0.f};
@@ -227,8 +269,11 @@ __device__ void invert_unit_lower(const float *Af, float *Tf, float *Y, int t) {
         const int m0 = 16 * (w >> 2), n0 = 8 * (w & 3);
         float c[4] = {0.f, 0.f, 0.f, 0.f};
         tile_mma(c, Tf + (32 + m0) * kLdA + 32, kLdA, Y, kLdY, n0, 4, lane);
-        tile_store(Tf + 32 * kLdA, kLdA, m0, n0, c, -1.f, lane);
+        const int R = 32 + m0 + g, C = n0 + 2 * tq;
+        st_tt_pair(tp, tpp, R, C, -c[0], -c[1], bg, bb);
+        st_tt_pair(tp, tpp, R + 8, C, -c[2], -c[3], bg, bb);
     }
+    fence_proxy_async_shared();
     named_sync(kBarIntra, kIntra);
 }
 
@@ -242,8 +287,8 @@ __device__ __forceinline__ void load_kq(uint32_t dst, uint32_t bar, const CUtens
     tma_load_2d(gst + 1024, tb, h & ~3, c0, bar);
     tma_load_3d(dst, tk, 0, hq, c0, bar);
     tma_load_3d(dst + 8192, tq, 0, hq, c0, bar);
-    tma_load_3d(dst + 16384, tk, 64, hq, c0, bar);
-    tma_load_3d(dst + 24576, tq, 64, hq, c0, bar);
+    tma_load_3d(dst + kAtomKQ, tk, 64, hq, c0, bar);
+    tma_load_3d(dst + kAtomKQ + 8192, tq, 64, hq, c0, bar);
 }
 
 __device__ __forceinline__ void load_v(uint32_t dst, uint32_t bar, const CUtensorMap *tv, int h, int c0) {
@@ -307,7 +352,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     const uint32_t id_gram = idesc_bf16(128, 64, false, false);
     const uint32_t id_w = idesc_bf16(128, 64, true, false);
-    const uint32_t id_u = idesc_bf16(128, 64, false, true, true);
+    const uint32_t id_qw = idesc_bf16(128, 128, false, false, true);  // [X1' | U^T] -= S [Q; W]^T
     const uint32_t id_x = idesc_bf16(128, 64, false, false);
     const uint32_t id_ds = idesc_bf16(128, 128, false, true);  // state update, accumulates into S
 
@@ -349,6 +394,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 tmem_st32(tmem + lane_bits + kColS + 32 * c4, v);
             }
+            {  // X1' accumulates onto zero
+                uint32_t z[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) z[j] = 0u;
+                tmem_st16u(tmem + lane_bits + kColX1 + 32 * ch, z);
+                tmem_st16u(tmem + lane_bits + kColX1 + 32 * ch + 16, z);
+            }
             tmem_wait_st();
             for (int n = 0; n < nchunks; ++n) {
                 const uint32_t gcn = gn + n, b = gcn & 1;
@@ -369,7 +421,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (tid == 0) {
 #pragma unroll
                     for (int s = 0; s < 4; ++s)
-                        mma_bf16(tmem + kColW, (smem_desc(kq, 16384, 1024) + uint64_t((s * 2048) >> 4)),
+                        mma_bf16(tmem + kColW, (smem_desc(kq, kAtomKQ, 1024) + uint64_t((s * 2048) >> 4)),
                                  (smem_desc(sb, 16, 1024) + uint64_t((kOffTp + s * 32) >> 4)), id_w, s > 0);
 #pragma unroll
                     for (int s = 0; s < 4; ++s)
@@ -409,23 +461,29 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     float v[32];
                     tmem_ld32(tmem + lane_bits + kColW + 32 * ch, v);
                     tmem_wait_ld();
-                    store_row_bf16(sb + kOffWT, row, 4 * ch, v, 4);
+                    // W[r][i] (token-major, d_k contiguous) for this thread's d_k index
+                    // i = row and tokens r = 32 ch + j, in the W rows of atom column i / 64
+                    const uint32_t wb = kq + (row >> 6) * kAtomKQ + 16384 + (row & 7) * 2;
+                    const uint32_t c8 = (row & 63) >> 3;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int r = 32 * ch + j;
+                        st_shared_b16(wb + r * 128 + ((c8 ^ uint32_t(r & 7)) << 4), v[j]);
+                    }
                 }
                 fence_proxy_async_shared();
                 tc_fence_before();
                 named_sync(kBarChain, kChain);
-                // (4) U^T = U~^T - S W^T and (5) X1 = S Q^T
+                // (4) and (5) as one product of N = 128 with A negated:
+                // [X1' | U^T] = [0 | U~^T] - S [Q; W]^T, so X1' = -S Q^T (its columns
+                // were zeroed after the previous output) and U^T = U~^T - S W^T
                 if (tid == 0) {
                     tc_fence_after();
 #pragma unroll
-                    for (int s = 0; s < 8; ++s)
-                        mma_bf16_ts(tmem + colU, tmem + kColSb + 8 * s,
-                                    (smem_desc(sb, 16384, 1024) + uint64_t((kOffWT + s * 2048) >> 4)), id_u, 1);
-#pragma unroll
                     for (int s = 0; s < 8; ++s) {
-                        const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+                        const uint32_t off = (s >> 2) * kAtomKQ + (s & 3) * 32;
                         mma_bf16_ts(tmem + kColX1, tmem + kColSb + 8 * s,
-                                 (smem_desc(kq, 16, 1024) + uint64_t((8192 + off) >> 4)), id_x, s > 0);
+                                    (smem_desc(kq + 8192, 16, 1024) + uint64_t(off >> 4)), id_qw, 1);
                     }
                     mma_commit(bars + 8 * kBarC);
                     bulk_wait_read();  // the previous chunk's output store has read the staging tile
@@ -466,7 +524,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                     for (int s = 0; s < 4; ++s)
                         mma_bf16_ts(tmem + kColS, tmem + kColUlb + 8 * s,
-                                    (smem_desc(kq, 16384, 1024) + uint64_t((s * 2048) >> 4)), id_ds, 1);
+                                    (smem_desc(kq, kAtomKQ, 1024) + uint64_t((s * 2048) >> 4)), id_ds, 1);
                     mma_commit(bars + 8 * kBarC);
                 }
                 {
@@ -479,11 +537,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (tid == 0 && n + 2 < nchunks)
                     load_kq(kq, bars + 8 * (kBarTKQ + b), &tm_k, &tm_q, hq, c0 + 128, sb + kOffGst + b * 2048, &tm_g,
                             &tm_b, h);
-                // output O[r][i] = gamma_r X1[i][r] + X2[i][r], staged token-major
-                // (rows of 256 bytes); a full chunk leaves in
-                // one TMA store, a ragged last chunk row by row
+                // output O[r][i] = gamma_r X1[i][r] + X2[i][r] = X2[i][r] - gamma_r X1'[i][r],
+                // staged token-major (rows of 256 bytes); a full chunk leaves in one
+                // TMA store, a ragged last chunk row by row.  X1' is zeroed for the
+                // next chunk's merged product.
                 {
                     __nv_bfloat16 *Ot = reinterpret_cast<__nv_bfloat16 *>(smem + kOffOst);
+                    uint32_t z[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) z[j] = 0u;
 #pragma unroll
                     for (int sl = 0; sl < 2; ++sl) {
                         const int r0 = 32 * ch + 16 * sl;
@@ -493,10 +555,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                         for (int q = 0; q < 4; ++q) load4(vec + kVecGam + r0 + 4 * q, gm + 4 * q);
                         tmem_wait_ld();
+                        tmem_st16u(tmem + lane_bits + kColX1 + r0, z);
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
-                            Ot[(r0 + j) * 128 + row] = __float2bfloat16_rn(fmaf(gm[j], x1[j], x2[j]));
+                            Ot[(r0 + j) * 128 + row] = __float2bfloat16_rn(fmaf(-gm[j], x1[j], x2[j]));
                     }
+                    tmem_wait_st();
                 }
                 fence_proxy_async_shared();
                 tc_fence_before();
@@ -560,7 +624,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tc_fence_after();
 #pragma unroll
                     for (int s = 0; s < 8; ++s) {
-                        const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+                        const uint32_t off = (s >> 2) * kAtomKQ + (s & 3) * 32;
                         mma_bf16(tmem + kColGram, (smem_desc(kq, 16, 1024) + uint64_t((off) >> 4)), (smem_desc(kq, 16, 1024) + uint64_t((off) >> 4)),
                                  id_gram, s > 0);
                     }
@@ -601,11 +665,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
                 }
                 tc_fence_after();
-                if (gcn >= 1) {  // the chain has consumed the previous chunk's T' and T'' (over A)
-                    const bool ok = !intra_poll || mbar_wait(bars + 8 * kBarWT, ph_wt);
-                    ph_wt ^= 1u;
-                    if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
-                }
                 // A (fp32, for the inverse) and P (bf16 operand) from the Gram, in
                 // slices of 16 columns
                 {
@@ -646,27 +705,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 fence_proxy_async_shared();
                 tc_fence_before();
                 named_sync(kBarIntra, kIntra);
-                invert_unit_lower(Af, Tf, Yb, it);
-                // T' = T diag(beta gamma) and T'' = T diag(beta) as bf16 operands (over A)
-                for (int e = it; e < 64 * 8; e += kIntra) {
-                    const int r = e >> 3, c8 = e & 7;
-                    float tv[8], b1[8], b2[8], x1[8], x2[8];
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        load4(Tf + r * kLdA + 8 * c8 + 4 * q, tv + 4 * q);  // zero above the diagonal
-                        load4(vec + kVecBG + 8 * c8 + 4 * q, b1 + 4 * q);
-                        load4(bs + 8 * c8 + 4 * q, b2 + 4 * q);
-                    }
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        x1[u] = tv[u] * b1[u];
-                        x2[u] = tv[u] * b2[u];
-                    }
-                    st_shared_v4(sb + kOffTp + sw128_offset(r, c8), pack_bf16x8(x1));
-                    st_shared_v4(sb + kOffTpp + sw128_offset(r, c8), pack_bf16x8(x2));
+                if (gcn >= 1) {  // the chain has consumed the previous chunk's T' and T''
+                    const bool ok = !intra_poll || mbar_wait(bars + 8 * kBarWT, ph_wt);
+                    ph_wt ^= 1u;
+                    if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
                 }
-                fence_proxy_async_shared();
-                named_sync(kBarIntra, kIntra);
+                invert_to_operands(Af, Tf, Yb, it, sb + kOffTp, sb + kOffTpp, vec + kVecBG, bs);
                 if (it == 0) mbar_arrive(bars + 8 * (kBarFull + b));  // chunk gcn ready for the chain
                 // start the next chunk's Gram as soon as its q and k are in (the Gram
                 // accumulator was consumed by this chunk's decay-mask epilogue)
@@ -680,7 +724,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         const uint64_t dk = smem_desc(nkq, 16, 1024);
 #pragma unroll
                         for (int s = 0; s < 8; ++s) {
-                            const uint64_t d = dk + uint64_t(((s >> 2) * 16384 + (s & 3) * 32) >> 4);
+                            const uint64_t d = dk + uint64_t(((s >> 2) * kAtomKQ + (s & 3) * 32) >> 4);
                             mma_bf16(tmem + kColGram, d, d, id_gram, s > 0);
                         }
                         mma_commit(bars + 8 * kBarI);
