@@ -602,62 +602,68 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int it = tid - kChain;                 // 0..255
             const int irow = (warp & 3) * 32 + lane;     // tensor-memory lane of this thread
             const int ih = (warp - 8) >> 2;              // which 32-column half of a 64-column tile
+            // (1) for the chunk whose [K;Q] tile is at kqb, by one thread
+            auto issue_gram = [&](uint32_t kqb) {
+                tc_fence_after();
+                const uint64_t dk = smem_desc(kqb, 16, 1024);
+#pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    const uint64_t d = dk + uint64_t(((s >> 2) * kAtomKQ + (s & 3) * 32) >> 4);
+                    mma_bf16(tmem + kColGram, d, d, id_gram, s > 0);
+                }
+                mma_commit(bars + 8 * kBarI);
+            };
+            // gates of the chunk in buffer bb (arrived with its q and k) and their
+            // chunk-local prefix sums, by one warp; tokens past the sequence end get
+            // g = beta = 0 (the identity on S)
+            auto chunk_gates = [&](uint32_t bb, int Lc) {
+                float *vv = reinterpret_cast<float *>(smem + (bb ? kOffVec1 : kOffVec0));
+                const float *stg = reinterpret_cast<const float *>(smem + kOffGst + bb * 2048);
+                const int hc = h & 3;
+                const bool ok0 = 2 * lane < Lc, ok1 = 2 * lane + 1 < Lc;
+                const float g0 = ok0 ? fmaxf(stg[(2 * lane) * 4 + hc], kGFloor) : 0.f;
+                const float g1 = ok1 ? fmaxf(stg[(2 * lane + 1) * 4 + hc], kGFloor) : 0.f;
+                vv[kVecB + 2 * lane] = ok0 ? stg[256 + (2 * lane) * 4 + hc] : 0.f;
+                vv[kVecB + 2 * lane + 1] = ok1 ? stg[256 + (2 * lane + 1) * 4 + hc] : 0.f;
+                float incl = g0 + g1;
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    const float tt = __shfl_up_sync(0xffffffffu, incl, d);
+                    if (lane >= d) incl += tt;
+                }
+                const float excl = incl - (g0 + g1);
+                vv[kVecG + 2 * lane] = excl + g0;
+                vv[kVecG + 2 * lane + 1] = excl + g0 + g1;
+            };
+            // per-token vectors gamma, beta gamma, lambda and 1/gamma (threads 0-63)
+            auto chunk_vectors = [&](uint32_t bb, int Lc) {
+                float *vv = reinterpret_cast<float *>(smem + (bb ? kOffVec1 : kOffVec0));
+                const float G = vv[kVecG + it];
+                vv[kVecGam + it] = __expf(G);
+                vv[kVecBG + it] = vv[kVecB + it] * __expf(G);
+                vv[kVecLam + it] = it < Lc ? __expf(vv[kVecG + Lc - 1] - G) : 0.f;
+                vv[kVecIGam + it] = __expf(-G);
+            };
             for (int n = 0; n < nchunks; ++n) {
                 const uint32_t gcn = gn + n, b = gcn & 1;
-                const int c0 = t0 + n * 64, L = min(64, len - n * 64);
+                const int L = min(64, len - n * 64);
                 float *vec = reinterpret_cast<float *>(smem + (b ? kOffVec1 : kOffVec0));
                 float *gs = vec + kVecG, *bs = vec + kVecB;
                 const uint32_t kq = sb + (b ? kOffKQ1 : kOffKQ0);
                 const uint32_t pt = sb + (b ? kOffP1 : kOffP0);
-                if (gcn >= 2) {  // buffers b were last used by chunk gcn - 2
-                    const bool ok = !intra_poll || mbar_wait(bars + 8 * (kBarEmpty + b), (ph_empty >> b) & 1u);
-                    ph_empty ^= 1u << b;
-                    if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
-                }
-                if (n == 0) {  // later chunks had q, k and their Gram started by the previous chunk
-                    const bool ok = !intra_poll || mbar_wait(bars + 8 * (kBarTKQ + b), (ph_tkq >> b) & 1u);
+                if (n == 0) {  // later chunks are prepared at the end of the previous one
+                    bool ok = true;
+                    if (intra_poll) {
+                        if (gcn >= 2) ok = mbar_wait(bars + 8 * (kBarEmpty + b), (ph_empty >> b) & 1u);
+                        ok = ok && mbar_wait(bars + 8 * (kBarTKQ + b), (ph_tkq >> b) & 1u);
+                    }
+                    if (gcn >= 2) ph_empty ^= 1u << b;
                     ph_tkq ^= 1u << b;
                     if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
-                }
-                // (1) Gram
-                if (it == kIntraIssuer && n == 0) {
-                    tc_fence_after();
-#pragma unroll
-                    for (int s = 0; s < 8; ++s) {
-                        const uint32_t off = (s >> 2) * kAtomKQ + (s & 3) * 32;
-                        mma_bf16(tmem + kColGram, (smem_desc(kq, 16, 1024) + uint64_t((off) >> 4)), (smem_desc(kq, 16, 1024) + uint64_t((off) >> 4)),
-                                 id_gram, s > 0);
-                    }
-                    mma_commit(bars + 8 * kBarI);
-                }
-                // gates of this chunk (arrived with q and k) and their chunk-local
-                // prefix sums, by the first intra warp while the Gram runs; tokens
-                // past the sequence end get g = beta = 0 (the identity on S)
-                if (warp == 8) {
-                    const float *stg = reinterpret_cast<const float *>(smem + kOffGst + b * 2048);
-                    const int hc = h & 3;
-                    const bool ok0 = 2 * lane < L, ok1 = 2 * lane + 1 < L;
-                    const float g0 = ok0 ? fmaxf(stg[(2 * lane) * 4 + hc], kGFloor) : 0.f;
-                    const float g1 = ok1 ? fmaxf(stg[(2 * lane + 1) * 4 + hc], kGFloor) : 0.f;
-                    bs[2 * lane] = ok0 ? stg[256 + (2 * lane) * 4 + hc] : 0.f;
-                    bs[2 * lane + 1] = ok1 ? stg[256 + (2 * lane + 1) * 4 + hc] : 0.f;
-                    float incl = g0 + g1;
-#pragma unroll
-                    for (int d = 1; d < 32; d <<= 1) {
-                        const float tt = __shfl_up_sync(0xffffffffu, incl, d);
-                        if (lane >= d) incl += tt;
-                    }
-                    const float excl = incl - (g0 + g1);
-                    gs[2 * lane] = excl + g0;
-                    gs[2 * lane + 1] = excl + g0 + g1;
-                }
-                named_sync(kBarIntra, kIntra);
-                if (it < 64) {
-                    const float G = gs[it];
-                    vec[kVecGam + it] = __expf(G);
-                    vec[kVecBG + it] = bs[it] * __expf(G);
-                    vec[kVecLam + it] = it < L ? __expf(gs[L - 1] - G) : 0.f;
-                    vec[kVecIGam + it] = __expf(-G);
+                    if (it == kIntraIssuer) issue_gram(kq);
+                    if (warp == 8) chunk_gates(b, L);
+                    named_sync(kBarIntra, kIntra);
+                    if (it < 64) chunk_vectors(b, L);
                 }
                 {
                     const bool ok = !intra_poll || mbar_wait(bars + 8 * kBarI, ph_i);
@@ -712,23 +718,24 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 invert_to_operands(Af, Tf, Yb, it, sb + kOffTp, sb + kOffTpp, vec + kVecBG, bs);
                 if (it == 0) mbar_arrive(bars + 8 * (kBarFull + b));  // chunk gcn ready for the chain
-                // start the next chunk's Gram as soon as its q and k are in (the Gram
-                // accumulator was consumed by this chunk's decay-mask epilogue)
+                // the next chunk: once its q and k are in, warp 15 starts its Gram (the
+                // Gram accumulator was consumed by this chunk's decay masks) while warp
+                // 8 waits for its buffers and scans its gates
                 if (n + 1 < nchunks) {
-                    const uint32_t nb = b ^ 1u, nkq = sb + (nb ? kOffKQ1 : kOffKQ0);
+                    const uint32_t nb = b ^ 1u;
+                    const int L1 = min(64, len - (n + 1) * 64);
                     const bool ok = !intra_poll || mbar_wait(bars + 8 * (kBarTKQ + nb), (ph_tkq >> nb) & 1u);
                     ph_tkq ^= 1u << nb;
                     if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
-                    if (it == kIntraIssuer) {
-                        tc_fence_after();
-                        const uint64_t dk = smem_desc(nkq, 16, 1024);
-#pragma unroll
-                        for (int s = 0; s < 8; ++s) {
-                            const uint64_t d = dk + uint64_t(((s >> 2) * kAtomKQ + (s & 3) * 32) >> 4);
-                            mma_bf16(tmem + kColGram, d, d, id_gram, s > 0);
-                        }
-                        mma_commit(bars + 8 * kBarI);
+                    if (it == kIntraIssuer) issue_gram(sb + (nb ? kOffKQ1 : kOffKQ0));
+                    bool ok2 = true;
+                    if (warp == 8) {
+                        if (gcn + 1 >= 2) ok2 = mbar_wait(bars + 8 * (kBarEmpty + nb), (ph_empty >> nb) & 1u);
+                        if (ok2) chunk_gates(nb, L1);
                     }
+                    if (gcn + 1 >= 2) ph_empty ^= 1u << nb;
+                    if (named_sync_or(kBarIntra, kIntra, !ok2)) { aborted = true; break; }
+                    if (it < 64) chunk_vectors(nb, L1);
                 }
             }
         }
