@@ -323,8 +323,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const bool chain_poll = warp == 0, intra_poll = warp == 8;
     const uint32_t lane_bits = uint32_t((warp & 3) * 32) << 16;  // this warp's tensor-memory lane quarter
     WsHeader *hdr = a.sched.hdr;
-    if (hdr->status != GDN_OK) return;
 
+    // Set-up that needs nothing from the schedule kernel runs while it finishes
+    // (this kernel is launched as its programmatic dependent).
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i) mbar_init(bars + 8 * i, 1);
         fence_mbarrier_init();
@@ -342,6 +343,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
+    grid_dep_wait();  // the schedule and the workspace status word are written
+    if (hdr->status != GDN_OK) {
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+        return;
+    }
 
     const int hv = a.hv, hk = a.hk, group = hv / hk;
     const int total_units = a.num_seqs * hv;
@@ -830,8 +838,21 @@ cudaError_t launch_chunk_tc(const PrefillArgs &a, cudaStream_t stream, int num_s
     const int64_t units = int64_t(a.num_seqs) * a.hv;
     const int grid = int(units < num_sms ? units : num_sms);
     if (grid <= 0) return cudaSuccess;
-    chunk_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mo, mg, mb, a);
+    // launched as a programmatic dependent of the schedule kernel: its set-up
+    // overlaps the schedule, and it waits for the schedule's results on device
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(grid));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, chunk_tc_kernel, mq, mk, mv, mo, mg, mb, a);
     count_launch();
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

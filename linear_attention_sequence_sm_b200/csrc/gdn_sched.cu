@@ -14,6 +14,9 @@ __global__ void __launch_bounds__(kSchedThreads)
 schedule_kernel(int32_t num_seqs, int32_t tokens, int32_t batched_len, const int32_t *__restrict__ cu,
                 WsHeader *hdr, int32_t *order, int32_t *start, int32_t *len) {
     __shared__ int bad;
+    // the prefill kernel that follows may start its own set-up now; it waits for
+    // this kernel's results (griddepcontrol.wait) before reading them
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) {
         bad = -1;
         hdr->status = GDN_OK;
