@@ -425,3 +425,40 @@ int64_t gdn_oracle_num_chunks(const int64_t *cu_seqlens, int64_t num_seqs, int32
     for (int64_t n = 0; n < num_seqs; ++n) acc += (cu_seqlens[n + 1] - cu_seqlens[n] + chunk - 1) / chunk;
     return acc;
 }
+
+/* The input side of the mixer, for callers that hand over raw projections
+ * ("Gated Attention Architectures", the Gated DeltaNet code listing: q and k
+ * L2-normalised per head, the decay gate and the write gate as sigmoids of
+ * per-head logits; "Architecture Thread I", "Modern Architecture
+ * Improvements": L2 normalisation keeps ||k|| = 1 so that the transition's
+ * eigenvalue along k, 1 - beta ||k||^2, stays in (0, 1), and beta comes from
+ * a sigmoid).  In place, fp64, every array token-major as above.
+ *   prep_flags & 2 : q[t, h, :] <- q / max(||q||_2, 1e-12), the same for k
+ *   prep_flags & 4 : g[t, h] holds the decay logit a; alpha = sigmoid(a), so
+ *                    the log-decay becomes g = log sigmoid(a) (written as
+ *                    -log1p(e^-a) for a >= 0 and a - log1p(e^a) below, which
+ *                    are the same function); beta[t, h] holds the write
+ *                    logit b and becomes sigmoid(b) = 1 / (1 + e^-b).       */
+void gdn_oracle_prepare(int64_t tokens, int32_t hk, int32_t hv, int32_t dk, double *q, double *k, double *g,
+                        double *beta, uint32_t prep_flags) {
+    if (prep_flags & 2u) {
+        double *xs[2] = {q, k};
+        for (int which = 0; which < 2; ++which) {
+            double *x = xs[which];
+            for (int64_t r = 0; r < tokens * hk; ++r) {
+                double ss = 0.0;
+                for (int32_t i = 0; i < dk; ++i) ss += x[r * dk + i] * x[r * dk + i];
+                const double nrm = sqrt(ss);
+                const double den = nrm > 1e-12 ? nrm : 1e-12;
+                for (int32_t i = 0; i < dk; ++i) x[r * dk + i] /= den;
+            }
+        }
+    }
+    if (prep_flags & 4u) {
+        for (int64_t r = 0; r < tokens * hv; ++r) {
+            const double a = g[r];
+            g[r] = a >= 0.0 ? -log1p(exp(-a)) : a - log1p(exp(a));
+            beta[r] = 1.0 / (1.0 + exp(-beta[r]));
+        }
+    }
+}

@@ -82,6 +82,10 @@ def load(path: str | None = None):
         lib.gdn_oracle_chunkwise.restype = ctypes.c_int
         lib.gdn_oracle_num_chunks.argtypes = [U, ctypes.c_int64, ctypes.c_int32]
         lib.gdn_oracle_num_chunks.restype = ctypes.c_int64
+        D = ctypes.POINTER(ctypes.c_double)
+        lib.gdn_oracle_prepare.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                           D, D, D, D, ctypes.c_uint32]
+        lib.gdn_oracle_prepare.restype = None
         if path is None:
             _lib = lib
         return lib
@@ -229,3 +233,22 @@ def decode_step(q, k, v, g, beta, state, threads=None, lib=None):
     N = np.asarray(q).shape[0]
     cu = np.arange(N + 1, dtype=np.int64)
     return recurrent(q, k, v, g, beta, initial_state=state, cu_seqlens=cu, threads=threads, lib=lib)
+
+
+def prepare_inputs(q, k, g, beta, qk_l2norm=False, gate_logits=False, lib=None):
+    """fp64 copies of q, k, g, beta with the mixer's input side applied
+    (``gdn_oracle_prepare``): per-head L2 normalisation of q and k, and the
+    decay and write gates from their logits (g = log sigmoid(a),
+    beta = sigmoid(b)).  Arrays keep their shapes: q, k [..., Hk, d_k];
+    g, beta [..., Hv]."""
+    L = lib or load()
+    q64, k64 = _f64(q).copy(), _f64(k).copy()
+    g64, b64 = _f64(g).copy(), _f64(beta).copy()
+    hk, dk = q64.shape[-2], q64.shape[-1]
+    hv = g64.shape[-1]
+    tokens = q64.size // (hk * dk)
+    flags = (2 if qk_l2norm else 0) | (4 if gate_logits else 0)
+    L.gdn_oracle_prepare(ctypes.c_int64(tokens), ctypes.c_int32(hk), ctypes.c_int32(hv), ctypes.c_int32(dk),
+                         _dptr(q64), _dptr(k64), _dptr(g64), _dptr(b64), ctypes.c_uint32(flags))
+    return q64, k64, g64, b64
+

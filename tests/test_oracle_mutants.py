@@ -48,6 +48,12 @@ MUTANTS = [
      "S[i * dk + x] = exp(gl) * S[i * dk + x] + acc;", "S[i * dk + x] = S[i * dk + x] + acc;"),
     ("inter-chunk output term without gamma",
      "ot[i] = exp(G[r]) * inter + intra;", "ot[i] = inter + intra;"),
+    ("q left unnormalised",
+     "double *xs[2] = {q, k};", "double *xs[2] = {k, k};"),
+    ("sigmoid used as the log-decay",
+     "g[r] = a >= 0.0 ? -log1p(exp(-a)) : a - log1p(exp(a));", "g[r] = 1.0 / (1.0 + exp(-a));"),
+    ("log-decay of the negated logit",
+     "g[r] = a >= 0.0 ? -log1p(exp(-a)) : a - log1p(exp(a));", "g[r] = a >= 0.0 ? -a - log1p(exp(-a)) : -log1p(exp(a));"),
     ("A built with Gamma transposed",
      "a = p->beta[(c0 + r) * p->hv + h] * exp(G[r] - G[j]) * kk;",
      "a = p->beta[(c0 + r) * p->hv + h] * exp(G[j] - G[r]) * kk;"),
@@ -72,6 +78,9 @@ class _Bound:
     def decode_step(self, *a, **kw):
         return oracle.decode_step(*a, lib=self.lib, **kw)
 
+    def prepare_inputs(self, *a, **kw):
+        return oracle.prepare_inputs(*a, lib=self.lib, **kw)
+
 
 def _pin_calls(m):
     return [
@@ -85,6 +94,8 @@ def _pin_calls(m):
         lambda: pins.test_chunkwise_equals_recurrent(m, 4, True),
         lambda: pins.test_chunkwise_equals_recurrent(m, 16, False),
         lambda: pins.test_continuation(m, 13),
+        lambda: pins.test_prepare_closed_forms(m),
+        lambda: pins.test_prepared_one_token_closed_form(m),
     ]
 
 

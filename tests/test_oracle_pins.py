@@ -325,3 +325,54 @@ def test_unit_subset_matches_full(oracle_mod):
         np.testing.assert_array_equal(os_[n, :, h], o[n, :, h])
         np.testing.assert_array_equal(ss[n, h], sf[n, h])
     assert np.isnan(os_[0, :, 0]).all()
+
+
+def test_prepare_closed_forms(oracle_mod):
+    """The input side: log-sigmoid and sigmoid closed forms, and the
+    invariants of per-head L2 normalisation."""
+    rng = np.random.default_rng(40)
+    q = rng.standard_normal((7, 3, 8))
+    k = 5.0 * rng.standard_normal((7, 3, 8))
+    k[2, 1] = 0.0  # a zero row stays zero (the 1e-12 floor of the norm)
+    a = np.tile(np.array([0.0, 40.0, -40.0, 1.5, -3.0, 0.25]), (7, 1))
+    b = -a
+    q2, k2, g2, b2 = oracle_mod.prepare_inputs(q, k, a, b, qk_l2norm=True, gate_logits=True)
+    assert np.allclose(np.linalg.norm(q2, axis=-1), 1.0, atol=1e-15)
+    assert np.allclose(np.sum(q2 * q, axis=-1), np.linalg.norm(q, axis=-1), rtol=1e-14)
+    assert np.all(k2[2, 1] == 0.0)
+    kn = np.linalg.norm(k, axis=-1)
+    ok = kn > 0
+    assert np.allclose(np.linalg.norm(k2, axis=-1)[ok], 1.0, atol=1e-15)
+    # log sigmoid: g(0) = -ln 2; g(40) = -e^-40 to first order; g(-40) = -40 in fp64
+    assert abs(g2[0, 0] + np.log(2.0)) < 1e-16
+    assert abs(g2[0, 1] + np.exp(-40.0)) < 1e-33
+    assert g2[0, 2] == -40.0
+    # e^{log sigmoid(a)} + sigmoid(-a) = 1 ties the two gates together; sigmoid(0) = 1/2
+    assert np.allclose(np.exp(g2) + b2, 1.0, atol=2e-16)
+    assert b2[0, 0] == 0.5
+    # a positive scale of the raw projections does not change the normalised rows
+    q3, k3, _, _ = oracle_mod.prepare_inputs(3.7 * q, 0.01 * k, a, b, qk_l2norm=True)
+    assert np.allclose(q3, q2, atol=1e-15) and np.allclose(k3[ok], k2[ok], atol=1e-15)
+    # flags off: values unchanged
+    q4, k4, g4, b4 = oracle_mod.prepare_inputs(q, k, a, b)
+    assert np.array_equal(q4, q) and np.array_equal(k4, k) and np.array_equal(g4, a) and np.array_equal(b4, b)
+
+
+def test_prepared_one_token_closed_form(oracle_mod):
+    """From a zero state, one token of raw inputs gives
+    o = sigmoid(b) v (k . q) / (|k| |q|), whatever the decay logit."""
+    rng = np.random.default_rng(41)
+    d, hk, hv = 6, 1, 2
+    q = rng.standard_normal((1, 1, hk, d))
+    k = 3.0 * rng.standard_normal((1, 1, hk, d))
+    v = rng.standard_normal((1, 1, hv, d))
+    a = rng.standard_normal((1, 1, hv))
+    b = rng.standard_normal((1, 1, hv))
+    q2, k2, g2, b2 = oracle_mod.prepare_inputs(q, k, a, b, qk_l2norm=True, gate_logits=True)
+    o, sf = oracle_mod.recurrent(q2, k2, v, g2, b2)
+    cosine = float(np.dot(q[0, 0, 0], k[0, 0, 0]) / (np.linalg.norm(q[0, 0, 0]) * np.linalg.norm(k[0, 0, 0])))
+    for h in range(hv):
+        sig = 1.0 / (1.0 + np.exp(-b[0, 0, h]))
+        assert np.allclose(o[0, 0, h], sig * cosine * v[0, 0, h], rtol=1e-13, atol=1e-15)
+        assert np.allclose(sf[0, h], sig * np.outer(v[0, 0, h], k[0, 0, 0] / np.linalg.norm(k[0, 0, 0])),
+                           rtol=1e-13, atol=1e-15)
