@@ -27,7 +27,8 @@
  *   - Value head h reads query/key head h / (Hv / Hk) (grouped heads share
  *     their q/k head in contiguous groups); Hv % Hk must be 0.
  *   - Unchecked preconditions (documented, not verified): q and k are
- *     L2-normalised by the caller; beta in (0, 1); g <= 0.  The kernels
+ *     L2-normalised by the caller, beta in (0, 1) and g <= 0 -- unless the
+ *     flags below hand those steps to the library.  The kernels
  *     read g as max(g, -20): exp(-20) is about 2e-9, below fp32 resolution
  *     relative to the state, and the floor keeps the chunk-local prefix
  *     sums of g finite and accurate (g = -inf would make them undefined).
@@ -69,9 +70,21 @@ typedef enum {
 
 typedef enum { GDN_DTYPE_F32 = 0, GDN_DTYPE_BF16 = 1 } gdn_dtype_t;
 
-/* Flags for gdn_shape_t.flags. */
+/* Flags for gdn_shape_t.flags (and the flags argument of gdn_decode_step_ex). */
 #define GDN_FLAG_FORCE_SIMT 1u  /* run the fp32 CUDA-core kernel even where the
                                    tensor-core kernel applies (cross-checks) */
+/* The mixer's input side, done inside the kernels so that no separate pass
+ * over q, k, g and beta is needed ("Gated Attention Architectures", the
+ * Gated DeltaNet code listing: q and k L2-normalised per head, decay and
+ * write gates as sigmoids of per-head logits; "Architecture Thread I",
+ * "Modern Architecture Improvements": L2 normalisation keeps the
+ * transition's eigenvalue along k in (0, 1)).                              */
+#define GDN_FLAG_QK_L2NORM 2u    /* q and k are raw: each (token, head) row is
+                                    used as x / max(||x||_2, 1e-12)          */
+#define GDN_FLAG_GATE_LOGITS 4u  /* g holds the decay logit a and beta the
+                                    write logit b: alpha = sigmoid(a), i.e.
+                                    the log-decay is log sigmoid(a), and the
+                                    write strength is sigmoid(b)            */
 
 /* Shape of a prefill problem.
  *   batch, seq_len  without cu_seqlens: B sequences of T tokens each
@@ -176,6 +189,16 @@ GDN_API gdn_status_t gdn_decode_step(int32_t num_seqs, int32_t num_qk_heads, int
                              const void *q, const void *k, const void *v,
                              const float *g, const float *beta,
                              float *state, void *o, void *stream);
+
+/* gdn_decode_step with flags: GDN_FLAG_QK_L2NORM and GDN_FLAG_GATE_LOGITS
+ * (as for prefill: raw q and k normalised per head inside the kernel; g and
+ * beta given as logits).  flags = 0 is gdn_decode_step.  Other bits return
+ * GDN_ERR_INVALID_ARGUMENT. */
+GDN_API gdn_status_t gdn_decode_step_ex(int32_t num_seqs, int32_t num_qk_heads, int32_t num_v_heads,
+                                int32_t head_dim_k, int32_t head_dim_v, int32_t dtype,
+                                const void *q, const void *k, const void *v,
+                                const float *g, const float *beta,
+                                float *state, void *o, uint32_t flags, void *stream);
 
 /* Static text for a status code. */
 GDN_API const char *gdn_status_string(gdn_status_t status);

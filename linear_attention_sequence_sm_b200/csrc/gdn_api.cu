@@ -54,6 +54,8 @@ static gdn_status_t check_shape(const gdn_shape_t *s) {
                     s->num_v_heads, s->num_qk_heads);
     if (s->dtype != GDN_DTYPE_F32 && s->dtype != GDN_DTYPE_BF16)
         return fail(GDN_ERR_INVALID_ARGUMENT, "dtype %d is not GDN_DTYPE_F32 or GDN_DTYPE_BF16", s->dtype);
+    if (s->flags & ~(GDN_FLAG_FORCE_SIMT | GDN_FLAG_QK_L2NORM | GDN_FLAG_GATE_LOGITS))
+        return fail(GDN_ERR_INVALID_ARGUMENT, "unknown flag bits 0x%x", s->flags);
     if (s->chunk_size != 16 && s->chunk_size != 32 && s->chunk_size != 64)
         return fail(GDN_ERR_UNSUPPORTED, "chunk_size %d not in {16, 32, 64}", s->chunk_size);
     if (s->head_dim_k > 128 || s->head_dim_v > 128)
@@ -143,6 +145,7 @@ gdn_status_t gdn_chunk_forward(const gdn_shape_t *s, const void *q, const void *
     a.chunk = s->chunk_size;
     a.dtype = s->dtype;
     a.tokens = int32_t(tokens);
+    a.flags = s->flags & (GDN_FLAG_QK_L2NORM | GDN_FLAG_GATE_LOGITS);
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.s0 = initial_state; a.o = o; a.s_final = final_state;
     char *ws = static_cast<char *>(workspace);
     a.sched.hdr = reinterpret_cast<WsHeader *>(ws);
@@ -174,7 +177,15 @@ gdn_status_t gdn_read_device_status(const void *workspace, int32_t *device_statu
 gdn_status_t gdn_decode_step(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
                              const void *q, const void *k, const void *v, const float *g, const float *beta,
                              float *state, void *o, void *stream_) {
+    return gdn_decode_step_ex(n, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o, 0u, stream_);
+}
+
+gdn_status_t gdn_decode_step_ex(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
+                                const void *q, const void *k, const void *v, const float *g, const float *beta,
+                                float *state, void *o, uint32_t flags, void *stream_) {
     g_msg[0] = 0;
+    if (flags & ~(GDN_FLAG_QK_L2NORM | GDN_FLAG_GATE_LOGITS))
+        return fail(GDN_ERR_INVALID_ARGUMENT, "unknown decode flag bits 0x%x", flags);
     if (n < 0 || hk <= 0 || hv <= 0 || dk <= 0 || dv <= 0)
         return fail(GDN_ERR_INVALID_ARGUMENT, "bad decode shape");
     if (hv % hk != 0) return fail(GDN_ERR_INVALID_ARGUMENT, "num_v_heads must be a multiple of num_qk_heads");
@@ -189,7 +200,7 @@ gdn_status_t gdn_decode_step(int32_t n, int32_t hk, int32_t hv, int32_t dk, int3
     for (int i = 0; i < 7; ++i)
         if (!aligned16(ptrs[i])) return fail(GDN_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
     if (int64_t(n) * hv * dv * dk > (int64_t(1) << 40)) return fail(GDN_ERR_UNSUPPORTED, "state too large");
-    cudaError_t e = launch_decode(n, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o,
+    cudaError_t e = launch_decode(n, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o, flags,
                                   static_cast<cudaStream_t>(stream_));
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     return GDN_OK;

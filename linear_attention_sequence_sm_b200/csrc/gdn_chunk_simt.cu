@@ -114,10 +114,25 @@ chunk_simt_kernel(PrefillArgs a, int n_slices) {
             }
             if (tid < C) {
                 const size_t off = size_t(t0 + c0 + tid) * hv + h;
-                Gc[tid] = tid < Lc ? fmaxf(a.g[off], kGFloor) : 0.f;
-                Bc[tid] = tid < Lc ? a.beta[off] : 0.f;
+                const bool logits = a.flags & GDN_FLAG_GATE_LOGITS;
+                Gc[tid] = tid < Lc ? fmaxf(logits ? log_sigmoid(a.g[off]) : a.g[off], kGFloor) : 0.f;
+                Bc[tid] = tid < Lc ? (logits ? sigmoid(a.beta[off]) : a.beta[off]) : 0.f;
             }
             __syncthreads();
+            if (a.flags & GDN_FLAG_QK_L2NORM) {
+                // raw q and k: each row scaled by 1 / max(||row||, 1e-12), a warp per row
+                const int warp = tid >> 5, lane = tid & 31;
+                for (int rr = warp; rr < 2 * C; rr += kSimtThreads / 32) {
+                    float *row = (rr < C ? Kc + rr * ldk : Qc + (rr - C) * ldk);
+                    float ss = 0.f;
+                    for (int x = lane; x < dk; x += 32) ss = fmaf(row[x], row[x], ss);
+#pragma unroll
+                    for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+                    const float inv = inv_l2(ss);
+                    for (int x = lane; x < dk; x += 32) row[x] *= inv;
+                }
+                __syncthreads();
+            }
             // 2. cumulative log-decay inside the chunk
             if (tid == 0) {
                 float run = 0.f;

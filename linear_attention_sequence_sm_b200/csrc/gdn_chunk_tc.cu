@@ -89,9 +89,10 @@ constexpr uint32_t kOffOst = 131072;  // output staging: 64 tokens x 128 bf16, t
 constexpr uint32_t kOffAf = 147456;   // A, fp32 64 x kLdA (intra group)
 constexpr uint32_t kOffTf = kOffAf + 64 * kLdA * 4;  // T, fp32 64 x kLdA
 constexpr uint32_t kOffY = kOffTf + 64 * kLdA * 4;   // inverse scratch, 32 x kLdY fp32
-constexpr uint32_t kOffVec0 = kOffY + 32 * kLdY * 4;  // per-token vectors of buffer 0 (6 x 64 fp32)
-constexpr uint32_t kOffVec1 = kOffVec0 + 6 * 64 * 4;  // buffer 1
-constexpr uint32_t kOffGst = kOffVec1 + 6 * 64 * 4;   // gates by TMA, per [K;Q] buffer: g, beta as 64 tokens x 4 heads
+constexpr uint32_t kOffVec0 = kOffY + 32 * kLdY * 4;  // per-token vectors of buffer 0 (10 x 64 fp32)
+constexpr uint32_t kOffVec1 = kOffVec0 + 10 * 64 * 4; // buffer 1
+constexpr uint32_t kOffNrm = kOffVec1 + 10 * 64 * 4;  // 1/||k_r|| (0-63), 1/||q_r|| (64-127) of the next chunk
+constexpr uint32_t kOffGst = kOffNrm + 128 * 4;       // gates by TMA, per [K;Q] buffer: g, beta as 64 tokens x 4 heads
 constexpr uint32_t kOffTp = (kOffGst + 2 * 2048 + 1023) / 1024 * 1024;  // T' = T diag(beta gamma), bf16 64 x 64
 constexpr uint32_t kOffTpp = kOffTp + 8192;                               // T'' = T diag(beta)
 constexpr uint32_t kOffBar = kOffTpp + 8192;          // mbarriers, tensor-memory slot, unit slot
@@ -99,6 +100,15 @@ constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024; // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 per-block limit");
 // per-token vectors inside a buffer (floats)
 constexpr int kVecG = 0, kVecB = 64, kVecGam = 128, kVecBG = 192, kVecLam = 256, kVecIGam = 320;
+// per-token scales through which GDN_FLAG_QK_L2NORM normalises the raw q and k
+// (the plain instantiation reads beta and gamma instead): A rows beta / ||k||^2,
+// P rows 1 / ||q||, T'' columns beta / ||k||, output gamma / ||q||; the T'
+// columns (kVecBG) then carry beta gamma / ||k||^2.  With N_k = diag(||k||):
+// T = N_k (I + diag(beta / ||k||^2) M)^-1 N_k^-1 for M = strict(K K^T (.) Gamma)
+// of the raw K, so W = N_k W' and U~ = N_k U~' with the scaled T', T''; U =
+// N_k U', the state update U'^T diag(lambda) K needs no scale, and the output
+// is diag(gamma / ||q||) Q S^T + diag(1 / ||q||) (Q K^T (.) Gamma) U'.
+constexpr int kVecSa = 384, kVecSp = 448, kVecTpp = 512, kVecGo = 576;
 // mbarrier slots
 constexpr int kBarTKQ = 0, kBarTV = 2, kBarI = 3, kBarC = 4, kBarFull = 5, kBarEmpty = 7, kBarWT = 9, kNumBars = 10;
 // (kBarWT: "T' and T'' consumed", chain -> intra)
@@ -297,6 +307,9 @@ __device__ __forceinline__ void load_v(uint32_t dst, uint32_t bar, const CUtenso
     tma_load_3d(dst + 8192, tv, 64, h, c0, bar);
 }
 
+// kL2: GDN_FLAG_QK_L2NORM; kLogits: GDN_FLAG_GATE_LOGITS (compile-time, so the
+// plain path carries none of the input-side work)
+template <bool kL2, bool kLogits>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -311,6 +324,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float *Af = reinterpret_cast<float *>(smem + kOffAf);
     float *Tf = reinterpret_cast<float *>(smem + kOffTf);
     float *Yb = reinterpret_cast<float *>(smem + kOffY);
+    float *nrm = reinterpret_cast<float *>(smem + kOffNrm);
     const uint32_t bars = sb + kOffBar;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + kOffBar + 8 * kNumBars);
     int *s_unit = reinterpret_cast<int *>(smem + kOffBar + 8 * kNumBars + 4);
@@ -561,7 +575,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         tmem_ld16(tmem + lane_bits + kColX1 + r0, x1);
                         tmem_ld16(tmem + lane_bits + kColX2 + r0, x2);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) load4(vec + kVecGam + r0 + 4 * q, gm + 4 * q);
+                        for (int q = 0; q < 4; ++q) load4(vec + (kL2 ? kVecGo : kVecGam) + r0 + 4 * q, gm + 4 * q);
                         tmem_wait_ld();
                         tmem_st16u(tmem + lane_bits + kColX1 + r0, z);
 #pragma unroll
@@ -629,10 +643,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const float *stg = reinterpret_cast<const float *>(smem + kOffGst + bb * 2048);
                 const int hc = h & 3;
                 const bool ok0 = 2 * lane < Lc, ok1 = 2 * lane + 1 < Lc;
-                const float g0 = ok0 ? fmaxf(stg[(2 * lane) * 4 + hc], kGFloor) : 0.f;
-                const float g1 = ok1 ? fmaxf(stg[(2 * lane + 1) * 4 + hc], kGFloor) : 0.f;
-                vv[kVecB + 2 * lane] = ok0 ? stg[256 + (2 * lane) * 4 + hc] : 0.f;
-                vv[kVecB + 2 * lane + 1] = ok1 ? stg[256 + (2 * lane + 1) * 4 + hc] : 0.f;
+                constexpr bool logits = kLogits;
+                const float ga = stg[(2 * lane) * 4 + hc], gb = stg[(2 * lane + 1) * 4 + hc];
+                const float ba = stg[256 + (2 * lane) * 4 + hc], bb2 = stg[256 + (2 * lane + 1) * 4 + hc];
+                const float g0 = ok0 ? fmaxf(logits ? log_sigmoid_fast(ga) : ga, kGFloor) : 0.f;
+                const float g1 = ok1 ? fmaxf(logits ? log_sigmoid_fast(gb) : gb, kGFloor) : 0.f;
+                vv[kVecB + 2 * lane] = ok0 ? (logits ? sigmoid_fast(ba) : ba) : 0.f;
+                vv[kVecB + 2 * lane + 1] = ok1 ? (logits ? sigmoid_fast(bb2) : bb2) : 0.f;
                 float incl = g0 + g1;
 #pragma unroll
                 for (int d = 1; d < 32; d <<= 1) {
@@ -643,14 +660,45 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 vv[kVecG + 2 * lane] = excl + g0;
                 vv[kVecG + 2 * lane + 1] = excl + g0 + g1;
             };
-            // per-token vectors gamma, beta gamma, lambda and 1/gamma (threads 0-63)
+            // 1 / max(||row||, 1e-12) of the 64 k rows and 64 q rows of the [K;Q]
+            // tile at kqb (GDN_FLAG_QK_L2NORM), one row per thread of warps 9-12
+            constexpr bool l2 = kL2;
+            auto chunk_norms = [&](uint32_t kqb) {
+                const int R = it - 32;  // tile row: k rows 0-63, q rows 64-127
+                float ss[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        // piece p of the row in swizzled order: the 8 lanes that share a
+                        // shared-memory phase hit 8 different 16-byte bank groups
+                        const uint4 w = ld_shared_v4(kqb + c * kAtomKQ + R * 128 + (uint32_t(p ^ (R & 7)) << 4));
+                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const float lo = __uint_as_float(ws[u] << 16), hi = __uint_as_float(ws[u] & 0xffff0000u);
+                            ss[u] = fmaf(lo, lo, fmaf(hi, hi, ss[u]));
+                        }
+                    }
+                nrm[R] = inv_l2((ss[0] + ss[1]) + (ss[2] + ss[3]));
+            };
+            // per-token vectors gamma, beta gamma, lambda and 1/gamma, and the operand scales (threads 0-63)
             auto chunk_vectors = [&](uint32_t bb, int Lc) {
                 float *vv = reinterpret_cast<float *>(smem + (bb ? kOffVec1 : kOffVec0));
-                const float G = vv[kVecG + it];
-                vv[kVecGam + it] = __expf(G);
-                vv[kVecBG + it] = vv[kVecB + it] * __expf(G);
+                const float G = vv[kVecG + it], bt = vv[kVecB + it], gam = __expf(G);
+                vv[kVecGam + it] = gam;
                 vv[kVecLam + it] = it < Lc ? __expf(vv[kVecG + Lc - 1] - G) : 0.f;
                 vv[kVecIGam + it] = __expf(-G);
+                if constexpr (kL2) {
+                    const float ik = nrm[it], iq = nrm[64 + it];  // 1/||k_it||, 1/||q_it||
+                    vv[kVecBG + it] = bt * gam * ik * ik;
+                    vv[kVecSa + it] = bt * ik * ik;
+                    vv[kVecSp + it] = iq;
+                    vv[kVecTpp + it] = bt * ik;
+                    vv[kVecGo + it] = gam * iq;
+                } else {
+                    vv[kVecBG + it] = bt * gam;
+                }
             };
             for (int n = 0; n < nchunks; ++n) {
                 const uint32_t gcn = gn + n, b = gcn & 1;
@@ -670,6 +718,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
                     if (it == kIntraIssuer) issue_gram(kq);
                     if (warp == 8) chunk_gates(b, L);
+                    if (l2 && it >= 32 && it < 160) chunk_norms(kq);
                     named_sync(kBarIntra, kIntra);
                     if (it < 64) chunk_vectors(b, L);
                 }
@@ -684,7 +733,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 {
                     const int r = irow & 63;
                     const bool is_a = irow < 64;
-                    const float scale = is_a ? bs[r] : 1.f;
+                    float scale;
+                    if constexpr (kL2) scale = vec[(is_a ? kVecSa : kVecSp) + r];
+                    else scale = is_a ? bs[r] : 1.f;
                     const int lim = is_a ? r : r + 1;  // A: j < r;  P: j <= r
                     // Gamma_rj = e^(G_r - G_j).  While the chunk's total log-decay is
                     // at least -80, e^(-G_j) stays finite in fp32 and Gamma is the
@@ -724,7 +775,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     ph_wt ^= 1u;
                     if (named_sync_or(kBarIntra, kIntra, !ok)) { aborted = true; break; }
                 }
-                invert_to_operands(Af, Tf, Yb, it, sb + kOffTp, sb + kOffTpp, vec + kVecBG, bs);
+                invert_to_operands(Af, Tf, Yb, it, sb + kOffTp, sb + kOffTpp, vec + kVecBG, kL2 ? vec + kVecTpp : bs);
                 if (it == 0) mbar_arrive(bars + 8 * (kBarFull + b));  // chunk gcn ready for the chain
                 // the next chunk: once its q and k are in, warp 15 starts its Gram (the
                 // Gram accumulator was consumed by this chunk's decay masks) while warp
@@ -741,6 +792,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         if (gcn + 1 >= 2) ok2 = mbar_wait(bars + 8 * (kBarEmpty + nb), (ph_empty >> nb) & 1u);
                         if (ok2) chunk_gates(nb, L1);
                     }
+                    if (l2 && it >= 32 && it < 160) chunk_norms(sb + (nb ? kOffKQ1 : kOffKQ0));
                     if (gcn + 1 >= 2) ph_empty ^= 1u << nb;
                     if (named_sync_or(kBarIntra, kIntra, !ok2)) { aborted = true; break; }
                     if (it < 64) chunk_vectors(nb, L1);
@@ -833,7 +885,10 @@ cudaError_t launch_chunk_tc(const PrefillArgs &a, cudaStream_t stream, int num_s
         !make_map(&mv, a.v, a.hv, a.tokens) || !make_map(&mo, a.o, a.hv, a.tokens, true) ||
         !make_gate_map(&mg, a.g, a.hv, a.tokens) || !make_gate_map(&mb, a.beta, a.hv, a.tokens))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+    const bool l2 = a.flags & GDN_FLAG_QK_L2NORM, logits = a.flags & GDN_FLAG_GATE_LOGITS;
+    auto *kern = l2 ? (logits ? chunk_tc_kernel<true, true> : chunk_tc_kernel<true, false>)
+                    : (logits ? chunk_tc_kernel<false, true> : chunk_tc_kernel<false, false>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
     if (e != cudaSuccess) return e;
     const int64_t units = int64_t(a.num_seqs) * a.hv;
     const int grid = int(units < num_sms ? units : num_sms);
@@ -850,7 +905,7 @@ cudaError_t launch_chunk_tc(const PrefillArgs &a, cudaStream_t stream, int num_s
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, chunk_tc_kernel, mq, mk, mv, mo, mg, mb, a);
+    e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, mg, mb, a);
     count_launch();
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

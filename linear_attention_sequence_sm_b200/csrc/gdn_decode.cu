@@ -49,7 +49,7 @@ __device__ __forceinline__ void load_vec4(const __nv_bfloat16 *p, float out[4]) 
     out[0] = fa.x; out[1] = fa.y; out[2] = fb.x; out[3] = fb.y;
 }
 
-template <typename T>
+template <typename T, uint32_t flags>
 __global__ void __launch_bounds__(kDecodeWarps * 32, GDN_DECODE_MINBLOCKS)
 decode_d128_kernel(int32_t hk, int32_t hv, int32_t dv, const T *__restrict__ q, const T *__restrict__ k,
                    const T *__restrict__ v, const float *__restrict__ g, const float *__restrict__ beta,
@@ -63,9 +63,19 @@ decode_d128_kernel(int32_t hk, int32_t hv, int32_t dv, const T *__restrict__ q, 
     float kf[4], qf[4];
     load_vec4(k + (size_t(n) * hk + hq) * dk + 4 * lane, kf);
     load_vec4(q + (size_t(n) * hk + hq) * dk + 4 * lane, qf);
+    if constexpr ((flags & GDN_FLAG_QK_L2NORM) != 0) {
+        const float ik = inv_l2(warp_sum(kf[0] * kf[0] + kf[1] * kf[1] + kf[2] * kf[2] + kf[3] * kf[3]));
+        const float iq = inv_l2(warp_sum(qf[0] * qf[0] + qf[1] * qf[1] + qf[2] * qf[2] + qf[3] * qf[3]));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            kf[e] *= ik;
+            qf[e] *= iq;
+        }
+    }
     const float kq = warp_sum(kf[0] * qf[0] + kf[1] * qf[1] + kf[2] * qf[2] + kf[3] * qf[3]);
-    const float alpha = __expf(fmaxf(g[unit], kGFloor));
-    const float b = beta[unit];
+    constexpr bool logits = (flags & GDN_FLAG_GATE_LOGITS) != 0;
+    const float alpha = __expf(fmaxf(logits ? log_sigmoid(g[unit]) : g[unit], kGFloor));
+    const float b = logits ? sigmoid(beta[unit]) : beta[unit];
 
     float *S = state + size_t(unit) * dv * dk;
     const T *vrow = v + size_t(unit) * dv;
@@ -113,7 +123,7 @@ decode_d128_kernel(int32_t hk, int32_t hv, int32_t dv, const T *__restrict__ q, 
 }
 
 // Generic d_k <= 256: warp per row, lane l holds elements l, l+32, ...
-template <typename T>
+template <typename T, uint32_t flags>
 __global__ void __launch_bounds__(kDecodeWarps * 32)
 decode_generic_kernel(int32_t hk, int32_t hv, int32_t dk, int32_t dv, const T *__restrict__ q,
                       const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ g,
@@ -124,17 +134,30 @@ decode_generic_kernel(int32_t hk, int32_t hv, int32_t dk, int32_t dv, const T *_
     const int hq = h / (hv / hk);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     float kf[kMaxPer], qf[kMaxPer];
-    float kq = 0.f;
+    float kk = 0.f, qq = 0.f;
 #pragma unroll
     for (int e = 0; e < kMaxPer; ++e) {
         const int j = lane + 32 * e;
         kf[e] = j < dk ? to_f32(k[(size_t(n) * hk + hq) * dk + j]) : 0.f;
         qf[e] = j < dk ? to_f32(q[(size_t(n) * hk + hq) * dk + j]) : 0.f;
-        kq += kf[e] * qf[e];
+        kk += kf[e] * kf[e];
+        qq += qf[e] * qf[e];
     }
+    if constexpr ((flags & GDN_FLAG_QK_L2NORM) != 0) {
+        const float ik = inv_l2(warp_sum(kk)), iq = inv_l2(warp_sum(qq));
+#pragma unroll
+        for (int e = 0; e < kMaxPer; ++e) {
+            kf[e] *= ik;
+            qf[e] *= iq;
+        }
+    }
+    float kq = 0.f;
+#pragma unroll
+    for (int e = 0; e < kMaxPer; ++e) kq += kf[e] * qf[e];
     kq = warp_sum(kq);
-    const float alpha = __expf(fmaxf(g[unit], kGFloor));
-    const float b = beta[unit];
+    constexpr bool logits = (flags & GDN_FLAG_GATE_LOGITS) != 0;
+    const float alpha = __expf(fmaxf(logits ? log_sigmoid(g[unit]) : g[unit], kGFloor));
+    const float b = logits ? sigmoid(beta[unit]) : beta[unit];
     float *S = state + size_t(unit) * dv * dk;
     for (int i = warp; i < dv; i += kDecodeWarps) {
         float s[kMaxPer];
@@ -158,30 +181,52 @@ decode_generic_kernel(int32_t hk, int32_t hv, int32_t dk, int32_t dv, const T *_
     }
 }
 
-cudaError_t launch_decode(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
-                          const void *q, const void *k, const void *v, const float *g, const float *beta,
-                          float *state, void *o, cudaStream_t stream) {
-    const int64_t units = int64_t(n) * hv;
-    if (units > INT32_MAX) return cudaErrorInvalidValue;
-    const dim3 grid(static_cast<unsigned>(units)), block(kDecodeWarps * 32);
+template <uint32_t F>
+static void launch_decode_as(dim3 grid, dim3 block, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
+                             const void *q, const void *k, const void *v, const float *g, const float *beta,
+                             float *state, void *o, cudaStream_t stream) {
+    using bf = __nv_bfloat16;
     if (dk == 128) {
         if (dtype == GDN_DTYPE_BF16)
-            decode_d128_kernel<__nv_bfloat16><<<grid, block, 0, stream>>>(
-                hk, hv, dv, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
-                static_cast<const __nv_bfloat16 *>(v), g, beta, state, static_cast<__nv_bfloat16 *>(o));
+            decode_d128_kernel<bf, F><<<grid, block, 0, stream>>>(
+                hk, hv, dv, static_cast<const bf *>(q), static_cast<const bf *>(k), static_cast<const bf *>(v), g,
+                beta, state, static_cast<bf *>(o));
         else
-            decode_d128_kernel<float><<<grid, block, 0, stream>>>(
+            decode_d128_kernel<float, F><<<grid, block, 0, stream>>>(
                 hk, hv, dv, static_cast<const float *>(q), static_cast<const float *>(k),
                 static_cast<const float *>(v), g, beta, state, static_cast<float *>(o));
     } else {
         if (dtype == GDN_DTYPE_BF16)
-            decode_generic_kernel<__nv_bfloat16><<<grid, block, 0, stream>>>(
-                hk, hv, dk, dv, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
-                static_cast<const __nv_bfloat16 *>(v), g, beta, state, static_cast<__nv_bfloat16 *>(o));
+            decode_generic_kernel<bf, F><<<grid, block, 0, stream>>>(
+                hk, hv, dk, dv, static_cast<const bf *>(q), static_cast<const bf *>(k), static_cast<const bf *>(v),
+                g, beta, state, static_cast<bf *>(o));
         else
-            decode_generic_kernel<float><<<grid, block, 0, stream>>>(
+            decode_generic_kernel<float, F><<<grid, block, 0, stream>>>(
                 hk, hv, dk, dv, static_cast<const float *>(q), static_cast<const float *>(k),
                 static_cast<const float *>(v), g, beta, state, static_cast<float *>(o));
+    }
+}
+
+cudaError_t launch_decode(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
+                          const void *q, const void *k, const void *v, const float *g, const float *beta,
+                          float *state, void *o, uint32_t flags, cudaStream_t stream) {
+    const int64_t units = int64_t(n) * hv;
+    if (units > INT32_MAX) return cudaErrorInvalidValue;
+    const dim3 grid(static_cast<unsigned>(units)), block(kDecodeWarps * 32);
+    switch (flags) {
+        case 0: launch_decode_as<0>(grid, block, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o, stream); break;
+        case GDN_FLAG_QK_L2NORM:
+            launch_decode_as<GDN_FLAG_QK_L2NORM>(grid, block, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o,
+                                                 stream);
+            break;
+        case GDN_FLAG_GATE_LOGITS:
+            launch_decode_as<GDN_FLAG_GATE_LOGITS>(grid, block, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o,
+                                                   stream);
+            break;
+        default:
+            launch_decode_as<GDN_FLAG_QK_L2NORM | GDN_FLAG_GATE_LOGITS>(grid, block, hk, hv, dk, dv, dtype, q, k,
+                                                                       v, g, beta, state, o, stream);
+            break;
     }
     count_launch();
     return cudaGetLastError();

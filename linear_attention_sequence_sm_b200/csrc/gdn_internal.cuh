@@ -15,6 +15,21 @@ namespace gdn {
 // chunk-local prefix sums of g finite (g = -inf would give -inf - -inf).
 constexpr float kGFloor = -20.0f;
 
+// The input side of the mixer (GDN_FLAG_GATE_LOGITS, GDN_FLAG_QK_L2NORM):
+// log sigmoid(a) as -log1p(e^-a) for a >= 0 and a - log1p(e^a) below (the same
+// function, each form free of overflow); sigmoid(b); and the reciprocal of
+// max(||x||_2, 1e-12) from the sum of squares.
+__device__ __forceinline__ float log_sigmoid(float a) { return a >= 0.f ? -log1pf(expf(-a)) : a - log1pf(expf(a)); }
+__device__ __forceinline__ float sigmoid(float b) { return 1.f / (1.f + expf(-b)); }
+__device__ __forceinline__ float inv_l2(float sum_sq) { return 1.f / fmaxf(sqrtf(sum_sq), 1e-12f); }
+// The same two gates with the fast exponential and logarithm intrinsics, for
+// the bf16 tensor-core path: their absolute error in log sigmoid is about
+// 1e-7, far below that path's bf16 rounding.
+__device__ __forceinline__ float log_sigmoid_fast(float a) {
+    return a >= 0.f ? -__logf(1.f + __expf(-a)) : a - __logf(1.f + __expf(a));
+}
+__device__ __forceinline__ float sigmoid_fast(float b) { return __fdividef(1.f, 1.f + __expf(-b)); }
+
 // ---------------------------------------------------------------------------
 // Workspace layout of gdn_chunk_forward (all offsets 256-byte aligned).
 //   [0, 256)              WsHeader
@@ -79,6 +94,7 @@ cudaError_t launch_schedule(const gdn_shape_t &s, const int32_t *cu_seqlens, voi
 struct PrefillArgs {
     int32_t num_seqs, hk, hv, dk, dv, chunk, dtype;
     int32_t tokens;  // rows of q, k, v, o (B * T, or the packed total)
+    uint32_t flags;  // GDN_FLAG_QK_L2NORM | GDN_FLAG_GATE_LOGITS (input side in the kernels)
     const void *q, *k, *v;
     const float *g, *beta, *s0;
     void *o;
@@ -96,6 +112,6 @@ bool chunk_tc_supported(const gdn_shape_t &s);
 // Decode step.
 cudaError_t launch_decode(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
                           const void *q, const void *k, const void *v, const float *g, const float *beta,
-                          float *state, void *o, cudaStream_t stream);
+                          float *state, void *o, uint32_t flags, cudaStream_t stream);
 
 }  // namespace gdn

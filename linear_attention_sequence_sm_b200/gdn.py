@@ -30,10 +30,12 @@ GDN_ERR_DEVICE_CHECK = 6
 GDN_DTYPE_F32 = 0
 GDN_DTYPE_BF16 = 1
 GDN_FLAG_FORCE_SIMT = 1
+GDN_FLAG_QK_L2NORM = 2
+GDN_FLAG_GATE_LOGITS = 4
 
 EXPORTED = ("gdn_chunk_forward_workspace_size", "gdn_chunk_forward", "gdn_read_device_status",
             "gdn_decode_step", "gdn_status_string", "gdn_last_error_message", "gdn_launch_count",
-            "gdn_chunk_forward_noalloc")
+            "gdn_chunk_forward_noalloc", "gdn_decode_step_ex")
 
 
 class GdnError(RuntimeError):
@@ -66,6 +68,8 @@ def _load(path: str = LIB_PATH):
     lib.gdn_read_device_status.restype = st
     lib.gdn_decode_step.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.gdn_decode_step.restype = st
+    lib.gdn_decode_step_ex.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, ctypes.c_uint32, vp]
+    lib.gdn_decode_step_ex.restype = st
     lib.gdn_status_string.argtypes = [st]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_last_error_message.argtypes = []
@@ -114,7 +118,13 @@ def _need(t, name, dtype=None, device=None):
         raise ValueError(f"{name} is on {t.device}, expected {device}")
 
 
-def make_shape(q, v, cu_seqlens=None, chunk_size=64, force_simt=False) -> Shape:
+def input_flags(qk_l2norm=False, gate_logits=False) -> int:
+    """GDN_FLAG_QK_L2NORM / GDN_FLAG_GATE_LOGITS bits: raw q and k normalised
+    per head inside the kernels; g and beta given as logits."""
+    return (GDN_FLAG_QK_L2NORM if qk_l2norm else 0) | (GDN_FLAG_GATE_LOGITS if gate_logits else 0)
+
+
+def make_shape(q, v, cu_seqlens=None, chunk_size=64, force_simt=False, flags=0) -> Shape:
     if cu_seqlens is not None:
         T = q.shape[-3]
         B, N = 1, cu_seqlens.shape[0] - 1
@@ -124,7 +134,7 @@ def make_shape(q, v, cu_seqlens=None, chunk_size=64, force_simt=False) -> Shape:
         B, T = q.shape[0], q.shape[1]
         N = B
     return Shape(B, T, N, q.shape[-2], v.shape[-2], q.shape[-1], v.shape[-1], chunk_size, _dtype_code(q),
-                 GDN_FLAG_FORCE_SIMT if force_simt else 0)
+                 (GDN_FLAG_FORCE_SIMT if force_simt else 0) | flags)
 
 
 def workspace_size(shape: Shape) -> int:
@@ -135,9 +145,11 @@ def workspace_size(shape: Shape) -> int:
 
 def chunk_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_size=64,
                   output_final_state=True, out=None, final_state=None, workspace=None, force_simt=False,
-                  stream=None):
+                  stream=None, qk_l2norm=False, gate_logits=False):
     """Chunkwise prefill.  Returns (o, final_state or None).  Asynchronous on
-    ``stream`` (default: the current stream)."""
+    ``stream`` (default: the current stream).  ``qk_l2norm``: q and k are raw
+    and normalised per head in the kernel; ``gate_logits``: g and beta are
+    the decay and write logits (alpha = sigmoid(g), beta = sigmoid(beta))."""
     dev = q.device
     dt = q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -148,7 +160,7 @@ def chunk_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_s
     _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
     if k.shape != q.shape:
         raise ValueError("k must have the shape of q")
-    shape = make_shape(q, v, cu_seqlens, chunk_size, force_simt)
+    shape = make_shape(q, v, cu_seqlens, chunk_size, force_simt, input_flags(qk_l2norm, gate_logits))
     if out is None:
         out = torch.empty(v.shape, dtype=dt, device=dev)
     _need(out, "out", dt, dev)
@@ -166,7 +178,8 @@ def chunk_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_s
 
 
 def chunk_forward_noalloc(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_size=64,
-                          output_final_state=True, out=None, final_state=None, force_simt=False, stream=None):
+                          output_final_state=True, out=None, final_state=None, force_simt=False, stream=None,
+                          qk_l2norm=False, gate_logits=False):
     """chunk_forward for callers that cannot allocate device scratch: the
     library's built-in scratch array stands in for the workspace (at most
     16,384 sequences; calls that overlap on the GPU race on that array).
@@ -180,7 +193,7 @@ def chunk_forward_noalloc(q, k, v, g, beta, initial_state=None, cu_seqlens=None,
     _need(beta, "beta", torch.float32, dev)
     _need(initial_state, "initial_state", torch.float32, dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
-    shape = make_shape(q, v, cu_seqlens, chunk_size, force_simt)
+    shape = make_shape(q, v, cu_seqlens, chunk_size, force_simt, input_flags(qk_l2norm, gate_logits))
     if out is None:
         out = torch.empty(v.shape, dtype=dt, device=dev)
     _need(out, "out", dt, dev)
@@ -202,9 +215,10 @@ def read_device_status(workspace, stream=None) -> int:
     return st.value
 
 
-def decode_step(q, k, v, g, beta, state, out=None, stream=None):
+def decode_step(q, k, v, g, beta, state, out=None, stream=None, qk_l2norm=False, gate_logits=False):
     """One token per sequence; ``state`` [N, Hv, d_v, d_k] fp32 is updated in
-    place.  Returns o [N, Hv, d_v]."""
+    place.  Returns o [N, Hv, d_v].  ``qk_l2norm`` and ``gate_logits`` as for
+    chunk_forward."""
     dev, dt = q.device, q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, dt, dev)
@@ -216,8 +230,9 @@ def decode_step(q, k, v, g, beta, state, out=None, stream=None):
     _need(out, "out", dt, dev)
     N, hk, dk = q.shape
     hv, dv = v.shape[1], v.shape[2]
-    _check(LIB.gdn_decode_step(N, hk, hv, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
-                               _ptr(beta), _ptr(state), _ptr(out), _stream_handle(stream)))
+    _check(LIB.gdn_decode_step_ex(N, hk, hv, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                  _ptr(beta), _ptr(state), _ptr(out), input_flags(qk_l2norm, gate_logits),
+                                  _stream_handle(stream)))
     return out
 
 
