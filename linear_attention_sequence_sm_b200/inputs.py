@@ -212,6 +212,33 @@ def make_prefill_inputs(w: Workload):
     return out
 
 
+def make_raw_prefill_inputs(w: Workload):
+    """The workload's shapes with raw projections, for the input side done in
+    the kernels (GDN_FLAG_QK_L2NORM, GDN_FLAG_GATE_LOGITS): q and k rows
+    N(0,1) times a per-(token, head) norm factor uniform in [0.3, 6] (not
+    normalised), v N(0,1), decay logits a ~ N(1.5, 1) (alpha = sigmoid(a)) and
+    write logits b ~ N(0, 1) (beta = sigmoid(b)); states and cu_seqlens as in
+    make_prefill_inputs."""
+    import torch
+    base = make_prefill_inputs(w)
+    B, T, hk, hv, d = w.batch, w.seq_len, w.hk, w.hv, w.d
+    s = w.seed
+    st = _torch_dtype(w.dtype)
+    rows = B * T * hk
+
+    def raw(tag):
+        def f(z):
+            return z
+        x = _slabbed(s, tag, (B, T, hk, d), f, torch.float32, d)
+        sc = torch.from_numpy(0.3 + 5.7 * uniform(s, tag + "_scale", rows)).float().reshape(B, T, hk, 1)
+        return (x * sc).to(st)
+
+    base["q"], base["k"] = raw("raw_q"), raw("raw_k")
+    base["g"] = _slabbed(s, "raw_a", (B, T, hv), lambda z: z + 1.5, torch.float32, hv)
+    base["beta"] = _slabbed(s, "raw_b", (B, T, hv), lambda z: z, torch.float32, hv)
+    return base
+
+
 def make_decode_inputs(w: DecodeWorkload, step: int):
     """Fresh per-step q, k [N,Hk,d], v [N,Hv,d], g, beta [N,Hv] (seed + step)."""
     import torch
