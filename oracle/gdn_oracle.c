@@ -39,6 +39,12 @@
  *                             write S <- S - beta (S k - v) k^T
  *                             ("Architecture Thread I", the delta-rule
  *                             update), with no gate.
+ * and the mixer's two sides around the recurrence:
+ *   gdn_oracle_prepare       -- q, k L2-normalised per head; gates from
+ *                             their logits (the input side).
+ *   gdn_oracle_output_side   -- RMS normalisation of each output row with a
+ *                             scale and an optional SiLU or sigmoid gate
+ *                             (the output side).
  *
  * Layouts (all row-major, token-major, fp64):
  *   q, k          [T_total, Hk, d_k]
@@ -459,6 +465,48 @@ void gdn_oracle_prepare(int64_t tokens, int32_t hk, int32_t hv, int32_t dk, doub
             const double a = g[r];
             g[r] = a >= 0.0 ? -log1p(exp(-a)) : a - log1p(exp(a));
             beta[r] = 1.0 / (1.0 + exp(-beta[r]));
+        }
+    }
+}
+
+/* The mixer's output side, applied to the read-out o of the recurrence.
+ * "Architecture Thread I", "Modern Architecture Improvements": the mixer's
+ * output is RMS-normalised before the output projection (in place of a
+ * softmax-style denominator).  "The Transformer Isn't Alone Anymore" lists
+ * a gated RMSNorm in the Gated DeltaNet block; the Gated DeltaNet code
+ * listing of "Gated Attention Architectures" multiplies the normalised
+ * output by SiLU of a gate projection; the Gated Attention section of the
+ * same page names the sigmoid gate; the Qwen3-Next passage of "Architecture
+ * Thread I" holds the norm's scale as 1 + delta ("zero-centred").
+ * For every (token, value head) row o of d_v values:
+ *     ms  = (1 / d_v) sum_j o_j^2
+ *     y_i = o_i / sqrt(ms + eps) * s_i * act(z_i)
+ *   out_flags & 1 : act(z) = z / (1 + e^-z)      (SiLU)
+ *   out_flags & 2 : act(z) = 1 / (1 + e^-z)      (sigmoid)
+ *   neither       : act = 1 and z is not read
+ *   out_flags & 4 : s_i = 1 + w_i (zero-centred; w NULL reads as 0)
+ *   otherwise     : s_i = w_i (w NULL reads as 1)
+ *   out_flags & 8 : w is [Hv, d_v], a row per value head; otherwise [d_v]
+ * o, z, y are [tokens, Hv, d_v]; y may alias o. */
+void gdn_oracle_output_side(int64_t tokens, int32_t hv, int32_t dv, const double *o, const double *z,
+                            const double *w, double eps, uint32_t out_flags, double *y) {
+    for (int64_t t = 0; t < tokens; ++t) {
+        for (int32_t h = 0; h < hv; ++h) {
+            const int64_t row = (t * hv + h) * dv;
+            double ms = 0.0;
+            for (int32_t i = 0; i < dv; ++i) ms += o[row + i] * o[row + i];
+            ms /= dv;
+            const double inv_rms = 1.0 / sqrt(ms + eps);
+            const double *wr = w ? w + ((out_flags & 8u) ? (int64_t)h * dv : 0) : NULL;
+            for (int32_t i = 0; i < dv; ++i) {
+                double s;
+                if (out_flags & 4u) s = 1.0 + (wr ? wr[i] : 0.0);
+                else s = wr ? wr[i] : 1.0;
+                double gate = 1.0;
+                if (out_flags & 1u) gate = z[row + i] / (1.0 + exp(-z[row + i]));
+                else if (out_flags & 2u) gate = 1.0 / (1.0 + exp(-z[row + i]));
+                y[row + i] = o[row + i] * inv_rms * s * gate;
+            }
         }
     }
 }

@@ -86,6 +86,9 @@ def load(path: str | None = None):
         lib.gdn_oracle_prepare.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                            D, D, D, D, ctypes.c_uint32]
         lib.gdn_oracle_prepare.restype = None
+        lib.gdn_oracle_output_side.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, D, D, D,
+                                               ctypes.c_double, ctypes.c_uint32, D]
+        lib.gdn_oracle_output_side.restype = None
         if path is None:
             _lib = lib
         return lib
@@ -251,4 +254,41 @@ def prepare_inputs(q, k, g, beta, qk_l2norm=False, gate_logits=False, lib=None):
     L.gdn_oracle_prepare(ctypes.c_int64(tokens), ctypes.c_int32(hk), ctypes.c_int32(hv), ctypes.c_int32(dk),
                          _dptr(q64), _dptr(k64), _dptr(g64), _dptr(b64), ctypes.c_uint32(flags))
     return q64, k64, g64, b64
+
+
+# output-side flags of gdn_oracle_output_side (the oracle's own numbering)
+OUT_GATE_SILU, OUT_GATE_SIGMOID, OUT_ZERO_CENTRED, OUT_WEIGHT_PER_HEAD = 1, 2, 4, 8
+
+
+def output_side(o, z=None, weight=None, eps=1e-6, gate="silu", zero_centred=False, lib=None):
+    """The mixer's output side on o [..., Hv, d_v] in fp64
+    (``gdn_oracle_output_side``): each (token, value head) row divided by
+    its root mean square (+ eps inside the root), times the scale (w, or
+    1 + w when zero_centred; weight [d_v] shared by the heads or [Hv, d_v]
+    per head), times act(z) with act = SiLU or sigmoid (``gate``) when z is
+    given.  Returns a new array of o's shape."""
+    L = lib or load()
+    o64 = _f64(o).copy()
+    hv, dv = o64.shape[-2], o64.shape[-1]
+    tokens = o64.size // (hv * dv)
+    flags = 0
+    z64 = None
+    if z is not None:
+        z64 = _f64(z).copy()
+        assert z64.shape == o64.shape
+        flags |= {"silu": OUT_GATE_SILU, "sigmoid": OUT_GATE_SIGMOID}[gate]
+    w64 = None
+    if weight is not None:
+        w64 = _f64(weight).copy()
+        if w64.ndim == 2:
+            assert w64.shape == (hv, dv)
+            flags |= OUT_WEIGHT_PER_HEAD
+        else:
+            assert w64.shape == (dv,)
+    if zero_centred:
+        flags |= OUT_ZERO_CENTRED
+    y = np.empty_like(o64)
+    L.gdn_oracle_output_side(ctypes.c_int64(tokens), ctypes.c_int32(hv), ctypes.c_int32(dv), _dptr(o64),
+                             _dptr(z64), _dptr(w64), ctypes.c_double(eps), ctypes.c_uint32(flags), _dptr(y))
+    return y
 

@@ -54,6 +54,17 @@ MUTANTS = [
      "g[r] = a >= 0.0 ? -log1p(exp(-a)) : a - log1p(exp(a));", "g[r] = 1.0 / (1.0 + exp(-a));"),
     ("log-decay of the negated logit",
      "g[r] = a >= 0.0 ? -log1p(exp(-a)) : a - log1p(exp(a));", "g[r] = a >= 0.0 ? -a - log1p(exp(-a)) : -log1p(exp(a));"),
+    ("RMS over the sum of squares, not the mean",
+     "    ms /= dv;\n", "\n"),
+    ("eps outside the root",
+     "const double inv_rms = 1.0 / sqrt(ms + eps);", "const double inv_rms = 1.0 / (sqrt(ms) + eps);"),
+    ("SiLU gate without its z factor",
+     "gate = z[row + i] / (1.0 + exp(-z[row + i]));", "gate = 1.0 / (1.0 + exp(-z[row + i]));"),
+    ("zero-centred scale without its 1",
+     "if (out_flags & 4u) s = 1.0 + (wr ? wr[i] : 0.0);", "if (out_flags & 4u) s = (wr ? wr[i] : 0.0);"),
+    ("per-head scale rows ignored",
+     "const double *wr = w ? w + ((out_flags & 8u) ? (int64_t)h * dv : 0) : NULL;",
+     "const double *wr = w;"),
     ("A built with Gamma transposed",
      "a = p->beta[(c0 + r) * p->hv + h] * exp(G[r] - G[j]) * kk;",
      "a = p->beta[(c0 + r) * p->hv + h] * exp(G[j] - G[r]) * kk;"),
@@ -81,6 +92,9 @@ class _Bound:
     def prepare_inputs(self, *a, **kw):
         return oracle.prepare_inputs(*a, lib=self.lib, **kw)
 
+    def output_side(self, *a, **kw):
+        return oracle.output_side(*a, lib=self.lib, **kw)
+
 
 def _pin_calls(m):
     return [
@@ -96,6 +110,8 @@ def _pin_calls(m):
         lambda: pins.test_continuation(m, 13),
         lambda: pins.test_prepare_closed_forms(m),
         lambda: pins.test_prepared_one_token_closed_form(m),
+        lambda: pins.test_output_side_handworked(m),
+        lambda: pins.test_output_side_invariants(m),
     ]
 
 

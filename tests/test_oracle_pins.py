@@ -376,3 +376,51 @@ def test_prepared_one_token_closed_form(oracle_mod):
         assert np.allclose(o[0, 0, h], sig * cosine * v[0, 0, h], rtol=1e-13, atol=1e-15)
         assert np.allclose(sf[0, h], sig * np.outer(v[0, 0, h], k[0, 0, 0] / np.linalg.norm(k[0, 0, 0])),
                            rtol=1e-13, atol=1e-15)
+
+
+def test_output_side_handworked(oracle_mod):
+    """The output side on a two-channel row worked by hand: o = (3, 4) has
+    mean square 12.5, so the normalised row is (3, 4) / sqrt(12.5) =
+    (0.8485..., 1.1313...); sigmoid(ln 3) = 3/4, so SiLU(ln 3) = (3/4) ln 3;
+    SiLU(0) = 0 and sigmoid(0) = 1/2."""
+    o = np.array([[[3.0, 4.0]]])
+    r = np.sqrt(12.5)
+    y = oracle_mod.output_side(o, eps=0.0)
+    assert np.allclose(y, [[[3.0 / r, 4.0 / r]]], rtol=1e-15)
+    w = np.array([2.0, 0.5])
+    z = np.array([[[0.0, np.log(3.0)]]])
+    y = oracle_mod.output_side(o, z=z, weight=w, eps=0.0, gate="silu")
+    assert np.allclose(y, [[[0.0, 2.0 / r * 0.75 * np.log(3.0)]]], rtol=1e-15, atol=0)
+    y = oracle_mod.output_side(o, z=z, weight=w, eps=0.0, gate="sigmoid")
+    assert np.allclose(y, [[[0.5 * 6.0 / r, 0.75 * 2.0 / r]]], rtol=1e-15)
+    # eps inside the root: a constant row c gives c / sqrt(c^2 + eps)
+    c = np.full((1, 1, 5), 0.2)
+    y = oracle_mod.output_side(c, eps=0.01)
+    assert np.allclose(y, 0.2 / np.sqrt(0.04 + 0.01), rtol=1e-15)
+
+
+def test_output_side_invariants(oracle_mod):
+    """Invariants of RMS normalisation on random rows: mean(y^2) =
+    ms / (ms + eps) with unit scale; a positive rescaling of o leaves y
+    unchanged when eps = 0; the zero-centred scale 1 + w equals the plain
+    scale 1 + w; per-head scales act on their own head only."""
+    rng = np.random.default_rng(42)
+    T, hv, dv = 6, 3, 16
+    o = rng.standard_normal((T, hv, dv)) * rng.uniform(0.2, 3.0, (T, hv, 1))
+    ms = np.mean(o * o, axis=-1)
+    eps = 0.3
+    y = oracle_mod.output_side(o, eps=eps)
+    assert np.allclose(np.mean(y * y, axis=-1), ms / (ms + eps), rtol=1e-14)
+    assert np.allclose(oracle_mod.output_side(7.5 * o, eps=0.0), oracle_mod.output_side(o, eps=0.0), rtol=1e-14)
+    d = 0.1 * rng.standard_normal(dv)
+    assert np.allclose(oracle_mod.output_side(o, weight=d, eps=eps, zero_centred=True),
+                       oracle_mod.output_side(o, weight=1.0 + d, eps=eps), rtol=1e-15)
+    assert np.array_equal(oracle_mod.output_side(o, eps=eps, zero_centred=True), y)
+    wh = np.stack([np.full(dv, h + 1.0) for h in range(hv)])
+    yh = oracle_mod.output_side(o, weight=wh, eps=eps)
+    for h in range(hv):
+        assert np.allclose(yh[:, h], (h + 1.0) * y[:, h], rtol=1e-15)
+    # the gate multiplies elementwise: SiLU(z) = z sigmoid(z), against numpy
+    z = rng.standard_normal((T, hv, dv)) * 3.0
+    yg = oracle_mod.output_side(o, z=z, eps=eps, gate="silu")
+    assert np.allclose(yg, y * z / (1.0 + np.exp(-z)), rtol=1e-14)
