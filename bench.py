@@ -52,6 +52,8 @@ def parse_args(argv=None):
                    help="time only one of the two paths (used by profiling commands)")
     p.add_argument("--raw-inputs", action="store_true",
                    help="prefill on raw q/k and gate logits, normalised and gated inside the kernels")
+    p.add_argument("--output-norm", action="store_true",
+                   help="prefill with the output side (RMS norm, per-channel scale, SiLU gate) in the kernel")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
@@ -263,7 +265,17 @@ def run_ours(args):
         seed={"prefill": 1002, "long": 1003, "varlen": 1005}[args.workload] + rank)
     host = I.make_raw_prefill_inputs(w) if args.raw_inputs else I.make_prefill_inputs(w)
     flags = {"qk_l2norm": True, "gate_logits": True} if args.raw_inputs else {}
+    suffix = ("_raw_inputs" if args.raw_inputs else "") + ("_output_norm" if args.output_norm else "")
+    if args.output_norm:
+        host["out_gate"] = I.make_output_gate(w)
+        out_weight = I.make_output_weight(w).to(device)
     dev = {k: (v.to(device) if v is not None else None) for k, v in host.items()}
+
+    def out_norm(x):
+        if not args.output_norm:
+            return {}
+        return {"output_norm": gdn.OutputNorm(weight=out_weight, gate=x["out_gate"], eps=1e-6, activation="silu")}
+
     o = torch.empty_like(dev["v"])
     sf = torch.empty((w.num_seqs, w.hv, w.d, w.d), dtype=torch.float32, device=device)
     shape = gdn.make_shape(dev["q"], dev["v"], dev["cu_seqlens"], w.chunk)
@@ -273,7 +285,7 @@ def run_ours(args):
     def step():
         gdn.chunk_forward(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], initial_state=dev["initial_state"],
                           cu_seqlens=dev["cu_seqlens"], out=o, final_state=sf, workspace=ws, chunk_size=w.chunk,
-                          **flags)
+                          **flags, **out_norm(dev))
 
     ms = ms_max = float("nan")
     launches = 0
@@ -298,7 +310,7 @@ def run_ours(args):
     kernel_name = "gdn_chunk_tc" if gdn_tc_active(gdn, dev, w) else "gdn_chunk_simt"
     roofline = {"bound": "tensor", "achieved": achieved_tflops, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved_tflops / peaks["bf16_tflops"],
-                "traffic": kernel_traffic(f"{kernel_name}/{w.name}" + ("_raw_inputs" if args.raw_inputs else "")),
+                "traffic": kernel_traffic(f"{kernel_name}/{w.name}{suffix}"),
                 "kernel": kernel_name,
                 "peak_source": f"{peak_src} bf16 dense (burst)",
                 "flops_per_launch": flops, "algorithmic_bytes_per_launch": prefill_bytes(w)}
@@ -350,7 +362,8 @@ def run_ours(args):
         def e2e_step():
             x = {k: v.to(device, non_blocking=True) for k, v in pin.items()}
             oo, ss = gdn.chunk_forward(x["q"], x["k"], x["v"], x["g"], x["beta"], initial_state=x.get("initial_state"),
-                                       cu_seqlens=x.get("cu_seqlens"), chunk_size=w.chunk, workspace=ws, **flags)
+                                       cu_seqlens=x.get("cu_seqlens"), chunk_size=w.chunk, workspace=ws, **flags,
+                                       **out_norm(x))
             o_host.copy_(oo, non_blocking=True)
             sf_host.copy_(ss, non_blocking=True)
 
@@ -364,8 +377,8 @@ def run_ours(args):
                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
 
     cpu = None
-    # (raw inputs: the oracle would first need the input side; no CPU line then)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only != "decode" and not args.raw_inputs:
+    # (raw inputs or the output side: the timed oracle covers the plain path only; no CPU line then)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only != "decode" and not suffix:
         cpu = cpu_oracle_sample(w, host, args.cpu_seconds)
 
     if rank == 0:
@@ -373,7 +386,7 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded splitmix64 / Box-Muller)",
-            "config": {"workload": w.name + ("_raw_inputs" if args.raw_inputs else ""),
+            "config": {"workload": w.name + suffix,
                        "global_batch": w.num_seqs * world, "seq_len": w.seq_len,
                        "heads_qk_v": [w.hk, w.hv], "head_dim": w.d, "chunk": w.chunk,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",

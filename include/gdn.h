@@ -200,6 +200,63 @@ GDN_API gdn_status_t gdn_decode_step_ex(int32_t num_seqs, int32_t num_qk_heads, 
                                 const float *g, const float *beta,
                                 float *state, void *o, uint32_t flags, void *stream);
 
+/* The mixer's output side, applied to every (token, value head) output row
+ * o of d_v values before it is stored:
+ *
+ *     y_i = o_i / sqrt(mean_j(o_j^2) + eps) * s_i * act(z_i)
+ *
+ * RMS normalisation of the mixer output ahead of the output projection
+ * ("Architecture Thread I", "Modern Architecture Improvements"), with the
+ * gate of the gated RMSNorm ("The Transformer Isn't Alone Anymore", the
+ * model-reconstruction section; "Gated Attention Architectures", the
+ * Gated DeltaNet code listing, whose gate is SiLU of a projection; the
+ * same page's Gated Attention section for the sigmoid form) and the
+ * zero-centred scale 1 + delta of the Qwen3-Next passage of "Architecture
+ * Thread I".  The normalisation runs in fp32 on the unrounded output. */
+#define GDN_OUT_GATE_SILU 1u        /* act(z) = z * sigmoid(z)                 */
+#define GDN_OUT_GATE_SIGMOID 2u     /* act(z) = sigmoid(z)                     */
+#define GDN_OUT_ZERO_CENTRED 4u     /* s_i = 1 + w_i (else s_i = w_i)          */
+#define GDN_OUT_WEIGHT_PER_HEAD 8u  /* w is [Hv, d_v] (else [d_v], shared by
+                                       all value heads)                       */
+typedef struct {
+    const float *weight;  /* fp32 scale w, [d_v] or [Hv, d_v], 16-byte aligned;
+                             NULL reads as w = 1 (plain) or w = 0 (zero-
+                             centred), i.e. a unit scale either way          */
+    const void *gate;     /* z, [tokens, Hv, d_v] of the problem's dtype,
+                             16-byte aligned; NULL = no gate (then neither
+                             gate flag may be set; with a gate exactly one
+                             must be)                                        */
+    float eps;            /* added to the mean square; finite and > 0        */
+    uint32_t flags;       /* GDN_OUT_* bits; others are invalid              */
+} gdn_output_side_t;
+
+/* gdn_chunk_forward with the output side applied: `o` receives y instead of
+ * the raw read-out.  out_side = NULL is gdn_chunk_forward.  The tensor-core
+ * kernel applies it in its output epilogue (the gate tile arrives by TMA
+ * beside the chunk); the fp32 CUDA-core kernel, whose blocks each own a
+ * slice of d_v, stores o and then runs one more kernel over o in place.
+ * Invalid output-side arguments return GDN_ERR_INVALID_ARGUMENT or
+ * GDN_ERR_MISALIGNED before any launch. */
+GDN_API gdn_status_t gdn_chunk_forward_out(const gdn_shape_t *shape,
+                                   const void *q, const void *k, const void *v,
+                                   const float *g, const float *beta,
+                                   const float *initial_state,
+                                   const int32_t *cu_seqlens,
+                                   const gdn_output_side_t *out_side,
+                                   void *o, float *final_state,
+                                   void *workspace, size_t workspace_bytes,
+                                   void *stream);
+
+/* gdn_decode_step_ex with the output side applied inside the decode kernel
+ * (gate z: [N, Hv, d_v]).  out_side = NULL is gdn_decode_step_ex.  With an
+ * output side, d_v must be at most 256 (GDN_ERR_UNSUPPORTED otherwise). */
+GDN_API gdn_status_t gdn_decode_step_out(int32_t num_seqs, int32_t num_qk_heads, int32_t num_v_heads,
+                                 int32_t head_dim_k, int32_t head_dim_v, int32_t dtype,
+                                 const void *q, const void *k, const void *v,
+                                 const float *g, const float *beta,
+                                 float *state, const gdn_output_side_t *out_side,
+                                 void *o, uint32_t flags, void *stream);
+
 /* Static text for a status code. */
 GDN_API const char *gdn_status_string(gdn_status_t status);
 

@@ -68,6 +68,33 @@ static gdn_status_t check_shape(const gdn_shape_t *s) {
     return GDN_OK;
 }
 
+// Validates an output-side descriptor (NULL = none) and converts it for the
+// kernels.
+static gdn_status_t check_output_side(const gdn_output_side_t *os, OutSide *out) {
+    *out = OutSide{nullptr, nullptr, 0.f, 0u};
+    if (!os) return GDN_OK;
+    const uint32_t known = GDN_OUT_GATE_SILU | GDN_OUT_GATE_SIGMOID | GDN_OUT_ZERO_CENTRED | GDN_OUT_WEIGHT_PER_HEAD;
+    if (os->flags & ~known) return fail(GDN_ERR_INVALID_ARGUMENT, "unknown output-side flag bits 0x%x", os->flags);
+    const uint32_t gates = os->flags & (GDN_OUT_GATE_SILU | GDN_OUT_GATE_SIGMOID);
+    if (os->gate && gates != GDN_OUT_GATE_SILU && gates != GDN_OUT_GATE_SIGMOID)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "an output gate needs exactly one of GDN_OUT_GATE_SILU, "
+                                              "GDN_OUT_GATE_SIGMOID");
+    if (!os->gate && gates) return fail(GDN_ERR_INVALID_ARGUMENT, "a gate activation is set but gate is NULL");
+    if (!(os->eps > 0.f) || !(os->eps < 3.0e38f))
+        return fail(GDN_ERR_INVALID_ARGUMENT, "output-side eps must be finite and > 0");
+    if (os->gate && !aligned16(os->gate)) return fail(GDN_ERR_MISALIGNED, "output gate is not 16-byte aligned");
+    if (os->weight && !aligned16(os->weight))
+        return fail(GDN_ERR_MISALIGNED, "output-side weight is not 16-byte aligned");
+    *out = OutSide{os->weight, os->gate, os->eps, os->flags | kOutOn};
+    return GDN_OK;
+}
+
+static gdn_status_t chunk_forward_impl(const gdn_shape_t *s, const void *q, const void *k, const void *v,
+                                       const float *g, const float *beta, const float *initial_state,
+                                       const int32_t *cu_seqlens, const gdn_output_side_t *out_side, void *o,
+                                       float *final_state, void *workspace, size_t workspace_bytes,
+                                       void *stream_);
+
 }  // namespace gdn
 
 using namespace gdn;
@@ -104,8 +131,32 @@ gdn_status_t gdn_chunk_forward(const gdn_shape_t *s, const void *q, const void *
                                const float *g, const float *beta, const float *initial_state,
                                const int32_t *cu_seqlens, void *o, float *final_state, void *workspace,
                                size_t workspace_bytes, void *stream_) {
+    return chunk_forward_impl(s, q, k, v, g, beta, initial_state, cu_seqlens, nullptr, o, final_state, workspace,
+                              workspace_bytes, stream_);
+}
+
+gdn_status_t gdn_chunk_forward_out(const gdn_shape_t *s, const void *q, const void *k, const void *v,
+                                   const float *g, const float *beta, const float *initial_state,
+                                   const int32_t *cu_seqlens, const gdn_output_side_t *out_side, void *o,
+                                   float *final_state, void *workspace, size_t workspace_bytes, void *stream_) {
+    return chunk_forward_impl(s, q, k, v, g, beta, initial_state, cu_seqlens, out_side, o, final_state, workspace,
+                              workspace_bytes, stream_);
+}
+
+}  // extern "C"
+
+namespace gdn {
+
+static gdn_status_t chunk_forward_impl(const gdn_shape_t *s, const void *q, const void *k, const void *v,
+                                       const float *g, const float *beta, const float *initial_state,
+                                       const int32_t *cu_seqlens, const gdn_output_side_t *out_side, void *o,
+                                       float *final_state, void *workspace, size_t workspace_bytes,
+                                       void *stream_) {
     g_msg[0] = 0;
     gdn_status_t st = check_shape(s);
+    if (st != GDN_OK) return st;
+    OutSide out;
+    st = check_output_side(out_side, &out);
     if (st != GDN_OK) return st;
     const int64_t tokens = int64_t(s->batch) * s->seq_len;
     if (cu_seqlens) {
@@ -147,6 +198,7 @@ gdn_status_t gdn_chunk_forward(const gdn_shape_t *s, const void *q, const void *
     a.tokens = int32_t(tokens);
     a.flags = s->flags & (GDN_FLAG_QK_L2NORM | GDN_FLAG_GATE_LOGITS);
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.s0 = initial_state; a.o = o; a.s_final = final_state;
+    a.out = out;
     char *ws = static_cast<char *>(workspace);
     a.sched.hdr = reinterpret_cast<WsHeader *>(ws);
     a.sched.order = reinterpret_cast<const int32_t *>(ws + L.order_off);
@@ -157,8 +209,17 @@ gdn_status_t gdn_chunk_forward(const gdn_shape_t *s, const void *q, const void *
     const bool use_tc = major == 10 && !(s->flags & GDN_FLAG_FORCE_SIMT) && chunk_tc_supported(*s);
     e = use_tc ? launch_chunk_tc(a, stream, sms) : launch_chunk_simt(a, stream, sms);
     if (e != cudaSuccess) return cuda_fail(e, use_tc ? "tensor-core prefill launch" : "prefill launch");
+    // the tensor-core kernel applies the output side itself (with tokens to load)
+    if (out.flags && !(use_tc && tokens > 0)) {
+        e = launch_output_side(o, int32_t(tokens), s->num_v_heads, s->head_dim_v, s->dtype, out, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "output-side launch");
+    }
     return GDN_OK;
 }
+
+}  // namespace gdn
+
+extern "C" {
 
 gdn_status_t gdn_read_device_status(const void *workspace, int32_t *device_status, void *stream_) {
     g_msg[0] = 0;
@@ -183,7 +244,17 @@ gdn_status_t gdn_decode_step(int32_t n, int32_t hk, int32_t hv, int32_t dk, int3
 gdn_status_t gdn_decode_step_ex(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
                                 const void *q, const void *k, const void *v, const float *g, const float *beta,
                                 float *state, void *o, uint32_t flags, void *stream_) {
+    return gdn_decode_step_out(n, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, nullptr, o, flags, stream_);
+}
+
+gdn_status_t gdn_decode_step_out(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
+                                 const void *q, const void *k, const void *v, const float *g, const float *beta,
+                                 float *state, const gdn_output_side_t *out_side, void *o, uint32_t flags,
+                                 void *stream_) {
     g_msg[0] = 0;
+    OutSide out;
+    gdn_status_t st = check_output_side(out_side, &out);
+    if (st != GDN_OK) return st;
     if (flags & ~(GDN_FLAG_QK_L2NORM | GDN_FLAG_GATE_LOGITS))
         return fail(GDN_ERR_INVALID_ARGUMENT, "unknown decode flag bits 0x%x", flags);
     if (n < 0 || hk <= 0 || hv <= 0 || dk <= 0 || dv <= 0)
@@ -192,6 +263,8 @@ gdn_status_t gdn_decode_step_ex(int32_t n, int32_t hk, int32_t hv, int32_t dk, i
     if (dtype != GDN_DTYPE_F32 && dtype != GDN_DTYPE_BF16)
         return fail(GDN_ERR_INVALID_ARGUMENT, "dtype %d is not GDN_DTYPE_F32 or GDN_DTYPE_BF16", dtype);
     if (dk > 256) return fail(GDN_ERR_UNSUPPORTED, "decode supports d_k <= 256 (got %d)", dk);
+    if (out.flags && dv > 256)
+        return fail(GDN_ERR_UNSUPPORTED, "decode with an output side supports d_v <= 256 (got %d)", dv);
     if (n == 0) return GDN_OK;
     if (!q || !k || !v || !g || !beta || !state || !o)
         return fail(GDN_ERR_INVALID_ARGUMENT, "decode pointers must be non-NULL");
@@ -200,7 +273,7 @@ gdn_status_t gdn_decode_step_ex(int32_t n, int32_t hk, int32_t hv, int32_t dk, i
     for (int i = 0; i < 7; ++i)
         if (!aligned16(ptrs[i])) return fail(GDN_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
     if (int64_t(n) * hv * dv * dk > (int64_t(1) << 40)) return fail(GDN_ERR_UNSUPPORTED, "state too large");
-    cudaError_t e = launch_decode(n, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o, flags,
+    cudaError_t e = launch_decode(n, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o, flags, out,
                                   static_cast<cudaStream_t>(stream_));
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     return GDN_OK;

@@ -98,6 +98,14 @@ constexpr uint32_t kOffTpp = kOffTp + 8192;                               // T''
 constexpr uint32_t kOffBar = kOffTpp + 8192;          // mbarriers, tensor-memory slot, unit slot
 constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024; // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 per-block limit");
+// With the output side: the chunk's gate tile z (64 tokens x 128 bf16,
+// token-major, by TMA one chunk ahead) after the barriers.  The per-token
+// partial sums of squares use the chunk's P buffer, whose product has
+// completed by the output epilogue.
+constexpr uint32_t kOffZ = (kOffBar + 128 + 1023) / 1024 * 1024;
+constexpr uint32_t kBytesZ = 64 * 128 * 2;
+constexpr uint32_t kSmemBytesOut = kOffZ + kBytesZ + 1024;
+static_assert(kSmemBytesOut <= 232448, "shared memory over the sm_100 per-block limit");
 // per-token vectors inside a buffer (floats)
 constexpr int kVecG = 0, kVecB = 64, kVecGam = 128, kVecBG = 192, kVecLam = 256, kVecIGam = 320;
 // per-token scales through which GDN_FLAG_QK_L2NORM normalises the raw q and k
@@ -110,8 +118,10 @@ constexpr int kVecG = 0, kVecB = 64, kVecGam = 128, kVecBG = 192, kVecLam = 256,
 // is diag(gamma / ||q||) Q S^T + diag(1 / ||q||) (Q K^T (.) Gamma) U'.
 constexpr int kVecSa = 384, kVecSp = 448, kVecTpp = 512, kVecGo = 576;
 // mbarrier slots
-constexpr int kBarTKQ = 0, kBarTV = 2, kBarI = 3, kBarC = 4, kBarFull = 5, kBarEmpty = 7, kBarWT = 9, kNumBars = 10;
-// (kBarWT: "T' and T'' consumed", chain -> intra)
+constexpr int kBarTKQ = 0, kBarTV = 2, kBarI = 3, kBarC = 4, kBarFull = 5, kBarEmpty = 7, kBarWT = 9, kBarZ = 10,
+              kNumBars = 11;
+// (kBarWT: "T' and T'' consumed", chain -> intra; kBarZ: gate tile landed)
+static_assert(8 * kNumBars + 8 <= 128, "barrier slots overflow their region");
 
 // Tensor-memory columns (128 lanes each): fp32 accumulators, and bf16 A
 // operands packed two elements per column: the copy of S for (4) and (5), and
@@ -307,14 +317,41 @@ __device__ __forceinline__ void load_v(uint32_t dst, uint32_t bar, const CUtenso
     tma_load_3d(dst + 8192, tv, 64, h, c0, bar);
 }
 
-// kL2: GDN_FLAG_QK_L2NORM; kLogits: GDN_FLAG_GATE_LOGITS (compile-time, so the
-// plain path carries none of the input-side work)
-template <bool kL2, bool kLogits>
+// The output side's gate tile of chunk c0, value head h (rows past the last
+// token read as zeros).
+__device__ __forceinline__ void load_z(uint32_t dst, uint32_t bar, const CUtensorMap *tz, int h, int c0) {
+    mbar_arrive_expect_tx(bar, kBytesZ);
+    tma_load_3d(dst, tz, 0, h, c0, bar);
+}
+
+// Column sums over a warp of 16 values per lane, transposed: afterwards lanes
+// 2t and 2t + 1 return the sum over all 32 lanes of x[t] (t = 0..15).  Four
+// halving exchanges (each lane keeps the half of its values selected by its
+// lane bit and adds its partner's copy of that half) and a final pairwise
+// add: 16 shuffles instead of the 80 of 16 separate reductions.
+__device__ __forceinline__ float warp_colsum16(float (&x)[16], int lane) {
+#pragma unroll
+    for (int n = 8, bit = 16; n >= 1; n >>= 1, bit >>= 1) {
+        const bool up = (lane & bit) != 0;
+#pragma unroll
+        for (int m = 0; m < n; ++m) {
+            const float send = up ? x[m] : x[m + n];
+            const float keep = up ? x[m + n] : x[m];
+            x[m] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+        }
+    }
+    return x[0] + __shfl_xor_sync(0xffffffffu, x[0], 1);
+}
+
+// kL2: GDN_FLAG_QK_L2NORM; kLogits: GDN_FLAG_GATE_LOGITS; kOut: the output
+// side in the output epilogue (compile-time, so the plain path carries none
+// of the input- or output-side work)
+template <bool kL2, bool kLogits, bool kOut>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                 const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_b,
-                const PrefillArgs a) {
+                const __grid_constant__ CUtensorMap tm_z, const PrefillArgs a) {
     extern __shared__ unsigned char smem_raw[];
     // Align to 1024 bytes with a byte offset on the shared array itself (not
     // through an integer cast), so that the compiler keeps every access below in
@@ -369,7 +406,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int total_units = a.num_seqs * hv;
     __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(a.o);
     uint32_t gn = 0;  // chunks this CTA has processed so far (selects buffers and barrier phases)
-    uint32_t ph_full = 0, ph_empty = 0, ph_tkq = 0, ph_v = 0, ph_i = 0, ph_c = 0, ph_wt = 0;
+    uint32_t ph_full = 0, ph_empty = 0, ph_tkq = 0, ph_v = 0, ph_i = 0, ph_c = 0, ph_wt = 0, ph_z = 0;
     bool aborted = false;
 
     const uint32_t id_gram = idesc_bf16(128, 64, false, false);
@@ -396,12 +433,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 load_kq(sb + (((gn + 1) & 1) ? kOffKQ1 : kOffKQ0), bars + 8 * (kBarTKQ + ((gn + 1) & 1)), &tm_k,
                         &tm_q, hq, t0 + 64, sb + kOffGst + ((gn + 1) & 1) * 2048, &tm_g, &tm_b, h);
             load_v(sb + kOffV, bars + 8 * kBarTV, &tm_v, h, t0);
+            if (kOut && a.out.z) load_z(sb + kOffZ, bars + 8 * kBarZ, &tm_z, h, t0);
         }
 
         if (is_chain) {
             // ============ chain group: thread = (state row, half of the columns) ============
             const int row = (warp & 3) * 32 + lane;
             const int ch = warp >> 2;
+            // output side: this thread's channel scale, and whether a gate tile comes
+            const float out_s = kOut ? out_scale(a.out, h, row, 128) : 0.f;
+            const bool zgate = kOut && a.out.z != nullptr;
             // initial state into tensor memory
 #pragma unroll
             for (int c4 = 2 * ch; c4 < 2 * ch + 2; ++c4) {
@@ -563,7 +604,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 // staged token-major (rows of 256 bytes); a full chunk leaves in one
                 // TMA store, a ragged last chunk row by row.  X1' is zeroed for the
                 // next chunk's merged product.
-                {
+                if constexpr (!kOut) {
                     __nv_bfloat16 *Ot = reinterpret_cast<__nv_bfloat16 *>(smem + kOffOst);
                     uint32_t z[16];
 #pragma unroll
@@ -584,9 +625,74 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                     tmem_wait_st();
                 }
+                else {
+                    // output side: y = O / sqrt(mean_i O[r][i]^2 + eps) * s_i * act(z[r][i]).
+                    // Pass 1 leaves O (fp32) in X2's columns, zeroes X1', and per token
+                    // sums O^2 over this warp's 32 value rows into the consumed P buffer.
+                    __nv_bfloat16 *Ot = reinterpret_cast<__nv_bfloat16 *>(smem + kOffOst);
+                    float *red = reinterpret_cast<float *>(smem + (b ? kOffP1 : kOffP0));
+                    const int quad = warp & 3;
+                    uint32_t zr[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) zr[j] = 0u;
+#pragma unroll
+                    for (int sl = 0; sl < 2; ++sl) {
+                        const int r0 = 32 * ch + 16 * sl;
+                        float x1[16], x2[16], gm[16];
+                        tmem_ld16(tmem + lane_bits + kColX1 + r0, x1);
+                        tmem_ld16(tmem + lane_bits + kColX2 + r0, x2);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) load4(vec + (kL2 ? kVecGo : kVecGam) + r0 + 4 * q, gm + 4 * q);
+                        tmem_wait_ld();
+                        tmem_st16u(tmem + lane_bits + kColX1 + r0, zr);
+                        uint32_t ob[16];
+                        float sq[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float ov = fmaf(-gm[j], x1[j], x2[j]);
+                            ob[j] = __float_as_uint(ov);
+                            sq[j] = ov * ov;
+                        }
+                        tmem_st16u(tmem + lane_bits + kColX2 + r0, ob);
+                        const float part = warp_colsum16(sq, lane);
+                        if ((lane & 1) == 0) red[(r0 + (lane >> 1)) * 4 + quad] = part;
+                    }
+                    tmem_wait_st();
+                    {
+                        bool ok = true;
+                        if (zgate) {
+                            ok = mbar_wait(bars + 8 * kBarZ, ph_z);
+                            ph_z ^= 1u;
+                        }
+                        if (named_sync_or(kBarChain, kChain, !ok)) { aborted = true; break; }
+                    }
+                    // pass 2: scale, gate and stage for the store
+                    const __nv_bfloat16 *Zt = reinterpret_cast<const __nv_bfloat16 *>(smem + kOffZ);
+                    const float eps = a.out.eps;
+                    const uint32_t oflags = a.out.flags;
+#pragma unroll
+                    for (int sl = 0; sl < 2; ++sl) {
+                        const int r0 = 32 * ch + 16 * sl;
+                        float ov[16];
+                        tmem_ld16(tmem + lane_bits + kColX2 + r0, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int r = r0 + j;
+                            const float4 pr = *reinterpret_cast<const float4 *>(red + 4 * r);
+                            const float ms = ((pr.x + pr.y) + (pr.z + pr.w)) * (1.f / 128.f);
+                            float y = ov[j] * out_s * rsqrtf(ms + eps);
+                            if (zgate) y *= out_gate_fast(oflags, __bfloat162float(Zt[r * 128 + row]));
+                            Ot[r * 128 + row] = __float2bfloat16_rn(y);
+                        }
+                    }
+                }
                 fence_proxy_async_shared();
                 tc_fence_before();
                 named_sync(kBarChain, kChain);
+                // the gate tile is read: the next chunk's may come in
+                if (kOut && zgate && tid == 0 && n + 1 < nchunks)
+                    load_z(sb + kOffZ, bars + 8 * kBarZ, &tm_z, h, c0 + 64);
                 if (L == 64) {
                     if (tid == 0) {
                         tma_store_3d(&tm_o, sb + kOffOst, 0, h, c0);
@@ -880,15 +986,26 @@ cudaError_t launch_chunk_tc(const PrefillArgs &a, cudaStream_t stream, int num_s
     // With no tokens at all there is nothing to load; the fp32 kernel writes
     // the final states (= initial states) of the empty sequences.
     if (a.tokens <= 0) return launch_chunk_simt(a, stream, num_sms);
-    CUtensorMap mq, mk, mv, mo, mg, mb;
+    CUtensorMap mq, mk, mv, mo, mg, mb, mz;
     if (!make_map(&mq, a.q, a.hk, a.tokens) || !make_map(&mk, a.k, a.hk, a.tokens) ||
         !make_map(&mv, a.v, a.hv, a.tokens) || !make_map(&mo, a.o, a.hv, a.tokens, true) ||
         !make_gate_map(&mg, a.g, a.hv, a.tokens) || !make_gate_map(&mb, a.beta, a.hv, a.tokens))
         return cudaErrorInvalidValue;
+    mz = mo;  // not read unless the output side has a gate
+    if (a.out.flags && a.out.z && !make_map(&mz, a.out.z, a.hv, a.tokens, true)) return cudaErrorInvalidValue;
     const bool l2 = a.flags & GDN_FLAG_QK_L2NORM, logits = a.flags & GDN_FLAG_GATE_LOGITS;
-    auto *kern = l2 ? (logits ? chunk_tc_kernel<true, true> : chunk_tc_kernel<true, false>)
-                    : (logits ? chunk_tc_kernel<false, true> : chunk_tc_kernel<false, false>);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+    const bool out = a.out.flags != 0;
+    using KernFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
+                            PrefillArgs);
+    static const KernFn table[8] = {
+        chunk_tc_kernel<false, false, false>, chunk_tc_kernel<false, true, false>,
+        chunk_tc_kernel<true, false, false>,  chunk_tc_kernel<true, true, false>,
+        chunk_tc_kernel<false, false, true>,  chunk_tc_kernel<false, true, true>,
+        chunk_tc_kernel<true, false, true>,   chunk_tc_kernel<true, true, true>,
+    };
+    const KernFn kern = table[(out ? 4 : 0) + (l2 ? 2 : 0) + (logits ? 1 : 0)];
+    const uint32_t smem_bytes = out ? kSmemBytesOut : kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_bytes));
     if (e != cudaSuccess) return e;
     const int64_t units = int64_t(a.num_seqs) * a.hv;
     const int grid = int(units < num_sms ? units : num_sms);
@@ -898,14 +1015,14 @@ cudaError_t launch_chunk_tc(const PrefillArgs &a, cudaStream_t stream, int num_s
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(grid));
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.dynamicSmemBytes = smem_bytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, mg, mb, a);
+    e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, mg, mb, mz, a);
     count_launch();
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

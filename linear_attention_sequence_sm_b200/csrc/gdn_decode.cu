@@ -27,6 +27,11 @@ namespace gdn {
 #endif
 constexpr int kDecodeWarps = 4;     // warps per block; a block owns one (sequence, head)
 constexpr int kRowBatch = GDN_DECODE_ROWS;  // rows in flight per warp
+// Template bit (beside the GDN_FLAG_* input-side bits): the output side is
+// applied in the kernel.  The rows of o then wait in shared memory until the
+// whole vector is known, for its root mean square.
+constexpr uint32_t kDecOut = 1u << 8;
+constexpr int kDecOutMaxDv = 256;
 
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
@@ -53,8 +58,10 @@ template <typename T, uint32_t flags>
 __global__ void __launch_bounds__(kDecodeWarps * 32, GDN_DECODE_MINBLOCKS)
 decode_d128_kernel(int32_t hk, int32_t hv, int32_t dv, const T *__restrict__ q, const T *__restrict__ k,
                    const T *__restrict__ v, const float *__restrict__ g, const float *__restrict__ beta,
-                   float *__restrict__ state, T *__restrict__ o) {
+                   float *__restrict__ state, T *__restrict__ o, const OutSide os) {
     constexpr int dk = 128;
+    constexpr bool kOut = (flags & kDecOut) != 0;
+    __shared__ float ob[kOut ? kDecOutMaxDv : 1], red[kDecodeWarps];
     const int unit = blockIdx.x;            // sequence * hv + head
     const int n = unit / hv, h = unit % hv;
     const int hq = h / (hv / hk);
@@ -117,8 +124,35 @@ decode_d128_kernel(int32_t hk, int32_t hv, int32_t dv, const T *__restrict__ q, 
             sn.z = fmaf(alpha, s[r].z, u * kf[2]);
             sn.w = fmaf(alpha, s[r].w, u * kf[3]);
             store4(S + size_t(i0 + r) * dk + 4 * lane, sn);
-            if (lane == r) orow[i0 + r] = from_f32<T>(fmaf(alpha, rq[r], u * kq));
+            if (lane == r) {
+                const float ov = fmaf(alpha, rq[r], u * kq);
+                if constexpr (kOut) ob[i0 + r] = ov;
+                else orow[i0 + r] = from_f32<T>(ov);
+            }
         }
+    }
+    if constexpr (kOut) decode_output_side(ob, red, dv, unit, h, os, orow);
+}
+
+// Output side over the block's d_v outputs in shared memory (kDecOut).
+template <typename T>
+__device__ __forceinline__ void decode_output_side(const float *ob, float *red, int dv, int unit, int h,
+                                                   const OutSide &os, T *orow) {
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float ss = 0.f;
+    for (int i = threadIdx.x; i < dv; i += kDecodeWarps * 32) ss = fmaf(ob[i], ob[i], ss);
+    ss = warp_sum(ss);
+    if (lane == 0) red[warp] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDecodeWarps; ++w) tot += red[w];
+    const float inv_rms = rsqrtf(tot / float(dv) + os.eps);
+    const T *z = os.z ? static_cast<const T *>(os.z) + size_t(unit) * dv : nullptr;
+    for (int i = threadIdx.x; i < dv; i += kDecodeWarps * 32) {
+        const float gz = z ? out_gate(os.flags, to_f32(z[i])) : 1.f;
+        orow[i] = from_f32<T>(ob[i] * inv_rms * out_scale(os, h, i, dv) * gz);
     }
 }
 
@@ -127,8 +161,11 @@ template <typename T, uint32_t flags>
 __global__ void __launch_bounds__(kDecodeWarps * 32)
 decode_generic_kernel(int32_t hk, int32_t hv, int32_t dk, int32_t dv, const T *__restrict__ q,
                       const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ g,
-                      const float *__restrict__ beta, float *__restrict__ state, T *__restrict__ o) {
+                      const float *__restrict__ beta, float *__restrict__ state, T *__restrict__ o,
+                      const OutSide os) {
     constexpr int kMaxPer = 8;  // 8 * 32 = 256 elements
+    constexpr bool kOut = (flags & kDecOut) != 0;
+    __shared__ float ob[kOut ? kDecOutMaxDv : 1], red[kDecodeWarps];
     const int unit = blockIdx.x;
     const int n = unit / hv, h = unit % hv;
     const int hq = h / (hv / hk);
@@ -177,57 +214,65 @@ decode_generic_kernel(int32_t hk, int32_t hv, int32_t dk, int32_t dv, const T *_
             const int j = lane + 32 * e;
             if (j < dk) S[size_t(i) * dk + j] = fmaf(alpha, s[e], u * kf[e]);
         }
-        if (lane == 0) o[size_t(unit) * dv + i] = from_f32<T>(fmaf(alpha, rq, u * kq));
+        if (lane == 0) {
+            const float ov = fmaf(alpha, rq, u * kq);
+            if constexpr (kOut) ob[i] = ov;
+            else o[size_t(unit) * dv + i] = from_f32<T>(ov);
+        }
     }
+    if constexpr (kOut) decode_output_side(ob, red, dv, unit, h, os, o + size_t(unit) * dv);
 }
 
 template <uint32_t F>
 static void launch_decode_as(dim3 grid, dim3 block, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
                              const void *q, const void *k, const void *v, const float *g, const float *beta,
-                             float *state, void *o, cudaStream_t stream) {
+                             float *state, void *o, const OutSide &os, cudaStream_t stream) {
     using bf = __nv_bfloat16;
     if (dk == 128) {
         if (dtype == GDN_DTYPE_BF16)
             decode_d128_kernel<bf, F><<<grid, block, 0, stream>>>(
                 hk, hv, dv, static_cast<const bf *>(q), static_cast<const bf *>(k), static_cast<const bf *>(v), g,
-                beta, state, static_cast<bf *>(o));
+                beta, state, static_cast<bf *>(o), os);
         else
             decode_d128_kernel<float, F><<<grid, block, 0, stream>>>(
                 hk, hv, dv, static_cast<const float *>(q), static_cast<const float *>(k),
-                static_cast<const float *>(v), g, beta, state, static_cast<float *>(o));
+                static_cast<const float *>(v), g, beta, state, static_cast<float *>(o), os);
     } else {
         if (dtype == GDN_DTYPE_BF16)
             decode_generic_kernel<bf, F><<<grid, block, 0, stream>>>(
                 hk, hv, dk, dv, static_cast<const bf *>(q), static_cast<const bf *>(k), static_cast<const bf *>(v),
-                g, beta, state, static_cast<bf *>(o));
+                g, beta, state, static_cast<bf *>(o), os);
         else
             decode_generic_kernel<float, F><<<grid, block, 0, stream>>>(
                 hk, hv, dk, dv, static_cast<const float *>(q), static_cast<const float *>(k),
-                static_cast<const float *>(v), g, beta, state, static_cast<float *>(o));
+                static_cast<const float *>(v), g, beta, state, static_cast<float *>(o), os);
     }
 }
 
 cudaError_t launch_decode(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
                           const void *q, const void *k, const void *v, const float *g, const float *beta,
-                          float *state, void *o, uint32_t flags, cudaStream_t stream) {
+                          float *state, void *o, uint32_t flags, const OutSide &os, cudaStream_t stream) {
     const int64_t units = int64_t(n) * hv;
     if (units > INT32_MAX) return cudaErrorInvalidValue;
+    if (os.flags && dv > kDecOutMaxDv) return cudaErrorInvalidValue;
     const dim3 grid(static_cast<unsigned>(units)), block(kDecodeWarps * 32);
-    switch (flags) {
-        case 0: launch_decode_as<0>(grid, block, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o, stream); break;
-        case GDN_FLAG_QK_L2NORM:
-            launch_decode_as<GDN_FLAG_QK_L2NORM>(grid, block, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o,
-                                                 stream);
-            break;
-        case GDN_FLAG_GATE_LOGITS:
-            launch_decode_as<GDN_FLAG_GATE_LOGITS>(grid, block, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o,
-                                                   stream);
-            break;
-        default:
-            launch_decode_as<GDN_FLAG_QK_L2NORM | GDN_FLAG_GATE_LOGITS>(grid, block, hk, hv, dk, dv, dtype, q, k,
-                                                                       v, g, beta, state, o, stream);
-            break;
+    constexpr uint32_t L2 = GDN_FLAG_QK_L2NORM, LG = GDN_FLAG_GATE_LOGITS;
+    const uint32_t f = (flags & (L2 | LG)) | (os.flags ? kDecOut : 0u);
+#define GDN_DECODE_CASE(F)                                                                                  \
+    case F: launch_decode_as<F>(grid, block, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o, os, stream); \
+        break;
+    switch (f) {
+        GDN_DECODE_CASE(0u)
+        GDN_DECODE_CASE(L2)
+        GDN_DECODE_CASE(LG)
+        GDN_DECODE_CASE(L2 | LG)
+        GDN_DECODE_CASE(kDecOut)
+        GDN_DECODE_CASE(kDecOut | L2)
+        GDN_DECODE_CASE(kDecOut | LG)
+        GDN_DECODE_CASE(kDecOut | L2 | LG)
+        default: return cudaErrorInvalidValue;
     }
+#undef GDN_DECODE_CASE
     count_launch();
     return cudaGetLastError();
 }

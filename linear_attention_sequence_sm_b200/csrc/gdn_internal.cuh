@@ -91,6 +91,37 @@ void count_launch();
 cudaError_t launch_schedule(const gdn_shape_t &s, const int32_t *cu_seqlens, void *workspace,
                             cudaStream_t stream);
 
+// The output side as the kernels see it (gdn_output_side_t plus an enable
+// bit): y = o / sqrt(mean(o^2) + eps) * s * act(z).
+constexpr uint32_t kOutOn = 1u << 31;
+struct OutSide {
+    const float *w;   // scale, or NULL
+    const void *z;    // gate, or NULL
+    float eps;
+    uint32_t flags;   // GDN_OUT_* | kOutOn; 0 = no output side
+};
+
+// The scale s_i of row channel i of value head h.
+__device__ __forceinline__ float out_scale(const OutSide &os, int h, int i, int dv) {
+    const float w = os.w ? os.w[((os.flags & GDN_OUT_WEIGHT_PER_HEAD) ? size_t(h) * dv : 0) + i]
+                         : ((os.flags & GDN_OUT_ZERO_CENTRED) ? 0.f : 1.f);
+    return (os.flags & GDN_OUT_ZERO_CENTRED) ? 1.f + w : w;
+}
+
+// act(z) for the gate kinds (1 without a gate).
+__device__ __forceinline__ float out_gate(uint32_t flags, float z) {
+    if (flags & GDN_OUT_GATE_SILU) return z * sigmoid(z);
+    if (flags & GDN_OUT_GATE_SIGMOID) return sigmoid(z);
+    return 1.f;
+}
+
+// The same with the fast sigmoid (bf16 outputs).
+__device__ __forceinline__ float out_gate_fast(uint32_t flags, float z) {
+    if (flags & GDN_OUT_GATE_SILU) return z * sigmoid_fast(z);
+    if (flags & GDN_OUT_GATE_SIGMOID) return sigmoid_fast(z);
+    return 1.f;
+}
+
 struct PrefillArgs {
     int32_t num_seqs, hk, hv, dk, dv, chunk, dtype;
     int32_t tokens;  // rows of q, k, v, o (B * T, or the packed total)
@@ -100,6 +131,7 @@ struct PrefillArgs {
     void *o;
     float *s_final;
     Sched sched;
+    OutSide out;     // output side (flags 0: none)
 };
 
 // fp32 CUDA-core chunkwise kernel (any dtype, d_k, d_v <= 128, C in {16,32,64}).
@@ -109,9 +141,14 @@ cudaError_t launch_chunk_simt(const PrefillArgs &a, cudaStream_t stream, int num
 cudaError_t launch_chunk_tc(const PrefillArgs &a, cudaStream_t stream, int num_sms);
 bool chunk_tc_supported(const gdn_shape_t &s);
 
+// The output side as its own pass over o, in place (for the CUDA-core prefill,
+// whose blocks each own a slice of d_v).
+cudaError_t launch_output_side(void *o, int32_t tokens, int32_t hv, int32_t dv, int32_t dtype, const OutSide &os,
+                               cudaStream_t stream);
+
 // Decode step.
 cudaError_t launch_decode(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
                           const void *q, const void *k, const void *v, const float *g, const float *beta,
-                          float *state, void *o, uint32_t flags, cudaStream_t stream);
+                          float *state, void *o, uint32_t flags, const OutSide &os, cudaStream_t stream);
 
 }  // namespace gdn

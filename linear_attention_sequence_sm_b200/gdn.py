@@ -32,10 +32,14 @@ GDN_DTYPE_BF16 = 1
 GDN_FLAG_FORCE_SIMT = 1
 GDN_FLAG_QK_L2NORM = 2
 GDN_FLAG_GATE_LOGITS = 4
+GDN_OUT_GATE_SILU = 1
+GDN_OUT_GATE_SIGMOID = 2
+GDN_OUT_ZERO_CENTRED = 4
+GDN_OUT_WEIGHT_PER_HEAD = 8
 
 EXPORTED = ("gdn_chunk_forward_workspace_size", "gdn_chunk_forward", "gdn_read_device_status",
             "gdn_decode_step", "gdn_status_string", "gdn_last_error_message", "gdn_launch_count",
-            "gdn_chunk_forward_noalloc", "gdn_decode_step_ex")
+            "gdn_chunk_forward_noalloc", "gdn_decode_step_ex", "gdn_chunk_forward_out", "gdn_decode_step_out")
 
 
 class GdnError(RuntimeError):
@@ -49,6 +53,11 @@ class Shape(ctypes.Structure):
                 ("num_qk_heads", ctypes.c_int32), ("num_v_heads", ctypes.c_int32),
                 ("head_dim_k", ctypes.c_int32), ("head_dim_v", ctypes.c_int32),
                 ("chunk_size", ctypes.c_int32), ("dtype", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+
+
+class OutputSideC(ctypes.Structure):
+    _fields_ = [("weight", ctypes.c_void_p), ("gate", ctypes.c_void_p), ("eps", ctypes.c_float),
+                ("flags", ctypes.c_uint32)]
 
 
 def _load(path: str = LIB_PATH):
@@ -70,6 +79,13 @@ def _load(path: str = LIB_PATH):
     lib.gdn_decode_step.restype = st
     lib.gdn_decode_step_ex.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, ctypes.c_uint32, vp]
     lib.gdn_decode_step_ex.restype = st
+    osp = ctypes.POINTER(OutputSideC)
+    lib.gdn_chunk_forward_out.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp, vp, osp, vp, vp, vp,
+                                          ctypes.c_size_t, vp]
+    lib.gdn_chunk_forward_out.restype = st
+    lib.gdn_decode_step_out.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, osp, vp,
+                                        ctypes.c_uint32, vp]
+    lib.gdn_decode_step_out.restype = st
     lib.gdn_status_string.argtypes = [st]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_last_error_message.argtypes = []
@@ -124,6 +140,41 @@ def input_flags(qk_l2norm=False, gate_logits=False) -> int:
     return (GDN_FLAG_QK_L2NORM if qk_l2norm else 0) | (GDN_FLAG_GATE_LOGITS if gate_logits else 0)
 
 
+class OutputNorm:
+    """The mixer's output side, applied in the kernels to every (token, value
+    head) output row o: y = o / sqrt(mean(o^2) + eps) * s * act(gate).
+
+    weight        fp32 [d_v] (shared by the value heads) or [Hv, d_v], or None
+                  for a unit scale; with ``zero_centred`` the scale is
+                  1 + weight.
+    gate          the gate pre-activation z, shaped and typed like o, or None.
+    activation    "silu" (z * sigmoid(z)) or "sigmoid" (used with a gate).
+    """
+
+    def __init__(self, weight=None, gate=None, eps=1e-6, activation="silu", zero_centred=False):
+        if activation not in ("silu", "sigmoid"):
+            raise ValueError(f"activation must be 'silu' or 'sigmoid', got {activation!r}")
+        self.weight, self.gate, self.eps = weight, gate, float(eps)
+        self.activation, self.zero_centred = activation, bool(zero_centred)
+
+    def c_struct(self, o: torch.Tensor) -> OutputSideC:
+        hv, dv = o.shape[-2], o.shape[-1]
+        flags = GDN_OUT_ZERO_CENTRED if self.zero_centred else 0
+        if self.weight is not None:
+            _need(self.weight, "output weight", torch.float32, o.device)
+            if tuple(self.weight.shape) == (hv, dv):
+                flags |= GDN_OUT_WEIGHT_PER_HEAD
+            elif tuple(self.weight.shape) != (dv,):
+                raise ValueError(f"output weight must be [{dv}] or [{hv}, {dv}], got {tuple(self.weight.shape)}")
+        if self.gate is not None:
+            _need(self.gate, "output gate", o.dtype, o.device)
+            if self.gate.shape != o.shape:
+                raise ValueError(f"output gate must have o's shape {tuple(o.shape)}, got {tuple(self.gate.shape)}")
+            flags |= GDN_OUT_GATE_SILU if self.activation == "silu" else GDN_OUT_GATE_SIGMOID
+        return OutputSideC(None if self.weight is None else self.weight.data_ptr(),
+                           None if self.gate is None else self.gate.data_ptr(), self.eps, flags)
+
+
 def make_shape(q, v, cu_seqlens=None, chunk_size=64, force_simt=False, flags=0) -> Shape:
     if cu_seqlens is not None:
         T = q.shape[-3]
@@ -145,11 +196,12 @@ def workspace_size(shape: Shape) -> int:
 
 def chunk_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_size=64,
                   output_final_state=True, out=None, final_state=None, workspace=None, force_simt=False,
-                  stream=None, qk_l2norm=False, gate_logits=False):
+                  stream=None, qk_l2norm=False, gate_logits=False, output_norm: OutputNorm | None = None):
     """Chunkwise prefill.  Returns (o, final_state or None).  Asynchronous on
     ``stream`` (default: the current stream).  ``qk_l2norm``: q and k are raw
     and normalised per head in the kernel; ``gate_logits``: g and beta are
-    the decay and write logits (alpha = sigmoid(g), beta = sigmoid(beta))."""
+    the decay and write logits (alpha = sigmoid(g), beta = sigmoid(beta));
+    ``output_norm``: the output side applied before o is stored."""
     dev = q.device
     dt = q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -171,6 +223,13 @@ def chunk_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_s
     nbytes = workspace_size(shape)
     if workspace is None or workspace.numel() < nbytes:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    if output_norm is not None:
+        osc = output_norm.c_struct(out)
+        _check(LIB.gdn_chunk_forward_out(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                         _ptr(initial_state), _ptr(cu_seqlens), ctypes.byref(osc), _ptr(out),
+                                         _ptr(final_state), _ptr(workspace), workspace.numel(),
+                                         _stream_handle(stream)))
+        return out, final_state
     _check(LIB.gdn_chunk_forward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
                                  _ptr(initial_state), _ptr(cu_seqlens), _ptr(out), _ptr(final_state),
                                  _ptr(workspace), workspace.numel(), _stream_handle(stream)))
@@ -215,10 +274,11 @@ def read_device_status(workspace, stream=None) -> int:
     return st.value
 
 
-def decode_step(q, k, v, g, beta, state, out=None, stream=None, qk_l2norm=False, gate_logits=False):
+def decode_step(q, k, v, g, beta, state, out=None, stream=None, qk_l2norm=False, gate_logits=False,
+                output_norm: OutputNorm | None = None):
     """One token per sequence; ``state`` [N, Hv, d_v, d_k] fp32 is updated in
-    place.  Returns o [N, Hv, d_v].  ``qk_l2norm`` and ``gate_logits`` as for
-    chunk_forward."""
+    place.  Returns o [N, Hv, d_v].  ``qk_l2norm``, ``gate_logits`` and
+    ``output_norm`` (gate [N, Hv, d_v]) as for chunk_forward."""
     dev, dt = q.device, q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, dt, dev)
@@ -230,6 +290,12 @@ def decode_step(q, k, v, g, beta, state, out=None, stream=None, qk_l2norm=False,
     _need(out, "out", dt, dev)
     N, hk, dk = q.shape
     hv, dv = v.shape[1], v.shape[2]
+    if output_norm is not None:
+        osc = output_norm.c_struct(out)
+        _check(LIB.gdn_decode_step_out(N, hk, hv, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                       _ptr(beta), _ptr(state), ctypes.byref(osc), _ptr(out),
+                                       input_flags(qk_l2norm, gate_logits), _stream_handle(stream)))
+        return out
     _check(LIB.gdn_decode_step_ex(N, hk, hv, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
                                   _ptr(beta), _ptr(state), _ptr(out), input_flags(qk_l2norm, gate_logits),
                                   _stream_handle(stream)))

@@ -239,6 +239,22 @@ def make_raw_prefill_inputs(w: Workload):
     return base
 
 
+def make_output_gate(w: Workload):
+    """The output side's gate pre-activation z, shaped like o: N(0, 2^2)
+    (SiLU then spans its negative dip and its near-identity range), rounded
+    once to the storage dtype."""
+    import torch
+    B, T, hv, d = w.batch, w.seq_len, w.hv, w.d
+    return _slabbed(w.seed, "out_gate", (B, T, hv, d), lambda z: 2.0 * z, _torch_dtype(w.dtype), d)
+
+
+def make_output_weight(w: Workload):
+    """The output side's per-channel scale, shared by the value heads:
+    N(1, 0.1^2) fp32 (a trained RMSNorm scale stays near 1)."""
+    import torch
+    return torch.from_numpy(normal(w.seed, "out_weight", (w.d,), mean=1.0, std=0.1)).to(torch.float32)
+
+
 def make_decode_inputs(w: DecodeWorkload, step: int):
     """Fresh per-step q, k [N,Hk,d], v [N,Hv,d], g, beta [N,Hv] (seed + step)."""
     import torch

@@ -131,3 +131,50 @@ def test_product_path_has_no_oracle_or_cpu_fallback():
             if fn.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, fn)).read()
                 assert not re.search(r"(from|import)\s+oracle|gdn_oracle|libgdn_oracle", text), fn
+
+
+def _call_out(gdn, shape, osc, **over):
+    p = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, o=FAKE, ws=FAKE, wsb=1 << 20)
+    p.update(over)
+    vp = ctypes.c_void_p
+    return gdn.LIB.gdn_chunk_forward_out(ctypes.byref(shape), vp(p["q"]), vp(p["k"]), vp(p["v"]), vp(p["g"]),
+                                         vp(p["beta"]), None, None, None if osc is None else ctypes.byref(osc),
+                                         vp(p["o"]), None, vp(p["ws"]), p["wsb"], None)
+
+
+@pytest.mark.parametrize("weight,gate,eps,flags,code", [
+    (None, FAKE, 1e-6, 0, 1),            # a gate without an activation
+    (None, FAKE, 1e-6, 1 | 2, 1),        # two activations
+    (None, None, 1e-6, 1, 1),            # an activation without a gate
+    (None, None, 0.0, 0, 1),             # eps must be > 0
+    (None, None, float("nan"), 0, 1),    # and finite
+    (None, None, float("inf"), 0, 1),
+    (None, None, 1e-6, 16, 1),           # unknown bit
+    (None, FAKE + 8, 1e-6, 1, 3),        # misaligned gate
+    (FAKE + 4, None, 1e-6, 0, 3),        # misaligned weight
+])
+def test_output_side_rejected(gdn, weight, gate, eps, flags, code):
+    osc = gdn.OutputSideC(weight, gate, eps, flags)
+    assert _call_out(gdn, _shape(gdn), osc) == code
+    assert gdn.LIB.gdn_last_error_message().decode() != ""
+    vp = ctypes.c_void_p
+    st = gdn.LIB.gdn_decode_step_out(4, 2, 4, 128, 128, 1, *([vp(FAKE)] * 6), ctypes.byref(osc), vp(FAKE), 0, None)
+    assert st == code
+
+
+def test_output_side_decode_dv_limit(gdn):
+    vp = ctypes.c_void_p
+    osc = gdn.OutputSideC(None, None, 1e-6, 0)
+    st = gdn.LIB.gdn_decode_step_out(4, 2, 4, 128, 512, 1, *([vp(FAKE)] * 6), ctypes.byref(osc), vp(FAKE), 0, None)
+    assert st == gdn.GDN_ERR_UNSUPPORTED
+
+
+def test_output_side_valid_reaches_the_device_check(gdn):
+    """A valid descriptor passes validation (no GPU here: the call then fails
+    on the device query, GDN_ERR_CUDA); NULL means no output side."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("only meaningful without a GPU")
+    osc = gdn.OutputSideC(FAKE, FAKE, 1e-6, 1 | 4 | 8)
+    assert _call_out(gdn, _shape(gdn), osc) == gdn.GDN_ERR_CUDA
+    assert _call_out(gdn, _shape(gdn), None) == gdn.GDN_ERR_CUDA
