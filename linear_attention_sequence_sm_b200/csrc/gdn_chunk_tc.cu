@@ -99,12 +99,12 @@ constexpr uint32_t kOffBar = kOffTpp + 8192;          // mbarriers, tensor-memor
 constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024; // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 per-block limit");
 // With the output side: the chunk's gate tile z (64 tokens x 128 bf16,
-// token-major, by TMA one chunk ahead) after the barriers.  The per-token
-// partial sums of squares use the chunk's P buffer, whose product has
-// completed by the output epilogue.
+// token-major, by TMA one chunk ahead) and the per-token partial sums of
+// squares after the barriers.
 constexpr uint32_t kOffZ = (kOffBar + 128 + 1023) / 1024 * 1024;
 constexpr uint32_t kBytesZ = 64 * 128 * 2;
-constexpr uint32_t kSmemBytesOut = kOffZ + kBytesZ + 1024;
+constexpr uint32_t kOffRed = kOffZ + kBytesZ;  // per token, 4 partial sums of squares (fp32 64 x 4)
+constexpr uint32_t kSmemBytesOut = kOffRed + 64 * 4 * 4 + 1024;
 static_assert(kSmemBytesOut <= 232448, "shared memory over the sm_100 per-block limit");
 // per-token vectors inside a buffer (floats)
 constexpr int kVecG = 0, kVecB = 64, kVecGam = 128, kVecBG = 192, kVecLam = 256, kVecIGam = 320;
@@ -465,6 +465,71 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tmem_st16u(tmem + lane_bits + kColX1 + 32 * ch + 16, z);
             }
             tmem_wait_st();
+            // Output side, second half, for the chunk whose O (fp32) waits in X2's
+            // columns (tokens cp .. cp + Lp - 1): per token the root mean square
+            // over the 128 value rows (column sums of O^2 per warp, then 4 partial
+            // sums per token), scale, gate, stage and store; then the gate tile of
+            // the chunk at cz may come in.  It runs while the tensor cores work on
+            // the next chunk's merged product (4)+(5), which leaves X2 alone.
+            auto out_deferred = [&](int cp, int Lp, bool load_next, int cz) -> bool {
+                __nv_bfloat16 *Ot = reinterpret_cast<__nv_bfloat16 *>(smem + kOffOst);
+                float *red = reinterpret_cast<float *>(smem + kOffRed);
+                const __nv_bfloat16 *Zt = reinterpret_cast<const __nv_bfloat16 *>(smem + kOffZ);
+                float ov[2][16];
+#pragma unroll
+                for (int sl = 0; sl < 2; ++sl) tmem_ld16(tmem + lane_bits + kColX2 + 32 * ch + 16 * sl, ov[sl]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int sl = 0; sl < 2; ++sl) {
+                    float sq[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) sq[j] = ov[sl][j] * ov[sl][j];
+                    const float part = warp_colsum16(sq, lane);
+                    if ((lane & 1) == 0) red[(32 * ch + 16 * sl + (lane >> 1)) * 4 + (warp & 3)] = part;
+                }
+                bool ok = true;
+                if (zgate) {
+                    ok = mbar_wait(bars + 8 * kBarZ, ph_z);
+                    ph_z ^= 1u;
+                }
+                // (also orders the staging writes after tid 0's wait for the last store)
+                if (named_sync_or(kBarChain, kChain, !ok)) return false;
+                float inv_rms;  // of token 32 ch + lane
+                {
+                    const float4 pr = *reinterpret_cast<const float4 *>(red + 4 * (32 * ch + lane));
+                    inv_rms = rsqrtf(((pr.x + pr.y) + (pr.z + pr.w)) * (1.f / 128.f) + a.out.eps);
+                }
+                const uint32_t oflags = a.out.flags;
+#pragma unroll
+                for (int sl = 0; sl < 2; ++sl)
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int r = 32 * ch + 16 * sl + j;
+                        float y = ov[sl][j] * out_s * __shfl_sync(0xffffffffu, inv_rms, 16 * sl + j);
+                        if (zgate) y *= out_gate_fast(oflags, __bfloat162float(Zt[r * 128 + row]));
+                        Ot[r * 128 + row] = __float2bfloat16_rn(y);
+                    }
+                fence_proxy_async_shared();
+                named_sync(kBarChain, kChain);
+                if (Lp == 64) {
+                    if (tid == 0) {
+                        tma_store_3d(&tm_o, sb + kOffOst, 0, h, cp);
+                        bulk_commit();
+                    }
+                } else {
+                    for (int e = tid; e < 64 * 16; e += kChain) {
+                        const int r = e >> 4, c = e & 15;
+                        if (r < Lp) {
+                            const uint4 val = *reinterpret_cast<const uint4 *>(smem + kOffOst + r * 256 + c * 16);
+                            *reinterpret_cast<uint4 *>(o + (size_t(cp + r) * hv + h) * 128 + c * 8) = val;
+                        }
+                    }
+                    named_sync(kBarChain, kChain);
+                }
+                // the gate tile has been read by every thread (barriers above)
+                if (load_next && zgate && tid == 0) load_z(sb + kOffZ, bars + 8 * kBarZ, &tm_z, h, cz);
+                return true;
+            };
             for (int n = 0; n < nchunks; ++n) {
                 const uint32_t gcn = gn + n, b = gcn & 1;
                 const int c0 = t0 + n * 64, L = min(64, len - n * 64);
@@ -551,6 +616,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     mma_commit(bars + 8 * kBarC);
                     bulk_wait_read();  // the previous chunk's output store has read the staging tile
                 }
+                // output side: the previous chunk (a full one: only a sequence's last
+                // chunk is ragged) finishes under this product; its gate tile then
+                // makes room for this chunk's
+                if constexpr (kOut)
+                    if (n > 0 && !out_deferred(c0 - 64, 64, true, c0)) { aborted = true; break; }
                 {
                     const bool ok = !chain_poll || mbar_wait(bars + 8 * kBarC, ph_c);
                     ph_c ^= 1u;
@@ -626,15 +696,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tmem_wait_st();
                 }
                 else {
-                    // output side: y = O / sqrt(mean_i O[r][i]^2 + eps) * s_i * act(z[r][i]).
-                    // Pass 1 leaves O (fp32) in X2's columns, zeroes X1', and per token
-                    // sums O^2 over this warp's 32 value rows into the consumed P buffer.
-                    __nv_bfloat16 *Ot = reinterpret_cast<__nv_bfloat16 *>(smem + kOffOst);
-                    float *red = reinterpret_cast<float *>(smem + (b ? kOffP1 : kOffP0));
-                    const int quad = warp & 3;
-                    uint32_t zr[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) zr[j] = 0u;
+                    // output side, first half: O = X2 - gamma X1' (fp32) into X2's columns and
+                    // X1' zeroed; the rest runs under the next chunk's merged product
 #pragma unroll
                     for (int sl = 0; sl < 2; ++sl) {
                         const int r0 = 32 * ch + 16 * sl;
@@ -644,71 +707,47 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                         for (int q = 0; q < 4; ++q) load4(vec + (kL2 ? kVecGo : kVecGam) + r0 + 4 * q, gm + 4 * q);
                         tmem_wait_ld();
-                        tmem_st16u(tmem + lane_bits + kColX1 + r0, zr);
-                        uint32_t ob[16];
-                        float sq[16];
+                        uint32_t ob[16], zr[16];
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
-                            const float ov = fmaf(-gm[j], x1[j], x2[j]);
-                            ob[j] = __float_as_uint(ov);
-                            sq[j] = ov * ov;
+                            ob[j] = __float_as_uint(fmaf(-gm[j], x1[j], x2[j]));
+                            zr[j] = 0u;
                         }
+                        tmem_st16u(tmem + lane_bits + kColX1 + r0, zr);
                         tmem_st16u(tmem + lane_bits + kColX2 + r0, ob);
-                        const float part = warp_colsum16(sq, lane);
-                        if ((lane & 1) == 0) red[(r0 + (lane >> 1)) * 4 + quad] = part;
                     }
                     tmem_wait_st();
-                    {
-                        bool ok = true;
-                        if (zgate) {
-                            ok = mbar_wait(bars + 8 * kBarZ, ph_z);
-                            ph_z ^= 1u;
-                        }
-                        if (named_sync_or(kBarChain, kChain, !ok)) { aborted = true; break; }
-                    }
-                    // pass 2: scale, gate and stage for the store
-                    const __nv_bfloat16 *Zt = reinterpret_cast<const __nv_bfloat16 *>(smem + kOffZ);
-                    const float eps = a.out.eps;
-                    const uint32_t oflags = a.out.flags;
-#pragma unroll
-                    for (int sl = 0; sl < 2; ++sl) {
-                        const int r0 = 32 * ch + 16 * sl;
-                        float ov[16];
-                        tmem_ld16(tmem + lane_bits + kColX2 + r0, ov);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int r = r0 + j;
-                            const float4 pr = *reinterpret_cast<const float4 *>(red + 4 * r);
-                            const float ms = ((pr.x + pr.y) + (pr.z + pr.w)) * (1.f / 128.f);
-                            float y = ov[j] * out_s * rsqrtf(ms + eps);
-                            if (zgate) y *= out_gate_fast(oflags, __bfloat162float(Zt[r * 128 + row]));
-                            Ot[r * 128 + row] = __float2bfloat16_rn(y);
-                        }
-                    }
                 }
                 fence_proxy_async_shared();
                 tc_fence_before();
                 named_sync(kBarChain, kChain);
-                // the gate tile is read: the next chunk's may come in
-                if (kOut && zgate && tid == 0 && n + 1 < nchunks)
-                    load_z(sb + kOffZ, bars + 8 * kBarZ, &tm_z, h, c0 + 64);
-                if (L == 64) {
-                    if (tid == 0) {
-                        tma_store_3d(&tm_o, sb + kOffOst, 0, h, c0);
-                        bulk_commit();
-                    }
-                } else {
-                    for (int e = tid; e < 64 * 16; e += kChain) {
-                        const int r = e >> 4, c = e & 15;
-                        if (r < L) {
-                            const uint4 val = *reinterpret_cast<const uint4 *>(smem + kOffOst + r * 256 + c * 16);
-                            *reinterpret_cast<uint4 *>(o + (size_t(c0 + r) * hv + h) * 128 + c * 8) = val;
+                if constexpr (!kOut) {
+                    if (L == 64) {
+                        if (tid == 0) {
+                            tma_store_3d(&tm_o, sb + kOffOst, 0, h, c0);
+                            bulk_commit();
                         }
+                    } else {
+                        for (int e = tid; e < 64 * 16; e += kChain) {
+                            const int r = e >> 4, c = e & 15;
+                            if (r < L) {
+                                const uint4 val =
+                                    *reinterpret_cast<const uint4 *>(smem + kOffOst + r * 256 + c * 16);
+                                *reinterpret_cast<uint4 *>(o + (size_t(c0 + r) * hv + h) * 128 + c * 8) = val;
+                            }
+                        }
+                        named_sync(kBarChain, kChain);
                     }
-                    named_sync(kBarChain, kChain);
                 }
                 if (tid == 0) mbar_arrive(bars + 8 * (kBarEmpty + b));  // buffers b may be refilled
+            }
+            if constexpr (kOut) {
+                if (!aborted && nchunks > 0) {
+                    const int cl = t0 + (nchunks - 1) * 64;
+                    if (tid == 0) bulk_wait_read();  // the previous store has read the staging tile
+                    if (!out_deferred(cl, len - (nchunks - 1) * 64, false, 0)) aborted = true;
+                    tc_fence_before();
+                }
             }
             if (!aborted) {
                 // final state out of tensor memory
