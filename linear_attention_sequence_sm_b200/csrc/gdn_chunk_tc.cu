@@ -49,6 +49,12 @@
 // group polls the mbarriers.  A full chunk of output leaves through one TMA
 // store of the staged tile.
 //
+// With the output side (a template instance of its own), each output row is
+// RMS-normalised, scaled and gated before it is stored: after (6)+(7) the
+// chain leaves O in fp32 in X2's columns, and the row reductions, scale, gate
+// and store of that chunk run under the next chunk's merged product (4)+(5).
+// The gate tile arrives by TMA one chunk ahead.
+//
 // One CTA per SM (shared memory and the 512 tensor-memory columns force it)
 // takes units longest sequence first from an atomic counter.  Every wait is
 // bounded; a timeout records GDN_ERR_DEVICE_CHECK (bad_index -2) in the

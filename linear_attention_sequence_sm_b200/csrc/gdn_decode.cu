@@ -11,6 +11,10 @@
 // and written once.  Decode is bound by that traffic ("The Transformer Isn't
 // Alone Anymore": the recurrent state is read and updated every step).
 //
+// With the output side (gdn_decode_step_out) the d_v outputs of the block's
+// (sequence, head) wait in shared memory; one block reduction gives their
+// root mean square, and y = o / rms * s * act(z) is written once.
+//
 // d_k = 128: a warp owns whole rows; lane l holds s_i[4l .. 4l+3] as one
 // float4 (a row is one coalesced 512-byte segment).  Each warp keeps
 // kRowBatch rows of loads in flight before reducing, for memory-level
