@@ -39,6 +39,11 @@
  *                             write S <- S - beta (S k - v) k^T
  *                             ("Architecture Thread I", the delta-rule
  *                             update), with no gate.
+ *   gdn_oracle_kda_recurrent / gdn_oracle_kda_chunkwise -- Kimi Delta
+ *                             Attention ("Gated Attention Architectures",
+ *                             section 8): one decay per key channel; the
+ *                             token recurrence and an independent chunked
+ *                             form derived from it.
  * and the mixer's two sides around the recurrence:
  *   gdn_oracle_prepare       -- q, k L2-normalised per head; gates from
  *                             their logits (the input side).
@@ -300,9 +305,180 @@ static void chunkwise_unit(const gdn_oracle_problem *p, const gdn_oracle_chunk_o
 }
 
 /* ------------------------------------------------------------------ */
+/* 4. Kimi Delta Attention (KDA): one decay per key channel.            */
+/* ------------------------------------------------------------------ */
+/* "Gated Attention Architectures", section 8 (Kimi Delta Attention),
+ * "Mathematical Formulation": S_t = (I - beta_t k_t k_t^T) D_t S_{t-1}
+ * + beta_t k_t v_t^T and o_t = S_t^T q_t, with D_t = diag(alpha_t) holding
+ * one decay per key channel.  That page's state is d_k x d_v; in this
+ * oracle's orientation (d_v x d_k, the transpose) the same update reads
+ *     S_t = S_{t-1} D_t (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *     o_t = S_t q_t,
+ * so each row s of S becomes s' = alpha_t .* s, then
+ * s <- s' + beta_t (v_i - s' . k_t) k_t.  With every alpha_t[c] equal this
+ * is the gated delta rule above (the page: KDA reduces to Gated DeltaNet
+ * when the decay collapses to a scalar).
+ * g is read as [T, Hv, d_k]: alpha_t[c] = exp(g[t, h, c]). */
+static int kda_recurrent_unit(const gdn_oracle_problem *p, int64_t unit, double *S) {
+    const int64_t n = unit / p->hv;
+    const int h = (int)(unit % p->hv);
+    const int hq = h / (p->hv / p->hk);
+    const int dk = p->dk, dv = p->dv;
+    double *alpha = malloc(sizeof(double) * dk);
+    double *sd = malloc(sizeof(double) * dk);
+    if (!alpha || !sd) {
+        free(alpha);
+        free(sd);
+        return -1;
+    }
+    if (p->s0) memcpy(S, p->s0 + unit * (int64_t)dv * dk, sizeof(double) * dv * dk);
+    else memset(S, 0, sizeof(double) * dv * dk);
+    for (int64_t t = p->cu_seqlens[n]; t < p->cu_seqlens[n + 1]; ++t) {
+        const double *kt = p->k + (t * p->hk + hq) * dk;
+        const double *qt = p->q + (t * p->hk + hq) * dk;
+        const double *vt = p->v + (t * p->hv + h) * dv;
+        const double *gt = p->g + (t * p->hv + h) * dk;
+        const double beta = p->beta[t * p->hv + h];
+        for (int j = 0; j < dk; ++j) alpha[j] = exp(gt[j]);
+        for (int i = 0; i < dv; ++i) {
+            /* the decayed row S_{t-1} D_t, and its prediction for k_t */
+            double pred = 0.0;
+            for (int j = 0; j < dk; ++j) {
+                sd[j] = alpha[j] * S[i * dk + j];
+                pred += sd[j] * kt[j];
+            }
+            const double ui = beta * (vt[i] - pred);
+            for (int j = 0; j < dk; ++j) S[i * dk + j] = sd[j] + ui * kt[j];
+        }
+        if (p->o) {
+            double *ot = p->o + (t * p->hv + h) * dv;
+            for (int i = 0; i < dv; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < dk; ++j) acc += S[i * dk + j] * qt[j];
+                ot[i] = acc;
+            }
+        }
+    }
+    if (p->s_final) memcpy(p->s_final + unit * (int64_t)dv * dk, S, sizeof(double) * dv * dk);
+    free(alpha);
+    free(sd);
+    return 0;
+}
+
+/* KDA in chunks of C tokens, derived here from the recurrence above (the
+ * page names a chunkwise WY algorithm with the decay absorbed into the keys;
+ * it prints none).  Within a chunk with start state S0 and the per-channel
+ * cumulative log-decay G_r[c] = g_0[c] + ... + g_r[c]:
+ *   S_r = S0 diag(e^{G_r}) + sum_{j<=r} u_j (k_j .* e^{G_r - G_j})^T
+ *   u_r = beta_r (v_r - S_{r-1} D_r k_r), which unrolls to
+ *   (I + A) U = diag(beta) V - diag(beta) K+ S0^T with
+ *   A_rj = beta_r sum_c k_r[c] k_j[c] e^{G_r[c] - G_j[c]}  (j < r),
+ *   K+_r = k_r .* e^{G_r};  so U = T diag(beta) V - T diag(beta) K+ S0^T,
+ *   T = (I + A)^-1;
+ *   o_r = S0 (q_r .* e^{G_r}) + sum_{j<=r} (sum_c q_r[c] k_j[c] e^{G_r[c] - G_j[c]}) u_j;
+ *   S_C = S0 diag(e^{G_last}) + sum_j u_j (k_j .* e^{G_last - G_j})^T.
+ * Every exponent above is a difference G_r - G_j with j <= r (or G itself),
+ * so with g <= 0 nothing overflows; the masked products are formed term by
+ * term, not as products of separately scaled matrices. */
+static int kda_chunk_unit(const gdn_oracle_problem *p, int C, int64_t unit, double *S) {
+    const int64_t n = unit / p->hv;
+    const int h = (int)(unit % p->hv);
+    const int hq = h / (p->hv / p->hk);
+    const int dk = p->dk, dv = p->dv;
+    double *G = malloc(sizeof(double) * C * dk);
+    double *A = malloc(sizeof(double) * C * C);
+    double *T = malloc(sizeof(double) * C * C);
+    double *W = malloc(sizeof(double) * C * dk);
+    double *U = malloc(sizeof(double) * C * dv);
+    double *O = malloc(sizeof(double) * C * dv);
+    double *Sn = malloc(sizeof(double) * dv * dk);
+    int rc = 0;
+    if (!G || !A || !T || !W || !U || !O || !Sn) {
+        rc = -1;
+        goto done;
+    }
+    if (p->s0) memcpy(S, p->s0 + unit * (int64_t)dv * dk, sizeof(double) * dv * dk);
+    else memset(S, 0, sizeof(double) * dv * dk);
+    const int64_t t_begin = p->cu_seqlens[n], t_end = p->cu_seqlens[n + 1];
+    for (int64_t c0 = t_begin; c0 < t_end; c0 += C) {
+        const int L = (int)((t_end - c0) < C ? (t_end - c0) : C);
+#define KDA_K(r, c) p->k[((c0 + (r)) * p->hk + hq) * dk + (c)]
+#define KDA_Q(r, c) p->q[((c0 + (r)) * p->hk + hq) * dk + (c)]
+#define KDA_V(r, i) p->v[((c0 + (r)) * p->hv + h) * dv + (i)]
+#define KDA_B(r) p->beta[(c0 + (r)) * p->hv + h]
+        for (int r = 0; r < L; ++r)
+            for (int c = 0; c < dk; ++c)
+                G[r * dk + c] = (r ? G[(r - 1) * dk + c] : 0.0) + p->g[((c0 + r) * p->hv + h) * dk + c];
+        /* A (strictly lower) and T = (I + A)^-1 by forward substitution */
+        for (int r = 0; r < L; ++r)
+            for (int j = 0; j < L; ++j) {
+                double a = 0.0;
+                if (j < r) {
+                    for (int c = 0; c < dk; ++c) a += KDA_K(r, c) * KDA_K(j, c) * exp(G[r * dk + c] - G[j * dk + c]);
+                    a *= KDA_B(r);
+                }
+                A[r * L + j] = a;
+            }
+        for (int col = 0; col < L; ++col)
+            for (int r = 0; r < L; ++r) {
+                double x = (r == col) ? 1.0 : 0.0;
+                for (int j = col; j < r; ++j) x -= A[r * L + j] * T[j * L + col];
+                T[r * L + col] = r < col ? 0.0 : x;
+            }
+        /* W = T diag(beta) K+ */
+        for (int r = 0; r < L; ++r)
+            for (int c = 0; c < dk; ++c) {
+                double acc = 0.0;
+                for (int j = 0; j <= r; ++j) acc += T[r * L + j] * KDA_B(j) * KDA_K(j, c) * exp(G[j * dk + c]);
+                W[r * dk + c] = acc;
+            }
+        /* U = T diag(beta) V - W S0^T */
+        for (int r = 0; r < L; ++r)
+            for (int i = 0; i < dv; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j <= r; ++j) acc += T[r * L + j] * KDA_B(j) * KDA_V(j, i);
+                for (int c = 0; c < dk; ++c) acc -= W[r * dk + c] * S[i * dk + c];
+                U[r * dv + i] = acc;
+            }
+        /* outputs from the chunk's start state and the corrected values */
+        for (int r = 0; r < L; ++r)
+            for (int i = 0; i < dv; ++i) {
+                double acc = 0.0;
+                for (int c = 0; c < dk; ++c) acc += S[i * dk + c] * KDA_Q(r, c) * exp(G[r * dk + c]);
+                for (int j = 0; j <= r; ++j) {
+                    double m = 0.0;
+                    for (int c = 0; c < dk; ++c) m += KDA_Q(r, c) * KDA_K(j, c) * exp(G[r * dk + c] - G[j * dk + c]);
+                    acc += m * U[j * dv + i];
+                }
+                O[r * dv + i] = acc;
+            }
+        if (p->o)
+            for (int r = 0; r < L; ++r)
+                memcpy(p->o + ((c0 + r) * p->hv + h) * dv, O + r * dv, sizeof(double) * dv);
+        /* state at the end of the chunk */
+        const double *Gl = G + (L - 1) * dk;
+        for (int i = 0; i < dv; ++i)
+            for (int c = 0; c < dk; ++c) {
+                double acc = S[i * dk + c] * exp(Gl[c]);
+                for (int j = 0; j < L; ++j) acc += U[j * dv + i] * KDA_K(j, c) * exp(Gl[c] - G[j * dk + c]);
+                Sn[i * dk + c] = acc;
+            }
+        memcpy(S, Sn, sizeof(double) * dv * dk);
+#undef KDA_K
+#undef KDA_Q
+#undef KDA_V
+#undef KDA_B
+    }
+    if (p->s_final) memcpy(p->s_final + unit * (int64_t)dv * dk, S, sizeof(double) * dv * dk);
+done:
+    free(G); free(A); free(T); free(W); free(U); free(O); free(Sn);
+    return rc;
+}
+
+/* ------------------------------------------------------------------ */
 /* Threading: units are independent, so threads take units round-robin. */
 /* ------------------------------------------------------------------ */
-enum { KIND_RECURRENT = 0, KIND_DELTA = 1, KIND_CHUNK = 2 };
+enum { KIND_RECURRENT = 0, KIND_DELTA = 1, KIND_CHUNK = 2, KIND_KDA = 3, KIND_KDA_CHUNK = 4 };
 
 typedef struct {
     int kind;
@@ -343,6 +519,8 @@ static void *worker(void *vp) {
             const int64_t unit = a->units ? a->units[i] : i;
             if (a->kind == KIND_RECURRENT) recurrent_unit(p, unit, S, buf);
             else if (a->kind == KIND_DELTA) delta_error_unit(p, unit, S, buf);
+            else if (a->kind == KIND_KDA) a->failed |= kda_recurrent_unit(p, unit, S) != 0;
+            else if (a->kind == KIND_KDA_CHUNK) a->failed |= kda_chunk_unit(p, a->co->chunk, unit, S) != 0;
             else chunkwise_unit(p, a->co, unit, &sc, a->chunk_base[unit / p->hv]);
         }
     }
@@ -377,6 +555,7 @@ static int run(int kind, const gdn_oracle_problem *p, const gdn_oracle_chunk_out
     if (n_threads > 256) n_threads = 256;
     if (n_threads > n_units && n_units > 0) n_threads = (int)n_units;
 
+    if (kind == KIND_KDA_CHUNK && (!co || co->chunk <= 0)) return -1;
     int64_t *chunk_base = NULL;
     if (kind == KIND_CHUNK) {
         if (!co || co->chunk <= 0) return -1;
@@ -423,6 +602,17 @@ int gdn_oracle_delta_error_form(const gdn_oracle_problem *p, const int64_t *unit
 int gdn_oracle_chunkwise(const gdn_oracle_problem *p, const gdn_oracle_chunk_out *co, const int64_t *units,
                          int64_t n_units, int n_threads) {
     return run(KIND_CHUNK, p, co, units, n_units, n_threads);
+}
+
+/* KDA: the problem's g is [T, Hv, d_k] (one log-decay per key channel). */
+int gdn_oracle_kda_recurrent(const gdn_oracle_problem *p, const int64_t *units, int64_t n_units, int n_threads) {
+    return run(KIND_KDA, p, NULL, units, n_units, n_threads);
+}
+
+int gdn_oracle_kda_chunkwise(const gdn_oracle_problem *p, int32_t chunk, const int64_t *units, int64_t n_units,
+                             int n_threads) {
+    gdn_oracle_chunk_out co = {chunk, NULL, NULL, NULL, NULL, NULL, NULL};
+    return run(KIND_KDA_CHUNK, p, &co, units, n_units, n_threads);
 }
 
 /* Number of chunks the chunkwise form uses (size of its intermediates). */

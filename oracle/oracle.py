@@ -89,6 +89,10 @@ def load(path: str | None = None):
         lib.gdn_oracle_output_side.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, D, D, D,
                                                ctypes.c_double, ctypes.c_uint32, D]
         lib.gdn_oracle_output_side.restype = None
+        lib.gdn_oracle_kda_recurrent.argtypes = [P, U, ctypes.c_int64, ctypes.c_int]
+        lib.gdn_oracle_kda_recurrent.restype = ctypes.c_int
+        lib.gdn_oracle_kda_chunkwise.argtypes = [P, ctypes.c_int32, U, ctypes.c_int64, ctypes.c_int]
+        lib.gdn_oracle_kda_chunkwise.restype = ctypes.c_int
         if path is None:
             _lib = lib
         return lib
@@ -291,4 +295,42 @@ def output_side(o, z=None, weight=None, eps=1e-6, gate="silu", zero_centred=Fals
     L.gdn_oracle_output_side(ctypes.c_int64(tokens), ctypes.c_int32(hv), ctypes.c_int32(dv), _dptr(o64),
                              _dptr(z64), _dptr(w64), ctypes.c_double(eps), ctypes.c_uint32(flags), _dptr(y))
     return y
+
+
+def _kda_run(name, q, k, v, g, beta, initial_state, cu_seqlens, units, threads, lib, extra=()):
+    """KDA: g holds one log-decay per key channel, [..., Hv, d_k]."""
+    g64 = _f64(g)
+    q, k, v, g0, beta, s0, cu, batched, dims = _prepare(q, k, v, g64[..., 0], beta, initial_state, cu_seqlens)
+    N, Ttot, hk, hv, dk, dv = dims
+    gk = np.ascontiguousarray(g64.reshape(Ttot, hv, dk))
+    o = np.full((Ttot, hv, dv), np.nan)
+    sf = np.full((N, hv, dv, dk), np.nan)
+    prob = _problem(q, k, v, gk, beta, s0, cu, o, sf, dims)
+    keep, uptr, nu = _units_arg(units)
+    fn = getattr(lib or load(), name)
+    rc = fn(ctypes.byref(prob), *extra, uptr, nu, threads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"oracle {name} failed ({rc})")
+    return _finish(o, sf, batched, dims)
+
+
+def kda_recurrent(q, k, v, g, beta, initial_state=None, cu_seqlens=None, units=None, threads=None, lib=None):
+    """Kimi Delta Attention, token recurrence (``gdn_oracle_kda_recurrent``):
+    g [..., Hv, d_k] is the per-key-channel log-decay.  Returns (o, final_state)."""
+    return _kda_run("gdn_oracle_kda_recurrent", q, k, v, g, beta, initial_state, cu_seqlens, units, threads, lib)
+
+
+def kda_chunkwise(q, k, v, g, beta, chunk, initial_state=None, cu_seqlens=None, units=None, threads=None, lib=None):
+    """Kimi Delta Attention in chunks of ``chunk`` tokens (``gdn_oracle_kda_chunkwise``),
+    an independent formulation derived from the recurrence."""
+    return _kda_run("gdn_oracle_kda_chunkwise", q, k, v, g, beta, initial_state, cu_seqlens, units, threads, lib,
+                    extra=(ctypes.c_int32(chunk),))
+
+
+def kda_decode_step(q, k, v, g, beta, state, threads=None, lib=None):
+    """One KDA token per sequence: q,k [N,Hk,dk], v [N,Hv,dv], g [N,Hv,dk],
+    beta [N,Hv], state [N,Hv,dv,dk].  Returns (o, new_state)."""
+    N = np.asarray(q).shape[0]
+    cu = np.arange(N + 1, dtype=np.int64)
+    return kda_recurrent(q, k, v, g, beta, initial_state=state, cu_seqlens=cu, threads=threads, lib=lib)
 

@@ -65,6 +65,19 @@ MUTANTS = [
     ("per-head scale rows ignored",
      "const double *wr = w ? w + ((out_flags & 8u) ? (int64_t)h * dv : 0) : NULL;",
      "const double *wr = w;"),
+    ("KDA prediction from the undecayed row",
+     "pred += sd[j] * kt[j];", "pred += S[i * dk + j] * kt[j];"),
+    ("KDA decay of one channel for all",
+     "for (int j = 0; j < dk; ++j) alpha[j] = exp(gt[j]);", "for (int j = 0; j < dk; ++j) alpha[j] = exp(gt[0]);"),
+    ("KDA write without beta",
+     "const double ui = beta * (vt[i] - pred);", "const double ui = (vt[i] - pred);"),
+    ("KDA chunk A with the decay transposed",
+     "a += KDA_K(r, c) * KDA_K(j, c) * exp(G[r * dk + c] - G[j * dk + c]);",
+     "a += KDA_K(r, c) * KDA_K(j, c) * exp(G[j * dk + c] - G[r * dk + c]);"),
+    ("KDA chunk output without the start-state decay",
+     "acc += S[i * dk + c] * KDA_Q(r, c) * exp(G[r * dk + c]);", "acc += S[i * dk + c] * KDA_Q(r, c);"),
+    ("KDA chunk end state without the decay of the writes",
+     "acc += U[j * dv + i] * KDA_K(j, c) * exp(Gl[c] - G[j * dk + c]);", "acc += U[j * dv + i] * KDA_K(j, c);"),
     ("A built with Gamma transposed",
      "a = p->beta[(c0 + r) * p->hv + h] * exp(G[r] - G[j]) * kk;",
      "a = p->beta[(c0 + r) * p->hv + h] * exp(G[j] - G[r]) * kk;"),
@@ -95,6 +108,12 @@ class _Bound:
     def output_side(self, *a, **kw):
         return oracle.output_side(*a, lib=self.lib, **kw)
 
+    def kda_recurrent(self, *a, **kw):
+        return oracle.kda_recurrent(*a, lib=self.lib, **kw)
+
+    def kda_chunkwise(self, *a, **kw):
+        return oracle.kda_chunkwise(*a, lib=self.lib, **kw)
+
 
 def _pin_calls(m):
     return [
@@ -112,6 +131,11 @@ def _pin_calls(m):
         lambda: pins.test_prepared_one_token_closed_form(m),
         lambda: pins.test_output_side_handworked(m),
         lambda: pins.test_output_side_invariants(m),
+        lambda: pins.test_kda_scalar_decay_is_gated_delta_rule(m),
+        lambda: pins.test_kda_brute_force_explicit_matrices(m),
+        lambda: pins.test_kda_beta_zero_is_channel_decay(m),
+        lambda: pins.test_kda_one_token(m),
+        lambda: pins.test_kda_chunkwise_equals_recurrent(m, 4),
     ]
 
 

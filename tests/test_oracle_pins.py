@@ -424,3 +424,86 @@ def test_output_side_invariants(oracle_mod):
     z = rng.standard_normal((T, hv, dv)) * 3.0
     yg = oracle_mod.output_side(o, z=z, eps=eps, gate="silu")
     assert np.allclose(yg, y * z / (1.0 + np.exp(-z)), rtol=1e-14)
+
+
+def _kda_problem(rng, T, hk, hv, d, s0=True, g_scale=1.0):
+    q, k, v, g, beta, S0 = _rand_problem(rng, T, hk, hv, d, d, s0=s0)
+    gk = -g_scale * np.logaddexp(0.0, rng.standard_normal((1, T, hv, d)))
+    return q, k, v, gk, beta, S0
+
+
+def test_kda_scalar_decay_is_gated_delta_rule(oracle_mod):
+    """KDA with the same decay on every key channel is the gated delta rule
+    ("Gated Attention Architectures", section 8: KDA reduces to Gated
+    DeltaNet when the decay collapses to a scalar per head)."""
+    rng = np.random.default_rng(50)
+    q, k, v, g, beta, S0 = _rand_problem(rng, 41, 2, 4, 8, 8)
+    gk = np.repeat(g[..., None], 8, axis=-1)
+    o1, s1 = oracle_mod.kda_recurrent(q, k, v, gk, beta, initial_state=S0)
+    o2, s2 = oracle_mod.recurrent(q, k, v, g, beta, initial_state=S0)
+    assert np.allclose(o1, o2, rtol=1e-12, atol=1e-13) and np.allclose(s1, s2, rtol=1e-12, atol=1e-13)
+
+
+def test_kda_brute_force_explicit_matrices(oracle_mod):
+    """KDA against explicit d x d transition matrices: with M_t =
+    diag(alpha_t)(I - beta_t k_t k_t^T) (this build's orientation, the
+    transpose of the page's (I - beta k k^T) D_t), S_t = S_{t-1} M_t +
+    beta_t v_t k_t^T and o_t = S_t q_t, multiplied out token by token."""
+    rng = np.random.default_rng(51)
+    T, d = 9, 5
+    q, k, v, gk, beta, S0 = _kda_problem(rng, T, 1, 1, d)
+    o, sf = oracle_mod.kda_recurrent(q, k, v, gk, beta, initial_state=S0)
+    S = S0[0, 0].copy()
+    for t in range(T):
+        kt, qt, vt, bt = k[0, t, 0], q[0, t, 0], v[0, t, 0], beta[0, t, 0]
+        M = np.diag(np.exp(gk[0, t, 0])) @ (np.eye(d) - bt * np.outer(kt, kt))
+        S = S @ M + bt * np.outer(vt, kt)
+        assert np.allclose(o[0, t, 0], S @ qt, rtol=1e-12, atol=1e-13)
+    assert np.allclose(sf[0, 0], S, rtol=1e-12, atol=1e-13)
+
+
+def test_kda_beta_zero_is_channel_decay(oracle_mod):
+    """beta = 0: only the decay acts, per key channel: S_T = S_0 diag(e^{sum g})
+    and o_t = S_0 (e^{G_t} .* q_t)."""
+    rng = np.random.default_rng(52)
+    q, k, v, gk, beta, S0 = _kda_problem(rng, 12, 1, 2, 6)
+    beta = np.zeros_like(beta)
+    o, sf = oracle_mod.kda_recurrent(q, k, v, gk, beta, initial_state=S0)
+    G = np.cumsum(gk[0], axis=0)  # [T, hv, d]
+    for h in range(2):
+        assert np.allclose(sf[0, h], S0[0, h] * np.exp(G[-1, h])[None, :], rtol=1e-13)
+        for t in range(12):
+            assert np.allclose(o[0, t, h], S0[0, h] @ (np.exp(G[t, h]) * q[0, t, 0]), rtol=1e-12, atol=1e-14)
+
+
+def test_kda_one_token(oracle_mod):
+    """One token from a start state S: o = S D q + beta (v - S D k)(k . q)
+    with D = diag(alpha); from zero, o = beta v (k . q) whatever the decay."""
+    rng = np.random.default_rng(53)
+    q, k, v, gk, beta, S0 = _kda_problem(rng, 1, 1, 1, 7)
+    D = np.exp(gk[0, 0, 0])
+    S, kt, qt, vt, bt = S0[0, 0], k[0, 0, 0], q[0, 0, 0], v[0, 0, 0], beta[0, 0, 0]
+    o, _ = oracle_mod.kda_recurrent(q, k, v, gk, beta, initial_state=S0)
+    ref = S @ (D * qt) + bt * (vt - S @ (D * kt)) * (kt @ qt)
+    assert np.allclose(o[0, 0, 0], ref, rtol=1e-13)
+    o0, _ = oracle_mod.kda_recurrent(q, k, v, gk, beta)
+    assert np.allclose(o0[0, 0, 0], bt * vt * (kt @ qt), rtol=1e-13)
+
+
+@pytest.mark.parametrize("C", [1, 4, 16])
+def test_kda_chunkwise_equals_recurrent(oracle_mod, C):
+    """The KDA chunked form (derived separately, masked products formed term
+    by term) against the token recurrence, batched and packed, with start
+    states and strong per-channel decay."""
+    rng = np.random.default_rng(54)
+    q, k, v, gk, beta, S0 = _kda_problem(rng, 45, 2, 4, 8, g_scale=3.0)
+    o1, s1 = oracle_mod.kda_recurrent(q, k, v, gk, beta, initial_state=S0)
+    o2, s2 = oracle_mod.kda_chunkwise(q, k, v, gk, beta, C, initial_state=S0)
+    assert np.allclose(o1, o2, rtol=1e-11, atol=1e-13) and np.allclose(s1, s2, rtol=1e-11, atol=1e-13)
+    lens = [0, 7, 17, 21]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    s0v = 0.3 * rng.standard_normal((4, 4, 8, 8))
+    o3, s3 = oracle_mod.kda_recurrent(q[0], k[0], v[0], gk[0], beta[0], initial_state=s0v, cu_seqlens=cu)
+    o4, s4 = oracle_mod.kda_chunkwise(q[0], k[0], v[0], gk[0], beta[0], C, initial_state=s0v, cu_seqlens=cu)
+    assert np.allclose(o3, o4, rtol=1e-11, atol=1e-13) and np.allclose(s3, s4, rtol=1e-11, atol=1e-13)
+    assert np.array_equal(s3[0], s0v[0])  # the empty sequence keeps its state
