@@ -54,6 +54,9 @@ def parse_args(argv=None):
                    help="prefill on raw q/k and gate logits, normalised and gated inside the kernels")
     p.add_argument("--output-norm", action="store_true",
                    help="prefill with the output side (RMS norm, per-channel scale, SiLU gate) in the kernel")
+    p.add_argument("--kda", action="store_true",
+                   help="Kimi Delta Attention (one decay per key channel) instead of the gated delta rule: "
+                        "CUDA-core prefill (ALU roofline) and decode (HBM roofline)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
@@ -265,7 +268,11 @@ def run_ours(args):
         seed={"prefill": 1002, "long": 1003, "varlen": 1005}[args.workload] + rank)
     host = I.make_raw_prefill_inputs(w) if args.raw_inputs else I.make_prefill_inputs(w)
     flags = {"qk_l2norm": True, "gate_logits": True} if args.raw_inputs else {}
-    suffix = ("_raw_inputs" if args.raw_inputs else "") + ("_output_norm" if args.output_norm else "")
+    suffix = ("_kda" if args.kda else "") + ("_raw_inputs" if args.raw_inputs else "") + \
+        ("_output_norm" if args.output_norm else "")
+    if args.kda:
+        host["g"] = I.make_kda_gates(w)
+    fwd = gdn.kda_forward if args.kda else gdn.chunk_forward
     if args.output_norm:
         host["out_gate"] = I.make_output_gate(w)
         out_weight = I.make_output_weight(w).to(device)
@@ -283,7 +290,7 @@ def run_ours(args):
     stream = torch.cuda.current_stream(device)
 
     def step():
-        gdn.chunk_forward(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], initial_state=dev["initial_state"],
+        fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], initial_state=dev["initial_state"],
                           cu_seqlens=dev["cu_seqlens"], out=o, final_state=sf, workspace=ws, chunk_size=w.chunk,
                           **flags, **out_norm(dev))
 
@@ -314,6 +321,17 @@ def run_ours(args):
                 "kernel": kernel_name,
                 "peak_source": f"{peak_src} bf16 dense (burst)",
                 "flops_per_launch": flops, "algorithmic_bytes_per_launch": prefill_bytes(w)}
+    if args.kda:
+        # token-order recurrence on CUDA cores: 7 d_v d_k fp32 flops per (token, value head)
+        # (decay, two dot products, rank-1 write); peak = SMs x 128 fp32 lanes x 2 x max SM clock
+        kflops = kda_flops_per_vhead_token(w.d) * tokens * w.hv
+        alu_peak = FP32_LANES_PER_SM * 2 * torch.cuda.get_device_properties(device).multi_processor_count * \
+            (clocks.summary().get("sm_max_mhz") or 1965) * 1e6 / 1e12
+        achieved = kflops / (ms / 1e3) / 1e12
+        roofline = {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s",
+                    "frac": achieved / alu_peak, "traffic": kernel_traffic(f"gdn_kda/{w.name}{suffix}"),
+                    "kernel": "gdn_kda", "peak_source": "fp32 FMA lanes x 2 x max SM clock (derived)",
+                    "flops_per_launch": kflops, "algorithmic_bytes_per_launch": prefill_bytes(w, kda=True)}
 
     # ---- decode: 256 sequences, fp32 state 512 MiB, in place ----
     decode = None
@@ -328,10 +346,15 @@ def run_ours(args):
         od = torch.empty((dw.num_seqs, dw.hv, dw.d), dtype=torch.bfloat16, device=device)
         it = [0]
 
+        if args.kda:
+            for s_, x in enumerate(ring):
+                x["g"] = I.make_kda_decode_gates(dw, s_).to(device)
+
         def dstep():
             x = ring[it[0] % len(ring)]
             it[0] += 1
-            gdn.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state, out=od)
+            (gdn.kda_decode_step if args.kda else gdn.decode_step)(x["q"], x["k"], x["v"], x["g"], x["beta"], state,
+                                                                   out=od)
 
         for _ in range(max(3, args.warmup)):
             dstep()
@@ -339,12 +362,13 @@ def run_ours(args):
         with ClockSampler(device.index) as dclocks:
             dms = timed(dstep, args.decode_steps, stream)
         dms = max_over_ranks(dms, device, world)
-        dbytes = decode_bytes(dw)
+        dbytes = decode_bytes(dw, kda=args.kda)
         dgbs = dbytes / (dms / 1e3) / 1e9
         decode = {"value": world * dgbs, "unit": "GB/s", "ms_per_step": dms, "steps": args.decode_steps,
                   "tokens_per_s": world * dw.num_seqs / (dms / 1e3), "workload": dw.name,
                   "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                               "frac": dgbs / peaks["hbm_gbs"], "traffic": kernel_traffic(f"gdn_decode/{dw.name}"),
+                               "frac": dgbs / peaks["hbm_gbs"],
+                               "traffic": kernel_traffic(f"gdn_decode/{dw.name}" + ("_kda" if args.kda else "")),
                                "kernel": "gdn_decode", "peak_source": f"{peak_src} HBM copy",
                                "bytes_per_launch": dbytes},
                   "clocks": dclocks.summary()}
@@ -361,7 +385,7 @@ def run_ours(args):
 
         def e2e_step():
             x = {k: v.to(device, non_blocking=True) for k, v in pin.items()}
-            oo, ss = gdn.chunk_forward(x["q"], x["k"], x["v"], x["g"], x["beta"], initial_state=x.get("initial_state"),
+            oo, ss = fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], initial_state=x.get("initial_state"),
                                        cu_seqlens=x.get("cu_seqlens"), chunk_size=w.chunk, workspace=ws, **flags,
                                        **out_norm(x))
             o_host.copy_(oo, non_blocking=True)
@@ -417,21 +441,31 @@ def useful_flops_per_vhead_token(group: int, d: int = 128, chunk: int = 64) -> i
     return 6 * d * d + 3 * chunk * d + 2 * chunk * d // group
 
 
-def prefill_bytes(w) -> int:
+FP32_LANES_PER_SM = 128
+
+
+def kda_flops_per_vhead_token(d: int = 128) -> int:
+    """Kimi Delta Attention in token order: per state element a decay
+    multiply, two dot-product FMAs (s'.k, s'.q) and the rank-1 write FMA."""
+    return 7 * d * d
+
+
+def prefill_bytes(w, kda: bool = False) -> int:
     """Mandatory HBM bytes of one prefill: q, k, v, o once, g and beta, the
-    initial state (if any) and the final state."""
+    initial state (if any) and the final state (KDA: g per key channel)."""
     esz = 2 if w.dtype == "bf16" else 4
     t = w.total_tokens
-    b = t * w.hk * w.d * esz * 2 + t * w.hv * w.d * esz * 2 + t * w.hv * 8
+    b = t * w.hk * w.d * esz * 2 + t * w.hv * w.d * esz * 2 + t * w.hv * (4 * w.d + 4 if kda else 8)
     b += w.num_seqs * w.hv * w.d * w.d * 4 * (2 if w.s0_std > 0 else 1)
     return b
 
 
-def decode_bytes(dw) -> int:
+def decode_bytes(dw, kda: bool = False) -> int:
     """Bytes one decode step must move: the fp32 state read and written once,
-    plus q, k, v, o (bf16) and g, beta (fp32)."""
+    plus q, k, v, o (bf16) and g, beta (fp32; KDA: g per key channel)."""
     s = dw.num_seqs * dw.hv * dw.d * dw.d * 4
-    return 2 * s + dw.num_seqs * (2 * dw.hk * dw.d * 2 + 2 * dw.hv * dw.d * 2 + 2 * dw.hv * 4)
+    gb = dw.hv * (4 * dw.d + 4) if kda else 2 * dw.hv * 4
+    return 2 * s + dw.num_seqs * (2 * dw.hk * dw.d * 2 + 2 * dw.hv * dw.d * 2 + gb)
 
 
 def main(argv=None):

@@ -257,6 +257,46 @@ GDN_API gdn_status_t gdn_decode_step_out(int32_t num_seqs, int32_t num_qk_heads,
                                  float *state, const gdn_output_side_t *out_side,
                                  void *o, uint32_t flags, void *stream);
 
+/* Kimi Delta Attention: the delta rule with one decay per key channel
+ * ("Gated Attention Architectures", section 8, "Mathematical Formulation":
+ * S_t = (I - beta_t k_t k_t^T) D_t S_{t-1} + beta_t k_t v_t^T, o_t = S_t^T q_t,
+ * D_t = diag(alpha_t)).  With this library's d_v x d_k state the update is
+ *     S_t = S_{t-1} diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *     o_t = S_t q_t,   alpha_t[c] = exp(g[t, h, c]),
+ * which is the gated delta rule when every alpha_t[c] is the same.
+ * Arguments are those of gdn_chunk_forward_out except
+ *   g     [tokens, Hv, d_k] fp32: one log-decay per key channel (with
+ *         GDN_FLAG_GATE_LOGITS: one decay logit per key channel, alpha =
+ *         sigmoid(logit)); read as max(g, -20) like the scalar gate.
+ * shape->chunk_size is checked as for gdn_chunk_forward but not used: the
+ * kernel walks the tokens of each sequence in order on CUDA cores, the state
+ * in registers (a block per sequence, value head and 32 rows of d_v), since
+ * the decay-masked key products of a chunked form are not plain matrix
+ * products.  Supports d_k <= 128 and d_v <= 128, fp32 or bf16; the input
+ * flags; an output side (applied as a second pass over o).  The workspace is
+ * that of gdn_chunk_forward for the same shape. */
+GDN_API gdn_status_t gdn_kda_forward(const gdn_shape_t *shape,
+                             const void *q, const void *k, const void *v,
+                             const float *g, const float *beta,
+                             const float *initial_state,
+                             const int32_t *cu_seqlens,
+                             const gdn_output_side_t *out_side,
+                             void *o, float *final_state,
+                             void *workspace, size_t workspace_bytes,
+                             void *stream);
+
+/* One Kimi Delta Attention token per sequence, state updated in place: per
+ * state row s_i, s' = alpha .* s_i, u_i = beta (v_i - s' . k),
+ * s_i <- s' + u_i k^T, o_i = s' . q + u_i (k . q); one read and one write of
+ * S.  g is [N, Hv, d_k] fp32; the other arguments are those of
+ * gdn_decode_step_out (out_side may be NULL). */
+GDN_API gdn_status_t gdn_kda_decode_step(int32_t num_seqs, int32_t num_qk_heads, int32_t num_v_heads,
+                                 int32_t head_dim_k, int32_t head_dim_v, int32_t dtype,
+                                 const void *q, const void *k, const void *v,
+                                 const float *g, const float *beta,
+                                 float *state, const gdn_output_side_t *out_side,
+                                 void *o, uint32_t flags, void *stream);
+
 /* Static text for a status code. */
 GDN_API const char *gdn_status_string(gdn_status_t status);
 

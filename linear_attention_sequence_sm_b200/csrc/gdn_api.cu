@@ -93,7 +93,11 @@ static gdn_status_t chunk_forward_impl(const gdn_shape_t *s, const void *q, cons
                                        const float *g, const float *beta, const float *initial_state,
                                        const int32_t *cu_seqlens, const gdn_output_side_t *out_side, void *o,
                                        float *final_state, void *workspace, size_t workspace_bytes,
-                                       void *stream_);
+                                       void *stream_, bool kda = false);
+static gdn_status_t decode_impl(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
+                                const void *q, const void *k, const void *v, const float *g, const float *beta,
+                                float *state, const gdn_output_side_t *out_side, void *o, uint32_t flags,
+                                void *stream_, bool kda);
 
 }  // namespace gdn
 
@@ -143,6 +147,14 @@ gdn_status_t gdn_chunk_forward_out(const gdn_shape_t *s, const void *q, const vo
                               workspace_bytes, stream_);
 }
 
+gdn_status_t gdn_kda_forward(const gdn_shape_t *s, const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const float *initial_state, const int32_t *cu_seqlens,
+                             const gdn_output_side_t *out_side, void *o, float *final_state, void *workspace,
+                             size_t workspace_bytes, void *stream_) {
+    return chunk_forward_impl(s, q, k, v, g, beta, initial_state, cu_seqlens, out_side, o, final_state, workspace,
+                              workspace_bytes, stream_, true);
+}
+
 }  // extern "C"
 
 namespace gdn {
@@ -151,7 +163,7 @@ static gdn_status_t chunk_forward_impl(const gdn_shape_t *s, const void *q, cons
                                        const float *g, const float *beta, const float *initial_state,
                                        const int32_t *cu_seqlens, const gdn_output_side_t *out_side, void *o,
                                        float *final_state, void *workspace, size_t workspace_bytes,
-                                       void *stream_) {
+                                       void *stream_, bool kda) {
     g_msg[0] = 0;
     gdn_status_t st = check_shape(s);
     if (st != GDN_OK) return st;
@@ -206,6 +218,15 @@ static gdn_status_t chunk_forward_impl(const gdn_shape_t *s, const void *q, cons
     a.sched.len = reinterpret_cast<const int32_t *>(ws + L.len_off);
     if (s->num_seqs == 0) return GDN_OK;
 
+    if (kda) {
+        e = launch_kda_prefill(a, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "KDA prefill launch");
+        if (out.flags) {
+            e = launch_output_side(o, int32_t(tokens), s->num_v_heads, s->head_dim_v, s->dtype, out, stream);
+            if (e != cudaSuccess) return cuda_fail(e, "output-side launch");
+        }
+        return GDN_OK;
+    }
     const bool use_tc = major == 10 && !(s->flags & GDN_FLAG_FORCE_SIMT) && chunk_tc_supported(*s);
     e = use_tc ? launch_chunk_tc(a, stream, sms) : launch_chunk_simt(a, stream, sms);
     if (e != cudaSuccess) return cuda_fail(e, use_tc ? "tensor-core prefill launch" : "prefill launch");
@@ -251,6 +272,24 @@ gdn_status_t gdn_decode_step_out(int32_t n, int32_t hk, int32_t hv, int32_t dk, 
                                  const void *q, const void *k, const void *v, const float *g, const float *beta,
                                  float *state, const gdn_output_side_t *out_side, void *o, uint32_t flags,
                                  void *stream_) {
+    return decode_impl(n, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, out_side, o, flags, stream_, false);
+}
+
+gdn_status_t gdn_kda_decode_step(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
+                                 const void *q, const void *k, const void *v, const float *g, const float *beta,
+                                 float *state, const gdn_output_side_t *out_side, void *o, uint32_t flags,
+                                 void *stream_) {
+    return decode_impl(n, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, out_side, o, flags, stream_, true);
+}
+
+}  // extern "C"
+
+namespace gdn {
+
+static gdn_status_t decode_impl(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
+                                const void *q, const void *k, const void *v, const float *g, const float *beta,
+                                float *state, const gdn_output_side_t *out_side, void *o, uint32_t flags,
+                                void *stream_, bool kda) {
     g_msg[0] = 0;
     OutSide out;
     gdn_status_t st = check_output_side(out_side, &out);
@@ -273,10 +312,12 @@ gdn_status_t gdn_decode_step_out(int32_t n, int32_t hk, int32_t hv, int32_t dk, 
     for (int i = 0; i < 7; ++i)
         if (!aligned16(ptrs[i])) return fail(GDN_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
     if (int64_t(n) * hv * dv * dk > (int64_t(1) << 40)) return fail(GDN_ERR_UNSUPPORTED, "state too large");
-    cudaError_t e = launch_decode(n, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o, flags, out,
-                                  static_cast<cudaStream_t>(stream_));
-    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    cudaError_t e = kda ? launch_kda_decode(n, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o, flags, out,
+                                            static_cast<cudaStream_t>(stream_))
+                        : launch_decode(n, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o, flags, out,
+                                        static_cast<cudaStream_t>(stream_));
+    if (e != cudaSuccess) return cuda_fail(e, kda ? "KDA decode launch" : "decode launch");
     return GDN_OK;
 }
 
-}  // extern "C"
+}  // namespace gdn

@@ -330,25 +330,6 @@ __device__ __forceinline__ void load_z(uint32_t dst, uint32_t bar, const CUtenso
     tma_load_3d(dst, tz, 0, h, c0, bar);
 }
 
-// Column sums over a warp of 16 values per lane, transposed: afterwards lanes
-// 2t and 2t + 1 return the sum over all 32 lanes of x[t] (t = 0..15).  Four
-// halving exchanges (each lane keeps the half of its values selected by its
-// lane bit and adds its partner's copy of that half) and a final pairwise
-// add: 16 shuffles instead of the 80 of 16 separate reductions.
-__device__ __forceinline__ float warp_colsum16(float (&x)[16], int lane) {
-#pragma unroll
-    for (int n = 8, bit = 16; n >= 1; n >>= 1, bit >>= 1) {
-        const bool up = (lane & bit) != 0;
-#pragma unroll
-        for (int m = 0; m < n; ++m) {
-            const float send = up ? x[m] : x[m + n];
-            const float keep = up ? x[m + n] : x[m];
-            x[m] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
-        }
-    }
-    return x[0] + __shfl_xor_sync(0xffffffffu, x[0], 1);
-}
-
 // kL2: GDN_FLAG_QK_L2NORM; kLogits: GDN_FLAG_GATE_LOGITS; kOut: the output
 // side in the output epilogue (compile-time, so the plain path carries none
 // of the input- or output-side work)

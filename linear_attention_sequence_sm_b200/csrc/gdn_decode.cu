@@ -36,6 +36,11 @@ constexpr int kRowBatch = GDN_DECODE_ROWS;  // rows in flight per warp
 // whole vector is known, for its root mean square.
 constexpr uint32_t kDecOut = 1u << 8;
 constexpr int kDecOutMaxDv = 256;
+// Template bit: Kimi Delta Attention, g holds one log-decay per key channel
+// ([N, Hv, d_k]): each row becomes s' = alpha .* s, p = s' . k, r = s' . q,
+// u = beta (v - p), s <- s' + u k, o = r + u (k . q) ("Gated Attention
+// Architectures", section 8; with all alpha[c] equal, the gated delta rule).
+constexpr uint32_t kDecKda = 1u << 9;
 
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
@@ -85,7 +90,28 @@ decode_d128_kernel(int32_t hk, int32_t hv, int32_t dv, const T *__restrict__ q, 
     }
     const float kq = warp_sum(kf[0] * qf[0] + kf[1] * qf[1] + kf[2] * qf[2] + kf[3] * qf[3]);
     constexpr bool logits = (flags & GDN_FLAG_GATE_LOGITS) != 0;
-    const float alpha = __expf(fmaxf(logits ? log_sigmoid(g[unit]) : g[unit], kGFloor));
+    constexpr bool kKda = (flags & kDecKda) != 0;
+    // GDN: one decay alpha; KDA: al[e] for this lane's channels, and the dot
+    // products take alpha .* k and alpha .* q
+    float alpha = 1.f, al[4], ak[4], aq[4];
+    if constexpr (kKda) {
+        float gg[4];
+        load_vec4(g + size_t(unit) * dk + 4 * lane, gg);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            al[e] = __expf(fmaxf(logits ? log_sigmoid(gg[e]) : gg[e], kGFloor));
+            ak[e] = al[e] * kf[e];
+            aq[e] = al[e] * qf[e];
+        }
+    } else {
+        alpha = __expf(fmaxf(logits ? log_sigmoid(g[unit]) : g[unit], kGFloor));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            al[e] = alpha;
+            ak[e] = kf[e];
+            aq[e] = qf[e];
+        }
+    }
     const float b = logits ? sigmoid(beta[unit]) : beta[unit];
 
     float *S = state + size_t(unit) * dv * dk;
@@ -104,8 +130,8 @@ decode_d128_kernel(int32_t hk, int32_t hv, int32_t dv, const T *__restrict__ q, 
 #pragma unroll
         for (int r = 0; r < kRowBatch; ++r) {
             if (i0 + r < dv) {
-                p[r] = s[r].x * kf[0] + s[r].y * kf[1] + s[r].z * kf[2] + s[r].w * kf[3];
-                rq[r] = s[r].x * qf[0] + s[r].y * qf[1] + s[r].z * qf[2] + s[r].w * qf[3];
+                p[r] = s[r].x * ak[0] + s[r].y * ak[1] + s[r].z * ak[2] + s[r].w * ak[3];
+                rq[r] = s[r].x * aq[0] + s[r].y * aq[1] + s[r].z * aq[2] + s[r].w * aq[3];
             } else {
                 p[r] = rq[r] = 0.f;
             }
@@ -121,15 +147,16 @@ decode_d128_kernel(int32_t hk, int32_t hv, int32_t dv, const T *__restrict__ q, 
 #pragma unroll
         for (int r = 0; r < kRowBatch; ++r) {
             if (i0 + r >= dv) continue;
-            const float u = b * (vr[r] - alpha * p[r]);
+            // GDN: p and rq are undecayed, alpha applies here; KDA: already decayed
+            const float u = kKda ? b * (vr[r] - p[r]) : b * (vr[r] - alpha * p[r]);
             float4 sn;
-            sn.x = fmaf(alpha, s[r].x, u * kf[0]);
-            sn.y = fmaf(alpha, s[r].y, u * kf[1]);
-            sn.z = fmaf(alpha, s[r].z, u * kf[2]);
-            sn.w = fmaf(alpha, s[r].w, u * kf[3]);
+            sn.x = fmaf(al[0], s[r].x, u * kf[0]);
+            sn.y = fmaf(al[1], s[r].y, u * kf[1]);
+            sn.z = fmaf(al[2], s[r].z, u * kf[2]);
+            sn.w = fmaf(al[3], s[r].w, u * kf[3]);
             store4(S + size_t(i0 + r) * dk + 4 * lane, sn);
             if (lane == r) {
-                const float ov = fmaf(alpha, rq[r], u * kq);
+                const float ov = kKda ? fmaf(u, kq, rq[r]) : fmaf(alpha, rq[r], u * kq);
                 if constexpr (kOut) ob[i0 + r] = ov;
                 else orow[i0 + r] = from_f32<T>(ov);
             }
@@ -197,7 +224,20 @@ decode_generic_kernel(int32_t hk, int32_t hv, int32_t dk, int32_t dv, const T *_
     for (int e = 0; e < kMaxPer; ++e) kq += kf[e] * qf[e];
     kq = warp_sum(kq);
     constexpr bool logits = (flags & GDN_FLAG_GATE_LOGITS) != 0;
-    const float alpha = __expf(fmaxf(logits ? log_sigmoid(g[unit]) : g[unit], kGFloor));
+    constexpr bool kKda = (flags & kDecKda) != 0;
+    float alpha = 1.f, al[kMaxPer];
+    if constexpr (kKda) {
+#pragma unroll
+        for (int e = 0; e < kMaxPer; ++e) {
+            const int j = lane + 32 * e;
+            const float gg = j < dk ? g[size_t(unit) * dk + j] : 0.f;
+            al[e] = __expf(fmaxf(logits ? log_sigmoid(gg) : gg, kGFloor));
+        }
+    } else {
+        alpha = __expf(fmaxf(logits ? log_sigmoid(g[unit]) : g[unit], kGFloor));
+#pragma unroll
+        for (int e = 0; e < kMaxPer; ++e) al[e] = alpha;
+    }
     const float b = logits ? sigmoid(beta[unit]) : beta[unit];
     float *S = state + size_t(unit) * dv * dk;
     for (int i = warp; i < dv; i += kDecodeWarps) {
@@ -207,19 +247,21 @@ decode_generic_kernel(int32_t hk, int32_t hv, int32_t dk, int32_t dv, const T *_
         for (int e = 0; e < kMaxPer; ++e) {
             const int j = lane + 32 * e;
             s[e] = j < dk ? S[size_t(i) * dk + j] : 0.f;
-            p += s[e] * kf[e];
-            rq += s[e] * qf[e];
+            const float sd = kKda ? al[e] * s[e] : s[e];  // KDA: the decayed row
+            p += sd * kf[e];
+            rq += sd * qf[e];
         }
         p = warp_sum(p);
         rq = warp_sum(rq);
-        const float u = b * (to_f32(v[size_t(unit) * dv + i]) - alpha * p);
+        const float u = kKda ? b * (to_f32(v[size_t(unit) * dv + i]) - p)
+                             : b * (to_f32(v[size_t(unit) * dv + i]) - alpha * p);
 #pragma unroll
         for (int e = 0; e < kMaxPer; ++e) {
             const int j = lane + 32 * e;
-            if (j < dk) S[size_t(i) * dk + j] = fmaf(alpha, s[e], u * kf[e]);
+            if (j < dk) S[size_t(i) * dk + j] = fmaf(al[e], s[e], u * kf[e]);
         }
         if (lane == 0) {
-            const float ov = fmaf(alpha, rq, u * kq);
+            const float ov = kKda ? fmaf(u, kq, rq) : fmaf(alpha, rq, u * kq);
             if constexpr (kOut) ob[i] = ov;
             else o[size_t(unit) * dv + i] = from_f32<T>(ov);
         }
@@ -253,15 +295,16 @@ static void launch_decode_as(dim3 grid, dim3 block, int32_t hk, int32_t hv, int3
     }
 }
 
-cudaError_t launch_decode(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
-                          const void *q, const void *k, const void *v, const float *g, const float *beta,
-                          float *state, void *o, uint32_t flags, const OutSide &os, cudaStream_t stream) {
+static cudaError_t launch_decode_any(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
+                                     const void *q, const void *k, const void *v, const float *g,
+                                     const float *beta, float *state, void *o, uint32_t flags, const OutSide &os,
+                                     bool kda, cudaStream_t stream) {
     const int64_t units = int64_t(n) * hv;
     if (units > INT32_MAX) return cudaErrorInvalidValue;
     if (os.flags && dv > kDecOutMaxDv) return cudaErrorInvalidValue;
     const dim3 grid(static_cast<unsigned>(units)), block(kDecodeWarps * 32);
     constexpr uint32_t L2 = GDN_FLAG_QK_L2NORM, LG = GDN_FLAG_GATE_LOGITS;
-    const uint32_t f = (flags & (L2 | LG)) | (os.flags ? kDecOut : 0u);
+    const uint32_t f = (flags & (L2 | LG)) | (os.flags ? kDecOut : 0u) | (kda ? kDecKda : 0u);
 #define GDN_DECODE_CASE(F)                                                                                  \
     case F: launch_decode_as<F>(grid, block, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o, os, stream); \
         break;
@@ -274,11 +317,31 @@ cudaError_t launch_decode(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t
         GDN_DECODE_CASE(kDecOut | L2)
         GDN_DECODE_CASE(kDecOut | LG)
         GDN_DECODE_CASE(kDecOut | L2 | LG)
+        GDN_DECODE_CASE(kDecKda)
+        GDN_DECODE_CASE(kDecKda | L2)
+        GDN_DECODE_CASE(kDecKda | LG)
+        GDN_DECODE_CASE(kDecKda | L2 | LG)
+        GDN_DECODE_CASE(kDecKda | kDecOut)
+        GDN_DECODE_CASE(kDecKda | kDecOut | L2)
+        GDN_DECODE_CASE(kDecKda | kDecOut | LG)
+        GDN_DECODE_CASE(kDecKda | kDecOut | L2 | LG)
         default: return cudaErrorInvalidValue;
     }
 #undef GDN_DECODE_CASE
     count_launch();
     return cudaGetLastError();
+}
+
+cudaError_t launch_decode(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
+                          const void *q, const void *k, const void *v, const float *g, const float *beta,
+                          float *state, void *o, uint32_t flags, const OutSide &os, cudaStream_t stream) {
+    return launch_decode_any(n, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o, flags, os, false, stream);
+}
+
+cudaError_t launch_kda_decode(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
+                              const void *q, const void *k, const void *v, const float *g, const float *beta,
+                              float *state, void *o, uint32_t flags, const OutSide &os, cudaStream_t stream) {
+    return launch_decode_any(n, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, o, flags, os, true, stream);
 }
 
 }  // namespace gdn

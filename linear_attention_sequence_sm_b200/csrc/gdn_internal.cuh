@@ -91,6 +91,25 @@ void count_launch();
 cudaError_t launch_schedule(const gdn_shape_t &s, const int32_t *cu_seqlens, void *workspace,
                             cudaStream_t stream);
 
+// Column sums over a warp of 16 values per lane, transposed: afterwards lanes
+// 2t and 2t + 1 return the sum over all 32 lanes of x[t] (t = 0..15).  Four
+// halving exchanges (each lane keeps the half of its values selected by its
+// lane bit and adds its partner's copy of that half) and a final pairwise
+// add: 16 shuffles instead of the 80 of 16 separate reductions.
+__device__ __forceinline__ float warp_colsum16(float (&x)[16], int lane) {
+#pragma unroll
+    for (int n = 8, bit = 16; n >= 1; n >>= 1, bit >>= 1) {
+        const bool up = (lane & bit) != 0;
+#pragma unroll
+        for (int m = 0; m < n; ++m) {
+            const float send = up ? x[m] : x[m + n];
+            const float keep = up ? x[m + n] : x[m];
+            x[m] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+        }
+    }
+    return x[0] + __shfl_xor_sync(0xffffffffu, x[0], 1);
+}
+
 // The output side as the kernels see it (gdn_output_side_t plus an enable
 // bit): y = o / sqrt(mean(o^2) + eps) * s * act(z).
 constexpr uint32_t kOutOn = 1u << 31;
@@ -151,6 +170,12 @@ bool chunk_tc_supported(const gdn_shape_t &s);
 // whose blocks each own a slice of d_v).
 cudaError_t launch_output_side(void *o, int32_t tokens, int32_t hv, int32_t dv, int32_t dtype, const OutSide &os,
                                cudaStream_t stream);
+
+// Kimi Delta Attention: prefill (token order, CUDA cores) and decode.
+cudaError_t launch_kda_prefill(const PrefillArgs &a, cudaStream_t stream);
+cudaError_t launch_kda_decode(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
+                              const void *q, const void *k, const void *v, const float *g, const float *beta,
+                              float *state, void *o, uint32_t flags, const OutSide &os, cudaStream_t stream);
 
 // Decode step.
 cudaError_t launch_decode(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,

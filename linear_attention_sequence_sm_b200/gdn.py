@@ -39,7 +39,8 @@ GDN_OUT_WEIGHT_PER_HEAD = 8
 
 EXPORTED = ("gdn_chunk_forward_workspace_size", "gdn_chunk_forward", "gdn_read_device_status",
             "gdn_decode_step", "gdn_status_string", "gdn_last_error_message", "gdn_launch_count",
-            "gdn_chunk_forward_noalloc", "gdn_decode_step_ex", "gdn_chunk_forward_out", "gdn_decode_step_out")
+            "gdn_chunk_forward_noalloc", "gdn_decode_step_ex", "gdn_chunk_forward_out", "gdn_decode_step_out",
+            "gdn_kda_forward", "gdn_kda_decode_step")
 
 
 class GdnError(RuntimeError):
@@ -86,6 +87,10 @@ def _load(path: str = LIB_PATH):
     lib.gdn_decode_step_out.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, osp, vp,
                                         ctypes.c_uint32, vp]
     lib.gdn_decode_step_out.restype = st
+    lib.gdn_kda_forward.argtypes = lib.gdn_chunk_forward_out.argtypes
+    lib.gdn_kda_forward.restype = st
+    lib.gdn_kda_decode_step.argtypes = lib.gdn_decode_step_out.argtypes
+    lib.gdn_kda_decode_step.restype = st
     lib.gdn_status_string.argtypes = [st]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_last_error_message.argtypes = []
@@ -299,6 +304,68 @@ def decode_step(q, k, v, g, beta, state, out=None, stream=None, qk_l2norm=False,
     _check(LIB.gdn_decode_step_ex(N, hk, hv, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
                                   _ptr(beta), _ptr(state), _ptr(out), input_flags(qk_l2norm, gate_logits),
                                   _stream_handle(stream)))
+    return out
+
+
+def kda_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, output_final_state=True, out=None,
+                final_state=None, workspace=None, stream=None, qk_l2norm=False, gate_logits=False,
+                output_norm: OutputNorm | None = None, chunk_size=64):
+    """Kimi Delta Attention prefill (one decay per key channel): g is
+    [..., Hv, d_k] fp32.  Returns (o, final_state or None).  Other arguments
+    as for chunk_forward; ``chunk_size`` is validated but unused (the kernel
+    walks the tokens in order)."""
+    dev = q.device
+    dt = q.dtype
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, dt, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(initial_state, "initial_state", torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    if k.shape != q.shape:
+        raise ValueError("k must have the shape of q")
+    if tuple(g.shape) != tuple(v.shape[:-1]) + (q.shape[-1],):
+        raise ValueError(f"KDA g must be [..., Hv, d_k] = {tuple(v.shape[:-1]) + (q.shape[-1],)}, got {tuple(g.shape)}")
+    shape = make_shape(q, v, cu_seqlens, chunk_size, False, input_flags(qk_l2norm, gate_logits))
+    if out is None:
+        out = torch.empty(v.shape, dtype=dt, device=dev)
+    _need(out, "out", dt, dev)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((shape.num_seqs, shape.num_v_heads, shape.head_dim_v, shape.head_dim_k),
+                                  dtype=torch.float32, device=dev)
+    _need(final_state, "final_state", torch.float32, dev)
+    nbytes = workspace_size(shape)
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    osc = output_norm.c_struct(out) if output_norm is not None else None
+    _check(LIB.gdn_kda_forward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                               _ptr(initial_state), _ptr(cu_seqlens), None if osc is None else ctypes.byref(osc),
+                               _ptr(out), _ptr(final_state), _ptr(workspace), workspace.numel(),
+                               _stream_handle(stream)))
+    return out, final_state
+
+
+def kda_decode_step(q, k, v, g, beta, state, out=None, stream=None, qk_l2norm=False, gate_logits=False,
+                    output_norm: OutputNorm | None = None):
+    """One Kimi Delta Attention token per sequence: g [N, Hv, d_k] fp32;
+    ``state`` [N, Hv, d_v, d_k] fp32 updated in place.  Returns o [N, Hv, d_v]."""
+    dev, dt = q.device, q.dtype
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, dt, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(state, "state", torch.float32, dev)
+    N, hk, dk = q.shape
+    hv, dv = v.shape[1], v.shape[2]
+    if tuple(g.shape) != (N, hv, dk):
+        raise ValueError(f"KDA g must be [{N}, {hv}, {dk}], got {tuple(g.shape)}")
+    if out is None:
+        out = torch.empty(v.shape, dtype=dt, device=dev)
+    _need(out, "out", dt, dev)
+    osc = output_norm.c_struct(out) if output_norm is not None else None
+    _check(LIB.gdn_kda_decode_step(N, hk, hv, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                   _ptr(beta), _ptr(state), None if osc is None else ctypes.byref(osc), _ptr(out),
+                                   input_flags(qk_l2norm, gate_logits), _stream_handle(stream)))
     return out
 
 

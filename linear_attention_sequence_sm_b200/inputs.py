@@ -239,6 +239,16 @@ def make_raw_prefill_inputs(w: Workload):
     return base
 
 
+def make_kda_gates(w: Workload):
+    """Kimi Delta Attention's per-key-channel log-decay, [B, T, Hv, d] fp32,
+    with the scalar gate's recipe drawn once per channel:
+    g = -g_scale * softplus(N(0,1) + g_shift)."""
+    import torch
+    B, T, hv, d = w.batch, w.seq_len, w.hv, w.d
+    return _slabbed(w.seed, "kda_g", (B, T, hv, d), lambda z: -w.g_scale * _softplus(z + w.g_shift),
+                    torch.float32, d)
+
+
 def make_output_gate(w: Workload):
     """The output side's gate pre-activation z, shaped like o: N(0, 2^2)
     (SiLU then spans its negative dip and its near-identity range), rounded
@@ -267,6 +277,14 @@ def make_decode_inputs(w: DecodeWorkload, step: int):
     g = -_softplus(normal(s, "dg", (N, hv)))
     return {"q": _round(q, w.dtype), "k": _round(k, w.dtype), "v": _round(v, w.dtype),
             "g": torch.from_numpy(g).to(torch.float32), "beta": torch.from_numpy(beta).to(torch.float32)}
+
+
+def make_kda_decode_gates(w: DecodeWorkload, step: int):
+    """Kimi Delta Attention decode: a per-key-channel log-decay [N, Hv, d],
+    -softplus(N(0,1)) per channel (seed + step)."""
+    import torch
+    g = -_softplus(normal(w.seed + step, "dkda_g", (w.num_seqs, w.hv, w.d)))
+    return torch.from_numpy(g).to(torch.float32)
 
 
 def make_decode_state(w: DecodeWorkload):

@@ -334,3 +334,18 @@ def kda_decode_step(q, k, v, g, beta, state, threads=None, lib=None):
     cu = np.arange(N + 1, dtype=np.int64)
     return kda_recurrent(q, k, v, g, beta, initial_state=state, cu_seqlens=cu, threads=threads, lib=lib)
 
+
+def prepare_kda_inputs(q, k, g, beta, qk_l2norm=False, gate_logits=False, lib=None):
+    """The input side for KDA: as ``prepare_inputs``, with g [..., Hv, d_k]
+    holding one logit per key channel (each becomes log sigmoid of itself;
+    the transform is elementwise, so the channels pass as extra heads)."""
+    q64, k64, _, b64 = prepare_inputs(q, k, np.zeros_like(_f64(beta)), beta, qk_l2norm=qk_l2norm,
+                                      gate_logits=gate_logits, lib=lib)
+    g64 = _f64(g).copy()
+    if gate_logits:
+        flat = g64.reshape(-1, g64.shape[-2] * g64.shape[-1])
+        _, _, gp, _ = prepare_inputs(np.zeros((flat.shape[0], 1, 1)), np.zeros((flat.shape[0], 1, 1)), flat,
+                                     np.zeros_like(flat), gate_logits=True, lib=lib)
+        g64 = gp.reshape(g64.shape)
+    return q64, k64, g64, b64
+
