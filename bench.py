@@ -57,6 +57,8 @@ def parse_args(argv=None):
     p.add_argument("--kda", action="store_true",
                    help="Kimi Delta Attention (one decay per key channel) instead of the gated delta rule: "
                         "CUDA-core prefill (ALU roofline) and decode (HBM roofline)")
+    p.add_argument("--mtp", type=int, default=0,
+                   help="decode: verify K draft tokens per sequence in one pass (state after every token kept)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
@@ -349,10 +351,22 @@ def run_ours(args):
         if args.kda:
             for s_, x in enumerate(ring):
                 x["g"] = I.make_kda_decode_gates(dw, s_).to(device)
+        if args.mtp > 0:
+            # K draft tokens per sequence: [N, K, H, d] inputs, one snapshot per token
+            K = args.mtp
+            ring = []
+            for s_ in range(4):
+                xs = [I.make_decode_inputs(dw, s_ * K + j) for j in range(K)]
+                ring.append({n: torch.stack([x_[n] for x_ in xs], dim=1).to(device) for n in xs[0]})
+            snaps = torch.empty((dw.num_seqs, K, dw.hv, dw.d, dw.d), dtype=torch.float32, device=device)
+            od = torch.empty((dw.num_seqs, K, dw.hv, dw.d), dtype=torch.bfloat16, device=device)
 
         def dstep():
             x = ring[it[0] % len(ring)]
             it[0] += 1
+            if args.mtp > 0:
+                gdn.decode_multi(x["q"], x["k"], x["v"], x["g"], x["beta"], state, out=od, snapshots=snaps)
+                return
             (gdn.kda_decode_step if args.kda else gdn.decode_step)(x["q"], x["k"], x["v"], x["g"], x["beta"], state,
                                                                    out=od)
 
@@ -362,13 +376,15 @@ def run_ours(args):
         with ClockSampler(device.index) as dclocks:
             dms = timed(dstep, args.decode_steps, stream)
         dms = max_over_ranks(dms, device, world)
-        dbytes = decode_bytes(dw, kda=args.kda)
+        dbytes = decode_bytes(dw, kda=args.kda, mtp=args.mtp)
         dgbs = dbytes / (dms / 1e3) / 1e9
         decode = {"value": world * dgbs, "unit": "GB/s", "ms_per_step": dms, "steps": args.decode_steps,
-                  "tokens_per_s": world * dw.num_seqs / (dms / 1e3), "workload": dw.name,
+                  "tokens_per_s": world * dw.num_seqs * max(1, args.mtp) / (dms / 1e3),
+                  "workload": dw.name + (f"_mtp{args.mtp}" if args.mtp > 0 else ""),
                   "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                "frac": dgbs / peaks["hbm_gbs"],
-                               "traffic": kernel_traffic(f"gdn_decode/{dw.name}" + ("_kda" if args.kda else "")),
+                               "traffic": kernel_traffic(f"gdn_decode/{dw.name}" + ("_kda" if args.kda else "")
+                                                         + (f"_mtp{args.mtp}" if args.mtp > 0 else "")),
                                "kernel": "gdn_decode", "peak_source": f"{peak_src} HBM copy",
                                "bytes_per_launch": dbytes},
                   "clocks": dclocks.summary()}
@@ -460,12 +476,17 @@ def prefill_bytes(w, kda: bool = False) -> int:
     return b
 
 
-def decode_bytes(dw, kda: bool = False) -> int:
+def decode_bytes(dw, kda: bool = False, mtp: int = 0) -> int:
     """Bytes one decode step must move: the fp32 state read and written once,
-    plus q, k, v, o (bf16) and g, beta (fp32; KDA: g per key channel)."""
+    plus q, k, v, o (bf16) and g, beta (fp32; KDA: g per key channel).  With
+    mtp = K draft tokens: the state read once and K snapshots written, and K
+    tokens' inputs and outputs."""
     s = dw.num_seqs * dw.hv * dw.d * dw.d * 4
     gb = dw.hv * (4 * dw.d + 4) if kda else 2 * dw.hv * 4
-    return 2 * s + dw.num_seqs * (2 * dw.hk * dw.d * 2 + 2 * dw.hv * dw.d * 2 + gb)
+    per_tok = dw.num_seqs * (2 * dw.hk * dw.d * 2 + 2 * dw.hv * dw.d * 2 + gb)
+    if mtp > 0:
+        return s * (1 + mtp) + per_tok * mtp
+    return 2 * s + per_tok
 
 
 def main(argv=None):

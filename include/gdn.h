@@ -297,6 +297,36 @@ GDN_API gdn_status_t gdn_kda_decode_step(int32_t num_seqs, int32_t num_qk_heads,
                                  float *state, const gdn_output_side_t *out_side,
                                  void *o, uint32_t flags, void *stream);
 
+/* Several decode tokens per sequence in one pass, for verifying draft
+ * tokens: multi-token prediction drafts a few tokens ahead and the model
+ * confirms several at once ("Architecture Thread I", the Qwen3-Next
+ * passage).  For each sequence the K = num_tokens tokens are applied in
+ * order from `state` with the decode step's update; o receives every
+ * token's output and `snapshots` the state after every token.  `state` is
+ * only read: after checking the drafts, gdn_decode_commit moves the state
+ * of the accepted prefix into it.  One read of S and K snapshot writes,
+ * instead of K reads and K writes for K decode steps.
+ *   q, k       [N, K, Hk, d_k] dtype;  v, o [N, K, Hv, d_v] dtype
+ *   g, beta    [N, K, Hv] fp32
+ *   state      [N, Hv, d_v, d_k] fp32 (read only)
+ *   snapshots  [N, K, Hv, d_v, d_k] fp32 (written; must not overlap state)
+ *   flags      GDN_FLAG_QK_L2NORM, GDN_FLAG_GATE_LOGITS
+ * Supports d_k = 128 and 1 <= K <= 16 (GDN_ERR_UNSUPPORTED otherwise). */
+GDN_API gdn_status_t gdn_decode_multi(int32_t num_seqs, int32_t num_tokens, int32_t num_qk_heads,
+                              int32_t num_v_heads, int32_t head_dim_k, int32_t head_dim_v, int32_t dtype,
+                              const void *q, const void *k, const void *v,
+                              const float *g, const float *beta, const float *state,
+                              float *snapshots, void *o, uint32_t flags, void *stream);
+
+/* Keeps the accepted prefix of a gdn_decode_multi call: for each sequence
+ * n, accepted[n] (device int32 [N]) in 1..K copies snapshot accepted[n] - 1
+ * into state[n]; 0 keeps state[n].  Values outside 0..K leave state[n]
+ * alone and, if bad_count (device int32) is not NULL, add one to it.
+ * Shapes as for gdn_decode_multi. */
+GDN_API gdn_status_t gdn_decode_commit(int32_t num_seqs, int32_t num_tokens, int32_t num_v_heads,
+                               int32_t head_dim_k, int32_t head_dim_v, const float *snapshots,
+                               const int32_t *accepted, float *state, int32_t *bad_count, void *stream);
+
 /* Static text for a status code. */
 GDN_API const char *gdn_status_string(gdn_status_t status);
 

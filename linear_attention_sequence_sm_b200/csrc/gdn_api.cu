@@ -321,3 +321,49 @@ static gdn_status_t decode_impl(int32_t n, int32_t hk, int32_t hv, int32_t dk, i
 }
 
 }  // namespace gdn
+
+extern "C" {
+
+gdn_status_t gdn_decode_multi(int32_t n, int32_t ntok, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
+                              const void *q, const void *k, const void *v, const float *g, const float *beta,
+                              const float *state, float *snapshots, void *o, uint32_t flags, void *stream_) {
+    g_msg[0] = 0;
+    if (flags & ~(GDN_FLAG_QK_L2NORM | GDN_FLAG_GATE_LOGITS))
+        return fail(GDN_ERR_INVALID_ARGUMENT, "unknown flag bits 0x%x", flags);
+    if (n < 0 || hk <= 0 || hv <= 0 || dk <= 0 || dv <= 0 || ntok <= 0)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "bad multi-token decode shape");
+    if (hv % hk != 0) return fail(GDN_ERR_INVALID_ARGUMENT, "num_v_heads must be a multiple of num_qk_heads");
+    if (dtype != GDN_DTYPE_F32 && dtype != GDN_DTYPE_BF16)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "dtype %d is not GDN_DTYPE_F32 or GDN_DTYPE_BF16", dtype);
+    if (dk != 128) return fail(GDN_ERR_UNSUPPORTED, "multi-token decode supports d_k = 128 (got %d)", dk);
+    if (ntok > 16) return fail(GDN_ERR_UNSUPPORTED, "multi-token decode takes at most 16 tokens (got %d)", ntok);
+    if (n == 0) return GDN_OK;
+    const void *ptrs[] = {q, k, v, g, beta, state, snapshots, o};
+    const char *names[] = {"q", "k", "v", "g", "beta", "state", "snapshots", "o"};
+    for (int i = 0; i < 8; ++i) {
+        if (!ptrs[i]) return fail(GDN_ERR_INVALID_ARGUMENT, "%s is NULL", names[i]);
+        if (!aligned16(ptrs[i])) return fail(GDN_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+    }
+    if (int64_t(n) * ntok * hv * dv * dk > (int64_t(1) << 40)) return fail(GDN_ERR_UNSUPPORTED, "too large");
+    cudaError_t e = launch_decode_multi(n, ntok, hk, hv, dk, dv, dtype, q, k, v, g, beta, state, snapshots, o,
+                                        flags, static_cast<cudaStream_t>(stream_));
+    if (e != cudaSuccess) return cuda_fail(e, "multi-token decode launch");
+    return GDN_OK;
+}
+
+gdn_status_t gdn_decode_commit(int32_t n, int32_t ntok, int32_t hv, int32_t dk, int32_t dv, const float *snapshots,
+                               const int32_t *accepted, float *state, int32_t *bad_count, void *stream_) {
+    g_msg[0] = 0;
+    if (n < 0 || hv <= 0 || dk <= 0 || dv <= 0 || ntok <= 0)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "bad commit shape");
+    if ((int64_t(dv) * dk) % 4 != 0) return fail(GDN_ERR_UNSUPPORTED, "d_v * d_k must be a multiple of 4");
+    if (n == 0) return GDN_OK;
+    if (!snapshots || !accepted || !state) return fail(GDN_ERR_INVALID_ARGUMENT, "NULL argument");
+    if (!aligned16(snapshots) || !aligned16(state)) return fail(GDN_ERR_MISALIGNED, "state or snapshots misaligned");
+    cudaError_t e = launch_decode_commit(n, ntok, hv, dk, dv, snapshots, accepted, state, bad_count,
+                                         static_cast<cudaStream_t>(stream_));
+    if (e != cudaSuccess) return cuda_fail(e, "commit launch");
+    return GDN_OK;
+}
+
+}  // extern "C"

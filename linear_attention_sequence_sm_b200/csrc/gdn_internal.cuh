@@ -177,6 +177,14 @@ cudaError_t launch_kda_decode(int32_t n, int32_t hk, int32_t hv, int32_t dk, int
                               const void *q, const void *k, const void *v, const float *g, const float *beta,
                               float *state, void *o, uint32_t flags, const OutSide &os, cudaStream_t stream);
 
+// Multi-token decode (draft verification) and its commit.
+cudaError_t launch_decode_multi(int32_t n, int32_t ntok, int32_t hk, int32_t hv, int32_t dk, int32_t dv,
+                                int32_t dtype, const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, const float *state, float *snap, void *o, uint32_t flags,
+                                cudaStream_t stream);
+cudaError_t launch_decode_commit(int32_t n, int32_t ntok, int32_t hv, int32_t dk, int32_t dv, const float *snap,
+                                 const int32_t *accepted, float *state, int32_t *bad, cudaStream_t stream);
+
 // Decode step.
 cudaError_t launch_decode(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
                           const void *q, const void *k, const void *v, const float *g, const float *beta,

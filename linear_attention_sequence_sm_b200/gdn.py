@@ -40,7 +40,7 @@ GDN_OUT_WEIGHT_PER_HEAD = 8
 EXPORTED = ("gdn_chunk_forward_workspace_size", "gdn_chunk_forward", "gdn_read_device_status",
             "gdn_decode_step", "gdn_status_string", "gdn_last_error_message", "gdn_launch_count",
             "gdn_chunk_forward_noalloc", "gdn_decode_step_ex", "gdn_chunk_forward_out", "gdn_decode_step_out",
-            "gdn_kda_forward", "gdn_kda_decode_step")
+            "gdn_kda_forward", "gdn_kda_decode_step", "gdn_decode_multi", "gdn_decode_commit")
 
 
 class GdnError(RuntimeError):
@@ -91,6 +91,10 @@ def _load(path: str = LIB_PATH):
     lib.gdn_kda_forward.restype = st
     lib.gdn_kda_decode_step.argtypes = lib.gdn_decode_step_out.argtypes
     lib.gdn_kda_decode_step.restype = st
+    lib.gdn_decode_multi.argtypes = [i32] * 7 + [vp] * 8 + [ctypes.c_uint32, vp]
+    lib.gdn_decode_multi.restype = st
+    lib.gdn_decode_commit.argtypes = [i32] * 5 + [vp] * 4 + [vp]
+    lib.gdn_decode_commit.restype = st
     lib.gdn_status_string.argtypes = [st]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_last_error_message.argtypes = []
@@ -367,6 +371,46 @@ def kda_decode_step(q, k, v, g, beta, state, out=None, stream=None, qk_l2norm=Fa
                                    _ptr(beta), _ptr(state), None if osc is None else ctypes.byref(osc), _ptr(out),
                                    input_flags(qk_l2norm, gate_logits), _stream_handle(stream)))
     return out
+
+
+def decode_multi(q, k, v, g, beta, state, out=None, snapshots=None, stream=None, qk_l2norm=False,
+                 gate_logits=False):
+    """K decode tokens per sequence in one pass (draft verification): q, k
+    [N, K, Hk, 128], v [N, K, Hv, d_v], g, beta [N, K, Hv]; ``state``
+    [N, Hv, d_v, 128] fp32 is only read.  Returns (o [N, K, Hv, d_v],
+    snapshots [N, K, Hv, d_v, 128] fp32: the state after each token)."""
+    dev, dt = q.device, q.dtype
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, dt, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(state, "state", torch.float32, dev)
+    N, K, hk, dk = q.shape
+    hv, dv = v.shape[2], v.shape[3]
+    if out is None:
+        out = torch.empty(v.shape, dtype=dt, device=dev)
+    if snapshots is None:
+        snapshots = torch.empty((N, K, hv, dv, dk), dtype=torch.float32, device=dev)
+    _need(out, "out", dt, dev)
+    _need(snapshots, "snapshots", torch.float32, dev)
+    _check(LIB.gdn_decode_multi(N, K, hk, hv, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                _ptr(beta), _ptr(state), _ptr(snapshots), _ptr(out),
+                                input_flags(qk_l2norm, gate_logits), _stream_handle(stream)))
+    return out, snapshots
+
+
+def decode_commit(snapshots, accepted, state, bad_count=None, stream=None):
+    """state[n] <- snapshots[n, accepted[n] - 1] for accepted[n] in 1..K
+    (0 keeps state[n]); ``accepted`` int32 [N] on the device."""
+    dev = state.device
+    _need(snapshots, "snapshots", torch.float32, dev)
+    _need(accepted, "accepted", torch.int32, dev)
+    _need(state, "state", torch.float32, dev)
+    _need(bad_count, "bad_count", torch.int32, dev)
+    N, K, hv, dv, dk = snapshots.shape
+    _check(LIB.gdn_decode_commit(N, K, hv, dk, dv, _ptr(snapshots), _ptr(accepted), _ptr(state), _ptr(bad_count),
+                                 _stream_handle(stream)))
+    return state
 
 
 def launch_count() -> int:

@@ -349,3 +349,20 @@ def prepare_kda_inputs(q, k, g, beta, qk_l2norm=False, gate_logits=False, lib=No
         g64 = gp.reshape(g64.shape)
     return q64, k64, g64, b64
 
+
+def decode_multi(q, k, v, g, beta, state, threads=None, lib=None):
+    """K decode tokens per sequence with the state after every token:
+    q, k [N, K, Hk, dk], v [N, K, Hv, dv], g, beta [N, K, Hv], state
+    [N, Hv, dv, dk].  Returns (o [N, K, Hv, dv], snapshots [N, K, Hv, dv, dk]).
+    A composition of ``decode_step`` (the pinned token recurrence), one token
+    at a time; no arithmetic of its own."""
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    S = _f64(state).copy()
+    N, K = q.shape[:2]
+    o = np.empty(v.shape)
+    snaps = np.empty((N, K) + S.shape[1:])
+    for j in range(K):
+        o[:, j], S = decode_step(q[:, j], k[:, j], v[:, j], g[:, j], beta[:, j], S, threads=threads, lib=lib)
+        snaps[:, j] = S
+    return o, snaps
+

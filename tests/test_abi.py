@@ -178,3 +178,24 @@ def test_output_side_valid_reaches_the_device_check(gdn):
     osc = gdn.OutputSideC(FAKE, FAKE, 1e-6, 1 | 4 | 8)
     assert _call_out(gdn, _shape(gdn), osc) == gdn.GDN_ERR_CUDA
     assert _call_out(gdn, _shape(gdn), None) == gdn.GDN_ERR_CUDA
+
+
+def test_decode_multi_and_commit_argument_checks(gdn):
+    vp = ctypes.c_void_p
+    f = gdn.LIB.gdn_decode_multi
+    ptrs = [vp(FAKE)] * 8
+    assert f(4, 3, 2, 4, 64, 128, 1, *ptrs, 0, None) == gdn.GDN_ERR_UNSUPPORTED   # d_k != 128
+    assert f(4, 17, 2, 4, 128, 128, 1, *ptrs, 0, None) == gdn.GDN_ERR_UNSUPPORTED  # more than 16 tokens
+    assert f(4, 0, 2, 4, 128, 128, 1, *ptrs, 0, None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert f(4, 3, 2, 3, 128, 128, 1, *ptrs, 0, None) == gdn.GDN_ERR_INVALID_ARGUMENT  # Hv % Hk
+    assert f(4, 3, 2, 4, 128, 128, 1, *ptrs, 8, None) == gdn.GDN_ERR_INVALID_ARGUMENT  # unknown flag
+    bad = [vp(FAKE)] * 6 + [vp(FAKE + 4), vp(FAKE)]
+    assert f(4, 3, 2, 4, 128, 128, 1, *bad, 0, None) == gdn.GDN_ERR_MISALIGNED
+    nul = [vp(FAKE)] * 6 + [None, vp(FAKE)]
+    assert f(4, 3, 2, 4, 128, 128, 1, *nul, 0, None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert f(0, 3, 2, 4, 128, 128, 1, *ptrs, 0, None) == gdn.GDN_OK
+    c = gdn.LIB.gdn_decode_commit
+    assert c(4, 3, 4, 128, 128, None, vp(FAKE), vp(FAKE), None, None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert c(4, 3, 4, 128, 128, vp(FAKE + 8), vp(FAKE), vp(FAKE), None, None) == gdn.GDN_ERR_MISALIGNED
+    assert c(4, 3, 4, 3, 3, vp(FAKE), vp(FAKE), vp(FAKE), None, None) == gdn.GDN_ERR_UNSUPPORTED
+    assert c(0, 3, 4, 128, 128, None, None, None, None, None) == gdn.GDN_OK
