@@ -604,6 +604,432 @@ int gdn_oracle_chunkwise(const gdn_oracle_problem *p, const gdn_oracle_chunk_out
     return run(KIND_CHUNK, p, co, units, n_units, n_threads);
 }
 
+/* ------------------------------------------------------------------ */
+/* 5. Gradients (training).                                             */
+/* ------------------------------------------------------------------ */
+/* The pages frame the chunkwise algorithm as the way to train the layer
+ * ("Architecture Thread I", the DeltaNet/Gated DeltaNet training remarks;
+ * "Gated Attention Architectures", sections 2 and 3).  For upstream
+ * gradients dO (of every output) and dS_T (of each final state) these are
+ * the gradients of L = sum dO . O + sum dS_T . S_T with respect to q, k, v,
+ * g, beta and the initial state.
+ *
+ * gdn_oracle_backward: reverse mode of the token recurrence, written out
+ * by hand.  Per token, with s' = alpha S_{t-1}, p = s' k, u = beta (v - p),
+ * S_t = s' + u k^T, o = S_t q (row form of the forward above), and dS the
+ * gradient of S_t accumulated from later tokens:
+ *   dS += dO_t q^T;              dq += S_t^T dO_t
+ *   du = dS k;                    dk += dS^T u
+ *   dbeta += du . (v - p);        dv = beta du;      dp = -beta du
+ *   ds' = dS + dp k^T;            dk += s'^T dp
+ *   dalpha = <ds', S_{t-1}>;      dg = alpha dalpha; dS_{t-1} = alpha ds'
+ * dq and dk are returned per VALUE head ([T, Hv, d_k]): summing the heads of
+ * a group gives the gradient of the shared q/k head. */
+typedef struct {
+    const double *dO;   /* [T, Hv, dv] */
+    const double *dSf;  /* [N, Hv, dv, dk] or NULL (zero) */
+    double *dq, *dk;    /* [T, Hv, dk] */
+    double *dv;         /* [T, Hv, dv] */
+    double *dg, *dbeta; /* [T, Hv] */
+    double *dS0;        /* [N, Hv, dv, dk] or NULL */
+} gdn_oracle_grads;
+
+static int backward_unit(const gdn_oracle_problem *p, const gdn_oracle_grads *gr, int64_t unit) {
+    const int64_t n = unit / p->hv;
+    const int h = (int)(unit % p->hv);
+    const int hq = h / (p->hv / p->hk);
+    const int dk = p->dk, dv = p->dv;
+    const int64_t t0 = p->cu_seqlens[n], T = p->cu_seqlens[n + 1] - t0;
+    const size_t ssz = (size_t)dv * dk;
+    double *Sh = malloc(sizeof(double) * ssz * (size_t)(T + 1)); /* S_{-1} .. S_{T-1} */
+    double *dS = malloc(sizeof(double) * ssz);
+    double *dsp = malloc(sizeof(double) * ssz);
+    double *pk = malloc(sizeof(double) * dv), *u = malloc(sizeof(double) * dv), *du = malloc(sizeof(double) * dv);
+    if (!Sh || !dS || !dsp || !pk || !u || !du) {
+        free(Sh); free(dS); free(dsp); free(pk); free(u); free(du);
+        return -1;
+    }
+    if (p->s0) memcpy(Sh, p->s0 + unit * (int64_t)ssz, sizeof(double) * ssz);
+    else memset(Sh, 0, sizeof(double) * ssz);
+    for (int64_t t = 0; t < T; ++t) { /* forward, keeping every state */
+        const int64_t tt = t0 + t;
+        const double *kt = p->k + (tt * p->hk + hq) * dk;
+        const double *vt = p->v + (tt * p->hv + h) * dv;
+        const double alpha = exp(p->g[tt * p->hv + h]), beta = p->beta[tt * p->hv + h];
+        const double *Sp = Sh + ssz * t;
+        double *Sn = Sh + ssz * (t + 1);
+        for (int i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) acc += alpha * Sp[i * dk + j] * kt[j];
+            const double ui = beta * (vt[i] - acc);
+            for (int j = 0; j < dk; ++j) Sn[i * dk + j] = alpha * Sp[i * dk + j] + ui * kt[j];
+        }
+    }
+    if (gr->dSf) memcpy(dS, gr->dSf + unit * (int64_t)ssz, sizeof(double) * ssz);
+    else memset(dS, 0, sizeof(double) * ssz);
+    for (int64_t t = T - 1; t >= 0; --t) {
+        const int64_t tt = t0 + t;
+        const double *kt = p->k + (tt * p->hk + hq) * dk;
+        const double *qt = p->q + (tt * p->hk + hq) * dk;
+        const double *vt = p->v + (tt * p->hv + h) * dv;
+        const double *dOt = gr->dO + (tt * p->hv + h) * dv;
+        const double alpha = exp(p->g[tt * p->hv + h]), beta = p->beta[tt * p->hv + h];
+        const double *Sp = Sh + ssz * t, *St = Sh + ssz * (t + 1);
+        double *dqt = gr->dq + (tt * p->hv + h) * dk, *dkt = gr->dk + (tt * p->hv + h) * dk;
+        double *dvt = gr->dv + (tt * p->hv + h) * dv;
+        for (int j = 0; j < dk; ++j) {
+            dqt[j] = 0.0;
+            dkt[j] = 0.0;
+        }
+        /* o = S_t q */
+        for (int i = 0; i < dv; ++i)
+            for (int j = 0; j < dk; ++j) {
+                dS[i * dk + j] += dOt[i] * qt[j];
+                dqt[j] += St[i * dk + j] * dOt[i];
+            }
+        /* the forward quantities of this token */
+        for (int i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) acc += alpha * Sp[i * dk + j] * kt[j];
+            pk[i] = acc;
+            u[i] = beta * (vt[i] - acc);
+        }
+        double dbeta = 0.0, dalpha = 0.0;
+        for (int i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) acc += dS[i * dk + j] * kt[j];
+            du[i] = acc;
+            dbeta += acc * (vt[i] - pk[i]);
+            dvt[i] = beta * acc;
+        }
+        for (int i = 0; i < dv; ++i) {
+            const double dpi = -beta * du[i];
+            for (int j = 0; j < dk; ++j) {
+                dkt[j] += u[i] * dS[i * dk + j] + dpi * alpha * Sp[i * dk + j];
+                dsp[i * dk + j] = dS[i * dk + j] + dpi * kt[j];
+                dalpha += dsp[i * dk + j] * Sp[i * dk + j];
+            }
+        }
+        for (size_t e = 0; e < ssz; ++e) dS[e] = alpha * dsp[e];
+        gr->dbeta[tt * p->hv + h] = dbeta;
+        gr->dg[tt * p->hv + h] = alpha * dalpha;
+    }
+    if (gr->dS0) memcpy(gr->dS0 + unit * (int64_t)ssz, dS, sizeof(double) * ssz);
+    free(Sh); free(dS); free(dsp); free(pk); free(u); free(du);
+    return 0;
+}
+
+typedef struct {
+    const gdn_oracle_problem *p;
+    const gdn_oracle_grads *gr;
+    int32_t chunk; /* 0: token recurrence; > 0: the chunked form */
+    int tid, nthreads, failed;
+} bwd_arg;
+
+static int backward_chunk_unit(const gdn_oracle_problem *p, const gdn_oracle_grads *gr, int64_t unit, int C);
+
+static void *bwd_worker(void *vp) {
+    bwd_arg *a = (bwd_arg *)vp;
+    const int64_t units = a->p->num_seqs * a->p->hv;
+    for (int64_t u = a->tid; u < units; u += a->nthreads) {
+        const int rc = a->chunk > 0 ? backward_chunk_unit(a->p, a->gr, u, a->chunk) : backward_unit(a->p, a->gr, u);
+        if (rc != 0) a->failed = 1;
+    }
+    return NULL;
+}
+
+static int run_backward(const gdn_oracle_problem *p, const gdn_oracle_grads *gr, int32_t chunk, int n_threads) {
+    if (validate(p) != 0 || !gr || !gr->dO || !gr->dq || !gr->dk || !gr->dv || !gr->dg || !gr->dbeta) return -1;
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > 256) n_threads = 256;
+    pthread_t th[256];
+    bwd_arg args[256];
+    int failed = 0;
+    for (int i = 0; i < n_threads; ++i) {
+        args[i] = (bwd_arg){p, gr, chunk, i, n_threads, 0};
+        if (pthread_create(&th[i], NULL, bwd_worker, &args[i]) != 0) {
+            bwd_worker(&args[i]);
+            th[i] = 0;
+        }
+    }
+    for (int i = 0; i < n_threads; ++i) {
+        if (th[i]) pthread_join(th[i], NULL);
+        failed |= args[i].failed;
+    }
+    return failed ? -2 : 0;
+}
+
+int gdn_oracle_backward(const gdn_oracle_problem *p, const gdn_oracle_grads *gr, int n_threads) {
+    return run_backward(p, gr, 0, n_threads);
+}
+
+/* gdn_oracle_backward_chunkwise: the gradients through the chunked form
+ * (the chunk forms of section 2 above), derived here by differentiating
+ * those matrix expressions; an independent formulation of the same
+ * gradients.  For a chunk with start state S0 and end-state gradient dS:
+ *   S_C = gamma_L S0 + U^T diag(lambda) K      -> dS0 = gamma_L dS, dU_j = lambda_j dS k_j,
+ *                                                 dk_j += lambda_j dS^T u_j, dlambda_j = u_j^T dS k_j
+ *   O = diag(gamma) Q S0^T + P U, P = QK^T (.) Gamma (lower, with diagonal)
+ *                                              -> dS0 += dO^T diag(gamma) Q, dq += diag(gamma) dO S0,
+ *                                                 dU += P^T dO, dP = dO U^T
+ *   U = U~ - W S0^T                             -> dW = -dU S0, dS0 -= dU^T W
+ *   W = T diag(beta gamma) K, U~ = T diag(beta) V
+ *                                              -> dT = dW (diag(bg) K)^T + dU (diag(beta) V)^T, ...
+ *   T = (I + A)^-1                              -> dA = -T^T dT T^T (strictly lower part)
+ *   A = diag(beta) (K K^T (.) Gamma) (strictly lower)
+ * and the decays through G (Gamma_rj = e^(G_r - G_j), gamma_r = e^(G_r),
+ * lambda_j = e^(G_last - G_j)), then dg_t = sum_{r >= t} dG_r.  The result
+ * must equal the token recurrence's. */
+static int backward_chunk_unit(const gdn_oracle_problem *p, const gdn_oracle_grads *gr, int64_t unit, int C) {
+    const int64_t n = unit / p->hv;
+    const int h = (int)(unit % p->hv);
+    const int hq = h / (p->hv / p->hk);
+    const int dk = p->dk, dv = p->dv;
+    const int64_t t0 = p->cu_seqlens[n], T = p->cu_seqlens[n + 1] - t0;
+    const int64_t nch = (T + C - 1) / C;
+    const size_t ssz = (size_t)dv * dk;
+    double *S0s = malloc(sizeof(double) * ssz * (size_t)(nch + 1));
+    double *dS = malloc(sizeof(double) * ssz), *dS0 = malloc(sizeof(double) * ssz);
+    double *G = malloc(sizeof(double) * C), *gam = malloc(sizeof(double) * C), *lam = malloc(sizeof(double) * C);
+    double *A = malloc(sizeof(double) * C * C), *Tm = malloc(sizeof(double) * C * C);
+    double *Gm = malloc(sizeof(double) * C * C), *KK = malloc(sizeof(double) * C * C), *QK = malloc(sizeof(double) * C * C);
+    double *W = malloc(sizeof(double) * C * dk), *U = malloc(sizeof(double) * C * dv);
+    double *dU = malloc(sizeof(double) * C * dv), *dW = malloc(sizeof(double) * C * dk);
+    double *dT = malloc(sizeof(double) * C * C), *dA = malloc(sizeof(double) * C * C), *tmp = malloc(sizeof(double) * C * C);
+    double *dGam = malloc(sizeof(double) * C * C);
+    double *dQ = malloc(sizeof(double) * C * dk), *dK = malloc(sizeof(double) * C * dk);
+    double *dG = malloc(sizeof(double) * C), *dgam = malloc(sizeof(double) * C), *dlam = malloc(sizeof(double) * C);
+    double *dbg = malloc(sizeof(double) * C), *dbeta = malloc(sizeof(double) * C);
+    int rc = 0;
+    if (!S0s || !dS || !dS0 || !G || !gam || !lam || !A || !Tm || !Gm || !KK || !QK || !W || !U || !dU || !dW ||
+        !dT || !dA || !tmp || !dGam || !dQ || !dK || !dG || !dgam || !dlam || !dbg || !dbeta) {
+        rc = -1;
+        goto done;
+    }
+#define BK(r, c) p->k[((t0 + c0 + (r)) * p->hk + hq) * dk + (c)]
+#define BQ(r, c) p->q[((t0 + c0 + (r)) * p->hk + hq) * dk + (c)]
+#define BV(r, i) p->v[((t0 + c0 + (r)) * p->hv + h) * dv + (i)]
+#define BB(r) p->beta[(t0 + c0 + (r)) * p->hv + h]
+#define BG(r) p->g[(t0 + c0 + (r)) * p->hv + h]
+    /* forward over chunks: the start state of every chunk */
+    if (p->s0) memcpy(S0s, p->s0 + unit * (int64_t)ssz, sizeof(double) * ssz);
+    else memset(S0s, 0, sizeof(double) * ssz);
+    for (int64_t c = 0; c < nch; ++c) {
+        const int64_t c0 = c * C;
+        const double *S = S0s + ssz * c;
+        double *Sn = S0s + ssz * (c + 1);
+        const int L = (int)((T - c0) < C ? (T - c0) : C);
+        memcpy(Sn, S, sizeof(double) * ssz);
+        for (int t = 0; t < L; ++t) { /* the token recurrence within the chunk */
+            const double alpha = exp(BG(t)), beta = BB(t);
+            for (int i = 0; i < dv; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < dk; ++j) acc += alpha * Sn[i * dk + j] * BK(t, j);
+                const double ui = beta * (BV(t, i) - acc);
+                for (int j = 0; j < dk; ++j) Sn[i * dk + j] = alpha * Sn[i * dk + j] + ui * BK(t, j);
+            }
+        }
+    }
+    if (gr->dSf) memcpy(dS, gr->dSf + unit * (int64_t)ssz, sizeof(double) * ssz);
+    else memset(dS, 0, sizeof(double) * ssz);
+    for (int64_t c = nch - 1; c >= 0; --c) {
+        const int64_t c0 = c * C;
+        const double *S0 = S0s + ssz * c;
+        const int L = (int)((T - c0) < C ? (T - c0) : C);
+        /* the chunk's forward quantities */
+        for (int r = 0; r < L; ++r) G[r] = (r ? G[r - 1] : 0.0) + BG(r);
+        for (int r = 0; r < L; ++r) {
+            gam[r] = exp(G[r]);
+            lam[r] = exp(G[L - 1] - G[r]);
+        }
+        const double gL = exp(G[L - 1]);
+        for (int r = 0; r < L; ++r)
+            for (int j = 0; j < L; ++j) {
+                double kk = 0.0, qk = 0.0;
+                for (int x = 0; x < dk; ++x) {
+                    kk += BK(r, x) * BK(j, x);
+                    qk += BQ(r, x) * BK(j, x);
+                }
+                KK[r * L + j] = kk;
+                QK[r * L + j] = qk;
+                Gm[r * L + j] = j <= r ? exp(G[r] - G[j]) : 0.0;
+                A[r * L + j] = j < r ? BB(r) * Gm[r * L + j] * kk : 0.0;
+            }
+        for (int col = 0; col < L; ++col)
+            for (int r = 0; r < L; ++r) {
+                double x = (r == col) ? 1.0 : 0.0;
+                for (int j = col; j < r; ++j) x -= A[r * L + j] * Tm[j * L + col];
+                Tm[r * L + col] = r < col ? 0.0 : x;
+            }
+        for (int r = 0; r < L; ++r) {
+            for (int x = 0; x < dk; ++x) {
+                double acc = 0.0;
+                for (int j = 0; j <= r; ++j) acc += Tm[r * L + j] * BB(j) * gam[j] * BK(j, x);
+                W[r * dk + x] = acc;
+            }
+            for (int i = 0; i < dv; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j <= r; ++j) acc += Tm[r * L + j] * BB(j) * BV(j, i);
+                for (int x = 0; x < dk; ++x) acc -= W[r * dk + x] * S0[i * dk + x];
+                U[r * dv + i] = acc;
+            }
+        }
+        for (int r = 0; r < L; ++r) {
+            dgam[r] = dlam[r] = dbg[r] = dbeta[r] = 0.0;
+            for (int x = 0; x < dk; ++x) dQ[r * dk + x] = dK[r * dk + x] = 0.0;
+        }
+        for (int e = 0; e < L * L; ++e) dGam[e] = dT[e] = 0.0;
+        /* S_C = gL S0 + U^T diag(lambda) K */
+        double dgL = 0.0;
+        for (size_t e = 0; e < ssz; ++e) {
+            dS0[e] = gL * dS[e];
+            dgL += dS[e] * S0[e];
+        }
+        for (int j = 0; j < L; ++j) {
+            double dl = 0.0;
+            for (int i = 0; i < dv; ++i) {
+                double dsk = 0.0;
+                for (int x = 0; x < dk; ++x) dsk += dS[i * dk + x] * BK(j, x);
+                dU[j * dv + i] = lam[j] * dsk;
+                dl += U[j * dv + i] * dsk;
+            }
+            dlam[j] = dl;
+            for (int x = 0; x < dk; ++x) {
+                double acc = 0.0;
+                for (int i = 0; i < dv; ++i) acc += dS[i * dk + x] * U[j * dv + i];
+                dK[j * dk + x] += lam[j] * acc;
+            }
+        }
+        /* O = diag(gamma) Q S0^T + P U */
+        for (int r = 0; r < L; ++r) {
+            const double *dOr = gr->dO + ((t0 + c0 + r) * p->hv + h) * dv;
+            for (int x = 0; x < dk; ++x) {
+                double acc = 0.0;
+                for (int i = 0; i < dv; ++i) {
+                    acc += dOr[i] * S0[i * dk + x];
+                    dS0[i * dk + x] += dOr[i] * gam[r] * BQ(r, x);
+                }
+                dQ[r * dk + x] += gam[r] * acc;
+                dgam[r] += acc * BQ(r, x);
+            }
+            for (int j = 0; j <= r; ++j) {
+                const double Prj = Gm[r * L + j] * QK[r * L + j];
+                double dP = 0.0;
+                for (int i = 0; i < dv; ++i) {
+                    dU[j * dv + i] += Prj * dOr[i];
+                    dP += dOr[i] * U[j * dv + i];
+                }
+                /* P_rj = Gamma_rj (q_r . k_j) */
+                for (int x = 0; x < dk; ++x) {
+                    dQ[r * dk + x] += dP * Gm[r * L + j] * BK(j, x);
+                    dK[j * dk + x] += dP * Gm[r * L + j] * BQ(r, x);
+                }
+                dGam[r * L + j] += dP * QK[r * L + j];
+            }
+        }
+        /* U = U~ - W S0^T;  W = T diag(beta gamma) K;  U~ = T diag(beta) V */
+        for (int r = 0; r < L; ++r)
+            for (int x = 0; x < dk; ++x) {
+                double acc = 0.0;
+                for (int i = 0; i < dv; ++i) {
+                    acc -= dU[r * dv + i] * S0[i * dk + x];
+                    dS0[i * dk + x] -= dU[r * dv + i] * W[r * dk + x];
+                }
+                dW[r * dk + x] = acc;
+            }
+        for (int r = 0; r < L; ++r)
+            for (int j = 0; j <= r; ++j) {
+                double acc = 0.0;
+                for (int x = 0; x < dk; ++x) acc += dW[r * dk + x] * BB(j) * gam[j] * BK(j, x);
+                for (int i = 0; i < dv; ++i) acc += dU[r * dv + i] * BB(j) * BV(j, i);
+                dT[r * L + j] = acc;
+            }
+        for (int j = 0; j < L; ++j) {
+            /* dX_j = (T^T dW)_j, dY_j = (T^T dU~)_j */
+            for (int x = 0; x < dk; ++x) {
+                double dx = 0.0;
+                for (int r = j; r < L; ++r) dx += Tm[r * L + j] * dW[r * dk + x];
+                dK[j * dk + x] += BB(j) * gam[j] * dx;
+                dbg[j] += dx * BK(j, x);
+            }
+            double *dvj = gr->dv + ((t0 + c0 + j) * p->hv + h) * dv;
+            for (int i = 0; i < dv; ++i) {
+                double dy = 0.0;
+                for (int r = j; r < L; ++r) dy += Tm[r * L + j] * dU[r * dv + i];
+                dvj[i] = BB(j) * dy;
+                dbeta[j] += dy * BV(j, i);
+            }
+        }
+        /* T = (I + A)^-1: dA = -T^T dT T^T, strictly lower */
+        for (int r = 0; r < L; ++r)
+            for (int j = 0; j < L; ++j) {
+                double acc = 0.0;
+                for (int m = 0; m < L; ++m) acc += dT[r * L + m] * Tm[j * L + m]; /* (dT T^T)_rj */
+                tmp[r * L + j] = acc;
+            }
+        for (int r = 0; r < L; ++r)
+            for (int j = 0; j < L; ++j) {
+                double acc = 0.0;
+                if (j < r)
+                    for (int m = 0; m < L; ++m) acc += Tm[m * L + r] * tmp[m * L + j]; /* (T^T (dT T^T))_rj */
+                dA[r * L + j] = -acc;
+            }
+        /* A_rj = beta_r Gamma_rj (k_r . k_j), j < r */
+        for (int r = 0; r < L; ++r)
+            for (int j = 0; j < r; ++j) {
+                const double da = dA[r * L + j];
+                dbeta[r] += da * Gm[r * L + j] * KK[r * L + j];
+                dGam[r * L + j] += da * BB(r) * KK[r * L + j];
+                const double dkk = da * BB(r) * Gm[r * L + j];
+                for (int x = 0; x < dk; ++x) {
+                    dK[r * dk + x] += dkk * BK(j, x);
+                    dK[j * dk + x] += dkk * BK(r, x);
+                }
+            }
+        /* the decays through G */
+        for (int r = 0; r < L; ++r) {
+            dbeta[r] += dbg[r] * gam[r];
+            dgam[r] += dbg[r] * BB(r);
+        }
+        for (int r = 0; r < L; ++r) dG[r] = dgam[r] * gam[r] - dlam[r] * lam[r];
+        dG[L - 1] += dgL * gL;
+        for (int j = 0; j < L; ++j) dG[L - 1] += dlam[j] * lam[j];
+        for (int r = 0; r < L; ++r)
+            for (int j = 0; j <= r; ++j) {
+                const double e = dGam[r * L + j] * Gm[r * L + j];
+                dG[r] += e;
+                dG[j] -= e;
+            }
+        double run = 0.0;
+        for (int t = L - 1; t >= 0; --t) {
+            run += dG[t];
+            const int64_t tt = t0 + c0 + t;
+            gr->dg[tt * p->hv + h] = run;
+            gr->dbeta[tt * p->hv + h] = dbeta[t];
+            memcpy(gr->dq + (tt * p->hv + h) * dk, dQ + t * dk, sizeof(double) * dk);
+            memcpy(gr->dk + (tt * p->hv + h) * dk, dK + t * dk, sizeof(double) * dk);
+        }
+        memcpy(dS, dS0, sizeof(double) * ssz);
+    }
+#undef BK
+#undef BQ
+#undef BV
+#undef BB
+#undef BG
+    if (gr->dS0) memcpy(gr->dS0 + unit * (int64_t)ssz, dS, sizeof(double) * ssz);
+done:
+    free(S0s); free(dS); free(dS0); free(G); free(gam); free(lam); free(A); free(Tm); free(Gm); free(KK); free(QK);
+    free(W); free(U); free(dU); free(dW); free(dT); free(dA); free(tmp); free(dGam); free(dQ); free(dK); free(dG);
+    free(dgam); free(dlam); free(dbg); free(dbeta);
+    return rc;
+}
+
+int gdn_oracle_backward_chunkwise(const gdn_oracle_problem *p, const gdn_oracle_grads *gr, int32_t chunk,
+                                  int n_threads) {
+    if (chunk <= 0) return -1;
+    return run_backward(p, gr, chunk, n_threads);
+}
+
 /* KDA: the problem's g is [T, Hv, d_k] (one log-decay per key channel). */
 int gdn_oracle_kda_recurrent(const gdn_oracle_problem *p, const int64_t *units, int64_t n_units, int n_threads) {
     return run(KIND_KDA, p, NULL, units, n_units, n_threads);

@@ -61,6 +61,10 @@ class _ChunkOut(ctypes.Structure):
     ]
 
 
+class _Grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.POINTER(ctypes.c_double)) for n in ("dO", "dSf", "dq", "dk", "dv", "dg", "dbeta", "dS0")]
+
+
 def load(path: str | None = None):
     """Load (building first if needed) the oracle library; cached per process."""
     global _lib
@@ -89,6 +93,11 @@ def load(path: str | None = None):
         lib.gdn_oracle_output_side.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, D, D, D,
                                                ctypes.c_double, ctypes.c_uint32, D]
         lib.gdn_oracle_output_side.restype = None
+        GP = ctypes.POINTER(_Grads)
+        lib.gdn_oracle_backward.argtypes = [P, GP, ctypes.c_int]
+        lib.gdn_oracle_backward.restype = ctypes.c_int
+        lib.gdn_oracle_backward_chunkwise.argtypes = [P, GP, ctypes.c_int32, ctypes.c_int]
+        lib.gdn_oracle_backward_chunkwise.restype = ctypes.c_int
         lib.gdn_oracle_kda_recurrent.argtypes = [P, U, ctypes.c_int64, ctypes.c_int]
         lib.gdn_oracle_kda_recurrent.restype = ctypes.c_int
         lib.gdn_oracle_kda_chunkwise.argtypes = [P, ctypes.c_int32, U, ctypes.c_int64, ctypes.c_int]
@@ -365,4 +374,42 @@ def decode_multi(q, k, v, g, beta, state, threads=None, lib=None):
         o[:, j], S = decode_step(q[:, j], k[:, j], v[:, j], g[:, j], beta[:, j], S, threads=threads, lib=lib)
         snaps[:, j] = S
     return o, snaps
+
+
+def backward(q, k, v, g, beta, dO, dS_final=None, initial_state=None, cu_seqlens=None, chunk=None, threads=None,
+             lib=None):
+    """Gradients of L = sum dO . o + sum dS_final . S_final with respect to
+    q, k, v, g, beta and the initial state (``gdn_oracle_backward``: reverse
+    mode of the token recurrence; with ``chunk``: ``gdn_oracle_backward_chunkwise``,
+    the chunked form differentiated).  Returns a dict of fp64 arrays shaped
+    like the inputs: dq, dk (summed over the value heads of each q/k group),
+    dv, dg, dbeta, dS0."""
+    q, k, v, g, beta, s0, cu, batched, dims = _prepare(q, k, v, g, beta, initial_state, cu_seqlens)
+    N, Ttot, hk, hv, dk, dv = dims
+    dO64 = np.ascontiguousarray(_f64(dO).reshape(Ttot, hv, dv))
+    dSf = None if dS_final is None else np.ascontiguousarray(_f64(dS_final).reshape(N, hv, dv, dk))
+    out = {"dq": np.zeros((Ttot, hv, dk)), "dk": np.zeros((Ttot, hv, dk)), "dv": np.zeros((Ttot, hv, dv)),
+           "dg": np.zeros((Ttot, hv)), "dbeta": np.zeros((Ttot, hv)), "dS0": np.zeros((N, hv, dv, dk))}
+    gr = _Grads(_dptr(dO64), _dptr(dSf), _dptr(out["dq"]), _dptr(out["dk"]), _dptr(out["dv"]), _dptr(out["dg"]),
+                _dptr(out["dbeta"]), _dptr(out["dS0"]))
+    prob = _problem(q, k, v, g, beta, s0, cu, None, None, dims)
+    L = lib or load()
+    if chunk is None:
+        rc = L.gdn_oracle_backward(ctypes.byref(prob), ctypes.byref(gr), threads or default_threads())
+    else:
+        rc = L.gdn_oracle_backward_chunkwise(ctypes.byref(prob), ctypes.byref(gr), ctypes.c_int32(chunk),
+                                             threads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"oracle backward failed ({rc})")
+    G = hv // hk
+    for n in ("dq", "dk"):
+        out[n] = out[n].reshape(Ttot, hk, G, dk).sum(axis=2)
+    if batched is not None:
+        B, T = batched
+        out["dq"] = out["dq"].reshape(B, T, hk, dk)
+        out["dk"] = out["dk"].reshape(B, T, hk, dk)
+        out["dv"] = out["dv"].reshape(B, T, hv, dv)
+        out["dg"] = out["dg"].reshape(B, T, hv)
+        out["dbeta"] = out["dbeta"].reshape(B, T, hv)
+    return out
 

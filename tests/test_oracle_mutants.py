@@ -78,6 +78,16 @@ MUTANTS = [
      "acc += S[i * dk + c] * KDA_Q(r, c) * exp(G[r * dk + c]);", "acc += S[i * dk + c] * KDA_Q(r, c);"),
     ("KDA chunk end state without the decay of the writes",
      "acc += U[j * dv + i] * KDA_K(j, c) * exp(Gl[c] - G[j * dk + c]);", "acc += U[j * dv + i] * KDA_K(j, c);"),
+    ("backward: decay gradient without alpha",
+     "gr->dg[tt * p->hv + h] = alpha * dalpha;", "gr->dg[tt * p->hv + h] = dalpha;"),
+    ("backward: carried state gradient not decayed",
+     "for (size_t e = 0; e < ssz; ++e) dS[e] = alpha * dsp[e];", "for (size_t e = 0; e < ssz; ++e) dS[e] = dsp[e];"),
+    ("backward: key gradient without the write term",
+     "dkt[j] += u[i] * dS[i * dk + j] + dpi * alpha * Sp[i * dk + j];", "dkt[j] += dpi * alpha * Sp[i * dk + j];"),
+    ("backward chunked: inverse gradient with the wrong sign",
+     "dA[r * L + j] = -acc;", "dA[r * L + j] = acc;"),
+    ("backward chunked: end-state decay gradient dropped",
+     "dG[L - 1] += dgL * gL;", "dG[L - 1] += 0.0 * dgL;"),
     ("A built with Gamma transposed",
      "a = p->beta[(c0 + r) * p->hv + h] * exp(G[r] - G[j]) * kk;",
      "a = p->beta[(c0 + r) * p->hv + h] * exp(G[j] - G[r]) * kk;"),
@@ -108,6 +118,9 @@ class _Bound:
     def output_side(self, *a, **kw):
         return oracle.output_side(*a, lib=self.lib, **kw)
 
+    def backward(self, *a, **kw):
+        return oracle.backward(*a, lib=self.lib, **kw)
+
     def kda_recurrent(self, *a, **kw):
         return oracle.kda_recurrent(*a, lib=self.lib, **kw)
 
@@ -136,6 +149,8 @@ def _pin_calls(m):
         lambda: pins.test_kda_beta_zero_is_channel_decay(m),
         lambda: pins.test_kda_one_token(m),
         lambda: pins.test_kda_chunkwise_equals_recurrent(m, 4),
+        lambda: pins.test_backward_matches_finite_differences(m),
+        lambda: pins.test_backward_chunkwise_equals_token_recurrence(m, 4),
     ]
 
 

@@ -507,3 +507,79 @@ def test_kda_chunkwise_equals_recurrent(oracle_mod, C):
     o4, s4 = oracle_mod.kda_chunkwise(q[0], k[0], v[0], gk[0], beta[0], C, initial_state=s0v, cu_seqlens=cu)
     assert np.allclose(o3, o4, rtol=1e-11, atol=1e-13) and np.allclose(s3, s4, rtol=1e-11, atol=1e-13)
     assert np.array_equal(s3[0], s0v[0])  # the empty sequence keeps its state
+
+
+def _fd_grads(oracle_mod, args, dO, dSf, names, h=1e-6, cu=None):
+    """Central finite differences of L = sum dO . o + sum dSf . S_T through the
+    (pinned) forward recurrence."""
+    def loss(a):
+        o, sf = oracle_mod.recurrent(a["q"], a["k"], a["v"], a["g"], a["beta"], initial_state=a["s0"], cu_seqlens=cu)
+        return float((o * dO).sum() + (sf * dSf).sum())
+    out = {}
+    for name in names:
+        x = args[name]
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            ap, am = dict(args), dict(args)
+            ap[name] = x.copy()
+            am[name] = x.copy()
+            ap[name][idx] += h
+            am[name][idx] -= h
+            fd[idx] = (loss(ap) - loss(am)) / (2 * h)
+        out[name] = fd
+    return out
+
+
+def test_backward_matches_finite_differences(oracle_mod):
+    """Every gradient of the hand-written reverse recurrence against central
+    differences of the forward recurrence (grouped heads, a start state,
+    unnormalised keys)."""
+    rng = np.random.default_rng(60)
+    T, hk, hv, d = 7, 1, 2, 3
+    q, k, v, g, beta, S0 = _rand_problem(rng, T, hk, hv, d, d, unit_keys=False)
+    k *= 0.6
+    dO = rng.standard_normal(v.shape)
+    dSf = rng.standard_normal(S0.shape)
+    gr = oracle_mod.backward(q, k, v, g, beta, dO, dSf, initial_state=S0)
+    args = dict(q=q, k=k, v=v, g=g, beta=beta, s0=S0)
+    fd = _fd_grads(oracle_mod, args, dO, dSf, list(args))
+    for name, key in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("g", "dg"), ("beta", "dbeta"), ("s0", "dS0")):
+        ref = fd[name]
+        got = gr[key].reshape(ref.shape)
+        assert np.allclose(got, ref, rtol=1e-6, atol=1e-7), (name, np.abs(got - ref).max())
+
+
+def test_backward_varlen_finite_differences(oracle_mod):
+    """Packed sequences (one empty): gradients stay inside their sequence and
+    an empty sequence passes dS_final straight to dS0."""
+    rng = np.random.default_rng(61)
+    lens = [3, 0, 4]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    T, hk, hv, d = sum(lens), 1, 1, 3
+    q, k, v, g, beta, _ = _rand_problem(rng, T, hk, hv, d, d, s0=False)
+    q, k, v, g, beta = q[0], k[0], v[0], g[0], beta[0]
+    S0 = 0.3 * rng.standard_normal((3, hv, d, d))
+    dO = rng.standard_normal(v.shape)
+    dSf = rng.standard_normal(S0.shape)
+    gr = oracle_mod.backward(q, k, v, g, beta, dO, dSf, initial_state=S0, cu_seqlens=cu)
+    args = dict(q=q, k=k, v=v, g=g, beta=beta, s0=S0)
+    fd = _fd_grads(oracle_mod, args, dO, dSf, ["k", "g", "s0"], cu=cu)
+    assert np.allclose(gr["dk"], fd["k"], rtol=1e-6, atol=1e-7)
+    assert np.allclose(gr["dg"], fd["g"], rtol=1e-6, atol=1e-7)
+    assert np.allclose(gr["dS0"], fd["s0"], rtol=1e-6, atol=1e-7)
+    assert np.array_equal(gr["dS0"][1], dSf[1])
+
+
+@pytest.mark.parametrize("C", [1, 4, 16])
+def test_backward_chunkwise_equals_token_recurrence(oracle_mod, C):
+    """The chunked form differentiated (matrix calculus through the WY
+    inverse and the decay masks) against the token recurrence's reverse
+    mode: two derivations of the same gradients."""
+    rng = np.random.default_rng(62)
+    q, k, v, g, beta, S0 = _rand_problem(rng, 37, 2, 4, 8, 8, g_scale=2.0)
+    dO = rng.standard_normal(v.shape)
+    dSf = rng.standard_normal(S0.shape)
+    a = oracle_mod.backward(q, k, v, g, beta, dO, dSf, initial_state=S0)
+    b = oracle_mod.backward(q, k, v, g, beta, dO, dSf, initial_state=S0, chunk=C)
+    for n in a:
+        assert np.allclose(a[n], b[n], rtol=1e-10, atol=1e-11), (n, np.abs(a[n] - b[n]).max())
