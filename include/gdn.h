@@ -327,6 +327,37 @@ GDN_API gdn_status_t gdn_decode_commit(int32_t num_seqs, int32_t num_tokens, int
                                int32_t head_dim_k, int32_t head_dim_v, const float *snapshots,
                                const int32_t *accepted, float *state, int32_t *bad_count, void *stream);
 
+/* Gradients for training ("Architecture Thread I", the Gated DeltaNet
+ * section, and "Gated Attention Architectures", sections 2 and 3: the
+ * chunked form is how the layer is trained).  For the upstream gradients
+ * d_o (of o) and d_final_state (of the final states; NULL = zero), writes
+ * the gradients of L = sum d_o . o + sum d_final_state . S_final:
+ *   dq, dk             [tokens, Hk, d_k] fp32 (summed over the value heads
+ *                      of each q/k group)
+ *   dv                 [tokens, Hv, d_v] fp32
+ *   dg, dbeta          [tokens, Hv] fp32 (dg is zero where g < -20, the
+ *                      kernels' floor on g)
+ *   d_initial_state    [N, Hv, d_v, d_k] fp32, or NULL
+ * Inputs are those of gdn_chunk_forward (the plain path: no input-side
+ * flags, GDN_ERR_UNSUPPORTED otherwise); d_o has the dtype of v.  fp32 on
+ * CUDA cores: the forward chunk states are recomputed and kept in the
+ * workspace (one d_v x d_k state per 32-token chunk and value head, plus
+ * the schedule; gdn_chunk_backward_workspace_size), then the chunks are
+ * walked backward.  dq, dk, dg and dbeta are accumulated with atomic adds
+ * (their summation order, and so their last bits, can vary between runs).
+ * d_k, d_v <= 128. */
+GDN_API gdn_status_t gdn_chunk_backward_workspace_size(const gdn_shape_t *shape, size_t *bytes);
+GDN_API gdn_status_t gdn_chunk_backward(const gdn_shape_t *shape,
+                                const void *q, const void *k, const void *v,
+                                const float *g, const float *beta,
+                                const float *initial_state,
+                                const int32_t *cu_seqlens,
+                                const void *d_o, const float *d_final_state,
+                                float *dq, float *dk, float *dv, float *dg, float *dbeta,
+                                float *d_initial_state,
+                                void *workspace, size_t workspace_bytes,
+                                void *stream);
+
 /* Static text for a status code. */
 GDN_API const char *gdn_status_string(gdn_status_t status);
 

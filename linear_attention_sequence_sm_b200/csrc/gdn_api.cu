@@ -367,3 +367,92 @@ gdn_status_t gdn_decode_commit(int32_t n, int32_t ntok, int32_t hv, int32_t dk, 
 }
 
 }  // extern "C"
+
+extern "C" {
+
+static size_t bwd_sched_bytes(const gdn_shape_t *s) { return (ws_layout(s->num_seqs).total + 255) / 256 * 256; }
+
+gdn_status_t gdn_chunk_backward_workspace_size(const gdn_shape_t *s, size_t *bytes) {
+    g_msg[0] = 0;
+    if (!bytes) return fail(GDN_ERR_INVALID_ARGUMENT, "bytes is NULL");
+    gdn_status_t st = check_shape(s);
+    if (st != GDN_OK) return st;
+    const int64_t tokens = int64_t(s->batch) * s->seq_len;
+    *bytes = bwd_sched_bytes(s) +
+             backward_ckpt_bytes(int32_t(tokens), s->num_seqs, s->num_v_heads, s->head_dim_k, s->head_dim_v);
+    return GDN_OK;
+}
+
+gdn_status_t gdn_chunk_backward(const gdn_shape_t *s, const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, const float *initial_state, const int32_t *cu_seqlens,
+                                const void *d_o, const float *d_final_state, float *dq, float *dk, float *dv,
+                                float *dg, float *dbeta, float *d_initial_state, void *workspace,
+                                size_t workspace_bytes, void *stream_) {
+    g_msg[0] = 0;
+    gdn_status_t st = check_shape(s);
+    if (st != GDN_OK) return st;
+    if (s->flags & (GDN_FLAG_QK_L2NORM | GDN_FLAG_GATE_LOGITS))
+        return fail(GDN_ERR_UNSUPPORTED, "the backward takes prepared inputs (no input-side flags)");
+    const int64_t tokens = int64_t(s->batch) * s->seq_len;
+    if (cu_seqlens) {
+        if (s->batch != 1) return fail(GDN_ERR_INVALID_ARGUMENT, "batch must be 1 with cu_seqlens");
+    } else if (s->num_seqs != s->batch) {
+        return fail(GDN_ERR_INVALID_ARGUMENT, "num_seqs (%d) must equal batch (%d) without cu_seqlens",
+                    s->num_seqs, s->batch);
+    }
+    if (tokens > 0 && (!q || !k || !v || !g || !beta || !d_o || !dq || !dk || !dv || !dg || !dbeta))
+        return fail(GDN_ERR_INVALID_ARGUMENT, "inputs, d_o and the gradient outputs must be non-NULL");
+    if (!workspace) return fail(GDN_ERR_INVALID_ARGUMENT, "workspace is NULL");
+    size_t need = 0;
+    gdn_chunk_backward_workspace_size(s, &need);
+    if (workspace_bytes < need)
+        return fail(GDN_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+    const void *ptrs[] = {q, k, v, g, beta, initial_state, cu_seqlens, d_o, d_final_state, dq, dk, dv, dg, dbeta,
+                          d_initial_state};
+    const char *names[] = {"q", "k", "v", "g", "beta", "initial_state", "cu_seqlens", "d_o", "d_final_state",
+                           "dq", "dk", "dv", "dg", "dbeta", "d_initial_state"};
+    for (int i = 0; i < 15; ++i)
+        if (ptrs[i] && !aligned16(ptrs[i])) return fail(GDN_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(GDN_ERR_MISALIGNED, "workspace is not 256-byte aligned");
+    int major = 0;
+    if (device_sm_count(&major) <= 0) return fail(GDN_ERR_CUDA, "no usable CUDA device");
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    cudaError_t e = launch_schedule(*s, cu_seqlens, workspace, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "schedule kernel launch");
+    if (tokens > 0) {
+        const size_t qk = size_t(tokens) * s->num_qk_heads * s->head_dim_k * sizeof(float);
+        const size_t gb = size_t(tokens) * s->num_v_heads * sizeof(float);
+        if ((e = cudaMemsetAsync(dq, 0, qk, stream)) != cudaSuccess ||
+            (e = cudaMemsetAsync(dk, 0, qk, stream)) != cudaSuccess ||
+            (e = cudaMemsetAsync(dg, 0, gb, stream)) != cudaSuccess ||
+            (e = cudaMemsetAsync(dbeta, 0, gb, stream)) != cudaSuccess)
+            return cuda_fail(e, "clearing the gradient accumulators");
+    }
+    const WsLayout L = ws_layout(s->num_seqs);
+    PrefillArgs a;
+    a.num_seqs = s->num_seqs;
+    a.hk = s->num_qk_heads;
+    a.hv = s->num_v_heads;
+    a.dk = s->head_dim_k;
+    a.dv = s->head_dim_v;
+    a.chunk = s->chunk_size;
+    a.dtype = s->dtype;
+    a.tokens = int32_t(tokens);
+    a.flags = 0;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.s0 = initial_state; a.o = nullptr; a.s_final = nullptr;
+    a.out = OutSide{nullptr, nullptr, 0.f, 0u};
+    char *ws = static_cast<char *>(workspace);
+    a.sched.hdr = reinterpret_cast<WsHeader *>(ws);
+    a.sched.order = reinterpret_cast<const int32_t *>(ws + L.order_off);
+    a.sched.start = reinterpret_cast<const int32_t *>(ws + L.start_off);
+    a.sched.len = reinterpret_cast<const int32_t *>(ws + L.len_off);
+    if (s->num_seqs == 0) return GDN_OK;
+    float *ckpt = reinterpret_cast<float *>(ws + bwd_sched_bytes(s));
+    e = launch_chunk_backward(a, d_o, d_final_state, dq, dk, dv, dg, dbeta, d_initial_state, ckpt, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+    return GDN_OK;
+}
+
+}  // extern "C"
+

@@ -1,0 +1,469 @@
+// gdn_backward.cu -- gradients of the chunked gated delta rule (training),
+// fp32 on CUDA cores.
+//
+// The pages present the chunked form as the way to train the layer
+// ("Architecture Thread I", the Gated DeltaNet section; "Gated Attention
+// Architectures", sections 2 and 3).  For upstream gradients dO and dS_T,
+// the kernel returns the gradients of L = sum dO . O + sum dS_T . S_T with
+// respect to q, k, v, g, beta and the initial state.
+//
+// Per chunk of C tokens with start state S0 (G, gamma, Gamma, lambda, A, T,
+// W, U~, U, P as in the forward):
+//   S_C = gamma_L S0 + U^T diag(lambda) K,  O = diag(gamma) Q S0^T + P U,
+//   U = U~ - W S0^T,  W = T diag(beta gamma) K,  U~ = T diag(beta) V,
+//   T = (I + A)^-1,  A = strict(diag(beta)(K K^T (.) Gamma)),  P = Q K^T (.) Gamma.
+// Reverse mode through these, for the chunk's end-state gradient dS:
+//   dS0 = gamma_L dS + dO^T diag(gamma) Q - dU^T W        (the previous chunk's dS)
+//   dU = diag(lambda) K dS^T + P^T dO,   dP = dO U^T (lower, with diagonal)
+//   dW = -dU S0,  dT = dW (diag(bg) K)^T + dU (diag(beta) V)^T,  dA = -T^T dT T^T
+//   dq, dk, dv, dbeta from the products; dg from the decays through the prefix sums G.
+// Every row slice of d_v enters dS, dU, dv and dS0 alone, and dq, dk, dbeta
+// and dg linearly, so a block owns (sequence, value head, 32 rows of d_v)
+// and adds its share of the shared gradients with atomics.
+//
+// Pass 1 runs the chunks forward and stores each chunk's start state (the
+// block's rows) in the workspace; pass 2 walks the chunks backward,
+// recomputing the chunk's forward quantities from its stored start state.
+#include "gdn_internal.cuh"
+
+namespace gdn {
+
+constexpr int kBwdThreads = 256;
+constexpr int kBwdC = 32;    // tokens per chunk
+constexpr int kBwdRows = 32; // rows of d_v per block
+
+struct BwdSmem {
+    int ldk, ldc, ldv;
+    size_t k, q, w, dw, dq, dk, s0, ds, v, u, du, dO, t, gm, kk, qk, dt, da, vec, total;
+};
+
+__host__ __device__ inline BwdSmem bwd_smem(int dk) {
+    BwdSmem s;
+    s.ldk = dk + 1;
+    s.ldc = kBwdC + 1;
+    s.ldv = kBwdRows + 1;
+    size_t off = 0;
+    auto take = [&](size_t n) { size_t o = off; off += n; return o; };
+    s.k = take(size_t(kBwdC) * s.ldk);
+    s.q = take(size_t(kBwdC) * s.ldk);
+    s.w = take(size_t(kBwdC) * s.ldk);
+    s.dw = take(size_t(kBwdC) * s.ldk);
+    s.dq = take(size_t(kBwdC) * s.ldk);
+    s.dk = take(size_t(kBwdC) * s.ldk);
+    s.s0 = take(size_t(kBwdRows) * s.ldk);
+    s.ds = take(size_t(kBwdRows) * s.ldk);
+    s.v = take(size_t(kBwdC) * s.ldv);
+    s.u = take(size_t(kBwdC) * s.ldv);
+    s.du = take(size_t(kBwdC) * s.ldv);
+    s.dO = take(size_t(kBwdC) * s.ldv);
+    s.t = take(size_t(kBwdC) * s.ldc);
+    s.gm = take(size_t(kBwdC) * s.ldc);
+    s.kk = take(size_t(kBwdC) * s.ldc);
+    s.qk = take(size_t(kBwdC) * s.ldc);
+    s.dt = take(size_t(kBwdC) * s.ldc);
+    s.da = take(size_t(kBwdC) * s.ldc);
+    s.vec = take(size_t(16) * kBwdC);
+    s.total = off;
+    return s;
+}
+
+// per-token vectors inside the vec block
+enum { kVG = 0, kVGam, kVLam, kVB, kVBG, kVDG, kVDGam, kVDLam, kVDBG, kVDB, kVNum };
+
+// checkpoint slot of chunk c of the sequence starting at token t0, sequence n:
+// floor(t0 / C) + n + c never collides between sequences
+__device__ __forceinline__ size_t bwd_slot(int t0, int n, int c) { return size_t(t0 / kBwdC + n + c); }
+
+template <typename T>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, float *dq, float *dk, float *dv,
+                      float *dg, float *dbeta, float *dS0_out, float *ckpt, int n_slices) {
+    if (a.sched.hdr->status != GDN_OK) return;
+    extern __shared__ float smem[];
+    const int dkd = a.dk, dvd = a.dv, hv = a.hv, hk = a.hk;
+    const BwdSmem L = bwd_smem(dkd);
+    const int ldk = L.ldk, ldc = L.ldc, ldv = L.ldv;
+    float *K = smem + L.k, *Q = smem + L.q, *W = smem + L.w, *dW = smem + L.dw, *dQ = smem + L.dq,
+          *dK = smem + L.dk, *S0 = smem + L.s0, *dS = smem + L.ds, *V = smem + L.v, *U = smem + L.u,
+          *dU = smem + L.du, *dOs = smem + L.dO, *Tm = smem + L.t, *Gm = smem + L.gm, *KK = smem + L.kk,
+          *QK = smem + L.qk, *dT = smem + L.dt, *dA = smem + L.da, *vec = smem + L.vec;
+    float *vG = vec + kVG * kBwdC, *vGam = vec + kVGam * kBwdC, *vLam = vec + kVLam * kBwdC,
+          *vB = vec + kVB * kBwdC, *vBG = vec + kVBG * kBwdC, *vdG = vec + kVDG * kBwdC,
+          *vdGam = vec + kVDGam * kBwdC, *vdLam = vec + kVDLam * kBwdC, *vdBG = vec + kVDBG * kBwdC,
+          *vdB = vec + kVDB * kBwdC;
+    __shared__ float red[kBwdThreads / 32];
+    const int tid = threadIdx.x;
+    const T *q = static_cast<const T *>(a.q);
+    const T *k = static_cast<const T *>(a.k);
+    const T *v = static_cast<const T *>(a.v);
+    const T *dO = static_cast<const T *>(dO_);
+
+    const int blk = blockIdx.x;
+    const int rank = blk / (hv * n_slices);
+    const int h = (blk / n_slices) % hv;
+    const int slice = blk % n_slices;
+    const int seq = a.sched.order[rank];
+    const int t0 = a.sched.start[seq], len = a.sched.len[seq];
+    const int hq = h / (hv / hk);
+    const int i0 = slice * kBwdRows;
+    const int nr = min(kBwdRows, dvd - i0);
+    const size_t sbase = (size_t(seq) * hv + h) * size_t(dvd) * dkd;
+    const int nch = (len + kBwdC - 1) / kBwdC;
+    auto ck = [&](int c) { return ckpt + (bwd_slot(t0, seq, c) * hv + h) * size_t(dvd) * dkd + size_t(i0) * dkd; };
+
+    // one chunk's inputs and forward quantities (A, T, W, U~, U; the masks)
+    auto chunk_forward = [&](int c, int Lc) {
+        const int c0 = t0 + c * kBwdC;
+        for (int idx = tid; idx < kBwdC * dkd; idx += kBwdThreads) {
+            const int r = idx / dkd, x = idx % dkd;
+            const bool ok = r < Lc;
+            K[r * ldk + x] = ok ? to_f32(k[(size_t(c0 + r) * hk + hq) * dkd + x]) : 0.f;
+            Q[r * ldk + x] = ok ? to_f32(q[(size_t(c0 + r) * hk + hq) * dkd + x]) : 0.f;
+        }
+        for (int idx = tid; idx < kBwdC * kBwdRows; idx += kBwdThreads) {
+            const int r = idx / kBwdRows, i = idx % kBwdRows;
+            V[r * ldv + i] = (r < Lc && i < nr) ? to_f32(v[(size_t(c0 + r) * hv + h) * dvd + i0 + i]) : 0.f;
+        }
+        if (tid < kBwdC) {
+            const size_t gb = size_t(c0 + tid) * hv + h;
+            vG[tid] = tid < Lc ? fmaxf(a.g[gb], kGFloor) : 0.f;
+            vB[tid] = tid < Lc ? a.beta[gb] : 0.f;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            float run = 0.f;
+            for (int r = 0; r < kBwdC; ++r) {
+                run += vG[r];
+                vG[r] = run;
+            }
+        }
+        __syncthreads();
+        if (tid < kBwdC) {
+            const float gam = __expf(vG[tid]);
+            vGam[tid] = gam;
+            vLam[tid] = tid < Lc ? __expf(vG[Lc - 1] - vG[tid]) : 0.f;
+            vBG[tid] = vB[tid] * gam;
+        }
+        for (int p = tid; p < kBwdC * kBwdC; p += kBwdThreads) {
+            const int r = p / kBwdC, j = p % kBwdC;
+            float kk = 0.f, qk = 0.f;
+            if (j <= r)
+                for (int x = 0; x < dkd; ++x) {
+                    kk = fmaf(K[r * ldk + x], K[j * ldk + x], kk);
+                    qk = fmaf(Q[r * ldk + x], K[j * ldk + x], qk);
+                }
+            KK[r * ldc + j] = kk;
+            QK[r * ldc + j] = qk;
+            Gm[r * ldc + j] = j <= r ? __expf(vG[r] - vG[j]) : 0.f;
+        }
+        __syncthreads();
+        // T = (I + A)^-1, A_rj = beta_r Gamma_rj KK_rj (j < r); one column per thread
+        if (tid < kBwdC) {
+            const int col = tid;
+            for (int r = 0; r < kBwdC; ++r) {
+                float x = r == col ? 1.f : 0.f;
+                if (r > col)
+                    for (int j = col; j < r; ++j) x = fmaf(-vB[r] * Gm[r * ldc + j] * KK[r * ldc + j], Tm[j * ldc + col], x);
+                Tm[r * ldc + col] = r < col ? 0.f : x;
+            }
+        }
+        __syncthreads();
+        for (int idx = tid; idx < kBwdC * dkd; idx += kBwdThreads) {
+            const int r = idx / dkd, x = idx % dkd;
+            float acc = 0.f;
+            for (int j = 0; j <= r; ++j) acc = fmaf(Tm[r * ldc + j] * vBG[j], K[j * ldk + x], acc);
+            W[r * ldk + x] = acc;
+        }
+        __syncthreads();
+        for (int idx = tid; idx < kBwdC * kBwdRows; idx += kBwdThreads) {
+            const int r = idx / kBwdRows, i = idx % kBwdRows;
+            float acc = 0.f;
+            for (int j = 0; j <= r; ++j) acc = fmaf(Tm[r * ldc + j] * vB[j], V[j * ldv + i], acc);
+            for (int x = 0; x < dkd; ++x) acc = fmaf(-W[r * ldk + x], S0[i * ldk + x], acc);
+            U[r * ldv + i] = acc;
+        }
+        __syncthreads();
+    };
+
+    // ---- pass 1: chunk start states into the workspace ----
+    for (int idx = tid; idx < kBwdRows * dkd; idx += kBwdThreads) {
+        const int i = idx / dkd, x = idx % dkd;
+        S0[i * ldk + x] = (a.s0 && i < nr) ? a.s0[sbase + size_t(i0 + i) * dkd + x] : 0.f;
+    }
+    __syncthreads();
+    for (int c = 0; c < nch; ++c) {
+        const int Lc = min(kBwdC, len - c * kBwdC);
+        float *dst = ck(c);
+        for (int idx = tid; idx < nr * dkd; idx += kBwdThreads) dst[idx] = S0[(idx / dkd) * ldk + idx % dkd];
+        chunk_forward(c, Lc);
+        const float gl = __expf(vG[Lc - 1]);
+        for (int idx = tid; idx < kBwdRows * dkd; idx += kBwdThreads) {
+            const int i = idx / dkd, x = idx % dkd;
+            float acc = gl * S0[i * ldk + x];
+            for (int j = 0; j < Lc; ++j) acc = fmaf(U[j * ldv + i] * vLam[j], K[j * ldk + x], acc);
+            S0[i * ldk + x] = acc;
+        }
+        __syncthreads();
+    }
+
+    // ---- pass 2: backward over the chunks ----
+    for (int idx = tid; idx < kBwdRows * dkd; idx += kBwdThreads) {
+        const int i = idx / dkd, x = idx % dkd;
+        dS[i * ldk + x] = (dSf && i < nr) ? dSf[sbase + size_t(i0 + i) * dkd + x] : 0.f;
+    }
+    for (int c = nch - 1; c >= 0; --c) {
+        const int Lc = min(kBwdC, len - c * kBwdC);
+        const int c0 = t0 + c * kBwdC;
+        const float *src = ck(c);
+        for (int idx = tid; idx < kBwdRows * dkd; idx += kBwdThreads) {
+            const int i = idx / dkd, x = idx % dkd;
+            S0[i * ldk + x] = i < nr ? src[i * dkd + x] : 0.f;
+        }
+        __syncthreads();
+        chunk_forward(c, Lc);
+        for (int idx = tid; idx < kBwdC * kBwdRows; idx += kBwdThreads) {
+            const int r = idx / kBwdRows, i = idx % kBwdRows;
+            dOs[r * ldv + i] = (r < Lc && i < nr) ? to_f32(dO[(size_t(c0 + r) * hv + h) * dvd + i0 + i]) : 0.f;
+        }
+        for (int idx = tid; idx < kBwdC * dkd; idx += kBwdThreads) {
+            dQ[(idx / dkd) * ldk + idx % dkd] = 0.f;
+            dK[(idx / dkd) * ldk + idx % dkd] = 0.f;
+        }
+        if (tid < kBwdC) vdGam[tid] = vdLam[tid] = vdBG[tid] = vdB[tid] = vdG[tid] = 0.f;
+        // dgamma_L = <dS, S0> over the block's rows
+        float part = 0.f;
+        for (int idx = tid; idx < kBwdRows * dkd; idx += kBwdThreads) {
+            const int i = idx / dkd, x = idx % dkd;
+            part = fmaf(dS[i * ldk + x], S0[i * ldk + x], part);
+        }
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
+        if ((tid & 31) == 0) red[tid >> 5] = part;
+        __syncthreads();
+        float dgl = 0.f;
+        for (int w = 0; w < kBwdThreads / 32; ++w) dgl += red[w];
+        // dU from the end state, and lambda's gradient: Z_ji = dS_i . k_j
+        for (int idx = tid; idx < kBwdC * kBwdRows; idx += kBwdThreads) {
+            const int j = idx / kBwdRows, i = idx % kBwdRows;
+            float z = 0.f;
+            for (int x = 0; x < dkd; ++x) z = fmaf(dS[i * ldk + x], K[j * ldk + x], z);
+            dU[j * ldv + i] = vLam[j] * z;
+            dT[j * ldc + i] = U[j * ldv + i] * z;  // scratch: U_ji Z_ji, summed below
+        }
+        __syncthreads();
+        if (tid < kBwdC) {
+            float s = 0.f;
+            for (int i = 0; i < kBwdRows; ++i) s += dT[tid * ldc + i];
+            vdLam[tid] = s;
+        }
+        // dK_j += lambda_j dS^T u_j;  output terms: Y_r = dO_r S0 -> dQ_r += gamma_r Y_r, dgamma_r += Y_r . q_r
+        for (int idx = tid; idx < kBwdC * dkd; idx += kBwdThreads) {
+            const int j = idx / dkd, x = idx % dkd;
+            float acc = 0.f, y = 0.f;
+            for (int i = 0; i < kBwdRows; ++i) {
+                acc = fmaf(U[j * ldv + i], dS[i * ldk + x], acc);
+                y = fmaf(dOs[j * ldv + i], S0[i * ldk + x], y);
+            }
+            dK[j * ldk + x] += vLam[j] * acc;
+            dQ[j * ldk + x] += vGam[j] * y;
+            dW[j * ldk + x] = y * Q[j * ldk + x];  // scratch for dgamma
+        }
+        __syncthreads();
+        if (tid < kBwdC) {
+            float s = 0.f;
+            for (int x = 0; x < dkd; ++x) s += dW[tid * ldk + x];
+            vdGam[tid] += s;
+        }
+        // dP_rj = dO_r . u_j (j <= r); dU_j += sum_r P_rj dO_r
+        for (int p = tid; p < kBwdC * kBwdC; p += kBwdThreads) {
+            const int r = p / kBwdC, j = p % kBwdC;
+            float d = 0.f;
+            if (j <= r)
+                for (int i = 0; i < kBwdRows; ++i) d = fmaf(dOs[r * ldv + i], U[j * ldv + i], d);
+            dT[r * ldc + j] = d;  // dP, kept in dT's storage until dT is formed
+        }
+        __syncthreads();
+        for (int idx = tid; idx < kBwdC * kBwdRows; idx += kBwdThreads) {
+            const int j = idx / kBwdRows, i = idx % kBwdRows;
+            float acc = dU[j * ldv + i];
+            for (int r = j; r < kBwdC; ++r) acc = fmaf(Gm[r * ldc + j] * QK[r * ldc + j], dOs[r * ldv + i], acc);
+            dU[j * ldv + i] = acc;
+        }
+        // P = QK (.) Gamma: dQ_r += sum_j dP_rj Gamma_rj k_j, dK_j += sum_r dP_rj Gamma_rj q_r; dGamma (in dA) = dP QK
+        for (int idx = tid; idx < kBwdC * dkd; idx += kBwdThreads) {
+            const int r = idx / dkd, x = idx % dkd;
+            float aq = 0.f, ak = 0.f;
+            for (int j = 0; j <= r; ++j) aq = fmaf(dT[r * ldc + j] * Gm[r * ldc + j], K[j * ldk + x], aq);
+            for (int i = r; i < kBwdC; ++i) ak = fmaf(dT[i * ldc + r] * Gm[i * ldc + r], Q[i * ldk + x], ak);
+            dQ[r * ldk + x] += aq;
+            dK[r * ldk + x] += ak;
+        }
+        for (int p = tid; p < kBwdC * kBwdC; p += kBwdThreads) {
+            const int r = p / kBwdC, j = p % kBwdC;
+            dA[r * ldc + j] = j <= r ? dT[r * ldc + j] * QK[r * ldc + j] : 0.f;  // dGamma so far
+        }
+        __syncthreads();
+        // dW = -dU S0; dS0 = gamma_L dS + dO^T diag(gamma) Q - dU^T W (in place over dS)
+        for (int idx = tid; idx < kBwdC * dkd; idx += kBwdThreads) {
+            const int r = idx / dkd, x = idx % dkd;
+            float acc = 0.f;
+            for (int i = 0; i < kBwdRows; ++i) acc = fmaf(-dU[r * ldv + i], S0[i * ldk + x], acc);
+            dW[r * ldk + x] = acc;
+        }
+        const float gL = __expf(vG[Lc - 1]);
+        for (int idx = tid; idx < kBwdRows * dkd; idx += kBwdThreads) {
+            const int i = idx / dkd, x = idx % dkd;
+            float acc = gL * dS[i * ldk + x];
+            for (int r = 0; r < Lc; ++r) {
+                acc = fmaf(dOs[r * ldv + i] * vGam[r], Q[r * ldk + x], acc);
+                acc = fmaf(-dU[r * ldv + i], W[r * ldk + x], acc);
+            }
+            dS[i * ldk + x] = acc;
+        }
+        __syncthreads();
+        // dT_rj = dW_r . (bg_j k_j) + dU_r . (beta_j v_j), j <= r
+        for (int p = tid; p < kBwdC * kBwdC; p += kBwdThreads) {
+            const int r = p / kBwdC, j = p % kBwdC;
+            float d = 0.f;
+            if (j <= r) {
+                for (int x = 0; x < dkd; ++x) d = fmaf(dW[r * ldk + x], K[j * ldk + x], d);
+                d *= vBG[j];
+                float e = 0.f;
+                for (int i = 0; i < kBwdRows; ++i) e = fmaf(dU[r * ldv + i], V[j * ldv + i], e);
+                d = fmaf(vB[j], e, d);
+            }
+            dT[r * ldc + j] = d;
+        }
+        __syncthreads();
+        // dX_j = sum_r T_rj dW_r: dK_j += bg_j dX_j, dbg_j = dX_j . k_j;
+        // dY_j = sum_r T_rj dU_r: dv_j = beta_j dY_j, dbeta_j += dY_j . v_j
+        for (int idx = tid; idx < kBwdC * dkd; idx += kBwdThreads) {
+            const int j = idx / dkd, x = idx % dkd;
+            float dx = 0.f;
+            for (int r = j; r < kBwdC; ++r) dx = fmaf(Tm[r * ldc + j], dW[r * ldk + x], dx);
+            dK[j * ldk + x] = fmaf(vBG[j], dx, dK[j * ldk + x]);
+            Q[j * ldk + x] = dx * K[j * ldk + x];  // scratch for dbg (Q is no longer needed; dW is still read)
+        }
+        for (int idx = tid; idx < kBwdC * kBwdRows; idx += kBwdThreads) {
+            const int j = idx / kBwdRows, i = idx % kBwdRows;
+            float dy = 0.f;
+            for (int r = j; r < kBwdC; ++r) dy = fmaf(Tm[r * ldc + j], dU[r * ldv + i], dy);
+            if (j < Lc && i < nr) dv[(size_t(c0 + j) * hv + h) * dvd + i0 + i] = vB[j] * dy;
+            U[j * ldv + i] = dy * V[j * ldv + i];  // scratch for dbeta (U is no longer needed)
+        }
+        __syncthreads();
+        if (tid < kBwdC) {
+            float s = 0.f;
+            for (int x = 0; x < dkd; ++x) s += Q[tid * ldk + x];
+            vdBG[tid] = s;
+            float b = 0.f;
+            for (int i = 0; i < kBwdRows; ++i) b += U[tid * ldv + i];
+            vdB[tid] = b;
+        }
+        // dA = -T^T dT T^T (strictly lower): first M = dT T^T into W's storage
+        for (int p = tid; p < kBwdC * kBwdC; p += kBwdThreads) {
+            const int r = p / kBwdC, j = p % kBwdC;
+            float acc = 0.f;
+            for (int m = 0; m <= j; ++m) acc = fmaf(dT[r * ldc + m], Tm[j * ldc + m], acc);
+            W[r * ldk + j] = acc;
+        }
+        __syncthreads();
+        for (int p = tid; p < kBwdC * kBwdC; p += kBwdThreads) {
+            const int r = p / kBwdC, j = p % kBwdC;
+            float acc = 0.f;
+            if (j < r)
+                for (int m = r; m < kBwdC; ++m) acc = fmaf(Tm[m * ldc + r], W[m * ldk + j], acc);
+            // A_rj = beta_r Gamma_rj KK_rj: dbeta_r, dGamma_rj, and dKK_rj into dT's storage
+            const float da = -acc;
+            dT[r * ldc + j] = j < r ? da * vB[r] * Gm[r * ldc + j] : 0.f;
+            if (j < r) dA[r * ldc + j] += da * vB[r] * KK[r * ldc + j];
+            dW[r * ldk + j] = j < r ? da * Gm[r * ldc + j] * KK[r * ldc + j] : 0.f;  // dbeta terms (W still read)
+        }
+        __syncthreads();
+        if (tid < kBwdC) {
+            float s = 0.f;
+            for (int j = 0; j < tid; ++j) s += dW[tid * ldk + j];
+            vdB[tid] += s;
+        }
+        // dK_r += sum_j dKK_rj k_j + sum_j dKK_jr k_j
+        for (int idx = tid; idx < kBwdC * dkd; idx += kBwdThreads) {
+            const int r = idx / dkd, x = idx % dkd;
+            float acc = 0.f;
+            for (int j = 0; j < r; ++j) acc = fmaf(dT[r * ldc + j], K[j * ldk + x], acc);
+            for (int j = r + 1; j < kBwdC; ++j) acc = fmaf(dT[j * ldc + r], K[j * ldk + x], acc);
+            dK[r * ldk + x] += acc;
+        }
+        __syncthreads();
+        // decays: beta gamma, gamma, lambda, gamma_L and Gamma through G, then dg = reverse prefix sums
+        if (tid < kBwdC) {
+            const int r = tid;
+            vdB[r] = fmaf(vdBG[r], vGam[r], vdB[r]);
+            const float dgam = fmaf(vdBG[r], vB[r], vdGam[r]);
+            float dG = dgam * vGam[r] - vdLam[r] * vLam[r];
+            for (int j = 0; j <= r; ++j) dG = fmaf(dA[r * ldc + j], Gm[r * ldc + j], dG);
+            for (int i = r; i < kBwdC; ++i) dG = fmaf(-dA[i * ldc + r], Gm[i * ldc + r], dG);
+            vdG[r] = dG;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            float extra = dgl * gL;
+            for (int j = 0; j < Lc; ++j) extra = fmaf(vdLam[j], vLam[j], extra);
+            vdG[Lc - 1] += extra;
+            float run = 0.f;
+            for (int t = Lc - 1; t >= 0; --t) {
+                run += vdG[t];
+                vdG[t] = run;
+            }
+        }
+        __syncthreads();
+        // the block's share of the shared gradients
+        for (int idx = tid; idx < Lc * dkd; idx += kBwdThreads) {
+            const int r = idx / dkd, x = idx % dkd;
+            const size_t o = (size_t(c0 + r) * hk + hq) * dkd + x;
+            atomicAdd(dq + o, dQ[r * ldk + x]);
+            atomicAdd(dk + o, dK[r * ldk + x]);
+        }
+        if (tid < Lc) {
+            atomicAdd(dg + size_t(c0 + tid) * hv + h, vdG[tid]);
+            atomicAdd(dbeta + size_t(c0 + tid) * hv + h, vdB[tid]);
+        }
+        __syncthreads();
+    }
+    if (dS0_out)
+        for (int idx = tid; idx < nr * dkd; idx += kBwdThreads) {
+            const int i = idx / dkd, x = idx % dkd;
+            dS0_out[sbase + size_t(i0 + i) * dkd + x] = dS[i * ldk + x];
+        }
+}
+
+size_t backward_ckpt_bytes(int32_t tokens, int32_t num_seqs, int32_t hv, int32_t dk, int32_t dv) {
+    const size_t slots = size_t(tokens) / kBwdC + size_t(num_seqs) + 1;
+    return slots * size_t(hv) * size_t(dv) * size_t(dk) * sizeof(float);
+}
+
+cudaError_t launch_chunk_backward(const PrefillArgs &a, const void *dO, const float *dSf, float *dq, float *dk,
+                                  float *dv, float *dg, float *dbeta, float *dS0, float *ckpt, cudaStream_t stream) {
+    const int n_slices = (a.dv + kBwdRows - 1) / kBwdRows;
+    const int64_t blocks = int64_t(a.num_seqs) * a.hv * n_slices;
+    if (blocks <= 0) return cudaSuccess;
+    if (blocks > INT32_MAX || a.dk > 128 || a.dv > 128) return cudaErrorInvalidValue;
+    const size_t bytes = bwd_smem(a.dk).total * sizeof(float);
+    cudaError_t e;
+    if (a.dtype == GDN_DTYPE_BF16) {
+        e = cudaFuncSetAttribute(chunk_backward_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(bytes));
+        if (e != cudaSuccess) return e;
+        chunk_backward_kernel<__nv_bfloat16><<<unsigned(blocks), kBwdThreads, bytes, stream>>>(
+            a, dO, dSf, dq, dk, dv, dg, dbeta, dS0, ckpt, n_slices);
+    } else {
+        e = cudaFuncSetAttribute(chunk_backward_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(bytes));
+        if (e != cudaSuccess) return e;
+        chunk_backward_kernel<float><<<unsigned(blocks), kBwdThreads, bytes, stream>>>(a, dO, dSf, dq, dk, dv, dg,
+                                                                                      dbeta, dS0, ckpt, n_slices);
+    }
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

@@ -185,6 +185,11 @@ cudaError_t launch_decode_multi(int32_t n, int32_t ntok, int32_t hk, int32_t hv,
 cudaError_t launch_decode_commit(int32_t n, int32_t ntok, int32_t hv, int32_t dk, int32_t dv, const float *snap,
                                  const int32_t *accepted, float *state, int32_t *bad, cudaStream_t stream);
 
+// Backward (training): checkpoint bytes and the kernel.
+size_t backward_ckpt_bytes(int32_t tokens, int32_t num_seqs, int32_t hv, int32_t dk, int32_t dv);
+cudaError_t launch_chunk_backward(const PrefillArgs &a, const void *dO, const float *dSf, float *dq, float *dk,
+                                  float *dv, float *dg, float *dbeta, float *dS0, float *ckpt, cudaStream_t stream);
+
 // Decode step.
 cudaError_t launch_decode(int32_t n, int32_t hk, int32_t hv, int32_t dk, int32_t dv, int32_t dtype,
                           const void *q, const void *k, const void *v, const float *g, const float *beta,

@@ -40,7 +40,8 @@ GDN_OUT_WEIGHT_PER_HEAD = 8
 EXPORTED = ("gdn_chunk_forward_workspace_size", "gdn_chunk_forward", "gdn_read_device_status",
             "gdn_decode_step", "gdn_status_string", "gdn_last_error_message", "gdn_launch_count",
             "gdn_chunk_forward_noalloc", "gdn_decode_step_ex", "gdn_chunk_forward_out", "gdn_decode_step_out",
-            "gdn_kda_forward", "gdn_kda_decode_step", "gdn_decode_multi", "gdn_decode_commit")
+            "gdn_kda_forward", "gdn_kda_decode_step", "gdn_decode_multi", "gdn_decode_commit",
+            "gdn_chunk_backward_workspace_size", "gdn_chunk_backward")
 
 
 class GdnError(RuntimeError):
@@ -95,6 +96,10 @@ def _load(path: str = LIB_PATH):
     lib.gdn_decode_multi.restype = st
     lib.gdn_decode_commit.argtypes = [i32] * 5 + [vp] * 4 + [vp]
     lib.gdn_decode_commit.restype = st
+    lib.gdn_chunk_backward_workspace_size.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(ctypes.c_size_t)]
+    lib.gdn_chunk_backward_workspace_size.restype = st
+    lib.gdn_chunk_backward.argtypes = [ctypes.POINTER(Shape)] + [vp] * 15 + [vp, ctypes.c_size_t, vp]
+    lib.gdn_chunk_backward.restype = st
     lib.gdn_status_string.argtypes = [st]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_last_error_message.argtypes = []
@@ -411,6 +416,37 @@ def decode_commit(snapshots, accepted, state, bad_count=None, stream=None):
     _check(LIB.gdn_decode_commit(N, K, hv, dk, dv, _ptr(snapshots), _ptr(accepted), _ptr(state), _ptr(bad_count),
                                  _stream_handle(stream)))
     return state
+
+
+def chunk_backward(q, k, v, g, beta, d_o, d_final_state=None, initial_state=None, cu_seqlens=None,
+                   want_d_initial_state=True, workspace=None, stream=None):
+    """Gradients of sum d_o . o + sum d_final_state . S_final (training).
+    Returns a dict of fp32 tensors: dq, dk (shaped like q), dv (like v),
+    dg, dbeta (like g), d_initial_state ([N, Hv, d_v, d_k], or None)."""
+    dev, dt = q.device, q.dtype
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (d_o, "d_o")):
+        _need(t, n, dt, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(initial_state, "initial_state", torch.float32, dev)
+    _need(d_final_state, "d_final_state", torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    shape = make_shape(q, v, cu_seqlens, 32)
+    n = ctypes.c_size_t(0)
+    _check(LIB.gdn_chunk_backward_workspace_size(ctypes.byref(shape), ctypes.byref(n)))
+    if workspace is None or workspace.numel() < n.value:
+        workspace = torch.empty(n.value, dtype=torch.uint8, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {"dq": torch.empty(q.shape, **f32), "dk": torch.empty(k.shape, **f32), "dv": torch.empty(v.shape, **f32),
+           "dg": torch.empty(g.shape, **f32), "dbeta": torch.empty(beta.shape, **f32),
+           "d_initial_state": torch.empty((shape.num_seqs, shape.num_v_heads, shape.head_dim_v, shape.head_dim_k),
+                                          **f32) if want_d_initial_state else None}
+    _check(LIB.gdn_chunk_backward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                  _ptr(initial_state), _ptr(cu_seqlens), _ptr(d_o), _ptr(d_final_state),
+                                  _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]),
+                                  _ptr(out["dbeta"]), _ptr(out["d_initial_state"]), _ptr(workspace),
+                                  workspace.numel(), _stream_handle(stream)))
+    return out
 
 
 def launch_count() -> int:

@@ -1,0 +1,96 @@
+"""GPU parity of the gradients (training) against the fp64 oracle's reverse
+mode of the token recurrence ("Architecture Thread I", the Gated DeltaNet
+section; "Gated Attention Architectures", sections 2 and 3), per
+(sequence, head) slice: dq, dk per q/k head, dv, dg, dbeta per value head,
+and the initial-state gradient.
+
+The kernel computes in fp32 from the given (bf16 or fp32) values, so both
+input types are held to one bar, GRAD_BAR: fp32 rounding over sums of
+O(C d) terms per chunk, carried through T / C chunks of the state-gradient
+recurrence, stays well below 1e-4 relative on these sizes; 2e-4 leaves room
+for the atomic summation order of dq, dk, dg and dbeta."""
+import numpy as np
+import pytest
+import torch
+
+from linear_attention_sequence_sm_b200 import inputs as I
+from parity import to_f64, slices
+
+pytestmark = pytest.mark.gpu
+
+DEV = torch.device("cuda:0")
+GRAD_BAR = 2e-4
+
+
+def bwd_inputs(seed, B, T, hk, hv, d, dtype, seq_lens=None, s0_std=0.05):
+    w = I.custom(f"bwd_{seed}", batch=B, seq_len=T, hk=hk, hv=hv, d=d, chunk=32, dtype=dtype, seed=seed,
+                 s0_std=s0_std, seq_lens=seq_lens)
+    inp = I.make_prefill_inputs(w)
+    td = torch.float32 if dtype == "f32" else torch.bfloat16
+    inp["dO"] = torch.from_numpy(I.normal(seed, "bwd_do", tuple(inp["v"].shape))).to(td)
+    inp["dSf"] = torch.from_numpy(I.normal(seed, "bwd_dsf", (w.num_seqs, hv, d, d), std=0.1)).float()
+    return inp
+
+
+def run_both(inp, with_dsf=True):
+    from linear_attention_sequence_sm_b200 import gdn
+    from oracle import oracle
+    d = {k: (v.to(DEV) if v is not None else None) for k, v in inp.items()}
+    gg = gdn.chunk_backward(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"],
+                            d_final_state=d["dSf"] if with_dsf else None, initial_state=d["initial_state"],
+                            cu_seqlens=d["cu_seqlens"])
+    torch.cuda.synchronize()
+    cu = None if inp["cu_seqlens"] is None else inp["cu_seqlens"].numpy().astype(np.int64)
+    ref = oracle.backward(*(to_f64(inp[n]) for n in ("q", "k", "v", "g", "beta", "dO")),
+                          dS_final=to_f64(inp["dSf"]) if with_dsf else None,
+                          initial_state=to_f64(inp["initial_state"]), cu_seqlens=cu)
+    return gg, ref
+
+
+def worst_errors(inp, gg, ref):
+    """Max rel-L2 over (sequence, head) slices of each gradient."""
+    hk, hv = inp["q"].shape[-2], inp["v"].shape[-2]
+    out = {}
+    for name, heads in (("dq", hk), ("dk", hk), ("dv", hv), ("dg", hv), ("dbeta", hv)):
+        got = to_f64(gg[name]).reshape(-1, heads, *gg[name].shape[len(inp["q"].shape[:-2]) + 1:])
+        want = np.asarray(ref[name]).reshape(got.shape)
+        w = 0.0
+        for n, a, b in slices(inp):
+            for h in range(heads):
+                if b > a:
+                    r = want[a:b, h]
+                    w = max(w, np.linalg.norm(got[a:b, h] - r) / max(np.linalg.norm(r), 1e-30))
+        out[name] = w
+    g0, r0 = to_f64(gg["d_initial_state"]), ref["dS0"]
+    out["dS0"] = max(np.linalg.norm(g0[n, h] - r0[n, h]) / max(np.linalg.norm(r0[n, h]), 1e-30)
+                     for n in range(r0.shape[0]) for h in range(hv))
+    return out
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("d", [128, 64])
+def test_backward_parity(dtype, d):
+    inp = bwd_inputs(300 + d, B=2, T=100, hk=2, hv=4, d=d, dtype=dtype)
+    gg, ref = run_both(inp)
+    errs = worst_errors(inp, gg, ref)
+    print(dtype, d, errs)
+    assert max(errs.values()) <= GRAD_BAR, errs
+
+
+def test_backward_varlen_edges():
+    lens = [1, 31, 32, 33, 0, 70, 5]
+    inp = bwd_inputs(310, B=1, T=sum(lens), hk=1, hv=2, d=128, dtype="bf16", seq_lens=lens)
+    gg, ref = run_both(inp)
+    errs = worst_errors(inp, gg, ref)
+    print(errs)
+    assert max(errs.values()) <= GRAD_BAR, errs
+    # the empty sequence passes its final-state gradient straight through
+    assert torch.allclose(gg["d_initial_state"][4], inp["dSf"][4].to(DEV), rtol=0, atol=0)
+
+
+def test_backward_small_dims_without_final_gradient():
+    inp = bwd_inputs(320, B=3, T=45, hk=1, hv=3, d=16, dtype="f32")
+    gg, ref = run_both(inp, with_dsf=False)
+    errs = worst_errors(inp, gg, ref)
+    print(errs)
+    assert max(errs.values()) <= GRAD_BAR, errs
