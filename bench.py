@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import ctypes
 import json
 import os
 import statistics
@@ -57,6 +58,9 @@ def parse_args(argv=None):
     p.add_argument("--kda", action="store_true",
                    help="Kimi Delta Attention (one decay per key channel) instead of the gated delta rule: "
                         "CUDA-core prefill (ALU roofline) and decode (HBM roofline)")
+    p.add_argument("--backward", action="store_true",
+                   help="time the gradients (training) on the prefill workload instead of the forward "
+                        "(CUDA-core kernel, fp32 ALU roofline)")
     p.add_argument("--mtp", type=int, default=0,
                    help="decode: verify K draft tokens per sequence in one pass (state after every token kept)")
     p.add_argument("--no-e2e", action="store_true")
@@ -271,7 +275,7 @@ def run_ours(args):
     host = I.make_raw_prefill_inputs(w) if args.raw_inputs else I.make_prefill_inputs(w)
     flags = {"qk_l2norm": True, "gate_logits": True} if args.raw_inputs else {}
     suffix = ("_kda" if args.kda else "") + ("_raw_inputs" if args.raw_inputs else "") + \
-        ("_output_norm" if args.output_norm else "")
+        ("_output_norm" if args.output_norm else "") + ("_backward" if args.backward else "")
     if args.kda:
         host["g"] = I.make_kda_gates(w)
     fwd = gdn.kda_forward if args.kda else gdn.chunk_forward
@@ -291,7 +295,18 @@ def run_ours(args):
     ws = torch.empty(gdn.workspace_size(shape), dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
 
+    if args.backward:
+        dev["dO"] = torch.from_numpy(I.normal(w.seed, "bwd_do", tuple(host["v"].shape))).to(dev["v"].dtype).to(device)
+        bshape = gdn.make_shape(dev["q"], dev["v"], dev["cu_seqlens"], 32)
+        nb = ctypes.c_size_t(0)
+        gdn.LIB.gdn_chunk_backward_workspace_size(ctypes.byref(bshape), ctypes.byref(nb))
+        bws = torch.empty(nb.value, dtype=torch.uint8, device=device)
+
     def step():
+        if args.backward:
+            gdn.chunk_backward(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev["dO"],
+                               initial_state=dev["initial_state"], cu_seqlens=dev["cu_seqlens"], workspace=bws)
+            return
         fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], initial_state=dev["initial_state"],
                           cu_seqlens=dev["cu_seqlens"], out=o, final_state=sf, workspace=ws, chunk_size=w.chunk,
                           **flags, **out_norm(dev))
@@ -323,6 +338,17 @@ def run_ours(args):
                 "kernel": kernel_name,
                 "peak_source": f"{peak_src} bf16 dense (burst)",
                 "flops_per_launch": flops, "algorithmic_bytes_per_launch": prefill_bytes(w)}
+    if args.backward:
+        # reverse mode of the token recurrence: 20 d^2 flops per (token, value head) (the forward
+        # recomputed, 6 d^2, and the backward, 14 d^2); fp32 on CUDA cores
+        bflops = 20 * w.d * w.d * tokens * w.hv
+        alu_peak = FP32_LANES_PER_SM * 2 * torch.cuda.get_device_properties(device).multi_processor_count * \
+            (clocks.summary().get("sm_max_mhz") or 1965) * 1e6 / 1e12
+        achieved = bflops / (ms / 1e3) / 1e12
+        roofline = {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s",
+                    "frac": achieved / alu_peak, "traffic": kernel_traffic(f"gdn_backward/{w.name}{suffix}"),
+                    "kernel": "gdn_backward", "peak_source": "fp32 FMA lanes x 2 x max SM clock (derived)",
+                    "flops_per_launch": bflops}
     if args.kda:
         # token-order recurrence on CUDA cores: 7 d_v d_k fp32 flops per (token, value head)
         # (decay, two dot products, rank-1 write); peak = SMs x 128 fp32 lanes x 2 x max SM clock

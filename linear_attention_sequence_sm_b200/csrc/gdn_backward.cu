@@ -34,7 +34,7 @@ constexpr int kBwdRows = 32; // rows of d_v per block
 
 struct BwdSmem {
     int ldk, ldc, ldv;
-    size_t k, q, w, dw, dq, dk, s0, ds, v, u, du, dO, t, gm, kk, qk, dt, da, vec, total;
+    size_t k, q, w, dw, dq, dk, s0, ds, v, u, du, dO, t, gm, kk, qk, dt, da, sm, se, vec, total;
 };
 
 __host__ __device__ inline BwdSmem bwd_smem(int dk) {
@@ -62,6 +62,8 @@ __host__ __device__ inline BwdSmem bwd_smem(int dk) {
     s.qk = take(size_t(kBwdC) * s.ldc);
     s.dt = take(size_t(kBwdC) * s.ldc);
     s.da = take(size_t(kBwdC) * s.ldc);
+    s.sm = take(size_t(kBwdC) * s.ldc);  // C x C scratch: dT T^T
+    s.se = take(size_t(kBwdC) * s.ldc);  // C x C scratch: the dbeta terms of dA
     s.vec = take(size_t(16) * kBwdC);
     s.total = off;
     return s;
@@ -86,7 +88,8 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
     float *K = smem + L.k, *Q = smem + L.q, *W = smem + L.w, *dW = smem + L.dw, *dQ = smem + L.dq,
           *dK = smem + L.dk, *S0 = smem + L.s0, *dS = smem + L.ds, *V = smem + L.v, *U = smem + L.u,
           *dU = smem + L.du, *dOs = smem + L.dO, *Tm = smem + L.t, *Gm = smem + L.gm, *KK = smem + L.kk,
-          *QK = smem + L.qk, *dT = smem + L.dt, *dA = smem + L.da, *vec = smem + L.vec;
+          *QK = smem + L.qk, *dT = smem + L.dt, *dA = smem + L.da, *sM = smem + L.sm, *sE = smem + L.se,
+          *vec = smem + L.vec;
     float *vG = vec + kVG * kBwdC, *vGam = vec + kVGam * kBwdC, *vLam = vec + kVLam * kBwdC,
           *vB = vec + kVB * kBwdC, *vBG = vec + kVBG * kBwdC, *vdG = vec + kVDG * kBwdC,
           *vdGam = vec + kVDGam * kBwdC, *vdLam = vec + kVDLam * kBwdC, *vdBG = vec + kVDBG * kBwdC,
@@ -360,29 +363,29 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
             for (int i = 0; i < kBwdRows; ++i) b += U[tid * ldv + i];
             vdB[tid] = b;
         }
-        // dA = -T^T dT T^T (strictly lower): first M = dT T^T into W's storage
+        // dA = -T^T dT T^T (strictly lower): first M = dT T^T
         for (int p = tid; p < kBwdC * kBwdC; p += kBwdThreads) {
             const int r = p / kBwdC, j = p % kBwdC;
             float acc = 0.f;
             for (int m = 0; m <= j; ++m) acc = fmaf(dT[r * ldc + m], Tm[j * ldc + m], acc);
-            W[r * ldk + j] = acc;
+            sM[r * ldc + j] = acc;
         }
         __syncthreads();
         for (int p = tid; p < kBwdC * kBwdC; p += kBwdThreads) {
             const int r = p / kBwdC, j = p % kBwdC;
             float acc = 0.f;
             if (j < r)
-                for (int m = r; m < kBwdC; ++m) acc = fmaf(Tm[m * ldc + r], W[m * ldk + j], acc);
+                for (int m = r; m < kBwdC; ++m) acc = fmaf(Tm[m * ldc + r], sM[m * ldc + j], acc);
             // A_rj = beta_r Gamma_rj KK_rj: dbeta_r, dGamma_rj, and dKK_rj into dT's storage
             const float da = -acc;
             dT[r * ldc + j] = j < r ? da * vB[r] * Gm[r * ldc + j] : 0.f;
             if (j < r) dA[r * ldc + j] += da * vB[r] * KK[r * ldc + j];
-            dW[r * ldk + j] = j < r ? da * Gm[r * ldc + j] * KK[r * ldc + j] : 0.f;  // dbeta terms (W still read)
+            sE[r * ldc + j] = j < r ? da * Gm[r * ldc + j] * KK[r * ldc + j] : 0.f;  // dbeta terms
         }
         __syncthreads();
         if (tid < kBwdC) {
             float s = 0.f;
-            for (int j = 0; j < tid; ++j) s += dW[tid * ldk + j];
+            for (int j = 0; j < tid; ++j) s += sE[tid * ldc + j];
             vdB[tid] += s;
         }
         // dK_r += sum_j dKK_rj k_j + sum_j dKK_jr k_j
