@@ -76,6 +76,41 @@ enum { kVG = 0, kVGam, kVLam, kVB, kVBG, kVDG, kVDGam, kVDLam, kVDBG, kVDB, kVNu
 // floor(t0 / C) + n + c never collides between sequences
 __device__ __forceinline__ size_t bwd_slot(int t0, int n, int c) { return size_t(t0 / kBwdC + n + c); }
 
+// out(m, n, sum_k a(m, k) b(k, n)) for m < M <= 32, n < N <= 32 TN, over the
+// block's 256 threads: warp w takes rows 4w .. 4w + 3 and lane l the columns
+// l + 32 i (i < TN), so b's reads are consecutive across a warp and a's are
+// broadcasts; 4 TN multiply-adds per 4 + TN shared-memory loads.  a and b are
+// element accessors, so scales, transposes and stacked operands need no copy.
+// A given (M, N, TN) always maps an output element to the same thread, so
+// products of one shape that accumulate into one array need no barrier
+// between them.
+template <int TN, class FA, class FB, class FO>
+__device__ __forceinline__ void bgemm(int M, int N, int K, FA a, FB b, FO out) {
+    const int m0 = 4 * (threadIdx.x >> 5), l = threadIdx.x & 31;
+    if (m0 >= M) return;
+    float acc[4][TN];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int i = 0; i < TN; ++i) acc[j][i] = 0.f;
+    for (int kk = 0; kk < K; ++kk) {
+        float av[4], bv[TN];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) av[j] = (m0 + j < M) ? a(m0 + j, kk) : 0.f;
+#pragma unroll
+        for (int i = 0; i < TN; ++i) bv[i] = (l + 32 * i < N) ? b(kk, l + 32 * i) : 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int i = 0; i < TN; ++i) acc[j][i] = fmaf(av[j], bv[i], acc[j][i]);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int i = 0; i < TN; ++i)
+            if (m0 + j < M && l + 32 * i < N) out(m0 + j, l + 32 * i, acc[j][i]);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, float *dq, float *dk, float *dv,
@@ -115,19 +150,20 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
     auto ck = [&](int c) { return ckpt + (bwd_slot(t0, seq, c) * hv + h) * size_t(dvd) * dkd + size_t(i0) * dkd; };
 
     // one chunk's inputs and forward quantities (A, T, W, U~, U; the masks)
+    constexpr int C = kBwdC, R = kBwdRows;
     auto chunk_forward = [&](int c, int Lc) {
-        const int c0 = t0 + c * kBwdC;
-        for (int idx = tid; idx < kBwdC * dkd; idx += kBwdThreads) {
+        const int c0 = t0 + c * C;
+        for (int idx = tid; idx < C * dkd; idx += kBwdThreads) {
             const int r = idx / dkd, x = idx % dkd;
             const bool ok = r < Lc;
             K[r * ldk + x] = ok ? to_f32(k[(size_t(c0 + r) * hk + hq) * dkd + x]) : 0.f;
             Q[r * ldk + x] = ok ? to_f32(q[(size_t(c0 + r) * hk + hq) * dkd + x]) : 0.f;
         }
-        for (int idx = tid; idx < kBwdC * kBwdRows; idx += kBwdThreads) {
-            const int r = idx / kBwdRows, i = idx % kBwdRows;
+        for (int idx = tid; idx < C * R; idx += kBwdThreads) {
+            const int r = idx / R, i = idx % R;
             V[r * ldv + i] = (r < Lc && i < nr) ? to_f32(v[(size_t(c0 + r) * hv + h) * dvd + i0 + i]) : 0.f;
         }
-        if (tid < kBwdC) {
+        if (tid < C) {
             const size_t gb = size_t(c0 + tid) * hv + h;
             vG[tid] = tid < Lc ? fmaxf(a.g[gb], kGFloor) : 0.f;
             vB[tid] = tid < Lc ? a.beta[gb] : 0.f;
@@ -135,35 +171,32 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
         __syncthreads();
         if (tid == 0) {
             float run = 0.f;
-            for (int r = 0; r < kBwdC; ++r) {
+            for (int r = 0; r < C; ++r) {
                 run += vG[r];
                 vG[r] = run;
             }
         }
+        // K K^T and Q K^T (lower, with the diagonal)
+        bgemm<1>(C, C, dkd, [&](int r, int x) { return K[r * ldk + x]; }, [&](int x, int j) { return K[j * ldk + x]; },
+                 [&](int r, int j, float acc) { KK[r * ldc + j] = j <= r ? acc : 0.f; });
+        bgemm<1>(C, C, dkd, [&](int r, int x) { return Q[r * ldk + x]; }, [&](int x, int j) { return K[j * ldk + x]; },
+                 [&](int r, int j, float acc) { QK[r * ldc + j] = j <= r ? acc : 0.f; });
         __syncthreads();
-        if (tid < kBwdC) {
+        if (tid < C) {
             const float gam = __expf(vG[tid]);
             vGam[tid] = gam;
             vLam[tid] = tid < Lc ? __expf(vG[Lc - 1] - vG[tid]) : 0.f;
             vBG[tid] = vB[tid] * gam;
         }
-        for (int p = tid; p < kBwdC * kBwdC; p += kBwdThreads) {
-            const int r = p / kBwdC, j = p % kBwdC;
-            float kk = 0.f, qk = 0.f;
-            if (j <= r)
-                for (int x = 0; x < dkd; ++x) {
-                    kk = fmaf(K[r * ldk + x], K[j * ldk + x], kk);
-                    qk = fmaf(Q[r * ldk + x], K[j * ldk + x], qk);
-                }
-            KK[r * ldc + j] = kk;
-            QK[r * ldc + j] = qk;
+        for (int p = tid; p < C * C; p += kBwdThreads) {
+            const int r = p / C, j = p % C;
             Gm[r * ldc + j] = j <= r ? __expf(vG[r] - vG[j]) : 0.f;
         }
         __syncthreads();
         // T = (I + A)^-1, A_rj = beta_r Gamma_rj KK_rj (j < r); one column per thread
-        if (tid < kBwdC) {
+        if (tid < C) {
             const int col = tid;
-            for (int r = 0; r < kBwdC; ++r) {
+            for (int r = 0; r < C; ++r) {
                 float x = r == col ? 1.f : 0.f;
                 if (r > col)
                     for (int j = col; j < r; ++j) x = fmaf(-vB[r] * Gm[r * ldc + j] * KK[r * ldc + j], Tm[j * ldc + col], x);
@@ -171,71 +204,64 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
             }
         }
         __syncthreads();
-        for (int idx = tid; idx < kBwdC * dkd; idx += kBwdThreads) {
-            const int r = idx / dkd, x = idx % dkd;
-            float acc = 0.f;
-            for (int j = 0; j <= r; ++j) acc = fmaf(Tm[r * ldc + j] * vBG[j], K[j * ldk + x], acc);
-            W[r * ldk + x] = acc;
-        }
+        // W = T diag(beta gamma) K
+        bgemm<4>(C, dkd, C, [&](int r, int j) { return Tm[r * ldc + j] * vBG[j]; },
+                 [&](int j, int x) { return K[j * ldk + x]; }, [&](int r, int x, float acc) { W[r * ldk + x] = acc; });
         __syncthreads();
-        for (int idx = tid; idx < kBwdC * kBwdRows; idx += kBwdThreads) {
-            const int r = idx / kBwdRows, i = idx % kBwdRows;
-            float acc = 0.f;
-            for (int j = 0; j <= r; ++j) acc = fmaf(Tm[r * ldc + j] * vB[j], V[j * ldv + i], acc);
-            for (int x = 0; x < dkd; ++x) acc = fmaf(-W[r * ldk + x], S0[i * ldk + x], acc);
-            U[r * ldv + i] = acc;
-        }
+        // U = T diag(beta) V - W S0^T
+        bgemm<1>(C, R, C, [&](int r, int j) { return Tm[r * ldc + j] * vB[j]; },
+                 [&](int j, int i) { return V[j * ldv + i]; }, [&](int r, int i, float acc) { U[r * ldv + i] = acc; });
+        bgemm<1>(C, R, dkd, [&](int r, int x) { return -W[r * ldk + x]; },
+                 [&](int x, int i) { return S0[i * ldk + x]; }, [&](int r, int i, float acc) { U[r * ldv + i] += acc; });
         __syncthreads();
     };
 
     // ---- pass 1: chunk start states into the workspace ----
-    for (int idx = tid; idx < kBwdRows * dkd; idx += kBwdThreads) {
+    for (int idx = tid; idx < R * dkd; idx += kBwdThreads) {
         const int i = idx / dkd, x = idx % dkd;
         S0[i * ldk + x] = (a.s0 && i < nr) ? a.s0[sbase + size_t(i0 + i) * dkd + x] : 0.f;
     }
     __syncthreads();
     for (int c = 0; c < nch; ++c) {
-        const int Lc = min(kBwdC, len - c * kBwdC);
+        const int Lc = min(C, len - c * C);
         float *dst = ck(c);
         for (int idx = tid; idx < nr * dkd; idx += kBwdThreads) dst[idx] = S0[(idx / dkd) * ldk + idx % dkd];
         chunk_forward(c, Lc);
         const float gl = __expf(vG[Lc - 1]);
-        for (int idx = tid; idx < kBwdRows * dkd; idx += kBwdThreads) {
-            const int i = idx / dkd, x = idx % dkd;
-            float acc = gl * S0[i * ldk + x];
-            for (int j = 0; j < Lc; ++j) acc = fmaf(U[j * ldv + i] * vLam[j], K[j * ldk + x], acc);
-            S0[i * ldk + x] = acc;
-        }
+        // S <- gamma_L S + U^T diag(lambda) K
+        bgemm<4>(R, dkd, Lc, [&](int i, int j) { return U[j * ldv + i] * vLam[j]; },
+                 [&](int j, int x) { return K[j * ldk + x]; },
+                 [&](int i, int x, float acc) { S0[i * ldk + x] = fmaf(gl, S0[i * ldk + x], acc); });
         __syncthreads();
     }
 
     // ---- pass 2: backward over the chunks ----
-    for (int idx = tid; idx < kBwdRows * dkd; idx += kBwdThreads) {
+    for (int idx = tid; idx < R * dkd; idx += kBwdThreads) {
         const int i = idx / dkd, x = idx % dkd;
         dS[i * ldk + x] = (dSf && i < nr) ? dSf[sbase + size_t(i0 + i) * dkd + x] : 0.f;
     }
     for (int c = nch - 1; c >= 0; --c) {
-        const int Lc = min(kBwdC, len - c * kBwdC);
-        const int c0 = t0 + c * kBwdC;
+        const int Lc = min(C, len - c * C);
+        const int c0 = t0 + c * C;
         const float *src = ck(c);
-        for (int idx = tid; idx < kBwdRows * dkd; idx += kBwdThreads) {
+        for (int idx = tid; idx < R * dkd; idx += kBwdThreads) {
             const int i = idx / dkd, x = idx % dkd;
             S0[i * ldk + x] = i < nr ? src[i * dkd + x] : 0.f;
         }
         __syncthreads();
         chunk_forward(c, Lc);
-        for (int idx = tid; idx < kBwdC * kBwdRows; idx += kBwdThreads) {
-            const int r = idx / kBwdRows, i = idx % kBwdRows;
+        for (int idx = tid; idx < C * R; idx += kBwdThreads) {
+            const int r = idx / R, i = idx % R;
             dOs[r * ldv + i] = (r < Lc && i < nr) ? to_f32(dO[(size_t(c0 + r) * hv + h) * dvd + i0 + i]) : 0.f;
         }
-        for (int idx = tid; idx < kBwdC * dkd; idx += kBwdThreads) {
+        for (int idx = tid; idx < C * dkd; idx += kBwdThreads) {
             dQ[(idx / dkd) * ldk + idx % dkd] = 0.f;
             dK[(idx / dkd) * ldk + idx % dkd] = 0.f;
         }
-        if (tid < kBwdC) vdGam[tid] = vdLam[tid] = vdBG[tid] = vdB[tid] = vdG[tid] = 0.f;
+        if (tid < C) vdGam[tid] = vdLam[tid] = vdBG[tid] = vdB[tid] = vdG[tid] = 0.f;
         // dgamma_L = <dS, S0> over the block's rows
         float part = 0.f;
-        for (int idx = tid; idx < kBwdRows * dkd; idx += kBwdThreads) {
+        for (int idx = tid; idx < R * dkd; idx += kBwdThreads) {
             const int i = idx / dkd, x = idx % dkd;
             part = fmaf(dS[i * ldk + x], S0[i * ldk + x], part);
         }
@@ -245,166 +271,114 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
         __syncthreads();
         float dgl = 0.f;
         for (int w = 0; w < kBwdThreads / 32; ++w) dgl += red[w];
-        // dU from the end state, and lambda's gradient: Z_ji = dS_i . k_j
-        for (int idx = tid; idx < kBwdC * kBwdRows; idx += kBwdThreads) {
-            const int j = idx / kBwdRows, i = idx % kBwdRows;
-            float z = 0.f;
-            for (int x = 0; x < dkd; ++x) z = fmaf(dS[i * ldk + x], K[j * ldk + x], z);
-            dU[j * ldv + i] = vLam[j] * z;
-            dT[j * ldc + i] = U[j * ldv + i] * z;  // scratch: U_ji Z_ji, summed below
+        // from the end state: Z_ji = dS_i . k_j, dU = diag(lambda) Z, dlambda_j = sum_i U_ji Z_ji
+        bgemm<1>(C, R, dkd, [&](int j, int x) { return K[j * ldk + x]; }, [&](int x, int i) { return dS[i * ldk + x]; },
+                 [&](int j, int i, float z) {
+                     dU[j * ldv + i] = vLam[j] * z;
+                     dT[j * ldc + i] = U[j * ldv + i] * z;  // scratch, summed below
+                 });
+        // dK_j += lambda_j dS^T u_j;  Y_r = dO_r S0: dQ_r += gamma_r Y_r, dgamma_r += Y_r . q_r
+        bgemm<4>(C, dkd, R, [&](int j, int i) { return U[j * ldv + i]; }, [&](int i, int x) { return dS[i * ldk + x]; },
+                 [&](int j, int x, float acc) { dK[j * ldk + x] += vLam[j] * acc; });
+        bgemm<4>(C, dkd, R, [&](int r, int i) { return dOs[r * ldv + i]; }, [&](int i, int x) { return S0[i * ldk + x]; },
+                 [&](int r, int x, float y) {
+                     dQ[r * ldk + x] += vGam[r] * y;
+                     dW[r * ldk + x] = y * Q[r * ldk + x];  // scratch for dgamma
+                 });
+        __syncthreads();
+        if (tid < C) {
+            float sl = 0.f, sg = 0.f;
+            for (int i = 0; i < R; ++i) sl += dT[tid * ldc + i];
+            for (int x = 0; x < dkd; ++x) sg += dW[tid * ldk + x];
+            vdLam[tid] = sl;
+            vdGam[tid] += sg;
         }
         __syncthreads();
-        if (tid < kBwdC) {
-            float s = 0.f;
-            for (int i = 0; i < kBwdRows; ++i) s += dT[tid * ldc + i];
-            vdLam[tid] = s;
-        }
-        // dK_j += lambda_j dS^T u_j;  output terms: Y_r = dO_r S0 -> dQ_r += gamma_r Y_r, dgamma_r += Y_r . q_r
-        for (int idx = tid; idx < kBwdC * dkd; idx += kBwdThreads) {
-            const int j = idx / dkd, x = idx % dkd;
-            float acc = 0.f, y = 0.f;
-            for (int i = 0; i < kBwdRows; ++i) {
-                acc = fmaf(U[j * ldv + i], dS[i * ldk + x], acc);
-                y = fmaf(dOs[j * ldv + i], S0[i * ldk + x], y);
-            }
-            dK[j * ldk + x] += vLam[j] * acc;
-            dQ[j * ldk + x] += vGam[j] * y;
-            dW[j * ldk + x] = y * Q[j * ldk + x];  // scratch for dgamma
-        }
+        // dP_rj = dO_r . u_j (j <= r), kept in dT's storage
+        bgemm<1>(C, C, R, [&](int r, int i) { return dOs[r * ldv + i]; }, [&](int i, int j) { return U[j * ldv + i]; },
+                 [&](int r, int j, float acc) { dT[r * ldc + j] = j <= r ? acc : 0.f; });
         __syncthreads();
-        if (tid < kBwdC) {
-            float s = 0.f;
-            for (int x = 0; x < dkd; ++x) s += dW[tid * ldk + x];
-            vdGam[tid] += s;
-        }
-        // dP_rj = dO_r . u_j (j <= r); dU_j += sum_r P_rj dO_r
-        for (int p = tid; p < kBwdC * kBwdC; p += kBwdThreads) {
-            const int r = p / kBwdC, j = p % kBwdC;
-            float d = 0.f;
-            if (j <= r)
-                for (int i = 0; i < kBwdRows; ++i) d = fmaf(dOs[r * ldv + i], U[j * ldv + i], d);
-            dT[r * ldc + j] = d;  // dP, kept in dT's storage until dT is formed
-        }
-        __syncthreads();
-        for (int idx = tid; idx < kBwdC * kBwdRows; idx += kBwdThreads) {
-            const int j = idx / kBwdRows, i = idx % kBwdRows;
-            float acc = dU[j * ldv + i];
-            for (int r = j; r < kBwdC; ++r) acc = fmaf(Gm[r * ldc + j] * QK[r * ldc + j], dOs[r * ldv + i], acc);
-            dU[j * ldv + i] = acc;
-        }
-        // P = QK (.) Gamma: dQ_r += sum_j dP_rj Gamma_rj k_j, dK_j += sum_r dP_rj Gamma_rj q_r; dGamma (in dA) = dP QK
-        for (int idx = tid; idx < kBwdC * dkd; idx += kBwdThreads) {
-            const int r = idx / dkd, x = idx % dkd;
-            float aq = 0.f, ak = 0.f;
-            for (int j = 0; j <= r; ++j) aq = fmaf(dT[r * ldc + j] * Gm[r * ldc + j], K[j * ldk + x], aq);
-            for (int i = r; i < kBwdC; ++i) ak = fmaf(dT[i * ldc + r] * Gm[i * ldc + r], Q[i * ldk + x], ak);
-            dQ[r * ldk + x] += aq;
-            dK[r * ldk + x] += ak;
-        }
-        for (int p = tid; p < kBwdC * kBwdC; p += kBwdThreads) {
-            const int r = p / kBwdC, j = p % kBwdC;
+        // dU_j += sum_r P_rj dO_r;  P = Q K^T (.) Gamma: dQ, dK and dGamma (in dA)
+        bgemm<1>(C, R, C, [&](int j, int r) { return Gm[r * ldc + j] * QK[r * ldc + j]; },
+                 [&](int r, int i) { return dOs[r * ldv + i]; }, [&](int j, int i, float acc) { dU[j * ldv + i] += acc; });
+        bgemm<4>(C, dkd, C, [&](int r, int j) { return dT[r * ldc + j] * Gm[r * ldc + j]; },
+                 [&](int j, int x) { return K[j * ldk + x]; }, [&](int r, int x, float acc) { dQ[r * ldk + x] += acc; });
+        bgemm<4>(C, dkd, C, [&](int r, int i) { return dT[i * ldc + r] * Gm[i * ldc + r]; },
+                 [&](int i, int x) { return Q[i * ldk + x]; }, [&](int r, int x, float acc) { dK[r * ldk + x] += acc; });
+        for (int p = tid; p < C * C; p += kBwdThreads) {
+            const int r = p / C, j = p % C;
             dA[r * ldc + j] = j <= r ? dT[r * ldc + j] * QK[r * ldc + j] : 0.f;  // dGamma so far
         }
         __syncthreads();
-        // dW = -dU S0; dS0 = gamma_L dS + dO^T diag(gamma) Q - dU^T W (in place over dS)
-        for (int idx = tid; idx < kBwdC * dkd; idx += kBwdThreads) {
-            const int r = idx / dkd, x = idx % dkd;
-            float acc = 0.f;
-            for (int i = 0; i < kBwdRows; ++i) acc = fmaf(-dU[r * ldv + i], S0[i * ldk + x], acc);
-            dW[r * ldk + x] = acc;
-        }
+        // dW = -dU S0;  dS0 = gamma_L dS + dO^T diag(gamma) Q - dU^T W (over dS)
         const float gL = __expf(vG[Lc - 1]);
-        for (int idx = tid; idx < kBwdRows * dkd; idx += kBwdThreads) {
-            const int i = idx / dkd, x = idx % dkd;
-            float acc = gL * dS[i * ldk + x];
-            for (int r = 0; r < Lc; ++r) {
-                acc = fmaf(dOs[r * ldv + i] * vGam[r], Q[r * ldk + x], acc);
-                acc = fmaf(-dU[r * ldv + i], W[r * ldk + x], acc);
-            }
-            dS[i * ldk + x] = acc;
-        }
+        bgemm<4>(C, dkd, R, [&](int r, int i) { return -dU[r * ldv + i]; }, [&](int i, int x) { return S0[i * ldk + x]; },
+                 [&](int r, int x, float acc) { dW[r * ldk + x] = acc; });
+        bgemm<4>(R, dkd, C, [&](int i, int r) { return dOs[r * ldv + i] * vGam[r]; },
+                 [&](int r, int x) { return Q[r * ldk + x]; },
+                 [&](int i, int x, float acc) { dS[i * ldk + x] = fmaf(gL, dS[i * ldk + x], acc); });
+        bgemm<4>(R, dkd, C, [&](int i, int r) { return -dU[r * ldv + i]; }, [&](int r, int x) { return W[r * ldk + x]; },
+                 [&](int i, int x, float acc) { dS[i * ldk + x] += acc; });
         __syncthreads();
         // dT_rj = dW_r . (bg_j k_j) + dU_r . (beta_j v_j), j <= r
-        for (int p = tid; p < kBwdC * kBwdC; p += kBwdThreads) {
-            const int r = p / kBwdC, j = p % kBwdC;
-            float d = 0.f;
-            if (j <= r) {
-                for (int x = 0; x < dkd; ++x) d = fmaf(dW[r * ldk + x], K[j * ldk + x], d);
-                d *= vBG[j];
-                float e = 0.f;
-                for (int i = 0; i < kBwdRows; ++i) e = fmaf(dU[r * ldv + i], V[j * ldv + i], e);
-                d = fmaf(vB[j], e, d);
-            }
-            dT[r * ldc + j] = d;
-        }
+        bgemm<1>(C, C, dkd, [&](int r, int x) { return dW[r * ldk + x]; },
+                 [&](int x, int j) { return K[j * ldk + x] * vBG[j]; },
+                 [&](int r, int j, float acc) { dT[r * ldc + j] = j <= r ? acc : 0.f; });
+        bgemm<1>(C, C, R, [&](int r, int i) { return dU[r * ldv + i]; }, [&](int i, int j) { return V[j * ldv + i] * vB[j]; },
+                 [&](int r, int j, float acc) {
+                     if (j <= r) dT[r * ldc + j] += acc;
+                 });
         __syncthreads();
-        // dX_j = sum_r T_rj dW_r: dK_j += bg_j dX_j, dbg_j = dX_j . k_j;
-        // dY_j = sum_r T_rj dU_r: dv_j = beta_j dY_j, dbeta_j += dY_j . v_j
-        for (int idx = tid; idx < kBwdC * dkd; idx += kBwdThreads) {
-            const int j = idx / dkd, x = idx % dkd;
-            float dx = 0.f;
-            for (int r = j; r < kBwdC; ++r) dx = fmaf(Tm[r * ldc + j], dW[r * ldk + x], dx);
-            dK[j * ldk + x] = fmaf(vBG[j], dx, dK[j * ldk + x]);
-            Q[j * ldk + x] = dx * K[j * ldk + x];  // scratch for dbg (Q is no longer needed; dW is still read)
-        }
-        for (int idx = tid; idx < kBwdC * kBwdRows; idx += kBwdThreads) {
-            const int j = idx / kBwdRows, i = idx % kBwdRows;
-            float dy = 0.f;
-            for (int r = j; r < kBwdC; ++r) dy = fmaf(Tm[r * ldc + j], dU[r * ldv + i], dy);
-            if (j < Lc && i < nr) dv[(size_t(c0 + j) * hv + h) * dvd + i0 + i] = vB[j] * dy;
-            U[j * ldv + i] = dy * V[j * ldv + i];  // scratch for dbeta (U is no longer needed)
-        }
+        // dX = T^T dW: dK_j += bg_j dX_j, dbg_j = dX_j . k_j;  dY = T^T dU: dv_j = beta_j dY_j, dbeta_j += dY_j . v_j
+        bgemm<4>(C, dkd, C, [&](int j, int r) { return Tm[r * ldc + j]; }, [&](int r, int x) { return dW[r * ldk + x]; },
+                 [&](int j, int x, float dx) {
+                     dK[j * ldk + x] = fmaf(vBG[j], dx, dK[j * ldk + x]);
+                     Q[j * ldk + x] = dx * K[j * ldk + x];  // scratch for dbg (Q is no longer needed)
+                 });
+        bgemm<1>(C, R, C, [&](int j, int r) { return Tm[r * ldc + j]; }, [&](int r, int i) { return dU[r * ldv + i]; },
+                 [&](int j, int i, float dy) {
+                     if (j < Lc && i < nr) dv[(size_t(c0 + j) * hv + h) * dvd + i0 + i] = vB[j] * dy;
+                     U[j * ldv + i] = dy * V[j * ldv + i];  // scratch for dbeta (U is no longer needed)
+                 });
         __syncthreads();
-        if (tid < kBwdC) {
-            float s = 0.f;
-            for (int x = 0; x < dkd; ++x) s += Q[tid * ldk + x];
-            vdBG[tid] = s;
-            float b = 0.f;
-            for (int i = 0; i < kBwdRows; ++i) b += U[tid * ldv + i];
-            vdB[tid] = b;
+        if (tid < C) {
+            float sb = 0.f, su = 0.f;
+            for (int x = 0; x < dkd; ++x) sb += Q[tid * ldk + x];
+            for (int i = 0; i < R; ++i) su += U[tid * ldv + i];
+            vdBG[tid] = sb;
+            vdB[tid] = su;
         }
-        // dA = -T^T dT T^T (strictly lower): first M = dT T^T
-        for (int p = tid; p < kBwdC * kBwdC; p += kBwdThreads) {
-            const int r = p / kBwdC, j = p % kBwdC;
-            float acc = 0.f;
-            for (int m = 0; m <= j; ++m) acc = fmaf(dT[r * ldc + m], Tm[j * ldc + m], acc);
-            sM[r * ldc + j] = acc;
-        }
+        // dA = -T^T dT T^T (strictly lower): M = dT T^T first
+        bgemm<1>(C, C, C, [&](int r, int m) { return dT[r * ldc + m]; }, [&](int m, int j) { return Tm[j * ldc + m]; },
+                 [&](int r, int j, float acc) { sM[r * ldc + j] = acc; });
         __syncthreads();
-        for (int p = tid; p < kBwdC * kBwdC; p += kBwdThreads) {
-            const int r = p / kBwdC, j = p % kBwdC;
-            float acc = 0.f;
-            if (j < r)
-                for (int m = r; m < kBwdC; ++m) acc = fmaf(Tm[m * ldc + r], sM[m * ldc + j], acc);
-            // A_rj = beta_r Gamma_rj KK_rj: dbeta_r, dGamma_rj, and dKK_rj into dT's storage
-            const float da = -acc;
-            dT[r * ldc + j] = j < r ? da * vB[r] * Gm[r * ldc + j] : 0.f;
-            if (j < r) dA[r * ldc + j] += da * vB[r] * KK[r * ldc + j];
-            sE[r * ldc + j] = j < r ? da * Gm[r * ldc + j] * KK[r * ldc + j] : 0.f;  // dbeta terms
-        }
+        // A_rj = beta_r Gamma_rj KK_rj: dbeta_r terms (sE), dGamma_rj (dA), dKK_rj (dT)
+        bgemm<1>(C, C, C, [&](int r, int m) { return Tm[m * ldc + r]; }, [&](int m, int j) { return sM[m * ldc + j]; },
+                 [&](int r, int j, float acc) {
+                     const float da = -acc;
+                     const bool low = j < r;
+                     dT[r * ldc + j] = low ? da * vB[r] * Gm[r * ldc + j] : 0.f;
+                     if (low) dA[r * ldc + j] += da * vB[r] * KK[r * ldc + j];
+                     sE[r * ldc + j] = low ? da * Gm[r * ldc + j] * KK[r * ldc + j] : 0.f;
+                 });
         __syncthreads();
-        if (tid < kBwdC) {
-            float s = 0.f;
-            for (int j = 0; j < tid; ++j) s += sE[tid * ldc + j];
-            vdB[tid] += s;
+        if (tid < C) {
+            float sv = 0.f;
+            for (int j = 0; j < tid; ++j) sv += sE[tid * ldc + j];
+            vdB[tid] += sv;
         }
-        // dK_r += sum_j dKK_rj k_j + sum_j dKK_jr k_j
-        for (int idx = tid; idx < kBwdC * dkd; idx += kBwdThreads) {
-            const int r = idx / dkd, x = idx % dkd;
-            float acc = 0.f;
-            for (int j = 0; j < r; ++j) acc = fmaf(dT[r * ldc + j], K[j * ldk + x], acc);
-            for (int j = r + 1; j < kBwdC; ++j) acc = fmaf(dT[j * ldc + r], K[j * ldk + x], acc);
-            dK[r * ldk + x] += acc;
-        }
+        // dK_r += sum_j (dKK_rj + dKK_jr) k_j
+        bgemm<4>(C, dkd, C, [&](int r, int j) { return j < r ? dT[r * ldc + j] : (j > r ? dT[j * ldc + r] : 0.f); },
+                 [&](int j, int x) { return K[j * ldk + x]; }, [&](int r, int x, float acc) { dK[r * ldk + x] += acc; });
         __syncthreads();
         // decays: beta gamma, gamma, lambda, gamma_L and Gamma through G, then dg = reverse prefix sums
-        if (tid < kBwdC) {
+        if (tid < C) {
             const int r = tid;
             vdB[r] = fmaf(vdBG[r], vGam[r], vdB[r]);
             const float dgam = fmaf(vdBG[r], vB[r], vdGam[r]);
             float dG = dgam * vGam[r] - vdLam[r] * vLam[r];
             for (int j = 0; j <= r; ++j) dG = fmaf(dA[r * ldc + j], Gm[r * ldc + j], dG);
-            for (int i = r; i < kBwdC; ++i) dG = fmaf(-dA[i * ldc + r], Gm[i * ldc + r], dG);
+            for (int i = r; i < C; ++i) dG = fmaf(-dA[i * ldc + r], Gm[i * ldc + r], dG);
             vdG[r] = dG;
         }
         __syncthreads();
