@@ -340,10 +340,10 @@ GDN_API gdn_status_t gdn_decode_commit(int32_t num_seqs, int32_t num_tokens, int
  *   d_initial_state    [N, Hv, d_v, d_k] fp32, or NULL
  * Inputs are those of gdn_chunk_forward (the plain path: no input-side
  * flags, GDN_ERR_UNSUPPORTED otherwise); d_o has the dtype of v.  fp32 on
- * CUDA cores: the forward chunk states are recomputed and kept in the
- * workspace (one d_v x d_k state per 32-token chunk and value head, plus
- * the schedule; gdn_chunk_backward_workspace_size), then the chunks are
- * walked backward.  dq, dk, dg and dbeta are accumulated with atomic adds
+ * CUDA cores: a forward pass keeps each 32-token chunk's start state and
+ * its intra-chunk products in the workspace (about 3 d_v d_k fp32 values
+ * per chunk and value head, plus the schedule; gdn_chunk_backward_
+ * workspace_size), then the chunks are walked backward.  dq, dk, dg and dbeta are accumulated with atomic adds
  * (their summation order, and so their last bits, can vary between runs).
  * d_k, d_v <= 128. */
 GDN_API gdn_status_t gdn_chunk_backward_workspace_size(const gdn_shape_t *shape, size_t *bytes);

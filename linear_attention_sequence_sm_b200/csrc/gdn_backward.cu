@@ -72,6 +72,11 @@ __host__ __device__ inline BwdSmem bwd_smem(int dk) {
 // per-token vectors inside the vec block
 enum { kVG = 0, kVGam, kVLam, kVB, kVBG, kVDG, kVDGam, kVDLam, kVDBG, kVDB, kVNum };
 
+// floats kept per (chunk, value head, row slice) for pass 2: K K^T, Q K^T, T, W, U
+__host__ __device__ inline size_t bwd_keep_floats(int dk) {
+    return size_t(3) * kBwdC * kBwdC + size_t(kBwdC) * dk + size_t(kBwdC) * kBwdRows;
+}
+
 // checkpoint slot of chunk c of the sequence starting at token t0, sequence n:
 // floor(t0 / C) + n + c never collides between sequences
 __device__ __forceinline__ size_t bwd_slot(int t0, int n, int c) { return size_t(t0 / kBwdC + n + c); }
@@ -114,7 +119,7 @@ __device__ __forceinline__ void bgemm(int M, int N, int K, FA a, FB b, FO out) {
 template <typename T>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, float *dq, float *dk, float *dv,
-                      float *dg, float *dbeta, float *dS0_out, float *ckpt, int n_slices) {
+                      float *dg, float *dbeta, float *dS0_out, float *ckpt, float *keep, int n_slices) {
     if (a.sched.hdr->status != GDN_OK) return;
     extern __shared__ float smem[];
     const int dkd = a.dk, dvd = a.dv, hv = a.hv, hk = a.hk;
@@ -148,10 +153,13 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
     const size_t sbase = (size_t(seq) * hv + h) * size_t(dvd) * dkd;
     const int nch = (len + kBwdC - 1) / kBwdC;
     auto ck = [&](int c) { return ckpt + (bwd_slot(t0, seq, c) * hv + h) * size_t(dvd) * dkd + size_t(i0) * dkd; };
+    // pass 1 keeps the chunk's K K^T, Q K^T, T, W and U (this block's rows) for pass 2
+    const size_t keep_sz = bwd_keep_floats(dkd);
+    auto kp = [&](int c) { return keep + ((bwd_slot(t0, seq, c) * hv + h) * n_slices + slice) * keep_sz; };
 
-    // one chunk's inputs and forward quantities (A, T, W, U~, U; the masks)
+    // one chunk's inputs, prefix sums, per-token decays and Gamma
     constexpr int C = kBwdC, R = kBwdRows;
-    auto chunk_forward = [&](int c, int Lc) {
+    auto chunk_inputs = [&](int c, int Lc) {
         const int c0 = t0 + c * C;
         for (int idx = tid; idx < C * dkd; idx += kBwdThreads) {
             const int r = idx / dkd, x = idx % dkd;
@@ -176,11 +184,6 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
                 vG[r] = run;
             }
         }
-        // K K^T and Q K^T (lower, with the diagonal)
-        bgemm<1>(C, C, dkd, [&](int r, int x) { return K[r * ldk + x]; }, [&](int x, int j) { return K[j * ldk + x]; },
-                 [&](int r, int j, float acc) { KK[r * ldc + j] = j <= r ? acc : 0.f; });
-        bgemm<1>(C, C, dkd, [&](int r, int x) { return Q[r * ldk + x]; }, [&](int x, int j) { return K[j * ldk + x]; },
-                 [&](int r, int j, float acc) { QK[r * ldc + j] = j <= r ? acc : 0.f; });
         __syncthreads();
         if (tid < C) {
             const float gam = __expf(vG[tid]);
@@ -192,6 +195,15 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
             const int r = p / C, j = p % C;
             Gm[r * ldc + j] = j <= r ? __expf(vG[r] - vG[j]) : 0.f;
         }
+        __syncthreads();
+    };
+    // the chunk's products: K K^T, Q K^T, T, W, U (after chunk_inputs)
+    auto chunk_products = [&]() {
+        // K K^T and Q K^T (lower, with the diagonal)
+        bgemm<1>(C, C, dkd, [&](int r, int x) { return K[r * ldk + x]; }, [&](int x, int j) { return K[j * ldk + x]; },
+                 [&](int r, int j, float acc) { KK[r * ldc + j] = j <= r ? acc : 0.f; });
+        bgemm<1>(C, C, dkd, [&](int r, int x) { return Q[r * ldk + x]; }, [&](int x, int j) { return K[j * ldk + x]; },
+                 [&](int r, int j, float acc) { QK[r * ldc + j] = j <= r ? acc : 0.f; });
         __syncthreads();
         // T = (I + A)^-1, A_rj = beta_r Gamma_rj KK_rj (j < r); one column per thread
         if (tid < C) {
@@ -216,6 +228,26 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
         __syncthreads();
     };
 
+    // K K^T, Q K^T, T (C x C each), W (C x d_k), U (C x 32) to / from the workspace
+    auto keep_io = [&](float *base, bool store) {
+        for (int e = tid; e < 3 * C * C; e += kBwdThreads) {
+            const int m = e / (C * C), r = (e / C) % C, j = e % C;
+            float *sm_ = m == 0 ? KK : (m == 1 ? QK : Tm);
+            if (store) base[e] = sm_[r * ldc + j];
+            else sm_[r * ldc + j] = base[e];
+        }
+        float *bw = base + 3 * C * C;
+        for (int e = tid; e < C * dkd; e += kBwdThreads) {
+            if (store) bw[e] = W[(e / dkd) * ldk + e % dkd];
+            else W[(e / dkd) * ldk + e % dkd] = bw[e];
+        }
+        float *bu = bw + C * dkd;
+        for (int e = tid; e < C * R; e += kBwdThreads) {
+            if (store) bu[e] = U[(e / R) * ldv + e % R];
+            else U[(e / R) * ldv + e % R] = bu[e];
+        }
+    };
+
     // ---- pass 1: chunk start states into the workspace ----
     for (int idx = tid; idx < R * dkd; idx += kBwdThreads) {
         const int i = idx / dkd, x = idx % dkd;
@@ -226,7 +258,9 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
         const int Lc = min(C, len - c * C);
         float *dst = ck(c);
         for (int idx = tid; idx < nr * dkd; idx += kBwdThreads) dst[idx] = S0[(idx / dkd) * ldk + idx % dkd];
-        chunk_forward(c, Lc);
+        chunk_inputs(c, Lc);
+        chunk_products();
+        keep_io(kp(c), true);
         const float gl = __expf(vG[Lc - 1]);
         // S <- gamma_L S + U^T diag(lambda) K
         bgemm<4>(R, dkd, Lc, [&](int i, int j) { return U[j * ldv + i] * vLam[j]; },
@@ -249,7 +283,8 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
             S0[i * ldk + x] = i < nr ? src[i * dkd + x] : 0.f;
         }
         __syncthreads();
-        chunk_forward(c, Lc);
+        chunk_inputs(c, Lc);
+        keep_io(kp(c), false);
         for (int idx = tid; idx < C * R; idx += kBwdThreads) {
             const int r = idx / R, i = idx % R;
             dOs[r * ldv + i] = (r < Lc && i < nr) ? to_f32(dO[(size_t(c0 + r) * hv + h) * dvd + i0 + i]) : 0.f;
@@ -413,9 +448,14 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
         }
 }
 
+static size_t bwd_slots(int32_t tokens, int32_t num_seqs) { return size_t(tokens) / kBwdC + size_t(num_seqs) + 1; }
+
+// chunk start states, then the kept per-chunk quantities (256-byte aligned)
 size_t backward_ckpt_bytes(int32_t tokens, int32_t num_seqs, int32_t hv, int32_t dk, int32_t dv) {
-    const size_t slots = size_t(tokens) / kBwdC + size_t(num_seqs) + 1;
-    return slots * size_t(hv) * size_t(dv) * size_t(dk) * sizeof(float);
+    const size_t slots = bwd_slots(tokens, num_seqs);
+    const size_t states = (slots * size_t(hv) * size_t(dv) * size_t(dk) * sizeof(float) + 255) / 256 * 256;
+    const size_t n_slices = (size_t(dv) + kBwdRows - 1) / kBwdRows;
+    return states + slots * size_t(hv) * n_slices * bwd_keep_floats(dk) * sizeof(float);
 }
 
 cudaError_t launch_chunk_backward(const PrefillArgs &a, const void *dO, const float *dSf, float *dq, float *dk,
@@ -425,19 +465,23 @@ cudaError_t launch_chunk_backward(const PrefillArgs &a, const void *dO, const fl
     if (blocks <= 0) return cudaSuccess;
     if (blocks > INT32_MAX || a.dk > 128 || a.dv > 128) return cudaErrorInvalidValue;
     const size_t bytes = bwd_smem(a.dk).total * sizeof(float);
+    const size_t slots = bwd_slots(a.tokens, a.num_seqs);
+    float *keep = ckpt + (slots * size_t(a.hv) * size_t(a.dv) * size_t(a.dk) * sizeof(float) + 255) / 256 * 256 /
+                             sizeof(float);
     cudaError_t e;
     if (a.dtype == GDN_DTYPE_BF16) {
         e = cudaFuncSetAttribute(chunk_backward_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(bytes));
         if (e != cudaSuccess) return e;
         chunk_backward_kernel<__nv_bfloat16><<<unsigned(blocks), kBwdThreads, bytes, stream>>>(
-            a, dO, dSf, dq, dk, dv, dg, dbeta, dS0, ckpt, n_slices);
+            a, dO, dSf, dq, dk, dv, dg, dbeta, dS0, ckpt, keep, n_slices);
     } else {
         e = cudaFuncSetAttribute(chunk_backward_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(bytes));
         if (e != cudaSuccess) return e;
         chunk_backward_kernel<float><<<unsigned(blocks), kBwdThreads, bytes, stream>>>(a, dO, dSf, dq, dk, dv, dg,
-                                                                                      dbeta, dS0, ckpt, n_slices);
+                                                                                      dbeta, dS0, ckpt, keep,
+                                                                                      n_slices);
     }
     count_launch();
     return cudaGetLastError();
