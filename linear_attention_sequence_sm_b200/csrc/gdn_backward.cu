@@ -24,6 +24,8 @@
 // Pass 1 runs the chunks forward and stores each chunk's start state (the
 // block's rows) in the workspace; pass 2 walks the chunks backward,
 // recomputing the chunk's forward quantities from its stored start state.
+#include <type_traits>
+
 #include "gdn_internal.cuh"
 
 namespace gdn {
@@ -116,12 +118,79 @@ __device__ __forceinline__ void bgemm(int M, int N, int K, FA a, FB b, FO out) {
             if (m0 + j < M && l + 32 * i < N) out(m0 + j, l + 32 * i, acc[j][i]);
 }
 
+// The same contract on the tensor cores: 16 x 8 output tiles per warp
+// (mma.sync m16n8k16, fp32 accumulation), tiles dealt to the 8 warps in a
+// fixed order, so again a given (M, N) always maps an element to the same
+// thread.  Each fp32 operand is split into a bf16 value and a bf16 residual,
+// x = hi + lo, and a b is formed as hi hi + hi lo + lo hi: about 16
+// mantissa bits, near the fp32 products of the CUDA-core path (the
+// gradients of the decays are sums with heavy cancellation, which a plain
+// bf16 product does not resolve).
+__device__ __forceinline__ void bwd_split2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+__device__ __forceinline__ void bwd_mma(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+template <class FA, class FB, class FO>
+__device__ __forceinline__ void tgemm(int M, int N, int K, FA a, FB b, FO out) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int mt = (M + 15) / 16, nt = (N + 7) / 8;
+    for (int tile = warp; tile < mt * nt; tile += kBwdThreads / 32) {
+        const int m0 = (tile % mt) * 16, n0 = (tile / mt) * 8;
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int k0 = 0; k0 < K; k0 += 16) {
+            auto A = [&](int r, int c) {
+                const int m = m0 + r, kk = k0 + c;
+                return (m < M && kk < K) ? a(m, kk) : 0.f;
+            };
+            auto B = [&](int r, int c) {
+                const int kk = k0 + r, n = n0 + c;
+                return (kk < K && n < N) ? b(kk, n) : 0.f;
+            };
+            uint32_t ah[4], al[4], bh[2], bl[2];
+            bwd_split2(A(g, 2 * t), A(g, 2 * t + 1), ah[0], al[0]);
+            bwd_split2(A(g + 8, 2 * t), A(g + 8, 2 * t + 1), ah[1], al[1]);
+            bwd_split2(A(g, 2 * t + 8), A(g, 2 * t + 9), ah[2], al[2]);
+            bwd_split2(A(g + 8, 2 * t + 8), A(g + 8, 2 * t + 9), ah[3], al[3]);
+            bwd_split2(B(2 * t, g), B(2 * t + 1, g), bh[0], bl[0]);
+            bwd_split2(B(2 * t + 8, g), B(2 * t + 9, g), bh[1], bl[1]);
+            bwd_mma(d, al, bh);
+            bwd_mma(d, ah, bl);
+            bwd_mma(d, ah, bh);
+        }
+        const int r0 = m0 + g, c0 = n0 + 2 * t;
+        if (r0 < M && c0 < N) out(r0, c0, d[0]);
+        if (r0 < M && c0 + 1 < N) out(r0, c0 + 1, d[1]);
+        if (r0 + 8 < M && c0 < N) out(r0 + 8, c0, d[2]);
+        if (r0 + 8 < M && c0 + 1 < N) out(r0 + 8, c0 + 1, d[3]);
+    }
+}
+
+// bf16 inputs: tensor-core tiles with split operands; fp32 inputs: fp32 CUDA-core tiles.
+template <bool kTC, int TN, class FA, class FB, class FO>
+__device__ __forceinline__ void prod(int M, int N, int K, FA a, FB b, FO out) {
+    if constexpr (kTC) tgemm(M, N, K, a, b, out);
+    else bgemm<TN>(M, N, K, a, b, out);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, float *dq, float *dk, float *dv,
                       float *dg, float *dbeta, float *dS0_out, float *ckpt, float *keep, int n_slices) {
     if (a.sched.hdr->status != GDN_OK) return;
     extern __shared__ float smem[];
+    constexpr bool kTC = std::is_same<T, __nv_bfloat16>::value;
     const int dkd = a.dk, dvd = a.dv, hv = a.hv, hk = a.hk;
     const BwdSmem L = bwd_smem(dkd);
     const int ldk = L.ldk, ldc = L.ldc, ldv = L.ldv;
@@ -200,9 +269,9 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
     // the chunk's products: K K^T, Q K^T, T, W, U (after chunk_inputs)
     auto chunk_products = [&]() {
         // K K^T and Q K^T (lower, with the diagonal)
-        bgemm<1>(C, C, dkd, [&](int r, int x) { return K[r * ldk + x]; }, [&](int x, int j) { return K[j * ldk + x]; },
+        prod<kTC, 1>(C, C, dkd, [&](int r, int x) { return K[r * ldk + x]; }, [&](int x, int j) { return K[j * ldk + x]; },
                  [&](int r, int j, float acc) { KK[r * ldc + j] = j <= r ? acc : 0.f; });
-        bgemm<1>(C, C, dkd, [&](int r, int x) { return Q[r * ldk + x]; }, [&](int x, int j) { return K[j * ldk + x]; },
+        prod<kTC, 1>(C, C, dkd, [&](int r, int x) { return Q[r * ldk + x]; }, [&](int x, int j) { return K[j * ldk + x]; },
                  [&](int r, int j, float acc) { QK[r * ldc + j] = j <= r ? acc : 0.f; });
         __syncthreads();
         // T = (I + A)^-1, A_rj = beta_r Gamma_rj KK_rj (j < r); one column per thread
@@ -217,13 +286,13 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
         }
         __syncthreads();
         // W = T diag(beta gamma) K
-        bgemm<4>(C, dkd, C, [&](int r, int j) { return Tm[r * ldc + j] * vBG[j]; },
+        prod<kTC, 4>(C, dkd, C, [&](int r, int j) { return Tm[r * ldc + j] * vBG[j]; },
                  [&](int j, int x) { return K[j * ldk + x]; }, [&](int r, int x, float acc) { W[r * ldk + x] = acc; });
         __syncthreads();
         // U = T diag(beta) V - W S0^T
-        bgemm<1>(C, R, C, [&](int r, int j) { return Tm[r * ldc + j] * vB[j]; },
+        prod<kTC, 1>(C, R, C, [&](int r, int j) { return Tm[r * ldc + j] * vB[j]; },
                  [&](int j, int i) { return V[j * ldv + i]; }, [&](int r, int i, float acc) { U[r * ldv + i] = acc; });
-        bgemm<1>(C, R, dkd, [&](int r, int x) { return -W[r * ldk + x]; },
+        prod<kTC, 1>(C, R, dkd, [&](int r, int x) { return -W[r * ldk + x]; },
                  [&](int x, int i) { return S0[i * ldk + x]; }, [&](int r, int i, float acc) { U[r * ldv + i] += acc; });
         __syncthreads();
     };
@@ -263,7 +332,7 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
         keep_io(kp(c), true);
         const float gl = __expf(vG[Lc - 1]);
         // S <- gamma_L S + U^T diag(lambda) K
-        bgemm<4>(R, dkd, Lc, [&](int i, int j) { return U[j * ldv + i] * vLam[j]; },
+        prod<kTC, 4>(R, dkd, Lc, [&](int i, int j) { return U[j * ldv + i] * vLam[j]; },
                  [&](int j, int x) { return K[j * ldk + x]; },
                  [&](int i, int x, float acc) { S0[i * ldk + x] = fmaf(gl, S0[i * ldk + x], acc); });
         __syncthreads();
@@ -307,15 +376,15 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
         float dgl = 0.f;
         for (int w = 0; w < kBwdThreads / 32; ++w) dgl += red[w];
         // from the end state: Z_ji = dS_i . k_j, dU = diag(lambda) Z, dlambda_j = sum_i U_ji Z_ji
-        bgemm<1>(C, R, dkd, [&](int j, int x) { return K[j * ldk + x]; }, [&](int x, int i) { return dS[i * ldk + x]; },
+        prod<kTC, 1>(C, R, dkd, [&](int j, int x) { return K[j * ldk + x]; }, [&](int x, int i) { return dS[i * ldk + x]; },
                  [&](int j, int i, float z) {
                      dU[j * ldv + i] = vLam[j] * z;
                      dT[j * ldc + i] = U[j * ldv + i] * z;  // scratch, summed below
                  });
         // dK_j += lambda_j dS^T u_j;  Y_r = dO_r S0: dQ_r += gamma_r Y_r, dgamma_r += Y_r . q_r
-        bgemm<4>(C, dkd, R, [&](int j, int i) { return U[j * ldv + i]; }, [&](int i, int x) { return dS[i * ldk + x]; },
+        prod<kTC, 4>(C, dkd, R, [&](int j, int i) { return U[j * ldv + i]; }, [&](int i, int x) { return dS[i * ldk + x]; },
                  [&](int j, int x, float acc) { dK[j * ldk + x] += vLam[j] * acc; });
-        bgemm<4>(C, dkd, R, [&](int r, int i) { return dOs[r * ldv + i]; }, [&](int i, int x) { return S0[i * ldk + x]; },
+        prod<kTC, 4>(C, dkd, R, [&](int r, int i) { return dOs[r * ldv + i]; }, [&](int i, int x) { return S0[i * ldk + x]; },
                  [&](int r, int x, float y) {
                      dQ[r * ldk + x] += vGam[r] * y;
                      dW[r * ldk + x] = y * Q[r * ldk + x];  // scratch for dgamma
@@ -330,15 +399,15 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
         }
         __syncthreads();
         // dP_rj = dO_r . u_j (j <= r), kept in dT's storage
-        bgemm<1>(C, C, R, [&](int r, int i) { return dOs[r * ldv + i]; }, [&](int i, int j) { return U[j * ldv + i]; },
+        prod<kTC, 1>(C, C, R, [&](int r, int i) { return dOs[r * ldv + i]; }, [&](int i, int j) { return U[j * ldv + i]; },
                  [&](int r, int j, float acc) { dT[r * ldc + j] = j <= r ? acc : 0.f; });
         __syncthreads();
         // dU_j += sum_r P_rj dO_r;  P = Q K^T (.) Gamma: dQ, dK and dGamma (in dA)
-        bgemm<1>(C, R, C, [&](int j, int r) { return Gm[r * ldc + j] * QK[r * ldc + j]; },
+        prod<kTC, 1>(C, R, C, [&](int j, int r) { return Gm[r * ldc + j] * QK[r * ldc + j]; },
                  [&](int r, int i) { return dOs[r * ldv + i]; }, [&](int j, int i, float acc) { dU[j * ldv + i] += acc; });
-        bgemm<4>(C, dkd, C, [&](int r, int j) { return dT[r * ldc + j] * Gm[r * ldc + j]; },
+        prod<kTC, 4>(C, dkd, C, [&](int r, int j) { return dT[r * ldc + j] * Gm[r * ldc + j]; },
                  [&](int j, int x) { return K[j * ldk + x]; }, [&](int r, int x, float acc) { dQ[r * ldk + x] += acc; });
-        bgemm<4>(C, dkd, C, [&](int r, int i) { return dT[i * ldc + r] * Gm[i * ldc + r]; },
+        prod<kTC, 4>(C, dkd, C, [&](int r, int i) { return dT[i * ldc + r] * Gm[i * ldc + r]; },
                  [&](int i, int x) { return Q[i * ldk + x]; }, [&](int r, int x, float acc) { dK[r * ldk + x] += acc; });
         for (int p = tid; p < C * C; p += kBwdThreads) {
             const int r = p / C, j = p % C;
@@ -347,30 +416,30 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
         __syncthreads();
         // dW = -dU S0;  dS0 = gamma_L dS + dO^T diag(gamma) Q - dU^T W (over dS)
         const float gL = __expf(vG[Lc - 1]);
-        bgemm<4>(C, dkd, R, [&](int r, int i) { return -dU[r * ldv + i]; }, [&](int i, int x) { return S0[i * ldk + x]; },
+        prod<kTC, 4>(C, dkd, R, [&](int r, int i) { return -dU[r * ldv + i]; }, [&](int i, int x) { return S0[i * ldk + x]; },
                  [&](int r, int x, float acc) { dW[r * ldk + x] = acc; });
-        bgemm<4>(R, dkd, C, [&](int i, int r) { return dOs[r * ldv + i] * vGam[r]; },
+        prod<kTC, 4>(R, dkd, C, [&](int i, int r) { return dOs[r * ldv + i] * vGam[r]; },
                  [&](int r, int x) { return Q[r * ldk + x]; },
                  [&](int i, int x, float acc) { dS[i * ldk + x] = fmaf(gL, dS[i * ldk + x], acc); });
-        bgemm<4>(R, dkd, C, [&](int i, int r) { return -dU[r * ldv + i]; }, [&](int r, int x) { return W[r * ldk + x]; },
+        prod<kTC, 4>(R, dkd, C, [&](int i, int r) { return -dU[r * ldv + i]; }, [&](int r, int x) { return W[r * ldk + x]; },
                  [&](int i, int x, float acc) { dS[i * ldk + x] += acc; });
         __syncthreads();
         // dT_rj = dW_r . (bg_j k_j) + dU_r . (beta_j v_j), j <= r
-        bgemm<1>(C, C, dkd, [&](int r, int x) { return dW[r * ldk + x]; },
+        prod<kTC, 1>(C, C, dkd, [&](int r, int x) { return dW[r * ldk + x]; },
                  [&](int x, int j) { return K[j * ldk + x] * vBG[j]; },
                  [&](int r, int j, float acc) { dT[r * ldc + j] = j <= r ? acc : 0.f; });
-        bgemm<1>(C, C, R, [&](int r, int i) { return dU[r * ldv + i]; }, [&](int i, int j) { return V[j * ldv + i] * vB[j]; },
+        prod<kTC, 1>(C, C, R, [&](int r, int i) { return dU[r * ldv + i]; }, [&](int i, int j) { return V[j * ldv + i] * vB[j]; },
                  [&](int r, int j, float acc) {
                      if (j <= r) dT[r * ldc + j] += acc;
                  });
         __syncthreads();
         // dX = T^T dW: dK_j += bg_j dX_j, dbg_j = dX_j . k_j;  dY = T^T dU: dv_j = beta_j dY_j, dbeta_j += dY_j . v_j
-        bgemm<4>(C, dkd, C, [&](int j, int r) { return Tm[r * ldc + j]; }, [&](int r, int x) { return dW[r * ldk + x]; },
+        prod<kTC, 4>(C, dkd, C, [&](int j, int r) { return Tm[r * ldc + j]; }, [&](int r, int x) { return dW[r * ldk + x]; },
                  [&](int j, int x, float dx) {
                      dK[j * ldk + x] = fmaf(vBG[j], dx, dK[j * ldk + x]);
                      Q[j * ldk + x] = dx * K[j * ldk + x];  // scratch for dbg (Q is no longer needed)
                  });
-        bgemm<1>(C, R, C, [&](int j, int r) { return Tm[r * ldc + j]; }, [&](int r, int i) { return dU[r * ldv + i]; },
+        prod<kTC, 1>(C, R, C, [&](int j, int r) { return Tm[r * ldc + j]; }, [&](int r, int i) { return dU[r * ldv + i]; },
                  [&](int j, int i, float dy) {
                      if (j < Lc && i < nr) dv[(size_t(c0 + j) * hv + h) * dvd + i0 + i] = vB[j] * dy;
                      U[j * ldv + i] = dy * V[j * ldv + i];  // scratch for dbeta (U is no longer needed)
@@ -384,11 +453,11 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
             vdB[tid] = su;
         }
         // dA = -T^T dT T^T (strictly lower): M = dT T^T first
-        bgemm<1>(C, C, C, [&](int r, int m) { return dT[r * ldc + m]; }, [&](int m, int j) { return Tm[j * ldc + m]; },
+        prod<kTC, 1>(C, C, C, [&](int r, int m) { return dT[r * ldc + m]; }, [&](int m, int j) { return Tm[j * ldc + m]; },
                  [&](int r, int j, float acc) { sM[r * ldc + j] = acc; });
         __syncthreads();
         // A_rj = beta_r Gamma_rj KK_rj: dbeta_r terms (sE), dGamma_rj (dA), dKK_rj (dT)
-        bgemm<1>(C, C, C, [&](int r, int m) { return Tm[m * ldc + r]; }, [&](int m, int j) { return sM[m * ldc + j]; },
+        prod<kTC, 1>(C, C, C, [&](int r, int m) { return Tm[m * ldc + r]; }, [&](int m, int j) { return sM[m * ldc + j]; },
                  [&](int r, int j, float acc) {
                      const float da = -acc;
                      const bool low = j < r;
@@ -403,7 +472,7 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
             vdB[tid] += sv;
         }
         // dK_r += sum_j (dKK_rj + dKK_jr) k_j
-        bgemm<4>(C, dkd, C, [&](int r, int j) { return j < r ? dT[r * ldc + j] : (j > r ? dT[j * ldc + r] : 0.f); },
+        prod<kTC, 4>(C, dkd, C, [&](int r, int j) { return j < r ? dT[r * ldc + j] : (j > r ? dT[j * ldc + r] : 0.f); },
                  [&](int j, int x) { return K[j * ldk + x]; }, [&](int r, int x, float acc) { dK[r * ldk + x] += acc; });
         __syncthreads();
         // decays: beta gamma, gamma, lambda, gamma_L and Gamma through G, then dg = reverse prefix sums

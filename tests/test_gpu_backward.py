@@ -4,11 +4,14 @@ section; "Gated Attention Architectures", sections 2 and 3), per
 (sequence, head) slice: dq, dk per q/k head, dv, dg, dbeta per value head,
 and the initial-state gradient.
 
-The kernel computes in fp32 from the given (bf16 or fp32) values, so both
-input types are held to one bar, GRAD_BAR: fp32 rounding over sums of
-O(C d) terms per chunk, carried through T / C chunks of the state-gradient
-recurrence, stays well below 1e-4 relative on these sizes; 2e-4 leaves room
-for the atomic summation order of dq, dk, dg and dbeta."""
+Bars, GRAD_BAR by input type:
+- fp32 inputs: the products run in fp32 on CUDA cores.  fp32 rounding over
+  sums of O(C d) terms per chunk, carried through T / C chunks of the
+  state-gradient recurrence, stays well below 1e-4 relative on these sizes;
+  2e-4 leaves room for the atomic summation order of dq, dk, dg and dbeta.
+- bf16 inputs: the products run on the tensor cores, each fp32 operand
+  split into a bf16 value and a bf16 residual (three products per tile,
+  about 16 mantissa bits, fp32 accumulation); the same 2e-4 holds."""
 import numpy as np
 import pytest
 import torch
@@ -19,7 +22,7 @@ from parity import to_f64, slices
 pytestmark = pytest.mark.gpu
 
 DEV = torch.device("cuda:0")
-GRAD_BAR = 2e-4
+GRAD_BAR = {"f32": 2e-4, "bf16": 2e-4}
 
 
 def bwd_inputs(seed, B, T, hk, hv, d, dtype, seq_lens=None, s0_std=0.05):
@@ -74,7 +77,7 @@ def test_backward_parity(dtype, d):
     gg, ref = run_both(inp)
     errs = worst_errors(inp, gg, ref)
     print(dtype, d, errs)
-    assert max(errs.values()) <= GRAD_BAR, errs
+    assert max(errs.values()) <= GRAD_BAR[dtype], errs
 
 
 def test_backward_varlen_edges():
@@ -83,7 +86,7 @@ def test_backward_varlen_edges():
     gg, ref = run_both(inp)
     errs = worst_errors(inp, gg, ref)
     print(errs)
-    assert max(errs.values()) <= GRAD_BAR, errs
+    assert max(errs.values()) <= GRAD_BAR["bf16"], errs
     # the empty sequence passes its final-state gradient straight through
     assert torch.allclose(gg["d_initial_state"][4], inp["dSf"][4].to(DEV), rtol=0, atol=0)
 
@@ -93,4 +96,4 @@ def test_backward_small_dims_without_final_gradient():
     gg, ref = run_both(inp, with_dsf=False)
     errs = worst_errors(inp, gg, ref)
     print(errs)
-    assert max(errs.values()) <= GRAD_BAR, errs
+    assert max(errs.values()) <= GRAD_BAR["f32"], errs
