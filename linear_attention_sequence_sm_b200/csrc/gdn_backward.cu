@@ -148,7 +148,8 @@ __device__ __forceinline__ void tgemm(int M, int N, int K, FA a, FB b, FO out) {
     const int mt = (M + 15) / 16, nt = (N + 7) / 8;
     for (int tile = warp; tile < mt * nt; tile += kBwdThreads / 32) {
         const int m0 = (tile % mt) * 16, n0 = (tile / mt) * 8;
-        float d[4] = {0.f, 0.f, 0.f, 0.f};
+        // three independent accumulators, so the three products of a step do not wait on each other
+        float d[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f}, d2[4] = {0.f, 0.f, 0.f, 0.f};
         for (int k0 = 0; k0 < K; k0 += 16) {
             auto A = [&](int r, int c) {
                 const int m = m0 + r, kk = k0 + c;
@@ -165,10 +166,12 @@ __device__ __forceinline__ void tgemm(int M, int N, int K, FA a, FB b, FO out) {
             bwd_split2(A(g + 8, 2 * t + 8), A(g + 8, 2 * t + 9), ah[3], al[3]);
             bwd_split2(B(2 * t, g), B(2 * t + 1, g), bh[0], bl[0]);
             bwd_split2(B(2 * t + 8, g), B(2 * t + 9, g), bh[1], bl[1]);
-            bwd_mma(d, al, bh);
-            bwd_mma(d, ah, bl);
+            bwd_mma(d1, al, bh);
+            bwd_mma(d2, ah, bl);
             bwd_mma(d, ah, bh);
         }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) d[e] += d1[e] + d2[e];
         const int r0 = m0 + g, c0 = n0 + 2 * t;
         if (r0 < M && c0 < N) out(r0, c0, d[0]);
         if (r0 < M && c0 + 1 < N) out(r0, c0 + 1, d[1]);
