@@ -208,6 +208,12 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
           *vdB = vec + kVDB * kBwdC;
     __shared__ float red[kBwdThreads / 32];
     const int tid = threadIdx.x;
+    // rows x d_k loops without a division: thread t takes column t & 127 of rows (t >> 7), (t >> 7) + 2, ...
+    auto rows_dk = [&](int nrows, auto &&f) {
+        const int x = tid & 127;
+        if (x < dkd)
+            for (int r = tid >> 7; r < nrows; r += kBwdThreads / 128) f(r, x);
+    };
     const T *q = static_cast<const T *>(a.q);
     const T *k = static_cast<const T *>(a.k);
     const T *v = static_cast<const T *>(a.v);
@@ -233,12 +239,11 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
     constexpr int C = kBwdC, R = kBwdRows;
     auto chunk_inputs = [&](int c, int Lc) {
         const int c0 = t0 + c * C;
-        for (int idx = tid; idx < C * dkd; idx += kBwdThreads) {
-            const int r = idx / dkd, x = idx % dkd;
+        rows_dk(C, [&](int r, int x) {
             const bool ok = r < Lc;
             K[r * ldk + x] = ok ? to_f32(k[(size_t(c0 + r) * hk + hq) * dkd + x]) : 0.f;
             Q[r * ldk + x] = ok ? to_f32(q[(size_t(c0 + r) * hk + hq) * dkd + x]) : 0.f;
-        }
+        });
         for (int idx = tid; idx < C * R; idx += kBwdThreads) {
             const int r = idx / R, i = idx % R;
             V[r * ldv + i] = (r < Lc && i < nr) ? to_f32(v[(size_t(c0 + r) * hv + h) * dvd + i0 + i]) : 0.f;
@@ -309,10 +314,10 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
             else sm_[r * ldc + j] = base[e];
         }
         float *bw = base + 3 * C * C;
-        for (int e = tid; e < C * dkd; e += kBwdThreads) {
-            if (store) bw[e] = W[(e / dkd) * ldk + e % dkd];
-            else W[(e / dkd) * ldk + e % dkd] = bw[e];
-        }
+        rows_dk(C, [&](int r, int x) {
+            if (store) bw[r * dkd + x] = W[r * ldk + x];
+            else W[r * ldk + x] = bw[r * dkd + x];
+        });
         float *bu = bw + C * dkd;
         for (int e = tid; e < C * R; e += kBwdThreads) {
             if (store) bu[e] = U[(e / R) * ldv + e % R];
@@ -321,15 +326,14 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
     };
 
     // ---- pass 1: chunk start states into the workspace ----
-    for (int idx = tid; idx < R * dkd; idx += kBwdThreads) {
-        const int i = idx / dkd, x = idx % dkd;
+    rows_dk(R, [&](int i, int x) {
         S0[i * ldk + x] = (a.s0 && i < nr) ? a.s0[sbase + size_t(i0 + i) * dkd + x] : 0.f;
-    }
+    });
     __syncthreads();
     for (int c = 0; c < nch; ++c) {
         const int Lc = min(C, len - c * C);
         float *dst = ck(c);
-        for (int idx = tid; idx < nr * dkd; idx += kBwdThreads) dst[idx] = S0[(idx / dkd) * ldk + idx % dkd];
+        rows_dk(nr, [&](int i, int x) { dst[i * dkd + x] = S0[i * ldk + x]; });
         chunk_inputs(c, Lc);
         chunk_products();
         keep_io(kp(c), true);
@@ -342,18 +346,14 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
     }
 
     // ---- pass 2: backward over the chunks ----
-    for (int idx = tid; idx < R * dkd; idx += kBwdThreads) {
-        const int i = idx / dkd, x = idx % dkd;
+    rows_dk(R, [&](int i, int x) {
         dS[i * ldk + x] = (dSf && i < nr) ? dSf[sbase + size_t(i0 + i) * dkd + x] : 0.f;
-    }
+    });
     for (int c = nch - 1; c >= 0; --c) {
         const int Lc = min(C, len - c * C);
         const int c0 = t0 + c * C;
         const float *src = ck(c);
-        for (int idx = tid; idx < R * dkd; idx += kBwdThreads) {
-            const int i = idx / dkd, x = idx % dkd;
-            S0[i * ldk + x] = i < nr ? src[i * dkd + x] : 0.f;
-        }
+        rows_dk(R, [&](int i, int x) { S0[i * ldk + x] = i < nr ? src[i * dkd + x] : 0.f; });
         __syncthreads();
         chunk_inputs(c, Lc);
         keep_io(kp(c), false);
@@ -361,17 +361,14 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
             const int r = idx / R, i = idx % R;
             dOs[r * ldv + i] = (r < Lc && i < nr) ? to_f32(dO[(size_t(c0 + r) * hv + h) * dvd + i0 + i]) : 0.f;
         }
-        for (int idx = tid; idx < C * dkd; idx += kBwdThreads) {
-            dQ[(idx / dkd) * ldk + idx % dkd] = 0.f;
-            dK[(idx / dkd) * ldk + idx % dkd] = 0.f;
-        }
+        rows_dk(C, [&](int r, int x) {
+            dQ[r * ldk + x] = 0.f;
+            dK[r * ldk + x] = 0.f;
+        });
         if (tid < C) vdGam[tid] = vdLam[tid] = vdBG[tid] = vdB[tid] = vdG[tid] = 0.f;
         // dgamma_L = <dS, S0> over the block's rows
         float part = 0.f;
-        for (int idx = tid; idx < R * dkd; idx += kBwdThreads) {
-            const int i = idx / dkd, x = idx % dkd;
-            part = fmaf(dS[i * ldk + x], S0[i * ldk + x], part);
-        }
+        rows_dk(R, [&](int i, int x) { part = fmaf(dS[i * ldk + x], S0[i * ldk + x], part); });
 #pragma unroll
         for (int m = 16; m > 0; m >>= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
         if ((tid & 31) == 0) red[tid >> 5] = part;
@@ -501,12 +498,11 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
         }
         __syncthreads();
         // the block's share of the shared gradients
-        for (int idx = tid; idx < Lc * dkd; idx += kBwdThreads) {
-            const int r = idx / dkd, x = idx % dkd;
+        rows_dk(Lc, [&](int r, int x) {
             const size_t o = (size_t(c0 + r) * hk + hq) * dkd + x;
             atomicAdd(dq + o, dQ[r * ldk + x]);
             atomicAdd(dk + o, dK[r * ldk + x]);
-        }
+        });
         if (tid < Lc) {
             atomicAdd(dg + size_t(c0 + tid) * hv + h, vdG[tid]);
             atomicAdd(dbeta + size_t(c0 + tid) * hv + h, vdB[tid]);
@@ -514,10 +510,7 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
         __syncthreads();
     }
     if (dS0_out)
-        for (int idx = tid; idx < nr * dkd; idx += kBwdThreads) {
-            const int i = idx / dkd, x = idx % dkd;
-            dS0_out[sbase + size_t(i0 + i) * dkd + x] = dS[i * ldk + x];
-        }
+        rows_dk(nr, [&](int i, int x) { dS0_out[sbase + size_t(i0 + i) * dkd + x] = dS[i * ldk + x]; });
 }
 
 static size_t bwd_slots(int32_t tokens, int32_t num_seqs) { return size_t(tokens) / kBwdC + size_t(num_seqs) + 1; }
