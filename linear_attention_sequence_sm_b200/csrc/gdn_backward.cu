@@ -282,14 +282,24 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
         prod<kTC, 1>(C, C, dkd, [&](int r, int x) { return Q[r * ldk + x]; }, [&](int x, int j) { return K[j * ldk + x]; },
                  [&](int r, int j, float acc) { QK[r * ldc + j] = j <= r ? acc : 0.f; });
         __syncthreads();
-        // T = (I + A)^-1, A_rj = beta_r Gamma_rj KK_rj (j < r); one column per thread
+        // T = (I + A)^-1, A_rj = beta_r Gamma_rj KK_rj (j < r): A formed by the block, then one column
+        // per thread by forward substitution with the column in registers (entries above the diagonal
+        // come out as exact zeros, the diagonal as 1)
+        for (int p = tid; p < C * C; p += kBwdThreads) {
+            const int r = p / C, j = p % C;
+            sM[r * ldc + j] = j < r ? vB[r] * Gm[r * ldc + j] * KK[r * ldc + j] : 0.f;
+        }
+        __syncthreads();
         if (tid < C) {
             const int col = tid;
+            float xs[C];
+#pragma unroll
             for (int r = 0; r < C; ++r) {
-                float x = r == col ? 1.f : 0.f;
-                if (r > col)
-                    for (int j = col; j < r; ++j) x = fmaf(-vB[r] * Gm[r * ldc + j] * KK[r * ldc + j], Tm[j * ldc + col], x);
-                Tm[r * ldc + col] = r < col ? 0.f : x;
+                float acc[4] = {r == col ? 1.f : 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int j = 0; j < r; ++j) acc[j & 3] = fmaf(-sM[r * ldc + j], xs[j], acc[j & 3]);
+                xs[r] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                Tm[r * ldc + col] = xs[r];
             }
         }
         __syncthreads();
