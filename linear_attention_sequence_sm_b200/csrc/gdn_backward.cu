@@ -74,6 +74,12 @@ __host__ __device__ inline BwdSmem bwd_smem(int dk) {
 // per-token vectors inside the vec block
 enum { kVG = 0, kVGam, kVLam, kVB, kVBG, kVDG, kVDGam, kVDLam, kVDBG, kVDB, kVNum };
 
+__device__ __forceinline__ float bwd_warp_sum(float x) {
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+    return x;
+}
+
 // floats kept per (chunk, value head, row slice) for pass 2: K K^T, Q K^T, T, W, U
 __host__ __device__ inline size_t bwd_keep_floats(int dk) {
     return size_t(3) * kBwdC * kBwdC + size_t(kBwdC) * dk + size_t(kBwdC) * kBwdRows;
@@ -400,12 +406,16 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
                      dW[r * ldk + x] = y * Q[r * ldk + x];  // scratch for dgamma
                  });
         __syncthreads();
-        if (tid < C) {
-            float sl = 0.f, sg = 0.f;
-            for (int i = 0; i < R; ++i) sl += dT[tid * ldc + i];
-            for (int x = 0; x < dkd; ++x) sg += dW[tid * ldk + x];
-            vdLam[tid] = sl;
-            vdGam[tid] += sg;
+        for (int r = tid >> 5; r < C; r += kBwdThreads / 32) {  // a warp per row, lanes over the columns
+            const int l = tid & 31;
+            float sl = l < R ? dT[r * ldc + l] : 0.f, sg = 0.f;
+            for (int x = l; x < dkd; x += 32) sg += dW[r * ldk + x];
+            sl = bwd_warp_sum(sl);
+            sg = bwd_warp_sum(sg);
+            if (l == 0) {
+                vdLam[r] = sl;
+                vdGam[r] += sg;
+            }
         }
         __syncthreads();
         // dP_rj = dO_r . u_j (j <= r), kept in dT's storage
@@ -455,12 +465,16 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
                      U[j * ldv + i] = dy * V[j * ldv + i];  // scratch for dbeta (U is no longer needed)
                  });
         __syncthreads();
-        if (tid < C) {
-            float sb = 0.f, su = 0.f;
-            for (int x = 0; x < dkd; ++x) sb += Q[tid * ldk + x];
-            for (int i = 0; i < R; ++i) su += U[tid * ldv + i];
-            vdBG[tid] = sb;
-            vdB[tid] = su;
+        for (int r = tid >> 5; r < C; r += kBwdThreads / 32) {  // a warp per row, lanes over the columns
+            const int l = tid & 31;
+            float su = l < R ? U[r * ldv + l] : 0.f, sb = 0.f;
+            for (int x = l; x < dkd; x += 32) sb += Q[r * ldk + x];
+            sb = bwd_warp_sum(sb);
+            su = bwd_warp_sum(su);
+            if (l == 0) {
+                vdBG[r] = sb;
+                vdB[r] = su;
+            }
         }
         // dA = -T^T dT T^T (strictly lower): M = dT T^T first
         prod<kTC, 1>(C, C, C, [&](int r, int m) { return dT[r * ldc + m]; }, [&](int m, int j) { return Tm[j * ldc + m]; },
