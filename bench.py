@@ -437,22 +437,62 @@ def run_ours(args):
         h2d = sum(t.numel() * t.element_size() for t in pin.values())
         d2h = o_host.numel() * o_host.element_size() + sf_host.numel() * sf_host.element_size()
 
+        # Steps overlap across three streams, double-buffered: step i's inputs copy in while step i-1
+        # computes and step i-2's results copy out (separate copy engines for the two directions).
+        # Every step still copies its own inputs from pinned host memory and its own results back.
+        s_in, s_out, comp = torch.cuda.Stream(device), torch.cuda.Stream(device), stream
+        dbuf = [{k: torch.empty_like(v, device=device) for k, v in pin.items()} for _ in range(2)]
+        obuf, sbuf = [torch.empty_like(o) for _ in range(2)], [torch.empty_like(sf) for _ in range(2)]
+        ohost = [o_host] + [torch.empty(o.shape, dtype=o.dtype).pin_memory()]
+        shost = [sf_host] + [torch.empty(sf.shape, dtype=sf.dtype).pin_memory()]
+        ev_in, ev_comp, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
+        for b in range(2):
+            ev_comp[b].record(comp)
+            ev_out[b].record(comp)
+        it = [0]
+
         def e2e_step():
-            x = {k: v.to(device, non_blocking=True) for k, v in pin.items()}
-            oo, ss = fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], initial_state=x.get("initial_state"),
-                                       cu_seqlens=x.get("cu_seqlens"), chunk_size=w.chunk, workspace=ws, **flags,
-                                       **out_norm(x))
-            o_host.copy_(oo, non_blocking=True)
-            sf_host.copy_(ss, non_blocking=True)
+            b = it[0] % 2
+            it[0] += 1
+            x = dbuf[b]
+            s_in.wait_event(ev_comp[b])  # the step that last read these input buffers has run
+            with torch.cuda.stream(s_in):
+                for k_ in x:
+                    x[k_].copy_(pin[k_], non_blocking=True)
+            ev_in[b].record(s_in)
+            comp.wait_event(ev_in[b])
+            comp.wait_event(ev_out[b])  # the results last held in these output buffers have left
+            with torch.cuda.stream(comp):
+                fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], initial_state=x.get("initial_state"),
+                    cu_seqlens=x.get("cu_seqlens"), chunk_size=w.chunk, out=obuf[b], final_state=sbuf[b],
+                    workspace=ws, **flags, **out_norm(x))
+            ev_comp[b].record(comp)
+            s_out.wait_event(ev_comp[b])
+            with torch.cuda.stream(s_out):
+                ohost[b].copy_(obuf[b], non_blocking=True)
+                shost[b].copy_(sbuf[b], non_blocking=True)
+            ev_out[b].record(s_out)
+
+        def e2e_timed(n):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(comp)
+            s_in.wait_stream(comp)
+            for _ in range(n):
+                e2e_step()
+            comp.wait_stream(s_out)
+            e1.record(comp)
+            e1.synchronize()
+            return e0.elapsed_time(e1) / n
 
         for _ in range(2):
             e2e_step()
         torch.cuda.synchronize(device)
         barrier(world, device)
-        e_ms = timed(e2e_step, max(3, min(args.steps, 20)), stream)
+        e_ms = e2e_timed(max(3, min(args.steps, 20)))
         e_ms = max_over_ranks(e_ms, device, world)
         e2e = {"value": world * tokens / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
+               "overlap": "copy-in, compute and copy-out of consecutive steps on three streams, double-buffered"}
 
     cpu = None
     # (raw inputs or the output side: the timed oracle covers the plain path only; no CPU line then)
