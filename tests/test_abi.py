@@ -199,3 +199,33 @@ def test_decode_multi_and_commit_argument_checks(gdn):
     assert c(4, 3, 4, 128, 128, vp(FAKE + 8), vp(FAKE), vp(FAKE), None, None) == gdn.GDN_ERR_MISALIGNED
     assert c(4, 3, 4, 3, 3, vp(FAKE), vp(FAKE), vp(FAKE), None, None) == gdn.GDN_ERR_UNSUPPORTED
     assert c(0, 3, 4, 128, 128, None, None, None, None, None) == gdn.GDN_OK
+
+
+def test_backward_and_kda_argument_checks(gdn):
+    """Refused before any device work: input-side flags on the backward,
+    NULL gradient outputs, a short workspace, misalignment; KDA with d_k > 128."""
+    vp = ctypes.c_void_p
+    s = _shape(gdn, chunk_size=32)
+    n = ctypes.c_size_t(0)
+    assert gdn.LIB.gdn_chunk_backward_workspace_size(ctypes.byref(s), ctypes.byref(n)) == gdn.GDN_OK
+    assert n.value > gdn.workspace_size(s)  # the chunk checkpoints come on top of the schedule
+
+    def bwd(shape, **over):
+        p = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, s0=None, cu=None, do=FAKE, dsf=None, dq=FAKE, dk=FAKE,
+                 dv=FAKE, dg=FAKE, db=FAKE, ds0=None, ws=FAKE, wsb=n.value)
+        p.update(over)
+        return gdn.LIB.gdn_chunk_backward(ctypes.byref(shape), *(vp(p[k]) for k in (
+            "q", "k", "v", "g", "beta", "s0", "cu", "do", "dsf", "dq", "dk", "dv", "dg", "db", "ds0", "ws")),
+            p["wsb"], None)
+
+    assert bwd(_shape(gdn, chunk_size=32, flags=2)) == gdn.GDN_ERR_UNSUPPORTED
+    assert bwd(s, dq=None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert bwd(s, wsb=1024) == gdn.GDN_ERR_WORKSPACE_TOO_SMALL
+    assert bwd(s, dv=FAKE + 4) == gdn.GDN_ERR_MISALIGNED
+    assert bwd(_shape(gdn, chunk_size=32, head_dim_k=256)) == gdn.GDN_ERR_UNSUPPORTED
+    ks = _shape(gdn, head_dim_k=160)
+    st = gdn.LIB.gdn_kda_forward(ctypes.byref(ks), *([vp(FAKE)] * 5), None, None, None, vp(FAKE), None, vp(FAKE),
+                                 1 << 20, None)
+    assert st == gdn.GDN_ERR_UNSUPPORTED
+    st = gdn.LIB.gdn_kda_decode_step(4, 2, 4, 512, 128, 1, *([vp(FAKE)] * 6), None, vp(FAKE), 0, None)
+    assert st == gdn.GDN_ERR_UNSUPPORTED
