@@ -339,6 +339,8 @@ def run_ours(args):
                 "traffic": kernel_traffic(f"{kernel_name}/{w.name}{suffix}"),
                 "kernel": kernel_name,
                 "peak_source": f"{peak_src} bf16 dense (burst)",
+                "frac_vs_sustained": achieved_tflops / peaks["bf16_tflops_sustained"],
+                "frac_vs_nominal_2250": achieved_tflops / 2250.0,
                 "flops_per_launch": flops, "algorithmic_bytes_per_launch": prefill_bytes(w)}
     if args.backward:
         # reverse mode of the token recurrence: 20 d^2 flops per (token, value head) (the forward
@@ -424,7 +426,7 @@ def run_ours(args):
                                "traffic": kernel_traffic(f"gdn_decode/{dw.name}" + ("_kda" if args.kda else "")
                                                          + (f"_mtp{args.mtp}" if args.mtp > 0 else "")),
                                "kernel": "gdn_decode", "peak_source": f"{peak_src} HBM copy",
-                               "bytes_per_launch": dbytes},
+                               "frac_vs_nominal_8000": dgbs / 8000.0, "bytes_per_launch": dbytes},
                   "clocks": dclocks.summary(), "cuda_graph": not args.no_graph}
         del state
 
