@@ -229,3 +229,19 @@ def test_backward_and_kda_argument_checks(gdn):
     assert st == gdn.GDN_ERR_UNSUPPORTED
     st = gdn.LIB.gdn_kda_decode_step(4, 2, 4, 512, 128, 1, *([vp(FAKE)] * 6), None, vp(FAKE), 0, None)
     assert st == gdn.GDN_ERR_UNSUPPORTED
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/gdn.h compiles as pedantic C99 (plain pointers and sizes, no
+    C++ or torch types in the ABI)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use.c"
+    src.write_text('#include "gdn.h"\nint main(void) { gdn_output_side_t o = {0}; (void)o; '
+                   'return (int)sizeof(gdn_shape_t); }\n')
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only",
+                        "-I", os.path.join(ROOT, "include"), str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
