@@ -241,31 +241,57 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
     const size_t keep_sz = bwd_keep_floats(dkd);
     auto kp = [&](int c) { return keep + ((bwd_slot(t0, seq, c) * hv + h) * n_slices + slice) * keep_sz; };
 
-    // one chunk's inputs, prefix sums, per-token decays and Gamma
+    // one chunk's inputs, prefix sums, per-token decays and Gamma.  Every
+    // thread issues all of its global loads before its first shared-memory
+    // store, so a group of loads costs about one memory latency, not one per row.
     constexpr int C = kBwdC, R = kBwdRows;
+    static_assert(C == 32 && kBwdThreads % 128 == 0, "one warp spans a chunk; d_k columns map to 128 threads");
+    constexpr int kRowStep = kBwdThreads / 128;     // rows apart of one thread's d_k-wide elements
+    constexpr int kRowsPer = C / kRowStep;          // C x d_k elements per thread
+    constexpr int kVPer = C * R / kBwdThreads;      // C x R elements per thread
+    const int colx = tid & 127, row0 = tid >> 7;
     auto chunk_inputs = [&](int c, int Lc) {
         const int c0 = t0 + c * C;
-        rows_dk(C, [&](int r, int x) {
-            const bool ok = r < Lc;
-            K[r * ldk + x] = ok ? to_f32(k[(size_t(c0 + r) * hk + hq) * dkd + x]) : 0.f;
-            Q[r * ldk + x] = ok ? to_f32(q[(size_t(c0 + r) * hk + hq) * dkd + x]) : 0.f;
-        });
-        for (int idx = tid; idx < C * R; idx += kBwdThreads) {
-            const int r = idx / R, i = idx % R;
-            V[r * ldv + i] = (r < Lc && i < nr) ? to_f32(v[(size_t(c0 + r) * hv + h) * dvd + i0 + i]) : 0.f;
+        float kr[kRowsPer], qr[kRowsPer], vr[kVPer], gr = 0.f, br = 0.f;
+#pragma unroll
+        for (int e = 0; e < kRowsPer; ++e) {
+            const int r = row0 + e * kRowStep;
+            const bool ok = r < Lc && colx < dkd;
+            const size_t o = (size_t(c0 + r) * hk + hq) * dkd + colx;
+            kr[e] = ok ? to_f32(k[o]) : 0.f;
+            qr[e] = ok ? to_f32(q[o]) : 0.f;
         }
-        if (tid < C) {
+#pragma unroll
+        for (int e = 0; e < kVPer; ++e) {
+            const int idx = tid + e * kBwdThreads, r = idx / R, i = idx % R;
+            vr[e] = (r < Lc && i < nr) ? to_f32(v[(size_t(c0 + r) * hv + h) * dvd + i0 + i]) : 0.f;
+        }
+        if (tid < Lc) {
             const size_t gb = size_t(c0 + tid) * hv + h;
-            vG[tid] = tid < Lc ? fmaxf(a.g[gb], kGFloor) : 0.f;
-            vB[tid] = tid < Lc ? a.beta[gb] : 0.f;
+            gr = fmaxf(a.g[gb], kGFloor);
+            br = a.beta[gb];
         }
-        __syncthreads();
-        if (tid == 0) {
-            float run = 0.f;
-            for (int r = 0; r < C; ++r) {
-                run += vG[r];
-                vG[r] = run;
+        if (colx < dkd)
+#pragma unroll
+            for (int e = 0; e < kRowsPer; ++e) {
+                const int r = row0 + e * kRowStep;
+                K[r * ldk + colx] = kr[e];
+                Q[r * ldk + colx] = qr[e];
             }
+#pragma unroll
+        for (int e = 0; e < kVPer; ++e) {
+            const int idx = tid + e * kBwdThreads;
+            V[(idx / R) * ldv + idx % R] = vr[e];
+        }
+        if (tid < C) {  // the first warp: inclusive prefix sums G of the clamped gates
+            const int l = tid;
+#pragma unroll
+            for (int m = 1; m < 32; m <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, gr, m);
+                if (l >= m) gr += y;
+            }
+            vG[l] = gr;
+            vB[l] = br;
         }
         __syncthreads();
         if (tid < C) {
@@ -321,30 +347,67 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
         __syncthreads();
     };
 
-    // K K^T, Q K^T, T (C x C each), W (C x d_k), U (C x 32) to / from the workspace
-    auto keep_io = [&](float *base, bool store) {
+    // K K^T, Q K^T, T (C x C each), W (C x d_k), U (C x 32) to the workspace
+    auto keep_store = [&](float *base) {
         for (int e = tid; e < 3 * C * C; e += kBwdThreads) {
             const int m = e / (C * C), r = (e / C) % C, j = e % C;
-            float *sm_ = m == 0 ? KK : (m == 1 ? QK : Tm);
-            if (store) base[e] = sm_[r * ldc + j];
-            else sm_[r * ldc + j] = base[e];
+            base[e] = (m == 0 ? KK : (m == 1 ? QK : Tm))[r * ldc + j];
         }
         float *bw = base + 3 * C * C;
-        rows_dk(C, [&](int r, int x) {
-            if (store) bw[r * dkd + x] = W[r * ldk + x];
-            else W[r * ldk + x] = bw[r * dkd + x];
-        });
+        rows_dk(C, [&](int r, int x) { bw[r * dkd + x] = W[r * ldk + x]; });
         float *bu = bw + C * dkd;
-        for (int e = tid; e < C * R; e += kBwdThreads) {
-            if (store) bu[e] = U[(e / R) * ldv + e % R];
-            else U[(e / R) * ldv + e % R] = bu[e];
+        for (int e = tid; e < C * R; e += kBwdThreads) bu[e] = U[(e / R) * ldv + e % R];
+    };
+    // and back, with the chunk's dO rows in the same group of loads
+    static_assert((C * C) % kBwdThreads == 0, "a thread's C x C elements stay in one matrix per step");
+    auto keep_load = [&](const float *base, int c0, int Lc) {
+        constexpr int kCC = 3 * C * C / kBwdThreads;
+        float cc[kCC], wr[kRowsPer], ur[kVPer], orow[kVPer];
+        const float *bw = base + 3 * C * C, *bu = bw + C * dkd;
+#pragma unroll
+        for (int e = 0; e < kCC; ++e) cc[e] = base[tid + e * kBwdThreads];
+#pragma unroll
+        for (int e = 0; e < kRowsPer; ++e)
+            wr[e] = colx < dkd ? bw[size_t(row0 + e * kRowStep) * dkd + colx] : 0.f;
+#pragma unroll
+        for (int e = 0; e < kVPer; ++e) {
+            const int idx = tid + e * kBwdThreads, r = idx / R, i = idx % R;
+            ur[e] = bu[idx];
+            orow[e] = (r < Lc && i < nr) ? to_f32(dO[(size_t(c0 + r) * hv + h) * dvd + i0 + i]) : 0.f;
         }
+#pragma unroll
+        for (int e = 0; e < kCC; ++e) {
+            const int idx = tid + e * kBwdThreads, r = (idx / C) % C, j = idx % C;
+            constexpr int kPerMat = C * C / kBwdThreads;
+            float *mat = e / kPerMat == 0 ? KK : (e / kPerMat == 1 ? QK : Tm);
+            mat[r * ldc + j] = cc[e];
+        }
+        if (colx < dkd)
+#pragma unroll
+            for (int e = 0; e < kRowsPer; ++e) W[(row0 + e * kRowStep) * ldk + colx] = wr[e];
+#pragma unroll
+        for (int e = 0; e < kVPer; ++e) {
+            const int idx = tid + e * kBwdThreads, r = idx / R, i = idx % R;
+            U[r * ldv + i] = ur[e];
+            dOs[r * ldv + i] = orow[e];
+        }
+    };
+    // R rows of d_k floats (row stride d_k; rows >= nvalid, or all rows for a null source, are zeros)
+    static_assert(kBwdRows == kBwdC, "state row slices use the chunk's row mapping");
+    auto load_rows = [&](float *dst, const float *src, int nvalid) {
+        float t[kRowsPer];
+#pragma unroll
+        for (int e = 0; e < kRowsPer; ++e) {
+            const int r = row0 + e * kRowStep;
+            t[e] = (src && r < nvalid && colx < dkd) ? src[size_t(r) * dkd + colx] : 0.f;
+        }
+        if (colx < dkd)
+#pragma unroll
+            for (int e = 0; e < kRowsPer; ++e) dst[(row0 + e * kRowStep) * ldk + colx] = t[e];
     };
 
     // ---- pass 1: chunk start states into the workspace ----
-    rows_dk(R, [&](int i, int x) {
-        S0[i * ldk + x] = (a.s0 && i < nr) ? a.s0[sbase + size_t(i0 + i) * dkd + x] : 0.f;
-    });
+    load_rows(S0, a.s0 ? a.s0 + sbase + size_t(i0) * dkd : nullptr, nr);
     __syncthreads();
     for (int c = 0; c < nch; ++c) {
         const int Lc = min(C, len - c * C);
@@ -352,7 +415,7 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
         rows_dk(nr, [&](int i, int x) { dst[i * dkd + x] = S0[i * ldk + x]; });
         chunk_inputs(c, Lc);
         chunk_products();
-        keep_io(kp(c), true);
+        keep_store(kp(c));
         const float gl = __expf(vG[Lc - 1]);
         // S <- gamma_L S + U^T diag(lambda) K
         prod<kTC, 4>(R, dkd, Lc, [&](int i, int j) { return U[j * ldv + i] * vLam[j]; },
@@ -362,21 +425,13 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
     }
 
     // ---- pass 2: backward over the chunks ----
-    rows_dk(R, [&](int i, int x) {
-        dS[i * ldk + x] = (dSf && i < nr) ? dSf[sbase + size_t(i0 + i) * dkd + x] : 0.f;
-    });
+    load_rows(dS, dSf ? dSf + sbase + size_t(i0) * dkd : nullptr, nr);
     for (int c = nch - 1; c >= 0; --c) {
         const int Lc = min(C, len - c * C);
         const int c0 = t0 + c * C;
-        const float *src = ck(c);
-        rows_dk(R, [&](int i, int x) { S0[i * ldk + x] = i < nr ? src[i * dkd + x] : 0.f; });
-        __syncthreads();
+        load_rows(S0, ck(c), nr);
         chunk_inputs(c, Lc);
-        keep_io(kp(c), false);
-        for (int idx = tid; idx < C * R; idx += kBwdThreads) {
-            const int r = idx / R, i = idx % R;
-            dOs[r * ldv + i] = (r < Lc && i < nr) ? to_f32(dO[(size_t(c0 + r) * hv + h) * dvd + i0 + i]) : 0.f;
-        }
+        keep_load(kp(c), c0, Lc);
         rows_dk(C, [&](int r, int x) {
             dQ[r * ldk + x] = 0.f;
             dK[r * ldk + x] = 0.f;
@@ -499,7 +554,9 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
         prod<kTC, 4>(C, dkd, C, [&](int r, int j) { return j < r ? dT[r * ldc + j] : (j > r ? dT[j * ldc + r] : 0.f); },
                  [&](int j, int x) { return K[j * ldk + x]; }, [&](int r, int x, float acc) { dK[r * ldk + x] += acc; });
         __syncthreads();
-        // decays: beta gamma, gamma, lambda, gamma_L and Gamma through G, then dg = reverse prefix sums
+        // decays: beta gamma, gamma, lambda, gamma_L and Gamma through G, then dg = reverse prefix
+        // sums of dG (the first warp, a lane per token; gamma_L = e^(G_L) and every lambda_j =
+        // e^(G_L - G_j) also reach G_L, the last token's)
         if (tid < C) {
             const int r = tid;
             vdB[r] = fmaf(vdBG[r], vGam[r], vdB[r]);
@@ -507,18 +564,14 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
             float dG = dgam * vGam[r] - vdLam[r] * vLam[r];
             for (int j = 0; j <= r; ++j) dG = fmaf(dA[r * ldc + j], Gm[r * ldc + j], dG);
             for (int i = r; i < C; ++i) dG = fmaf(-dA[i * ldc + r], Gm[i * ldc + r], dG);
-            vdG[r] = dG;
-        }
-        __syncthreads();
-        if (tid == 0) {
-            float extra = dgl * gL;
-            for (int j = 0; j < Lc; ++j) extra = fmaf(vdLam[j], vLam[j], extra);
-            vdG[Lc - 1] += extra;
-            float run = 0.f;
-            for (int t = Lc - 1; t >= 0; --t) {
-                run += vdG[t];
-                vdG[t] = run;
+            const float extra = dgl * gL + bwd_warp_sum(r < Lc ? vdLam[r] * vLam[r] : 0.f);
+            float run = r < Lc ? dG + (r == Lc - 1 ? extra : 0.f) : 0.f;
+#pragma unroll
+            for (int m = 1; m < 32; m <<= 1) {
+                const float y = __shfl_down_sync(0xffffffffu, run, m);
+                if (r + m < 32) run += y;
             }
+            vdG[r] = run;
         }
         __syncthreads();
         // the block's share of the shared gradients
