@@ -39,11 +39,17 @@ struct BwdSmem {
     size_t k, q, w, dw, dq, dk, s0, ds, v, u, du, dO, t, gm, kk, qk, dt, da, sm, se, vec, total;
 };
 
-__host__ __device__ inline BwdSmem bwd_smem(int dk) {
+// Row strides (floats) of the shared arrays.  The CUDA-core tiles (tc = false)
+// read a row per lane, so an odd stride puts the 32 lanes in 32 banks.  The
+// tensor-core tiles read fragment element (g, 2t) of lane 4g + t, as row g or
+// as column g: a stride of 4 mod 8 maps the column form to bank 8t + g (all
+// distinct) and the row form to at most 2 lanes a bank, where an odd stride
+// gives g + 2t (up to 4 a bank) in both.
+__host__ __device__ inline BwdSmem bwd_smem(int dk, bool tc) {
     BwdSmem s;
-    s.ldk = dk + 1;
-    s.ldc = kBwdC + 1;
-    s.ldv = kBwdRows + 1;
+    s.ldk = tc ? dk + (12 - dk % 8) % 8 : dk + 1;
+    s.ldc = kBwdC + (tc ? 4 : 1);
+    s.ldv = kBwdRows + (tc ? 4 : 1);
     size_t off = 0;
     auto take = [&](size_t n) { size_t o = off; off += n; return o; };
     s.k = take(size_t(kBwdC) * s.ldk);
@@ -201,7 +207,7 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
     extern __shared__ float smem[];
     constexpr bool kTC = std::is_same<T, __nv_bfloat16>::value;
     const int dkd = a.dk, dvd = a.dv, hv = a.hv, hk = a.hk;
-    const BwdSmem L = bwd_smem(dkd);
+    const BwdSmem L = bwd_smem(dkd, kTC);
     const int ldk = L.ldk, ldc = L.ldc, ldv = L.ldv;
     float *K = smem + L.k, *Q = smem + L.q, *W = smem + L.w, *dW = smem + L.dw, *dQ = smem + L.dq,
           *dK = smem + L.dk, *S0 = smem + L.s0, *dS = smem + L.ds, *V = smem + L.v, *U = smem + L.u,
@@ -606,7 +612,7 @@ cudaError_t launch_chunk_backward(const PrefillArgs &a, const void *dO, const fl
     const int64_t blocks = int64_t(a.num_seqs) * a.hv * n_slices;
     if (blocks <= 0) return cudaSuccess;
     if (blocks > INT32_MAX || a.dk > 128 || a.dv > 128) return cudaErrorInvalidValue;
-    const size_t bytes = bwd_smem(a.dk).total * sizeof(float);
+    const size_t bytes = bwd_smem(a.dk, a.dtype == GDN_DTYPE_BF16).total * sizeof(float);
     const size_t slots = bwd_slots(a.tokens, a.num_seqs);
     float *keep = ckpt + (slots * size_t(a.hv) * size_t(a.dv) * size_t(a.dk) * sizeof(float) + 255) / 256 * 256 /
                              sizeof(float);
