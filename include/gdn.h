@@ -339,8 +339,10 @@ GDN_API gdn_status_t gdn_decode_commit(int32_t num_seqs, int32_t num_tokens, int
  *                      kernels' floor on g)
  *   d_initial_state    [N, Hv, d_v, d_k] fp32, or NULL
  * Inputs are those of gdn_chunk_forward (the plain path: no input-side
- * flags, GDN_ERR_UNSUPPORTED otherwise); d_o has the dtype of v.  fp32 on
- * CUDA cores: a forward pass keeps each 32-token chunk's start state and
+ * flags, GDN_ERR_UNSUPPORTED otherwise); d_o has the dtype of v.  fp32
+ * arithmetic; for bf16 inputs the products run as tensor-core tiles with
+ * each fp32 operand split into two bf16 parts and fp32 accumulation, for
+ * fp32 inputs as CUDA-core tiles.  A forward pass keeps each 32-token chunk's start state and
  * its intra-chunk products in the workspace (about 3 d_v d_k fp32 values
  * per chunk and value head, plus the schedule; gdn_chunk_backward_
  * workspace_size), then the chunks are walked backward.  dq, dk, dg and dbeta are accumulated with atomic adds

@@ -1,5 +1,6 @@
 // gdn_backward.cu -- gradients of the chunked gated delta rule (training),
-// fp32 on CUDA cores.
+// fp32 arithmetic: products as split-bf16 tensor-core tiles for bf16 inputs,
+// as CUDA-core tiles for fp32 inputs.
 //
 // The pages present the chunked form as the way to train the layer
 // ("Architecture Thread I", the Gated DeltaNet section; "Gated Attention

@@ -148,6 +148,51 @@ def _need(t, name, dtype=None, device=None):
         raise ValueError(f"{name} is on {t.device}, expected {device}")
 
 
+def _expect(t, name, shape):
+    """``t`` (if given) must have exactly ``shape``: the library takes bare
+    pointers and derives every extent from q and v, so a tensor of another
+    shape would be read or written out of bounds on the device."""
+    if t is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _prefill_shapes(q, k, v, g, beta, initial_state, cu_seqlens, kda=False):
+    """Shape checks of the prefill and backward inputs (before any device
+    check, so they hold for tensors anywhere).  Returns (N, Hv, d_v, d_k)."""
+    if cu_seqlens is not None:
+        if q.dim() not in (3, 4) or (q.dim() == 4 and q.shape[0] != 1):
+            raise ValueError(f"with cu_seqlens q must be [T, Hk, d_k] or [1, T, Hk, d_k], got {tuple(q.shape)}")
+        if cu_seqlens.dim() != 1 or cu_seqlens.shape[0] < 1:
+            raise ValueError(f"cu_seqlens must be [N + 1], got {tuple(cu_seqlens.shape)}")
+        n_seqs = cu_seqlens.shape[0] - 1
+    else:
+        if q.dim() != 4:
+            raise ValueError(f"batched q must be [B, T, Hk, d_k], got {tuple(q.shape)}")
+        n_seqs = q.shape[0]
+    _expect(k, "k", q.shape)
+    if v.dim() != q.dim() or tuple(v.shape[:-2]) != tuple(q.shape[:-2]):
+        raise ValueError(f"v must be [{', '.join(map(str, q.shape[:-2]))}, Hv, d_v], got {tuple(v.shape)}")
+    hv, dv, dk = v.shape[-2], v.shape[-1], q.shape[-1]
+    _expect(g, "g", tuple(v.shape[:-1]) + ((dk,) if kda else ()))
+    _expect(beta, "beta", v.shape[:-1])
+    _expect(initial_state, "initial_state", (n_seqs, hv, dv, dk))
+    return n_seqs, hv, dv, dk
+
+
+def _decode_shapes(q, k, v, g, beta, state, kda=False):
+    """Shape checks of one decode step: q, k [N, Hk, d_k], v [N, Hv, d_v],
+    g [N, Hv] ([N, Hv, d_k] for KDA), beta [N, Hv], state [N, Hv, d_v, d_k]."""
+    if q.dim() != 3:
+        raise ValueError(f"decode q must be [N, Hk, d_k], got {tuple(q.shape)}")
+    _expect(k, "k", q.shape)
+    if v.dim() != 3 or v.shape[0] != q.shape[0]:
+        raise ValueError(f"decode v must be [{q.shape[0]}, Hv, d_v], got {tuple(v.shape)}")
+    n, hv, dv, dk = q.shape[0], v.shape[1], v.shape[2], q.shape[2]
+    _expect(g, "g", (n, hv, dk) if kda else (n, hv))
+    _expect(beta, "beta", (n, hv))
+    _expect(state, "state", (n, hv, dv, dk))
+
+
 def input_flags(qk_l2norm=False, gate_logits=False) -> int:
     """GDN_FLAG_QK_L2NORM / GDN_FLAG_GATE_LOGITS bits: raw q and k normalised
     per head inside the kernels; g and beta given as logits."""
@@ -216,6 +261,9 @@ def chunk_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_s
     and normalised per head in the kernel; ``gate_logits``: g and beta are
     the decay and write logits (alpha = sigmoid(g), beta = sigmoid(beta));
     ``output_norm``: the output side applied before o is stored."""
+    n_seqs, hv, dv, dk = _prefill_shapes(q, k, v, g, beta, initial_state, cu_seqlens)
+    _expect(out, "out", v.shape)
+    _expect(final_state, "final_state", (n_seqs, hv, dv, dk))
     dev = q.device
     dt = q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -224,8 +272,6 @@ def chunk_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_s
     _need(beta, "beta", torch.float32, dev)
     _need(initial_state, "initial_state", torch.float32, dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
-    if k.shape != q.shape:
-        raise ValueError("k must have the shape of q")
     shape = make_shape(q, v, cu_seqlens, chunk_size, force_simt, input_flags(qk_l2norm, gate_logits))
     if out is None:
         out = torch.empty(v.shape, dtype=dt, device=dev)
@@ -258,6 +304,9 @@ def chunk_forward_noalloc(q, k, v, g, beta, initial_state=None, cu_seqlens=None,
     16,384 sequences; calls that overlap on the GPU race on that array).
     Output tensors are still the caller's (allocated here only when not
     given)."""
+    n_seqs, hv, dv, dk = _prefill_shapes(q, k, v, g, beta, initial_state, cu_seqlens)
+    _expect(out, "out", v.shape)
+    _expect(final_state, "final_state", (n_seqs, hv, dv, dk))
     dev = q.device
     dt = q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -293,6 +342,8 @@ def decode_step(q, k, v, g, beta, state, out=None, stream=None, qk_l2norm=False,
     """One token per sequence; ``state`` [N, Hv, d_v, d_k] fp32 is updated in
     place.  Returns o [N, Hv, d_v].  ``qk_l2norm``, ``gate_logits`` and
     ``output_norm`` (gate [N, Hv, d_v]) as for chunk_forward."""
+    _decode_shapes(q, k, v, g, beta, state)
+    _expect(out, "out", v.shape)
     dev, dt = q.device, q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, dt, dev)
@@ -323,6 +374,9 @@ def kda_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, output_fi
     [..., Hv, d_k] fp32.  Returns (o, final_state or None).  Other arguments
     as for chunk_forward; ``chunk_size`` is validated but unused (the kernel
     walks the tokens in order)."""
+    n_seqs, hv, dv, dk = _prefill_shapes(q, k, v, g, beta, initial_state, cu_seqlens, kda=True)
+    _expect(out, "out", v.shape)
+    _expect(final_state, "final_state", (n_seqs, hv, dv, dk))
     dev = q.device
     dt = q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -331,10 +385,6 @@ def kda_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, output_fi
     _need(beta, "beta", torch.float32, dev)
     _need(initial_state, "initial_state", torch.float32, dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
-    if k.shape != q.shape:
-        raise ValueError("k must have the shape of q")
-    if tuple(g.shape) != tuple(v.shape[:-1]) + (q.shape[-1],):
-        raise ValueError(f"KDA g must be [..., Hv, d_k] = {tuple(v.shape[:-1]) + (q.shape[-1],)}, got {tuple(g.shape)}")
     shape = make_shape(q, v, cu_seqlens, chunk_size, False, input_flags(qk_l2norm, gate_logits))
     if out is None:
         out = torch.empty(v.shape, dtype=dt, device=dev)
@@ -358,6 +408,8 @@ def kda_decode_step(q, k, v, g, beta, state, out=None, stream=None, qk_l2norm=Fa
                     output_norm: OutputNorm | None = None):
     """One Kimi Delta Attention token per sequence: g [N, Hv, d_k] fp32;
     ``state`` [N, Hv, d_v, d_k] fp32 updated in place.  Returns o [N, Hv, d_v]."""
+    _decode_shapes(q, k, v, g, beta, state, kda=True)
+    _expect(out, "out", v.shape)
     dev, dt = q.device, q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, dt, dev)
@@ -366,8 +418,6 @@ def kda_decode_step(q, k, v, g, beta, state, out=None, stream=None, qk_l2norm=Fa
     _need(state, "state", torch.float32, dev)
     N, hk, dk = q.shape
     hv, dv = v.shape[1], v.shape[2]
-    if tuple(g.shape) != (N, hv, dk):
-        raise ValueError(f"KDA g must be [{N}, {hv}, {dk}], got {tuple(g.shape)}")
     if out is None:
         out = torch.empty(v.shape, dtype=dt, device=dev)
     _need(out, "out", dt, dev)
@@ -384,6 +434,17 @@ def decode_multi(q, k, v, g, beta, state, out=None, snapshots=None, stream=None,
     [N, K, Hk, 128], v [N, K, Hv, d_v], g, beta [N, K, Hv]; ``state``
     [N, Hv, d_v, 128] fp32 is only read.  Returns (o [N, K, Hv, d_v],
     snapshots [N, K, Hv, d_v, 128] fp32: the state after each token)."""
+    if q.dim() != 4:
+        raise ValueError(f"multi-token decode q must be [N, K, Hk, d_k], got {tuple(q.shape)}")
+    _expect(k, "k", q.shape)
+    if v.dim() != 4 or tuple(v.shape[:2]) != tuple(q.shape[:2]):
+        raise ValueError(f"v must be [{q.shape[0]}, {q.shape[1]}, Hv, d_v], got {tuple(v.shape)}")
+    n_, k_, hv_, dv_, dk_ = q.shape[0], q.shape[1], v.shape[2], v.shape[3], q.shape[3]
+    _expect(g, "g", (n_, k_, hv_))
+    _expect(beta, "beta", (n_, k_, hv_))
+    _expect(state, "state", (n_, hv_, dv_, dk_))
+    _expect(out, "out", v.shape)
+    _expect(snapshots, "snapshots", (n_, k_, hv_, dv_, dk_))
     dev, dt = q.device, q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, dt, dev)
@@ -407,6 +468,13 @@ def decode_multi(q, k, v, g, beta, state, out=None, snapshots=None, stream=None,
 def decode_commit(snapshots, accepted, state, bad_count=None, stream=None):
     """state[n] <- snapshots[n, accepted[n] - 1] for accepted[n] in 1..K
     (0 keeps state[n]); ``accepted`` int32 [N] on the device."""
+    if snapshots.dim() != 5:
+        raise ValueError(f"snapshots must be [N, K, Hv, d_v, d_k], got {tuple(snapshots.shape)}")
+    n_, _, hv_, dv_, dk_ = snapshots.shape
+    _expect(accepted, "accepted", (n_,))
+    _expect(state, "state", (n_, hv_, dv_, dk_))
+    if bad_count is not None and bad_count.numel() < 1:
+        raise ValueError("bad_count must hold at least one int32")
     dev = state.device
     _need(snapshots, "snapshots", torch.float32, dev)
     _need(accepted, "accepted", torch.int32, dev)
@@ -423,6 +491,9 @@ def chunk_backward(q, k, v, g, beta, d_o, d_final_state=None, initial_state=None
     """Gradients of sum d_o . o + sum d_final_state . S_final (training).
     Returns a dict of fp32 tensors: dq, dk (shaped like q), dv (like v),
     dg, dbeta (like g), d_initial_state ([N, Hv, d_v, d_k], or None)."""
+    n_seqs, hv, dv, dk = _prefill_shapes(q, k, v, g, beta, initial_state, cu_seqlens)
+    _expect(d_o, "d_o", v.shape)
+    _expect(d_final_state, "d_final_state", (n_seqs, hv, dv, dk))
     dev, dt = q.device, q.dtype
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (d_o, "d_o")):
         _need(t, n, dt, dev)
