@@ -88,6 +88,16 @@ MUTANTS = [
      "dA[r * L + j] = -acc;", "dA[r * L + j] = acc;"),
     ("backward chunked: end-state decay gradient dropped",
      "dG[L - 1] += dgL * gL;", "dG[L - 1] += 0.0 * dgL;"),
+    ("recurrence stops one token early",
+     "for (int64_t t = p->cu_seqlens[n]; t < p->cu_seqlens[n + 1]; ++t) {",
+     "for (int64_t t = p->cu_seqlens[n]; t < p->cu_seqlens[n + 1] - 1; ++t) {"),
+    ("every sequence starts from the first sequence's state",
+     "if (p->s0) memcpy(S, p->s0 + unit * (int64_t)dv * dk,", "if (p->s0) memcpy(S, p->s0 + (int64_t)h * dv * dk,"),
+    ("chunk grid on the packed token index, not the sequence start",
+     "for (int64_t c0 = t_begin; c0 < t_end; c0 += C, ++chunk_idx) {",
+     "for (int64_t c0 = t_begin - t_begin % C; c0 < t_end; c0 += C, ++chunk_idx) {"),
+    ("backward: reverse walk stops before the first token",
+     "for (int64_t t = T - 1; t >= 0; --t) {", "for (int64_t t = T - 1; t >= 1; --t) {"),
     ("A built with Gamma transposed",
      "a = p->beta[(c0 + r) * p->hv + h] * exp(G[r] - G[j]) * kk;",
      "a = p->beta[(c0 + r) * p->hv + h] * exp(G[j] - G[r]) * kk;"),
@@ -140,6 +150,7 @@ def _pin_calls(m):
         lambda: pins.test_chunkwise_equals_recurrent(m, 4, True),
         lambda: pins.test_chunkwise_equals_recurrent(m, 16, False),
         lambda: pins.test_continuation(m, 13),
+        lambda: pins.test_varlen_equals_per_sequence(m),
         lambda: pins.test_prepare_closed_forms(m),
         lambda: pins.test_prepared_one_token_closed_form(m),
         lambda: pins.test_output_side_handworked(m),
