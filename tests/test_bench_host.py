@@ -61,6 +61,29 @@ def test_reference_arm_exits_quietly_on_other_ranks():
     assert r.returncode == 0 and r.stdout.strip() == ""
 
 
+def test_reference_arm_line():
+    """Rank 0 of the reference arm prints one JSON line with the bench
+    contract's keys: the oracle timed on the host cores, its own line doubling
+    as cpu_baseline and e2e (no host-device copies)."""
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "1"], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
+    assert d["steps"] == 1 and d["warmup"] == 1 and d["n_gpus"] == 1 and d["higher_is_better"] is True
+    assert d["config"]["workload"] == "prefill_bf16_B4_T4096_hk16_hv32_d128_C64"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert abs(d["ms_per_step"] - 1e3 * 4 * 4096 / d["value"]) <= 1e-6 * d["ms_per_step"]
+
+
 def test_roofline_counts():
     from linear_attention_sequence_sm_b200 import inputs as I
     # 6 d^2 + 3 C d + 2 C d / G at d = 128, C = 64, G = 2
