@@ -25,7 +25,7 @@
  *     a NULL initial state means zeros.
  *   - the output at t reads the state AFTER the update at t.
  *
- * Three independent formulations live here:
+ * Independent formulations live here:
  *   gdn_oracle_recurrent   -- the token recurrence (the oracle proper).
  *   gdn_oracle_chunkwise   -- the chunked form with a per-chunk cumulative
  *                             decay and the WY/UT triangular factor, derived
@@ -44,7 +44,14 @@
  *                             section 8): one decay per key channel; the
  *                             token recurrence and an independent chunked
  *                             form derived from it.
+ *   gdn_oracle_backward / gdn_oracle_backward_chunkwise -- the gradients:
+ *                             the reverse mode of the token recurrence, and
+ *                             an independent derivation through the chunk
+ *                             forms.
  * and the mixer's two sides around the recurrence:
+ *   gdn_oracle_short_conv    -- the short causal depthwise convolution of
+ *                             the projections, with an optional SiLU, and
+ *                             its per-sequence conv state (the input side).
  *   gdn_oracle_prepare       -- q, k L2-normalised per head; gates from
  *                             their logits (the input side).
  *   gdn_oracle_output_side   -- RMS normalisation of each output row with a
@@ -1125,4 +1132,53 @@ void gdn_oracle_output_side(int64_t tokens, int32_t hv, int32_t dv, const double
             }
         }
     }
+}
+
+/* The short causal convolution of the mixer's input side, with an optional
+ * SiLU after it.  "Architecture Thread I", "Modern Architecture
+ * Improvements", items 2 and the module structure that follows it: after
+ * the linear projections, q and k pass through a short convolution, SiLU and
+ * L2 normalisation, and v through a short convolution and SiLU.  The page
+ * gives neither the width nor the tap order; this oracle takes the plain
+ * causal depthwise reading: one filter of W taps per channel, and
+ *     y[t, c] = act( sum_{j=0}^{W-1} w[c, j] x[t - (W-1) + j, c] ),
+ * so w[c, W-1] multiplies the current token.  Inputs before a sequence's
+ * first token come from that sequence's conv state (its W-1 preceding
+ * inputs, oldest first), or are zero when no state is given; a sequence
+ * never reads another's tokens.  act is SiLU, a / (1 + e^-a), when silu is
+ * set, the identity otherwise.
+ *   x, y        [tokens, channels], token-major; y must not alias x
+ *   w           [channels, W]
+ *   cu_seqlens  [num_seqs + 1]
+ *   state_in    [num_seqs, channels, W-1] or NULL (zeros)
+ *   state_out   [num_seqs, channels, W-1] or NULL: the last W-1 inputs seen
+ *               by the sequence (reaching into state_in when it is shorter);
+ *               it may alias state_in (entry i is written after every read
+ *               of entries <= i)
+ * Returns 0, or -1 for W < 1 or a bad cu_seqlens. */
+int gdn_oracle_short_conv(int64_t tokens, int32_t channels, int32_t width, const double *x, const double *w,
+                          const int64_t *cu_seqlens, int64_t num_seqs, const double *state_in, double *y,
+                          double *state_out, int32_t silu) {
+    if (width < 1 || channels < 1 || num_seqs < 0) return -1;
+    if (cu_seqlens[0] != 0 || cu_seqlens[num_seqs] != tokens) return -1;
+    for (int64_t n = 0; n < num_seqs; ++n)
+        if (cu_seqlens[n + 1] < cu_seqlens[n]) return -1;
+    const int32_t hist = width - 1;
+    for (int64_t n = 0; n < num_seqs; ++n) {
+        const int64_t s = cu_seqlens[n], e = cu_seqlens[n + 1];
+        for (int32_t c = 0; c < channels; ++c) {
+            const double *st = state_in ? state_in + (n * channels + c) * (int64_t)hist : NULL;
+            /* the input at token u of this sequence's timeline (u < s reaches into the state) */
+#define CONV_IN(u) ((u) >= s ? x[(u) * channels + c] : (st ? st[hist - (s - (u))] : 0.0))
+            for (int64_t t = s; t < e; ++t) {
+                double acc = 0.0;
+                for (int32_t j = 0; j < width; ++j) acc += w[(int64_t)c * width + j] * CONV_IN(t - hist + j);
+                y[t * channels + c] = silu ? acc / (1.0 + exp(-acc)) : acc;
+            }
+            if (state_out)
+                for (int32_t i = 0; i < hist; ++i) state_out[(n * channels + c) * (int64_t)hist + i] = CONV_IN(e - hist + i);
+#undef CONV_IN
+        }
+    }
+    return 0;
 }

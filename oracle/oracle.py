@@ -93,6 +93,9 @@ def load(path: str | None = None):
         lib.gdn_oracle_output_side.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, D, D, D,
                                                ctypes.c_double, ctypes.c_uint32, D]
         lib.gdn_oracle_output_side.restype = None
+        lib.gdn_oracle_short_conv.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, D, D, U,
+                                              ctypes.c_int64, D, D, D, ctypes.c_int32]
+        lib.gdn_oracle_short_conv.restype = ctypes.c_int
         GP = ctypes.POINTER(_Grads)
         lib.gdn_oracle_backward.argtypes = [P, GP, ctypes.c_int]
         lib.gdn_oracle_backward.restype = ctypes.c_int
@@ -267,6 +270,47 @@ def prepare_inputs(q, k, g, beta, qk_l2norm=False, gate_logits=False, lib=None):
     L.gdn_oracle_prepare(ctypes.c_int64(tokens), ctypes.c_int32(hk), ctypes.c_int32(hv), ctypes.c_int32(dk),
                          _dptr(q64), _dptr(k64), _dptr(g64), _dptr(b64), ctypes.c_uint32(flags))
     return q64, k64, g64, b64
+
+
+def short_conv(x, weight, cu_seqlens=None, state=None, silu=True, lib=None):
+    """The input side's short causal convolution in fp64
+    (``gdn_oracle_short_conv``): one filter of W taps per channel along the
+    tokens of each sequence, y[t] = act(sum_j w[j] x[t - (W-1) + j]) with the
+    last tap on the current token, then SiLU when ``silu``.
+
+    x is [B, T, *channel dims] (batched) or [T, *channel dims] with
+    ``cu_seqlens`` [N + 1]; weight is [*channel dims, W]; state (the W-1
+    inputs before each sequence, oldest first) is [N, *channel dims, W-1] or
+    None for zeros.  Returns (y shaped like x, the state after each sequence
+    [N, *channel dims, W-1])."""
+    L = lib or load()
+    x64 = _f64(x)
+    w64 = _f64(weight)
+    width = w64.shape[-1]
+    ch_shape = w64.shape[:-1]
+    channels = int(np.prod(ch_shape))
+    if cu_seqlens is None:
+        B, T = x64.shape[0], x64.shape[1]
+        assert x64.shape[2:] == ch_shape, (x64.shape, ch_shape)
+        cu = np.arange(B + 1, dtype=np.int64) * T
+    else:
+        assert x64.shape[1:] == ch_shape, (x64.shape, ch_shape)
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    n = cu.shape[0] - 1
+    tokens = x64.size // channels
+    s64 = None
+    if state is not None:
+        s64 = _f64(state)
+        assert s64.shape == (n, *ch_shape, width - 1), (s64.shape, (n, *ch_shape, width - 1))
+    y = np.empty_like(x64)
+    s_out = np.empty((n, *ch_shape, width - 1))
+    rc = L.gdn_oracle_short_conv(ctypes.c_int64(tokens), ctypes.c_int32(channels), ctypes.c_int32(width),
+                                 _dptr(x64), _dptr(w64), cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                 ctypes.c_int64(n), _dptr(s64), _dptr(y), _dptr(s_out),
+                                 ctypes.c_int32(1 if silu else 0))
+    if rc != 0:
+        raise ValueError("oracle short_conv rejected its arguments")
+    return y, s_out
 
 
 # output-side flags of gdn_oracle_output_side (the oracle's own numbering)

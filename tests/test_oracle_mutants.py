@@ -98,6 +98,16 @@ MUTANTS = [
      "for (int64_t c0 = t_begin - t_begin % C; c0 < t_end; c0 += C, ++chunk_idx) {"),
     ("backward: reverse walk stops before the first token",
      "for (int64_t t = T - 1; t >= 0; --t) {", "for (int64_t t = T - 1; t >= 1; --t) {"),
+    ("conv taps reversed",
+     "acc += w[(int64_t)c * width + j] * CONV_IN(t - hist + j);",
+     "acc += w[(int64_t)c * width + (width - 1 - j)] * CONV_IN(t - hist + j);"),
+    ("conv reads across the sequence start",
+     "#define CONV_IN(u) ((u) >= s ?", "#define CONV_IN(u) ((u) >= 0 ?"),
+    ("conv state ignored",
+     "(st ? st[hist - (s - (u))] : 0.0)", "(0.0)"),
+    ("conv activation a sigmoid, not SiLU",
+     "y[t * channels + c] = silu ? acc / (1.0 + exp(-acc)) : acc;",
+     "y[t * channels + c] = silu ? 1.0 / (1.0 + exp(-acc)) : acc;"),
     ("A built with Gamma transposed",
      "a = p->beta[(c0 + r) * p->hv + h] * exp(G[r] - G[j]) * kk;",
      "a = p->beta[(c0 + r) * p->hv + h] * exp(G[j] - G[r]) * kk;"),
@@ -137,6 +147,9 @@ class _Bound:
     def kda_chunkwise(self, *a, **kw):
         return oracle.kda_chunkwise(*a, lib=self.lib, **kw)
 
+    def short_conv(self, *a, **kw):
+        return oracle.short_conv(*a, lib=self.lib, **kw)
+
 
 def _pin_calls(m):
     return [
@@ -162,6 +175,9 @@ def _pin_calls(m):
         lambda: pins.test_kda_chunkwise_equals_recurrent(m, 4),
         lambda: pins.test_backward_matches_finite_differences(m),
         lambda: pins.test_backward_chunkwise_equals_token_recurrence(m, 4),
+        lambda: pins.test_short_conv_identity_and_shift(m),
+        lambda: pins.test_short_conv_equals_numpy_correlate(m),
+        lambda: pins.test_short_conv_continuation(m),
     ]
 
 

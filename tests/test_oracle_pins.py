@@ -583,3 +583,89 @@ def test_backward_chunkwise_equals_token_recurrence(oracle_mod, C):
     b = oracle_mod.backward(q, k, v, g, beta, dO, dSf, initial_state=S0, chunk=C)
     for n in a:
         assert np.allclose(a[n], b[n], rtol=1e-10, atol=1e-11), (n, np.abs(a[n] - b[n]).max())
+
+
+# ---------------------------------------------------------------------------
+# The input side's short causal convolution ("Architecture Thread I",
+# "Modern Architecture Improvements": projection -> short conv -> SiLU)
+# ---------------------------------------------------------------------------
+
+def _conv_case(rng, lens, channels=(2, 3), W=4):
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    x = rng.standard_normal((sum(lens), *channels))
+    w = rng.standard_normal((*channels, W))
+    st = rng.standard_normal((len(lens), *channels, W - 1))
+    return cu, x, w, st
+
+
+def test_short_conv_identity_and_shift(oracle_mod):
+    """The last tap is the current token: a kernel (0, .., 0, 1) is the
+    identity; (1, 0, .., 0) delays by W - 1 tokens, reading the conv state
+    (or zeros) before the sequence's first token."""
+    rng = np.random.default_rng(70)
+    W = 4
+    cu, x, _, st = _conv_case(rng, [6, 2], channels=(3,), W=W)
+    ident = np.zeros((3, W))
+    ident[:, -1] = 1.0
+    y, s = oracle_mod.short_conv(x, ident, cu_seqlens=cu, state=st, silu=False)
+    assert np.array_equal(y, x)
+    delay = np.zeros((3, W))
+    delay[:, 0] = 1.0
+    y, s = oracle_mod.short_conv(x, delay, cu_seqlens=cu, silu=False)
+    assert np.array_equal(y[:3], np.zeros((3, 3))) and np.array_equal(y[3:6], x[0:3])
+    assert np.array_equal(y[6:8], np.zeros((2, 3)))  # the second sequence never sees the first
+    y, s = oracle_mod.short_conv(x, delay, cu_seqlens=cu, state=st, silu=False)
+    assert np.array_equal(y[0:3], st[0].T) and np.array_equal(y[6:8], st[1].T[0:2])
+    # the state after a sequence: its last W - 1 inputs, oldest first; the 2-token sequence keeps
+    # the newest entry of its incoming state in front of its two inputs
+    assert np.array_equal(s[0], x[3:6].T)
+    assert np.array_equal(s[1][:, 0], st[1][:, -1]) and np.array_equal(s[1][:, 1:], x[6:8].T)
+
+
+def test_short_conv_equals_numpy_correlate(oracle_mod):
+    """Against numpy's correlation of (state, sequence) with each channel's
+    filter, and SiLU against scipy's logistic: packed sequences of lengths
+    0 to 9, W = 1, 2 and 4."""
+    from scipy.special import expit
+    rng = np.random.default_rng(71)
+    for W in (1, 2, 4):
+        lens = [5, 0, 1, 9, 2]
+        cu, x, w, st = _conv_case(rng, lens, W=W)
+        y, s = oracle_mod.short_conv(x, w, cu_seqlens=cu, state=st, silu=False)
+        ys, _ = oracle_mod.short_conv(x, w, cu_seqlens=cu, state=st, silu=True)
+        for n in range(len(lens)):
+            a, b = cu[n], cu[n + 1]
+            for c0 in range(2):
+                for c1 in range(3):
+                    full = np.concatenate([st[n, c0, c1], x[a:b, c0, c1]])
+                    if b > a:
+                        ref = np.correlate(full, w[c0, c1], mode="valid")
+                        assert np.allclose(y[a:b, c0, c1], ref, rtol=1e-13, atol=1e-13)
+                    assert np.allclose(s[n, c0, c1], full[len(full) - (W - 1):], rtol=0, atol=0)
+        assert np.allclose(ys, y * expit(y), rtol=1e-13, atol=1e-15)
+    zero, _ = oracle_mod.short_conv(np.zeros((1, 3, 2)), np.ones((2, 4)), silu=True)
+    assert np.array_equal(zero, np.zeros((1, 3, 2)))  # SiLU(0) = 0
+
+
+def test_short_conv_continuation(oracle_mod):
+    """A sequence cut in pieces, each started from the state the previous
+    piece left, gives the uncut result, pieces shorter than W - 1 included."""
+    rng = np.random.default_rng(72)
+    cu, x, w, st = _conv_case(rng, [14], W=4)
+    y, s = oracle_mod.short_conv(x, w, cu_seqlens=cu, state=st)
+    parts, state = [], st
+    for a, b in ((0, 5), (5, 6), (6, 8), (8, 8), (8, 14)):
+        yp, state = oracle_mod.short_conv(x[a:b], w, cu_seqlens=np.array([0, b - a]), state=state)
+        parts.append(yp)
+    assert np.array_equal(np.concatenate(parts), y) and np.array_equal(state, s)
+
+
+def test_short_conv_batched_equals_packed(oracle_mod):
+    """The batched layout [B, T, ...] is the packed one with equal lengths."""
+    rng = np.random.default_rng(73)
+    x = rng.standard_normal((3, 7, 2, 3))
+    w = rng.standard_normal((2, 3, 4))
+    st = rng.standard_normal((3, 2, 3, 3))
+    yb, sb = oracle_mod.short_conv(x, w, state=st)
+    yp, sp = oracle_mod.short_conv(x.reshape(21, 2, 3), w, cu_seqlens=np.array([0, 7, 14, 21]), state=st)
+    assert np.array_equal(yb.reshape(21, 2, 3), yp) and np.array_equal(sb, sp)
