@@ -1,6 +1,7 @@
 """Host logic of bench.py, on CPU: the replica aggregation across ranks (two
-gloo processes), the reference arm on a non-zero rank, and the algorithmic
-byte/FLOP counts behind the roofline fields."""
+gloo processes), the reference arm (its JSON line on rank 0, silence on the
+others), the algorithmic byte/FLOP counts behind the roofline fields, the
+traffic lookup and the clock record."""
 import json
 import os
 import socket
@@ -108,3 +109,33 @@ def test_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
     src.write_text("kernel v2")
     assert bench.kernel_traffic("k") is None
     assert bench.kernel_traffic("missing") is None
+
+
+def test_clock_sampler_against_a_fake_nvml(monkeypatch):
+    """The clock record of the bench line, from a fake NVML: the median SM
+    clock, the maximum, and the clock-event reasons decoded from NVML's bit
+    values (idle and applications-clock bits are not slowdowns and are not
+    reported); without NVML the record is empty, not an error."""
+    import types
+    clocks = iter([1965, 1500, 1965, 1965, 1200])
+    bits = iter([0x0, 0x4, 0x4 | 0x40, 0x1 | 0x2, 0x8 | 0x20])
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=0, nvmlInit=lambda: None, nvmlDeviceGetHandleByIndex=lambda i: ("gpu", i),
+        nvmlDeviceGetMaxClockInfo=lambda h, c: 1965, nvmlDeviceGetClockInfo=lambda h, c: next(clocks),
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: next(bits))
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    cs = bench.ClockSampler(0)
+    for _ in range(5):
+        cs._sample()
+    s = cs.summary()
+    assert s["sm_mhz"] == 1965 and s["sm_max_mhz"] == 1965 and s["samples"] == 5
+    assert s["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_power_cap", "sw_thermal_slowdown"]
+
+    def no_nvml():
+        raise RuntimeError("no driver")
+
+    monkeypatch.setitem(sys.modules, "pynvml", types.SimpleNamespace(nvmlInit=no_nvml))
+    empty = bench.ClockSampler(0)
+    with empty:
+        pass
+    assert empty.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
