@@ -403,6 +403,25 @@ def prepare_kda_inputs(q, k, g, beta, qk_l2norm=False, gate_logits=False, lib=No
     return q64, k64, g64, b64
 
 
+def conv_input_side(q, k, v, conv_q, conv_k, conv_v, cu_seqlens=None, states=None, lib=None):
+    """The input side up to the recurrence's q, k and v, as "Architecture
+    Thread I" ("Modern Architecture Improvements") orders it: q and k pass
+    through the short causal convolution, SiLU and per-head L2
+    normalisation; v through the short convolution and SiLU.  A composition
+    of ``short_conv`` and ``prepare_inputs`` (both pinned), no arithmetic of
+    its own.  conv_q, conv_k are [Hk, d_k, W] and conv_v [Hv, d_v, W];
+    ``states`` is None or a dict of conv states {"q", "k", "v"} each
+    [N, H, d, W-1].  Returns (q, k, v, the conv states after each sequence)."""
+    st = states or {}
+    cq, sq = short_conv(q, conv_q, cu_seqlens=cu_seqlens, state=st.get("q"), silu=True, lib=lib)
+    ck, sk = short_conv(k, conv_k, cu_seqlens=cu_seqlens, state=st.get("k"), silu=True, lib=lib)
+    cv, sv = short_conv(v, conv_v, cu_seqlens=cu_seqlens, state=st.get("v"), silu=True, lib=lib)
+    lead = cq.shape[:-2]
+    zeros = np.zeros(lead + (1,))
+    qn, kn, _, _ = prepare_inputs(cq, ck, zeros, zeros, qk_l2norm=True, lib=lib)
+    return qn, kn, cv, {"q": sq, "k": sk, "v": sv}
+
+
 def decode_multi(q, k, v, g, beta, state, threads=None, lib=None):
     """K decode tokens per sequence with the state after every token:
     q, k [N, K, Hk, dk], v [N, K, Hv, dv], g, beta [N, K, Hv], state

@@ -669,3 +669,36 @@ def test_short_conv_batched_equals_packed(oracle_mod):
     yb, sb = oracle_mod.short_conv(x, w, state=st)
     yp, sp = oracle_mod.short_conv(x.reshape(21, 2, 3), w, cu_seqlens=np.array([0, 7, 14, 21]), state=st)
     assert np.array_equal(yb.reshape(21, 2, 3), yp) and np.array_equal(sb, sp)
+
+
+def test_conv_input_side_composition(oracle_mod):
+    """The composed input side: with width-1 unit filters and the SiLU
+    undone it is the L2 normalisation alone; each output row of q and k has
+    unit norm; v is the SiLU of the convolution; a prefill's conv states
+    carry a continuation exactly."""
+    from scipy.special import expit
+    rng = np.random.default_rng(74)
+    T, hk, hv, dk, dv, W = 11, 2, 4, 8, 6, 4
+    q = rng.standard_normal((1, T, hk, dk))
+    k = rng.standard_normal((1, T, hk, dk))
+    v = rng.standard_normal((1, T, hv, dv))
+    wq, wk, wv = (rng.standard_normal((h, d, W)) for h, d in ((hk, dk), (hk, dk), (hv, dv)))
+    qn, kn, vc, st = oracle_mod.conv_input_side(q, k, v, wq, wk, wv)
+    assert np.allclose(np.linalg.norm(qn, axis=-1), 1.0, rtol=0, atol=1e-12)
+    assert np.allclose(np.linalg.norm(kn, axis=-1), 1.0, rtol=0, atol=1e-12)
+    plain_v, _ = oracle_mod.short_conv(v, wv, silu=False)
+    assert np.allclose(vc, plain_v * expit(plain_v), rtol=1e-13, atol=1e-15)
+    # width-1 unit filters: conv = identity, so q -> L2(SiLU(q)); compare against prepare on SiLU(q)
+    one_q, one_k, one_v = np.ones((hk, dk, 1)), np.ones((hk, dk, 1)), np.ones((hv, dv, 1))
+    q1, k1, v1, _ = oracle_mod.conv_input_side(q, k, v, one_q, one_k, one_v)
+    sq, sk = q * expit(q), k * expit(k)
+    pq, pk, _, _ = oracle_mod.prepare_inputs(sq, sk, np.zeros((1, T, 1)), np.zeros((1, T, 1)), qk_l2norm=True)
+    assert np.allclose(q1, pq, rtol=1e-13, atol=1e-15) and np.allclose(k1, pk, rtol=1e-13, atol=1e-15)
+    assert np.allclose(v1, v * expit(v), rtol=1e-13, atol=1e-15)
+    # a prefill of the first 7 tokens, then the rest from its conv states
+    a = oracle_mod.conv_input_side(q[:, :7], k[:, :7], v[:, :7], wq, wk, wv)
+    b = oracle_mod.conv_input_side(q[:, 7:], k[:, 7:], v[:, 7:], wq, wk, wv, states=a[3])
+    for i in range(3):
+        assert np.array_equal(np.concatenate([a[i], b[i]], axis=1), (qn, kn, vc)[i])
+    for n in ("q", "k", "v"):
+        assert np.array_equal(b[3][n], st[n])
