@@ -28,12 +28,22 @@ _lib = None
 
 
 def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:
-    """Compile the oracle (plain C11, fp64, no fast-math) into a shared library."""
-    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
-        return out
+    """Compile the oracle (plain C11, fp64, no fast-math) into a shared library.
+    A library is reused only if it was built from a source of the same
+    content (its SHA-256 is kept beside it), whatever the files' times."""
+    import hashlib
+    with open(src, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()
+    stamp = out + ".sha256"
+    if not force and os.path.exists(out) and os.path.exists(stamp):
+        with open(stamp) as f:
+            if f.read().strip() == digest:
+                return out
     cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", "-fno-fast-math",
            "-ffp-contract=off", "-o", out, src, "-lm"]
     subprocess.run(cmd, check=True)
+    with open(stamp, "w") as f:
+        f.write(digest + "\n")
     return out
 
 
