@@ -7,6 +7,7 @@ without a GPU driver (calls then fail with GDN_ERR_CUDA).
 from __future__ import annotations
 
 import glob
+import hashlib
 import os
 import subprocess
 import sys
@@ -29,11 +30,25 @@ def _deps():
     return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [os.path.join(ROOT, "include", "gdn.h")]
 
 
+def _digest() -> str:
+    """SHA-256 over the names and contents of every source and header and the
+    compiler flags: the library is current only for exactly these inputs
+    (file times say nothing once a tree is copied or checked out)."""
+    h = hashlib.sha256()
+    for p in _deps():
+        h.update(os.path.relpath(p, ROOT).encode() + b"\0")
+        with open(p, "rb") as f:
+            h.update(f.read())
+    h.update(" ".join(ARCH + FLAGS).encode())
+    return h.hexdigest()
+
+
 def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+    stamp = LIB + ".sha256"
+    if not (os.path.exists(LIB) and os.path.exists(stamp)):
         return False
-    t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(p) <= t for p in _deps())
+    with open(stamp) as f:
+        return f.read().strip() == _digest()
 
 
 def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False) -> str:
@@ -67,6 +82,8 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
+    with open(LIB + ".sha256", "w") as f:
+        f.write(_digest() + "\n")
     return LIB
 
 
