@@ -68,27 +68,72 @@ def prefill_errors(inp, o_gpu, sf_gpu, o_ref, sf_ref, units=None):
     return worst_o, worst_s
 
 
-def oracle_units_sliced(inp, units, hv, hk):
-    """Oracle outputs for the listed (sequence, head) units, each run on its own
-    head's slice of the inputs (keeps host memory bounded at full sizes).
-    Returns {unit: (o [T_n, d_v], final state [d_v, d_k])}."""
+def _seq_bounds(inp):
+    """(start, end) token bounds of every sequence in the flattened token axis."""
+    q = inp["q"]
+    if inp["cu_seqlens"] is None:
+        B, T = q.shape[0], q.shape[1]
+        return [(b * T, (b + 1) * T) for b in range(B)]
+    cu = inp["cu_seqlens"].tolist()
+    return [(cu[n], cu[n + 1]) for n in range(len(cu) - 1)]
+
+
+def _segment_rel(err2, ref2, starts):
+    """Max over token segments (each from one start to the next) of
+    sqrt(sum err2) / max(sqrt(sum ref2), 1e-30), per head column."""
+    if len(starts) == 0:
+        return 0.0
+    e = np.add.reduceat(err2, starts, axis=0)
+    r = np.add.reduceat(ref2, starts, axis=0)
+    return float((np.sqrt(e) / np.maximum(np.sqrt(r), 1e-30)).max())
+
+
+def full_prefill_errors(inp, o_gpu, sf_gpu, chunk=64, threads=None):
+    """Every (sequence, value head) unit of a prefill against the fp64 oracle.
+
+    The oracle runs a few q/k heads at a time (with their value heads), so
+    host memory stays bounded at full sizes.  Returns a dict:
+      o_slice  max rel-L2 over (sequence, head) slices of o (the parity metric)
+      o_chunk  max rel-L2 over (sequence, head, chunk of ``chunk`` tokens)
+               slices of o, so that one wrong chunk cannot hide in a long slice
+      state    max rel-L2 over the (sequence, head) final states
+      units    (sequence, head) units compared
+    """
     from oracle import oracle
+    threads = threads or oracle.default_threads()
+    hk, hv = inp["q"].shape[-2], inp["v"].shape[-2]
     G = hv // hk
-    q, k, v = inp["q"], inp["k"], inp["v"]
-    res = {}
-    for u in units:
-        n, h = divmod(u, hv)
-        hq = h // G
-        if inp["cu_seqlens"] is None:
-            qs, ks = q[n, :, hq:hq + 1], k[n, :, hq:hq + 1]
-            vs, gs, bs = v[n, :, h:h + 1], inp["g"][n, :, h:h + 1], inp["beta"][n, :, h:h + 1]
-        else:
-            cu = inp["cu_seqlens"].tolist()
-            a, b = cu[n], cu[n + 1]
-            qs, ks = q[0, a:b, hq:hq + 1], k[0, a:b, hq:hq + 1]
-            vs, gs, bs = v[0, a:b, h:h + 1], inp["g"][0, a:b, h:h + 1], inp["beta"][0, a:b, h:h + 1]
-        s0 = None if inp["initial_state"] is None else to_f64(inp["initial_state"][n:n + 1, h:h + 1])
-        o, sf = oracle.recurrent(to_f64(qs)[None], to_f64(ks)[None], to_f64(vs)[None], to_f64(gs)[None],
-                                 to_f64(bs)[None], initial_state=s0)
-        res[u] = (o[0, :, 0], sf[0, 0])
+    bounds = _seq_bounds(inp)
+    N = len(bounds)
+    seq_starts = np.array([a for a, b in bounds if b > a], dtype=np.int64)
+    chunk_starts = np.array([t for a, b in bounds for t in range(a, b, chunk)], dtype=np.int64)
+    dv = inp["v"].shape[-1]
+    og_all = o_gpu.detach().reshape(-1, hv, dv)
+    sg_all = None if sf_gpu is None else sf_gpu.detach()
+    per_call = max(1, min(hk, -(-threads // max(1, N * G))))
+    cu = None if inp["cu_seqlens"] is None else inp["cu_seqlens"].numpy().astype(np.int64)
+    res = {"o_slice": 0.0, "o_chunk": 0.0, "state": 0.0, "units": 0}
+    for q0 in range(0, hk, per_call):
+        q1 = min(hk, q0 + per_call)
+        h0, h1 = q0 * G, q1 * G
+        q = to_f64(inp["q"][..., q0:q1, :])
+        k = to_f64(inp["k"][..., q0:q1, :])
+        v = to_f64(inp["v"][..., h0:h1, :])
+        g = to_f64(inp["g"][..., h0:h1])
+        b = to_f64(inp["beta"][..., h0:h1])
+        s0 = None if inp["initial_state"] is None else to_f64(inp["initial_state"][:, h0:h1])
+        o_ref, s_ref = oracle.recurrent(q, k, v, g, b, initial_state=s0, cu_seqlens=cu, threads=threads)
+        o_ref = np.asarray(o_ref).reshape(-1, h1 - h0, dv)
+        og = to_f64(og_all[:, h0:h1].cpu())
+        err2 = ((og - o_ref) ** 2).sum(axis=-1)
+        ref2 = (o_ref ** 2).sum(axis=-1)
+        res["o_slice"] = max(res["o_slice"], _segment_rel(err2, ref2, seq_starts))
+        res["o_chunk"] = max(res["o_chunk"], _segment_rel(err2, ref2, chunk_starts))
+        if sg_all is not None:
+            sg = to_f64(sg_all[:, h0:h1].cpu())
+            e = np.sqrt(((sg - s_ref) ** 2).sum(axis=(-2, -1)))
+            r = np.maximum(np.sqrt((s_ref ** 2).sum(axis=(-2, -1))), 1e-30)
+            res["state"] = max(res["state"], float((e / r).max()))
+        res["units"] += N * (h1 - h0)
+        del q, k, v, g, b, s0, o_ref, s_ref, og, err2, ref2
     return res

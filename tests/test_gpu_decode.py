@@ -10,14 +10,21 @@ from parity import BAR, to_f64
 pytestmark = pytest.mark.gpu
 
 
-def _run(w, steps, units=None, dtype="bf16"):
+def _rel(x, ref, axes):
+    """Per-(sequence, head) relative L2 errors, norms over ``axes``."""
+    e = np.sqrt(((x - ref) ** 2).sum(axis=axes))
+    return e / np.maximum(np.sqrt((ref ** 2).sum(axis=axes)), 1e-30)
+
+
+def _run(w, steps):
+    """``steps`` decode steps of workload ``w`` on the GPU (state in place) and
+    in the oracle; every (sequence, head) unit's output compared at every
+    step, and the state after the last step.  Returns (worst o, worst state)."""
     from linear_attention_sequence_sm_b200 import gdn
     from oracle import oracle
     dev = torch.device("cuda:0")
     state = I.make_decode_state(w)
     ref_state = to_f64(state)
-    if units is not None:
-        ref_state = ref_state.copy()
     st = state.to(dev)
     worst_o = 0.0
     for step in range(steps):
@@ -26,33 +33,9 @@ def _run(w, steps, units=None, dtype="bf16"):
         o = gdn.decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], st)
         torch.cuda.synchronize()
         xs = {k: to_f64(v) for k, v in x.items()}
-        if units is None:
-            o_ref, ref_state = oracle.decode_step(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], ref_state)
-            og = to_f64(o)
-            for n in range(w.num_seqs):
-                for h in range(w.hv):
-                    e = np.linalg.norm(og[n, h] - o_ref[n, h]) / max(np.linalg.norm(o_ref[n, h]), 1e-30)
-                    worst_o = max(worst_o, e)
-        else:
-            # sampled units: run the oracle on those (sequence, head) pairs only
-            og = to_f64(o)
-            for u in units:
-                n, h = divmod(u, w.hv)
-                hq = h // (w.hv // w.hk)
-                o_ref, s_new = oracle.decode_step(xs["q"][n:n + 1, hq:hq + 1], xs["k"][n:n + 1, hq:hq + 1],
-                                                  xs["v"][n:n + 1, h:h + 1], xs["g"][n:n + 1, h:h + 1],
-                                                  xs["beta"][n:n + 1, h:h + 1], ref_state[n:n + 1, h:h + 1])
-                ref_state[n, h] = s_new[0, 0]
-                e = np.linalg.norm(og[n, h] - o_ref[0, 0]) / max(np.linalg.norm(o_ref[0, 0]), 1e-30)
-                worst_o = max(worst_o, e)
-    sg = to_f64(st)
-    worst_s = 0.0
-    for n in range(w.num_seqs):
-        for h in range(w.hv):
-            if units is not None and n * w.hv + h not in units:
-                continue
-            e = np.linalg.norm(sg[n, h] - ref_state[n, h]) / max(np.linalg.norm(ref_state[n, h]), 1e-30)
-            worst_s = max(worst_s, e)
+        o_ref, ref_state = oracle.decode_step(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], ref_state)
+        worst_o = max(worst_o, float(_rel(to_f64(o), o_ref, (-1,)).max()))
+    worst_s = float(_rel(to_f64(st), ref_state, (-2, -1)).max())
     return worst_o, worst_s
 
 
@@ -64,12 +47,13 @@ def test_decode_small(dtype, d):
     assert eo <= BAR[dtype] and es <= BAR[dtype], (eo, es)
 
 
-def test_decode_full_size_sampled():
+def test_decode_full_size_all_units():
     """256 sequences, 16/32 heads, d=128, fp32 state of 512 MiB updated in
-    place; 24 steps checked on 6 sampled (sequence, head) units."""
+    place; every (sequence, head) unit checked at each of 64 steps, and the
+    whole state after them."""
     w = I.decode_bf16()
-    units = [0, 31, 4000, 5555, 8000, 256 * 32 - 1]
-    eo, es = _run(w, 24, units=units)
+    eo, es = _run(w, 64)
+    print(f"PARITY {w.name}: 64 steps, all {w.num_seqs * w.hv} units: o {eo:.3e} state {es:.3e}")
     assert eo <= BAR["bf16"] and es <= BAR["bf16"], (eo, es)
 
 
