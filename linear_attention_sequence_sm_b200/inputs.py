@@ -69,16 +69,32 @@ def normal(seed: int, tag: str, shape, mean: float = 0.0, std: float = 1.0, offs
 def _slabbed(seed: int, tag: str, shape, fn, out_dtype, row_elems: int, slab_rows: int = 8192):
     """Draw normals for ``shape`` slab by slab along the leading flattened rows
     (each row = ``row_elems`` elements), apply ``fn`` (elementwise or per-row)
-    and store into a torch tensor of ``out_dtype``."""
+    and store into a torch tensor of ``out_dtype``.  Slabs are drawn on a pool
+    of host threads (numpy releases the interpreter lock inside its array
+    operations); every slab is a fixed range of counters of the stream, so the
+    values do not depend on the thread count or the order of completion."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
     import torch
     n = int(np.prod(shape))
     rows = n // row_elems
     out = torch.empty(n, dtype=out_dtype)
-    for r0 in range(0, rows, slab_rows):
+
+    def slab(r0):
         r1 = min(rows, r0 + slab_rows)
         off = r0 * row_elems
         z = normal(seed, tag, ((r1 - r0), row_elems), offset=off)
         out[off:r1 * row_elems] = torch.from_numpy(np.ascontiguousarray(fn(z).reshape(-1))).to(out_dtype)
+
+    starts = list(range(0, rows, slab_rows))
+    workers = min(len(starts), len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else 8, 32)
+    if workers <= 1:
+        for r0 in starts:
+            slab(r0)
+    else:
+        with ThreadPoolExecutor(max_workers=workers) as ex:
+            list(ex.map(slab, starts))
     return out.reshape(shape)
 
 
