@@ -13,9 +13,15 @@ independent replica on its own GPU (the problems are independent; there is
 no data-path collective): "scaling" is "weak" and the value is the tokens
 of all ranks over the slowest rank's device time.
 
+The two other prefill workloads are timed in the same run and reported
+under "long" (65,536 tokens, 16/48 heads, initial states) and "varlen" (32
+packed sequences of 128..8192 tokens): each with its own roofline, e2e and
+CPU baseline.
+
 --impl reference times the fp64 CPU oracle on the host cores instead (on
-rank 0 only), each step a bounded sample of (sequence, head) units of the
-same workload, extrapolated to the workload's tokens/s.
+rank 0 only): every step runs the oracle over the whole 4 x 4096 workload
+(all (sequence, head) units), with the same code that times the GPU arm's
+CPU baseline.
 """
 from __future__ import annotations
 
@@ -67,6 +73,8 @@ def parse_args(argv=None):
                    help="decode: launch each step instead of replaying the ring of steps as one CUDA graph")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extra", action="store_true",
+                   help="time only the headline prefill workload (not the long-context and varlen records)")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
     return p.parse_args(argv)
 
@@ -196,31 +204,52 @@ def timed(fn, steps, stream):
     return start.elapsed_time(end) / steps
 
 
-def cpu_oracle_sample(w, inp, target_s: float):
-    """Time the fp64 oracle on whole (sequence, head) units of the workload and
-    extrapolate to the full workload's tokens/s."""
-    import numpy as np
-    from oracle import oracle
-    f64 = lambda t: None if t is None else t.to(dtype=__import__("torch").float64).numpy()
-    q, k, v, g, b = (f64(inp[n]) for n in ("q", "k", "v", "g", "beta"))
-    s0 = f64(inp["initial_state"])
-    threads = oracle.default_threads()
-    total_units = w.num_seqs * w.hv
-    # calibrate with one round of `threads` units, then run a sample of about target_s
-    cal = list(range(min(threads, total_units)))
-    t0 = time.perf_counter()
-    oracle.recurrent(q, k, v, g, b, initial_state=s0, units=cal, threads=threads)
-    t_cal = time.perf_counter() - t0
-    rounds = max(1, int(target_s / max(t_cal, 1e-3)))
-    n_units = min(total_units, rounds * len(cal))
-    units = list(range(n_units))
-    t0 = time.perf_counter()
-    oracle.recurrent(q, k, v, g, b, initial_state=s0, units=units, threads=threads)
-    t = time.perf_counter() - t0
-    full = t * total_units / n_units
-    return {"value": w.total_tokens / full, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{n_units} of {total_units} (sequence, v-head) units of {w.name} (whole sequences, "
-                      f"{t:.1f} s wall), extrapolated to the full workload"}
+def host_cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+class OracleRun:
+    """The fp64 oracle over every (sequence, head) unit of a workload.
+
+    The fp64 copies of the inputs are made once, outside any timing, and
+    ``run()`` times one pass of the oracle over the whole workload on all host
+    cores.  The GPU arm's CPU baseline and the reference arm both use this."""
+
+    def __init__(self, w, inp):
+        from oracle import oracle
+        self.oracle = oracle
+        f64 = lambda t: None if t is None else t.to(dtype=__import__("torch").float64).numpy()
+        self.args = [f64(inp[n]) for n in ("q", "k", "v", "g", "beta")]
+        self.s0 = f64(inp["initial_state"])
+        self.cu = None if inp["cu_seqlens"] is None else inp["cu_seqlens"].numpy().astype("int64")
+        self.threads = oracle.default_threads()
+        self.w = w
+
+    def run(self) -> float:
+        t0 = time.perf_counter()
+        self.oracle.recurrent(*self.args, initial_state=self.s0, cu_seqlens=self.cu, threads=self.threads)
+        return time.perf_counter() - t0
+
+
+def cpu_baseline(w, inp, target_s: float):
+    """Whole-workload passes of the oracle until about ``target_s`` seconds
+    (at least one); tokens/s = tokens / mean seconds per pass."""
+    r = OracleRun(w, inp)
+    times = [r.run()]
+    while sum(times) < target_s and len(times) < 50:
+        times.append(r.run())
+    per = statistics.mean(times)
+    return {"value": w.total_tokens / per, "unit": "tokens/s", "cores": r.threads, "kind": "oracle",
+            "cpu_model": host_cpu_model(), "seconds_per_pass": per,
+            "sample": f"the whole workload {w.name} (all {w.num_seqs * w.hv} (sequence, v-head) units), "
+                      f"{len(times)} pass(es), not extrapolated"}
 
 
 def run_reference(args):
@@ -228,59 +257,112 @@ def run_reference(args):
     if rank != 0:
         return 0
     from linear_attention_sequence_sm_b200 import inputs as I
-    from oracle import oracle
-    import numpy as np
     w = I.prefill_bf16()
-    inp = I.make_prefill_inputs(w)
-    f64 = lambda t: None if t is None else t.to(dtype=__import__("torch").float64).numpy()
-    q, k, v, g, b = (f64(inp[n]) for n in ("q", "k", "v", "g", "beta"))
-    threads = oracle.default_threads()
-    total_units = w.num_seqs * w.hv
-    per_step = min(total_units, threads)  # one unit per host thread per step
+    r = OracleRun(w, I.make_prefill_inputs(w))
     times = []
     for i in range(args.warmup + args.steps):
-        units = [(i * per_step + j) % total_units for j in range(per_step)]
-        t0 = time.perf_counter()
-        oracle.recurrent(q, k, v, g, b, units=units, threads=threads)
-        dt = time.perf_counter() - t0
+        dt = r.run()
         if i >= args.warmup:
             times.append(dt)
-    step_s = statistics.mean(times) * total_units / per_step  # extrapolated full-workload step
+    step_s = statistics.mean(times)
     value = w.total_tokens / step_s
-    sample = f"{per_step} of {total_units} (sequence, v-head) units per step of {w.name}, extrapolated"
+    sample = f"the whole workload {w.name} (all {w.num_seqs * w.hv} (sequence, v-head) units) every step"
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded splitmix64)",
         "config": {"workload": w.name, "global_batch": w.batch, "seq_len": w.seq_len, "parallelism": "none (host cores)"},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": r.threads, "kind": "oracle",
+                         "cpu_model": host_cpu_model(), "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
     return 0
 
 
-def run_ours(args):
+def e2e_record(fwd, w, host, ws, flags, out_norm, steps, device, world, stream):
+    """The prefill through the public call with host buffers: every step copies
+    its inputs from pinned host memory and its outputs (o and the final
+    states) back, inside the timed region."""
     import torch
-    rank, world, local_rank = dist_env()
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    device = torch.device("cuda", local_rank)
-    torch.cuda.set_device(device)
+    pin = {k: v.pin_memory() for k, v in host.items() if v is not None}
+    dv0 = next(iter(v for k, v in pin.items() if k == "v"))
+    o_shape, sf_shape = dv0.shape, (w.num_seqs, w.hv, w.d, w.d)
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = dv0.numel() * dv0.element_size() + w.num_seqs * w.hv * w.d * w.d * 4
+
+    # Steps overlap across three streams, double-buffered: step i's inputs copy in while step i-1
+    # computes and step i-2's results copy out (separate copy engines for the two directions).
+    # Every step still copies its own inputs from pinned host memory and its own results back.
+    s_in, s_out, comp = torch.cuda.Stream(device), torch.cuda.Stream(device), stream
+    dbuf = [{k: torch.empty_like(v, device=device) for k, v in pin.items()} for _ in range(2)]
+    obuf = [torch.empty(o_shape, dtype=dv0.dtype, device=device) for _ in range(2)]
+    sbuf = [torch.empty(sf_shape, dtype=torch.float32, device=device) for _ in range(2)]
+    ohost = [torch.empty(o_shape, dtype=dv0.dtype).pin_memory() for _ in range(2)]
+    shost = [torch.empty(sf_shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    ev_in, ev_comp, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
+    for b in range(2):
+        ev_comp[b].record(comp)
+        ev_out[b].record(comp)
+    it = [0]
+
+    def e2e_step():
+        b = it[0] % 2
+        it[0] += 1
+        x = dbuf[b]
+        s_in.wait_event(ev_comp[b])  # the step that last read these input buffers has run
+        with torch.cuda.stream(s_in):
+            for k_ in x:
+                x[k_].copy_(pin[k_], non_blocking=True)
+        ev_in[b].record(s_in)
+        comp.wait_event(ev_in[b])
+        comp.wait_event(ev_out[b])  # the results last held in these output buffers have left
+        with torch.cuda.stream(comp):
+            fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], initial_state=x.get("initial_state"),
+                cu_seqlens=x.get("cu_seqlens"), chunk_size=w.chunk, out=obuf[b], final_state=sbuf[b],
+                workspace=ws, **flags, **out_norm(x))
+        ev_comp[b].record(comp)
+        s_out.wait_event(ev_comp[b])
+        with torch.cuda.stream(s_out):
+            ohost[b].copy_(obuf[b], non_blocking=True)
+            shost[b].copy_(sbuf[b], non_blocking=True)
+        ev_out[b].record(s_out)
+
+    def e2e_timed(n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(comp)
+        s_in.wait_stream(comp)
+        for _ in range(n):
+            e2e_step()
+        comp.wait_stream(s_out)
+        e1.record(comp)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    e_ms = max_over_ranks(e2e_timed(max(3, min(steps, 20))), device, world)
+    del dbuf, obuf, sbuf
+    return {"value": world * w.total_tokens / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
+            "overlap": "copy-in, compute and copy-out of consecutive steps on three streams, double-buffered"}
+
+
+def prefill_record(args, w, host, device, world, rank, peaks, peak_src, e2e=True, cpu=True):
+    """Times the prefill of workload ``w`` (inputs resident in HBM) and returns
+    its record: ms per step (max over ranks), tokens/s of all ranks, the
+    roofline of the dominant kernel, the e2e figure and the CPU baseline."""
+    import torch
     from linear_attention_sequence_sm_b200 import gdn
     from linear_attention_sequence_sm_b200 import inputs as I
-
-    peaks, peak_src = load_peaks()
-    w = {"prefill": I.prefill_bf16, "long": I.long_bf16, "varlen": I.varlen_bf16}[args.workload](
-        seed={"prefill": 1002, "long": 1003, "varlen": 1005}[args.workload] + rank)
-    host = I.make_raw_prefill_inputs(w) if args.raw_inputs else I.make_prefill_inputs(w)
     flags = {"qk_l2norm": True, "gate_logits": True} if args.raw_inputs else {}
     suffix = ("_kda" if args.kda else "") + ("_raw_inputs" if args.raw_inputs else "") + \
         ("_output_norm" if args.output_norm else "") + ("_backward" if args.backward else "")
     if args.kda:
         host["g"] = I.make_kda_gates(w)
     fwd = gdn.kda_forward if args.kda else gdn.chunk_forward
+    out_weight = None
     if args.output_norm:
         host["out_gate"] = I.make_output_gate(w)
         out_weight = I.make_output_weight(w).to(device)
@@ -310,27 +392,23 @@ def run_ours(args):
                                initial_state=dev["initial_state"], cu_seqlens=dev["cu_seqlens"], workspace=bws)
             return
         fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], initial_state=dev["initial_state"],
-                          cu_seqlens=dev["cu_seqlens"], out=o, final_state=sf, workspace=ws, chunk_size=w.chunk,
-                          **flags, **out_norm(dev))
+            cu_seqlens=dev["cu_seqlens"], out=o, final_state=sf, workspace=ws, chunk_size=w.chunk,
+            **flags, **out_norm(dev))
 
-    ms = ms_max = float("nan")
-    launches = 0
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    n0 = gdn.launch_count()
     clocks = ClockSampler(device.index)
-    if args.only in ("all", "prefill"):
-        for _ in range(max(3, args.warmup)):
-            step()
+    with clocks:
+        ms = timed(step, args.steps, stream)
         torch.cuda.synchronize(device)
-        barrier(world, device)
-        torch.cuda.synchronize(device)
-        n0 = gdn.launch_count()
-        with clocks:
-            ms = timed(step, args.steps, stream)
-            torch.cuda.synchronize(device)
-        launches = gdn.launch_count() - n0
-        barrier(world, device)
-        ms_max = max_over_ranks(ms, device, world)
+    launches = gdn.launch_count() - n0
+    barrier(world, device)
+    ms_max = max_over_ranks(ms, device, world)
     tokens = w.total_tokens
-    value = aggregate_value(tokens, ms_max, world)
     flops = useful_flops_per_vhead_token(w.hv // w.hk) * tokens * w.hv
     achieved_tflops = flops / (ms / 1e3) / 1e12
     kernel_name = "gdn_chunk_tc" if gdn_tc_active(gdn, dev, w) else "gdn_chunk_simt"
@@ -342,12 +420,12 @@ def run_ours(args):
                 "frac_vs_sustained": achieved_tflops / peaks["bf16_tflops_sustained"],
                 "frac_vs_nominal_2250": achieved_tflops / 2250.0,
                 "flops_per_launch": flops, "algorithmic_bytes_per_launch": prefill_bytes(w)}
+    alu_peak = FP32_LANES_PER_SM * 2 * torch.cuda.get_device_properties(device).multi_processor_count * \
+        (clocks.summary().get("sm_max_mhz") or 1965) * 1e6 / 1e12
     if args.backward:
         # reverse mode of the token recurrence: 20 d^2 flops per (token, value head) (the forward
         # recomputed, 6 d^2, and the backward, 14 d^2); fp32 on CUDA cores
         bflops = 20 * w.d * w.d * tokens * w.hv
-        alu_peak = FP32_LANES_PER_SM * 2 * torch.cuda.get_device_properties(device).multi_processor_count * \
-            (clocks.summary().get("sm_max_mhz") or 1965) * 1e6 / 1e12
         achieved = bflops / (ms / 1e3) / 1e12
         roofline = {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s",
                     "frac": achieved / alu_peak, "traffic": kernel_traffic(f"gdn_backward/{w.name}{suffix}"),
@@ -357,163 +435,149 @@ def run_ours(args):
         # token-order recurrence on CUDA cores: 7 d_v d_k fp32 flops per (token, value head)
         # (decay, two dot products, rank-1 write); peak = SMs x 128 fp32 lanes x 2 x max SM clock
         kflops = kda_flops_per_vhead_token(w.d) * tokens * w.hv
-        alu_peak = FP32_LANES_PER_SM * 2 * torch.cuda.get_device_properties(device).multi_processor_count * \
-            (clocks.summary().get("sm_max_mhz") or 1965) * 1e6 / 1e12
         achieved = kflops / (ms / 1e3) / 1e12
         roofline = {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s",
                     "frac": achieved / alu_peak, "traffic": kernel_traffic(f"gdn_kda/{w.name}{suffix}"),
                     "kernel": "gdn_kda", "peak_source": "fp32 FMA lanes x 2 x max SM clock (derived)",
                     "flops_per_launch": kflops, "algorithmic_bytes_per_launch": prefill_bytes(w, kda=True)}
+    rec = {"workload": w.name + suffix, "ms_per_step": ms_max, "tokens_per_s": aggregate_value(tokens, ms_max, world),
+           "tokens": tokens, "roofline": roofline, "gpu_launches": launches, "clocks": clocks.summary(),
+           "config": {"global_batch": w.num_seqs * world, "seq_len": w.seq_len, "heads_qk_v": [w.hk, w.hv],
+                      "head_dim": w.d, "chunk": w.chunk, "initial_state": w.s0_std > 0,
+                      "l2": f"inputs larger than L2 ({prefill_bytes(w) / 1e6:.0f} MB of mandatory traffic per step)"}}
+    del o, sf
+    if e2e and not args.no_e2e and not args.backward:
+        rec["e2e"] = e2e_record(fwd, w, host, ws, flags, out_norm, args.steps, device, world, stream)
+    # (raw inputs, the output side, KDA or gradients: the timed oracle covers the plain forward only)
+    if cpu and rank == 0 and world == 1 and not args.no_cpu_baseline and not suffix:
+        rec["cpu_baseline"] = cpu_baseline(w, host, args.cpu_seconds)
+    del dev, ws
+    torch.cuda.empty_cache()
+    return rec
 
-    # ---- decode: 256 sequences, fp32 state 512 MiB, in place ----
-    decode = None
+
+def decode_record(args, device, world, rank, peaks, peak_src):
+    """Times the decode step of the 256-sequence workload (state in place)."""
+    import torch
+    from linear_attention_sequence_sm_b200 import gdn
+    from linear_attention_sequence_sm_b200 import inputs as I
     dw = I.decode_bf16()
-    if args.only == "prefill":
-        args.decode_steps = 0
-    if args.decode_steps > 0:
-        gen = torch.Generator(device=device)
-        gen.manual_seed(dw.seed + rank)
-        state = torch.randn((dw.num_seqs, dw.hv, dw.d, dw.d), generator=gen, device=device) * dw.s0_std
-        ring = [{k: v.to(device) for k, v in I.make_decode_inputs(dw, s).items()} for s in range(8)]
-        od = torch.empty((dw.num_seqs, dw.hv, dw.d), dtype=torch.bfloat16, device=device)
-        it = [0]
+    stream = torch.cuda.current_stream(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(dw.seed + rank)
+    state = torch.randn((dw.num_seqs, dw.hv, dw.d, dw.d), generator=gen, device=device) * dw.s0_std
+    ring = [{k: v.to(device) for k, v in I.make_decode_inputs(dw, s).items()} for s in range(8)]
+    od = torch.empty((dw.num_seqs, dw.hv, dw.d), dtype=torch.bfloat16, device=device)
+    it = [0]
+    if args.kda:
+        for s_, x in enumerate(ring):
+            x["g"] = I.make_kda_decode_gates(dw, s_).to(device)
+    if args.mtp > 0:
+        # K draft tokens per sequence: [N, K, H, d] inputs, one snapshot per token
+        K = args.mtp
+        ring = []
+        for s_ in range(4):
+            xs = [I.make_decode_inputs(dw, s_ * K + j) for j in range(K)]
+            ring.append({n: torch.stack([x_[n] for x_ in xs], dim=1).to(device) for n in xs[0]})
+        snaps = torch.empty((dw.num_seqs, K, dw.hv, dw.d, dw.d), dtype=torch.float32, device=device)
+        od = torch.empty((dw.num_seqs, K, dw.hv, dw.d), dtype=torch.bfloat16, device=device)
 
-        if args.kda:
-            for s_, x in enumerate(ring):
-                x["g"] = I.make_kda_decode_gates(dw, s_).to(device)
+    def dstep():
+        x = ring[it[0] % len(ring)]
+        it[0] += 1
         if args.mtp > 0:
-            # K draft tokens per sequence: [N, K, H, d] inputs, one snapshot per token
-            K = args.mtp
-            ring = []
-            for s_ in range(4):
-                xs = [I.make_decode_inputs(dw, s_ * K + j) for j in range(K)]
-                ring.append({n: torch.stack([x_[n] for x_ in xs], dim=1).to(device) for n in xs[0]})
-            snaps = torch.empty((dw.num_seqs, K, dw.hv, dw.d, dw.d), dtype=torch.float32, device=device)
-            od = torch.empty((dw.num_seqs, K, dw.hv, dw.d), dtype=torch.bfloat16, device=device)
+            gdn.decode_multi(x["q"], x["k"], x["v"], x["g"], x["beta"], state, out=od, snapshots=snaps)
+            return
+        (gdn.kda_decode_step if args.kda else gdn.decode_step)(x["q"], x["k"], x["v"], x["g"], x["beta"], state,
+                                                               out=od)
 
-        def dstep():
-            x = ring[it[0] % len(ring)]
-            it[0] += 1
-            if args.mtp > 0:
-                gdn.decode_multi(x["q"], x["k"], x["v"], x["g"], x["beta"], state, out=od, snapshots=snaps)
-                return
-            (gdn.kda_decode_step if args.kda else gdn.decode_step)(x["q"], x["k"], x["v"], x["g"], x["beta"], state,
-                                                                   out=od)
-
-        for _ in range(max(3, args.warmup)):
-            dstep()
+    for _ in range(max(3, args.warmup)):
+        dstep()
+    torch.cuda.synchronize(device)
+    run, per_call = dstep, 1
+    graph = None
+    if not args.no_graph:
+        # the ring of steps captured once and replayed: no host launch gaps between steps
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(len(ring)):
+                dstep()
+        graph.replay()
         torch.cuda.synchronize(device)
-        run, per_call = dstep, 1
-        if not args.no_graph:
-            # the ring of steps captured once and replayed: no host launch gaps between steps
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph):
-                for _ in range(len(ring)):
-                    dstep()
-            graph.replay()
-            torch.cuda.synchronize(device)
-            run, per_call = graph.replay, len(ring)
-        with ClockSampler(device.index) as dclocks:
-            dms = timed(run, max(1, args.decode_steps // per_call), stream) / per_call
-        dms = max_over_ranks(dms, device, world)
-        dbytes = decode_bytes(dw, kda=args.kda, mtp=args.mtp)
-        dgbs = dbytes / (dms / 1e3) / 1e9
-        decode = {"value": world * dgbs, "unit": "GB/s", "ms_per_step": dms, "steps": args.decode_steps,
-                  "tokens_per_s": world * dw.num_seqs * max(1, args.mtp) / (dms / 1e3),
-                  "workload": dw.name + (f"_mtp{args.mtp}" if args.mtp > 0 else ""),
-                  "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                               "frac": dgbs / peaks["hbm_gbs"],
-                               "traffic": kernel_traffic(f"gdn_decode/{dw.name}" + ("_kda" if args.kda else "")
-                                                         + (f"_mtp{args.mtp}" if args.mtp > 0 else "")),
-                               "kernel": "gdn_decode", "peak_source": f"{peak_src} HBM copy",
-                               "frac_vs_nominal_8000": dgbs / 8000.0, "bytes_per_launch": dbytes},
-                  "clocks": dclocks.summary(), "cuda_graph": not args.no_graph}
-        del state
+        run, per_call = graph.replay, len(ring)
+    barrier(world, device)
+    n0 = gdn.launch_count()
+    with ClockSampler(device.index) as dclocks:
+        dms = timed(run, max(1, args.decode_steps // per_call), stream) / per_call
+    # kernels replayed from the graph are not counted by the library's host-side counter
+    launches = (gdn.launch_count() - n0) if graph is None else len(ring) * max(1, args.decode_steps // per_call)
+    dms = max_over_ranks(dms, device, world)
+    dbytes = decode_bytes(dw, kda=args.kda, mtp=args.mtp)
+    dgbs = dbytes / (dms / 1e3) / 1e9
+    rec = {"value": world * dgbs, "unit": "GB/s", "ms_per_step": dms, "steps": args.decode_steps,
+           "tokens_per_s": world * dw.num_seqs * max(1, args.mtp) / (dms / 1e3),
+           "workload": dw.name + (f"_mtp{args.mtp}" if args.mtp > 0 else ""),
+           "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": dgbs / peaks["hbm_gbs"],
+                        "traffic": kernel_traffic(f"gdn_decode/{dw.name}" + ("_kda" if args.kda else "")
+                                                  + (f"_mtp{args.mtp}" if args.mtp > 0 else "")),
+                        "kernel": "gdn_decode", "peak_source": f"{peak_src} HBM copy",
+                        "frac_vs_nominal_8000": dgbs / 8000.0, "bytes_per_launch": dbytes},
+           "gpu_launches": launches, "clocks": dclocks.summary(), "cuda_graph": not args.no_graph}
+    del graph, state, ring
+    torch.cuda.empty_cache()
+    return rec
 
-    # ---- end to end through the public API with host buffers ----
-    e2e = None
-    if not args.no_e2e and args.only != "decode":
-        pin = {k: v.pin_memory() for k, v in host.items() if v is not None}
-        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-        sf_host = torch.empty(sf.shape, dtype=sf.dtype).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in pin.values())
-        d2h = o_host.numel() * o_host.element_size() + sf_host.numel() * sf_host.element_size()
 
-        # Steps overlap across three streams, double-buffered: step i's inputs copy in while step i-1
-        # computes and step i-2's results copy out (separate copy engines for the two directions).
-        # Every step still copies its own inputs from pinned host memory and its own results back.
-        s_in, s_out, comp = torch.cuda.Stream(device), torch.cuda.Stream(device), stream
-        dbuf = [{k: torch.empty_like(v, device=device) for k, v in pin.items()} for _ in range(2)]
-        obuf, sbuf = [torch.empty_like(o) for _ in range(2)], [torch.empty_like(sf) for _ in range(2)]
-        ohost = [o_host] + [torch.empty(o.shape, dtype=o.dtype).pin_memory()]
-        shost = [sf_host] + [torch.empty(sf.shape, dtype=sf.dtype).pin_memory()]
-        ev_in, ev_comp, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
-        for b in range(2):
-            ev_comp[b].record(comp)
-            ev_out[b].record(comp)
-        it = [0]
+def run_ours(args):
+    import torch
+    rank, world, local_rank = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    from linear_attention_sequence_sm_b200 import inputs as I
 
-        def e2e_step():
-            b = it[0] % 2
-            it[0] += 1
-            x = dbuf[b]
-            s_in.wait_event(ev_comp[b])  # the step that last read these input buffers has run
-            with torch.cuda.stream(s_in):
-                for k_ in x:
-                    x[k_].copy_(pin[k_], non_blocking=True)
-            ev_in[b].record(s_in)
-            comp.wait_event(ev_in[b])
-            comp.wait_event(ev_out[b])  # the results last held in these output buffers have left
-            with torch.cuda.stream(comp):
-                fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], initial_state=x.get("initial_state"),
-                    cu_seqlens=x.get("cu_seqlens"), chunk_size=w.chunk, out=obuf[b], final_state=sbuf[b],
-                    workspace=ws, **flags, **out_norm(x))
-            ev_comp[b].record(comp)
-            s_out.wait_event(ev_comp[b])
-            with torch.cuda.stream(s_out):
-                ohost[b].copy_(obuf[b], non_blocking=True)
-                shost[b].copy_(sbuf[b], non_blocking=True)
-            ev_out[b].record(s_out)
+    peaks, peak_src = load_peaks()
+    makers = {"prefill": (I.prefill_bf16, 1002), "long": (I.long_bf16, 1003), "varlen": (I.varlen_bf16, 1005)}
+    mk, seed = makers[args.workload]
+    w = mk(seed=seed + rank)
+    host = I.make_raw_prefill_inputs(w) if args.raw_inputs else I.make_prefill_inputs(w)
 
-        def e2e_timed(n):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(comp)
-            s_in.wait_stream(comp)
-            for _ in range(n):
-                e2e_step()
-            comp.wait_stream(s_out)
-            e1.record(comp)
-            e1.synchronize()
-            return e0.elapsed_time(e1) / n
+    head = None
+    if args.only in ("all", "prefill"):
+        head = prefill_record(args, w, host, device, world, rank, peaks, peak_src)
+    del host
+    # the other two prefill workloads, each with its own record (plain forward only)
+    extra = {}
+    plain = not (args.kda or args.raw_inputs or args.output_norm or args.backward)
+    if args.only == "all" and args.workload == "prefill" and plain and not args.no_extra:
+        for name in ("long", "varlen"):
+            mk2, seed2 = makers[name]
+            w2 = mk2(seed=seed2 + rank)
+            extra[name] = prefill_record(args, w2, I.make_prefill_inputs(w2), device, world, rank, peaks, peak_src)
 
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize(device)
-        barrier(world, device)
-        e_ms = e2e_timed(max(3, min(args.steps, 20)))
-        e_ms = max_over_ranks(e_ms, device, world)
-        e2e = {"value": world * tokens / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
-               "overlap": "copy-in, compute and copy-out of consecutive steps on three streams, double-buffered"}
-
-    cpu = None
-    # (raw inputs or the output side: the timed oracle covers the plain path only; no CPU line then)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only != "decode" and not suffix:
-        cpu = cpu_oracle_sample(w, host, args.cpu_seconds)
+    decode = None
+    if args.only in ("all", "decode") and args.decode_steps > 0:
+        decode = decode_record(args, device, world, rank, peaks, peak_src)
 
     if rank == 0:
-        print(json.dumps({
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded splitmix64 / Box-Muller)",
-            "config": {"workload": w.name + suffix,
-                       "global_batch": w.num_seqs * world, "seq_len": w.seq_len,
-                       "heads_qk_v": [w.hk, w.hv], "head_dim": w.d, "chunk": w.chunk,
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": f"inputs larger than L2 ({prefill_bytes(w) / 1e6:.0f} MB of mandatory traffic per step)"},
-            "roofline": roofline, "decode": decode, "e2e": e2e, "cpu_baseline": cpu,
-            "gpu_launches": launches, "clocks": clocks.summary(),
-        }), flush=True)
+        ms_max = head["ms_per_step"] if head else float("nan")
+        line = {
+            "metric": METRIC, "value": head["tokens_per_s"] if head else None, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded splitmix64 / Box-Muller)",
+            "config": dict({"workload": head["workload"] if head else w.name,
+                            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                           **(head["config"] if head else {})),
+            "roofline": head["roofline"] if head else None, "decode": decode,
+            "e2e": head.get("e2e") if head else None, "cpu_baseline": head.get("cpu_baseline") if head else None,
+            "gpu_launches": head["gpu_launches"] if head else 0, "clocks": head["clocks"] if head else None,
+        }
+        line.update(extra)
+        print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

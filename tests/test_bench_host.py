@@ -81,6 +81,7 @@ def test_reference_arm_line():
     assert d["config"]["workload"] == "prefill_bf16_B4_T4096_hk16_hv32_d128_C64"
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert "whole workload" in cb["sample"] and cb["cpu_model"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert abs(d["ms_per_step"] - 1e3 * 4 * 4096 / d["value"]) <= 1e-6 * d["ms_per_step"]
 
@@ -139,3 +140,14 @@ def test_clock_sampler_against_a_fake_nvml(monkeypatch):
     with empty:
         pass
     assert empty.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+
+def test_cpu_baseline_times_the_whole_workload():
+    """The GPU arm's CPU baseline runs the same oracle pass as the reference
+    arm: the whole workload, no extrapolation; tokens/s = tokens / seconds per
+    pass."""
+    from linear_attention_sequence_sm_b200 import inputs as I
+    w = I.custom("cpu_base", batch=2, seq_len=256, hk=2, hv=4, d=32, chunk=64, dtype="bf16", seed=5)
+    cb = bench.cpu_baseline(w, I.make_prefill_inputs(w), target_s=0.0)
+    assert cb["kind"] == "oracle" and "not extrapolated" in cb["sample"] and "all 8" in cb["sample"]
+    assert cb["value"] == pytest.approx(w.total_tokens / cb["seconds_per_pass"])
