@@ -130,9 +130,15 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
 
 
-def _stream_handle(stream):
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return ctypes.c_void_p(s.cuda_stream)
+def _stream_handle(stream, dev):
+    """The stream a call enqueues on: ``stream``, or the current stream of the
+    tensors' device ``dev``.  A stream of another device is rejected: the
+    library would launch on it with pointers into ``dev``'s memory."""
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    elif stream.device != dev:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {dev}")
+    return ctypes.c_void_p(stream.cuda_stream)
 
 
 def _need(t, name, dtype=None, device=None):
@@ -285,14 +291,16 @@ def chunk_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_s
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     if output_norm is not None:
         osc = output_norm.c_struct(out)
-        _check(LIB.gdn_chunk_forward_out(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
-                                         _ptr(initial_state), _ptr(cu_seqlens), ctypes.byref(osc), _ptr(out),
-                                         _ptr(final_state), _ptr(workspace), workspace.numel(),
-                                         _stream_handle(stream)))
+        with torch.cuda.device(dev):  # the library launches on the current device
+            _check(LIB.gdn_chunk_forward_out(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                             _ptr(initial_state), _ptr(cu_seqlens), ctypes.byref(osc), _ptr(out),
+                                             _ptr(final_state), _ptr(workspace), workspace.numel(),
+                                             _stream_handle(stream, dev)))
         return out, final_state
-    _check(LIB.gdn_chunk_forward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
-                                 _ptr(initial_state), _ptr(cu_seqlens), _ptr(out), _ptr(final_state),
-                                 _ptr(workspace), workspace.numel(), _stream_handle(stream)))
+    with torch.cuda.device(dev):  # the library launches on the current device
+        _check(LIB.gdn_chunk_forward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                     _ptr(initial_state), _ptr(cu_seqlens), _ptr(out), _ptr(final_state),
+                                     _ptr(workspace), workspace.numel(), _stream_handle(stream, dev)))
     return out, final_state
 
 
@@ -323,9 +331,10 @@ def chunk_forward_noalloc(q, k, v, g, beta, initial_state=None, cu_seqlens=None,
         final_state = torch.empty((shape.num_seqs, shape.num_v_heads, shape.head_dim_v, shape.head_dim_k),
                                   dtype=torch.float32, device=dev)
     _need(final_state, "final_state", torch.float32, dev)
-    _check(LIB.gdn_chunk_forward_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
-                                         _ptr(initial_state), _ptr(cu_seqlens), _ptr(out), _ptr(final_state),
-                                         _stream_handle(stream)))
+    with torch.cuda.device(dev):  # the library launches on the current device
+        _check(LIB.gdn_chunk_forward_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                             _ptr(initial_state), _ptr(cu_seqlens), _ptr(out), _ptr(final_state),
+                                             _stream_handle(stream, dev)))
     return out, final_state
 
 
@@ -333,7 +342,9 @@ def read_device_status(workspace, stream=None) -> int:
     """Synchronise the stream and return the device status word of the last
     gdn_chunk_forward that used ``workspace``."""
     st = ctypes.c_int32(-1)
-    _check(LIB.gdn_read_device_status(_ptr(workspace), ctypes.byref(st), _stream_handle(stream)))
+    dev = workspace.device
+    with torch.cuda.device(dev):  # the library launches on the current device
+        _check(LIB.gdn_read_device_status(_ptr(workspace), ctypes.byref(st), _stream_handle(stream, dev)))
     return st.value
 
 
@@ -357,13 +368,15 @@ def decode_step(q, k, v, g, beta, state, out=None, stream=None, qk_l2norm=False,
     hv, dv = v.shape[1], v.shape[2]
     if output_norm is not None:
         osc = output_norm.c_struct(out)
-        _check(LIB.gdn_decode_step_out(N, hk, hv, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
-                                       _ptr(beta), _ptr(state), ctypes.byref(osc), _ptr(out),
-                                       input_flags(qk_l2norm, gate_logits), _stream_handle(stream)))
+        with torch.cuda.device(dev):  # the library launches on the current device
+            _check(LIB.gdn_decode_step_out(N, hk, hv, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                           _ptr(beta), _ptr(state), ctypes.byref(osc), _ptr(out),
+                                           input_flags(qk_l2norm, gate_logits), _stream_handle(stream, dev)))
         return out
-    _check(LIB.gdn_decode_step_ex(N, hk, hv, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
-                                  _ptr(beta), _ptr(state), _ptr(out), input_flags(qk_l2norm, gate_logits),
-                                  _stream_handle(stream)))
+    with torch.cuda.device(dev):  # the library launches on the current device
+        _check(LIB.gdn_decode_step_ex(N, hk, hv, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                      _ptr(beta), _ptr(state), _ptr(out), input_flags(qk_l2norm, gate_logits),
+                                      _stream_handle(stream, dev)))
     return out
 
 
@@ -397,10 +410,11 @@ def kda_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, output_fi
     if workspace is None or workspace.numel() < nbytes:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     osc = output_norm.c_struct(out) if output_norm is not None else None
-    _check(LIB.gdn_kda_forward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
-                               _ptr(initial_state), _ptr(cu_seqlens), None if osc is None else ctypes.byref(osc),
-                               _ptr(out), _ptr(final_state), _ptr(workspace), workspace.numel(),
-                               _stream_handle(stream)))
+    with torch.cuda.device(dev):  # the library launches on the current device
+        _check(LIB.gdn_kda_forward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                   _ptr(initial_state), _ptr(cu_seqlens), None if osc is None else ctypes.byref(osc),
+                                   _ptr(out), _ptr(final_state), _ptr(workspace), workspace.numel(),
+                                   _stream_handle(stream, dev)))
     return out, final_state
 
 
@@ -422,9 +436,10 @@ def kda_decode_step(q, k, v, g, beta, state, out=None, stream=None, qk_l2norm=Fa
         out = torch.empty(v.shape, dtype=dt, device=dev)
     _need(out, "out", dt, dev)
     osc = output_norm.c_struct(out) if output_norm is not None else None
-    _check(LIB.gdn_kda_decode_step(N, hk, hv, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
-                                   _ptr(beta), _ptr(state), None if osc is None else ctypes.byref(osc), _ptr(out),
-                                   input_flags(qk_l2norm, gate_logits), _stream_handle(stream)))
+    with torch.cuda.device(dev):  # the library launches on the current device
+        _check(LIB.gdn_kda_decode_step(N, hk, hv, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                       _ptr(beta), _ptr(state), None if osc is None else ctypes.byref(osc), _ptr(out),
+                                       input_flags(qk_l2norm, gate_logits), _stream_handle(stream, dev)))
     return out
 
 
@@ -459,9 +474,10 @@ def decode_multi(q, k, v, g, beta, state, out=None, snapshots=None, stream=None,
         snapshots = torch.empty((N, K, hv, dv, dk), dtype=torch.float32, device=dev)
     _need(out, "out", dt, dev)
     _need(snapshots, "snapshots", torch.float32, dev)
-    _check(LIB.gdn_decode_multi(N, K, hk, hv, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
-                                _ptr(beta), _ptr(state), _ptr(snapshots), _ptr(out),
-                                input_flags(qk_l2norm, gate_logits), _stream_handle(stream)))
+    with torch.cuda.device(dev):  # the library launches on the current device
+        _check(LIB.gdn_decode_multi(N, K, hk, hv, dk, dv, _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                    _ptr(beta), _ptr(state), _ptr(snapshots), _ptr(out),
+                                    input_flags(qk_l2norm, gate_logits), _stream_handle(stream, dev)))
     return out, snapshots
 
 
@@ -481,8 +497,9 @@ def decode_commit(snapshots, accepted, state, bad_count=None, stream=None):
     _need(state, "state", torch.float32, dev)
     _need(bad_count, "bad_count", torch.int32, dev)
     N, K, hv, dv, dk = snapshots.shape
-    _check(LIB.gdn_decode_commit(N, K, hv, dk, dv, _ptr(snapshots), _ptr(accepted), _ptr(state), _ptr(bad_count),
-                                 _stream_handle(stream)))
+    with torch.cuda.device(dev):  # the library launches on the current device
+        _check(LIB.gdn_decode_commit(N, K, hv, dk, dv, _ptr(snapshots), _ptr(accepted), _ptr(state), _ptr(bad_count),
+                                     _stream_handle(stream, dev)))
     return state
 
 
@@ -512,11 +529,12 @@ def chunk_backward(q, k, v, g, beta, d_o, d_final_state=None, initial_state=None
            "dg": torch.empty(g.shape, **f32), "dbeta": torch.empty(beta.shape, **f32),
            "d_initial_state": torch.empty((shape.num_seqs, shape.num_v_heads, shape.head_dim_v, shape.head_dim_k),
                                           **f32) if want_d_initial_state else None}
-    _check(LIB.gdn_chunk_backward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
-                                  _ptr(initial_state), _ptr(cu_seqlens), _ptr(d_o), _ptr(d_final_state),
-                                  _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]),
-                                  _ptr(out["dbeta"]), _ptr(out["d_initial_state"]), _ptr(workspace),
-                                  workspace.numel(), _stream_handle(stream)))
+    with torch.cuda.device(dev):  # the library launches on the current device
+        _check(LIB.gdn_chunk_backward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                      _ptr(initial_state), _ptr(cu_seqlens), _ptr(d_o), _ptr(d_final_state),
+                                      _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]),
+                                      _ptr(out["dbeta"]), _ptr(out["d_initial_state"]), _ptr(workspace),
+                                      workspace.numel(), _stream_handle(stream, dev)))
     return out
 
 

@@ -165,3 +165,16 @@ def test_multi_token_decode_and_commit_shapes():
         gdn.decode_commit(snaps, acc, torch.zeros(N, HV, DV, 64))
     with pytest.raises(ValueError, match="bad_count"):
         gdn.decode_commit(snaps, acc, st, bad_count=torch.zeros(0, dtype=torch.int32))
+
+
+def test_stream_of_another_device_is_rejected():
+    """The library launches on the stream it is given with pointers into the
+    tensors' device: a stream of another device is refused in the binding,
+    and without one the tensors' own device's current stream is used."""
+    import types
+    from linear_attention_sequence_sm_b200 import gdn
+    other = types.SimpleNamespace(device=torch.device("cuda", 1), cuda_stream=77)
+    with pytest.raises(ValueError, match="stream is on cuda:1"):
+        gdn._stream_handle(other, torch.device("cuda", 0))
+    same = types.SimpleNamespace(device=torch.device("cuda", 0), cuda_stream=1234)
+    assert gdn._stream_handle(same, torch.device("cuda", 0)).value == 1234
