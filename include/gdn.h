@@ -152,9 +152,10 @@ GDN_API gdn_status_t gdn_chunk_forward(const gdn_shape_t *shape,
  * every GPU that loads the library, held until the process exits, enough
  * for at most 16,384 sequences per call (more returns GDN_ERR_UNSUPPORTED
  * with a message; nothing is launched).  Arguments and results are those of
- * gdn_chunk_forward.  The first call on a device looks up the array's device
- * address once (cudaGetSymbolAddress, with that device current); make that
- * first call before any stream capture.  No call allocates or frees memory.
+ * gdn_chunk_forward.  Every call looks up the array's device address in the
+ * current device's context (cudaGetSymbolAddress, a host-side query); the
+ * first lookup in a context may load the library's device code, so make the
+ * first call on a device before any stream capture.  No call allocates or frees memory.
  * All calls on a device share the one array: calls that overlap on the GPU
  * (two streams, or two host threads) race on it and give wrong results, so
  * serialise them.  Each call re-initialises the scratch before use, so what

@@ -17,7 +17,6 @@
 // work counter before the prefill kernel reads them), so stale contents from
 // an earlier call do no harm.
 #include <cstdio>
-#include <mutex>
 
 #include "gdn_internal.cuh"
 
@@ -31,26 +30,19 @@ static_assert(kNoAllocScratchBytes % 256 == 0, "scratch size must keep 256-byte 
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch per device ordinal, resolved once per
-// device with that device current (the host-side symbol is only a stand-in
-// and must never be passed to a kernel).
-constexpr int kMaxDevices = 64;
-static void *g_scratch_ptr[kMaxDevices];
-static std::mutex g_scratch_mu;
-
+// Device address of g_noalloc_scratch in the current device's context,
+// looked up on every call with that device current.  The host-side symbol is
+// only a stand-in and must never be passed to a kernel; and an address kept
+// from an earlier call could belong to another context (after
+// cudaDeviceReset the module is loaded anew, and a caller's own driver-API
+// context holds its own instance of the module), so nothing is cached.  The
+// lookup is a host-side query (no synchronisation); the first one in a
+// context may load the library's device code.
 static cudaError_t scratch_address(void **out) {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    *out = p;
     return cudaSuccess;
 }
 

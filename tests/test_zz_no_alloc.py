@@ -5,19 +5,19 @@ Callers such as a plugin that its host runtime gives only tensor pointers
 request path, use this entry point: its scratch is a device array built into
 the library instead of a caller-allocated workspace.  This file checks,
 through the C ABI, that two calls in a row (the second finding the first
-call's leftovers in the shared array) give the same results as
-gdn_chunk_forward with a workspace, within the bf16 parity bar, and that a
-problem too large for the array is refused before any launch.  The file name
+call's leftovers in the shared array) give exactly the results of
+gdn_chunk_forward with a workspace (both run the same deterministic kernels
+on the same inputs), on the tensor-core path and on the fp32 CUDA-core path,
+each after a call with more sequences, and that a problem too large for the
+array is refused before any launch.  The file name
 makes pytest collect it last.
 """
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
 from linear_attention_sequence_sm_b200 import inputs as I
-from parity import BAR, prefill_errors, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -28,9 +28,9 @@ def _device_inputs(w):
     return inp, {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
 
 
-def _noalloc_call(gdn, d, chunk):
+def _noalloc_call(gdn, d, chunk, force_simt=False):
     """Call gdn_chunk_forward_noalloc directly through ctypes."""
-    shape = gdn.make_shape(d["q"], d["v"], d["cu_seqlens"], chunk)
+    shape = gdn.make_shape(d["q"], d["v"], d["cu_seqlens"], chunk, force_simt)
     o = torch.full_like(d["v"], float("nan"))
     sf = torch.full((shape.num_seqs, shape.num_v_heads, shape.head_dim_v, shape.head_dim_k), float("nan"),
                     dtype=torch.float32, device=d["q"].device)
@@ -44,19 +44,24 @@ def _noalloc_call(gdn, d, chunk):
 
 def test_noalloc_matches_workspace_entry_point_twice():
     from linear_attention_sequence_sm_b200 import gdn
-    workloads = [
-        I.custom("noalloc_varlen", 1, 0, 2, 4, 128, 64, "bf16", seed=61, s0_std=0.02,
-                 seq_lens=[130, 1, 64, 0, 257, 33]),
-        I.custom("noalloc_batched", batch=3, seq_len=200, hk=2, hv=4, d=128, chunk=64, dtype="bf16", seed=62),
+    # (workload, force the fp32 CUDA-core kernel); each call after the first
+    # finds fewer sequences than the call before left in the shared array
+    cases = [
+        (I.custom("noalloc_varlen", 1, 0, 2, 4, 128, 64, "bf16", seed=61, s0_std=0.02,
+                  seq_lens=[130, 1, 64, 0, 257, 33]), False),
+        (I.custom("noalloc_batched", batch=3, seq_len=200, hk=2, hv=4, d=128, chunk=64, dtype="bf16", seed=62),
+         False),
+        (I.custom("noalloc_fp32_d16", batch=2, seq_len=90, hk=2, hv=2, d=16, chunk=16, dtype="f32", seed=63,
+                  s0_std=0.05), False),
+        (I.custom("noalloc_simt", 1, 0, 1, 3, 128, 64, "bf16", seed=64, s0_std=0.02, seq_lens=[65, 2]), True),
     ]
-    for w in workloads:  # two calls in a row on the shared scratch array
+    for w, simt in cases:  # calls in a row on the shared scratch array
         inp, d = _device_inputs(w)
-        o_na, sf_na = _noalloc_call(gdn, d, w.chunk)
+        o_na, sf_na = _noalloc_call(gdn, d, w.chunk, force_simt=simt)
         o_ws, sf_ws = gdn.chunk_forward(d["q"], d["k"], d["v"], d["g"], d["beta"], initial_state=d["initial_state"],
-                                        cu_seqlens=d["cu_seqlens"], chunk_size=w.chunk)
+                                        cu_seqlens=d["cu_seqlens"], chunk_size=w.chunk, force_simt=simt)
         torch.cuda.synchronize()
-        eo, es = prefill_errors(inp, o_na, sf_na, to_f64(o_ws), to_f64(sf_ws))
-        assert eo <= BAR["bf16"] and es <= BAR["bf16"], (w.name, eo, es)
+        assert torch.equal(o_na, o_ws) and torch.equal(sf_na, sf_ws), w.name
         assert torch.isfinite(o_na.float()).all() and torch.isfinite(sf_na).all()
 
 
