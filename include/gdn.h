@@ -85,6 +85,15 @@ typedef enum { GDN_DTYPE_F32 = 0, GDN_DTYPE_BF16 = 1 } gdn_dtype_t;
                                     write logit b: alpha = sigmoid(a), i.e.
                                     the log-decay is log sigmoid(a), and the
                                     write strength is sigmoid(b)            */
+/* The bf16 tensor-core prefill (d_k = d_v = 128, C = 64) normally runs as two
+ * kernels: the chunks' triangular WY factors T = (I + A)^-1 for all chunks at
+ * once (they do not depend on the state), kept in the workspace, then the
+ * state-carrying chunk loop that reads them.  This flag runs it as a single
+ * kernel that inverts each chunk's factor in place, one chunk ahead of the
+ * state; its workspace holds only the schedule tables (a few bytes per
+ * sequence) instead of 8 KiB per (chunk, value head), and it needs the value
+ * heads in multiples of 4.  The results agree within rounding.             */
+#define GDN_FLAG_ONE_KERNEL 8u
 
 /* Shape of a prefill problem.
  *   batch, seq_len  without cu_seqlens: B sequences of T tokens each
@@ -108,7 +117,11 @@ typedef struct {
 } gdn_shape_t;
 
 /* Bytes of device workspace gdn_chunk_forward needs for `shape` (a pure
- * function of the shape; the caller allocates it, 256-byte aligned). */
+ * function of the shape; the caller allocates it, 256-byte aligned).  For
+ * the two-kernel tensor-core path this includes 8 KiB per (chunk, value
+ * head) for the chunk factors: at most ((tokens + 63 N) / 64) Hv tiles.  A
+ * workspace below this size but at least the size queried with
+ * GDN_FLAG_ONE_KERNEL set runs the single-kernel path instead. */
 GDN_API gdn_status_t gdn_chunk_forward_workspace_size(const gdn_shape_t *shape, size_t *bytes);
 
 /* Chunkwise prefill ("Gated Attention Architectures", sections 2 and 3: the
@@ -152,7 +165,8 @@ GDN_API gdn_status_t gdn_chunk_forward(const gdn_shape_t *shape,
  * every GPU that loads the library, held until the process exits, enough
  * for at most 16,384 sequences per call (more returns GDN_ERR_UNSUPPORTED
  * with a message; nothing is launched).  Arguments and results are those of
- * gdn_chunk_forward.  Every call looks up the array's device address in the
+ * gdn_chunk_forward with GDN_FLAG_ONE_KERNEL set (the scratch holds no chunk
+ * factors).  Every call looks up the array's device address in the
  * current device's context (cudaGetSymbolAddress, a host-side query); the
  * first lookup in a context may load the library's device code, so make the
  * first call on a device before any stream capture.  No call allocates or frees memory.
@@ -360,6 +374,41 @@ GDN_API gdn_status_t gdn_chunk_backward(const gdn_shape_t *shape,
                                 float *d_initial_state,
                                 void *workspace, size_t workspace_bytes,
                                 void *stream);
+
+/* The input side's short causal convolution, with an optional SiLU after it
+ * ("Architecture Thread I", "Modern Architecture Improvements": after the
+ * projections, q and k pass through a short convolution, SiLU and L2
+ * normalisation -- the last step is GDN_FLAG_QK_L2NORM of the mixer calls --
+ * and v through a short convolution and SiLU).  Causal and depthwise, one
+ * filter of W taps per channel:
+ *     y[t, c] = act( sum_{j<W} weight[c, j] x[t - (W-1) + j, c] ),
+ * the last tap on the current token; act = SiLU with GDN_CONV_SILU, else the
+ * identity.  Inputs before a sequence's first token come from the
+ * sequence's conv state, its W-1 preceding inputs oldest first (zeros when
+ * state_in is NULL); a sequence never reads another's tokens.
+ *   num_seqs, seq_len, cu_seqlens
+ *                   N sequences: without cu_seqlens, of seq_len tokens each
+ *                   (tokens = N * seq_len); with cu_seqlens ([N + 1] int32
+ *                   device array of sequence starts, as for
+ *                   gdn_chunk_forward; seq_len ignored), packed.  Its
+ *                   contents are not checked: contents that break its
+ *                   contract give unspecified values, never an access out
+ *                   of bounds.
+ *   x, y            [tokens, channels] of `dtype` (q, k or v as [tokens,
+ *                   H, d] with channels = H * d); y must not overlap x.
+ *   weight          [channels, W] fp32.
+ *   state_in        [N, channels, W-1] fp32, or NULL for zeros.
+ *   state_out       [N, channels, W-1] fp32, or NULL: each sequence's last
+ *                   W-1 inputs (reaching into state_in when the sequence is
+ *                   shorter), for decode to continue from; must not overlap
+ *                   state_in.
+ * 1 <= W <= 8; channels a multiple of 4.  HBM-bound: one read of x and one
+ * write of y. */
+#define GDN_CONV_SILU 1u
+GDN_API gdn_status_t gdn_short_conv(int32_t num_seqs, int32_t seq_len, const int32_t *cu_seqlens, int64_t tokens,
+                                    int32_t channels, int32_t width, int32_t dtype, const void *x,
+                                    const float *weight, const float *state_in, float *state_out, void *y,
+                                    uint32_t flags, void *stream);
 
 /* Static text for a status code. */
 GDN_API const char *gdn_status_string(gdn_status_t status);

@@ -54,7 +54,7 @@ static gdn_status_t check_shape(const gdn_shape_t *s) {
                     s->num_v_heads, s->num_qk_heads);
     if (s->dtype != GDN_DTYPE_F32 && s->dtype != GDN_DTYPE_BF16)
         return fail(GDN_ERR_INVALID_ARGUMENT, "dtype %d is not GDN_DTYPE_F32 or GDN_DTYPE_BF16", s->dtype);
-    if (s->flags & ~(GDN_FLAG_FORCE_SIMT | GDN_FLAG_QK_L2NORM | GDN_FLAG_GATE_LOGITS))
+    if (s->flags & ~(GDN_FLAG_FORCE_SIMT | GDN_FLAG_QK_L2NORM | GDN_FLAG_GATE_LOGITS | GDN_FLAG_ONE_KERNEL))
         return fail(GDN_ERR_INVALID_ARGUMENT, "unknown flag bits 0x%x", s->flags);
     if (s->chunk_size != 16 && s->chunk_size != 32 && s->chunk_size != 64)
         return fail(GDN_ERR_UNSUPPORTED, "chunk_size %d not in {16, 32, 64}", s->chunk_size);
@@ -127,7 +127,8 @@ gdn_status_t gdn_chunk_forward_workspace_size(const gdn_shape_t *s, size_t *byte
     if (!bytes) return fail(GDN_ERR_INVALID_ARGUMENT, "bytes is NULL");
     gdn_status_t st = check_shape(s);
     if (st != GDN_OK) return st;
-    *bytes = ws_layout(s->num_seqs).total;
+    const bool split = chunk_split_supported(*s) && !(s->flags & (GDN_FLAG_ONE_KERNEL | GDN_FLAG_FORCE_SIMT));
+    *bytes = split ? split_layout(*s).total : ws_layout(s->num_seqs).total;
     return GDN_OK;
 }
 
@@ -196,8 +197,7 @@ static gdn_status_t chunk_forward_impl(const gdn_shape_t *s, const void *q, cons
     if (sms <= 0) return fail(GDN_ERR_CUDA, "no usable CUDA device");
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
 
-    cudaError_t e = launch_schedule(*s, cu_seqlens, workspace, stream);
-    if (e != cudaSuccess) return cuda_fail(e, "schedule kernel launch");
+    cudaError_t e = cudaSuccess;
 
     PrefillArgs a;
     a.num_seqs = s->num_seqs;
@@ -216,9 +216,15 @@ static gdn_status_t chunk_forward_impl(const gdn_shape_t *s, const void *q, cons
     a.sched.order = reinterpret_cast<const int32_t *>(ws + L.order_off);
     a.sched.start = reinterpret_cast<const int32_t *>(ws + L.start_off);
     a.sched.len = reinterpret_cast<const int32_t *>(ws + L.len_off);
-    if (s->num_seqs == 0) return GDN_OK;
+    a.sched.chunk_base = nullptr;
+    if (s->num_seqs == 0) {  // nothing to compute; the status word still reads GDN_OK
+        e = launch_schedule(*s, cu_seqlens, workspace, stream);
+        return e == cudaSuccess ? GDN_OK : cuda_fail(e, "schedule kernel launch");
+    }
 
     if (kda) {
+        e = launch_schedule(*s, cu_seqlens, workspace, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "schedule kernel launch");
         e = launch_kda_prefill(a, stream);
         if (e != cudaSuccess) return cuda_fail(e, "KDA prefill launch");
         if (out.flags) {
@@ -227,7 +233,28 @@ static gdn_status_t chunk_forward_impl(const gdn_shape_t *s, const void *q, cons
         }
         return GDN_OK;
     }
-    const bool use_tc = major == 10 && !(s->flags & GDN_FLAG_FORCE_SIMT) && chunk_tc_supported(*s);
+    const bool tc_arch = major == 10 && !(s->flags & GDN_FLAG_FORCE_SIMT);
+    // The two-kernel tensor-core path needs the full queried workspace (it keeps
+    // every chunk's inverse there); with less, or with the output side, the
+    // single-kernel tensor-core path runs where it applies.
+    const bool use_split = tc_arch && tokens > 0 && !out.flags && !(s->flags & GDN_FLAG_ONE_KERNEL) &&
+                           chunk_split_supported(*s) && workspace_bytes >= split_layout(*s).total;
+    const bool use_tc = !use_split && tc_arch && chunk_tc_supported(*s);
+    if (use_split) {
+        const SplitLayout SL = split_layout(*s);
+        int32_t *cbase = reinterpret_cast<int32_t *>(ws + SL.cbase_off);
+        __nv_bfloat16 *tinv = reinterpret_cast<__nv_bfloat16 *>(ws + SL.tinv_off);
+        e = launch_schedule(*s, cu_seqlens, workspace, stream, cbase);
+        if (e != cudaSuccess) return cuda_fail(e, "schedule kernel launch");
+        a.sched.chunk_base = cbase;
+        e = launch_chunk_inverse(a, tinv, SL.max_chunks, stream, sms);
+        if (e != cudaSuccess) return cuda_fail(e, "chunk inverse launch");
+        e = launch_chunk_chain(a, tinv, SL.max_chunks, stream, sms);
+        if (e != cudaSuccess) return cuda_fail(e, "tensor-core chunk loop launch");
+        return GDN_OK;
+    }
+    e = launch_schedule(*s, cu_seqlens, workspace, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "schedule kernel launch");
     e = use_tc ? launch_chunk_tc(a, stream, sms) : launch_chunk_simt(a, stream, sms);
     if (e != cudaSuccess) return cuda_fail(e, use_tc ? "tensor-core prefill launch" : "prefill launch");
     // the tensor-core kernel applies the output side itself (with tokens to load)
@@ -447,6 +474,7 @@ gdn_status_t gdn_chunk_backward(const gdn_shape_t *s, const void *q, const void 
     a.sched.order = reinterpret_cast<const int32_t *>(ws + L.order_off);
     a.sched.start = reinterpret_cast<const int32_t *>(ws + L.start_off);
     a.sched.len = reinterpret_cast<const int32_t *>(ws + L.len_off);
+    a.sched.chunk_base = nullptr;
     if (s->num_seqs == 0) return GDN_OK;
     float *ckpt = reinterpret_cast<float *>(ws + bwd_sched_bytes(s));
     e = launch_chunk_backward(a, d_o, d_final_state, dq, dk, dv, dg, dbeta, d_initial_state, ckpt, stream);
@@ -456,3 +484,42 @@ gdn_status_t gdn_chunk_backward(const gdn_shape_t *s, const void *q, const void 
 
 }  // extern "C"
 
+extern "C" {
+
+gdn_status_t gdn_short_conv(int32_t num_seqs, int32_t seq_len, const int32_t *cu_seqlens, int64_t tokens,
+                            int32_t channels, int32_t width, int32_t dtype, const void *x, const float *weight,
+                            const float *state_in, float *state_out, void *y, uint32_t flags, void *stream_) {
+    g_msg[0] = 0;
+    if (flags & ~GDN_CONV_SILU) return fail(GDN_ERR_INVALID_ARGUMENT, "unknown convolution flag bits 0x%x", flags);
+    if (num_seqs < 0 || tokens < 0 || channels <= 0)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "bad convolution shape");
+    if (dtype != GDN_DTYPE_F32 && dtype != GDN_DTYPE_BF16)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "dtype %d is not GDN_DTYPE_F32 or GDN_DTYPE_BF16", dtype);
+    if (width < 1 || width > 8) return fail(GDN_ERR_UNSUPPORTED, "convolution width %d not in 1..8", width);
+    if (channels % 4 != 0) return fail(GDN_ERR_UNSUPPORTED, "channels (%d) must be a multiple of 4", channels);
+    if (int64_t(channels) / 4 > int64_t(65535) * 128)
+        return fail(GDN_ERR_UNSUPPORTED, "too many channels (%d)", channels);
+    if (tokens > INT32_MAX) return fail(GDN_ERR_UNSUPPORTED, "more than 2^31-1 tokens");
+    if (!cu_seqlens && int64_t(num_seqs) * seq_len != tokens)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "tokens (%lld) must equal num_seqs * seq_len without cu_seqlens",
+                    (long long)tokens);
+    if (num_seqs == 0 && tokens > 0) return fail(GDN_ERR_INVALID_ARGUMENT, "tokens without sequences");
+    if (num_seqs == 0) return GDN_OK;
+    if (!weight || (tokens > 0 && (!x || !y)))
+        return fail(GDN_ERR_INVALID_ARGUMENT, "x, weight and y must be non-NULL");
+    if (tokens > 0 && x == y) return fail(GDN_ERR_INVALID_ARGUMENT, "y must not alias x");
+    if (width > 1 && state_in && state_in == state_out)
+        return fail(GDN_ERR_INVALID_ARGUMENT, "state_out must not alias state_in");
+    const void *ptrs[] = {x, weight, state_in, state_out, y, cu_seqlens};
+    const char *names[] = {"x", "weight", "state_in", "state_out", "y", "cu_seqlens"};
+    for (int i = 0; i < 6; ++i)
+        if (ptrs[i] && !aligned16(ptrs[i])) return fail(GDN_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+    if (device_sm_count(nullptr) <= 0) return fail(GDN_ERR_CUDA, "no usable CUDA device");
+    cudaError_t e = launch_short_conv(num_seqs, seq_len, cu_seqlens, int32_t(tokens), channels, width, dtype, x,
+                                      weight, state_in, state_out, y, (flags & GDN_CONV_SILU) != 0,
+                                      static_cast<cudaStream_t>(stream_));
+    if (e != cudaSuccess) return cuda_fail(e, "short convolution launch");
+    return GDN_OK;
+}
+
+}  // extern "C"

@@ -140,62 +140,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kBytesKQ = 4 * 8192 + 2 * 1024;  // four 64 x 64 bf16 boxes and two 64 x 4 fp32 gate boxes
 constexpr uint32_t kBytesV = 2 * 8192;
 
-__device__ __forceinline__ void named_sync(int id, int count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
-// Barrier over one warp group that also ORs a predicate across it.
-__device__ __forceinline__ bool named_sync_or(int id, int count, bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"(uint32_t(pred)), "r"(id), "r"(count)
-        : "memory");
-    return r != 0;
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void store_row_bf16(uint32_t tile, int row, int chunk0, const float *x, int nchunks) {
-#pragma unroll
-    for (int c = 0; c < nchunks; ++c) st_shared_v4(tile + sw128_offset(row, chunk0 + c), pack_bf16x8(x + 8 * c));
-}
-
-__device__ __forceinline__ void load4(const float *p, float *x) {
-    const float4 t = *reinterpret_cast<const float4 *>(p);
-    x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
-}
-
-// c += X[0:16, 0:8nk] Z[0:8nk, n0:n0+8] for row-major fp32 blocks X (stride
-// ldx, rows from its first row) and Z (stride ldz), one warp, tf32 inputs.
-__device__ __forceinline__ void tile_mma(float (&c)[4], const float *X, int ldx, const float *Z, int ldz, int n0,
-                                         int nk, int lane) {
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-        if (s >= nk) break;
-        const int k = 8 * s;
-        const uint32_t av[4] = {to_tf32(X[g * ldx + k + t]), to_tf32(X[(g + 8) * ldx + k + t]),
-                                to_tf32(X[g * ldx + k + t + 4]), to_tf32(X[(g + 8) * ldx + k + t + 4])};
-        const uint32_t bv[2] = {to_tf32(Z[(k + t) * ldz + n0 + g]), to_tf32(Z[(k + t + 4) * ldz + n0 + g])};
-        mma_tf32_16x8x8(c, av, bv);
-    }
-}
-
-// D[m0.., n0..] (16 x 8 tile) = sgn * c.
-__device__ __forceinline__ void tile_store(float *D, int ldd, int m0, int n0, const float (&c)[4], float sgn,
-                                           int lane) {
-    const int g = lane >> 2, t = lane & 3;
-    *reinterpret_cast<float2 *>(D + (m0 + g) * ldd + n0 + 2 * t) = make_float2(sgn * c[0], sgn * c[1]);
-    *reinterpret_cast<float2 *>(D + (m0 + g + 8) * ldd + n0 + 2 * t) = make_float2(sgn * c[2], sgn * c[3]);
-}
-
 // T' = T diag(beta gamma) and T'' = T diag(beta) entries (R, C), (R, C + 1) as
 // bf16 pairs in the 128-byte-swizzled 64 x 64 operand tiles at tp and tpp.
 __device__ __forceinline__ void st_tt_pair(uint32_t tp, uint32_t tpp, int R, int C, float v0, float v1,
@@ -950,54 +894,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
-}
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
-// [tokens, heads, 128] bf16 viewed as a 3-D tensor (d fastest), boxes of
-// 64 (d) x 1 (head) x 64 (tokens), 128-byte swizzle; rows past the last token
-// read as zeros.
-// [tokens, heads] fp32 gates viewed as 2-D, boxes of 4 heads x 64 tokens (the
-// inner box must span at least 16 bytes; the kernel picks its head's column).
-bool make_gate_map(CUtensorMap *map, const float *base, int heads, int tokens) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    const cuuint64_t dims[2] = {cuuint64_t(heads), cuuint64_t(tokens)};
-    const cuuint64_t strides[1] = {cuuint64_t(heads) * 4};
-    const cuuint32_t box[2] = {4, 64};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// With `out` set: boxes of 128 (d) x 1 x 64 tokens, no swizzle -- the
-// token-major output tile staged in shared memory.
-bool make_map(CUtensorMap *map, const void *base, int heads, int tokens, bool out = false) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    const cuuint64_t dims[3] = {128, cuuint64_t(heads), cuuint64_t(tokens)};
-    const cuuint64_t strides[2] = {128 * 2, cuuint64_t(heads) * 128 * 2};
-    const cuuint32_t box[3] = {out ? 128u : 64u, 1, 64};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, out ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace

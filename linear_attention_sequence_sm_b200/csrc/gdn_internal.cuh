@@ -2,6 +2,7 @@
 // libgdn.so (host launch layer and kernels).  Not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -42,7 +43,8 @@ struct WsHeader {
     int32_t bad_index;     // first offending cu_seqlens index (diagnostics)
     uint32_t next_unit;    // work counter of the persistent prefill kernels
     int32_t num_seqs;
-    int32_t pad[60];
+    int32_t total_chunks;  // chunks of all sequences (the two-kernel path: chunk_base filled)
+    int32_t pad[59];
 };
 static_assert(sizeof(WsHeader) == 256, "header must be 256 bytes");
 
@@ -62,12 +64,47 @@ inline WsLayout ws_layout(int32_t num_seqs) {
     return L;
 }
 
+// The two-kernel tensor-core path appends to the schedule tables
+//   chunk_base [N + 1]    first chunk of each sequence in the chunk order
+//                         (sequence by sequence, chunks in token order);
+//                         chunk_base[N] = total chunks
+//   tinv                  per (chunk, value head) the 64 x 64 bf16 inverse T
+//                         of the chunk's WY representation, row-major,
+//                         [max_chunks][Hv][64][64]
+// max_chunks bounds the chunk count for the shape: (tokens + 63 N) / 64 (each
+// sequence adds at most one partial chunk).
+struct SplitLayout {
+    WsLayout sched;
+    size_t cbase_off, tinv_off, total;
+    int64_t max_chunks;
+};
+
+inline int64_t max_chunks_bound(const gdn_shape_t &s) {
+    // sum over sequences of ceil(L_n / 64) <= (sum L_n + 63 N) / 64 (also
+    // covers the batched layout: B ceil(T / 64) <= (B T + 63 B) / 64)
+    return (int64_t(s.batch) * s.seq_len + 63 * int64_t(s.num_seqs)) / 64;
+}
+
+inline SplitLayout split_layout(const gdn_shape_t &s) {
+    SplitLayout L;
+    L.sched = ws_layout(s.num_seqs);
+    size_t off = L.sched.total;
+    L.cbase_off = off; off = align256(off + 4 * (size_t(s.num_seqs) + 1));
+    off = (off + 1023) & ~size_t(1023);
+    L.tinv_off = off;
+    L.max_chunks = max_chunks_bound(s);
+    off += size_t(L.max_chunks) * size_t(s.num_v_heads) * 64 * 64 * 2;
+    L.total = align256(off);
+    return L;
+}
+
 // Pointers into the workspace, as the kernels see them.
 struct Sched {
     WsHeader *hdr;
     const int32_t *order;
     const int32_t *start;
     const int32_t *len;
+    const int32_t *chunk_base;  // two-kernel path only (else NULL)
 };
 
 // Element access for the two storage types.
@@ -87,9 +124,10 @@ gdn_status_t set_error(gdn_status_t st, const char *text);
 void count_launch();
 
 // Prefill schedule: validates cu_seqlens (or synthesises the batched layout)
-// and fills the workspace tables.  One block.
+// and fills the workspace tables (with chunk_base when it is not NULL).  One
+// block.
 cudaError_t launch_schedule(const gdn_shape_t &s, const int32_t *cu_seqlens, void *workspace,
-                            cudaStream_t stream);
+                            cudaStream_t stream, int32_t *chunk_base = nullptr);
 
 // Column sums over a warp of 16 values per lane, transposed: afterwards lanes
 // 2t and 2t + 1 return the sum over all 32 lanes of x[t] (t = 0..15).  Four
@@ -162,9 +200,27 @@ struct PrefillArgs {
 // fp32 CUDA-core chunkwise kernel (any dtype, d_k, d_v <= 128, C in {16,32,64}).
 cudaError_t launch_chunk_simt(const PrefillArgs &a, cudaStream_t stream, int num_sms);
 
-// Tensor-core chunkwise kernel (bf16, d = 128, C = 64).
+// Tensor maps (gdn_tma.cu): gates [tokens, heads] fp32 in boxes of 4 heads x
+// 64 tokens; [tokens, heads, 128] bf16 in boxes of 64 x 1 x 64, 128-byte
+// swizzle (out: 128 x 1 x 64, no swizzle); rows x 64 bf16 tiles of 64 rows,
+// 128-byte swizzle.
+bool make_gate_map(CUtensorMap *map, const float *base, int heads, int tokens);
+bool make_map(CUtensorMap *map, const void *base, int heads, int tokens, bool out = false);
+bool make_tile_map(CUtensorMap *map, const void *base, int64_t rows);
+
+// Tensor-core chunkwise kernel (bf16, d = 128, C = 64) as one kernel.
 cudaError_t launch_chunk_tc(const PrefillArgs &a, cudaStream_t stream, int num_sms);
 bool chunk_tc_supported(const gdn_shape_t &s);
+
+// The two-kernel tensor-core path (bf16, d = 128, C = 64, any head counts):
+// the chunk inverses T for all chunks (gdn_chunk_inv.cu), then the
+// state-carrying chunk loop that reads them (gdn_chunk_chain.cu).  Both are
+// programmatic dependents of the schedule kernel, which fills chunk_base.
+bool chunk_split_supported(const gdn_shape_t &s);
+cudaError_t launch_chunk_inverse(const PrefillArgs &a, __nv_bfloat16 *tinv, int64_t max_chunks, cudaStream_t stream,
+                                 int num_sms);
+cudaError_t launch_chunk_chain(const PrefillArgs &a, const __nv_bfloat16 *tinv, int64_t max_chunks,
+                               cudaStream_t stream, int num_sms);
 
 // The output side as its own pass over o, in place (for the CUDA-core prefill,
 // whose blocks each own a slice of d_v).
@@ -184,6 +240,11 @@ cudaError_t launch_decode_multi(int32_t n, int32_t ntok, int32_t hk, int32_t hv,
                                 cudaStream_t stream);
 cudaError_t launch_decode_commit(int32_t n, int32_t ntok, int32_t hv, int32_t dk, int32_t dv, const float *snap,
                                  const int32_t *accepted, float *state, int32_t *bad, cudaStream_t stream);
+
+// The input side's short causal convolution (+ SiLU) and its conv states.
+cudaError_t launch_short_conv(int32_t n, int32_t seq_len, const int32_t *cu, int32_t tokens, int32_t channels,
+                              int32_t width, int32_t dtype, const void *x, const float *w, const float *state_in,
+                              float *state_out, void *y, bool silu, cudaStream_t stream);
 
 // Backward (training): checkpoint bytes and the kernel.
 size_t backward_ckpt_bytes(int32_t tokens, int32_t num_seqs, int32_t hv, int32_t dk, int32_t dv);

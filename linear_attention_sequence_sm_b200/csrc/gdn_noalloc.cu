@@ -69,6 +69,11 @@ extern "C" GDN_API gdn_status_t gdn_chunk_forward_noalloc(const gdn_shape_t *sha
                  cudaGetErrorString(e));
         return set_error(GDN_ERR_CUDA, msg);
     }
-    return gdn_chunk_forward(shape, q, k, v, g, beta, initial_state, cu_seqlens, o, final_state, scratch,
+    // the single-kernel path: its scratch is the schedule tables alone
+    if (!shape) return gdn_chunk_forward(shape, q, k, v, g, beta, initial_state, cu_seqlens, o, final_state,
+                                         scratch, kNoAllocScratchBytes, stream);
+    gdn_shape_t one = *shape;
+    one.flags |= GDN_FLAG_ONE_KERNEL;
+    return gdn_chunk_forward(&one, q, k, v, g, beta, initial_state, cu_seqlens, o, final_state, scratch,
                              kNoAllocScratchBytes, stream);
 }

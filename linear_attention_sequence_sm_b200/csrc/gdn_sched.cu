@@ -12,8 +12,9 @@ constexpr int kMaxRankedSeqs = 8192;
 
 __global__ void __launch_bounds__(kSchedThreads)
 schedule_kernel(int32_t num_seqs, int32_t tokens, int32_t batched_len, const int32_t *__restrict__ cu,
-                WsHeader *hdr, int32_t *order, int32_t *start, int32_t *len) {
+                WsHeader *hdr, int32_t *order, int32_t *start, int32_t *len, int32_t *chunk_base) {
     __shared__ int bad;
+    __shared__ int part[kSchedThreads];
     // the prefill kernel that follows may start its own set-up now; it waits for
     // this kernel's results (griddepcontrol.wait) before reading them
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -23,6 +24,7 @@ schedule_kernel(int32_t num_seqs, int32_t tokens, int32_t batched_len, const int
         hdr->bad_index = -1;
         hdr->next_unit = 0;
         hdr->num_seqs = num_seqs;
+        hdr->total_chunks = 0;
     }
     __syncthreads();
     for (int n = threadIdx.x; n < num_seqs; n += blockDim.x) {
@@ -48,6 +50,32 @@ schedule_kernel(int32_t num_seqs, int32_t tokens, int32_t batched_len, const int
         }
         return;
     }
+    if (chunk_base) {
+        // chunk_base = exclusive prefix sums of ceil(L_n / 64): each thread sums a
+        // contiguous run of sequences, the block scans the run totals, and each
+        // thread then writes its run's prefixes
+        const int per = (num_seqs + kSchedThreads - 1) / kSchedThreads;
+        const int n0 = min(num_seqs, int(threadIdx.x) * per), n1 = min(num_seqs, n0 + per);
+        int local = 0;
+        for (int n = n0; n < n1; ++n) local += (len[n] + 63) / 64;
+        part[threadIdx.x] = local;
+        __syncthreads();
+        for (int d = 1; d < kSchedThreads; d <<= 1) {  // inclusive Hillis-Steele scan
+            const int add = threadIdx.x >= unsigned(d) ? part[threadIdx.x - d] : 0;
+            __syncthreads();
+            part[threadIdx.x] += add;
+            __syncthreads();
+        }
+        int run = part[threadIdx.x] - local;
+        for (int n = n0; n < n1; ++n) {
+            chunk_base[n] = run;
+            run += (len[n] + 63) / 64;
+        }
+        if (threadIdx.x == kSchedThreads - 1) {
+            chunk_base[num_seqs] = part[kSchedThreads - 1];
+            hdr->total_chunks = part[kSchedThreads - 1];
+        }
+    }
     // longest first, ties by index: rank(n) = #{m : L_m > L_n or (L_m == L_n and m < n)}
     const bool rank_it = cu != nullptr && num_seqs <= kMaxRankedSeqs;
     for (int n = threadIdx.x; n < num_seqs; n += blockDim.x) {
@@ -66,14 +94,14 @@ schedule_kernel(int32_t num_seqs, int32_t tokens, int32_t batched_len, const int
 }
 
 cudaError_t launch_schedule(const gdn_shape_t &s, const int32_t *cu_seqlens, void *workspace,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, int32_t *chunk_base) {
     const WsLayout L = ws_layout(s.num_seqs);
     char *ws = static_cast<char *>(workspace);
     const int32_t tokens = s.batch * s.seq_len;
     schedule_kernel<<<1, kSchedThreads, 0, stream>>>(
         s.num_seqs, tokens, cu_seqlens ? 0 : s.seq_len, cu_seqlens, reinterpret_cast<WsHeader *>(ws),
         reinterpret_cast<int32_t *>(ws + L.order_off), reinterpret_cast<int32_t *>(ws + L.start_off),
-        reinterpret_cast<int32_t *>(ws + L.len_off));
+        reinterpret_cast<int32_t *>(ws + L.len_off), chunk_base);
     count_launch();
     return cudaGetLastError();
 }

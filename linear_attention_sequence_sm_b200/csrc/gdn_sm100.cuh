@@ -316,5 +316,65 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
                  : "memory");
 }
 
+// ---------------------------------------------------------------------------
+// Group barriers, small register/shared-memory helpers and warp-level tf32
+// products shared by the tensor-core prefill kernels.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void named_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Barrier over one warp group that also ORs a predicate across it.
+__device__ __forceinline__ bool named_sync_or(int id, int count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(uint32_t(pred)), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void store_row_bf16(uint32_t tile, int row, int chunk0, const float *x, int nchunks) {
+#pragma unroll
+    for (int c = 0; c < nchunks; ++c) st_shared_v4(tile + sw128_offset(row, chunk0 + c), pack_bf16x8(x + 8 * c));
+}
+
+__device__ __forceinline__ void load4(const float *p, float *x) {
+    const float4 t = *reinterpret_cast<const float4 *>(p);
+    x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
+}
+
+// c += X[0:16, 0:8nk] Z[0:8nk, n0:n0+8] for row-major fp32 blocks X (stride
+// ldx, rows from its first row) and Z (stride ldz), one warp, tf32 inputs.
+__device__ __forceinline__ void tile_mma(float (&c)[4], const float *X, int ldx, const float *Z, int ldz, int n0,
+                                         int nk, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+        if (s >= nk) break;
+        const int k = 8 * s;
+        const uint32_t av[4] = {to_tf32(X[g * ldx + k + t]), to_tf32(X[(g + 8) * ldx + k + t]),
+                                to_tf32(X[g * ldx + k + t + 4]), to_tf32(X[(g + 8) * ldx + k + t + 4])};
+        const uint32_t bv[2] = {to_tf32(Z[(k + t) * ldz + n0 + g]), to_tf32(Z[(k + t + 4) * ldz + n0 + g])};
+        mma_tf32_16x8x8(c, av, bv);
+    }
+}
+
+// D[m0.., n0..] (16 x 8 tile) = sgn * c.
+__device__ __forceinline__ void tile_store(float *D, int ldd, int m0, int n0, const float (&c)[4], float sgn,
+                                           int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    *reinterpret_cast<float2 *>(D + (m0 + g) * ldd + n0 + 2 * t) = make_float2(sgn * c[0], sgn * c[1]);
+    *reinterpret_cast<float2 *>(D + (m0 + g + 8) * ldd + n0 + 2 * t) = make_float2(sgn * c[2], sgn * c[3]);
+}
+
 }  // namespace sm100
 }  // namespace gdn

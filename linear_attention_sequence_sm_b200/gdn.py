@@ -32,16 +32,18 @@ GDN_DTYPE_BF16 = 1
 GDN_FLAG_FORCE_SIMT = 1
 GDN_FLAG_QK_L2NORM = 2
 GDN_FLAG_GATE_LOGITS = 4
+GDN_FLAG_ONE_KERNEL = 8
 GDN_OUT_GATE_SILU = 1
 GDN_OUT_GATE_SIGMOID = 2
 GDN_OUT_ZERO_CENTRED = 4
 GDN_OUT_WEIGHT_PER_HEAD = 8
+GDN_CONV_SILU = 1
 
 EXPORTED = ("gdn_chunk_forward_workspace_size", "gdn_chunk_forward", "gdn_read_device_status",
             "gdn_decode_step", "gdn_status_string", "gdn_last_error_message", "gdn_launch_count",
             "gdn_chunk_forward_noalloc", "gdn_decode_step_ex", "gdn_chunk_forward_out", "gdn_decode_step_out",
             "gdn_kda_forward", "gdn_kda_decode_step", "gdn_decode_multi", "gdn_decode_commit",
-            "gdn_chunk_backward_workspace_size", "gdn_chunk_backward")
+            "gdn_chunk_backward_workspace_size", "gdn_chunk_backward", "gdn_short_conv")
 
 
 class GdnError(RuntimeError):
@@ -100,6 +102,9 @@ def _load(path: str = LIB_PATH):
     lib.gdn_chunk_backward_workspace_size.restype = st
     lib.gdn_chunk_backward.argtypes = [ctypes.POINTER(Shape)] + [vp] * 15 + [vp, ctypes.c_size_t, vp]
     lib.gdn_chunk_backward.restype = st
+    lib.gdn_short_conv.argtypes = [i32, i32, vp, ctypes.c_int64, i32, i32, i32, vp, vp, vp, vp, vp,
+                                   ctypes.c_uint32, vp]
+    lib.gdn_short_conv.restype = st
     lib.gdn_status_string.argtypes = [st]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_last_error_message.argtypes = []
@@ -240,7 +245,7 @@ class OutputNorm:
                            None if self.gate is None else self.gate.data_ptr(), self.eps, flags)
 
 
-def make_shape(q, v, cu_seqlens=None, chunk_size=64, force_simt=False, flags=0) -> Shape:
+def make_shape(q, v, cu_seqlens=None, chunk_size=64, force_simt=False, flags=0, one_kernel=False) -> Shape:
     if cu_seqlens is not None:
         T = q.shape[-3]
         B, N = 1, cu_seqlens.shape[0] - 1
@@ -250,7 +255,7 @@ def make_shape(q, v, cu_seqlens=None, chunk_size=64, force_simt=False, flags=0) 
         B, T = q.shape[0], q.shape[1]
         N = B
     return Shape(B, T, N, q.shape[-2], v.shape[-2], q.shape[-1], v.shape[-1], chunk_size, _dtype_code(q),
-                 (GDN_FLAG_FORCE_SIMT if force_simt else 0) | flags)
+                 (GDN_FLAG_FORCE_SIMT if force_simt else 0) | (GDN_FLAG_ONE_KERNEL if one_kernel else 0) | flags)
 
 
 def workspace_size(shape: Shape) -> int:
@@ -261,12 +266,15 @@ def workspace_size(shape: Shape) -> int:
 
 def chunk_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_size=64,
                   output_final_state=True, out=None, final_state=None, workspace=None, force_simt=False,
-                  stream=None, qk_l2norm=False, gate_logits=False, output_norm: OutputNorm | None = None):
+                  stream=None, qk_l2norm=False, gate_logits=False, output_norm: OutputNorm | None = None,
+                  one_kernel=False):
     """Chunkwise prefill.  Returns (o, final_state or None).  Asynchronous on
     ``stream`` (default: the current stream).  ``qk_l2norm``: q and k are raw
     and normalised per head in the kernel; ``gate_logits``: g and beta are
     the decay and write logits (alpha = sigmoid(g), beta = sigmoid(beta));
-    ``output_norm``: the output side applied before o is stored."""
+    ``output_norm``: the output side applied before o is stored;
+    ``one_kernel``: the tensor-core path as one kernel (GDN_FLAG_ONE_KERNEL,
+    schedule-sized workspace)."""
     n_seqs, hv, dv, dk = _prefill_shapes(q, k, v, g, beta, initial_state, cu_seqlens)
     _expect(out, "out", v.shape)
     _expect(final_state, "final_state", (n_seqs, hv, dv, dk))
@@ -278,7 +286,7 @@ def chunk_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_s
     _need(beta, "beta", torch.float32, dev)
     _need(initial_state, "initial_state", torch.float32, dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
-    shape = make_shape(q, v, cu_seqlens, chunk_size, force_simt, input_flags(qk_l2norm, gate_logits))
+    shape = make_shape(q, v, cu_seqlens, chunk_size, force_simt, input_flags(qk_l2norm, gate_logits), one_kernel)
     if out is None:
         out = torch.empty(v.shape, dtype=dt, device=dev)
     _need(out, "out", dt, dev)
@@ -536,6 +544,57 @@ def chunk_backward(q, k, v, g, beta, d_o, d_final_state=None, initial_state=None
                                       _ptr(out["dbeta"]), _ptr(out["d_initial_state"]), _ptr(workspace),
                                       workspace.numel(), _stream_handle(stream, dev)))
     return out
+
+
+def short_conv(x, weight, cu_seqlens=None, state=None, silu=True, out=None, state_out=None,
+               want_state=True, stream=None):
+    """The input side's short causal convolution (depthwise, W taps per
+    channel, the last on the current token), then SiLU when ``silu``.
+    x is [B, T, *channel dims] (batched) or [T, *channel dims] /
+    [1, T, *channel dims] with ``cu_seqlens``; weight [*channel dims, W]
+    fp32; state (each sequence's W-1 preceding inputs, oldest first)
+    [N, *channel dims, W-1] fp32 or None for zeros.  Returns (y shaped like
+    x, the state after each sequence or None)."""
+    if weight.dim() < 2:
+        raise ValueError(f"weight must be [*channel dims, W], got {tuple(weight.shape)}")
+    ch = tuple(weight.shape[:-1])
+    width = weight.shape[-1]
+    nch = len(ch)
+    if cu_seqlens is not None:
+        if x.dim() not in (nch + 1, nch + 2) or (x.dim() == nch + 2 and x.shape[0] != 1):
+            raise ValueError(f"with cu_seqlens x must be [T, *{ch}] or [1, T, *{ch}], got {tuple(x.shape)}")
+        if cu_seqlens.dim() != 1 or cu_seqlens.shape[0] < 1:
+            raise ValueError(f"cu_seqlens must be [N + 1], got {tuple(cu_seqlens.shape)}")
+        n_seqs, seq_len = cu_seqlens.shape[0] - 1, 0
+    else:
+        if x.dim() != nch + 2:
+            raise ValueError(f"batched x must be [B, T, *{ch}], got {tuple(x.shape)}")
+        n_seqs, seq_len = x.shape[0], x.shape[1]
+    if tuple(x.shape[-nch:]) != ch:
+        raise ValueError(f"x's channel dims {tuple(x.shape[-nch:])} differ from the weight's {ch}")
+    _expect(state, "state", (n_seqs, *ch, width - 1))
+    _expect(out, "out", x.shape)
+    _expect(state_out, "state_out", (n_seqs, *ch, width - 1))
+    dev, dt = x.device, x.dtype
+    _need(x, "x", dt, dev)
+    _need(weight, "weight", torch.float32, dev)
+    _need(state, "state", torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    if out is None:
+        out = torch.empty_like(x)
+    _need(out, "out", dt, dev)
+    if state_out is None and want_state:
+        state_out = torch.empty((n_seqs, *ch, width - 1), dtype=torch.float32, device=dev)
+    _need(state_out, "state_out", torch.float32, dev)
+    channels = 1
+    for c in ch:
+        channels *= c
+    tokens = x.numel() // channels
+    with torch.cuda.device(dev):  # the library launches on the current device
+        _check(LIB.gdn_short_conv(n_seqs, seq_len, _ptr(cu_seqlens), tokens, channels, width, _dtype_code(x),
+                                  _ptr(x), _ptr(weight), _ptr(state), _ptr(state_out), _ptr(out),
+                                  GDN_CONV_SILU if silu else 0, _stream_handle(stream, dev)))
+    return out, state_out
 
 
 def launch_count() -> int:

@@ -51,20 +51,23 @@ def oracle_raw(inp, qk_l2norm, gate_logits):
                             cu_seqlens=cu)
 
 
-def gpu_raw(inp, chunk, qk_l2norm, gate_logits, force_simt=False):
+def gpu_raw(inp, chunk, qk_l2norm, gate_logits, path="default"):
     from linear_attention_sequence_sm_b200 import gdn
     dev = torch.device("cuda:0")
     d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
     o, sf = gdn.chunk_forward(d["q"], d["k"], d["v"], d["g"], d["beta"], initial_state=d["initial_state"],
-                              cu_seqlens=d["cu_seqlens"], chunk_size=chunk, force_simt=force_simt,
-                              qk_l2norm=qk_l2norm, gate_logits=gate_logits)
+                              cu_seqlens=d["cu_seqlens"], chunk_size=chunk, force_simt=path == "simt",
+                              one_kernel=path == "one", qk_l2norm=qk_l2norm, gate_logits=gate_logits)
     torch.cuda.synchronize()
     return o, sf
 
 
-@pytest.mark.parametrize("force_simt", [False, True])
+PATHS = ["default", "one", "simt"]  # two-kernel tensor-core, one-kernel tensor-core, fp32 CUDA cores
+
+
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("qk_l2norm,gate_logits", [(True, True), (True, False), (False, True)])
-def test_prefill_bf16_raw_inputs(force_simt, qk_l2norm, gate_logits):
+def test_prefill_bf16_raw_inputs(path, qk_l2norm, gate_logits):
     inp = raw_inputs(61, B=2, T=300, hk=2, hv=4, d=128, dtype="bf16", s0_std=0.02)
     if not qk_l2norm:  # the caller normalised q and k
         for n in ("q", "k"):
@@ -73,19 +76,19 @@ def test_prefill_bf16_raw_inputs(force_simt, qk_l2norm, gate_logits):
     if not gate_logits:  # the caller gave g <= 0 and beta in (0, 1)
         inp["g"] = torch.nn.functional.logsigmoid(inp["g"])
         inp["beta"] = torch.sigmoid(inp["beta"])
-    o, sf = gpu_raw(inp, 64, qk_l2norm, gate_logits, force_simt)
+    o, sf = gpu_raw(inp, 64, qk_l2norm, gate_logits, path)
     o_ref, sf_ref = oracle_raw(inp, qk_l2norm, gate_logits)
     eo, es = prefill_errors(inp, o, sf, o_ref, sf_ref)
     assert eo <= BAR["bf16"] and es <= BAR["bf16"], (eo, es)
 
 
-@pytest.mark.parametrize("force_simt", [False, True])
-def test_prefill_bf16_raw_varlen_edges(force_simt):
+@pytest.mark.parametrize("path", PATHS)
+def test_prefill_bf16_raw_varlen_edges(path):
     """Ragged lengths (1, 63, 64, 65, 0, 200, 7): padded rows of a chunk carry
     the next sequence's raw rows or zeros, and must not reach any output."""
     lens = [1, 63, 64, 65, 0, 200, 7]
     inp = raw_inputs(62, B=1, T=sum(lens), hk=1, hv=4, d=128, dtype="bf16", seq_lens=lens, s0_std=0.02)
-    o, sf = gpu_raw(inp, 64, True, True, force_simt)
+    o, sf = gpu_raw(inp, 64, True, True, path)
     o_ref, sf_ref = oracle_raw(inp, True, True)
     eo, es = prefill_errors(inp, o, sf, o_ref, sf_ref)
     assert eo <= BAR["bf16"] and es <= BAR["bf16"], (eo, es)

@@ -16,15 +16,17 @@ from parity import BAR, full_prefill_errors, gpu_prefill, oracle_prefill, prefil
 
 pytestmark = pytest.mark.gpu
 
-PATHS = [pytest.param(True, id="simt"), pytest.param(False, id="default")]
+# "simt": the fp32 CUDA-core kernel; "default": the two-kernel tensor-core path
+# where it applies; "one": the single-kernel tensor-core path
+PATHS = [pytest.param("simt", id="simt"), pytest.param("default", id="default"), pytest.param("one", id="one")]
 
 
-def _check(w, force_simt, bar=None):
+def _check(w, path, bar=None):
     inp = I.make_prefill_inputs(w)
-    o, sf = gpu_prefill(inp, w.chunk, force_simt=force_simt)
+    o, sf = gpu_prefill(inp, w.chunk, force_simt=path == "simt", one_kernel=path == "one")
     r = full_prefill_errors(inp, o, sf, chunk=64)
     bar = bar or BAR[w.dtype]
-    print(f"PARITY {w.name} {'simt' if force_simt else 'default'}: units {r['units']} o/slice {r['o_slice']:.3e} "
+    print(f"PARITY {w.name} {path}: units {r['units']} o/slice {r['o_slice']:.3e} "
           f"o/chunk {r['o_chunk']:.3e} state {r['state']:.3e} (bar {bar:g})")
     assert r["o_slice"] <= bar and r["o_chunk"] <= bar and r["state"] <= bar, f"{w.name}: {r} (bar {bar:g})"
     return r
@@ -32,40 +34,40 @@ def _check(w, force_simt, bar=None):
 
 def test_tiny_fp32_config():
     """B=1, T=64, 2 q/k and 2 v heads, d=16, C=16, fp32 (bar 1e-4)."""
-    _check(I.tiny_fp32(), force_simt=False)
+    _check(I.tiny_fp32(), "default")
 
 
 @pytest.mark.parametrize("C", [16, 32, 64])
 def test_fp32_d128_ragged(C):
     w = I.custom("fp32_d128", batch=2, seq_len=200, hk=2, hv=4, d=128, chunk=C, dtype="f32", seed=21,
                  s0_std=0.02)
-    _check(w, force_simt=False)
+    _check(w, "default")
 
 
-@pytest.mark.parametrize("force_simt", PATHS)
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("hk,hv", [(2, 4), (4, 12), (4, 4), (1, 3)])
-def test_bf16_d128_c64_batched(force_simt, hk, hv):
+def test_bf16_d128_c64_batched(path, hk, hv):
     w = I.custom(f"bf16_b2_T300_{hk}x{hv}", batch=2, seq_len=300, hk=hk, hv=hv, d=128, chunk=64, dtype="bf16",
                  seed=22 + hv, s0_std=0.02)
-    _check(w, force_simt)
+    _check(w, path)
 
 
-@pytest.mark.parametrize("force_simt", PATHS)
-def test_bf16_varlen_edges(force_simt):
+@pytest.mark.parametrize("path", PATHS)
+def test_bf16_varlen_edges(path):
     """Ragged lengths around the chunk size, a one-token and an empty sequence,
     per-sequence initial states."""
     w = I.custom("bf16_varlen_edges", 1, 0, 2, 4, 128, 64, "bf16", seed=23, s0_std=0.02,
                  seq_lens=[1, 63, 64, 65, 0, 200, 128, 7])
-    _check(w, force_simt)
+    _check(w, path)
 
 
-@pytest.mark.parametrize("force_simt", PATHS)
-def test_bf16_mild_decay_long(force_simt):
+@pytest.mark.parametrize("path", PATHS)
+def test_bf16_mild_decay_long(path):
     """The milder decay of the 4 x 4096 workload (g = -0.1 softplus(N(0,1)+2)),
     where errors have the most room to grow, over 1024 tokens."""
     w = I.custom("bf16_mild", batch=1, seq_len=1024, hk=2, hv=4, d=128, chunk=64, dtype="bf16", seed=24,
                  g_shift=2.0, g_scale=0.1)
-    _check(w, force_simt)
+    _check(w, path)
 
 
 @pytest.mark.parametrize("dk,dv,C,dtype", [(64, 96, 32, "bf16"), (32, 16, 16, "f32"), (128, 64, 64, "f32"),
@@ -91,8 +93,8 @@ def test_other_shapes_simt(dk, dv, C, dtype):
     assert eo <= BAR[dtype] and es <= BAR[dtype], (eo, es)
 
 
-@pytest.mark.parametrize("force_simt", PATHS)
-def test_degenerate_gates(force_simt):
+@pytest.mark.parametrize("path", PATHS)
+def test_degenerate_gates(path):
     """beta = 0 on some tokens (pure decay), g far below the kernel floor and
     g = 0 (no decay) on others: the oracle uses them exactly (g = -inf gives
     alpha = 0); the kernels read max(g, -20), a relative change below 1e-8."""
@@ -103,15 +105,15 @@ def test_degenerate_gates(force_simt):
     inp["g"][0, 50:52] = float("-inf")
     inp["g"][0, 100] = -1e4
     inp["g"][0, 120:180] = 0.0
-    o, sf = gpu_prefill(inp, 64, force_simt=force_simt)
+    o, sf = gpu_prefill(inp, 64, force_simt=path == "simt", one_kernel=path == "one")
     o_ref, sf_ref = oracle_prefill(inp)
     eo, es = prefill_errors(inp, o, sf, o_ref, sf_ref)
     assert eo <= BAR["bf16"] and es <= BAR["bf16"], (eo, es)
     assert torch.isfinite(o.float()).all() and torch.isfinite(sf).all()
 
 
-@pytest.mark.parametrize("force_simt", PATHS)
-def test_in_place_state_and_no_final(force_simt):
+@pytest.mark.parametrize("path", PATHS)
+def test_in_place_state_and_no_final(path):
     """final_state may alias initial_state; output_final_state=False works."""
     from linear_attention_sequence_sm_b200 import gdn
     w = I.custom("bf16_inplace", batch=2, seq_len=130, hk=1, hv=4, d=128, chunk=64, dtype="bf16", seed=27,
@@ -122,9 +124,10 @@ def test_in_place_state_and_no_final(force_simt):
     d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
     state = d["initial_state"].clone()
     o, sf = gdn.chunk_forward(d["q"], d["k"], d["v"], d["g"], d["beta"], initial_state=state, final_state=state,
-                              chunk_size=64, force_simt=force_simt)
+                              chunk_size=64, force_simt=path == "simt", one_kernel=path == "one")
     o2, none = gdn.chunk_forward(d["q"], d["k"], d["v"], d["g"], d["beta"], initial_state=d["initial_state"],
-                                 chunk_size=64, output_final_state=False, force_simt=force_simt)
+                                 chunk_size=64, output_final_state=False, force_simt=path == "simt",
+                                 one_kernel=path == "one")
     torch.cuda.synchronize()
     assert none is None and sf.data_ptr() == state.data_ptr()
     eo, es = prefill_errors(inp, o, state, o_ref, sf_ref)
@@ -179,20 +182,21 @@ def test_prefill_then_decode_equals_longer_prefill():
     assert eo <= BAR["bf16"] and es <= BAR["bf16"], (eo, es)
 
 
-def test_full_size_prefill_4x4096_all_units():
+@pytest.mark.parametrize("path", ["default", "one"])
+def test_full_size_prefill_4x4096_all_units(path):
     """The 4 x 4096 token, 16/32-head, d=128, C=64 bf16 workload at full size,
-    in the launch configuration the benchmark times; every (sequence, head)
-    unit against the oracle."""
-    _check(I.prefill_bf16(), force_simt=False)
+    in the launch configuration the benchmark times (the default path); every
+    (sequence, head) unit against the oracle."""
+    _check(I.prefill_bf16(), path)
 
 
 def test_full_size_varlen_all_units():
     """The 32-sequence packed workload (lengths 128..8192, per-sequence
     initial states) at full size, every unit."""
-    _check(I.varlen_bf16(), force_simt=False)
+    _check(I.varlen_bf16(), "default")
 
 
 def test_full_size_long_context_all_units():
     """The 65,536-token, 16/48-head (3 value heads per q/k head), d=128, C=64
     bf16 workload with initial states, at full size, every unit."""
-    _check(I.long_bf16(), force_simt=False)
+    _check(I.long_bf16(), "default")

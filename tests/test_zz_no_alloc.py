@@ -6,8 +6,9 @@ request path, use this entry point: its scratch is a device array built into
 the library instead of a caller-allocated workspace.  This file checks,
 through the C ABI, that two calls in a row (the second finding the first
 call's leftovers in the shared array) give exactly the results of
-gdn_chunk_forward with a workspace (both run the same deterministic kernels
-on the same inputs), on the tensor-core path and on the fp32 CUDA-core path,
+gdn_chunk_forward with a workspace and GDN_FLAG_ONE_KERNEL (both run the same
+deterministic kernels on the same inputs), on the tensor-core path and on
+the fp32 CUDA-core path,
 each after a call with more sequences, and that a problem too large for the
 array is refused before any launch.  The file name
 makes pytest collect it last.
@@ -59,7 +60,8 @@ def test_noalloc_matches_workspace_entry_point_twice():
         inp, d = _device_inputs(w)
         o_na, sf_na = _noalloc_call(gdn, d, w.chunk, force_simt=simt)
         o_ws, sf_ws = gdn.chunk_forward(d["q"], d["k"], d["v"], d["g"], d["beta"], initial_state=d["initial_state"],
-                                        cu_seqlens=d["cu_seqlens"], chunk_size=w.chunk, force_simt=simt)
+                                        cu_seqlens=d["cu_seqlens"], chunk_size=w.chunk, force_simt=simt,
+                                        one_kernel=True)
         torch.cuda.synchronize()
         assert torch.equal(o_na, o_ws) and torch.equal(sf_na, sf_ws), w.name
         assert torch.isfinite(o_na.float()).all() and torch.isfinite(sf_na).all()
