@@ -67,6 +67,9 @@ def parse_args(argv=None):
     p.add_argument("--backward", action="store_true",
                    help="time the gradients (training) on the prefill workload instead of the forward "
                         "(CUDA-core kernel, fp32 ALU roofline)")
+    p.add_argument("--conv", type=int, default=0,
+                   help="time the input side's short causal convolution with SiLU (this width) over q, k and v "
+                        "of the prefill workload instead of the mixer (HBM roofline)")
     p.add_argument("--mtp", type=int, default=0,
                    help="decode: verify K draft tokens per sequence in one pass (state after every token kept)")
     p.add_argument("--no-graph", action="store_true",
@@ -358,7 +361,8 @@ def prefill_record(args, w, host, device, world, rank, peaks, peak_src, e2e=True
     from linear_attention_sequence_sm_b200 import inputs as I
     flags = {"qk_l2norm": True, "gate_logits": True} if args.raw_inputs else {}
     suffix = ("_kda" if args.kda else "") + ("_raw_inputs" if args.raw_inputs else "") + \
-        ("_output_norm" if args.output_norm else "") + ("_backward" if args.backward else "")
+        ("_output_norm" if args.output_norm else "") + ("_backward" if args.backward else "") + \
+        (f"_conv{args.conv}" if args.conv else "")
     if args.kda:
         host["g"] = I.make_kda_gates(w)
     fwd = gdn.kda_forward if args.kda else gdn.chunk_forward
@@ -386,7 +390,18 @@ def prefill_record(args, w, host, device, world, rank, peaks, peak_src, e2e=True
         gdn.LIB.gdn_chunk_backward_workspace_size(ctypes.byref(bshape), ctypes.byref(nb))
         bws = torch.empty(nb.value, dtype=torch.uint8, device=device)
 
+    if args.conv:
+        convs = []
+        for n_, h_ in (("q", w.hk), ("k", w.hk), ("v", w.hv)):
+            wt = torch.from_numpy(I.normal(w.seed, "conv_" + n_, (h_, w.d, args.conv), std=args.conv ** -0.5))
+            convs.append((dev[n_], wt.float().to(device), torch.empty_like(dev[n_]),
+                          torch.empty((w.num_seqs, h_, w.d, args.conv - 1), dtype=torch.float32, device=device)))
+
     def step():
+        if args.conv:
+            for x_, wt_, y_, so_ in convs:
+                gdn.short_conv(x_, wt_, cu_seqlens=dev["cu_seqlens"], silu=True, out=y_, state_out=so_)
+            return
         if args.backward:
             gdn.chunk_backward(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev["dO"],
                                initial_state=dev["initial_state"], cu_seqlens=dev["cu_seqlens"], workspace=bws)
@@ -431,6 +446,13 @@ def prefill_record(args, w, host, device, world, rank, peaks, peak_src, e2e=True
                     "frac": achieved / alu_peak, "traffic": kernel_traffic(f"gdn_backward/{w.name}{suffix}"),
                     "kernel": "gdn_backward", "peak_source": "fp32 FMA lanes x 2 x max SM clock (derived)",
                     "flops_per_launch": bflops}
+    if args.conv:
+        # one read and one write of q, k and v, the filters, and the conv states written
+        cbytes = conv_bytes(w, args.conv)
+        cgbs = cbytes / (ms / 1e3) / 1e9
+        roofline = {"bound": "hbm", "achieved": cgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": cgbs / peaks["hbm_gbs"], "traffic": kernel_traffic(f"gdn_conv/{w.name}{suffix}"),
+                    "kernel": "gdn_conv", "peak_source": f"{peak_src} HBM copy", "bytes_per_step": cbytes}
     if args.kda:
         # token-order recurrence on CUDA cores: 7 d_v d_k fp32 flops per (token, value head)
         # (decay, two dot products, rank-1 write); peak = SMs x 128 fp32 lanes x 2 x max SM clock
@@ -446,7 +468,7 @@ def prefill_record(args, w, host, device, world, rank, peaks, peak_src, e2e=True
                       "head_dim": w.d, "chunk": w.chunk, "initial_state": w.s0_std > 0,
                       "l2": f"inputs larger than L2 ({prefill_bytes(w) / 1e6:.0f} MB of mandatory traffic per step)"}}
     del o, sf
-    if e2e and not args.no_e2e and not args.backward:
+    if e2e and not args.no_e2e and not args.backward and not args.conv:
         rec["e2e"] = e2e_record(fwd, w, host, ws, flags, out_norm, args.steps, device, world, stream)
     # (raw inputs, the output side, KDA or gradients: the timed oracle covers the plain forward only)
     if cpu and rank == 0 and world == 1 and not args.no_cpu_baseline and not suffix:
@@ -552,7 +574,7 @@ def run_ours(args):
     del host
     # the other two prefill workloads, each with its own record (plain forward only)
     extra = {}
-    plain = not (args.kda or args.raw_inputs or args.output_norm or args.backward)
+    plain = not (args.kda or args.raw_inputs or args.output_norm or args.backward or args.conv)
     if args.only == "all" and args.workload == "prefill" and plain and not args.no_extra:
         for name in ("long", "varlen"):
             mk2, seed2 = makers[name]
@@ -560,7 +582,7 @@ def run_ours(args):
             extra[name] = prefill_record(args, w2, I.make_prefill_inputs(w2), device, world, rank, peaks, peak_src)
 
     decode = None
-    if args.only in ("all", "decode") and args.decode_steps > 0:
+    if args.only in ("all", "decode") and args.decode_steps > 0 and not args.conv:
         decode = decode_record(args, device, world, rank, peaks, peak_src)
 
     if rank == 0:
@@ -618,6 +640,14 @@ def prefill_bytes(w, kda: bool = False) -> int:
     b = t * w.hk * w.d * esz * 2 + t * w.hv * w.d * esz * 2 + t * w.hv * (4 * w.d + 4 if kda else 8)
     b += w.num_seqs * w.hv * w.d * w.d * 4 * (2 if w.s0_std > 0 else 1)
     return b
+
+
+def conv_bytes(w, width: int) -> int:
+    """Algorithmic bytes of one --conv step: q, k and v read and written once
+    in the storage dtype, the fp32 filters read, the fp32 conv states written."""
+    es = 2 if w.dtype == "bf16" else 4
+    ch = 2 * w.hk * w.d + w.hv * w.d
+    return w.total_tokens * ch * es * 2 + ch * width * 4 + w.num_seqs * ch * (width - 1) * 4
 
 
 def decode_bytes(dw, kda: bool = False, mtp: int = 0) -> int:

@@ -231,6 +231,36 @@ def test_backward_and_kda_argument_checks(gdn):
     assert st == gdn.GDN_ERR_UNSUPPORTED
 
 
+def test_short_conv_argument_checks(gdn):
+    """Refused before any device work: widths outside 1..8, channels not a
+    multiple of 4, a token count that the batched layout does not give,
+    aliased outputs, misalignment; no sequences is a no-op; a valid call
+    reaches the device check."""
+    vp = ctypes.c_void_p
+    f = gdn.LIB.gdn_short_conv
+
+    def conv(n=2, seq_len=5, cu=None, tokens=10, ch=256, w=4, dt=1, x=FAKE, wt=FAKE, si=None, so=None, y=FAKE + 4096,
+             flags=1):
+        return f(n, seq_len, None if cu is None else vp(cu), tokens, ch, w, dt, vp(x) if x else None,
+                 vp(wt) if wt else None, vp(si) if si else None, vp(so) if so else None, vp(y) if y else None,
+                 flags, None)
+
+    assert conv(w=0) == gdn.GDN_ERR_UNSUPPORTED and conv(w=9) == gdn.GDN_ERR_UNSUPPORTED
+    assert conv(ch=6) == gdn.GDN_ERR_UNSUPPORTED
+    assert conv(tokens=11) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert conv(flags=2) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert conv(dt=7) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert conv(y=FAKE) == gdn.GDN_ERR_INVALID_ARGUMENT  # y aliases x
+    assert conv(si=FAKE + 8192, so=FAKE + 8192) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert conv(wt=None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    assert conv(x=FAKE + 4) == gdn.GDN_ERR_MISALIGNED
+    assert conv(n=0, tokens=0) == gdn.GDN_OK
+    assert conv(n=0, tokens=4, cu=FAKE) == gdn.GDN_ERR_INVALID_ARGUMENT
+    import torch
+    if not torch.cuda.is_available():  # with a GPU this call would launch on the fake pointers
+        assert conv() == gdn.GDN_ERR_CUDA  # everything valid: the next step needs a GPU
+
+
 def test_header_is_plain_c(tmp_path):
     """include/gdn.h compiles as pedantic C99 (plain pointers and sizes, no
     C++ or torch types in the ABI)."""
