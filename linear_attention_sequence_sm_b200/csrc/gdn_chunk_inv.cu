@@ -107,7 +107,7 @@ __device__ void invert_in_place(float *Af, float *Y, int t) {
         const int m0 = 16 * (w >> 2), n0 = 8 * (w & 3);
         float c[4] = {0.f, 0.f, 0.f, 0.f};
         tile_mma(c, Af + (32 + m0) * kLdA + 32, kLdA, Y, kLdY, n0, 4, lane);
-        tile_store(Af + (32 + m0) * kLdA, kLdA, m0, n0, c, -1.f, lane);
+        tile_store(Af + 32 * kLdA, kLdA, m0, n0, c, -1.f, lane);  // rows 32 + m0 .., columns n0 ..
     }
     __syncthreads();
 }

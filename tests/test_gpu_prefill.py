@@ -113,6 +113,21 @@ def test_degenerate_gates(path):
 
 
 @pytest.mark.parametrize("path", PATHS)
+def test_no_decay_every_chunk(path):
+    """g = 0 on every token (DeltaNet): nothing damps the far entries of the
+    chunks' WY factors, so every block of the triangular inverse carries
+    weight in the outputs (a decaying input hides a wrong far block)."""
+    w = I.custom("bf16_no_decay", batch=2, seq_len=200, hk=1, hv=4, d=128, chunk=64, dtype="bf16", seed=29,
+                 s0_std=0.02)
+    inp = I.make_prefill_inputs(w)
+    inp["g"].zero_()
+    o, sf = gpu_prefill(inp, 64, force_simt=path == "simt", one_kernel=path == "one")
+    r = full_prefill_errors(inp, o, sf, chunk=64)
+    print(f"PARITY bf16_no_decay {path}: o/slice {r['o_slice']:.3e} o/chunk {r['o_chunk']:.3e} state {r['state']:.3e}")
+    assert r["o_slice"] <= BAR["bf16"] and r["o_chunk"] <= BAR["bf16"] and r["state"] <= BAR["bf16"], r
+
+
+@pytest.mark.parametrize("path", PATHS)
 def test_in_place_state_and_no_final(path):
     """final_state may alias initial_state; output_final_state=False works."""
     from linear_attention_sequence_sm_b200 import gdn
