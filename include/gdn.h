@@ -91,7 +91,7 @@ typedef enum { GDN_DTYPE_F32 = 0, GDN_DTYPE_BF16 = 1 } gdn_dtype_t;
  * state-carrying chunk loop that reads them.  This flag runs it as a single
  * kernel that inverts each chunk's factor in place, one chunk ahead of the
  * state; its workspace holds only the schedule tables (a few bytes per
- * sequence) instead of 8 KiB per (chunk, value head), and it needs the value
+ * sequence) instead of 16 KiB per (chunk, value head), and it needs the value
  * heads in multiples of 4.  The results agree within rounding.             */
 #define GDN_FLAG_ONE_KERNEL 8u
 
@@ -118,7 +118,7 @@ typedef struct {
 
 /* Bytes of device workspace gdn_chunk_forward needs for `shape` (a pure
  * function of the shape; the caller allocates it, 256-byte aligned).  For
- * the two-kernel tensor-core path this includes 8 KiB per (chunk, value
+ * the two-kernel tensor-core path this includes 16 KiB per (chunk, value
  * head) for the chunk factors: at most ((tokens + 63 N) / 64) Hv tiles.  A
  * workspace below this size but at least the size queried with
  * GDN_FLAG_ONE_KERNEL set runs the single-kernel path instead. */

@@ -9,7 +9,9 @@
 //   Gamma_rj = e^(G_r - G_j),  G = chunk-local prefix sums of g,
 //   T = (I + A)^-1   (unit lower triangular, 64 x 64),
 //
-// and stores T as bf16.  None of this depends on the state, so it runs over
+// and stores the two column scalings the chunk loop multiplies by, T' = T
+// diag(beta gamma) and T'' = T diag(beta) (gamma = e^G), as bf16, each
+// rounded once from the fp32 T.  None of this depends on the state, so it runs over
 // the chunks of all sequences at once, before the kernel that carries the
 // state (gdn_chunk_chain.cu), which reads T instead of inverting on its
 // critical path.  Tokens past a sequence's end take beta = g = 0, so A is zero
@@ -43,9 +45,11 @@ constexpr uint32_t kOffK0 = 0, kOffK1 = kTileK;
 constexpr uint32_t kOffA = 2 * kTileK;                 // A, inverted in place into T
 constexpr uint32_t kOffY = kOffA + 64 * kLdA * 4;      // 32 x kLdY fp32
 constexpr uint32_t kOffVec = kOffY + 32 * kLdY * 4;    // per-token vectors (below)
-constexpr uint32_t kOffBar = kOffVec + 5 * 64 * 4;     // mbarriers, tensor-memory slot
+constexpr int kMaxGatedHeads = 8;                      // value heads per q/k head whose gates are prefetched
+constexpr uint32_t kOffGst = kOffVec + 6 * 64 * 4;     // gates by cp.async: [2 items][kMaxGatedHeads][g, beta][64]
+constexpr uint32_t kOffBar = kOffGst + 2 * kMaxGatedHeads * 2 * 64 * 4;  // mbarriers, tensor-memory slot
 constexpr uint32_t kSmemBytes = kOffBar + 64 + 1024;   // + alignment slack
-constexpr int kVecG = 0, kVecB = 64, kVecRow = 128, kVecCol = 192, kVecIk = 256;
+constexpr int kVecG = 0, kVecB = 64, kVecRow = 128, kVecCol = 192, kVecIk = 256, kVecTp = 320;
 constexpr int kBarK = 0, kBarMma = 2;  // K tile barriers (2 buffers), Gram completion
 constexpr uint32_t kTmemCols = 64;
 
@@ -169,12 +173,28 @@ chunk_inverse_kernel(const __grid_constant__ CUtensorMap tm_k, const PrefillArgs
         tma_load_3d(buf, &tm_k, 0, hq, t0, bar);
         tma_load_3d(buf + 8192, &tm_k, 64, hq, t0, bar);
     };
+    // the gates of an item's value heads (g, beta for 64 tokens; zeros past the end) by
+    // cp.async into buffer `buf`, one group per item; with more than kMaxGatedHeads value
+    // heads per q/k head the gates are read from global memory instead
+    const bool prefetch = group <= kMaxGatedHeads;
+    auto load_gates = [&](uint32_t buf, int hq, int t0, int L) {
+        if (prefetch) {
+            const uint32_t dst = sb + kOffGst + buf * (kMaxGatedHeads * 512);
+            for (int e = tid; e < group * 128; e += kThreads) {
+                const int j = e >> 7, isb = (e >> 6) & 1, r = e & 63;
+                const size_t i = size_t(t0 + min(r, L - 1)) * hv + hq * group + j;
+                cp_async_4(dst + uint32_t(e) * 4, (isb ? a.beta : a.g) + i, r < L);
+            }
+        }
+        cp_async_commit();
+    };
 
     int item = blockIdx.x;
     int gc = 0, hq = 0, t0 = 0, L = 0;
     if (item < total) {
         locate(item, gc, hq, t0, L);
         if (tid == 0) load_k(sb + kOffK0, hq, t0, bars + 8 * kBarK);
+        load_gates(0, hq, t0, L);
     }
     uint32_t ph_k[2] = {0u, 0u}, ph_m = 0u;
     for (uint32_t it = 0; item < total; ++it, item += gridDim.x) {
@@ -186,6 +206,10 @@ chunk_inverse_kernel(const __grid_constant__ CUtensorMap tm_k, const PrefillArgs
         if (nitem < total) {
             locate(nitem, ngc, nhq, nt0, nL);
             if (tid == 0) load_k(sb + (buf ? kOffK0 : kOffK1), nhq, nt0, bars + 8 * (kBarK + (buf ^ 1u)));
+            load_gates(buf ^ 1u, nhq, nt0, nL);
+            cp_async_wait_1();  // this item's gates (the next item's may still be in flight)
+        } else {
+            cp_async_wait_all();
         }
         {
             const bool ok = warp != 0 || mbar_wait(bars + 8 * (kBarK + buf), ph_k[buf]);
@@ -230,9 +254,15 @@ chunk_inverse_kernel(const __grid_constant__ CUtensorMap tm_k, const PrefillArgs
             // per lane); tokens past the end get g = beta = 0
             if (warp == 0) {
                 const bool ok0 = 2 * lane < L, ok1 = 2 * lane + 1 < L;
-                const size_t i0 = size_t(t0 + 2 * lane) * hv + h, i1 = i0 + hv;
-                const float ga = ok0 ? a.g[i0] : 0.f, gb = ok1 ? a.g[i1] : 0.f;
-                const float ba = ok0 ? a.beta[i0] : 0.f, bb = ok1 ? a.beta[i1] : 0.f;
+                float ga, gb, ba, bb;
+                if (prefetch) {
+                    const float *gs = reinterpret_cast<const float *>(smem + kOffGst) + buf * (kMaxGatedHeads * 128) + j * 128;
+                    ga = gs[2 * lane]; gb = gs[2 * lane + 1]; ba = gs[64 + 2 * lane]; bb = gs[64 + 2 * lane + 1];
+                } else {
+                    const size_t i0 = size_t(t0 + 2 * lane) * hv + h, i1 = i0 + hv;
+                    ga = ok0 ? a.g[i0] : 0.f; gb = ok1 ? a.g[i1] : 0.f;
+                    ba = ok0 ? a.beta[i0] : 0.f; bb = ok1 ? a.beta[i1] : 0.f;
+                }
                 const float g0 = ok0 ? fmaxf(kLogits ? log_sigmoid_fast(ga) : ga, kGFloor) : 0.f;
                 const float g1 = ok1 ? fmaxf(kLogits ? log_sigmoid_fast(gb) : gb, kGFloor) : 0.f;
                 vec[kVecB + 2 * lane] = ok0 ? (kLogits ? sigmoid_fast(ba) : ba) : 0.f;
@@ -259,6 +289,7 @@ chunk_inverse_kernel(const __grid_constant__ CUtensorMap tm_k, const PrefillArgs
                 const float ik = kL2 ? vec[kVecIk + tid] : 1.f;
                 vec[kVecRow + tid] = rank1 ? bt * __expf(G) * ik : bt * ik;
                 vec[kVecCol + tid] = rank1 ? __expf(-G) * ik : ik;
+                vec[kVecTp + tid] = bt * __expf(G) * ik;  // T' column scale beta gamma (/||k||)
             }
             if (j == 0) {  // the Gram is complete
                 const bool ok = warp != 0 || mbar_wait(bars + 8 * kBarMma, ph_m);
@@ -269,7 +300,8 @@ chunk_inverse_kernel(const __grid_constant__ CUtensorMap tm_k, const PrefillArgs
                 __syncthreads();
             }
             // A from the Gram: warp w reads its lane quarter (rows 16 (w % 4) ..
-            // + 15 in lanes 0-15) and 32 of the 64 columns
+            // + 15 in lanes 0-15) and 32 of the 64 columns; slices entirely above
+            // the diagonal are zeros without a tensor-memory read
             {
                 const int quarter = warp & 3, half = warp >> 2;
                 const int r = 16 * quarter + (lane & 15);
@@ -278,22 +310,30 @@ chunk_inverse_kernel(const __grid_constant__ CUtensorMap tm_k, const PrefillArgs
 #pragma unroll
                 for (int sl = 0; sl < 2; ++sl) {
                     const int j0 = 32 * half + 16 * sl;
-                    float v[16], cs[16], gj[16];
-                    tmem_ld16(tmem + (uint32_t(32 * quarter) << 16) + uint32_t(j0), v);
+                    float xo[16];
+                    if (j0 / 16 > quarter) {  // warp-uniform: every entry has j > r
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        load4(vec + kVecCol + j0 + 4 * q, cs + 4 * q);
-                        load4(vec + kVecG + j0 + 4 * q, gj + 4 * q);
-                    }
-                    tmem_wait_ld();
-                    if (valid) {
-                        float xo[16];
+                        for (int jj = 0; jj < 16; ++jj) xo[jj] = 0.f;
+                    } else {
+                        float v[16], cs[16];
+                        tmem_ld16(tmem + (uint32_t(32 * quarter) << 16) + uint32_t(j0), v);
 #pragma unroll
-                        for (int jj = 0; jj < 16; ++jj) {
-                            const float keep = (j0 + jj < r) ? 1.f : 0.f;
-                            xo[jj] = rank1 ? keep * rs * cs[jj] * v[jj]
-                                           : keep * rs * cs[jj] * __expf(fminf(Gr - gj[jj], 0.f)) * v[jj];
+                        for (int q = 0; q < 4; ++q) load4(vec + kVecCol + j0 + 4 * q, cs + 4 * q);
+                        tmem_wait_ld();
+                        if (rank1) {  // uniform across the CTA
+#pragma unroll
+                            for (int jj = 0; jj < 16; ++jj)
+                                xo[jj] = (j0 + jj < r) ? rs * cs[jj] * v[jj] : 0.f;
+                        } else {
+                            float gj[16];
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) load4(vec + kVecG + j0 + 4 * q, gj + 4 * q);
+#pragma unroll
+                            for (int jj = 0; jj < 16; ++jj)
+                                xo[jj] = (j0 + jj < r) ? rs * cs[jj] * __expf(fminf(Gr - gj[jj], 0.f)) * v[jj] : 0.f;
                         }
+                    }
+                    if (valid) {
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
                             *reinterpret_cast<float4 *>(Af + r * kLdA + j0 + 4 * q) =
@@ -304,13 +344,29 @@ chunk_inverse_kernel(const __grid_constant__ CUtensorMap tm_k, const PrefillArgs
             tc_fence_before();  // the tensor-memory reads are ordered before the next item's Gram
             __syncthreads();
             invert_in_place(Af, Yb, tid);
-            // T (bf16, row-major) to its slot: thread t stores 16 entries of row t / 4
+            // T' = T diag(beta gamma (/||k||)) and T'' = T diag(beta) (bf16, row-major, T' then
+            // T'') to the (chunk, head) slot: thread t stores 16 entries of row t / 4 of each
             {
                 const int r = tid >> 2, c0 = (tid & 3) * 16;
                 const float *src = Af + r * kLdA + c0;
-                uint4 *dst = reinterpret_cast<uint4 *>(tinv + ((size_t(gc) * hv + h) * 64 + r) * 64 + c0);
-                dst[0] = pack_bf16x8(src);
-                dst[1] = pack_bf16x8(src + 8);
+                uint4 *dst = reinterpret_cast<uint4 *>(tinv + ((size_t(gc) * hv + h) * 128 + r) * 64 + c0);
+                float tp[16], tpp[16];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float x[4], sp[4], sb[4];
+                    load4(src + 4 * q, x);
+                    load4(vec + kVecTp + c0 + 4 * q, sp);
+                    load4(vec + kVecB + c0 + 4 * q, sb);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        tp[4 * q + u] = x[u] * sp[u];
+                        tpp[4 * q + u] = x[u] * sb[u];
+                    }
+                }
+                dst[0] = pack_bf16x8(tp);
+                dst[1] = pack_bf16x8(tp + 8);
+                dst[64 * 64 / 8] = pack_bf16x8(tpp);  // T'' tile: 64 x 64 entries on
+                dst[64 * 64 / 8 + 1] = pack_bf16x8(tpp + 8);
             }
             __syncthreads();  // Af and the vectors are reused by the next head
         }
@@ -321,6 +377,7 @@ chunk_inverse_kernel(const __grid_constant__ CUtensorMap tm_k, const PrefillArgs
         __syncthreads();
         gc = ngc; hq = nhq; t0 = nt0; L = nL;
     }
+    cp_async_wait_all();
     if (aborted && tid == 0 && total > 0) {
         // let this thread's tensor-core work drain (bounded) before the tensor
         // memory is freed

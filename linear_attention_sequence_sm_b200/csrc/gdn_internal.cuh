@@ -68,9 +68,9 @@ inline WsLayout ws_layout(int32_t num_seqs) {
 //   chunk_base [N + 1]    first chunk of each sequence in the chunk order
 //                         (sequence by sequence, chunks in token order);
 //                         chunk_base[N] = total chunks
-//   tinv                  per (chunk, value head) the 64 x 64 bf16 inverse T
-//                         of the chunk's WY representation, row-major,
-//                         [max_chunks][Hv][64][64]
+//   tinv                  per (chunk, value head) T' = T diag(beta gamma) and
+//                         T'' = T diag(beta) of the chunk's WY factor
+//                         T = (I + A)^-1, bf16 row-major, [max_chunks][Hv][2][64][64]
 // max_chunks bounds the chunk count for the shape: (tokens + 63 N) / 64 (each
 // sequence adds at most one partial chunk).
 struct SplitLayout {
@@ -93,7 +93,7 @@ inline SplitLayout split_layout(const gdn_shape_t &s) {
     off = (off + 1023) & ~size_t(1023);
     L.tinv_off = off;
     L.max_chunks = max_chunks_bound(s);
-    off += size_t(L.max_chunks) * size_t(s.num_v_heads) * 64 * 64 * 2;
+    off += size_t(L.max_chunks) * size_t(s.num_v_heads) * 2 * 64 * 64 * 2;
     L.total = align256(off);
     return L;
 }

@@ -151,6 +151,8 @@ __device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src, bool v
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// Waits until at most one of this thread's committed cp.async groups is pending.
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 // Warp-level tf32 product (m16n8k8, fp32 accumulate) for small fp32 matrix
 // blocks; fragments: a = rows (g, g+8) x cols (t, t+4), b = rows (t, t+4) x
