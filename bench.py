@@ -426,7 +426,12 @@ def prefill_record(args, w, host, device, world, rank, peaks, peak_src, e2e=True
     tokens = w.total_tokens
     flops = useful_flops_per_vhead_token(w.hv // w.hk) * tokens * w.hv
     achieved_tflops = flops / (ms / 1e3) / 1e12
-    kernel_name = "gdn_chunk_tc" if gdn_tc_active(gdn, dev, w) else "gdn_chunk_simt"
+    # the default path: the single tensor-core kernel where the value heads come in
+    # multiples of 4, else the two-kernel form (chunk factors, then the chunk loop)
+    if not gdn_tc_active(gdn, dev, w):
+        kernel_name = "gdn_chunk_simt"
+    else:
+        kernel_name = "gdn_chunk_tc" if w.hv % 4 == 0 else "gdn_chunk_inverse+gdn_chunk_chain"
     roofline = {"bound": "tensor", "achieved": achieved_tflops, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved_tflops / peaks["bf16_tflops"],
                 "traffic": kernel_traffic(f"{kernel_name}/{w.name}{suffix}"),

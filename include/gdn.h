@@ -85,15 +85,21 @@ typedef enum { GDN_DTYPE_F32 = 0, GDN_DTYPE_BF16 = 1 } gdn_dtype_t;
                                     write logit b: alpha = sigmoid(a), i.e.
                                     the log-decay is log sigmoid(a), and the
                                     write strength is sigmoid(b)            */
-/* The bf16 tensor-core prefill (d_k = d_v = 128, C = 64) normally runs as two
- * kernels: the chunks' triangular WY factors T = (I + A)^-1 for all chunks at
- * once (they do not depend on the state), kept in the workspace, then the
- * state-carrying chunk loop that reads them.  This flag runs it as a single
- * kernel that inverts each chunk's factor in place, one chunk ahead of the
- * state; its workspace holds only the schedule tables (a few bytes per
- * sequence) instead of 16 KiB per (chunk, value head), and it needs the value
- * heads in multiples of 4.  The results agree within rounding.             */
+/* The bf16 tensor-core prefill (d_k = d_v = 128, C = 64) has two forms.  The
+ * single kernel inverts each chunk's triangular WY factor T = (I + A)^-1 in
+ * place, one chunk ahead of the state; its workspace holds only the schedule
+ * tables (a few bytes per sequence), and it needs the value heads in
+ * multiples of 4.  The two-kernel form computes the factors of all chunks at
+ * once (they do not depend on the state) into the workspace, 16 KiB per
+ * (chunk, value head), then runs the state-carrying chunk loop that reads
+ * them; it takes any head count.  By default the single kernel runs where it
+ * applies and the two-kernel form where it does not (value heads not a
+ * multiple of 4).  GDN_FLAG_SPLIT asks for the two-kernel form wherever it
+ * applies; GDN_FLAG_ONE_KERNEL never runs it (shapes the single kernel does
+ * not take then run the fp32 CUDA-core kernel).  Setting both is an invalid
+ * argument.  The results agree within rounding.                            */
 #define GDN_FLAG_ONE_KERNEL 8u
+#define GDN_FLAG_SPLIT 16u
 
 /* Shape of a prefill problem.
  *   batch, seq_len  without cu_seqlens: B sequences of T tokens each
@@ -117,11 +123,12 @@ typedef struct {
 } gdn_shape_t;
 
 /* Bytes of device workspace gdn_chunk_forward needs for `shape` (a pure
- * function of the shape; the caller allocates it, 256-byte aligned).  For
- * the two-kernel tensor-core path this includes 16 KiB per (chunk, value
- * head) for the chunk factors: at most ((tokens + 63 N) / 64) Hv tiles.  A
- * workspace below this size but at least the size queried with
- * GDN_FLAG_ONE_KERNEL set runs the single-kernel path instead. */
+ * function of the shape, flags included; the caller allocates it, 256-byte
+ * aligned).  Where the two-kernel tensor-core form runs, this includes
+ * 16 KiB per (chunk, value head) for the chunk factors: at most
+ * ((tokens + 63 N) / 64) Hv of them.  With a workspace below that size (but
+ * at least the size queried with GDN_FLAG_ONE_KERNEL set) the call runs as
+ * if GDN_FLAG_ONE_KERNEL were set. */
 GDN_API gdn_status_t gdn_chunk_forward_workspace_size(const gdn_shape_t *shape, size_t *bytes);
 
 /* Chunkwise prefill ("Gated Attention Architectures", sections 2 and 3: the

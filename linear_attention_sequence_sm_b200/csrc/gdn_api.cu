@@ -54,7 +54,10 @@ static gdn_status_t check_shape(const gdn_shape_t *s) {
                     s->num_v_heads, s->num_qk_heads);
     if (s->dtype != GDN_DTYPE_F32 && s->dtype != GDN_DTYPE_BF16)
         return fail(GDN_ERR_INVALID_ARGUMENT, "dtype %d is not GDN_DTYPE_F32 or GDN_DTYPE_BF16", s->dtype);
-    if (s->flags & ~(GDN_FLAG_FORCE_SIMT | GDN_FLAG_QK_L2NORM | GDN_FLAG_GATE_LOGITS | GDN_FLAG_ONE_KERNEL))
+    if ((s->flags & GDN_FLAG_ONE_KERNEL) && (s->flags & GDN_FLAG_SPLIT))
+        return fail(GDN_ERR_INVALID_ARGUMENT, "GDN_FLAG_ONE_KERNEL and GDN_FLAG_SPLIT are both set");
+    if (s->flags &
+        ~(GDN_FLAG_FORCE_SIMT | GDN_FLAG_QK_L2NORM | GDN_FLAG_GATE_LOGITS | GDN_FLAG_ONE_KERNEL | GDN_FLAG_SPLIT))
         return fail(GDN_ERR_INVALID_ARGUMENT, "unknown flag bits 0x%x", s->flags);
     if (s->chunk_size != 16 && s->chunk_size != 32 && s->chunk_size != 64)
         return fail(GDN_ERR_UNSUPPORTED, "chunk_size %d not in {16, 32, 64}", s->chunk_size);
@@ -70,6 +73,13 @@ static gdn_status_t check_shape(const gdn_shape_t *s) {
 
 // Validates an output-side descriptor (NULL = none) and converts it for the
 // kernels.
+// The two-kernel tensor-core form: asked for with GDN_FLAG_SPLIT, else taken
+// where the single kernel does not apply (value heads not a multiple of 4).
+static bool wants_split(const gdn_shape_t &s) {
+    if (!chunk_split_supported(s) || (s.flags & (GDN_FLAG_ONE_KERNEL | GDN_FLAG_FORCE_SIMT))) return false;
+    return (s.flags & GDN_FLAG_SPLIT) || !chunk_tc_supported(s);
+}
+
 static gdn_status_t check_output_side(const gdn_output_side_t *os, OutSide *out) {
     *out = OutSide{nullptr, nullptr, 0.f, 0u};
     if (!os) return GDN_OK;
@@ -127,8 +137,7 @@ gdn_status_t gdn_chunk_forward_workspace_size(const gdn_shape_t *s, size_t *byte
     if (!bytes) return fail(GDN_ERR_INVALID_ARGUMENT, "bytes is NULL");
     gdn_status_t st = check_shape(s);
     if (st != GDN_OK) return st;
-    const bool split = chunk_split_supported(*s) && !(s->flags & (GDN_FLAG_ONE_KERNEL | GDN_FLAG_FORCE_SIMT));
-    *bytes = split ? split_layout(*s).total : ws_layout(s->num_seqs).total;
+    *bytes = wants_split(*s) ? split_layout(*s).total : ws_layout(s->num_seqs).total;
     return GDN_OK;
 }
 
@@ -237,8 +246,8 @@ static gdn_status_t chunk_forward_impl(const gdn_shape_t *s, const void *q, cons
     // The two-kernel tensor-core path needs the full queried workspace (it keeps
     // every chunk's inverse there); with less, or with the output side, the
     // single-kernel tensor-core path runs where it applies.
-    const bool use_split = tc_arch && tokens > 0 && !out.flags && !(s->flags & GDN_FLAG_ONE_KERNEL) &&
-                           chunk_split_supported(*s) && workspace_bytes >= split_layout(*s).total;
+    const bool use_split =
+        tc_arch && tokens > 0 && !out.flags && wants_split(*s) && workspace_bytes >= split_layout(*s).total;
     const bool use_tc = !use_split && tc_arch && chunk_tc_supported(*s);
     if (use_split) {
         const SplitLayout SL = split_layout(*s);

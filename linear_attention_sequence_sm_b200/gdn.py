@@ -33,6 +33,7 @@ GDN_FLAG_FORCE_SIMT = 1
 GDN_FLAG_QK_L2NORM = 2
 GDN_FLAG_GATE_LOGITS = 4
 GDN_FLAG_ONE_KERNEL = 8
+GDN_FLAG_SPLIT = 16
 GDN_OUT_GATE_SILU = 1
 GDN_OUT_GATE_SIGMOID = 2
 GDN_OUT_ZERO_CENTRED = 4
@@ -245,7 +246,8 @@ class OutputNorm:
                            None if self.gate is None else self.gate.data_ptr(), self.eps, flags)
 
 
-def make_shape(q, v, cu_seqlens=None, chunk_size=64, force_simt=False, flags=0, one_kernel=False) -> Shape:
+def make_shape(q, v, cu_seqlens=None, chunk_size=64, force_simt=False, flags=0, one_kernel=False,
+               split=False) -> Shape:
     if cu_seqlens is not None:
         T = q.shape[-3]
         B, N = 1, cu_seqlens.shape[0] - 1
@@ -255,7 +257,8 @@ def make_shape(q, v, cu_seqlens=None, chunk_size=64, force_simt=False, flags=0, 
         B, T = q.shape[0], q.shape[1]
         N = B
     return Shape(B, T, N, q.shape[-2], v.shape[-2], q.shape[-1], v.shape[-1], chunk_size, _dtype_code(q),
-                 (GDN_FLAG_FORCE_SIMT if force_simt else 0) | (GDN_FLAG_ONE_KERNEL if one_kernel else 0) | flags)
+                 (GDN_FLAG_FORCE_SIMT if force_simt else 0) | (GDN_FLAG_ONE_KERNEL if one_kernel else 0) |
+                 (GDN_FLAG_SPLIT if split else 0) | flags)
 
 
 def workspace_size(shape: Shape) -> int:
@@ -267,14 +270,15 @@ def workspace_size(shape: Shape) -> int:
 def chunk_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_size=64,
                   output_final_state=True, out=None, final_state=None, workspace=None, force_simt=False,
                   stream=None, qk_l2norm=False, gate_logits=False, output_norm: OutputNorm | None = None,
-                  one_kernel=False):
+                  one_kernel=False, split=False):
     """Chunkwise prefill.  Returns (o, final_state or None).  Asynchronous on
     ``stream`` (default: the current stream).  ``qk_l2norm``: q and k are raw
     and normalised per head in the kernel; ``gate_logits``: g and beta are
     the decay and write logits (alpha = sigmoid(g), beta = sigmoid(beta));
     ``output_norm``: the output side applied before o is stored;
-    ``one_kernel``: the tensor-core path as one kernel (GDN_FLAG_ONE_KERNEL,
-    schedule-sized workspace)."""
+    ``one_kernel``: never the two-kernel tensor-core form (GDN_FLAG_ONE_KERNEL,
+    schedule-sized workspace); ``split``: the two-kernel form wherever it
+    applies (GDN_FLAG_SPLIT)."""
     n_seqs, hv, dv, dk = _prefill_shapes(q, k, v, g, beta, initial_state, cu_seqlens)
     _expect(out, "out", v.shape)
     _expect(final_state, "final_state", (n_seqs, hv, dv, dk))
@@ -286,7 +290,8 @@ def chunk_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk_s
     _need(beta, "beta", torch.float32, dev)
     _need(initial_state, "initial_state", torch.float32, dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
-    shape = make_shape(q, v, cu_seqlens, chunk_size, force_simt, input_flags(qk_l2norm, gate_logits), one_kernel)
+    shape = make_shape(q, v, cu_seqlens, chunk_size, force_simt, input_flags(qk_l2norm, gate_logits), one_kernel,
+                       split)
     if out is None:
         out = torch.empty(v.shape, dtype=dt, device=dev)
     _need(out, "out", dt, dev)

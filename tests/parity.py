@@ -15,14 +15,14 @@ def to_f64(t):
     return None if t is None else t.detach().to("cpu", torch.float64).numpy()
 
 
-def gpu_prefill(inp, chunk, force_simt=False, final_state=True, initial_state="inp", one_kernel=False):
+def gpu_prefill(inp, chunk, force_simt=False, final_state=True, initial_state="inp", split=False):
     from linear_attention_sequence_sm_b200 import gdn
     dev = torch.device("cuda:0")
     d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
     s0 = d["initial_state"] if initial_state == "inp" else initial_state
     o, sf = gdn.chunk_forward(d["q"], d["k"], d["v"], d["g"], d["beta"], initial_state=s0,
                               cu_seqlens=d["cu_seqlens"], chunk_size=chunk, output_final_state=final_state,
-                              force_simt=force_simt, one_kernel=one_kernel)
+                              force_simt=force_simt, split=split)
     torch.cuda.synchronize()
     return o, sf
 

@@ -58,6 +58,30 @@ def test_workspace_size(gdn):
     assert big > n
 
 
+def test_workspace_size_follows_the_path(gdn):
+    """The bf16 d=128 C=64 shape runs the single tensor-core kernel by default
+    (schedule-sized workspace); GDN_FLAG_SPLIT asks for the two-kernel form and
+    its 16 KiB per (chunk, value head); value heads not a multiple of 4 take
+    the two-kernel form by default."""
+    kw = dict(batch=2, seq_len=200, num_seqs=2, num_qk_heads=2, num_v_heads=8, head_dim_k=128, head_dim_v=128,
+              chunk_size=64, dtype=gdn.GDN_DTYPE_BF16)
+    one = gdn.workspace_size(_shape(gdn, **kw))
+    split = gdn.workspace_size(_shape(gdn, flags=gdn.GDN_FLAG_SPLIT, **kw))
+    assert split >= one + 2 * 4 * 8 * 16384  # 2 sequences x 4 chunks x 8 heads
+    assert gdn.workspace_size(_shape(gdn, flags=gdn.GDN_FLAG_ONE_KERNEL, **kw)) == one
+    odd = dict(kw, num_qk_heads=1, num_v_heads=6)
+    assert gdn.workspace_size(_shape(gdn, **odd)) > gdn.workspace_size(_shape(gdn, flags=gdn.GDN_FLAG_ONE_KERNEL,
+                                                                                **odd))
+    # the fp32 path never takes the two-kernel form
+    assert gdn.workspace_size(_shape(gdn, flags=gdn.GDN_FLAG_SPLIT, **dict(kw, dtype=gdn.GDN_DTYPE_F32))) == one
+
+
+def test_contradictory_path_flags_rejected(gdn):
+    n = ctypes.c_size_t(0)
+    s = _shape(gdn, flags=gdn.GDN_FLAG_SPLIT | gdn.GDN_FLAG_ONE_KERNEL)
+    assert gdn.LIB.gdn_chunk_forward_workspace_size(ctypes.byref(s), ctypes.byref(n)) == gdn.GDN_ERR_INVALID_ARGUMENT
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(num_v_heads=3), 1),          # Hv % Hk != 0
     (dict(dtype=7), 1),                # unknown dtype

@@ -57,12 +57,12 @@ def gpu_raw(inp, chunk, qk_l2norm, gate_logits, path="default"):
     d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
     o, sf = gdn.chunk_forward(d["q"], d["k"], d["v"], d["g"], d["beta"], initial_state=d["initial_state"],
                               cu_seqlens=d["cu_seqlens"], chunk_size=chunk, force_simt=path == "simt",
-                              one_kernel=path == "one", qk_l2norm=qk_l2norm, gate_logits=gate_logits)
+                              split=path == "split", qk_l2norm=qk_l2norm, gate_logits=gate_logits)
     torch.cuda.synchronize()
     return o, sf
 
 
-PATHS = ["default", "one", "simt"]  # two-kernel tensor-core, one-kernel tensor-core, fp32 CUDA cores
+PATHS = ["default", "split", "simt"]  # one-kernel tensor-core, two-kernel tensor-core, fp32 CUDA cores
 
 
 @pytest.mark.parametrize("path", PATHS)

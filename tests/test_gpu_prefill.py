@@ -16,14 +16,15 @@ from parity import BAR, full_prefill_errors, gpu_prefill, oracle_prefill, prefil
 
 pytestmark = pytest.mark.gpu
 
-# "simt": the fp32 CUDA-core kernel; "default": the two-kernel tensor-core path
-# where it applies; "one": the single-kernel tensor-core path
-PATHS = [pytest.param("simt", id="simt"), pytest.param("default", id="default"), pytest.param("one", id="one")]
+# "simt": the fp32 CUDA-core kernel; "default": the single-kernel tensor-core
+# path where it applies (the two-kernel one for value heads not a multiple of
+# 4); "split": the two-kernel tensor-core path
+PATHS = [pytest.param("simt", id="simt"), pytest.param("default", id="default"), pytest.param("split", id="split")]
 
 
 def _check(w, path, bar=None):
     inp = I.make_prefill_inputs(w)
-    o, sf = gpu_prefill(inp, w.chunk, force_simt=path == "simt", one_kernel=path == "one")
+    o, sf = gpu_prefill(inp, w.chunk, force_simt=path == "simt", split=path == "split")
     r = full_prefill_errors(inp, o, sf, chunk=64)
     bar = bar or BAR[w.dtype]
     print(f"PARITY {w.name} {path}: units {r['units']} o/slice {r['o_slice']:.3e} "
@@ -105,7 +106,7 @@ def test_degenerate_gates(path):
     inp["g"][0, 50:52] = float("-inf")
     inp["g"][0, 100] = -1e4
     inp["g"][0, 120:180] = 0.0
-    o, sf = gpu_prefill(inp, 64, force_simt=path == "simt", one_kernel=path == "one")
+    o, sf = gpu_prefill(inp, 64, force_simt=path == "simt", split=path == "split")
     o_ref, sf_ref = oracle_prefill(inp)
     eo, es = prefill_errors(inp, o, sf, o_ref, sf_ref)
     assert eo <= BAR["bf16"] and es <= BAR["bf16"], (eo, es)
@@ -121,7 +122,7 @@ def test_no_decay_every_chunk(path):
                  s0_std=0.02)
     inp = I.make_prefill_inputs(w)
     inp["g"].zero_()
-    o, sf = gpu_prefill(inp, 64, force_simt=path == "simt", one_kernel=path == "one")
+    o, sf = gpu_prefill(inp, 64, force_simt=path == "simt", split=path == "split")
     r = full_prefill_errors(inp, o, sf, chunk=64)
     print(f"PARITY bf16_no_decay {path}: o/slice {r['o_slice']:.3e} o/chunk {r['o_chunk']:.3e} state {r['state']:.3e}")
     assert r["o_slice"] <= BAR["bf16"] and r["o_chunk"] <= BAR["bf16"] and r["state"] <= BAR["bf16"], r
@@ -139,10 +140,10 @@ def test_in_place_state_and_no_final(path):
     d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
     state = d["initial_state"].clone()
     o, sf = gdn.chunk_forward(d["q"], d["k"], d["v"], d["g"], d["beta"], initial_state=state, final_state=state,
-                              chunk_size=64, force_simt=path == "simt", one_kernel=path == "one")
+                              chunk_size=64, force_simt=path == "simt", split=path == "split")
     o2, none = gdn.chunk_forward(d["q"], d["k"], d["v"], d["g"], d["beta"], initial_state=d["initial_state"],
                                  chunk_size=64, output_final_state=False, force_simt=path == "simt",
-                                 one_kernel=path == "one")
+                                 split=path == "split")
     torch.cuda.synchronize()
     assert none is None and sf.data_ptr() == state.data_ptr()
     eo, es = prefill_errors(inp, o, state, o_ref, sf_ref)
@@ -197,7 +198,7 @@ def test_prefill_then_decode_equals_longer_prefill():
     assert eo <= BAR["bf16"] and es <= BAR["bf16"], (eo, es)
 
 
-@pytest.mark.parametrize("path", ["default", "one"])
+@pytest.mark.parametrize("path", ["default", "split"])
 def test_full_size_prefill_4x4096_all_units(path):
     """The 4 x 4096 token, 16/32-head, d=128, C=64 bf16 workload at full size,
     in the launch configuration the benchmark times (the default path); every

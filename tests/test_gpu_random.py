@@ -33,7 +33,7 @@ def case(seed):
         lens, B, T = None, int(rng.integers(1, 4)), int(rng.integers(1, 300))
     return dict(hk=hk, hv=hv, d=d, dtype=dtype, lens=lens, B=B, T=T, s0=bool(rng.random() < 0.6),
                 l2=bool(rng.random() < 0.4), logits=bool(rng.random() < 0.4), out=bool(rng.random() < 0.4),
-                one=bool(rng.random() < 0.3))
+                split=bool(rng.random() < 0.3))
 
 
 @pytest.mark.parametrize("seed", range(24))
@@ -62,7 +62,7 @@ def test_random_prefill(seed):
     d = {k: (v.to(DEV) if v is not None else None) for k, v in inp.items()}
     o, sf = gdn.chunk_forward(d["q"], d["k"], d["v"], d["g"], d["beta"], initial_state=d["initial_state"],
                               cu_seqlens=d["cu_seqlens"], chunk_size=64, qk_l2norm=c["l2"], gate_logits=c["logits"],
-                              output_norm=on, one_kernel=c["one"])
+                              output_norm=on, split=c["split"])
     torch.cuda.synchronize()
     q, k, g, b = oracle.prepare_inputs(to_f64(inp["q"]), to_f64(inp["k"]), to_f64(inp["g"]), to_f64(inp["beta"]),
                                        qk_l2norm=c["l2"], gate_logits=c["logits"])
