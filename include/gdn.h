@@ -90,9 +90,9 @@ typedef enum { GDN_DTYPE_F32 = 0, GDN_DTYPE_BF16 = 1 } gdn_dtype_t;
  * place, one chunk ahead of the state; its workspace holds only the schedule
  * tables (a few bytes per sequence), and it needs the value heads in
  * multiples of 4.  The two-kernel form computes the factors of all chunks at
- * once (they do not depend on the state) into the workspace, 16 KiB per
- * (chunk, value head), then runs the state-carrying chunk loop that reads
- * them; it takes any head count.  By default the single kernel runs where it
+ * once (they do not depend on the state) into the workspace, 16,640 bytes
+ * per (chunk, value head), then runs the state-carrying chunk loop that
+ * reads them; it takes any head count.  By default the single kernel runs where it
  * applies and the two-kernel form where it does not (value heads not a
  * multiple of 4).  GDN_FLAG_SPLIT asks for the two-kernel form wherever it
  * applies; GDN_FLAG_ONE_KERNEL never runs it (shapes the single kernel does
@@ -125,7 +125,8 @@ typedef struct {
 /* Bytes of device workspace gdn_chunk_forward needs for `shape` (a pure
  * function of the shape, flags included; the caller allocates it, 256-byte
  * aligned).  Where the two-kernel tensor-core form runs, this includes
- * 16 KiB per (chunk, value head) for the chunk factors: at most
+ * 16,640 bytes per (chunk, value head) for the chunk factors (T', T'' and
+ * the decay prefix sums): at most
  * ((tokens + 63 N) / 64) Hv of them.  With a workspace below that size (but
  * at least the size queried with GDN_FLAG_ONE_KERNEL set) the call runs as
  * if GDN_FLAG_ONE_KERNEL were set. */

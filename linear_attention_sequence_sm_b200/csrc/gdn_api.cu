@@ -253,12 +253,13 @@ static gdn_status_t chunk_forward_impl(const gdn_shape_t *s, const void *q, cons
         const SplitLayout SL = split_layout(*s);
         int32_t *cbase = reinterpret_cast<int32_t *>(ws + SL.cbase_off);
         __nv_bfloat16 *tinv = reinterpret_cast<__nv_bfloat16 *>(ws + SL.tinv_off);
+        float *gcum = reinterpret_cast<float *>(ws + SL.gcum_off);
         e = launch_schedule(*s, cu_seqlens, workspace, stream, cbase);
         if (e != cudaSuccess) return cuda_fail(e, "schedule kernel launch");
         a.sched.chunk_base = cbase;
-        e = launch_chunk_inverse(a, tinv, SL.max_chunks, stream, sms);
+        e = launch_chunk_inverse(a, tinv, gcum, SL.max_chunks, stream, sms);
         if (e != cudaSuccess) return cuda_fail(e, "chunk inverse launch");
-        e = launch_chunk_chain(a, tinv, SL.max_chunks, stream, sms);
+        e = launch_chunk_chain(a, tinv, gcum, SL.max_chunks, stream, sms);
         if (e != cudaSuccess) return cuda_fail(e, "tensor-core chunk loop launch");
         return GDN_OK;
     }

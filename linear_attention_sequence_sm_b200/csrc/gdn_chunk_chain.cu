@@ -14,7 +14,7 @@
 //
 // Every product is one tcgen05.mma stream with M = 128 rows (the value index
 // of the state, or the key index for W), fp32 accumulators in tensor memory:
-//   (W)   W^T  = K^T T'^T             128 x 64 x 64     prep issuer
+//   (W)   W^T  = K^T T'^T             128 x 64 x 64     warp 14
 //   (U~)  U~^T = V^T T''^T            128 x 64 x 64     warp 13
 //   (XU)  U^T  = U~^T - S W^T         128 x 64 x 128    warp 12   } the state's
 //   (S7)  S   += (U^T diag(lambda)) K 128 x 128 x 64    warp 12   } critical path
@@ -33,12 +33,15 @@
 //   epilogue warps (4-7)  after (XU): U^T -> bf16, U^T diag(lambda) -> bf16;
 //                         after (X1), (X6): O staged and stored by TMA; then the
 //                         state pass of columns 96-127 for the next chunk
-//   prep warps (8-11)     one chunk ahead, state-independent: gates (cp.async,
-//                         two chunks ahead), per-token scales, the mask P from
-//                         the Gram, the epilogue of W^T
+//   prep warps (8-11)     one chunk ahead, state-independent: per-token scales
+//                         from the chunk's prefix sums G (computed by the factor
+//                         kernel, which took the same sums for T'; they arrive
+//                         with T' and T''), the mask P from the Gram, the
+//                         epilogue of W^T
 //   warps 12, 13, 14, 15  lane 0 issues the products above (14: Gram and W)
 // Tiles: K and Q in a ring of three chunks, T' and T'' in two, W^T and P in
-// two, V in one.  Roles hand over through mbarriers; every wait is bounded,
+// two, V in one.  Tensor-memory loads of a role are issued together and waited
+// for once.  Roles hand over through mbarriers; every wait is bounded,
 // and a timeout records GDN_ERR_DEVICE_CHECK (bad_index -2) and ends the
 // kernel after its own tensor-core work has drained.  With
 // GDN_FLAG_QK_L2NORM the factors 1/||q_r||, 1/||k_r|| are folded into P, the
@@ -69,14 +72,13 @@ constexpr uint32_t kWPBytes = 24576, kWP_W = 0, kWP_P = 16384;        // [2]: W^
 constexpr uint32_t kOffWP = kOffT + 2 * kTBytes;                      // 131072
 constexpr uint32_t kOffV = kOffWP + 2 * kWPBytes;                     // 180224: V (2 atoms x 64 rows)
 constexpr uint32_t kOffOst = kOffV + 16384;                           // 196608: output tile, 64 tokens x 256 B
-constexpr uint32_t kOffGst = kOffOst + 16384;                         // 212992: gates [2][g, beta][64]
-constexpr uint32_t kOffVec = kOffGst + 2 * 512;                       // 214016: token vectors [4]
+constexpr uint32_t kOffVec = kOffOst + 16384;                         // 212992: token vectors [4]
 constexpr int kVecFloats = 10 * 64;
-constexpr uint32_t kOffBar = kOffVec + 4 * kVecFloats * 4;            // 224256
+constexpr uint32_t kOffBar = kOffVec + 4 * kVecFloats * 4;            // 223232
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 per-block limit");
 // token vectors of a chunk (floats)
-constexpr int kVecG = 0, kVecB = 64, kVecGam = 128, kVecLam = 192, kVecPr = 256, kVecPc = 320, kVecGo = 384,
+constexpr int kVecG = 0, kVecGam = 128, kVecLam = 192, kVecPr = 256, kVecPc = 320, kVecGo = 384,
               kVecIk = 448, kVecIq = 512, kVecRank1 = 576;
 
 // mbarriers (arrival count 1 unless noted)
@@ -120,21 +122,27 @@ __device__ __forceinline__ bool group_wait(bool poller, uint32_t bar, uint32_t p
 }
 
 // The state pass of columns [c0, c0 + 32 kSlices) of this thread's state row:
-// the bf16 copy (A operand of (XU), (X1)) and S <- gC S in place.
+// the bf16 copy (A operand of (XU), (X1)) and S <- gC S in place.  Slices are
+// read two at a time, with one wait per pair.
+__device__ __forceinline__ void state_slice(uint32_t tmem_row, int c, float gC, float (&v)[32]) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+    tmem_st16u(tmem_row + kColSb + uint32_t(c / 2), pk);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] *= gC;
+    tmem_st32(tmem_row + kColS + uint32_t(c), v);
+}
 template <int kSlices>
 __device__ __forceinline__ void state_pass(uint32_t tmem_row, int c0, float gC) {
 #pragma unroll
-    for (int p = 0; p < kSlices; ++p) {
-        float v[32];
-        tmem_ld32(tmem_row + kColS + uint32_t(c0 + 32 * p), v);
+    for (int p = 0; p < kSlices; p += 2) {
+        float v0[32], v1[32];
+        tmem_ld32(tmem_row + kColS + uint32_t(c0 + 32 * p), v0);
+        if (p + 1 < kSlices) tmem_ld32(tmem_row + kColS + uint32_t(c0 + 32 * p + 32), v1);
         tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
-        tmem_st16u(tmem_row + kColSb + uint32_t((c0 + 32 * p) / 2), pk);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] *= gC;
-        tmem_st32(tmem_row + kColS + uint32_t(c0 + 32 * p), v);
+        state_slice(tmem_row, c0 + 32 * p, gC, v0);
+        if (p + 1 < kSlices) state_slice(tmem_row, c0 + 32 * p + 32, gC, v1);
     }
     tmem_wait_st();
 }
@@ -171,11 +179,11 @@ __device__ __forceinline__ void state_out(uint32_t tmem_row, float *dst, int c0)
     }
 }
 
-template <bool kL2, bool kLogits>
+template <bool kL2>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                   const __grid_constant__ CUtensorMap tm_t, const PrefillArgs a) {
+                   const __grid_constant__ CUtensorMap tm_t, const PrefillArgs a, const float *gcum) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sb = smem_u32(smem);
@@ -239,14 +247,16 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             tma_load_3d(dst + kKQ_Q, &tm_q, 0, hq, tok, b);
             tma_load_3d(dst + kKQ_Q + 8192, &tm_q, 64, hq, tok, b);
         };
-        auto load_t = [&](int c) {  // T', T'' of chunk c
+        auto load_t = [&](int c) {  // T', T'' and the prefix sums G of chunk c
             const uint32_t gc = gn + uint32_t(c), i = gc & 1u;
             const uint32_t dst = sb + kOffT + i * kTBytes;
             const uint32_t b = bar(kBT + int(i));
-            mbar_arrive_expect_tx(b, kBytesT);
+            mbar_arrive_expect_tx(b, kBytesT + 256);
             const int row = ((cbase + c) * hv + h) * 128;
             tma_load_2d(dst + kT_P, &tm_t, 0, row, b);
             tma_load_2d(dst + kT_PP, &tm_t, 0, row + 64, b);
+            bulk_load(sb + kOffVec + (gc & 3u) * (kVecFloats * 4) + kVecG * 4,
+                      gcum + (size_t(cbase + c) * hv + h) * 64, 256, b);
         };
         auto load_v = [&](int c) {
             mbar_arrive_expect_tx(bar(kBV), kBytesV);
@@ -327,21 +337,26 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     if (named_sync_or(kBarEpi, 128, !ok)) { aborted = true; break; }
                 }
                 tc_fence_after();
-#pragma unroll
-                for (int p = 0; p < 2; ++p) {
-                    float v[32], l[32];
-                    tmem_ld32(trow + kColU + 32 * p, v);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) load4(vec + kVecLam + 32 * p + 4 * q, l + 4 * q);
+                {
+                    float v[2][32];
+                    tmem_ld32(trow + kColU, v[0]);
+                    tmem_ld32(trow + kColU + 32, v[1]);
                     tmem_wait_ld();
-                    uint32_t pu[16], pl[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        pu[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
-                        pl[j] = pack_bf16x2(l[2 * j] * v[2 * j], l[2 * j + 1] * v[2 * j + 1]);
+                    for (int p = 0; p < 2; ++p) {
+                        uint32_t pu[16], pl[16];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            float l[4];
+                            load4(vec + kVecLam + 32 * p + 4 * q, l);
+                            pu[2 * q] = pack_bf16x2(v[p][4 * q], v[p][4 * q + 1]);
+                            pu[2 * q + 1] = pack_bf16x2(v[p][4 * q + 2], v[p][4 * q + 3]);
+                            pl[2 * q] = pack_bf16x2(l[0] * v[p][4 * q], l[1] * v[p][4 * q + 1]);
+                            pl[2 * q + 1] = pack_bf16x2(l[2] * v[p][4 * q + 2], l[3] * v[p][4 * q + 3]);
+                        }
+                        tmem_st16u(trow + kColSb + 16 * p, pu);
+                        tmem_st16u(trow + kColSb + 32 + 16 * p, pl);
                     }
-                    tmem_st16u(trow + kColSb + 16 * p, pu);
-                    tmem_st16u(trow + kColSb + 32 + 16 * p, pl);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -414,54 +429,14 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // ============ prep warps: chunk n's state-independent operands ============
             const int pt = tid - 32 * kWarpPrep;  // 0..127
             const bool poller = warp == kWarpPrep;
-            // gates by cp.async, two chunks ahead: g then beta, 64 tokens each (zeros past the end)
-            auto prefetch_gates = [&](int c) {
-                const uint32_t dst = sb + kOffGst + ((gn + uint32_t(c)) & 1u) * 512;
-                const int L = min(64, len - 64 * c);
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int r = 2 * lane + q;
-                    const size_t i = size_t(t0 + 64 * c + min(r, L - 1)) * hv + h;
-                    cp_async_4(dst + 4 * r, a.g + i, r < L);
-                    cp_async_4(dst + 256 + 4 * r, a.beta + i, r < L);
-                }
-                cp_async_commit();
-            };
-            if (warp == kWarpPrep && nchunks > 0) {
-                prefetch_gates(0);
-                if (nchunks > 1) prefetch_gates(1);
-            }
             for (int n = 0; n < nchunks; ++n) {
                 const uint32_t gc = gn + uint32_t(n), b = gc & 1u;
                 const int L = min(64, len - 64 * n);
                 float *vec = vecs(gc);
                 const uint32_t kq = sb + kOffKQ + (gc % 3u) * kKQBytes;
                 const uint32_t wp = sb + kOffWP + b * kWPBytes;
-                // gates and their chunk-local prefix sums (tokens past the end: g = beta = 0)
-                if (warp == kWarpPrep) {
-                    if (n + 1 < nchunks) cp_async_wait_1();
-                    else cp_async_wait_all();
-                    __syncwarp();
-                    const float *gs = reinterpret_cast<const float *>(smem + kOffGst + b * 512);
-                    const float ga = gs[2 * lane], gb = gs[2 * lane + 1];
-                    const float ba = gs[64 + 2 * lane], bb = gs[64 + 2 * lane + 1];
-                    const bool ok0 = 2 * lane < L, ok1 = 2 * lane + 1 < L;
-                    const float g0 = ok0 ? fmaxf(kLogits ? log_sigmoid_fast(ga) : ga, kGFloor) : 0.f;
-                    const float g1 = ok1 ? fmaxf(kLogits ? log_sigmoid_fast(gb) : gb, kGFloor) : 0.f;
-                    vec[kVecB + 2 * lane] = ok0 ? (kLogits ? sigmoid_fast(ba) : ba) : 0.f;
-                    vec[kVecB + 2 * lane + 1] = ok1 ? (kLogits ? sigmoid_fast(bb) : bb) : 0.f;
-                    float incl = g0 + g1;
-#pragma unroll
-                    for (int d = 1; d < 32; d <<= 1) {
-                        const float tt = __shfl_up_sync(0xffffffffu, incl, d);
-                        if (lane >= d) incl += tt;
-                    }
-                    const float excl = incl - (g0 + g1);
-                    vec[kVecG + 2 * lane] = excl + g0;
-                    vec[kVecG + 2 * lane + 1] = excl + g0 + g1;
-                    __syncwarp();
-                    if (n + 2 < nchunks) prefetch_gates(n + 2);  // this buffer's next use
-                }
+                // the chunk's prefix sums G arrive with its T' and T''
+                if (!group_wait(poller, bar(kBT + int(b)), (gc >> 1) & 1u, kBarPrep, 128)) { aborted = true; break; }
                 if constexpr (kL2) {
                     // 1 / max(||x||, 1e-12) of the 64 k rows (pt 0..63) and q rows (pt 64..127)
                     if (!group_wait(warp == kWarpPrep + 1, bar(kBKQ + int(gc % 3u)), (gc / 3u) & 1u, kBarPrep, 128)) {
@@ -486,9 +461,9 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             }
                         vec[(pt < 64 ? kVecIk : kVecIq) + R] = inv_l2(ss);
                     }
+                    named_sync(kBarPrep, 128);
                 }
-                named_sync(kBarPrep, 128);
-                // per-token scales (tokens past the end: lambda = beta = 0)
+                // per-token scales (tokens past the end: lambda = 0)
                 if (pt < 64) {
                     const float G = vec[kVecG + pt], gam = __expf(G);
                     const float ik = kL2 ? vec[kVecIk + pt] : 1.f, iq = kL2 ? vec[kVecIq + pt] : 1.f;
@@ -516,35 +491,43 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     const bool valid = lane < 16;
                     const bool rank1 = vec[kVecRank1] != 0.f;
                     const float pr = vec[kVecPr + r], Gr = vec[kVecG + r];
+                    // the warp's slices two at a time: both tensor-memory loads, one wait
 #pragma unroll
-                    for (int sl = 0; sl < 4; ++sl) {
-                        const int j0 = 16 * sl;
-                        float x[16];
-                        if (sl > quarter) {  // warp-uniform: every entry has j > r
+                    for (int s2 = 0; s2 < 4; s2 += 2) {
+                        float v[2][16];
 #pragma unroll
-                            for (int jj = 0; jj < 16; ++jj) x[jj] = 0.f;
-                        } else {
-                            float v[16], pc[16];
-                            tmem_ld16(tmem + lane_bits + kColGram + uint32_t(j0), v);
+                        for (int u = 0; u < 2; ++u)
+                            if (s2 + u <= quarter) tmem_ld16(tmem + lane_bits + kColGram + uint32_t(16 * (s2 + u)), v[u]);
+                        if (s2 <= quarter) tmem_wait_ld();
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) load4(vec + kVecPc + j0 + 4 * q, pc + 4 * q);
-                            tmem_wait_ld();
-                            if (rank1) {
+                        for (int u = 0; u < 2; ++u) {
+                            const int sl = s2 + u, j0 = 16 * sl;
+                            float x[16];
+                            if (sl > quarter) {  // warp-uniform: every entry has j > r
 #pragma unroll
-                                for (int jj = 0; jj < 16; ++jj) x[jj] = (j0 + jj <= r) ? pr * pc[jj] * v[jj] : 0.f;
+                                for (int jj = 0; jj < 16; ++jj) x[jj] = 0.f;
                             } else {
-                                float gj[16];
+                                float pc[16];
 #pragma unroll
-                                for (int q = 0; q < 4; ++q) load4(vec + kVecG + j0 + 4 * q, gj + 4 * q);
+                                for (int q = 0; q < 4; ++q) load4(vec + kVecPc + j0 + 4 * q, pc + 4 * q);
+                                if (rank1) {
 #pragma unroll
-                                for (int jj = 0; jj < 16; ++jj)
-                                    x[jj] = (j0 + jj <= r) ? pr * pc[jj] * __expf(fminf(Gr - gj[jj], 0.f)) * v[jj] : 0.f;
+                                    for (int jj = 0; jj < 16; ++jj) x[jj] = (j0 + jj <= r) ? pr * pc[jj] * v[u][jj] : 0.f;
+                                } else {
+                                    float gj[16];
+#pragma unroll
+                                    for (int q = 0; q < 4; ++q) load4(vec + kVecG + j0 + 4 * q, gj + 4 * q);
+#pragma unroll
+                                    for (int jj = 0; jj < 16; ++jj)
+                                        x[jj] = (j0 + jj <= r) ? pr * pc[jj] * __expf(fminf(Gr - gj[jj], 0.f)) * v[u][jj]
+                                                               : 0.f;
+                                }
                             }
-                        }
-                        if (valid) {
-                            const uint32_t base = wp + kWP_P + uint32_t(r) * 128;
-                            st_shared_v4(base + (uint32_t((2 * sl) ^ (r & 7)) << 4), pack_bf16x8(x));
-                            st_shared_v4(base + (uint32_t((2 * sl + 1) ^ (r & 7)) << 4), pack_bf16x8(x + 8));
+                            if (valid) {
+                                const uint32_t base = wp + kWP_P + uint32_t(r) * 128;
+                                st_shared_v4(base + (uint32_t((2 * sl) ^ (r & 7)) << 4), pack_bf16x8(x));
+                                st_shared_v4(base + (uint32_t((2 * sl + 1) ^ (r & 7)) << 4), pack_bf16x8(x + 8));
+                            }
                         }
                     }
                 }
@@ -556,15 +539,15 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 {
                     const int c = (warp & 3) * 32 + lane;  // d_k index = tensor-memory lane
                     const uint32_t base = wp + kWP_W + uint32_t(c) * 128;
+                    float v[2][32];
+                    tmem_ld32(tmem + lane_bits + kColW, v[0]);
+                    tmem_ld32(tmem + lane_bits + kColW + 32, v[1]);
+                    tmem_wait_ld();
 #pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        float v[32];
-                        tmem_ld32(tmem + lane_bits + kColW + 32 * p, v);
-                        tmem_wait_ld();
+                    for (int p = 0; p < 2; ++p)
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
-                            st_shared_v4(base + (uint32_t((4 * p + q) ^ (c & 7)) << 4), pack_bf16x8(v + 8 * q));
-                    }
+                            st_shared_v4(base + (uint32_t((4 * p + q) ^ (c & 7)) << 4), pack_bf16x8(v[p] + 8 * q));
                 }
                 fence_proxy_async_shared();
                 tc_fence_before();
@@ -694,7 +677,6 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
 
     if (warp >= kWarpEpi && warp < kWarpPrep && tid == 32 * kWarpEpi) bulk_wait_all();
-    if (warp == kWarpPrep) cp_async_wait_all();
     if (aborted) {
         // let this thread's own tensor-core work drain (bounded) before the tensor
         // memory is freed
@@ -720,18 +702,19 @@ bool chunk_split_supported(const gdn_shape_t &s) {
     return s.dtype == GDN_DTYPE_BF16 && s.head_dim_k == 128 && s.head_dim_v == 128 && s.chunk_size == 64;
 }
 
-cudaError_t launch_chunk_chain(const PrefillArgs &a, const __nv_bfloat16 *tinv, int64_t max_chunks,
-                               cudaStream_t stream, int num_sms) {
+cudaError_t launch_chunk_chain(const PrefillArgs &a, const __nv_bfloat16 *tinv, const float *gcum,
+                               int64_t max_chunks, cudaStream_t stream, int num_sms) {
     CUtensorMap mq, mk, mv, mo, mt;
     if (!make_map(&mq, a.q, a.hk, a.tokens) || !make_map(&mk, a.k, a.hk, a.tokens) ||
         !make_map(&mv, a.v, a.hv, a.tokens) || !make_map(&mo, a.o, a.hv, a.tokens, true) ||
         !make_tile_map(&mt, tinv, max_chunks * a.hv * 128))
         return cudaErrorInvalidValue;
-    const bool l2 = a.flags & GDN_FLAG_QK_L2NORM, logits = a.flags & GDN_FLAG_GATE_LOGITS;
-    using KernFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, PrefillArgs);
-    static const KernFn table[4] = {chunk_chain_kernel<false, false>, chunk_chain_kernel<false, true>,
-                                    chunk_chain_kernel<true, false>, chunk_chain_kernel<true, true>};
-    const KernFn kern = table[(l2 ? 2 : 0) + (logits ? 1 : 0)];
+    // (the gate logits were turned into decays by the chunk-factor kernel, which
+    // hands over the prefix sums G)
+    const bool l2 = a.flags & GDN_FLAG_QK_L2NORM;
+    using KernFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, PrefillArgs,
+                            const float *);
+    const KernFn kern = l2 ? chunk_chain_kernel<true> : chunk_chain_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
     if (e != cudaSuccess) return e;
     const int64_t units = int64_t(a.num_seqs) * a.hv;
@@ -747,7 +730,7 @@ cudaError_t launch_chunk_chain(const PrefillArgs &a, const __nv_bfloat16 *tinv, 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, mt, a);
+    e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, mt, a, gcum);
     count_launch();
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

@@ -129,7 +129,8 @@ __device__ __forceinline__ int seq_of_chunk(const int32_t *chunk_base, int num_s
 
 template <bool kL2, bool kLogits>
 __global__ void __launch_bounds__(kThreads, 3)
-chunk_inverse_kernel(const __grid_constant__ CUtensorMap tm_k, const PrefillArgs a, __nv_bfloat16 *tinv) {
+chunk_inverse_kernel(const __grid_constant__ CUtensorMap tm_k, const PrefillArgs a, __nv_bfloat16 *tinv,
+                     float *gcum) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sb = smem_u32(smem);
@@ -276,6 +277,9 @@ chunk_inverse_kernel(const __grid_constant__ CUtensorMap tm_k, const PrefillArgs
                 const float excl = incl - (g0 + g1);
                 vec[kVecG + 2 * lane] = excl + g0;
                 vec[kVecG + 2 * lane + 1] = excl + g0 + g1;
+                // the chunk loop takes its decays from these same sums
+                reinterpret_cast<float2 *>(gcum + (size_t(gc) * hv + h) * 64)[lane] =
+                    make_float2(excl + g0, excl + g0 + g1);
             }
             __syncthreads();
             // row and column scales of the mask.  While the chunk's total log-decay
@@ -393,12 +397,12 @@ chunk_inverse_kernel(const __grid_constant__ CUtensorMap tm_k, const PrefillArgs
 
 }  // namespace
 
-cudaError_t launch_chunk_inverse(const PrefillArgs &a, __nv_bfloat16 *tinv, int64_t max_chunks, cudaStream_t stream,
-                                 int num_sms) {
+cudaError_t launch_chunk_inverse(const PrefillArgs &a, __nv_bfloat16 *tinv, float *gcum, int64_t max_chunks,
+                                 cudaStream_t stream, int num_sms) {
     CUtensorMap mk;
     if (!make_map(&mk, a.k, a.hk, a.tokens)) return cudaErrorInvalidValue;
     const bool l2 = a.flags & GDN_FLAG_QK_L2NORM, logits = a.flags & GDN_FLAG_GATE_LOGITS;
-    using KernFn = void (*)(CUtensorMap, PrefillArgs, __nv_bfloat16 *);
+    using KernFn = void (*)(CUtensorMap, PrefillArgs, __nv_bfloat16 *, float *);
     static const KernFn table[4] = {chunk_inverse_kernel<false, false>, chunk_inverse_kernel<false, true>,
                                     chunk_inverse_kernel<true, false>, chunk_inverse_kernel<true, true>};
     const KernFn kern = table[(l2 ? 2 : 0) + (logits ? 1 : 0)];
@@ -418,7 +422,7 @@ cudaError_t launch_chunk_inverse(const PrefillArgs &a, __nv_bfloat16 *tinv, int6
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, mk, a, tinv);
+    e = cudaLaunchKernelEx(&cfg, kern, mk, a, tinv, gcum);
     count_launch();
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

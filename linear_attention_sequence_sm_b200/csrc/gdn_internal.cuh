@@ -71,11 +71,14 @@ inline WsLayout ws_layout(int32_t num_seqs) {
 //   tinv                  per (chunk, value head) T' = T diag(beta gamma) and
 //                         T'' = T diag(beta) of the chunk's WY factor
 //                         T = (I + A)^-1, bf16 row-major, [max_chunks][Hv][2][64][64]
+//   gcum                  per (chunk, value head) the chunk-local prefix sums G
+//                         of the log-decay (tokens past the end carry g = 0),
+//                         fp32 [max_chunks][Hv][64]
 // max_chunks bounds the chunk count for the shape: (tokens + 63 N) / 64 (each
 // sequence adds at most one partial chunk).
 struct SplitLayout {
     WsLayout sched;
-    size_t cbase_off, tinv_off, total;
+    size_t cbase_off, tinv_off, gcum_off, total;
     int64_t max_chunks;
 };
 
@@ -94,6 +97,8 @@ inline SplitLayout split_layout(const gdn_shape_t &s) {
     L.tinv_off = off;
     L.max_chunks = max_chunks_bound(s);
     off += size_t(L.max_chunks) * size_t(s.num_v_heads) * 2 * 64 * 64 * 2;
+    L.gcum_off = off;
+    off += size_t(L.max_chunks) * size_t(s.num_v_heads) * 64 * 4;
     L.total = align256(off);
     return L;
 }
@@ -217,10 +222,10 @@ bool chunk_tc_supported(const gdn_shape_t &s);
 // state-carrying chunk loop that reads them (gdn_chunk_chain.cu).  Both are
 // programmatic dependents of the schedule kernel, which fills chunk_base.
 bool chunk_split_supported(const gdn_shape_t &s);
-cudaError_t launch_chunk_inverse(const PrefillArgs &a, __nv_bfloat16 *tinv, int64_t max_chunks, cudaStream_t stream,
-                                 int num_sms);
-cudaError_t launch_chunk_chain(const PrefillArgs &a, const __nv_bfloat16 *tinv, int64_t max_chunks,
-                               cudaStream_t stream, int num_sms);
+cudaError_t launch_chunk_inverse(const PrefillArgs &a, __nv_bfloat16 *tinv, float *gcum, int64_t max_chunks,
+                                 cudaStream_t stream, int num_sms);
+cudaError_t launch_chunk_chain(const PrefillArgs &a, const __nv_bfloat16 *tinv, const float *gcum,
+                               int64_t max_chunks, cudaStream_t stream, int num_sms);
 
 // The output side as its own pass over o, in place (for the CUDA-core prefill,
 // whose blocks each own a slice of d_v).
