@@ -132,6 +132,23 @@ typedef struct {
  * if GDN_FLAG_ONE_KERNEL were set. */
 GDN_API gdn_status_t gdn_chunk_forward_workspace_size(const gdn_shape_t *shape, size_t *bytes);
 
+/* Kernel paths of gdn_chunk_forward. */
+#define GDN_PATH_SIMT 0          /* fp32 CUDA-core kernel                      */
+#define GDN_PATH_TC_ONE_KERNEL 1 /* single tensor-core kernel                  */
+#define GDN_PATH_TC_SPLIT 2      /* two-kernel tensor-core form (chunk factors
+                                    for all chunks, then the chunk loop)      */
+
+/* Which path gdn_chunk_forward takes for `shape` with a workspace of
+ * `workspace_bytes` on the current device, written to *path (a GDN_PATH_*
+ * value).  The page has no counterpart for this query: it lets a caller see
+ * that a shape runs on the CUDA cores (an fp32 or non-128 head size, or the
+ * flags), or that a workspace below the two-kernel size kept a shape of
+ * value heads not a multiple of 4 off the tensor cores.  Errors: those of
+ * gdn_chunk_forward_workspace_size, GDN_ERR_WORKSPACE_TOO_SMALL below the
+ * minimum workspace, GDN_ERR_CUDA without a usable device.  Launches
+ * nothing. */
+GDN_API gdn_status_t gdn_chunk_forward_path(const gdn_shape_t *shape, size_t workspace_bytes, int32_t *path);
+
 /* Chunkwise prefill ("Gated Attention Architectures", sections 2 and 3: the
  * WY representation of the generalised Householder transitions, extended
  * with per-chunk cumulative decay products, and the decay-masked chunk

@@ -80,6 +80,19 @@ static bool wants_split(const gdn_shape_t &s) {
     return (s.flags & GDN_FLAG_SPLIT) || !chunk_tc_supported(s);
 }
 
+// The kernel path of a prefill call (GDN kernels; KDA has its own).  One
+// function serves the call and the path query, so the two cannot disagree.
+static int32_t select_path(const gdn_shape_t &s, int major, bool out_side, size_t workspace_bytes) {
+    const int64_t tokens = int64_t(s.batch) * s.seq_len;
+    const bool tc_arch = major == 10 && !(s.flags & GDN_FLAG_FORCE_SIMT);
+    // the two-kernel form needs the full queried workspace (it keeps every
+    // chunk's factors there) and has no output side
+    if (tc_arch && tokens > 0 && !out_side && wants_split(s) && workspace_bytes >= split_layout(s).total)
+        return GDN_PATH_TC_SPLIT;
+    if (tc_arch && chunk_tc_supported(s)) return GDN_PATH_TC_ONE_KERNEL;
+    return GDN_PATH_SIMT;
+}
+
 static gdn_status_t check_output_side(const gdn_output_side_t *os, OutSide *out) {
     *out = OutSide{nullptr, nullptr, 0.f, 0u};
     if (!os) return GDN_OK;
@@ -138,6 +151,20 @@ gdn_status_t gdn_chunk_forward_workspace_size(const gdn_shape_t *s, size_t *byte
     gdn_status_t st = check_shape(s);
     if (st != GDN_OK) return st;
     *bytes = wants_split(*s) ? split_layout(*s).total : ws_layout(s->num_seqs).total;
+    return GDN_OK;
+}
+
+gdn_status_t gdn_chunk_forward_path(const gdn_shape_t *s, size_t workspace_bytes, int32_t *path) {
+    g_msg[0] = 0;
+    if (!path) return fail(GDN_ERR_INVALID_ARGUMENT, "path is NULL");
+    gdn_status_t st = check_shape(s);
+    if (st != GDN_OK) return st;
+    const size_t need = ws_layout(s->num_seqs).total;
+    if (workspace_bytes < need)
+        return fail(GDN_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+    int major = 0;
+    if (device_sm_count(&major) <= 0) return fail(GDN_ERR_CUDA, "no usable CUDA device");
+    *path = select_path(*s, major, false, workspace_bytes);
     return GDN_OK;
 }
 
@@ -242,13 +269,8 @@ static gdn_status_t chunk_forward_impl(const gdn_shape_t *s, const void *q, cons
         }
         return GDN_OK;
     }
-    const bool tc_arch = major == 10 && !(s->flags & GDN_FLAG_FORCE_SIMT);
-    // The two-kernel tensor-core path needs the full queried workspace (it keeps
-    // every chunk's inverse there); with less, or with the output side, the
-    // single-kernel tensor-core path runs where it applies.
-    const bool use_split =
-        tc_arch && tokens > 0 && !out.flags && wants_split(*s) && workspace_bytes >= split_layout(*s).total;
-    const bool use_tc = !use_split && tc_arch && chunk_tc_supported(*s);
+    const int32_t path = select_path(*s, major, out.flags != 0, workspace_bytes);
+    const bool use_split = path == GDN_PATH_TC_SPLIT, use_tc = path == GDN_PATH_TC_ONE_KERNEL;
     if (use_split) {
         const SplitLayout SL = split_layout(*s);
         int32_t *cbase = reinterpret_cast<int32_t *>(ws + SL.cbase_off);

@@ -44,7 +44,12 @@ EXPORTED = ("gdn_chunk_forward_workspace_size", "gdn_chunk_forward", "gdn_read_d
             "gdn_decode_step", "gdn_status_string", "gdn_last_error_message", "gdn_launch_count",
             "gdn_chunk_forward_noalloc", "gdn_decode_step_ex", "gdn_chunk_forward_out", "gdn_decode_step_out",
             "gdn_kda_forward", "gdn_kda_decode_step", "gdn_decode_multi", "gdn_decode_commit",
-            "gdn_chunk_backward_workspace_size", "gdn_chunk_backward", "gdn_short_conv")
+            "gdn_chunk_backward_workspace_size", "gdn_chunk_backward", "gdn_short_conv",
+            "gdn_chunk_forward_path")
+GDN_PATH_SIMT = 0
+GDN_PATH_TC_ONE_KERNEL = 1
+GDN_PATH_TC_SPLIT = 2
+PATH_NAMES = {GDN_PATH_SIMT: "simt", GDN_PATH_TC_ONE_KERNEL: "tc_one_kernel", GDN_PATH_TC_SPLIT: "tc_split"}
 
 
 class GdnError(RuntimeError):
@@ -73,6 +78,8 @@ def _load(path: str = LIB_PATH):
     vp, i32, st = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int
     lib.gdn_chunk_forward_workspace_size.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(ctypes.c_size_t)]
     lib.gdn_chunk_forward_workspace_size.restype = st
+    lib.gdn_chunk_forward_path.argtypes = [ctypes.POINTER(Shape), ctypes.c_size_t, ctypes.POINTER(ctypes.c_int32)]
+    lib.gdn_chunk_forward_path.restype = st
     lib.gdn_chunk_forward.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                       ctypes.c_size_t, vp]
     lib.gdn_chunk_forward.restype = st
@@ -259,6 +266,17 @@ def make_shape(q, v, cu_seqlens=None, chunk_size=64, force_simt=False, flags=0, 
     return Shape(B, T, N, q.shape[-2], v.shape[-2], q.shape[-1], v.shape[-1], chunk_size, _dtype_code(q),
                  (GDN_FLAG_FORCE_SIMT if force_simt else 0) | (GDN_FLAG_ONE_KERNEL if one_kernel else 0) |
                  (GDN_FLAG_SPLIT if split else 0) | flags)
+
+
+def forward_path(shape: Shape, workspace_bytes: int | None = None) -> str:
+    """The kernel path gdn_chunk_forward takes for ``shape`` on the current
+    device ("simt", "tc_one_kernel" or "tc_split"), with a workspace of
+    ``workspace_bytes`` (default: the queried size)."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace_size(shape)
+    p = ctypes.c_int32(-1)
+    _check(LIB.gdn_chunk_forward_path(ctypes.byref(shape), ctypes.c_size_t(workspace_bytes), ctypes.byref(p)))
+    return PATH_NAMES[p.value]
 
 
 def workspace_size(shape: Shape) -> int:

@@ -76,6 +76,24 @@ def test_workspace_size_follows_the_path(gdn):
     assert gdn.workspace_size(_shape(gdn, flags=gdn.GDN_FLAG_SPLIT, **dict(kw, dtype=gdn.GDN_DTYPE_F32))) == one
 
 
+def test_path_query_arguments(gdn):
+    """The path query checks its arguments before it looks for a device (this
+    host has none, so a well-formed query reports GDN_ERR_CUDA)."""
+    p = ctypes.c_int32(-1)
+    s = _shape(gdn)
+    assert gdn.LIB.gdn_chunk_forward_path(ctypes.byref(s), ctypes.c_size_t(1 << 20), None) == \
+        gdn.GDN_ERR_INVALID_ARGUMENT
+    assert gdn.LIB.gdn_chunk_forward_path(ctypes.byref(s), ctypes.c_size_t(0), ctypes.byref(p)) == \
+        gdn.GDN_ERR_WORKSPACE_TOO_SMALL
+    bad = _shape(gdn, num_v_heads=3)
+    assert gdn.LIB.gdn_chunk_forward_path(ctypes.byref(bad), ctypes.c_size_t(1 << 20), ctypes.byref(p)) == \
+        gdn.GDN_ERR_INVALID_ARGUMENT
+    import torch
+    if not torch.cuda.is_available():
+        st = gdn.LIB.gdn_chunk_forward_path(ctypes.byref(s), ctypes.c_size_t(gdn.workspace_size(s)), ctypes.byref(p))
+        assert st == gdn.GDN_ERR_CUDA and p.value == -1
+
+
 def test_contradictory_path_flags_rejected(gdn):
     n = ctypes.c_size_t(0)
     s = _shape(gdn, flags=gdn.GDN_FLAG_SPLIT | gdn.GDN_FLAG_ONE_KERNEL)

@@ -216,3 +216,41 @@ def test_full_size_long_context_all_units():
     """The 65,536-token, 16/48-head (3 value heads per q/k head), d=128, C=64
     bf16 workload with initial states, at full size, every unit."""
     _check(I.long_bf16(), "default")
+
+
+def test_path_query_matches_the_launches():
+    """gdn_chunk_forward_path names the path the call then takes: one launch
+    after the schedule for a single kernel, two for the two-kernel form.  Value
+    heads not a multiple of 4 take the two-kernel form with the queried
+    workspace and the CUDA-core kernel with only the single-kernel size."""
+    import ctypes
+    from linear_attention_sequence_sm_b200 import gdn
+    dev = torch.device("cuda:0")
+
+    def run(hk, hv, dtype, small=False, **kw):
+        w = I.custom(f"path_{hk}_{hv}", batch=1, seq_len=130, hk=hk, hv=hv, d=128, chunk=64, dtype=dtype, seed=71)
+        inp = I.make_prefill_inputs(w)
+        d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+        shape = gdn.make_shape(d["q"], d["v"], None, 64, **kw)
+        nbytes = gdn.workspace_size(gdn.make_shape(d["q"], d["v"], None, 64, one_kernel=True)) if small else \
+            gdn.workspace_size(shape)
+        path = gdn.forward_path(shape, nbytes)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        o = torch.empty_like(d["v"])
+        p = lambda t: ctypes.c_void_p(t.data_ptr())
+        n0 = gdn.launch_count()
+        st = gdn.LIB.gdn_chunk_forward(ctypes.byref(shape), p(d["q"]), p(d["k"]), p(d["v"]), p(d["g"]), p(d["beta"]),
+                                       None, None, p(o), None, p(ws), nbytes,
+                                       ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        torch.cuda.synchronize()
+        assert st == gdn.GDN_OK and gdn.read_device_status(ws) == gdn.GDN_OK
+        assert torch.isfinite(o.float()).all()
+        return path, gdn.launch_count() - n0
+
+    assert run(2, 8, "bf16") == ("tc_one_kernel", 2)
+    assert run(2, 8, "bf16", split=True) == ("tc_split", 3)
+    assert run(2, 6, "bf16") == ("tc_split", 3)
+    assert run(2, 6, "bf16", small=True) == ("simt", 2)
+    assert run(2, 6, "bf16", one_kernel=True) == ("simt", 2)
+    assert run(2, 8, "f32") == ("simt", 2)
+    assert run(2, 8, "bf16", force_simt=True) == ("simt", 2)
