@@ -72,6 +72,9 @@ def parse_args(argv=None):
                         "of the prefill workload instead of the mixer (HBM roofline)")
     p.add_argument("--mtp", type=int, default=0,
                    help="decode: verify K draft tokens per sequence in one pass (state after every token kept)")
+    p.add_argument("--split", action="store_true",
+                   help="prefill through the two-kernel tensor-core form (chunk factors for all chunks, then the "
+                        "chunk loop) instead of the default single kernel")
     p.add_argument("--no-graph", action="store_true",
                    help="decode: launch each step instead of replaying the ring of steps as one CUDA graph")
     p.add_argument("--no-e2e", action="store_true")
@@ -108,12 +111,16 @@ def kernel_traffic(kernel: str):
     e = entries.get(kernel)
     if not e:
         return None
-    src = os.path.join(ROOT, e["source"])
-    if not os.path.exists(src):
-        return None
-    with open(src, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()
-    return e["bytes_per_launch"] if sha == e["source_sha256"] else None
+    # one source, or several (a path of more than one kernel): all unchanged
+    sources = e.get("sources") or [{"source": e["source"], "source_sha256": e["source_sha256"]}]
+    for item in sources:
+        src = os.path.join(ROOT, item["source"])
+        if not os.path.exists(src):
+            return None
+        with open(src, "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != item["source_sha256"]:
+                return None
+    return e["bytes_per_launch"]
 
 
 class ClockSampler:
@@ -360,7 +367,8 @@ def prefill_record(args, w, host, device, world, rank, peaks, peak_src, e2e=True
     from linear_attention_sequence_sm_b200 import gdn
     from linear_attention_sequence_sm_b200 import inputs as I
     flags = {"qk_l2norm": True, "gate_logits": True} if args.raw_inputs else {}
-    suffix = ("_kda" if args.kda else "") + ("_raw_inputs" if args.raw_inputs else "") + \
+    suffix = ("_kda" if args.kda else "") + ("_split" if args.split else "") + \
+        ("_raw_inputs" if args.raw_inputs else "") + \
         ("_output_norm" if args.output_norm else "") + ("_backward" if args.backward else "") + \
         (f"_conv{args.conv}" if args.conv else "")
     if args.kda:
@@ -379,7 +387,8 @@ def prefill_record(args, w, host, device, world, rank, peaks, peak_src, e2e=True
 
     o = torch.empty_like(dev["v"])
     sf = torch.empty((w.num_seqs, w.hv, w.d, w.d), dtype=torch.float32, device=device)
-    shape = gdn.make_shape(dev["q"], dev["v"], dev["cu_seqlens"], w.chunk)
+    split = {"split": True} if args.split and not args.kda else {}
+    shape = gdn.make_shape(dev["q"], dev["v"], dev["cu_seqlens"], w.chunk, **split)
     ws = torch.empty(gdn.workspace_size(shape), dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
 
@@ -408,7 +417,7 @@ def prefill_record(args, w, host, device, world, rank, peaks, peak_src, e2e=True
             return
         fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], initial_state=dev["initial_state"],
             cu_seqlens=dev["cu_seqlens"], out=o, final_state=sf, workspace=ws, chunk_size=w.chunk,
-            **flags, **out_norm(dev))
+            **flags, **out_norm(dev), **split)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -430,8 +439,10 @@ def prefill_record(args, w, host, device, world, rank, peaks, peak_src, e2e=True
     # multiples of 4, else the two-kernel form (chunk factors, then the chunk loop)
     if not gdn_tc_active(gdn, dev, w):
         kernel_name = "gdn_chunk_simt"
+    elif w.hv % 4 == 0 and not split:
+        kernel_name = "gdn_chunk_tc"
     else:
-        kernel_name = "gdn_chunk_tc" if w.hv % 4 == 0 else "gdn_chunk_inverse+gdn_chunk_chain"
+        kernel_name = "gdn_chunk_inverse+gdn_chunk_chain"
     roofline = {"bound": "tensor", "achieved": achieved_tflops, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved_tflops / peaks["bf16_tflops"],
                 "traffic": kernel_traffic(f"{kernel_name}/{w.name}{suffix}"),
