@@ -529,9 +529,11 @@ gdn_status_t gdn_short_conv(int32_t num_seqs, int32_t seq_len, const int32_t *cu
         return fail(GDN_ERR_INVALID_ARGUMENT, "dtype %d is not GDN_DTYPE_F32 or GDN_DTYPE_BF16", dtype);
     if (width < 1 || width > 8) return fail(GDN_ERR_UNSUPPORTED, "convolution width %d not in 1..8", width);
     if (channels % 4 != 0) return fail(GDN_ERR_UNSUPPORTED, "channels (%d) must be a multiple of 4", channels);
-    if (int64_t(channels) / 4 > int64_t(65535) * 128)
-        return fail(GDN_ERR_UNSUPPORTED, "too many channels (%d)", channels);
     if (tokens > INT32_MAX) return fail(GDN_ERR_UNSUPPORTED, "more than 2^31-1 tokens");
+    // at most one thread per token and 4 channels, 256 threads a block, in a 1-D grid
+    if (tokens * (int64_t(channels) / 4) / 256 >= int64_t(INT32_MAX))
+        return fail(GDN_ERR_UNSUPPORTED, "too many (token, channel) groups: %lld tokens x %d channels",
+                    static_cast<long long>(tokens), channels);
     if (!cu_seqlens && int64_t(num_seqs) * seq_len != tokens)
         return fail(GDN_ERR_INVALID_ARGUMENT, "tokens (%lld) must equal num_seqs * seq_len without cu_seqlens",
                     (long long)tokens);

@@ -10,25 +10,28 @@
 // zero; the state after each sequence (its last W-1 inputs) is returned so
 // that decode can continue.
 //
-// HBM-bound: one read of x and one write of y.  A thread owns a segment of
-// kConvSeg tokens of the packed layout and 4 consecutive channels (one 8- or
-// 16-byte vector per token, coalesced across the warp).  It finds the
-// sequence of its first token by binary search over the sequence starts,
-// fills its W-1 token history from the inputs before the segment (or the
-// state), and walks its tokens, resetting the history at each sequence start
-// and writing the state after each sequence's last token.  Loads run
-// kConvPre tokens ahead.  Empty sequences pass their state through in a
-// second, small kernel.  Every index is bounded by the sizes, so contents of
-// cu_seqlens that break its contract give unspecified values, never an
-// access out of bounds.
+// HBM-bound: one read of x and one write of y.  The work is spread for
+// memory-level parallelism: a thread owns kConvTok consecutive tokens of the
+// packed layout and 4 consecutive channels (one 8- or 16-byte vector per
+// token; consecutive threads take consecutive channel groups, so a warp reads
+// whole rows), loads its W-1+kConvTok input rows at once (the W-1 halo rows
+// come again from L1/L2, not from HBM), and finds the sequence of each of its
+// tokens by binary search over the sequence starts, stepping on at sequence
+// boundaries.  A tap before its token's sequence start reads the sequence's
+// conv state (or zero).  The thread holding a sequence's last token writes
+// the sequence's conv state, its last W-1 inputs (reaching into the incoming
+// state when the sequence is shorter); a small second kernel passes the state
+// of empty sequences through.  Weights of width 4 arrive as one 16-byte load
+// per channel: the load/store pipe, not DRAM, is what this kernel runs out of
+// first, so it is fed few and wide instructions.  Every index is bounded by
+// the sizes, so contents of cu_seqlens that break its contract give
+// unspecified values, never an access out of bounds.
 #include "gdn_internal.cuh"
 
 namespace gdn {
 
-constexpr int kConvSeg = 64;      // tokens per thread
-constexpr int kConvPre = 8;       // tokens loaded ahead
-constexpr int kConvThreads = 128; // 4 channels each: 512 channels per block
-
+constexpr int kConvTok = 8;         // tokens per thread
+constexpr int kConvThreads = 256;
 struct ConvArgs {
     const int32_t *cu;  // [N + 1], or NULL: N sequences of seq_len tokens
     int32_t n, seq_len, tokens, channels;
@@ -66,23 +69,54 @@ __device__ __forceinline__ void store4(__nv_bfloat16 *p, const float (&v)[4]) {
     *reinterpret_cast<uint2 *>(p) = u;
 }
 
+// xr[i][e] for a row index known only at run time (the boundary path; the
+// compiler keeps the array in registers and selects)
+template <int R>
+__device__ __forceinline__ float xr_at(const float (&xr)[R][4], int i, int e) {
+    float v = 0.f;
+#pragma unroll
+    for (int k = 0; k < R; ++k) v = (k == i) ? xr[k][e] : v;
+    return v;
+}
+
 template <typename T, int W>
-__global__ void __launch_bounds__(kConvThreads) short_conv_kernel(const ConvArgs a) {
-    constexpr int H = W - 1;
-    const int64_t c0 = (int64_t(blockIdx.y) * kConvThreads + threadIdx.x) * 4;
-    if (c0 >= a.channels) return;
-    const int32_t t0 = int32_t(blockIdx.x) * kConvSeg;
+__global__ void __launch_bounds__(kConvThreads, 3) short_conv_kernel(const ConvArgs a) {
+    constexpr int H = W - 1, R = H + kConvTok;
+    const int64_t cgs = a.channels / 4;
+    const int64_t idx = int64_t(blockIdx.x) * kConvThreads + threadIdx.x;
+    const int64_t tg = idx / cgs;
+    const int64_t c0 = (idx - tg * cgs) * 4;
+    const int64_t t0 = tg * kConvTok;
     if (t0 >= a.tokens) return;
-    const int32_t t1 = min(t0 + kConvSeg, a.tokens);
     const T *x = static_cast<const T *>(a.x);
     T *y = static_cast<T *>(a.y);
     const int64_t C = a.channels;
 
+    // input rows t0 - H .. t0 + kConvTok - 1 (zeros outside 0 .. tokens - 1), all loads first
+    float xr[R][4];
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+        const int64_t u = t0 - H + i;
+        if (u >= 0 && u < a.tokens) {
+            load4(x + u * C + c0, xr[i]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) xr[i][e] = 0.f;
+        }
+    }
     float w[4][W];
+    if constexpr (W == 4) {  // one 16-byte load per channel (rows of 4 taps are 16-byte aligned)
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
+        for (int e = 0; e < 4; ++e) {
+            const float4 f = *reinterpret_cast<const float4 *>(a.w + (c0 + e) * 4);
+            w[e][0] = f.x; w[e][1] = f.y; w[e][2] = f.z; w[e][3] = f.w;
+        }
+    } else {
 #pragma unroll
-        for (int j = 0; j < W; ++j) w[e][j] = a.w[(c0 + e) * W + j];
+        for (int e = 0; e < 4; ++e)
+#pragma unroll
+            for (int j = 0; j < W; ++j) w[e][j] = a.w[(c0 + e) * W + j];
+    }
 
     // the sequence of the first token: the last n with cu[n] <= t0 (first entry above t0, minus one)
     int32_t lo = 0, hi = a.n + 1;
@@ -92,80 +126,100 @@ __global__ void __launch_bounds__(kConvThreads) short_conv_kernel(const ConvArgs
         else hi = mid;
     }
     int32_t n = min(max(lo - 1, 0), a.n - 1);
-    int32_t start = conv_cu(a, n), next = conv_cu(a, n + 1);
+    int64_t start = conv_cu(a, n), next = conv_cu(a, n + 1);
 
-    // history: the W-1 inputs before t0, oldest first
-    float hist[H > 0 ? H : 1][4];
+    auto silu_inplace = [&](float (&out)[4]) {
+        // SiLU: x / (1 + e^-x) with the fast exponential and division (relative
+        // error a few ulp of fp32, far inside the output's rounding; for x below
+        // about -88 the denominator is infinite and the result the limit 0)
+        if (a.silu)
 #pragma unroll
-    for (int i = 0; i < H; ++i) {
-        const int32_t u = t0 - H + i;
-        if (u >= start && u >= 0) {
-            load4(x + int64_t(u) * C + c0, hist[i]);
-        } else {
-            const int32_t si = H - (start - u);
+            for (int e = 0; e < 4; ++e) out[e] = __fdividef(out[e], 1.f + __expf(-out[e]));
+    };
+    if (t0 - H >= start && t0 + kConvTok <= next && t0 + kConvTok <= a.tokens) {
+        // the common case: every token of the group, with all its taps, inside one sequence
+        T *yb = y + t0 * C + c0;
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                hist[i][e] = (a.state_in && si >= 0 && si < H) ? a.state_in[(int64_t(n) * C + c0 + e) * H + si] : 0.f;
-        }
-    }
-
-    for (int32_t tb = t0; tb < t1; tb += kConvPre) {
-        float xv[kConvPre][4];
-#pragma unroll
-        for (int p = 0; p < kConvPre; ++p)
-            if (tb + p < t1) load4(x + int64_t(tb + p) * C + c0, xv[p]);
-#pragma unroll
-        for (int p = 0; p < kConvPre; ++p) {
-            const int32_t t = tb + p;
-            if (t >= t1) break;
-            while (t >= next && n < a.n - 1) {  // a sequence starts at t: reset from its state
-                ++n;
-                start = next;
-                next = conv_cu(a, n + 1);
-#pragma unroll
-                for (int i = 0; i < H; ++i)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        hist[i][e] = a.state_in ? a.state_in[(int64_t(n) * C + c0 + e) * H + i] : 0.f;
-            }
+        for (int p = 0; p < kConvTok; ++p) {
             float out[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                float acc = w[e][H] * xv[p][e];
+                float acc = 0.f;
 #pragma unroll
-                for (int j = 0; j < H; ++j) acc = fmaf(w[e][j], hist[j][e], acc);
-                out[e] = a.silu ? acc / (1.f + expf(-acc)) : acc;
+                for (int j = 0; j < W; ++j) acc = fmaf(w[e][j], xr[p + j][e], acc);
+                out[e] = acc;
             }
-            store4(y + int64_t(t) * C + c0, out);
+            silu_inplace(out);
+            store4(yb + int64_t(p) * C, out);
+        }
+        if (a.state_out && H > 0 && t0 + kConvTok == next)  // the sequence's last H inputs: rows kConvTok ..
 #pragma unroll
-            for (int i = 0; i + 1 < H; ++i)
+            for (int e = 0; e < 4; ++e)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) hist[i][e] = hist[i + 1][e];
-            if (H > 0)
+                for (int i = 0; i < H; ++i) a.state_out[(int64_t(n) * C + c0 + e) * H + i] = xr[kConvTok + i][e];
+        return;
+    }
+    for (int p = 0; p < kConvTok; ++p) {
+        const int64_t t = t0 + p;
+        if (t >= a.tokens) break;
+        while (t >= next && n < a.n - 1) {  // a sequence starts at or before t
+            ++n;
+            start = next;
+            next = conv_cu(a, n + 1);
+        }
+        float out[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) hist[H > 0 ? H - 1 : 0][e] = xv[p][e];
-            if (t == next - 1 && a.state_out)
+        for (int e = 0; e < 4; ++e) {
+            float acc = 0.f;
 #pragma unroll
-                for (int i = 0; i < H; ++i)
+            for (int j = 0; j < W; ++j) {
+                const int64_t u = t - H + j;  // tap j of token t
+                float v;
+                if (u >= start) {
+                    v = xr_at(xr, p + j, e);
+                } else {
+                    const int64_t si = H - (start - u);  // oldest first in the conv state
+                    v = (a.state_in && si >= 0 && si < H) ? a.state_in[(int64_t(n) * C + c0 + e) * H + si] : 0.f;
+                }
+                acc = fmaf(w[e][j], v, acc);
+            }
+            out[e] = acc;
+        }
+        silu_inplace(out);
+        store4(y + t * C + c0, out);
+        if (a.state_out && H > 0 && t == next - 1) {  // the sequence's last H inputs, oldest first
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) a.state_out[(int64_t(n) * C + c0 + e) * H + i] = hist[i][e];
+            for (int e = 0; e < 4; ++e)
+#pragma unroll
+                for (int i = 0; i < H; ++i) {
+                    const int64_t u = t - H + 1 + i;
+                    float v;
+                    if (u >= start) {
+                        v = xr_at(xr, p + 1 + i, e);
+                    } else {
+                        const int64_t si = H - (start - u);
+                        v = (a.state_in && si >= 0 && si < H) ? a.state_in[(int64_t(n) * C + c0 + e) * H + si] : 0.f;
+                    }
+                    a.state_out[(int64_t(n) * C + c0 + e) * H + i] = v;
+                }
         }
     }
 }
 
-// empty sequences: state_out = state_in (zeros without one)
-__global__ void short_conv_empty_kernel(const ConvArgs a, int32_t hist) {
+// Empty sequences (no thread of the convolution sees them): the conv state
+// passes through (zeros without an incoming state).
+__global__ void short_conv_empty_kernel(const ConvArgs a, int32_t H) {
     const int32_t n = blockIdx.x;
     if (conv_cu(a, n + 1) != conv_cu(a, n)) return;
-    const int64_t per = int64_t(a.channels) * hist;
+    const int64_t per = int64_t(a.channels) * H;
     for (int64_t i = threadIdx.x; i < per; i += blockDim.x)
         a.state_out[int64_t(n) * per + i] = a.state_in ? a.state_in[int64_t(n) * per + i] : 0.f;
 }
 
 template <typename T>
 static cudaError_t launch_conv_as(const ConvArgs &a, int32_t width, cudaStream_t stream) {
-    const dim3 grid(unsigned((a.tokens + kConvSeg - 1) / kConvSeg),
-                    unsigned((a.channels / 4 + kConvThreads - 1) / kConvThreads));
+    const int64_t threads = (int64_t(a.tokens) + kConvTok - 1) / kConvTok * (a.channels / 4);
+    const unsigned grid = unsigned((threads + kConvThreads - 1) / kConvThreads);
     switch (width) {
         case 1: short_conv_kernel<T, 1><<<grid, kConvThreads, 0, stream>>>(a); break;
         case 2: short_conv_kernel<T, 2><<<grid, kConvThreads, 0, stream>>>(a); break;
@@ -185,7 +239,8 @@ cudaError_t launch_short_conv(int32_t n, int32_t seq_len, const int32_t *cu, int
                               float *state_out, void *y, bool silu, cudaStream_t stream) {
     if (n <= 0) return cudaSuccess;
     if (width < 1 || width > 8 || channels <= 0 || channels % 4 != 0 || tokens < 0) return cudaErrorInvalidValue;
-    if (int64_t(channels) / 4 > int64_t(65535) * kConvThreads) return cudaErrorInvalidValue;
+    const int64_t threads = (int64_t(tokens) + kConvTok - 1) / kConvTok * (channels / 4);
+    if ((threads + kConvThreads - 1) / kConvThreads > int64_t(0x7fffffff)) return cudaErrorInvalidValue;
     ConvArgs a{cu, n, seq_len, tokens, channels, x, w, state_in, state_out, y, silu ? 1 : 0};
     cudaError_t e = cudaSuccess;
     if (tokens > 0) {

@@ -1,20 +1,21 @@
-"""The index walk of the short-convolution kernel (csrc/gdn_conv.cu), written
+"""The index walk of the short-convolution kernels (csrc/gdn_conv.cu), written
 out in Python thread by thread and run on CPU against the fp64 oracle.
 
-The kernel gives each thread a segment of kConvSeg consecutive tokens of the
-packed layout and a group of channels.  A segment may start inside a
-sequence, span several short ones, or include empty ones; the thread finds
-the sequence of its first token by binary search over cu_seqlens, fills its
-W-1 token history from the inputs before the segment (or from the
-sequence's conv state, or zeros, before the sequence's first token), and
-walks its tokens, resetting the history at each sequence start and writing
-the conv state after each sequence's last token.  Empty sequences get their
-state passed through by a second kernel.  This file checks that walk; the
-GPU parity test checks the kernel itself."""
+The convolution kernel gives each thread kConvTok consecutive tokens of the
+packed layout and a group of channels.  The thread loads the input rows from
+W-1 before its first token to its last token (zeros outside the tensor),
+finds the sequence of its first token by binary search over cu_seqlens, and
+for each of its tokens steps on to the token's sequence; a tap before the
+sequence's first token reads the sequence's conv state (or zero).  The thread
+holding a sequence's last token writes that sequence's last W-1 inputs,
+reaching into the incoming state when the sequence is shorter; a second
+kernel passes the state of empty sequences through.  This file checks that
+walk with several tokens-per-thread counts; the GPU parity test checks the
+kernels themselves."""
 import numpy as np
 import pytest
 
-SEG = 64  # tokens per thread segment, as kConvSeg in the kernel
+TOK = 8  # tokens per thread, as kConvTok in the kernel
 
 
 def upper_bound(cu, t):
@@ -29,8 +30,8 @@ def upper_bound(cu, t):
     return lo
 
 
-def walk(x, w, cu, state_in, silu, seg=SEG):
-    """The kernels' arithmetic and indexing, per (segment, channel) thread,
+def walk(x, w, cu, state_in, silu, tok=TOK):
+    """The kernels' arithmetic and indexing, per (token group, channel) thread,
     in fp64 so that only the walk, not the rounding, is under test."""
     T, C = x.shape
     W = w.shape[1]
@@ -38,29 +39,30 @@ def walk(x, w, cu, state_in, silu, seg=SEG):
     N = len(cu) - 1
     y = np.full((T, C), np.nan)
     s_out = np.full((N, C, H), np.nan)
+
+    def from_state(n, c, start, u):
+        si = H - (start - u)  # oldest first in the conv state
+        return state_in[n, c, si] if (state_in is not None and 0 <= si < H) else 0.0
+
     for c in range(C):
-        for t0 in range(0, T, seg):
-            t1 = min(t0 + seg, T)
-            n = upper_bound(cu, t0) - 1  # cu[n] <= t0 < cu[n + 1]
-            hist = []
-            for i in range(H):
-                u = t0 - H + i
-                if u >= cu[n]:
-                    hist.append(x[u, c])
-                else:
-                    hist.append(state_in[n, c, H - (cu[n] - u)] if state_in is not None else 0.0)
-            for t in range(t0, t1):
-                while t >= cu[n + 1]:
+        for t0 in range(0, T, tok):
+            rows = {u: (x[u, c] if 0 <= u < T else 0.0) for u in range(t0 - H, t0 + tok)}
+            n = min(max(upper_bound(cu, t0) - 1, 0), N - 1)
+            start, nxt = cu[n], cu[n + 1]
+            for t in range(t0, min(t0 + tok, T)):
+                while t >= nxt and n < N - 1:
                     n += 1
-                    hist = [state_in[n, c, i] if state_in is not None else 0.0 for i in range(H)]
-                acc = w[c, H] * x[t, c]
-                for j in range(H):
-                    acc += w[c, j] * hist[j]
+                    start, nxt = nxt, cu[n + 1]
+                acc = 0.0
+                for j in range(W):
+                    u = t - H + j
+                    acc += w[c, j] * (rows[u] if u >= start else from_state(n, c, start, u))
                 y[t, c] = acc / (1.0 + np.exp(-acc)) if silu else acc
-                hist = hist[1:] + [x[t, c]]
-                if t == cu[n + 1] - 1:
-                    s_out[n, c] = hist
-    # second kernel: empty sequences pass their state through
+                if t == nxt - 1:  # the sequence's last token: its conv state
+                    for i in range(H):
+                        u = t - H + 1 + i
+                        s_out[n, c, i] = rows[u] if u >= start else from_state(n, c, start, u)
+    # the second kernel: empty sequences pass their state through
     for n in range(N):
         if cu[n + 1] == cu[n]:
             s_out[n] = state_in[n] if state_in is not None else 0.0
@@ -71,7 +73,7 @@ def walk(x, w, cu, state_in, silu, seg=SEG):
 def test_walk_matches_oracle(oracle_mod, case):
     rng = np.random.default_rng(900 + case)
     W = [1, 2, 3, 4, 4, 4, 5, 8, 4, 4, 2, 4][case]
-    seg = [64, 64, 64, 64, 5, 3, 7, 4, 1, 2, 64, 9][case]
+    seg = [8, 8, 8, 8, 5, 3, 7, 4, 1, 2, 64, 9][case]
     n = int(rng.integers(1, 9))
     lens = [int(v) for v in rng.integers(0, 3 * seg + 4, size=n)]
     if case % 3 == 0:

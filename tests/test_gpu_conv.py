@@ -54,8 +54,9 @@ def test_conv_batched(dtype, W):
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("with_state", [False, True])
 def test_conv_varlen_edges(dtype, with_state):
-    """Empty sequences, sequences shorter than W - 1, and segment boundaries
-    inside and between sequences; 16 heads of 128 (several channel blocks)."""
+    """Empty sequences, sequences shorter than W - 1, and the boundaries of the
+    threads' token groups
+    inside and between sequences; 16 heads of 128 (several channel groups)."""
     lens = [0, 1, 2, 63, 64, 65, 0, 130, 3, 200]
     x, w, st, cu = conv_case(50, (sum(lens),), (16, 128), 4, dtype, lens=lens, with_state=with_state)
     y, so, y_ref, s_ref = run_both(x, w, st, cu)
