@@ -198,8 +198,9 @@ GDN_API gdn_status_t gdn_chunk_forward(const gdn_shape_t *shape,
  * All calls on a device share the one array: calls that overlap on the GPU
  * (two streams, or two host threads) race on it and give wrong results, so
  * serialise them.  Each call re-initialises the scratch before use, so what
- * an earlier call left there is harmless.  The device status word of a
- * cu_seqlens check cannot be read back through this entry point. */
+ * an earlier call left there is harmless.  gdn_noalloc_read_device_status
+ * reads back the device status word the last call on the current device
+ * left in the array. */
 GDN_API gdn_status_t gdn_chunk_forward_noalloc(const gdn_shape_t *shape,
                                        const void *q, const void *k, const void *v,
                                        const float *g, const float *beta,
@@ -210,8 +211,19 @@ GDN_API gdn_status_t gdn_chunk_forward_noalloc(const gdn_shape_t *shape,
 
 /* Reads the device status word that gdn_chunk_forward left in `workspace`
  * (GDN_OK or GDN_ERR_DEVICE_CHECK) into *device_status.  Synchronises
- * `stream`.  This is the only entry point that waits for the GPU. */
+ * `stream`.  This and gdn_noalloc_read_device_status are the only entry
+ * points that wait for the GPU. */
 GDN_API gdn_status_t gdn_read_device_status(const void *workspace, int32_t *device_status, void *stream);
+
+/* The same for gdn_chunk_forward_noalloc: reads the device status word that
+ * the last such call on the current device left in the library's built-in
+ * scratch array (a cu_seqlens rejected on the device, or a tensor-core wait
+ * that timed out, reads GDN_ERR_DEVICE_CHECK; o and final_state are then
+ * not written).  Synchronises `stream`.  Like the scratch array itself it
+ * has no counterpart in the source pages.  Errors: GDN_ERR_INVALID_ARGUMENT
+ * for a NULL device_status, GDN_ERR_CUDA when the array's address cannot be
+ * resolved or the read fails. */
+GDN_API gdn_status_t gdn_noalloc_read_device_status(int32_t *device_status, void *stream);
 
 /* One decode token for each of N sequences, state updated in place
  * ("The Transformer Isn't Alone Anymore": the recurrent state is read and

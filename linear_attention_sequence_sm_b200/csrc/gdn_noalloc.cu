@@ -77,3 +77,18 @@ extern "C" GDN_API gdn_status_t gdn_chunk_forward_noalloc(const gdn_shape_t *sha
     return gdn_chunk_forward(&one, q, k, v, g, beta, initial_state, cu_seqlens, o, final_state, scratch,
                              kNoAllocScratchBytes, stream);
 }
+
+extern "C" GDN_API gdn_status_t gdn_noalloc_read_device_status(int32_t *device_status, void *stream) {
+    using namespace gdn;
+    if (!device_status) return set_error(GDN_ERR_INVALID_ARGUMENT, "device_status is NULL");
+    void *scratch = nullptr;
+    const cudaError_t e = scratch_address(&scratch);
+    if (e != cudaSuccess) {
+        char msg[200];
+        snprintf(msg, sizeof(msg), "resolving the device address of the built-in scratch array failed: %s",
+                 cudaGetErrorString(e));
+        return set_error(GDN_ERR_CUDA, msg);
+    }
+    // the array starts with the same header a caller's workspace does
+    return gdn_read_device_status(scratch, device_status, stream);
+}

@@ -45,7 +45,7 @@ EXPORTED = ("gdn_chunk_forward_workspace_size", "gdn_chunk_forward", "gdn_read_d
             "gdn_chunk_forward_noalloc", "gdn_decode_step_ex", "gdn_chunk_forward_out", "gdn_decode_step_out",
             "gdn_kda_forward", "gdn_kda_decode_step", "gdn_decode_multi", "gdn_decode_commit",
             "gdn_chunk_backward_workspace_size", "gdn_chunk_backward", "gdn_short_conv",
-            "gdn_chunk_forward_path")
+            "gdn_chunk_forward_path", "gdn_noalloc_read_device_status")
 GDN_PATH_SIMT = 0
 GDN_PATH_TC_ONE_KERNEL = 1
 GDN_PATH_TC_SPLIT = 2
@@ -80,6 +80,8 @@ def _load(path: str = LIB_PATH):
     lib.gdn_chunk_forward_workspace_size.restype = st
     lib.gdn_chunk_forward_path.argtypes = [ctypes.POINTER(Shape), ctypes.c_size_t, ctypes.POINTER(ctypes.c_int32)]
     lib.gdn_chunk_forward_path.restype = st
+    lib.gdn_noalloc_read_device_status.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
+    lib.gdn_noalloc_read_device_status.restype = st
     lib.gdn_chunk_forward.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                       ctypes.c_size_t, vp]
     lib.gdn_chunk_forward.restype = st
@@ -376,6 +378,16 @@ def read_device_status(workspace, stream=None) -> int:
     dev = workspace.device
     with torch.cuda.device(dev):  # the library launches on the current device
         _check(LIB.gdn_read_device_status(_ptr(workspace), ctypes.byref(st), _stream_handle(stream, dev)))
+    return st.value
+
+
+def noalloc_read_device_status(device=None, stream=None) -> int:
+    """Synchronise the stream and return the device status word of the last
+    gdn_chunk_forward_noalloc on ``device`` (default: the current device)."""
+    st = ctypes.c_int32(-1)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        _check(LIB.gdn_noalloc_read_device_status(ctypes.byref(st), _stream_handle(stream, dev)))
     return st.value
 
 

@@ -94,6 +94,17 @@ def test_path_query_arguments(gdn):
         assert st == gdn.GDN_ERR_CUDA and p.value == -1
 
 
+def test_noalloc_status_arguments(gdn):
+    """The built-in array's status reader refuses a NULL output; on a host
+    without a GPU it reports GDN_ERR_CUDA rather than reading anything."""
+    assert gdn.LIB.gdn_noalloc_read_device_status(None, None) == gdn.GDN_ERR_INVALID_ARGUMENT
+    import torch
+    if not torch.cuda.is_available():
+        st = ctypes.c_int32(-1)
+        assert gdn.LIB.gdn_noalloc_read_device_status(ctypes.byref(st), None) == gdn.GDN_ERR_CUDA
+        assert st.value == -1 and gdn.LIB.gdn_last_error_message().decode() != ""
+
+
 def test_contradictory_path_flags_rejected(gdn):
     n = ctypes.c_size_t(0)
     s = _shape(gdn, flags=gdn.GDN_FLAG_SPLIT | gdn.GDN_FLAG_ONE_KERNEL)

@@ -67,6 +67,28 @@ def test_noalloc_matches_workspace_entry_point_twice():
         assert torch.isfinite(o_na.float()).all() and torch.isfinite(sf_na).all()
 
 
+def test_noalloc_device_status_reads_back():
+    """A cu_seqlens rejected on the device shows in the built-in array's status
+    word (and the outputs stay unwritten); the next good call clears it."""
+    from linear_attention_sequence_sm_b200 import gdn
+    dev = torch.device("cuda:0")
+    T, hk, hv, d = 100, 1, 4, 128
+    gen = torch.Generator(device="cpu").manual_seed(81)
+    q = torch.nn.functional.normalize(torch.randn(1, T, hk, d, generator=gen), dim=-1).bfloat16().to(dev)
+    v = torch.randn(1, T, hv, d, generator=gen).bfloat16().to(dev)
+    g = (-torch.rand(1, T, hv, generator=gen)).to(dev)
+    b = torch.rand(1, T, hv, generator=gen).to(dev)
+    bad = torch.tensor([0, 60, 40, 100], dtype=torch.int32, device=dev)
+    o = torch.full_like(v, 7.0)
+    gdn.chunk_forward_noalloc(q, q, v, g, b, cu_seqlens=bad, out=o)
+    assert gdn.noalloc_read_device_status(dev) == gdn.GDN_ERR_DEVICE_CHECK
+    assert (o == 7.0).all()
+    good = torch.tensor([0, 50, 100], dtype=torch.int32, device=dev)
+    gdn.chunk_forward_noalloc(q, q, v, g, b, cu_seqlens=good, out=o)
+    assert gdn.noalloc_read_device_status(dev) == gdn.GDN_OK
+    assert not (o == 7.0).all()
+
+
 def test_noalloc_refuses_too_many_sequences():
     from linear_attention_sequence_sm_b200 import gdn
     dev = torch.device("cuda:0")
