@@ -320,13 +320,18 @@ GDN_API gdn_status_t gdn_decode_step_out(int32_t num_seqs, int32_t num_qk_heads,
  *   g     [tokens, Hv, d_k] fp32: one log-decay per key channel (with
  *         GDN_FLAG_GATE_LOGITS: one decay logit per key channel, alpha =
  *         sigmoid(logit)); read as max(g, -20) like the scalar gate.
- * shape->chunk_size is checked as for gdn_chunk_forward but not used: the
- * kernel walks the tokens of each sequence in order on CUDA cores, the state
- * in registers (a block per sequence, value head and 32 rows of d_v), since
- * the decay-masked key products of a chunked form are not plain matrix
- * products.  Supports d_k <= 128 and d_v <= 128, fp32 or bf16; the input
- * flags; an output side (applied as a second pass over o).  The workspace is
- * that of gdn_chunk_forward for the same shape. */
+ * Two paths.  bf16 with d_k = d_v = 128 and C = 64 runs the chunkwise WY
+ * form on the tensor cores: a first kernel forms every chunk's decay-masked
+ * products, its triangular factor and the decay-scaled keys and queries at
+ * once, then the chunk loop carries the state through tcgen05 products.  It
+ * needs the workspace gdn_kda_forward_workspace_size returns (66,048 bytes
+ * per (chunk, value head) on top of the schedule tables).  Every other shape,
+ * GDN_FLAG_FORCE_SIMT, or a smaller workspace walks the tokens of each
+ * sequence in order on CUDA cores (state in registers, a block per sequence,
+ * value head and 32 rows of d_v; shape->chunk_size is checked but not used),
+ * with the workspace of gdn_chunk_forward.  Supports d_k <= 128 and
+ * d_v <= 128, fp32 or bf16; the input flags; an output side (applied as a
+ * second pass over o). */
 GDN_API gdn_status_t gdn_kda_forward(const gdn_shape_t *shape,
                              const void *q, const void *k, const void *v,
                              const float *g, const float *beta,
@@ -336,6 +341,10 @@ GDN_API gdn_status_t gdn_kda_forward(const gdn_shape_t *shape,
                              void *o, float *final_state,
                              void *workspace, size_t workspace_bytes,
                              void *stream);
+
+/* Bytes of workspace gdn_kda_forward needs for `shape` (the tensor-core path's
+ * chunk operands where it applies, else the schedule tables alone). */
+GDN_API gdn_status_t gdn_kda_forward_workspace_size(const gdn_shape_t *shape, size_t *bytes);
 
 /* One Kimi Delta Attention token per sequence, state updated in place: per
  * state row s_i, s' = alpha .* s_i, u_i = beta (v_i - s' . k),

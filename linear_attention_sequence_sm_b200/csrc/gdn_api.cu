@@ -184,6 +184,16 @@ gdn_status_t gdn_chunk_forward_out(const gdn_shape_t *s, const void *q, const vo
                               workspace_bytes, stream_);
 }
 
+gdn_status_t gdn_kda_forward_workspace_size(const gdn_shape_t *s, size_t *bytes) {
+    g_msg[0] = 0;
+    if (!bytes) return fail(GDN_ERR_INVALID_ARGUMENT, "bytes is NULL");
+    gdn_status_t st = check_shape(s);
+    if (st != GDN_OK) return st;
+    const bool tc = kda_tc_supported(*s) && !(s->flags & GDN_FLAG_FORCE_SIMT);
+    *bytes = tc ? kda_layout(*s).total : ws_layout(s->num_seqs).total;
+    return GDN_OK;
+}
+
 gdn_status_t gdn_kda_forward(const gdn_shape_t *s, const void *q, const void *k, const void *v, const float *g,
                              const float *beta, const float *initial_state, const int32_t *cu_seqlens,
                              const gdn_output_side_t *out_side, void *o, float *final_state, void *workspace,
@@ -259,10 +269,24 @@ static gdn_status_t chunk_forward_impl(const gdn_shape_t *s, const void *q, cons
     }
 
     if (kda) {
-        e = launch_schedule(*s, cu_seqlens, workspace, stream);
-        if (e != cudaSuccess) return cuda_fail(e, "schedule kernel launch");
-        e = launch_kda_prefill(a, stream);
-        if (e != cudaSuccess) return cuda_fail(e, "KDA prefill launch");
+        // bf16 with d_k = d_v = 128 and C = 64 runs on the tensor cores when the
+        // workspace holds the chunk operands; otherwise the token-order kernel
+        const bool kda_tc = major == 10 && tokens > 0 && !(s->flags & GDN_FLAG_FORCE_SIMT) &&
+                            kda_tc_supported(*s) && workspace_bytes >= kda_layout(*s).total;
+        if (kda_tc) {
+            const KdaLayout KL = kda_layout(*s);
+            int32_t *cbase = reinterpret_cast<int32_t *>(ws + KL.cbase_off);
+            e = launch_schedule(*s, cu_seqlens, workspace, stream, cbase);
+            if (e != cudaSuccess) return cuda_fail(e, "schedule kernel launch");
+            a.sched.chunk_base = cbase;
+            e = launch_kda_tc(a, reinterpret_cast<unsigned char *>(ws + KL.items_off), stream, sms);
+            if (e != cudaSuccess) return cuda_fail(e, "tensor-core KDA prefill launch");
+        } else {
+            e = launch_schedule(*s, cu_seqlens, workspace, stream);
+            if (e != cudaSuccess) return cuda_fail(e, "schedule kernel launch");
+            e = launch_kda_prefill(a, stream);
+            if (e != cudaSuccess) return cuda_fail(e, "KDA prefill launch");
+        }
         if (out.flags) {
             e = launch_output_side(o, int32_t(tokens), s->num_v_heads, s->head_dim_v, s->dtype, out, stream);
             if (e != cudaSuccess) return cuda_fail(e, "output-side launch");

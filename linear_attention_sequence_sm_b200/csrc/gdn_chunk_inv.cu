@@ -30,6 +30,7 @@
 // so T is the factor of the normalised keys.  Every wait is bounded; a timeout
 // records GDN_ERR_DEVICE_CHECK (bad_index -3) in the workspace status word.
 #include "gdn_internal.cuh"
+#include "gdn_inverse.cuh"
 #include "gdn_sm100.cuh"
 
 namespace gdn {
@@ -38,8 +39,6 @@ using namespace sm100;
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kLdA = 68;  // fp32 row stride of A / T (16-byte aligned rows, 4 mod 8 against bank conflicts)
-constexpr int kLdY = 36;  // fp32 row stride of the block-product scratch
 constexpr uint32_t kTileK = 16384;  // one K tile: 2 atom columns x 64 rows x 128 bytes
 constexpr uint32_t kOffK0 = 0, kOffK1 = kTileK;
 constexpr uint32_t kOffA = 2 * kTileK;                 // A, inverted in place into T
@@ -52,80 +51,6 @@ constexpr uint32_t kSmemBytes = kOffBar + 64 + 1024;   // + alignment slack
 constexpr int kVecG = 0, kVecB = 64, kVecRow = 128, kVecCol = 192, kVecIk = 256, kVecTp = 320;
 constexpr int kBarK = 0, kBarMma = 2;  // K tile barriers (2 buffers), Gram completion
 constexpr uint32_t kTmemCols = 64;
-
-// T = (I + A)^-1 in place for the 64 x 64 strictly lower A in Af (everything
-// on and above the diagonal zero).  Called by all kThreads threads.
-__device__ void invert_in_place(float *Af, float *Y, int t) {
-    const int w = t >> 5, lane = t & 31;
-    // the four 16 x 16 diagonal blocks: thread (b, c) solves column c of block b
-    float x[16];
-    if (t < 64) {
-        const int b = t >> 4, c = t & 15;
-        const float *Ab = Af + (16 * b) * kLdA + 16 * b;
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float a[16];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) load4(Ab + r * kLdA + 4 * q, a + 4 * q);
-            float acc0 = (r == c) ? 1.f : 0.f, acc1 = 0.f;
-#pragma unroll
-            for (int jj = 0; jj < r; ++jj) {
-                if (jj & 1) acc1 = fmaf(-a[jj], x[jj], acc1);
-                else acc0 = fmaf(-a[jj], x[jj], acc0);
-            }
-            x[r] = acc0 + acc1;
-        }
-    }
-    __syncthreads();  // every diagonal block of A has been read
-    if (t < 64) {
-        const int b = t >> 4, c = t & 15;
-        float *Tb = Af + (16 * b) * kLdA + 16 * b;
-#pragma unroll
-        for (int r = 0; r < 16; ++r) Tb[r * kLdA + c] = x[r];
-    }
-    __syncthreads();
-    // 16 -> 32: in each 32 x 32 half p, Y = A21 T11, then T21 = -T22 Y
-    if (w < 4) {
-        const int p = w >> 1, n0 = 8 * (w & 1);
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-        tile_mma(c, Af + (32 * p + 16) * kLdA + 32 * p, kLdA, Af + (32 * p) * kLdA + 32 * p, kLdA, n0, 2, lane);
-        tile_store(Y + (16 * p) * kLdY, kLdY, 0, n0, c, 1.f, lane);
-    }
-    __syncthreads();
-    if (w < 4) {
-        const int p = w >> 1, n0 = 8 * (w & 1);
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-        tile_mma(c, Af + (32 * p + 16) * kLdA + 32 * p + 16, kLdA, Y + (16 * p) * kLdY, kLdY, n0, 2, lane);
-        tile_store(Af + (32 * p + 16) * kLdA + 32 * p, kLdA, 0, n0, c, -1.f, lane);
-    }
-    __syncthreads();
-    // 32 -> 64: Y = A21 T11 (32 x 32), then T21 = -T22 Y
-    {
-        const int m0 = 16 * (w >> 2), n0 = 8 * (w & 3);
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-        tile_mma(c, Af + (32 + m0) * kLdA, kLdA, Af, kLdA, n0, 4, lane);
-        tile_store(Y, kLdY, m0, n0, c, 1.f, lane);
-    }
-    __syncthreads();
-    {
-        const int m0 = 16 * (w >> 2), n0 = 8 * (w & 3);
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-        tile_mma(c, Af + (32 + m0) * kLdA + 32, kLdA, Y, kLdY, n0, 4, lane);
-        tile_store(Af + 32 * kLdA, kLdA, m0, n0, c, -1.f, lane);  // rows 32 + m0 .., columns n0 ..
-    }
-    __syncthreads();
-}
-
-// Sequence n holding global chunk gc: the largest n < N with chunk_base[n] <= gc.
-__device__ __forceinline__ int seq_of_chunk(const int32_t *chunk_base, int num_seqs, int gc) {
-    int lo = 0, hi = num_seqs - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (chunk_base[mid] <= gc) lo = mid;
-        else hi = mid - 1;
-    }
-    return lo;
-}
 
 template <bool kL2, bool kLogits>
 __global__ void __launch_bounds__(kThreads, 3)
@@ -164,7 +89,7 @@ chunk_inverse_kernel(const __grid_constant__ CUtensorMap tm_k, const PrefillArgs
     auto locate = [&](int item, int &gc, int &hq, int &t0, int &L) {
         gc = item / hk;
         hq = item - gc * hk;
-        const int n = seq_of_chunk(a.sched.chunk_base, a.num_seqs, gc);
+        const int n = chunk_sequence(a.sched.chunk_base, a.num_seqs, gc);
         const int c = gc - a.sched.chunk_base[n];
         t0 = a.sched.start[n] + 64 * c;
         L = min(64, a.sched.len[n] - 64 * c);

@@ -103,6 +103,28 @@ inline SplitLayout split_layout(const gdn_shape_t &s) {
     return L;
 }
 
+// Sequence n holding global chunk gc: the largest n < N with chunk_base[n] <= gc.
+__device__ __forceinline__ int chunk_sequence(const int32_t *chunk_base, int num_seqs, int gc) {
+    int lo = 0, hi = num_seqs - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (chunk_base[mid] <= gc) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Workspace of the tensor-core KDA prefill (gdn_kda_tc.cu): the schedule
+// tables, chunk_base, then per (chunk, value head) the chunk loop's operands
+// (K+, Q+, K^, T'', P as bf16 tiles and e^G_last), 66,048 bytes each.
+struct KdaLayout {
+    WsLayout sched;
+    size_t cbase_off, items_off, total;
+    int64_t max_chunks;
+};
+KdaLayout kda_layout(const gdn_shape_t &s);
+bool kda_tc_supported(const gdn_shape_t &s);
+
 // Pointers into the workspace, as the kernels see them.
 struct Sched {
     WsHeader *hdr;
@@ -226,6 +248,8 @@ cudaError_t launch_chunk_inverse(const PrefillArgs &a, __nv_bfloat16 *tinv, floa
                                  cudaStream_t stream, int num_sms);
 cudaError_t launch_chunk_chain(const PrefillArgs &a, const __nv_bfloat16 *tinv, const float *gcum,
                                int64_t max_chunks, cudaStream_t stream, int num_sms);
+// The tensor-core KDA prefill: factor kernel, then chunk loop (gdn_kda_tc.cu).
+cudaError_t launch_kda_tc(const PrefillArgs &a, unsigned char *items, cudaStream_t stream, int num_sms);
 
 // The output side as its own pass over o, in place (for the CUDA-core prefill,
 // whose blocks each own a slice of d_v).

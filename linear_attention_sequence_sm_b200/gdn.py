@@ -45,7 +45,7 @@ EXPORTED = ("gdn_chunk_forward_workspace_size", "gdn_chunk_forward", "gdn_read_d
             "gdn_chunk_forward_noalloc", "gdn_decode_step_ex", "gdn_chunk_forward_out", "gdn_decode_step_out",
             "gdn_kda_forward", "gdn_kda_decode_step", "gdn_decode_multi", "gdn_decode_commit",
             "gdn_chunk_backward_workspace_size", "gdn_chunk_backward", "gdn_short_conv",
-            "gdn_chunk_forward_path", "gdn_noalloc_read_device_status")
+            "gdn_chunk_forward_path", "gdn_noalloc_read_device_status", "gdn_kda_forward_workspace_size")
 GDN_PATH_SIMT = 0
 GDN_PATH_TC_ONE_KERNEL = 1
 GDN_PATH_TC_SPLIT = 2
@@ -80,6 +80,8 @@ def _load(path: str = LIB_PATH):
     lib.gdn_chunk_forward_workspace_size.restype = st
     lib.gdn_chunk_forward_path.argtypes = [ctypes.POINTER(Shape), ctypes.c_size_t, ctypes.POINTER(ctypes.c_int32)]
     lib.gdn_chunk_forward_path.restype = st
+    lib.gdn_kda_forward_workspace_size.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(ctypes.c_size_t)]
+    lib.gdn_kda_forward_workspace_size.restype = st
     lib.gdn_noalloc_read_device_status.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
     lib.gdn_noalloc_read_device_status.restype = st
     lib.gdn_chunk_forward.argtypes = [ctypes.POINTER(Shape), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
@@ -281,6 +283,13 @@ def forward_path(shape: Shape, workspace_bytes: int | None = None) -> str:
     return PATH_NAMES[p.value]
 
 
+def kda_workspace_size(shape: Shape) -> int:
+    """Bytes of workspace gdn_kda_forward needs for ``shape``."""
+    n = ctypes.c_size_t(0)
+    _check(LIB.gdn_kda_forward_workspace_size(ctypes.byref(shape), ctypes.byref(n)))
+    return n.value
+
+
 def workspace_size(shape: Shape) -> int:
     n = ctypes.c_size_t(0)
     _check(LIB.gdn_chunk_forward_workspace_size(ctypes.byref(shape), ctypes.byref(n)))
@@ -425,11 +434,12 @@ def decode_step(q, k, v, g, beta, state, out=None, stream=None, qk_l2norm=False,
 
 def kda_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, output_final_state=True, out=None,
                 final_state=None, workspace=None, stream=None, qk_l2norm=False, gate_logits=False,
-                output_norm: OutputNorm | None = None, chunk_size=64):
+                output_norm: OutputNorm | None = None, chunk_size=64, force_simt=False):
     """Kimi Delta Attention prefill (one decay per key channel): g is
     [..., Hv, d_k] fp32.  Returns (o, final_state or None).  Other arguments
-    as for chunk_forward; ``chunk_size`` is validated but unused (the kernel
-    walks the tokens in order)."""
+    as for chunk_forward.  bf16 with d = 128 and chunk_size 64 runs the
+    tensor-core chunkwise form; other shapes, or ``force_simt``, the
+    token-order CUDA-core kernel."""
     n_seqs, hv, dv, dk = _prefill_shapes(q, k, v, g, beta, initial_state, cu_seqlens, kda=True)
     _expect(out, "out", v.shape)
     _expect(final_state, "final_state", (n_seqs, hv, dv, dk))
@@ -441,7 +451,7 @@ def kda_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, output_fi
     _need(beta, "beta", torch.float32, dev)
     _need(initial_state, "initial_state", torch.float32, dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
-    shape = make_shape(q, v, cu_seqlens, chunk_size, False, input_flags(qk_l2norm, gate_logits))
+    shape = make_shape(q, v, cu_seqlens, chunk_size, force_simt, input_flags(qk_l2norm, gate_logits))
     if out is None:
         out = torch.empty(v.shape, dtype=dt, device=dev)
     _need(out, "out", dt, dev)
@@ -449,7 +459,7 @@ def kda_forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, output_fi
         final_state = torch.empty((shape.num_seqs, shape.num_v_heads, shape.head_dim_v, shape.head_dim_k),
                                   dtype=torch.float32, device=dev)
     _need(final_state, "final_state", torch.float32, dev)
-    nbytes = workspace_size(shape)
+    nbytes = kda_workspace_size(shape)
     if workspace is None or workspace.numel() < nbytes:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     osc = output_norm.c_struct(out) if output_norm is not None else None

@@ -88,7 +88,7 @@ def _segment_rel(err2, ref2, starts):
     return float((np.sqrt(e) / np.maximum(np.sqrt(r), 1e-30)).max())
 
 
-def full_prefill_errors(inp, o_gpu, sf_gpu, chunk=64, threads=None):
+def full_prefill_errors(inp, o_gpu, sf_gpu, chunk=64, threads=None, kda=False):
     """Every (sequence, value head) unit of a prefill against the fp64 oracle.
 
     The oracle runs a few q/k heads at a time (with their value heads), so
@@ -98,6 +98,8 @@ def full_prefill_errors(inp, o_gpu, sf_gpu, chunk=64, threads=None):
                slices of o, so that one wrong chunk cannot hide in a long slice
       state    max rel-L2 over the (sequence, head) final states
       units    (sequence, head) units compared
+    With ``kda`` the gates are per key channel ([..., Hv, d_k]) and the
+    oracle's KDA recurrence is the reference.
     """
     from oracle import oracle
     threads = threads or oracle.default_threads()
@@ -119,10 +121,11 @@ def full_prefill_errors(inp, o_gpu, sf_gpu, chunk=64, threads=None):
         q = to_f64(inp["q"][..., q0:q1, :])
         k = to_f64(inp["k"][..., q0:q1, :])
         v = to_f64(inp["v"][..., h0:h1, :])
-        g = to_f64(inp["g"][..., h0:h1])
+        g = to_f64(inp["g"][..., h0:h1, :]) if kda else to_f64(inp["g"][..., h0:h1])
         b = to_f64(inp["beta"][..., h0:h1])
         s0 = None if inp["initial_state"] is None else to_f64(inp["initial_state"][:, h0:h1])
-        o_ref, s_ref = oracle.recurrent(q, k, v, g, b, initial_state=s0, cu_seqlens=cu, threads=threads)
+        run = oracle.kda_recurrent if kda else oracle.recurrent
+        o_ref, s_ref = run(q, k, v, g, b, initial_state=s0, cu_seqlens=cu, threads=threads)
         o_ref = np.asarray(o_ref).reshape(-1, h1 - h0, dv)
         og = to_f64(og_all[:, h0:h1].cpu())
         err2 = ((og - o_ref) ** 2).sum(axis=-1)

@@ -132,3 +132,48 @@ def test_kda_decode(dtype, d, with_out):
     sg = to_f64(state)
     es = max(np.linalg.norm(sg[n, h] - ref[n, h]) / np.linalg.norm(ref[n, h]) for n in range(N) for h in range(hv))
     assert worst <= BAR[dtype] and es <= BAR[dtype], (worst, es)
+
+
+def test_kda_tensor_core_path_is_taken_and_matches_token_order():
+    """bf16, d = 128, C = 64 runs the tensor-core chunkwise form (its own launch
+    count: schedule, factors, chunk loop); the token-order kernel
+    (force_simt) agrees within rounding, and both meet the oracle."""
+    from linear_attention_sequence_sm_b200 import gdn
+    inp = kda_inputs(130, B=2, T=200, hk=2, hv=4, d=128, dtype="bf16")
+    n0 = gdn.launch_count()
+    o, sf = gpu_kda(inp)
+    assert gdn.launch_count() - n0 == 3
+    o2, sf2 = gpu_kda(inp, force_simt=True)
+    o_ref, sf_ref = oracle_kda(inp)
+    for oo, ss in ((o, sf), (o2, sf2)):
+        eo, es = prefill_errors(inp, oo, ss, o_ref, sf_ref)
+        assert eo <= BAR["bf16"] and es <= BAR["bf16"], (eo, es)
+
+
+@pytest.mark.parametrize("strong", [1, 40])
+def test_kda_tensor_core_strongly_decaying_channels(strong):
+    """Channels whose decay over a chunk passes e^-80 (here 3 per token for 64
+    tokens) leave the factorised Gram and are added with their exact
+    exponents; a few of them, and most of them."""
+    inp = kda_inputs(131, B=1, T=260, hk=1, hv=2, d=128, dtype="bf16")
+    g = inp["g"].clone()
+    g[..., :strong] = -3.0
+    inp["g"] = g
+    o, sf = gpu_kda(inp)
+    o_ref, sf_ref = oracle_kda(inp)
+    eo, es = prefill_errors(inp, o, sf, o_ref, sf_ref)
+    assert eo <= BAR["bf16"] and es <= BAR["bf16"], (eo, es)
+
+
+def test_kda_tensor_core_full_size_all_units():
+    """The 4 x 4096 prefill workload with per-channel decays, every (sequence,
+    value head) unit against the oracle, per slice and per 64-token chunk."""
+    from parity import full_prefill_errors
+    w = I.prefill_bf16()
+    inp = I.make_prefill_inputs(w)
+    inp["g"] = I.make_kda_gates(w)
+    o, sf = gpu_kda(inp)
+    err = full_prefill_errors(inp, o, sf, kda=True)
+    print(f"PARITY kda {w.name}: units {err['units']} o/slice {err['o_slice']:.3e} o/chunk {err['o_chunk']:.3e} "
+          f"state {err['state']:.3e}")
+    assert err["o_slice"] <= BAR["bf16"] and err["o_chunk"] <= BAR["bf16"] and err["state"] <= BAR["bf16"], err
