@@ -389,7 +389,8 @@ def prefill_record(args, w, host, device, world, rank, peaks, peak_src, e2e=True
     sf = torch.empty((w.num_seqs, w.hv, w.d, w.d), dtype=torch.float32, device=device)
     split = {"split": True} if args.split and not args.kda else {}
     shape = gdn.make_shape(dev["q"], dev["v"], dev["cu_seqlens"], w.chunk, **split)
-    ws = torch.empty(gdn.workspace_size(shape), dtype=torch.uint8, device=device)
+    ws = torch.empty(gdn.kda_workspace_size(shape) if args.kda else gdn.workspace_size(shape), dtype=torch.uint8,
+                     device=device)
     stream = torch.cuda.current_stream(device)
 
     if args.backward:
@@ -469,7 +470,17 @@ def prefill_record(args, w, host, device, world, rank, peaks, peak_src, e2e=True
         roofline = {"bound": "hbm", "achieved": cgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": cgbs / peaks["hbm_gbs"], "traffic": kernel_traffic(f"gdn_conv/{w.name}{suffix}"),
                     "kernel": "gdn_conv", "peak_source": f"{peak_src} HBM copy", "bytes_per_step": cbytes}
-    if args.kda:
+    if args.kda and gdn_tc_active(gdn, dev, w):
+        # the chunkwise WY form on the tensor cores: the gated delta rule's useful flops
+        # with the Gram per value head (G = 1: its decay differs per head)
+        kflops = useful_flops_per_vhead_token(1, w.d, w.chunk) * tokens * w.hv
+        achieved = kflops / (ms / 1e3) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": achieved / peaks["bf16_tflops"],
+                    "traffic": kernel_traffic(f"gdn_kda_factor+gdn_kda_chain/{w.name}{suffix}"),
+                    "kernel": "gdn_kda_factor+gdn_kda_chain", "peak_source": f"{peak_src} bf16 dense (burst)",
+                    "flops_per_launch": kflops, "algorithmic_bytes_per_launch": prefill_bytes(w, kda=True)}
+    elif args.kda:
         # token-order recurrence on CUDA cores: 7 d_v d_k fp32 flops per (token, value head)
         # (decay, two dot products, rank-1 write); peak = SMs x 128 fp32 lanes x 2 x max SM clock
         kflops = kda_flops_per_vhead_token(w.d) * tokens * w.hv

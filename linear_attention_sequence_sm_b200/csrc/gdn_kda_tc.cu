@@ -156,15 +156,26 @@ kda_factor_kernel(const PrefillArgs a, unsigned char *items) {
             }
         }
         __syncthreads();
-        // 2. prefix sums per channel, in place; the channels that decay past e^-80
-        if (tid < 128) {
+        // 2. prefix sums per channel, in place: each half of the tokens by its own
+        //    thread, then the second half offset by the first half's total
+        {
+            const int c = tid & 127, r0 = (tid >> 7) * 32;
             float acc = 0.f;
-            for (int r = 0; r < 64; ++r) {
-                acc += G[r * 128 + tid];
-                G[r * 128 + tid] = acc;
+#pragma unroll 8
+            for (int r = r0; r < r0 + 32; ++r) {
+                acc += G[r * 128 + c];
+                G[r * 128 + c] = acc;
             }
-            vec[kFVGl + tid] = acc;  // G_63 = G_(L-1): rows past the end carry g = 0
-            reinterpret_cast<float *>(it + kItGam)[tid] = __expf(acc);
+        }
+        __syncthreads();
+        if (tid >= 128) {
+            const int c = tid - 128;
+            const float base = G[31 * 128 + c];
+#pragma unroll 8
+            for (int r = 32; r < 64; ++r) G[r * 128 + c] += base;
+            const float gl = G[63 * 128 + c];
+            vec[kFVGl + c] = gl;  // G_63 = G_(L-1): rows past the end carry g = 0
+            reinterpret_cast<float *>(it + kItGam)[c] = __expf(gl);
         }
         __syncthreads();
         if (warp == 0) {
@@ -191,10 +202,14 @@ kda_factor_kernel(const PrefillArgs a, unsigned char *items) {
             const float sk = kL2 ? vec[kFVIk + r] : 1.f, sq = kL2 ? vec[kFVIq + r] : 1.f;
             const uint32_t kws[4] = {kw.x, kw.y, kw.z, kw.w}, qws[4] = {qw.x, qw.y, qw.z, qw.w};
             float kpv[8], kmv[8], khv[8], qpv[8];
+            float grv[8], glv[8];
+            load4(G + r * 128 + 8 * cc, grv);
+            load4(G + r * 128 + 8 * cc + 4, grv + 4);
+            load4(vec + kFVGl + 8 * cc, glv);
+            load4(vec + kFVGl + 8 * cc + 4, glv + 4);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int c = 8 * cc + u;
-                const float gr = G[r * 128 + c], gl = vec[kFVGl + c];
+                const float gr = grv[u], gl = glv[u];
                 const float kv = sk * __uint_as_float((u & 1) ? (kws[u >> 1] & 0xffff0000u) : (kws[u >> 1] << 16));
                 const float qv = sq * __uint_as_float((u & 1) ? (qws[u >> 1] & 0xffff0000u) : (qws[u >> 1] << 16));
                 const float eg = __expf(gr);
