@@ -94,6 +94,23 @@ def test_path_query_arguments(gdn):
         assert st == gdn.GDN_ERR_CUDA and p.value == -1
 
 
+def test_kda_workspace_size_follows_the_path(gdn):
+    """The tensor-core KDA form (bf16, d = 128, C = 64) needs its 66,048 bytes
+    per (chunk, value head) on top of the schedule; other shapes and
+    GDN_FLAG_FORCE_SIMT need only the schedule tables."""
+    kw = dict(batch=2, seq_len=200, num_seqs=2, num_qk_heads=2, num_v_heads=4, head_dim_k=128, head_dim_v=128,
+              chunk_size=64, dtype=gdn.GDN_DTYPE_BF16)
+    sched = gdn.workspace_size(_shape(gdn, flags=gdn.GDN_FLAG_ONE_KERNEL, **kw))
+    tc = gdn.kda_workspace_size(_shape(gdn, **kw))
+    assert tc >= sched + 2 * 4 * 4 * 66048  # 2 sequences x 4 chunks x 4 value heads
+    assert gdn.kda_workspace_size(_shape(gdn, flags=gdn.GDN_FLAG_FORCE_SIMT, **kw)) == sched
+    assert gdn.kda_workspace_size(_shape(gdn, **dict(kw, dtype=gdn.GDN_DTYPE_F32))) == sched
+    assert gdn.kda_workspace_size(_shape(gdn, **dict(kw, head_dim_k=64, head_dim_v=64))) == sched
+    n = ctypes.c_size_t(0)
+    bad = _shape(gdn, num_v_heads=3)
+    assert gdn.LIB.gdn_kda_forward_workspace_size(ctypes.byref(bad), ctypes.byref(n)) == gdn.GDN_ERR_INVALID_ARGUMENT
+
+
 def test_noalloc_status_arguments(gdn):
     """The built-in array's status reader refuses a NULL output; on a host
     without a GPU it reports GDN_ERR_CUDA rather than reading anything."""
