@@ -461,6 +461,10 @@ gdn_status_t gdn_chunk_backward_workspace_size(const gdn_shape_t *s, size_t *byt
     gdn_status_t st = check_shape(s);
     if (st != GDN_OK) return st;
     const int64_t tokens = int64_t(s->batch) * s->seq_len;
+    if (backward_tc_supported(*s) && !(s->flags & GDN_FLAG_FORCE_SIMT)) {
+        *bytes = bwd_tc_layout(*s).total;
+        return GDN_OK;
+    }
     *bytes = bwd_sched_bytes(s) +
              backward_ckpt_bytes(int32_t(tokens), s->num_seqs, s->num_v_heads, s->head_dim_k, s->head_dim_v);
     return GDN_OK;
@@ -476,6 +480,8 @@ gdn_status_t gdn_chunk_backward(const gdn_shape_t *s, const void *q, const void 
     if (st != GDN_OK) return st;
     if (s->flags & (GDN_FLAG_QK_L2NORM | GDN_FLAG_GATE_LOGITS))
         return fail(GDN_ERR_UNSUPPORTED, "the backward takes prepared inputs (no input-side flags)");
+    if (s->flags & (GDN_FLAG_ONE_KERNEL | GDN_FLAG_SPLIT))
+        return fail(GDN_ERR_UNSUPPORTED, "GDN_FLAG_ONE_KERNEL and GDN_FLAG_SPLIT select forward paths");
     const int64_t tokens = int64_t(s->batch) * s->seq_len;
     if (cu_seqlens) {
         if (s->batch != 1) return fail(GDN_ERR_INVALID_ARGUMENT, "batch must be 1 with cu_seqlens");
@@ -499,9 +505,16 @@ gdn_status_t gdn_chunk_backward(const gdn_shape_t *s, const void *q, const void 
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(GDN_ERR_MISALIGNED, "workspace is not 256-byte aligned");
     int major = 0;
-    if (device_sm_count(&major) <= 0) return fail(GDN_ERR_CUDA, "no usable CUDA device");
+    const int sms = device_sm_count(&major);
+    if (sms <= 0) return fail(GDN_ERR_CUDA, "no usable CUDA device");
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-    cudaError_t e = launch_schedule(*s, cu_seqlens, workspace, stream);
+    // the tensor-core form (bf16, d = 128) on sm_100 unless GDN_FLAG_FORCE_SIMT; its
+    // workspace size is what gdn_chunk_backward_workspace_size reports for such shapes
+    const bool tc = major == 10 && backward_tc_supported(*s) && !(s->flags & GDN_FLAG_FORCE_SIMT);
+    const BwdTcLayout TL = bwd_tc_layout(*s);
+    char *ws = static_cast<char *>(workspace);
+    cudaError_t e = tc ? launch_schedule(*s, cu_seqlens, workspace, stream, reinterpret_cast<int32_t *>(ws + TL.cbase_off))
+                       : launch_schedule(*s, cu_seqlens, workspace, stream);
     if (e != cudaSuccess) return cuda_fail(e, "schedule kernel launch");
     if (tokens > 0) {
         const size_t qk = size_t(tokens) * s->num_qk_heads * s->head_dim_k * sizeof(float);
@@ -525,13 +538,19 @@ gdn_status_t gdn_chunk_backward(const gdn_shape_t *s, const void *q, const void 
     a.flags = 0;
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.s0 = initial_state; a.o = nullptr; a.s_final = nullptr;
     a.out = OutSide{nullptr, nullptr, 0.f, 0u};
-    char *ws = static_cast<char *>(workspace);
     a.sched.hdr = reinterpret_cast<WsHeader *>(ws);
     a.sched.order = reinterpret_cast<const int32_t *>(ws + L.order_off);
     a.sched.start = reinterpret_cast<const int32_t *>(ws + L.start_off);
     a.sched.len = reinterpret_cast<const int32_t *>(ws + L.len_off);
     a.sched.chunk_base = nullptr;
     if (s->num_seqs == 0) return GDN_OK;
+    if (tc) {
+        a.sched.chunk_base = reinterpret_cast<const int32_t *>(ws + TL.cbase_off);
+        e = launch_backward_tc(a, d_o, d_final_state, dq, dk, dv, dg, dbeta, d_initial_state, nullptr,
+                               reinterpret_cast<unsigned char *>(ws), TL, stream, sms);
+        if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+        return GDN_OK;
+    }
     float *ckpt = reinterpret_cast<float *>(ws + bwd_sched_bytes(s));
     e = launch_chunk_backward(a, d_o, d_final_state, dq, dk, dv, dg, dbeta, d_initial_state, ckpt, stream);
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");

@@ -251,6 +251,22 @@ cudaError_t launch_chunk_chain(const PrefillArgs &a, const __nv_bfloat16 *tinv, 
 // The tensor-core KDA prefill: factor kernel, then chunk loop (gdn_kda_tc.cu).
 cudaError_t launch_kda_tc(const PrefillArgs &a, unsigned char *items, cudaStream_t stream, int num_sms);
 
+// The tensor-core backward (gdn_backward_tc.cu; bf16, d_k = d_v = 128): the
+// schedule tables, chunk_base, then per (chunk, value head) the factor item
+// (212,992 bytes) and two checkpoints (65,536 bytes each).
+struct BwdTcLayout {
+    WsLayout sched;
+    size_t cbase_off, items_off, ck_s_off, ck_ds_off, total;
+    int64_t max_chunks;
+};
+bool backward_tc_supported(const gdn_shape_t &s);
+BwdTcLayout bwd_tc_layout(const gdn_shape_t &s);
+// Factors, chains and gradients after the schedule kernel (which must fill
+// chunk_base); s_final, if not NULL, receives the final states.
+cudaError_t launch_backward_tc(const PrefillArgs &a, const void *dO, const float *dSf, float *dq, float *dk,
+                               float *dv, float *dg, float *dbeta, float *dS0, float *s_final, unsigned char *ws,
+                               const BwdTcLayout &L, cudaStream_t stream, int num_sms);
+
 // The output side as its own pass over o, in place (for the CUDA-core prefill,
 // whose blocks each own a slice of d_v).
 cudaError_t launch_output_side(void *o, int32_t tokens, int32_t hv, int32_t dv, int32_t dtype, const OutSide &os,

@@ -557,10 +557,12 @@ def decode_commit(snapshots, accepted, state, bad_count=None, stream=None):
 
 
 def chunk_backward(q, k, v, g, beta, d_o, d_final_state=None, initial_state=None, cu_seqlens=None,
-                   want_d_initial_state=True, workspace=None, stream=None):
+                   want_d_initial_state=True, workspace=None, stream=None, force_simt=False):
     """Gradients of sum d_o . o + sum d_final_state . S_final (training).
     Returns a dict of fp32 tensors: dq, dk (shaped like q), dv (like v),
-    dg, dbeta (like g), d_initial_state ([N, Hv, d_v, d_k], or None)."""
+    dg, dbeta (like g), d_initial_state ([N, Hv, d_v, d_k], or None).
+    bf16 inputs with d_k = d_v = 128 take the tensor-core kernels on sm_100
+    unless ``force_simt`` (GDN_FLAG_FORCE_SIMT) picks the single-kernel form."""
     n_seqs, hv, dv, dk = _prefill_shapes(q, k, v, g, beta, initial_state, cu_seqlens)
     _expect(d_o, "d_o", v.shape)
     _expect(d_final_state, "d_final_state", (n_seqs, hv, dv, dk))
@@ -572,7 +574,7 @@ def chunk_backward(q, k, v, g, beta, d_o, d_final_state=None, initial_state=None
     _need(initial_state, "initial_state", torch.float32, dev)
     _need(d_final_state, "d_final_state", torch.float32, dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
-    shape = make_shape(q, v, cu_seqlens, 32)
+    shape = make_shape(q, v, cu_seqlens, 32, force_simt=force_simt)
     n = ctypes.c_size_t(0)
     _check(LIB.gdn_chunk_backward_workspace_size(ctypes.byref(shape), ctypes.byref(n)))
     if workspace is None or workspace.numel() < n.value:
