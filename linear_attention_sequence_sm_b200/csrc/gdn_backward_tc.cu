@@ -160,6 +160,59 @@ __device__ __forceinline__ void colsum_add(float (&v)[32], bool valid, float *ds
     }
 }
 
+// Adds to the transaction count of the current phase without arriving.
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// Reads of an M = 64 accumulator with every lane busy (16x32bx2 shape):
+// threads 0-15 read lanes 0-15 of the warp's quarter (rows 16 (warp % 4) +
+// lane) at column `col`, threads 16-31 the same rows at `col + 32`.
+__device__ __forceinline__ void tmem_ld_h16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16], 32;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_ld_h32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32], 32;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Column sums over the 16 lanes of each half-warp, 16 values per lane: four
+// halving exchanges leave lane l with the sum of column l % 16; added into
+// dst[l % 16] (dst: this half-warp's columns).
+__device__ __forceinline__ void colsum16_add(float (&x)[16], float *dst, int lane) {
+#pragma unroll
+    for (int n = 8, bit = 8; n >= 1; n >>= 1, bit >>= 1) {
+        const bool up = (lane & bit) != 0;
+#pragma unroll
+        for (int m = 0; m < n; ++m) {
+            const float send = up ? x[m] : x[m + n];
+            const float keep = up ? x[m + n] : x[m];
+            x[m] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+        }
+    }
+    atomicAdd(dst + (lane & 15), x[0]);
+}
+
 // Waits on an mbarrier phase with every thread polling (bounded); true on
 // success for the whole block.
 __device__ __forceinline__ bool block_wait(uint32_t bar, uint32_t parity) {
@@ -669,10 +722,14 @@ bwd_chain_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, co
 constexpr uint32_t kDK = 0, kDQ = 16384;        // K, Q [64][128] (TMA)
 constexpr uint32_t kDV = 32768, kDO = 40960;    // V, dO: the half's 64 columns [64][64] (TMA)
 constexpr uint32_t kDT = 49152, kDTb = 65536, kDTbg = 81920;  // T, T diag(beta), T diag(beta gamma) pairs
-constexpr uint32_t kDS0 = 98304;   // S_c half pair [64][128]; then M = dT T^T (+0) and dKK (+16384) pairs
+constexpr uint32_t kDS0 = 98304;   // S_c half pair [64][128]
 constexpr uint32_t kDdS = 131072;  // dS_{c+1} half pair; then dU^T (+0) and dP (.) Gamma (+16384) pairs
 constexpr uint32_t kDR1 = 163840;  // W pair; then U^T (+0) and (U diag(lambda))^T (+16384); then dW pair
-constexpr uint32_t kDgO = 196608;  // diag(gamma) dO pair [64][64]; then P; then dT
+constexpr uint32_t kDgO = 196608;  // diag(gamma) dO pair [64][64]; then P, dT, M = dT T^T and dKK in turn
+// The next unit's inputs are loaded while this one finishes, each into its
+// buffer once the buffer's last reader has completed: after the third group
+// of products S_c, dS, Q, V, dO and T diag(beta); after the fourth W and
+// T diag(beta gamma); after the sixth T; after the seventh K.
 constexpr uint32_t kDVec = 212992;
 constexpr uint32_t kDBar = kDVec + 4096;
 constexpr uint32_t kDSmem = kDBar + 64 + 1024;
@@ -718,9 +775,11 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
     const int hv = a.hv, hk = a.hk, group = hv / hk;
     const int64_t total = aborted ? 0 : int64_t(hdr->total_chunks) * hv * 2;
     uint32_t lph = 0, mph = 0;
-    const int half = warp >> 2, r64 = 16 * (warp & 3) + (lane & 15);
-    const bool v64 = lane < 16;
-    const int c32 = 32 * half;  // this warp's columns of a 64-column accumulator
+    // accumulator reads: row rr of an M = 64 accumulator; of a 64-column one the 16
+    // columns cb .. cb + 15, of a 128-column one the 32 columns cb2 .. cb2 + 31
+    // (warp group wg = warp / 4 takes columns 64 wg ..)
+    const int wg = warp >> 2, rr = 16 * (warp & 3) + (lane & 15);
+    const int cb = 16 * wg + 32 * (lane >> 4), cb2 = 32 * (lane >> 4);
 
     // one group of products, then every thread waits for it
     auto group_done = [&]() -> bool {
@@ -736,10 +795,10 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
         tc_fence_before();
         __syncthreads();
     };
-    // 32 values (this lane's row, columns c0 .. c0 + 31 of a 64-column tile) as a split pair
-    auto stage32 = [&](uint32_t tile, int r, int c0, const float *x) {
+    // 16 values (row r, columns c0 .. c0 + 15 of a 64-column tile) as a split pair
+    auto stage16 = [&](uint32_t tile, int r, int c0, const float *x) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
             uint4 hi, lo;
             split8(x + 8 * c, hi, lo);
             const uint32_t off = sw128_offset(r, c0 / 8 + c);
@@ -748,43 +807,76 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
         }
     };
 
-    for (int64_t unit = blockIdx.x; unit < total; unit += gridDim.x) {
+    // a unit's coordinates
+    struct Unit {
+        int sh, i0, h, hq, t0, L;
+        const unsigned char *it, *cs0, *cds;
+    };
+    auto decode = [&](int64_t unit) {
+        Unit U;
         const int64_t item = unit >> 1;
-        const int sh = int(unit & 1), i0 = 64 * sh;
-        const int gc = int(item / hv), h = int(item - int64_t(gc) * hv), hq = h / group;
+        U.sh = int(unit & 1);
+        U.i0 = 64 * U.sh;
+        const int gc = int(item / hv);
+        U.h = int(item - int64_t(gc) * hv);
+        U.hq = U.h / group;
         const int n = chunk_sequence(a.sched.chunk_base, a.num_seqs, gc);
         const int c0 = gc - a.sched.chunk_base[n];
-        const int t0 = a.sched.start[n] + 64 * c0;
-        const int L = min(64, a.sched.len[n] - 64 * c0);
-        const unsigned char *it = items + size_t(item) * kItemBytes;
-        const unsigned char *cs0 = ck_s + size_t(item) * kCkBytes, *cds = ck_ds + size_t(item) * kCkBytes;
-
-        if (tid == 0) {
-            // K, Q, V and dO halves; T, T diag(beta), T diag(beta gamma); W; the two checkpoint halves
-            mbar_arrive_expect_tx(lbar, (2 * 16384 + 2 * 8192) + 3 * 16384 + 32768 + 2 * 32768);
-            tma_load_3d(sb + kDK, &tk, 0, hq, t0, lbar);
-            tma_load_3d(sb + kDK + 8192, &tk, 64, hq, t0, lbar);
-            tma_load_3d(sb + kDQ, &tq, 0, hq, t0, lbar);
-            tma_load_3d(sb + kDQ + 8192, &tq, 64, hq, t0, lbar);
-            tma_load_3d(sb + kDV, &tv, i0, h, t0, lbar);
-            tma_load_3d(sb + kDO, &tdo, i0, h, t0, lbar);
-            bulk_load(sb + kDT, it + kIT, 16384, lbar);
-            bulk_load(sb + kDTb, it + kITb, 16384, lbar);
-            bulk_load(sb + kDTbg, it + kITbg, 16384, lbar);
-            bulk_load(sb + kDR1, it + kIW, 32768, lbar);
-            // rows i0 .. i0 + 63 of each atom of the two checkpoint pairs
-            for (int q = 0; q < 4; ++q) {
-                const uint32_t src = uint32_t(q) * 16384 + uint32_t(sh) * 8192, dst = uint32_t(q) * 8192;
-                bulk_load(sb + kDS0 + dst, cs0 + src, 8192, lbar);
-                bulk_load(sb + kDdS + dst, cds + src, 8192, lbar);
+        U.t0 = a.sched.start[n] + 64 * c0;
+        U.L = min(64, a.sched.len[n] - 64 * c0);
+        U.it = items + size_t(item) * kItemBytes;
+        U.cs0 = ck_s + size_t(item) * kCkBytes;
+        U.cds = ck_ds + size_t(item) * kCkBytes;
+        return U;
+    };
+    // the unit's inputs, in the four sets the prefetch uses (thread 0; set 3 arrives)
+    auto load_set = [&](const Unit &U, int set) {
+        if (set == 0) {
+            mbar_expect_tx(lbar, 2 * 32768 + 16384 + 2 * 8192 + 16384);
+            for (int q = 0; q < 4; ++q) {  // rows i0 .. i0 + 63 of each atom of the two checkpoint pairs
+                const uint32_t src = uint32_t(q) * 16384 + uint32_t(U.sh) * 8192, dst = uint32_t(q) * 8192;
+                bulk_load(sb + kDS0 + dst, U.cs0 + src, 8192, lbar);
+                bulk_load(sb + kDdS + dst, U.cds + src, 8192, lbar);
             }
+            tma_load_3d(sb + kDQ, &tq, 0, U.hq, U.t0, lbar);
+            tma_load_3d(sb + kDQ + 8192, &tq, 64, U.hq, U.t0, lbar);
+            tma_load_3d(sb + kDV, &tv, U.i0, U.h, U.t0, lbar);
+            tma_load_3d(sb + kDO, &tdo, U.i0, U.h, U.t0, lbar);
+            bulk_load(sb + kDTb, U.it + kITb, 16384, lbar);
+        } else if (set == 1) {
+            mbar_expect_tx(lbar, 32768 + 16384);
+            bulk_load(sb + kDR1, U.it + kIW, 32768, lbar);
+            bulk_load(sb + kDTbg, U.it + kITbg, 16384, lbar);
+        } else if (set == 2) {
+            mbar_expect_tx(lbar, 16384);
+            bulk_load(sb + kDT, U.it + kIT, 16384, lbar);
+        } else {
+            mbar_arrive_expect_tx(lbar, 16384);
+            tma_load_3d(sb + kDK, &tk, 0, U.hq, U.t0, lbar);
+            tma_load_3d(sb + kDK + 8192, &tk, 64, U.hq, U.t0, lbar);
         }
+    };
+    bool pending = false;  // a load phase is open (thread 0)
+    if (tid == 0 && total > int64_t(blockIdx.x)) {
+        const Unit U = decode(blockIdx.x);
+        for (int set = 0; set < 4; ++set) load_set(U, set);
+        pending = true;
+    }
+
+    for (int64_t unit = blockIdx.x; unit < total; unit += gridDim.x) {
+        const Unit U = decode(unit);
+        const int i0 = U.i0, h = U.h, hq = U.hq, t0 = U.t0, L = U.L;
+        const int64_t next = unit + gridDim.x;
+        const bool has_next = next < total;
+        Unit N{};
+        if (tid == 0 && has_next) N = decode(next);
         if (tid < 64)
             for (int v = kVll; v < kVNum; ++v) vec[64 * v + tid] = 0.f;
         if (tid < 2) scal[tid] = 0.f;
         chunk_vectors(a, t0, L, h, cv, tid);
         if (!block_wait(lbar, lph)) { aborted = true; break; }
         lph ^= 1u;
+        if (tid == 0) pending = false;
         // diag(gamma) dO (rows < L) as a split pair
         for (int e = tid; e < 64 * 8; e += kThr) {
             const int r = e >> 3, ch = e & 7;
@@ -814,115 +906,99 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
             product(tmem + kTdQ, gO, S0mn, 64, 128, 4, false, false);
         }
         if (!group_done()) { aborted = true; break; }
-        // ---- E1
+        // ---- E1.  Every 64-column accumulator is read by all eight warps, 16 columns a
+        // thread (columns cb .. cb + 15 of row rr); 128-column ones 32 a thread (cb2 ..).
+        float zl[16];  // lambda_j Z_ij, kept for dU^T
         {
-            float u[32], z[32];
-            tmem_ld32(tlane(tmem, warp, kTSA + c32), u);
-            tmem_ld32(tlane(tmem, warp, kTSB + c32), z);
+            float u[16], ul[16], pr[16];
+            tmem_ld_h16(tlane(tmem, warp, kTSA + 16 * wg), u);
+            tmem_ld_h16(tlane(tmem, warp, kTSB + 16 * wg), zl);
             tmem_wait_ld();
-            float pr[32], ul[32];
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                const int j = c32 + q;
+            for (int q = 0; q < 16; ++q) {
+                const int j = cb + q;
                 const float lj = j < L ? cv.lam[j] : 0.f;
-                z[q] *= lj;  // lambda_j Z_ij
-                pr[q] = u[q] * z[q];
+                zl[q] *= lj;
+                pr[q] = u[q] * zl[q];
                 ul[q] = lj * u[q];
             }
-            tmem_st32(tlane(tmem, warp, kTSB + c32), z);
-            colsum_add(pr, v64, dll + c32, lane);
-            if (v64) {
-                stage32(sb + kDR1, r64, c32, u);
-                stage32(sb + kDR1 + 16384, r64, c32, ul);
-            }
+            colsum16_add(pr, dll + cb, lane);
+            stage16(sb + kDR1, rr, cb, u);
+            stage16(sb + kDR1 + 16384, rr, cb, ul);
             // P = Q K^T (.) Gamma (lower, rows < L)
-            tmem_ld32(tlane(tmem, warp, kTQK2 + c32), u);
+            tmem_ld_h16(tlane(tmem, warp, kTQK2 + 16 * wg), u);
             tmem_wait_ld();
-            if (v64) {
-                const float Gr = cv.G[r64];
+            const float Gr = cv.G[rr];
 #pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    const int j = c32 + q;
-                    u[q] = (j <= r64 && r64 < L) ? __expf(Gr - cv.G[j]) * u[q] : 0.f;
-                }
-                stage32(sb + kDgO, r64, c32, u);
+            for (int q = 0; q < 16; ++q) {
+                const int j = cb + q;
+                u[q] = (j <= rr && rr < L) ? __expf(Gr - cv.G[j]) * u[q] : 0.f;
             }
-            // gamma_r dgamma_r (dO S_c part) = sum_x Y'_rx q_rx over this warp's 64 columns
-            float part = 0.f;
-#pragma unroll 1
-            for (int p = 0; p < 2; ++p) {
-                tmem_ld32(tlane(tmem, warp, kTdQ + 64 * half + 32 * p), u);
-                tmem_wait_ld();
-                if (v64) {
+            stage16(sb + kDgO, rr, cb, u);
+            // gamma_r dgamma_r (dO S_c part) = sum_x Y'_rx q_rx over this thread's 32 columns
+            float y[32], part = 0.f;
+            tmem_ld_h32(tlane(tmem, warp, kTdQ + 64 * wg), y);
+            tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        float qv[8];
-                        unpack8(ld_shared_v4(sb + kDQ + uint32_t(half) * 8192 + sw128_offset(r64, 4 * p + c)), qv);
+            for (int c = 0; c < 4; ++c) {
+                float qv[8];
+                unpack8(ld_shared_v4(sb + kDQ + uint32_t(wg) * 8192 + sw128_offset(rr, cb2 / 8 + c)), qv);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) part = fmaf(u[8 * c + e], qv[e], part);
-                    }
-                }
+                for (int e = 0; e < 8; ++e) part = fmaf(y[8 * c + e], qv[e], part);
             }
-            if (v64) atomicAdd(dgg + r64, part);
+            atomicAdd(dgg + rr, part);
             // <dS_{c+1}, S_c> over the half
             float dot = 0.f;
             for (int e = tid; e < 64 * 16; e += kThr) {
                 const int r = e >> 4, a8 = (e >> 3) & 1, ch = e & 7;
                 const uint32_t off = uint32_t(a8) * 8192 + sw128_offset(r, ch);
-                float x[8], y[8];
+                float x[8], w8[8];
                 ld_pair8(sb + kDS0 + off, sb + kDS0 + 16384 + off, x);
-                ld_pair8(sb + kDdS + off, sb + kDdS + 16384 + off, y);
+                ld_pair8(sb + kDdS + off, sb + kDdS + 16384 + off, w8);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) dot = fmaf(x[q], y[q], dot);
+                for (int q = 0; q < 8; ++q) dot = fmaf(x[q], w8[q], dot);
             }
 #pragma unroll
             for (int m = 16; m > 0; m >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, m);
             if (lane == 0) atomicAdd(scal, dot);
         }
-        tmem_wait_st();
         stage_done();
-        // ---- G2: dU^T += dO^T P, dP = dO U^T, dK = (U diag(lambda)) dS
+        // ---- G2: dO^T P, dP = dO U^T, dK = (U diag(lambda)) dS
         if (tid == 0) {
             tc_fence_after();
             const Opd dOmn{sb + kDO, 0, 8192, true}, Pmn{sb + kDgO, 8192, 8192, true};
             const Opd dO{sb + kDO, 0, 8192, false}, Utmn{sb + kDR1, 8192, 8192, true};
             const Opd Ulmn{sb + kDR1 + 16384, 8192, 8192, true}, dSmn{sb + kDdS, 16384, 8192, true};
-            product(tmem + kTSB, dOmn, Pmn, 64, 64, 4, false, true);
+            product(tmem + kTSB, dOmn, Pmn, 64, 64, 4, false, false);
             product(tmem + kTSA, dO, Utmn, 64, 64, 4, false, false);
             product(tmem + kTdK, Ulmn, dSmn, 64, 128, 4, false, false);
         }
         if (!group_done()) { aborted = true; break; }
-        // ---- E2
+        // ---- E2: dU^T = lambda Z^T + dO^T P (columns < L); dP (.) Gamma and its dGamma sums
         {
-            float x[32], y[32];
-            tmem_ld32(tlane(tmem, warp, kTSB + c32), x);  // dU^T: rows i, columns r
+            float x[16], y[16];
+            tmem_ld_h16(tlane(tmem, warp, kTSB + 16 * wg), x);
             tmem_wait_ld();
-            if (v64) {
 #pragma unroll
-                for (int q = 0; q < 32; ++q)
-                    if (c32 + q >= L) x[q] = 0.f;
-                stage32(sb + kDdS, r64, c32, x);
-            }
-            tmem_ld32(tlane(tmem, warp, kTSA + c32), x);   // dP: rows r, columns j
-            tmem_ld32(tlane(tmem, warp, kTQK2 + c32), y);  // Q K^T
+            for (int q = 0; q < 16; ++q) x[q] = cb + q < L ? x[q] + zl[q] : 0.f;
+            stage16(sb + kDdS, rr, cb, x);
+            tmem_ld_h16(tlane(tmem, warp, kTSA + 16 * wg), x);   // dP: rows r, columns j
+            tmem_ld_h16(tlane(tmem, warp, kTQK2 + 16 * wg), y);  // Q K^T
             tmem_wait_ld();
             float rsum = 0.f;
-            const float Gr = cv.G[r64];
+            const float Gr = cv.G[rr];
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                const int j = c32 + q;
-                const bool ok = j <= r64 && r64 < L;
+            for (int q = 0; q < 16; ++q) {
+                const int j = cb + q;
+                const bool ok = j <= rr && rr < L;
                 const float gm = ok ? __expf(Gr - cv.G[j]) : 0.f;
-                const float dp = ok ? x[q] : 0.f;
-                x[q] = dp * gm;           // dP (.) Gamma
-                y[q] = x[q] * y[q];       // dGamma_rj Gamma_rj (the P part)
+                x[q] = ok ? x[q] * gm : 0.f;  // dP (.) Gamma
+                y[q] = x[q] * y[q];           // dGamma_rj Gamma_rj (the P part)
                 rsum += y[q];
             }
-            if (v64) {
-                stage32(sb + kDdS + 16384, r64, c32, x);
-                atomicAdd(rs + r64, rsum);
-            }
-            colsum_add(y, v64, cs + c32, lane);
+            stage16(sb + kDdS + 16384, rr, cb, x);
+            atomicAdd(rs + rr, rsum);
+            colsum16_add(y, cs + cb, lane);
         }
         stage_done();
         // ---- G3: dQ += (dP (.) Gamma) K, dK += (dP (.) Gamma)^T Q, dW = -dU S_c, dT2 = dU V^T, dV = T''^T dU
@@ -940,31 +1016,31 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
             product(tmem + kTSB, Tbmn, dUt, 64, 64, 4, false, false);
         }
         if (!group_done()) { aborted = true; break; }
+        if (tid == 0 && has_next) {
+            load_set(N, 0);
+            pending = true;
+        }
         // ---- E3: dv (this half's columns, rows < L); dW as a split pair
         {
-            float x[32];
-            tmem_ld32(tlane(tmem, warp, kTSB + c32), x);
+            float x[16];
+            tmem_ld_h16(tlane(tmem, warp, kTSB + 16 * wg), x);
             tmem_wait_ld();
-            if (v64 && r64 < L) {
-                float *dst = dv + (size_t(t0 + r64) * hv + h) * 128 + i0 + c32;
+            if (rr < L) {
+                float *dst = dv + (size_t(t0 + rr) * hv + h) * 128 + i0 + cb;
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
+                for (int q = 0; q < 4; ++q)
                     *reinterpret_cast<float4 *>(dst + 4 * q) = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
             }
-#pragma unroll 1
-            for (int p = 0; p < 2; ++p) {
-                tmem_ld32(tlane(tmem, warp, kTdW + 64 * half + 32 * p), x);
-                tmem_wait_ld();
-                if (v64) {
+            float y[32];
+            tmem_ld_h32(tlane(tmem, warp, kTdW + 64 * wg), y);
+            tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint4 hi, lo;
-                        split8(x + 8 * c, hi, lo);
-                        const uint32_t off = uint32_t(half) * 8192 + sw128_offset(r64, 4 * p + c);
-                        st_shared_v4(sb + kDR1 + off, hi);
-                        st_shared_v4(sb + kDR1 + 16384 + off, lo);
-                    }
-                }
+            for (int c = 0; c < 4; ++c) {
+                uint4 hi, lo;
+                split8(y + 8 * c, hi, lo);
+                const uint32_t off = uint32_t(wg) * 8192 + sw128_offset(rr, cb2 / 8 + c);
+                st_shared_v4(sb + kDR1 + off, hi);
+                st_shared_v4(sb + kDR1 + 16384 + off, lo);
             }
         }
         stage_done();
@@ -977,33 +1053,31 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
             product(tmem + kTdK, Tbgmn, dWmn, 64, 128, 4, false, true);
         }
         if (!group_done()) { aborted = true; break; }
+        if (tid == 0 && has_next) load_set(N, 1);
         // ---- E4: dT (lower, rows < L) as a split pair; T (.) dT1 and T (.) dT2 column sums
         {
-            float x1[32], x2[32];
-            tmem_ld32(tlane(tmem, warp, kTdT1 + c32), x1);
-            tmem_ld32(tlane(tmem, warp, kTSA + c32), x2);
-            tmem_wait_ld();
-            const bool ok = v64 && r64 < L;
-            float t[32];
-            if (v64) {
+            float x1[16], x2[16], t[16];
+            tmem_ld_h16(tlane(tmem, warp, kTdT1 + 16 * wg), x1);
+            tmem_ld_h16(tlane(tmem, warp, kTSA + 16 * wg), x2);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint32_t off = sw128_offset(r64, c32 / 8 + c);
-                    ld_pair8(sb + kDT + off, sb + kDT + 8192 + off, t + 8 * c);
-                }
+            for (int c = 0; c < 2; ++c) {
+                const uint32_t off = sw128_offset(rr, cb / 8 + c);
+                ld_pair8(sb + kDT + off, sb + kDT + 8192 + off, t + 8 * c);
             }
-            float p1[32], p2[32];
+            tmem_wait_ld();
+            const bool ok = rr < L;
+            float p1[16], p2[16];
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                const int j = c32 + q;
+            for (int q = 0; q < 16; ++q) {
+                const int j = cb + q;
                 const float tv = ok ? t[q] : 0.f;
                 p1[q] = tv * x1[q];
                 p2[q] = tv * x2[q];
-                x1[q] = (ok && j <= r64) ? fmaf(cv.bg[j], x1[q], cv.beta[j] * x2[q]) : 0.f;
+                x1[q] = (ok && j <= rr) ? fmaf(cv.bg[j], x1[q], cv.beta[j] * x2[q]) : 0.f;
             }
-            if (v64) stage32(sb + kDgO, r64, c32, x1);
-            colsum_add(p1, ok, dbgv + c32, lane);
-            colsum_add(p2, ok, dyv + c32, lane);
+            stage16(sb + kDgO, rr, cb, x1);
+            colsum16_add(p1, dbgv + cb, lane);
+            colsum16_add(p2, dyv + cb, lane);
         }
         stage_done();
         // ---- G5: M = dT T^T
@@ -1014,33 +1088,34 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
         }
         if (!group_done()) { aborted = true; break; }
         {
-            float x[32];
-            tmem_ld32(tlane(tmem, warp, kTSA + c32), x);
+            float x[16];
+            tmem_ld_h16(tlane(tmem, warp, kTSA + 16 * wg), x);
             tmem_wait_ld();
-            if (v64) stage32(sb + kDS0, r64, c32, x);
+            stage16(sb + kDgO, rr, cb, x);  // M (dT, its operand, is consumed)
         }
         stage_done();
         // ---- G6: dA = -T^T M, K K^T
         if (tid == 0) {
             tc_fence_after();
-            const Opd Tmn{sb + kDT, 8192, 8192, true}, Mmn{sb + kDS0, 8192, 8192, true};
+            const Opd Tmn{sb + kDT, 8192, 8192, true}, Mmn{sb + kDgO, 8192, 8192, true};
             const Opd K{sb + kDK, 0, 8192, false};
             product(tmem + kTSB, Tmn, Mmn, 64, 64, 4, true, false);
             product(tmem + kTKK2, K, K, 64, 64, 8, false, false);
         }
         if (!group_done()) { aborted = true; break; }
+        if (tid == 0 && has_next) load_set(N, 2);
         // ---- E6: from dA (strictly lower, rows < L): dbeta, dGamma, dKK
         {
-            float da[32], kk[32];
-            tmem_ld32(tlane(tmem, warp, kTSB + c32), da);
-            tmem_ld32(tlane(tmem, warp, kTKK2 + c32), kk);
+            float da[16], kk[16];
+            tmem_ld_h16(tlane(tmem, warp, kTSB + 16 * wg), da);
+            tmem_ld_h16(tlane(tmem, warp, kTKK2 + 16 * wg), kk);
             tmem_wait_ld();
-            const int j = r64;
+            const int j = rr;
             const float Gj = cv.G[j], bj = cv.beta[j];
-            float sab = 0.f, srs = 0.f, e[32];
+            float sab = 0.f, srs = 0.f, e[16];
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                const int m = c32 + q;
+            for (int q = 0; q < 16; ++q) {
+                const int m = cb + q;
                 const bool ok = m < j && j < L;
                 const float gm = ok ? __expf(Gj - cv.G[m]) : 0.f;
                 const float d = ok ? da[q] : 0.f;
@@ -1049,42 +1124,35 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
                 srs += e[q];
                 da[q] = d * bj * gm;  // dKK
             }
-            if (v64) {
-                atomicAdd(dab + j, sab);
-                atomicAdd(rs + j, srs);
-                stage32(sb + kDS0 + 16384, j, c32, da);
-            }
-            colsum_add(e, v64, cs + c32, lane);
+            atomicAdd(dab + j, sab);
+            atomicAdd(rs + j, srs);
+            stage16(sb + kDgO, j, cb, da);  // dKK (M is consumed)
+            colsum16_add(e, cs + cb, lane);
         }
         stage_done();
         // ---- G7: dK += dKK K + dKK^T K
         if (tid == 0) {
             tc_fence_after();
-            const Opd dKK{sb + kDS0 + 16384, 8192, 8192, false}, dKKmn{sb + kDS0 + 16384, 8192, 8192, true};
+            const Opd dKK{sb + kDgO, 8192, 8192, false}, dKKmn{sb + kDgO, 8192, 8192, true};
             const Opd Kmn{sb + kDK, 0, 8192, true};
             product(tmem + kTdK, dKK, Kmn, 64, 128, 4, false, true);
             product(tmem + kTdK, dKKmn, Kmn, 64, 128, 4, false, true);
         }
         if (!group_done()) { aborted = true; break; }
+        if (tid == 0 && has_next) load_set(N, 3);
         // ---- E7: dq, dk (this half's shares, rows < L); dG, dbeta, dg
-        {
 #pragma unroll 1
-            for (int which = 0; which < 2; ++which) {
-                float *base = which == 0 ? dq : dk;
-                const int col = which == 0 ? kTdQ : kTdK;
-#pragma unroll 1
-                for (int p = 0; p < 2; ++p) {
-                    float x[32];
-                    tmem_ld32(tlane(tmem, warp, col + 64 * half + 32 * p), x);
-                    tmem_wait_ld();
-                    if (v64 && r64 < L) {
-                        float *dst = base + (size_t(t0 + r64) * hk + hq) * 128 + 64 * half + 32 * p;
+        for (int which = 0; which < 2; ++which) {
+            float *base = which == 0 ? dq : dk;
+            float x[32];
+            tmem_ld_h32(tlane(tmem, warp, (which == 0 ? kTdQ : kTdK) + 64 * wg), x);
+            tmem_wait_ld();
+            if (rr < L) {
+                float *dst = base + (size_t(t0 + rr) * hk + hq) * 128 + 64 * wg + 32 * (lane >> 4);
 #pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            atomicAdd(reinterpret_cast<float4 *>(dst + 4 * q),
-                                      make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]));
-                    }
-                }
+                for (int q = 0; q < 8; ++q)
+                    atomicAdd(reinterpret_cast<float4 *>(dst + 4 * q),
+                              make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]));
             }
         }
         if (tid < 64) {
@@ -1120,6 +1188,10 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
     if (aborted && tid == 0 && total > 0) {
         mma_commit(mbar);
         (void)mbar_wait(mbar, mph);
+        if (pending) {  // loads in flight into this CTA's shared memory: let them land
+            mbar_arrive(lbar);
+            (void)mbar_wait(lbar, lph);
+        }
         record_abort(hdr, -8);
     }
     tc_fence_before();
