@@ -318,8 +318,10 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
     const int64_t total = aborted ? 0 : int64_t(hdr->total_chunks) * hv;
     uint32_t lph = 0, mph = 0;
     const int q4 = warp & 3, half = warp >> 2;
-    const int r64 = 16 * q4 + (lane & 15);  // this lane's row of an M = 64 accumulator (lanes 0-15)
-    const bool v64 = lane < 16;
+    // M = 64 accumulators, read with every lane busy: row rr; of a 64-column one the
+    // 16 columns cb .. cb + 15, of a 128-column one the 32 columns 64 half + cb2 ..
+    const int rr = 16 * q4 + (lane & 15);
+    const int cb = 16 * half + 32 * (lane >> 4), cb2 = 32 * (lane >> 4);
 
     for (int64_t item = blockIdx.x; item < total; item += gridDim.x) {
         const int gc = int(item / hv), h = int(item - int64_t(gc) * hv), hq = h / group;
@@ -354,35 +356,33 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
         tc_fence_after();
         // A (fp32, strictly lower) from K K^T; P = Q K^T (.) Gamma (lower, rows < L) as a split pair
         {
-            const int col0 = 32 * half;
-            float v[32];
-            tmem_ld32(tlane(tmem, warp, kTKK + col0), v);
+            float v[16];
+            tmem_ld_h16(tlane(tmem, warp, kTKK + 16 * half), v);
             tmem_wait_ld();
-            if (v64) {
-                const float br = cv.beta[r64], Gr = cv.G[r64];
+            const float br = cv.beta[rr], Gr = cv.G[rr];
 #pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                    const int j = col0 + u;
-                    Af[r64 * kLdA + j] = j < r64 ? br * __expf(Gr - cv.G[j]) * v[u] : 0.f;
+            for (int q = 0; q < 4; ++q) {
+                float x[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int j = cb + 4 * q + u;
+                    x[u] = j < rr ? br * __expf(Gr - cv.G[j]) * v[4 * q + u] : 0.f;
                 }
+                *reinterpret_cast<float4 *>(Af + rr * kLdA + cb + 4 * q) = make_float4(x[0], x[1], x[2], x[3]);
             }
-            tmem_ld32(tlane(tmem, warp, kTQK + col0), v);
+            tmem_ld_h16(tlane(tmem, warp, kTQK + 16 * half), v);
             tmem_wait_ld();
-            if (v64) {
-                const float Gr = cv.G[r64];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    float x[8];
+            for (int u = 0; u < 16; ++u) {
+                const int j = cb + u;
+                v[u] = (j <= rr && rr < L) ? __expf(Gr - cv.G[j]) * v[u] : 0.f;
+            }
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int j = col0 + 8 * c + u;
-                        x[u] = (j <= r64 && r64 < L) ? __expf(Gr - cv.G[j]) * v[8 * c + u] : 0.f;
-                    }
-                    uint4 hi, lo;
-                    split8(x, hi, lo);
-                    st_shared_v4(sb + kAP + sw128_offset(r64, 4 * half + c), hi);
-                    st_shared_v4(sb + kAP + 8192 + sw128_offset(r64, 4 * half + c), lo);
-                }
+            for (int c = 0; c < 2; ++c) {
+                uint4 hi, lo;
+                split8(v + 8 * c, hi, lo);
+                st_shared_v4(sb + kAP + sw128_offset(rr, cb / 8 + c), hi);
+                st_shared_v4(sb + kAP + 8192 + sw128_offset(rr, cb / 8 + c), lo);
             }
         }
         tc_fence_before();
@@ -433,49 +433,41 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
         mph ^= 1u;
         tc_fence_after();
         // W: pair to shared memory and the item, W diag(lambda) to shared memory;
-        // U~ diag(lambda) to the item (this warp: 64 of the 128 columns, one atom)
+        // U~ diag(lambda) to the item (columns 64 half + cb2 .. + 31: atom `half`)
         {
             const uint32_t atom = uint32_t(half) * 8192;
-#pragma unroll 1
-            for (int p = 0; p < 2; ++p) {
-                float v[32];
-                tmem_ld32(tlane(tmem, warp, kTW + 64 * half + 32 * p), v);
-                tmem_wait_ld();
-                if (v64) {
-                    const float lr = cv.lam[r64];
+            const float lr = cv.lam[rr];
+            float v[32];
+            tmem_ld_h32(tlane(tmem, warp, kTW + 64 * half), v);
+            tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint32_t off = atom + sw128_offset(r64, 4 * p + c);
-                        float wl[8];
+            for (int c = 0; c < 4; ++c) {
+                const uint32_t off = atom + sw128_offset(rr, cb2 / 8 + c);
+                float wl[8];
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) wl[u] = lr * v[8 * c + u];
-                        uint4 hi, lo;
-                        split8(v + 8 * c, hi, lo);
-                        st_shared_v4(sb + kAW + off, hi);
-                        st_shared_v4(sb + kAW + 16384 + off, lo);
-                        *reinterpret_cast<uint4 *>(it + kIW + off) = hi;
-                        *reinterpret_cast<uint4 *>(it + kIW + 16384 + off) = lo;
-                        split8(wl, hi, lo);
-                        st_shared_v4(sb + kAWl + off, hi);
-                        st_shared_v4(sb + kAWl + 16384 + off, lo);
-                    }
-                }
-                tmem_ld32(tlane(tmem, warp, kTU + 64 * half + 32 * p), v);
-                tmem_wait_ld();
-                if (v64) {
-                    const float lr = cv.lam[r64];
+                for (int u = 0; u < 8; ++u) wl[u] = lr * v[8 * c + u];
+                uint4 hi, lo;
+                split8(v + 8 * c, hi, lo);
+                st_shared_v4(sb + kAW + off, hi);
+                st_shared_v4(sb + kAW + 16384 + off, lo);
+                *reinterpret_cast<uint4 *>(it + kIW + off) = hi;
+                *reinterpret_cast<uint4 *>(it + kIW + 16384 + off) = lo;
+                split8(wl, hi, lo);
+                st_shared_v4(sb + kAWl + off, hi);
+                st_shared_v4(sb + kAWl + 16384 + off, lo);
+            }
+            tmem_ld_h32(tlane(tmem, warp, kTU + 64 * half), v);
+            tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint32_t off = atom + sw128_offset(r64, 4 * p + c);
-                        float ul[8];
+            for (int c = 0; c < 4; ++c) {
+                const uint32_t off = atom + sw128_offset(rr, cb2 / 8 + c);
+                float ul[8];
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) ul[u] = lr * v[8 * c + u];
-                        uint4 hi, lo;
-                        split8(ul, hi, lo);
-                        *reinterpret_cast<uint4 *>(it + kIUl + off) = hi;
-                        *reinterpret_cast<uint4 *>(it + kIUl + 16384 + off) = lo;
-                    }
-                }
+                for (int u = 0; u < 8; ++u) ul[u] = lr * v[8 * c + u];
+                uint4 hi, lo;
+                split8(ul, hi, lo);
+                *reinterpret_cast<uint4 *>(it + kIUl + off) = hi;
+                *reinterpret_cast<uint4 *>(it + kIUl + 16384 + off) = lo;
             }
         }
         fence_proxy_async_shared();
@@ -521,26 +513,21 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
         // X = diag(gamma) Q - P W (rows < L)
         {
             const uint32_t atom = uint32_t(half) * 8192;
-#pragma unroll 1
-            for (int p = 0; p < 2; ++p) {
-                float v[32];
-                tmem_ld32(tlane(tmem, warp, kTPW + 64 * half + 32 * p), v);
-                tmem_wait_ld();
-                if (v64) {
-                    const float gr = r64 < L ? cv.gam[r64] : 0.f;
+            float v[32];
+            tmem_ld_h32(tlane(tmem, warp, kTPW + 64 * half), v);
+            tmem_wait_ld();
+            const float gr = rr < L ? cv.gam[rr] : 0.f;
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint32_t off = atom + sw128_offset(r64, 4 * p + c);
-                        float qv[8], x[8];
-                        unpack8(ld_shared_v4(sb + kAQ + off), qv);
+            for (int c = 0; c < 4; ++c) {
+                const uint32_t off = atom + sw128_offset(rr, cb2 / 8 + c);
+                float qv[8], x[8];
+                unpack8(ld_shared_v4(sb + kAQ + off), qv);
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) x[u] = r64 < L ? fmaf(gr, qv[u], -v[8 * c + u]) : 0.f;
-                        uint4 hi, lo;
-                        split8(x, hi, lo);
-                        *reinterpret_cast<uint4 *>(it + kIX + off) = hi;
-                        *reinterpret_cast<uint4 *>(it + kIX + 16384 + off) = lo;
-                    }
-                }
+                for (int u = 0; u < 8; ++u) x[u] = rr < L ? fmaf(gr, qv[u], -v[8 * c + u]) : 0.f;
+                uint4 hi, lo;
+                split8(x, hi, lo);
+                *reinterpret_cast<uint4 *>(it + kIX + off) = hi;
+                *reinterpret_cast<uint4 *>(it + kIX + 16384 + off) = lo;
             }
         }
         tc_fence_before();
