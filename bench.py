@@ -454,7 +454,15 @@ def prefill_record(args, w, host, device, world, rank, peaks, peak_src, e2e=True
                 "flops_per_launch": flops, "algorithmic_bytes_per_launch": prefill_bytes(w)}
     alu_peak = FP32_LANES_PER_SM * 2 * torch.cuda.get_device_properties(device).multi_processor_count * \
         (clocks.summary().get("sm_max_mhz") or 1965) * 1e6 / 1e12
-    if args.backward:
+    if args.backward and backward_tc_active(gdn, dev, w):
+        # the tensor-core form: factors, chains, gradients (useful flops, each product once)
+        bflops = backward_flops_per_vhead_token(w.d) * tokens * w.hv
+        achieved = bflops / (ms / 1e3) / 1e12
+        kname = "gdn_bwd_factor+gdn_bwd_chain+gdn_bwd_grad"
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": achieved / peaks["bf16_tflops"], "traffic": kernel_traffic(f"{kname}/{w.name}{suffix}"),
+                    "kernel": kname, "peak_source": f"{peak_src} bf16 dense (burst)", "flops_per_launch": bflops}
+    elif args.backward:
         # reverse mode of the token recurrence: 20 d^2 flops per (token, value head) (the forward
         # recomputed, 6 d^2, and the backward, 14 d^2); fp32 on CUDA cores
         bflops = 20 * w.d * w.d * tokens * w.hv
@@ -639,6 +647,13 @@ def gdn_tc_active(gdn, dev, w) -> bool:
     return major == 10 and w.dtype == "bf16" and w.d == 128 and w.chunk == 64 and tc_built(gdn)
 
 
+def backward_tc_active(gdn, dev, w) -> bool:
+    """The backward takes the tensor-core kernels (bf16, d = 128, sm_100)."""
+    import torch
+    major, _ = torch.cuda.get_device_capability()
+    return major == 10 and w.dtype == "bf16" and w.d == 128 and w.hv % w.hk == 0
+
+
 def tc_built(gdn) -> bool:
     src = open(os.path.join(ROOT, "linear_attention_sequence_sm_b200", "csrc", "gdn_chunk_tc.cu")).read()
     return "tcgen05.mma" in src
@@ -651,6 +666,18 @@ def useful_flops_per_vhead_token(group: int, d: int = 128, chunk: int = 64) -> i
 
 
 FP32_LANES_PER_SM = 128
+
+
+def backward_flops_per_vhead_token(d: int = 128, chunk: int = 64) -> int:
+    """Useful flops of the tensor-core backward per (token, value head), every
+    product counted once (not the two or three instructions its split
+    operands take): the factors (K K^T, Q K^T, W, U~, P W: C x C x d each;
+    (W diag(lambda))^T K: d x d x C), the two chains (S M', dS M'^T: d x d x d;
+    U~^T diag(lambda) K, dO^T X: d x d x C), and the gradients (five
+    C x d x d products, thirteen C x C x d, two C x C x C):
+    36 C^2 d + 16 C d^2 + 4 d^3 + 4 C^3 per chunk."""
+    C = chunk
+    return (36 * C * C * d + 16 * C * d * d + 4 * d ** 3 + 4 * C ** 3) // C
 
 
 def kda_flops_per_vhead_token(d: int = 128) -> int:

@@ -400,15 +400,24 @@ GDN_API gdn_status_t gdn_decode_commit(int32_t num_seqs, int32_t num_tokens, int
  *                      kernels' floor on g)
  *   d_initial_state    [N, Hv, d_v, d_k] fp32, or NULL
  * Inputs are those of gdn_chunk_forward (the plain path: no input-side
- * flags, GDN_ERR_UNSUPPORTED otherwise); d_o has the dtype of v.  fp32
- * arithmetic; for bf16 inputs the products run as tensor-core tiles with
- * each fp32 operand split into two bf16 parts and fp32 accumulation, for
- * fp32 inputs as CUDA-core tiles.  A forward pass keeps each 32-token chunk's start state and
- * its intra-chunk products in the workspace (about 3 d_v d_k fp32 values
- * per chunk and value head, plus the schedule; gdn_chunk_backward_
- * workspace_size), then the chunks are walked backward.  dq, dk, dg and dbeta are accumulated with atomic adds
- * (their summation order, and so their last bits, can vary between runs).
- * d_k, d_v <= 128. */
+ * flags, GDN_ERR_UNSUPPORTED otherwise, and neither GDN_FLAG_ONE_KERNEL nor
+ * GDN_FLAG_SPLIT); d_o has the dtype of v.  d_k, d_v <= 128.  Two forms:
+ *   - bf16 with d_k = d_v = 128 on sm_100 (unless GDN_FLAG_FORCE_SIMT):
+ *     tcgen05 tensor-core kernels over chunks of 64 tokens -- the chunk
+ *     factors of every (chunk, value head), the state and state-gradient
+ *     recurrences (one product per chunk each, every chunk's boundary state
+ *     kept), then the gradients of every (chunk, value head, half of d_v).
+ *     Workspace: the schedule plus 344,064 bytes per (chunk, value head)
+ *     (gdn_chunk_backward_workspace_size).
+ *   - otherwise one kernel per (sequence, value head, 32 rows of d_v) that
+ *     walks 32-token chunks forward, keeping each chunk's start state and
+ *     intra-chunk products (about 3 d_v d_k fp32 values per chunk and value
+ *     head), then backward.
+ * fp32 results: products of fp32 operands split each operand into a bf16
+ * value and a bf16 residual (tensor cores, fp32 accumulation) for bf16
+ * inputs, fp32 CUDA-core tiles for fp32 inputs.  dq, dk, dg and dbeta are
+ * accumulated with atomic adds (their summation order, and so their last
+ * bits, can vary between runs). */
 GDN_API gdn_status_t gdn_chunk_backward_workspace_size(const gdn_shape_t *shape, size_t *bytes);
 GDN_API gdn_status_t gdn_chunk_backward(const gdn_shape_t *shape,
                                 const void *q, const void *k, const void *v,

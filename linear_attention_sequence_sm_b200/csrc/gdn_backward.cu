@@ -588,7 +588,8 @@ chunk_backward_kernel(const PrefillArgs a, const void *dO_, const float *dSf, fl
             atomicAdd(dk + o, dK[r * ldk + x]);
         });
         if (tid < Lc) {
-            atomicAdd(dg + size_t(c0 + tid) * hv + h, vdG[tid]);
+            // d max(g, floor) / dg: zero below the floor
+            if (a.g[size_t(c0 + tid) * hv + h] >= kGFloor) atomicAdd(dg + size_t(c0 + tid) * hv + h, vdG[tid]);
             atomicAdd(dbeta + size_t(c0 + tid) * hv + h, vdB[tid]);
         }
         __syncthreads();

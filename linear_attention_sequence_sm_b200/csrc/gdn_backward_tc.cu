@@ -1166,8 +1166,9 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
                 const float y = __shfl_down_sync(0xffffffffu, run, m);
                 if (tid + m < 32) run += y;
             }
-            if (r0 < L) atomicAdd(dg + size_t(t0 + r0) * hv + h, run);
-            if (r1 < L) atomicAdd(dg + size_t(t0 + r1) * hv + h, run - a0);
+            // d max(g, floor) / dg: zero below the floor
+            if (r0 < L && a.g[size_t(t0 + r0) * hv + h] >= kGFloor) atomicAdd(dg + size_t(t0 + r0) * hv + h, run);
+            if (r1 < L && a.g[size_t(t0 + r1) * hv + h] >= kGFloor) atomicAdd(dg + size_t(t0 + r1) * hv + h, run - a0);
         }
         tc_fence_before();
         __syncthreads();  // tensor memory, shared memory and the vectors are reused by the next unit

@@ -97,3 +97,78 @@ def test_backward_small_dims_without_final_gradient():
     errs = worst_errors(inp, gg, ref)
     print(errs)
     assert max(errs.values()) <= GRAD_BAR["f32"], errs
+
+
+# ---- the tensor-core form (bf16, d = 128: factors, state chains, gradients over chunks of 64)
+
+def test_backward_tc_chunk_boundaries():
+    """Sequences on both sides of the 64-token chunks the tensor-core form
+    uses (one, two and three chunks, a full and a one-token last chunk)."""
+    lens = [63, 64, 65, 127, 128, 129, 1, 192]
+    inp = bwd_inputs(330, B=1, T=sum(lens), hk=2, hv=4, d=128, dtype="bf16", seq_lens=lens)
+    gg, ref = run_both(inp)
+    errs = worst_errors(inp, gg, ref)
+    print(errs)
+    assert max(errs.values()) <= GRAD_BAR["bf16"], errs
+
+
+def test_backward_tc_long_chains():
+    """2048 tokens: the state and state-gradient chains over 32 chunks."""
+    inp = bwd_inputs(331, B=1, T=2048, hk=1, hv=2, d=128, dtype="bf16")
+    gg, ref = run_both(inp)
+    errs = worst_errors(inp, gg, ref)
+    print(errs)
+    assert max(errs.values()) <= GRAD_BAR["bf16"], errs
+
+
+def test_backward_tc_strong_decay():
+    """Gates at and just above the kernels' floor (-20): the decays
+    gamma_r = e^(G_r) underflow to zero inside every chunk (the oracle reads
+    g unfloored, so gates below the floor are left to the next test)."""
+    inp = bwd_inputs(332, B=2, T=150, hk=1, hv=2, d=128, dtype="bf16")
+    g = inp["g"].clone()
+    g[:, ::3] = -19.5
+    g[:, 1::3] = -20.0
+    inp["g"] = g
+    gg, ref = run_both(inp)
+    errs = worst_errors(inp, gg, ref)
+    print(errs)
+    assert max(errs.values()) <= GRAD_BAR["bf16"], errs
+
+
+@pytest.mark.parametrize("force_simt", [False, True])
+def test_backward_dg_zero_below_floor(force_simt):
+    """The kernels read g as max(g, -20), whose derivative is zero below the
+    floor: dg is exactly zero there, and the other gradients match the same
+    inputs with those gates raised to the floor."""
+    from linear_attention_sequence_sm_b200 import gdn
+    inp = bwd_inputs(334, B=2, T=150, hk=1, hv=2, d=128, dtype="bf16")
+    g = inp["g"].clone()
+    g[:, 5::7] = -25.0
+    d = {k: (v.to(DEV) if v is not None else None) for k, v in inp.items()}
+    below = g.to(DEV) < -20
+    a = gdn.chunk_backward(d["q"], d["k"], d["v"], g.to(DEV), d["beta"], d["dO"], d_final_state=d["dSf"],
+                           initial_state=d["initial_state"], force_simt=force_simt)
+    b = gdn.chunk_backward(d["q"], d["k"], d["v"], g.clamp_min(-20).to(DEV), d["beta"], d["dO"],
+                           d_final_state=d["dSf"], initial_state=d["initial_state"], force_simt=force_simt)
+    assert torch.count_nonzero(a["dg"][below]) == 0
+    assert torch.allclose(a["dg"][~below], b["dg"][~below], rtol=1e-5, atol=1e-6)
+    for name in ("dq", "dk", "dv", "dbeta", "d_initial_state"):
+        assert torch.allclose(a[name], b[name], rtol=1e-5, atol=1e-6), name
+
+
+def test_backward_tc_matches_single_kernel():
+    """The tensor-core form and the single-kernel form (GDN_FLAG_FORCE_SIMT)
+    agree on a ragged batch, with and without an initial state."""
+    from linear_attention_sequence_sm_b200 import gdn
+    for s0 in (0.05, 0.0):
+        inp = bwd_inputs(333, B=3, T=200, hk=2, hv=4, d=128, dtype="bf16", s0_std=s0)
+        d = {k: (v.to(DEV) if v is not None else None) for k, v in inp.items()}
+        args = (d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"])
+        kw = dict(d_final_state=d["dSf"], initial_state=d["initial_state"])
+        a = gdn.chunk_backward(*args, **kw)
+        b = gdn.chunk_backward(*args, force_simt=True, **kw)
+        for name in ("dq", "dk", "dv", "dg", "dbeta", "d_initial_state"):
+            x, y = a[name].double(), b[name].double()
+            rel = ((x - y).norm() / y.norm().clamp_min(1e-30)).item()
+            assert rel <= 2 * GRAD_BAR["bf16"], (s0, name, rel)
