@@ -122,18 +122,26 @@ struct Opd {
     }
 };
 
+// Start-address step (16-byte units, the descriptor's low field) of k-step s.
+__device__ __forceinline__ uint64_t kstep(const Opd &X, int s) {
+    return X.mn ? uint64_t(s) * 128u : uint64_t((uint32_t(s >> 2) * X.atom + uint32_t(s & 3) * 32) >> 4);
+}
+
 // D (+)= A B over nk k-steps, split parts combined as hi hi + hi lo + lo hi
-// (or hi, lo against an exact operand).  One thread issues.
+// (or hi, lo against an exact operand).  One thread issues; each part's
+// descriptor is built once and stepped through K by its start address.
 __device__ __forceinline__ void product(uint32_t d, const Opd &A, const Opd &B, int M, int N, int nk, bool neg,
                                         bool accumulate) {
     const uint32_t id = idesc_bf16(M, N, A.mn, B.mn, neg);
-    const int pa = A.part ? 2 : 1, pb = B.part ? 2 : 1;
-    bool acc = accumulate;
-    for (int s = 0; s < nk; ++s) {
-        mma_bf16(d, A.desc(s, 0), B.desc(s, 0), id, acc);
-        acc = true;
-        if (pb == 2) mma_bf16(d, A.desc(s, 0), B.desc(s, 1), id, 1);
-        if (pa == 2) mma_bf16(d, A.desc(s, 1), B.desc(s, 0), id, 1);
+    const uint64_t a0 = A.desc(0, 0), a1 = A.desc(0, 1), b0 = B.desc(0, 0), b1 = B.desc(0, 1);
+    const bool pa = A.part != 0, pb = B.part != 0;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+        if (s >= nk) break;
+        const uint64_t da = kstep(A, s), db = kstep(B, s);
+        mma_bf16(d, a0 + da, b0 + db, id, (accumulate || s > 0) ? 1u : 0u);
+        if (pb) mma_bf16(d, a0 + da, b1 + db, id, 1);
+        if (pa) mma_bf16(d, a1 + da, b0 + db, id, 1);
     }
 }
 
@@ -768,13 +776,16 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
     const int wg = warp >> 2, rr = 16 * (warp & 3) + (lane & 15);
     const int cb = 16 * wg + 32 * (lane >> 4), cb2 = 32 * (lane >> 4);
 
-    // one group of products, then every thread waits for it
-    auto group_done = [&]() -> bool {
-        if (tid == 0) mma_commit(mbar);
+    // every thread waits for the group of products last committed
+    auto group_wait = [&]() -> bool {
         const bool ok = block_wait(mbar, mph);
         mph ^= 1u;
         tc_fence_after();
         return ok;
+    };
+    auto group_done = [&]() -> bool {
+        if (tid == 0) mma_commit(mbar);
+        return group_wait();
     };
     // the staged operands are visible to the tensor cores, the accumulator reads are done
     auto stage_done = [&]() {
@@ -896,8 +907,9 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
         // ---- E1.  Every 64-column accumulator is read by all eight warps, 16 columns a
         // thread (columns cb .. cb + 15 of row rr); 128-column ones 32 a thread (cb2 ..).
         float zl[16];  // lambda_j Z_ij, kept for dU^T
+        float pr[16];  // U_ij lambda_j Z_ij, for dlambda lambda
         {
-            float u[16], ul[16], pr[16];
+            float u[16], ul[16];
             tmem_ld_h16(tlane(tmem, warp, kTSA + 16 * wg), u);
             tmem_ld_h16(tlane(tmem, warp, kTSB + 16 * wg), zl);
             tmem_wait_ld();
@@ -909,7 +921,6 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
                 pr[q] = u[q] * zl[q];
                 ul[q] = lj * u[q];
             }
-            colsum16_add(pr, dll + cb, lane);
             stage16(sb + kDR1, rr, cb, u);
             stage16(sb + kDR1 + 16384, rr, cb, ul);
             // P = Q K^T (.) Gamma (lower, rows < L)
@@ -922,7 +933,22 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
                 u[q] = (j <= rr && rr < L) ? __expf(Gr - cv.G[j]) * u[q] : 0.f;
             }
             stage16(sb + kDgO, rr, cb, u);
-            // gamma_r dgamma_r (dO S_c part) = sum_x Y'_rx q_rx over this thread's 32 columns
+        }
+        stage_done();
+        // ---- G2: dO^T P, dP = dO U^T, dK = (U diag(lambda)) dS
+        if (tid == 0) {
+            tc_fence_after();
+            const Opd dOmn{sb + kDO, 0, 8192, true}, Pmn{sb + kDgO, 8192, 8192, true};
+            const Opd dO{sb + kDO, 0, 8192, false}, Utmn{sb + kDR1, 8192, 8192, true};
+            const Opd Ulmn{sb + kDR1 + 16384, 8192, 8192, true}, dSmn{sb + kDdS, 16384, 8192, true};
+            product(tmem + kTSB, dOmn, Pmn, 64, 64, 4, false, false);
+            product(tmem + kTSA, dO, Utmn, 64, 64, 4, false, false);
+            product(tmem + kTdK, Ulmn, dSmn, 64, 128, 4, false, false);
+            mma_commit(mbar);
+        }
+        // (while G2 runs) dlambda lambda column sums; gamma_r dgamma_r; <dS_{c+1}, S_c>
+        {
+            colsum16_add(pr, dll + cb, lane);
             float y[32], part = 0.f;
             tmem_ld_h32(tlane(tmem, warp, kTdQ + 64 * wg), y);
             tmem_wait_ld();
@@ -934,7 +960,6 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
                 for (int e = 0; e < 8; ++e) part = fmaf(y[8 * c + e], qv[e], part);
             }
             atomicAdd(dgg + rr, part);
-            // <dS_{c+1}, S_c> over the half
             float dot = 0.f;
             for (int e = tid; e < 64 * 16; e += kThr) {
                 const int r = e >> 4, a8 = (e >> 3) & 1, ch = e & 7;
@@ -949,30 +974,20 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
             for (int m = 16; m > 0; m >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, m);
             if (lane == 0) atomicAdd(scal, dot);
         }
-        stage_done();
-        // ---- G2: dO^T P, dP = dO U^T, dK = (U diag(lambda)) dS
-        if (tid == 0) {
-            tc_fence_after();
-            const Opd dOmn{sb + kDO, 0, 8192, true}, Pmn{sb + kDgO, 8192, 8192, true};
-            const Opd dO{sb + kDO, 0, 8192, false}, Utmn{sb + kDR1, 8192, 8192, true};
-            const Opd Ulmn{sb + kDR1 + 16384, 8192, 8192, true}, dSmn{sb + kDdS, 16384, 8192, true};
-            product(tmem + kTSB, dOmn, Pmn, 64, 64, 4, false, false);
-            product(tmem + kTSA, dO, Utmn, 64, 64, 4, false, false);
-            product(tmem + kTdK, Ulmn, dSmn, 64, 128, 4, false, false);
-        }
-        if (!group_done()) { aborted = true; break; }
+        tc_fence_before();
+        if (!group_wait()) { aborted = true; break; }
         // ---- E2: dU^T = lambda Z^T + dO^T P (columns < L); dP (.) Gamma and its dGamma sums
+        float e2[16], rsum = 0.f;
         {
-            float x[16], y[16];
+            float x[16];
             tmem_ld_h16(tlane(tmem, warp, kTSB + 16 * wg), x);
             tmem_wait_ld();
 #pragma unroll
             for (int q = 0; q < 16; ++q) x[q] = cb + q < L ? x[q] + zl[q] : 0.f;
             stage16(sb + kDdS, rr, cb, x);
-            tmem_ld_h16(tlane(tmem, warp, kTSA + 16 * wg), x);   // dP: rows r, columns j
-            tmem_ld_h16(tlane(tmem, warp, kTQK2 + 16 * wg), y);  // Q K^T
+            tmem_ld_h16(tlane(tmem, warp, kTSA + 16 * wg), x);    // dP: rows r, columns j
+            tmem_ld_h16(tlane(tmem, warp, kTQK2 + 16 * wg), e2);  // Q K^T
             tmem_wait_ld();
-            float rsum = 0.f;
             const float Gr = cv.G[rr];
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
@@ -980,12 +995,10 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
                 const bool ok = j <= rr && rr < L;
                 const float gm = ok ? __expf(Gr - cv.G[j]) : 0.f;
                 x[q] = ok ? x[q] * gm : 0.f;  // dP (.) Gamma
-                y[q] = x[q] * y[q];           // dGamma_rj Gamma_rj (the P part)
-                rsum += y[q];
+                e2[q] = x[q] * e2[q];         // dGamma_rj Gamma_rj (the P part)
+                rsum += e2[q];
             }
             stage16(sb + kDdS + 16384, rr, cb, x);
-            atomicAdd(rs + rr, rsum);
-            colsum16_add(y, cs + cb, lane);
         }
         stage_done();
         // ---- G3: dQ += (dP (.) Gamma) K, dK += (dP (.) Gamma)^T Q, dW = -dU S_c, dT2 = dU V^T, dV = T''^T dU
@@ -1001,23 +1014,17 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
             product(tmem + kTdW, dUtmn, S0mn, 64, 128, 4, true, false);
             product(tmem + kTSA, dUtmn, V, 64, 64, 4, false, false);
             product(tmem + kTSB, Tbmn, dUt, 64, 64, 4, false, false);
+            mma_commit(mbar);
         }
-        if (!group_done()) { aborted = true; break; }
+        atomicAdd(rs + rr, rsum);
+        colsum16_add(e2, cs + cb, lane);
+        if (!group_wait()) { aborted = true; break; }
         if (tid == 0 && has_next) {
             load_set(N, 0);
             pending = true;
         }
-        // ---- E3: dv (this half's columns, rows < L); dW as a split pair
+        // ---- E3: dW as a split pair; dv (this half's columns, rows < L) while G4 runs
         {
-            float x[16];
-            tmem_ld_h16(tlane(tmem, warp, kTSB + 16 * wg), x);
-            tmem_wait_ld();
-            if (rr < L) {
-                float *dst = dv + (size_t(t0 + rr) * hv + h) * 128 + i0 + cb;
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<float4 *>(dst + 4 * q) = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
-            }
             float y[32];
             tmem_ld_h32(tlane(tmem, warp, kTdW + 64 * wg), y);
             tmem_wait_ld();
@@ -1038,8 +1045,21 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
             const Opd Tbgmn{sb + kDTbg, 8192, 8192, true}, dWmn{sb + kDR1, 16384, 8192, true};
             product(tmem + kTdT1, dW, K, 64, 64, 8, false, false);
             product(tmem + kTdK, Tbgmn, dWmn, 64, 128, 4, false, true);
+            mma_commit(mbar);
         }
-        if (!group_done()) { aborted = true; break; }
+        {
+            float x[16];
+            tmem_ld_h16(tlane(tmem, warp, kTSB + 16 * wg), x);
+            tmem_wait_ld();
+            if (rr < L) {
+                float *dst = dv + (size_t(t0 + rr) * hv + h) * 128 + i0 + cb;
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<float4 *>(dst + 4 * q) = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+            }
+        }
+        tc_fence_before();
+        if (!group_wait()) { aborted = true; break; }
         if (tid == 0 && has_next) load_set(N, 1);
         // ---- E4: dT (lower, rows < L) as a split pair; T (.) dT1 and T (.) dT2 column sums
         {
@@ -1063,17 +1083,18 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
                 x1[q] = (ok && j <= rr) ? fmaf(cv.bg[j], x1[q], cv.beta[j] * x2[q]) : 0.f;
             }
             stage16(sb + kDgO, rr, cb, x1);
+            stage_done();
+            // ---- G5: M = dT T^T
+            if (tid == 0) {
+                tc_fence_after();
+                const Opd dT{sb + kDgO, 8192, 8192, false}, T{sb + kDT, 8192, 8192, false};
+                product(tmem + kTSA, dT, T, 64, 64, 4, false, false);
+                mma_commit(mbar);
+            }
             colsum16_add(p1, dbgv + cb, lane);
             colsum16_add(p2, dyv + cb, lane);
         }
-        stage_done();
-        // ---- G5: M = dT T^T
-        if (tid == 0) {
-            tc_fence_after();
-            const Opd dT{sb + kDgO, 8192, 8192, false}, T{sb + kDT, 8192, 8192, false};
-            product(tmem + kTSA, dT, T, 64, 64, 4, false, false);
-        }
-        if (!group_done()) { aborted = true; break; }
+        if (!group_wait()) { aborted = true; break; }
         {
             float x[16];
             tmem_ld_h16(tlane(tmem, warp, kTSA + 16 * wg), x);
@@ -1111,21 +1132,22 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
                 srs += e[q];
                 da[q] = d * bj * gm;  // dKK
             }
+            stage16(sb + kDgO, j, cb, da);  // dKK (M is consumed)
+            stage_done();
+            // ---- G7: dK += dKK K + dKK^T K
+            if (tid == 0) {
+                tc_fence_after();
+                const Opd dKK{sb + kDgO, 8192, 8192, false}, dKKmn{sb + kDgO, 8192, 8192, true};
+                const Opd Kmn{sb + kDK, 0, 8192, true};
+                product(tmem + kTdK, dKK, Kmn, 64, 128, 4, false, true);
+                product(tmem + kTdK, dKKmn, Kmn, 64, 128, 4, false, true);
+                mma_commit(mbar);
+            }
             atomicAdd(dab + j, sab);
             atomicAdd(rs + j, srs);
-            stage16(sb + kDgO, j, cb, da);  // dKK (M is consumed)
             colsum16_add(e, cs + cb, lane);
         }
-        stage_done();
-        // ---- G7: dK += dKK K + dKK^T K
-        if (tid == 0) {
-            tc_fence_after();
-            const Opd dKK{sb + kDgO, 8192, 8192, false}, dKKmn{sb + kDgO, 8192, 8192, true};
-            const Opd Kmn{sb + kDK, 0, 8192, true};
-            product(tmem + kTdK, dKK, Kmn, 64, 128, 4, false, true);
-            product(tmem + kTdK, dKKmn, Kmn, 64, 128, 4, false, true);
-        }
-        if (!group_done()) { aborted = true; break; }
+        if (!group_wait()) { aborted = true; break; }
         if (tid == 0 && has_next) load_set(N, 3);
         // ---- E7: dq, dk (this half's shares, rows < L); dG, dbeta, dg
 #pragma unroll 1
