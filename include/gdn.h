@@ -415,9 +415,9 @@ GDN_API gdn_status_t gdn_decode_commit(int32_t num_seqs, int32_t num_tokens, int
  *     head), then backward.
  * fp32 results: products of fp32 operands split each operand into a bf16
  * value and a bf16 residual (tensor cores, fp32 accumulation) for bf16
- * inputs, fp32 CUDA-core tiles for fp32 inputs.  dq, dk, dg and dbeta are
- * accumulated with atomic adds (their summation order, and so their last
- * bits, can vary between runs). */
+ * inputs, fp32 CUDA-core tiles for fp32 inputs.  dg and dbeta (both forms)
+ * and dq, dk (the single-kernel form) are accumulated with atomic adds
+ * (their summation order, and so their last bits, can vary between runs). */
 GDN_API gdn_status_t gdn_chunk_backward_workspace_size(const gdn_shape_t *shape, size_t *bytes);
 GDN_API gdn_status_t gdn_chunk_backward(const gdn_shape_t *shape,
                                 const void *q, const void *k, const void *v,

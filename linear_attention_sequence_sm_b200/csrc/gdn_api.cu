@@ -519,8 +519,9 @@ gdn_status_t gdn_chunk_backward(const gdn_shape_t *s, const void *q, const void 
     if (tokens > 0) {
         const size_t qk = size_t(tokens) * s->num_qk_heads * s->head_dim_k * sizeof(float);
         const size_t gb = size_t(tokens) * s->num_v_heads * sizeof(float);
-        if ((e = cudaMemsetAsync(dq, 0, qk, stream)) != cudaSuccess ||
-            (e = cudaMemsetAsync(dk, 0, qk, stream)) != cudaSuccess ||
+        // the tensor-core form writes dq and dk whole (one CTA per chunk and q/k head)
+        if ((!tc && ((e = cudaMemsetAsync(dq, 0, qk, stream)) != cudaSuccess ||
+                     (e = cudaMemsetAsync(dk, 0, qk, stream)) != cudaSuccess)) ||
             (e = cudaMemsetAsync(dg, 0, gb, stream)) != cudaSuccess ||
             (e = cudaMemsetAsync(dbeta, 0, gb, stream)) != cudaSuccess)
             return cuda_fail(e, "clearing the gradient accumulators");

@@ -29,8 +29,9 @@
 //      the decay and beta gradients as row and column sums of these
 //      products, and dg as reverse prefix sums of dG inside the chunk.
 // Every d_v row enters dS, dU and dv alone and the shared gradients (dq, dk,
-// dg, dbeta) linearly, so the two halves of d_v are independent units whose
-// shares of the shared gradients are added with atomics.
+// dg, dbeta) linearly, so the two halves of d_v are independent units.  A CTA
+// takes the units of one (chunk, q/k head) in turn and sums their dq and dk
+// shares in registers; dg and dbeta shares are added with atomics.
 //
 // Precision: the tensor cores take bf16 operands.  q, k, v and dO are exact
 // in bf16; every fp32 operand is split into a bf16 value and a bf16
@@ -331,26 +332,51 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
     const int rr = 16 * q4 + (lane & 15);
     const int cb = 16 * half + 32 * (lane >> 4), cb2 = 32 * (lane >> 4);
 
-    for (int64_t item = blockIdx.x; item < total; item += gridDim.x) {
-        const int gc = int(item / hv), h = int(item - int64_t(gc) * hv), hq = h / group;
+    // an item's (value head, q/k head, first token, tokens)
+    auto decode = [&](int64_t item, int &h, int &hq, int &t0, int &L) {
+        const int gc = int(item / hv);
+        h = int(item - int64_t(gc) * hv);
+        hq = h / group;
         const int n = chunk_sequence(a.sched.chunk_base, a.num_seqs, gc);
         const int c0 = gc - a.sched.chunk_base[n];
-        const int t0 = a.sched.start[n] + 64 * c0;
-        const int L = min(64, a.sched.len[n] - 64 * c0);
-        unsigned char *it = items + size_t(item) * kItemBytes;
+        t0 = a.sched.start[n] + 64 * c0;
+        L = min(64, a.sched.len[n] - 64 * c0);
+    };
+    // K and V of an item (once the previous item's products are done), then Q (after its last reader)
+    auto load_kv = [&](int h, int hq, int t0) {
+        mbar_expect_tx(lbar, 2 * 16384);
+        tma_load_3d(sb + kAK, &tk, 0, hq, t0, lbar);
+        tma_load_3d(sb + kAK + 8192, &tk, 64, hq, t0, lbar);
+        tma_load_3d(sb + kAV, &tv, 0, h, t0, lbar);
+        tma_load_3d(sb + kAV + 8192, &tv, 64, h, t0, lbar);
+    };
+    auto load_q = [&](int hq, int t0) {
+        mbar_arrive_expect_tx(lbar, 16384);
+        tma_load_3d(sb + kAQ, &tq, 0, hq, t0, lbar);
+        tma_load_3d(sb + kAQ + 8192, &tq, 64, hq, t0, lbar);
+    };
+    bool pending = false;  // a load phase is open (thread 0)
+    if (tid == 0 && total > int64_t(blockIdx.x)) {
+        int h, hq, t0, L;
+        decode(blockIdx.x, h, hq, t0, L);
+        load_kv(h, hq, t0);
+        load_q(hq, t0);
+        pending = true;
+    }
 
-        if (tid == 0) {
-            mbar_arrive_expect_tx(lbar, 3 * 16384);
-            tma_load_3d(sb + kAK, &tk, 0, hq, t0, lbar);
-            tma_load_3d(sb + kAK + 8192, &tk, 64, hq, t0, lbar);
-            tma_load_3d(sb + kAQ, &tq, 0, hq, t0, lbar);
-            tma_load_3d(sb + kAQ + 8192, &tq, 64, hq, t0, lbar);
-            tma_load_3d(sb + kAV, &tv, 0, h, t0, lbar);
-            tma_load_3d(sb + kAV + 8192, &tv, 64, h, t0, lbar);
-        }
+    for (int64_t item = blockIdx.x; item < total; item += gridDim.x) {
+        int h, hq, t0, L;
+        decode(item, h, hq, t0, L);
+        unsigned char *it = items + size_t(item) * kItemBytes;
+        const int64_t next = item + gridDim.x;
+        const bool has_next = next < total;
+        int nh = 0, nhq = 0, nt0 = 0, nL = 0;
+        if (tid == 0 && has_next) decode(next, nh, nhq, nt0, nL);
+
         chunk_vectors(a, t0, L, h, cv, tid);
         if (!block_wait(lbar, lph)) { aborted = true; break; }
         lph ^= 1u;
+        if (tid == 0) pending = false;
         // K K^T and Q K^T (exact bf16 operands)
         if (tid == 0) {
             tc_fence_after();
@@ -396,35 +422,27 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
         tc_fence_before();
         __syncthreads();
         invert_in_place<true>(Af, Yb, tid);
-        // T, T diag(beta), T diag(beta gamma): split pairs to the item, the last two to shared memory too
-        {
-            const int r = tid >> 2, cq = (tid & 3) * 16;
+        // T diag(beta), T diag(beta gamma) as split pairs to shared memory; W and U~ issued;
+        // then T, T diag(beta), T diag(beta gamma) to the item while they run
+        const int tr = tid >> 2, tcq = (tid & 3) * 16;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                float t[8], tb[8], tbg[8];
+        for (int c = 0; c < 2; ++c) {
+            float tb[8], tbg[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int j = cq + 8 * c + u;
-                    t[u] = Af[r * kLdA + j];
-                    tb[u] = t[u] * cv.beta[j];
-                    tbg[u] = t[u] * cv.bg[j];
-                }
-                const uint32_t off = sw128_offset(r, cq / 8 + c);
-                uint4 hi, lo;
-                split8(t, hi, lo);
-                *reinterpret_cast<uint4 *>(it + kIT + off) = hi;
-                *reinterpret_cast<uint4 *>(it + kIT + 8192 + off) = lo;
-                split8(tb, hi, lo);
-                *reinterpret_cast<uint4 *>(it + kITb + off) = hi;
-                *reinterpret_cast<uint4 *>(it + kITb + 8192 + off) = lo;
-                st_shared_v4(sb + kATb + off, hi);
-                st_shared_v4(sb + kATb + 8192 + off, lo);
-                split8(tbg, hi, lo);
-                *reinterpret_cast<uint4 *>(it + kITbg + off) = hi;
-                *reinterpret_cast<uint4 *>(it + kITbg + 8192 + off) = lo;
-                st_shared_v4(sb + kATbg + off, hi);
-                st_shared_v4(sb + kATbg + 8192 + off, lo);
+            for (int u = 0; u < 8; ++u) {
+                const int j = tcq + 8 * c + u;
+                const float t = Af[tr * kLdA + j];
+                tb[u] = t * cv.beta[j];
+                tbg[u] = t * cv.bg[j];
             }
+            const uint32_t off = sw128_offset(tr, tcq / 8 + c);
+            uint4 hi, lo;
+            split8(tb, hi, lo);
+            st_shared_v4(sb + kATb + off, hi);
+            st_shared_v4(sb + kATb + 8192 + off, lo);
+            split8(tbg, hi, lo);
+            st_shared_v4(sb + kATbg + off, hi);
+            st_shared_v4(sb + kATbg + 8192 + off, lo);
         }
         fence_proxy_async_shared();
         __syncthreads();
@@ -437,20 +455,35 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
             product(tmem + kTU, Tb, Vmn, 64, 128, 4, false, false);
             mma_commit(mbar);
         }
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const uint32_t off = sw128_offset(tr, tcq / 8 + c);
+            float t[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) t[u] = Af[tr * kLdA + tcq + 8 * c + u];
+            uint4 hi, lo;
+            split8(t, hi, lo);
+            *reinterpret_cast<uint4 *>(it + kIT + off) = hi;
+            *reinterpret_cast<uint4 *>(it + kIT + 8192 + off) = lo;
+            *reinterpret_cast<uint4 *>(it + kITb + off) = ld_shared_v4(sb + kATb + off);
+            *reinterpret_cast<uint4 *>(it + kITb + 8192 + off) = ld_shared_v4(sb + kATb + 8192 + off);
+            *reinterpret_cast<uint4 *>(it + kITbg + off) = ld_shared_v4(sb + kATbg + off);
+            *reinterpret_cast<uint4 *>(it + kITbg + 8192 + off) = ld_shared_v4(sb + kATbg + 8192 + off);
+        }
         if (!block_wait(mbar, mph)) { aborted = true; break; }
         mph ^= 1u;
         tc_fence_after();
-        // W: pair to shared memory and the item, W diag(lambda) to shared memory;
-        // U~ diag(lambda) to the item (columns 64 half + cb2 .. + 31: atom `half`)
+        // W and W diag(lambda) as split pairs to shared memory (columns 64 half + cb2 ..: atom
+        // `half`); the last products issued; then W and U~ diag(lambda) to the item while they run
+        const uint32_t watom = uint32_t(half) * 8192;
+        const float lr = cv.lam[rr];
         {
-            const uint32_t atom = uint32_t(half) * 8192;
-            const float lr = cv.lam[rr];
             float v[32];
             tmem_ld_h32(tlane(tmem, warp, kTW + 64 * half), v);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const uint32_t off = atom + sw128_offset(rr, cb2 / 8 + c);
+                const uint32_t off = watom + sw128_offset(rr, cb2 / 8 + c);
                 float wl[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) wl[u] = lr * v[8 * c + u];
@@ -458,24 +491,9 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
                 split8(v + 8 * c, hi, lo);
                 st_shared_v4(sb + kAW + off, hi);
                 st_shared_v4(sb + kAW + 16384 + off, lo);
-                *reinterpret_cast<uint4 *>(it + kIW + off) = hi;
-                *reinterpret_cast<uint4 *>(it + kIW + 16384 + off) = lo;
                 split8(wl, hi, lo);
                 st_shared_v4(sb + kAWl + off, hi);
                 st_shared_v4(sb + kAWl + 16384 + off, lo);
-            }
-            tmem_ld_h32(tlane(tmem, warp, kTU + 64 * half), v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const uint32_t off = atom + sw128_offset(rr, cb2 / 8 + c);
-                float ul[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) ul[u] = lr * v[8 * c + u];
-                uint4 hi, lo;
-                split8(ul, hi, lo);
-                *reinterpret_cast<uint4 *>(it + kIUl + off) = hi;
-                *reinterpret_cast<uint4 *>(it + kIUl + 16384 + off) = lo;
             }
         }
         fence_proxy_async_shared();
@@ -490,9 +508,36 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
             product(tmem + kTPW, P, Wmn, 64, 128, 4, false, false);
             mma_commit(mbar);
         }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const uint32_t off = watom + sw128_offset(rr, cb2 / 8 + c);
+            *reinterpret_cast<uint4 *>(it + kIW + off) = ld_shared_v4(sb + kAW + off);
+            *reinterpret_cast<uint4 *>(it + kIW + 16384 + off) = ld_shared_v4(sb + kAW + 16384 + off);
+        }
+        {
+            float v[32];
+            tmem_ld_h32(tlane(tmem, warp, kTU + 64 * half), v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint32_t off = watom + sw128_offset(rr, cb2 / 8 + c);
+                float ul[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) ul[u] = lr * v[8 * c + u];
+                uint4 hi, lo;
+                split8(ul, hi, lo);
+                *reinterpret_cast<uint4 *>(it + kIUl + off) = hi;
+                *reinterpret_cast<uint4 *>(it + kIUl + 16384 + off) = lo;
+            }
+        }
+        tc_fence_before();
         if (!block_wait(mbar, mph)) { aborted = true; break; }
         mph ^= 1u;
         tc_fence_after();
+        if (tid == 0 && has_next) {  // K and V are free (their last products are done)
+            load_kv(nh, nhq, nt0);
+            pending = true;
+        }
         // M' = gamma_L I - (W diag(lambda))^T K: row y = 32 (warp % 4) + lane, 64 columns
         {
             const int y = 32 * q4 + lane;
@@ -538,12 +583,18 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
                 *reinterpret_cast<uint4 *>(it + kIX + 16384 + off) = lo;
             }
         }
+        fence_proxy_async_shared();
         tc_fence_before();
         __syncthreads();  // tensor memory and shared memory are reused by the next item
+        if (tid == 0 && has_next) load_q(nhq, nt0);  // Q's last reader (X) is done
     }
     if (aborted && tid == 0 && total > 0) {
         mma_commit(mbar);
         (void)mbar_wait(mbar, mph);
+        if (pending) {  // loads in flight into this CTA's shared memory: let them land
+            mbar_arrive(lbar);
+            (void)mbar_wait(lbar, lph);
+        }
         record_abort(hdr, -6);
     }
     tc_fence_before();
@@ -768,7 +819,12 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
     grid_dep_wait();
     bool aborted = hdr->status != GDN_OK;
     const int hv = a.hv, hk = a.hk, group = hv / hk;
-    const int64_t total = aborted ? 0 : int64_t(hdr->total_chunks) * hv * 2;
+    // Units come in groups of one (chunk, q/k head): its value heads' two halves of d_v in turn,
+    // so that dq and dk add up in registers and are written once, and K and Q (per group) and
+    // T, T diag(beta), T diag(beta gamma) (per value head) are loaded once.
+    const int upg = 2 * group;  // units per group
+    const int64_t groups = aborted ? 0 : int64_t(hdr->total_chunks) * hk;
+    const int64_t my_units = groups > int64_t(blockIdx.x) ? ((groups - 1 - blockIdx.x) / gridDim.x + 1) * upg : 0;
     uint32_t lph = 0, mph = 0;
     // accumulator reads: row rr of an M = 64 accumulator; of a 64-column one the 16
     // columns cb .. cb + 15, of a 128-column one the 32 columns cb2 .. cb2 + 31
@@ -805,19 +861,21 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
         }
     };
 
-    // a unit's coordinates
+    // the k-th unit of this CTA
     struct Unit {
-        int sh, i0, h, hq, t0, L;
+        int sh, i0, h, hq, t0, L, pos;
         const unsigned char *it, *cs0, *cds;
     };
-    auto decode = [&](int64_t unit) {
+    auto decode = [&](int64_t k) {
         Unit U;
-        const int64_t item = unit >> 1;
-        U.sh = int(unit & 1);
+        const int64_t gi = blockIdx.x + (k / upg) * gridDim.x;
+        U.pos = int(k % upg);
+        U.sh = U.pos & 1;
         U.i0 = 64 * U.sh;
-        const int gc = int(item / hv);
-        U.h = int(item - int64_t(gc) * hv);
-        U.hq = U.h / group;
+        const int gc = int(gi / hk);
+        U.hq = int(gi - int64_t(gc) * hk);
+        U.h = U.hq * group + (U.pos >> 1);
+        const int64_t item = int64_t(gc) * hv + U.h;
         const int n = chunk_sequence(a.sched.chunk_base, a.num_seqs, gc);
         const int c0 = gc - a.sched.chunk_base[n];
         U.t0 = a.sched.start[n] + 64 * c0;
@@ -827,47 +885,59 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
         U.cds = ck_ds + size_t(item) * kCkBytes;
         return U;
     };
-    // the unit's inputs, in the four sets the prefetch uses (thread 0; set 3 arrives)
+    // the unit's inputs, in the four sets the prefetch uses (thread 0; set 3 arrives).  Q and
+    // K only for a group's first unit, the three T tiles only for a value head's first half.
     auto load_set = [&](const Unit &U, int set) {
+        const bool new_group = U.pos == 0, new_head = U.sh == 0;
         if (set == 0) {
-            mbar_expect_tx(lbar, 2 * 32768 + 16384 + 2 * 8192 + 16384);
+            mbar_expect_tx(lbar, 2 * 32768 + 2 * 8192 + (new_group ? 16384 : 0) + (new_head ? 16384 : 0));
             for (int q = 0; q < 4; ++q) {  // rows i0 .. i0 + 63 of each atom of the two checkpoint pairs
                 const uint32_t src = uint32_t(q) * 16384 + uint32_t(U.sh) * 8192, dst = uint32_t(q) * 8192;
                 bulk_load(sb + kDS0 + dst, U.cs0 + src, 8192, lbar);
                 bulk_load(sb + kDdS + dst, U.cds + src, 8192, lbar);
             }
-            tma_load_3d(sb + kDQ, &tq, 0, U.hq, U.t0, lbar);
-            tma_load_3d(sb + kDQ + 8192, &tq, 64, U.hq, U.t0, lbar);
+            if (new_group) {
+                tma_load_3d(sb + kDQ, &tq, 0, U.hq, U.t0, lbar);
+                tma_load_3d(sb + kDQ + 8192, &tq, 64, U.hq, U.t0, lbar);
+            }
             tma_load_3d(sb + kDV, &tv, U.i0, U.h, U.t0, lbar);
             tma_load_3d(sb + kDO, &tdo, U.i0, U.h, U.t0, lbar);
-            bulk_load(sb + kDTb, U.it + kITb, 16384, lbar);
+            if (new_head) bulk_load(sb + kDTb, U.it + kITb, 16384, lbar);
         } else if (set == 1) {
-            mbar_expect_tx(lbar, 32768 + 16384);
+            mbar_expect_tx(lbar, 32768 + (new_head ? 16384 : 0));
             bulk_load(sb + kDR1, U.it + kIW, 32768, lbar);
-            bulk_load(sb + kDTbg, U.it + kITbg, 16384, lbar);
+            if (new_head) bulk_load(sb + kDTbg, U.it + kITbg, 16384, lbar);
         } else if (set == 2) {
-            mbar_expect_tx(lbar, 16384);
-            bulk_load(sb + kDT, U.it + kIT, 16384, lbar);
+            if (new_head) {
+                mbar_expect_tx(lbar, 16384);
+                bulk_load(sb + kDT, U.it + kIT, 16384, lbar);
+            }
         } else {
-            mbar_arrive_expect_tx(lbar, 16384);
-            tma_load_3d(sb + kDK, &tk, 0, U.hq, U.t0, lbar);
-            tma_load_3d(sb + kDK + 8192, &tk, 64, U.hq, U.t0, lbar);
+            mbar_arrive_expect_tx(lbar, new_group ? 16384 : 0);
+            if (new_group) {
+                tma_load_3d(sb + kDK, &tk, 0, U.hq, U.t0, lbar);
+                tma_load_3d(sb + kDK + 8192, &tk, 64, U.hq, U.t0, lbar);
+            }
         }
     };
     bool pending = false;  // a load phase is open (thread 0)
-    if (tid == 0 && total > int64_t(blockIdx.x)) {
-        const Unit U = decode(blockIdx.x);
+    if (tid == 0 && my_units > 0) {
+        const Unit U = decode(0);
         for (int set = 0; set < 4; ++set) load_set(U, set);
         pending = true;
     }
+    float accq[32], acck[32];  // this thread's 32 columns of dq and dk, summed over the group
 
-    for (int64_t unit = blockIdx.x; unit < total; unit += gridDim.x) {
-        const Unit U = decode(unit);
+    for (int64_t k = 0; k < my_units; ++k) {
+        const Unit U = decode(k);
         const int i0 = U.i0, h = U.h, hq = U.hq, t0 = U.t0, L = U.L;
-        const int64_t next = unit + gridDim.x;
-        const bool has_next = next < total;
+        const bool has_next = k + 1 < my_units;
         Unit N{};
-        if (tid == 0 && has_next) N = decode(next);
+        if (tid == 0 && has_next) N = decode(k + 1);
+        if (U.pos == 0) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) accq[q] = acck[q] = 0.f;
+        }
         if (tid < 64)
             for (int v = kVll; v < kVNum; ++v) vec[64 * v + tid] = 0.f;
         if (tid < 2) scal[tid] = 0.f;
@@ -1048,6 +1118,13 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
             mma_commit(mbar);
         }
         {
+            float y[32];
+            tmem_ld_h32(tlane(tmem, warp, kTdQ + 64 * wg), y);  // dQ: complete after G3
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 32; ++q) accq[q] += y[q];
+        }
+        {
             float x[16];
             tmem_ld_h16(tlane(tmem, warp, kTSB + 16 * wg), x);
             tmem_wait_ld();
@@ -1149,19 +1226,22 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
         }
         if (!group_wait()) { aborted = true; break; }
         if (tid == 0 && has_next) load_set(N, 3);
-        // ---- E7: dq, dk (this half's shares, rows < L); dG, dbeta, dg
-#pragma unroll 1
-        for (int which = 0; which < 2; ++which) {
-            float *base = which == 0 ? dq : dk;
+        // ---- E7: dK into the register sums; after the group's last unit dq and dk stored (rows < L)
+        {
             float x[32];
-            tmem_ld_h32(tlane(tmem, warp, (which == 0 ? kTdQ : kTdK) + 64 * wg), x);
+            tmem_ld_h32(tlane(tmem, warp, kTdK + 64 * wg), x);
             tmem_wait_ld();
-            if (rr < L) {
-                float *dst = base + (size_t(t0 + rr) * hk + hq) * 128 + 64 * wg + 32 * (lane >> 4);
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    atomicAdd(reinterpret_cast<float4 *>(dst + 4 * q),
-                              make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]));
+            for (int q = 0; q < 32; ++q) acck[q] += x[q];
+            if (U.pos == upg - 1 && rr < L) {
+                const size_t o = (size_t(t0 + rr) * hk + hq) * 128 + 64 * wg + 32 * (lane >> 4);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    *reinterpret_cast<float4 *>(dq + o + 4 * q) =
+                        make_float4(accq[4 * q], accq[4 * q + 1], accq[4 * q + 2], accq[4 * q + 3]);
+                    *reinterpret_cast<float4 *>(dk + o + 4 * q) =
+                        make_float4(acck[4 * q], acck[4 * q + 1], acck[4 * q + 2], acck[4 * q + 3]);
+                }
             }
         }
         if (tid < 64) {
@@ -1195,7 +1275,7 @@ bwd_grad_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, con
         tc_fence_before();
         __syncthreads();  // tensor memory, shared memory and the vectors are reused by the next unit
     }
-    if (aborted && tid == 0 && total > 0) {
+    if (aborted && tid == 0 && my_units > 0) {
         mma_commit(mbar);
         (void)mbar_wait(mbar, mph);
         if (pending) {  // loads in flight into this CTA's shared memory: let them land
