@@ -172,3 +172,38 @@ def test_backward_tc_matches_single_kernel():
             x, y = a[name].double(), b[name].double()
             rel = ((x - y).norm() / y.norm().clamp_min(1e-30)).item()
             assert rel <= 2 * GRAD_BAR["bf16"], (s0, name, rel)
+
+
+@pytest.mark.parametrize("case", ["bench_4x4096", "long_65536"])
+def test_backward_tc_full_size(case):
+    """Full size: the tensor-core form against the single-kernel form (itself
+    checked against the oracle above) on the 4 x 4096 bench workload (16 q/k,
+    32 value heads: every item and unit) and on one 65,536-token sequence
+    (chains of 1024 chunks), per (sequence, head) slice of every gradient."""
+    from linear_attention_sequence_sm_b200 import gdn
+    if case == "bench_4x4096":
+        w = I.custom("bwd_full", batch=4, seq_len=4096, hk=16, hv=32, d=128, chunk=64, dtype="bf16", seed=41,
+                     s0_std=0.05)
+    else:
+        w = I.custom("bwd_long", batch=1, seq_len=65536, hk=2, hv=4, d=128, chunk=64, dtype="bf16", seed=42,
+                     s0_std=0.05)
+    inp = I.make_prefill_inputs(w)
+    d = {k: (v.to(DEV) if v is not None else None) for k, v in inp.items()}
+    dO = torch.from_numpy(I.normal(w.seed, "bwd_do", tuple(inp["v"].shape))).to(torch.bfloat16).to(DEV)
+    dSf = torch.from_numpy(I.normal(w.seed, "bwd_dsf", (w.num_seqs, w.hv, 128, 128), std=0.1)).float().to(DEV)
+    args = (d["q"], d["k"], d["v"], d["g"], d["beta"], dO)
+    a = gdn.chunk_backward(*args, d_final_state=dSf, initial_state=d["initial_state"])
+    b = gdn.chunk_backward(*args, d_final_state=dSf, initial_state=d["initial_state"], force_simt=True)
+    torch.cuda.synchronize()
+    worst = {}
+    for name in ("dq", "dk", "dv", "dg", "dbeta"):
+        x, y = a[name].double(), b[name].double()
+        heads = x.shape[2]
+        x = x.reshape(w.batch, w.seq_len, heads, -1)
+        y = y.reshape(w.batch, w.seq_len, heads, -1)
+        diff = (x - y).norm(dim=(1, 3)) / y.norm(dim=(1, 3)).clamp_min(1e-30)  # per (sequence, head)
+        worst[name] = diff.max().item()
+    x, y = a["d_initial_state"].double(), b["d_initial_state"].double()
+    worst["dS0"] = ((x - y).norm(dim=(2, 3)) / y.norm(dim=(2, 3)).clamp_min(1e-30)).max().item()
+    print(case, worst)
+    assert max(worst.values()) <= 2 * GRAD_BAR["bf16"], worst
