@@ -169,6 +169,12 @@ __device__ __forceinline__ void colsum_add(float (&v)[32], bool valid, float *ds
     }
 }
 
+// Shared -> global bulk copy (one thread; completion through the bulk group).
+__device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+                 : "memory");
+}
+
 // Adds to the transaction count of the current phase without arriving.
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
@@ -288,7 +294,11 @@ constexpr uint32_t kAAf = 163840;                        // A, inverted into T: 
 constexpr uint32_t kAY = kAAf + 64 * kLdA * 4;           // 32 x kLdY fp32
 constexpr uint32_t kAVec = kAY + 32 * kLdY * 4;          // G, gamma, lambda, beta, beta gamma
 constexpr uint32_t kABar = kAVec + 5 * 64 * 4;           // load and product mbarriers, tensor-memory slot
-constexpr uint32_t kASmem = kABar + 64 + 1024;
+constexpr uint32_t kAT = (kABar + 64 + 1023) & ~1023u;   // T pair, staged for its copy to the item
+constexpr uint32_t kASmem = kAT + 16384 + 1024;
+// The item's tiles leave through shared memory as bulk copies: T, T diag(beta), T diag(beta gamma)
+// from their slots; W from kAW and U~ diag(lambda) from kATbg (its 32 KB span kATbg and kATb);
+// M' from kAW (with kAWl) and X from kATbg once the products that read those slots are done.
 static_assert(kASmem <= 232448, "factor kernel shared memory");
 // tensor memory (512 columns): K K^T 0, Q K^T 64 (M = 64); then W 128, U~ 256
 // (M = 64, 128 columns); then (W diag(lambda))^T K 384 (M = 128) and P W 0.
@@ -422,21 +432,24 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
         tc_fence_before();
         __syncthreads();
         invert_in_place<true>(Af, Yb, tid);
-        // T diag(beta), T diag(beta gamma) as split pairs to shared memory; W and U~ issued;
-        // then T, T diag(beta), T diag(beta gamma) to the item while they run
+        // T, T diag(beta), T diag(beta gamma) as split pairs to shared memory; copied to the item
+        // while W and U~ run
         const int tr = tid >> 2, tcq = (tid & 3) * 16;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-            float tb[8], tbg[8];
+            float t[8], tb[8], tbg[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int j = tcq + 8 * c + u;
-                const float t = Af[tr * kLdA + j];
-                tb[u] = t * cv.beta[j];
-                tbg[u] = t * cv.bg[j];
+                t[u] = Af[tr * kLdA + j];
+                tb[u] = t[u] * cv.beta[j];
+                tbg[u] = t[u] * cv.bg[j];
             }
             const uint32_t off = sw128_offset(tr, tcq / 8 + c);
             uint4 hi, lo;
+            split8(t, hi, lo);
+            st_shared_v4(sb + kAT + off, hi);
+            st_shared_v4(sb + kAT + 8192 + off, lo);
             split8(tb, hi, lo);
             st_shared_v4(sb + kATb + off, hi);
             st_shared_v4(sb + kATb + 8192 + off, lo);
@@ -448,6 +461,10 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
         __syncthreads();
         // W = (T diag(beta gamma)) K and U~ = (T diag(beta)) V   (M = 64, N = 128, K = 64)
         if (tid == 0) {
+            bulk_store(it + kIT, sb + kAT, 16384);
+            bulk_store(it + kITb, sb + kATb, 16384);
+            bulk_store(it + kITbg, sb + kATbg, 16384);
+            bulk_commit();
             tc_fence_after();
             const Opd Tbg{sb + kATbg, 8192, 8192, false}, Tb{sb + kATb, 8192, 8192, false};
             const Opd Kmn{sb + kAK, 0, 8192, true}, Vmn{sb + kAV, 0, 8192, true};
@@ -455,29 +472,16 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
             product(tmem + kTU, Tb, Vmn, 64, 128, 4, false, false);
             mma_commit(mbar);
         }
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const uint32_t off = sw128_offset(tr, tcq / 8 + c);
-            float t[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) t[u] = Af[tr * kLdA + tcq + 8 * c + u];
-            uint4 hi, lo;
-            split8(t, hi, lo);
-            *reinterpret_cast<uint4 *>(it + kIT + off) = hi;
-            *reinterpret_cast<uint4 *>(it + kIT + 8192 + off) = lo;
-            *reinterpret_cast<uint4 *>(it + kITb + off) = ld_shared_v4(sb + kATb + off);
-            *reinterpret_cast<uint4 *>(it + kITb + 8192 + off) = ld_shared_v4(sb + kATb + 8192 + off);
-            *reinterpret_cast<uint4 *>(it + kITbg + off) = ld_shared_v4(sb + kATbg + off);
-            *reinterpret_cast<uint4 *>(it + kITbg + 8192 + off) = ld_shared_v4(sb + kATbg + 8192 + off);
-        }
         if (!block_wait(mbar, mph)) { aborted = true; break; }
         mph ^= 1u;
         tc_fence_after();
-        // W and W diag(lambda) as split pairs to shared memory (columns 64 half + cb2 ..: atom
-        // `half`); the last products issued; then W and U~ diag(lambda) to the item while they run
-        const uint32_t watom = uint32_t(half) * 8192;
-        const float lr = cv.lam[rr];
+        // W, W diag(lambda) and U~ diag(lambda) as split pairs to shared memory (columns 64 half +
+        // cb2 ..: atom `half`); W and U~ diag(lambda) copied to the item while the last products run
+        if (tid == 0) bulk_wait_read();  // the T copies have read kATb, kATbg
+        __syncthreads();
         {
+            const uint32_t watom = uint32_t(half) * 8192;
+            const float lr = cv.lam[rr];
             float v[32];
             tmem_ld_h32(tlane(tmem, warp, kTW + 64 * half), v);
             tmem_wait_ld();
@@ -495,27 +499,6 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
                 st_shared_v4(sb + kAWl + off, hi);
                 st_shared_v4(sb + kAWl + 16384 + off, lo);
             }
-        }
-        fence_proxy_async_shared();
-        tc_fence_before();
-        __syncthreads();
-        // (W diag(lambda))^T K (M = 128, N = 128, K = 64) and P W (M = 64, N = 128, K = 64)
-        if (tid == 0) {
-            tc_fence_after();
-            const Opd Wl{sb + kAWl, 16384, 8192, true}, Kmn{sb + kAK, 0, 8192, true};
-            const Opd P{sb + kAP, 8192, 8192, false}, Wmn{sb + kAW, 16384, 8192, true};
-            product(tmem + kTM, Wl, Kmn, 128, 128, 4, false, false);
-            product(tmem + kTPW, P, Wmn, 64, 128, 4, false, false);
-            mma_commit(mbar);
-        }
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const uint32_t off = watom + sw128_offset(rr, cb2 / 8 + c);
-            *reinterpret_cast<uint4 *>(it + kIW + off) = ld_shared_v4(sb + kAW + off);
-            *reinterpret_cast<uint4 *>(it + kIW + 16384 + off) = ld_shared_v4(sb + kAW + 16384 + off);
-        }
-        {
-            float v[32];
             tmem_ld_h32(tlane(tmem, warp, kTU + 64 * half), v);
             tmem_wait_ld();
 #pragma unroll
@@ -526,11 +509,25 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
                 for (int u = 0; u < 8; ++u) ul[u] = lr * v[8 * c + u];
                 uint4 hi, lo;
                 split8(ul, hi, lo);
-                *reinterpret_cast<uint4 *>(it + kIUl + off) = hi;
-                *reinterpret_cast<uint4 *>(it + kIUl + 16384 + off) = lo;
+                st_shared_v4(sb + kATbg + off, hi);
+                st_shared_v4(sb + kATbg + 16384 + off, lo);
             }
         }
+        fence_proxy_async_shared();
         tc_fence_before();
+        __syncthreads();
+        // (W diag(lambda))^T K (M = 128, N = 128, K = 64) and P W (M = 64, N = 128, K = 64)
+        if (tid == 0) {
+            bulk_store(it + kIW, sb + kAW, 32768);
+            bulk_store(it + kIUl, sb + kATbg, 32768);
+            bulk_commit();
+            tc_fence_after();
+            const Opd Wl{sb + kAWl, 16384, 8192, true}, Kmn{sb + kAK, 0, 8192, true};
+            const Opd P{sb + kAP, 8192, 8192, false}, Wmn{sb + kAW, 16384, 8192, true};
+            product(tmem + kTM, Wl, Kmn, 128, 128, 4, false, false);
+            product(tmem + kTPW, P, Wmn, 64, 128, 4, false, false);
+            mma_commit(mbar);
+        }
         if (!block_wait(mbar, mph)) { aborted = true; break; }
         mph ^= 1u;
         tc_fence_after();
@@ -538,7 +535,10 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
             load_kv(nh, nhq, nt0);
             pending = true;
         }
-        // M' = gamma_L I - (W diag(lambda))^T K: row y = 32 (warp % 4) + lane, 64 columns
+        if (tid == 0) bulk_wait_read();  // the W and U~ diag(lambda) copies have read kAW, kATbg
+        __syncthreads();
+        // M' = gamma_L I - (W diag(lambda))^T K: row y = 32 (warp % 4) + lane, 64 columns;
+        // as a pair in kAW .. (value 32 KB, then residual 32 KB over kAWl)
         {
             const int y = 32 * q4 + lane;
             const float gl = cv.gam[63];
@@ -558,12 +558,12 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
                     uint4 hi, lo;
                     split8(x, hi, lo);
                     const uint32_t off = uint32_t(half) * 16384 + sw128_offset(y, 4 * p + c);
-                    *reinterpret_cast<uint4 *>(it + kIMp + off) = hi;
-                    *reinterpret_cast<uint4 *>(it + kIMp + 32768 + off) = lo;
+                    st_shared_v4(sb + kAW + off, hi);
+                    st_shared_v4(sb + kAW + 32768 + off, lo);
                 }
             }
         }
-        // X = diag(gamma) Q - P W (rows < L)
+        // X = diag(gamma) Q - P W (rows < L), as a pair in kATbg ..
         {
             const uint32_t atom = uint32_t(half) * 8192;
             float v[32];
@@ -579,9 +579,17 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
                 for (int u = 0; u < 8; ++u) x[u] = rr < L ? fmaf(gr, qv[u], -v[8 * c + u]) : 0.f;
                 uint4 hi, lo;
                 split8(x, hi, lo);
-                *reinterpret_cast<uint4 *>(it + kIX + off) = hi;
-                *reinterpret_cast<uint4 *>(it + kIX + 16384 + off) = lo;
+                st_shared_v4(sb + kATbg + off, hi);
+                st_shared_v4(sb + kATbg + 16384 + off, lo);
             }
+        }
+        fence_proxy_async_shared();
+        __syncthreads();
+        if (tid == 0) {
+            bulk_store(it + kIMp, sb + kAW, 65536);
+            bulk_store(it + kIX, sb + kATbg, 32768);
+            bulk_commit();
+            bulk_wait_read();  // the next item reuses these slots
         }
         fence_proxy_async_shared();
         tc_fence_before();
@@ -597,6 +605,7 @@ bwd_factor_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, c
         }
         record_abort(hdr, -6);
     }
+    if (tid == 0) bulk_wait_all();  // the item copies have landed
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 512);
