@@ -271,6 +271,33 @@ def test_decode_multi_and_commit_argument_checks(gdn):
     assert c(0, 3, 4, 128, 128, None, None, None, None, None) == gdn.GDN_OK
 
 
+def test_backward_workspace_size_follows_the_path(gdn):
+    """bf16 with d_k = d_v = 128 sizes the tensor-core backward: the schedule
+    and chunk_base, then 212,992 + 2 x 65,536 bytes per (chunk, value head)
+    slot; GDN_FLAG_FORCE_SIMT, fp32 or other head sizes size the single-kernel
+    form; the forward-path flags are refused by the backward."""
+    n = ctypes.c_size_t(0)
+    def size(**kw):
+        assert gdn.LIB.gdn_chunk_backward_workspace_size(ctypes.byref(_shape(gdn, **kw)), ctypes.byref(n)) == gdn.GDN_OK
+        return n.value
+    # 2 sequences of 200 tokens, 4 value heads: at most (400 + 63 * 2) // 64 = 8 chunks; the tables
+    # (header, order, start, len: 1024 bytes; chunk_base) end at 2048 after rounding to 1 KiB
+    tc = size(batch=2, seq_len=200, num_seqs=2)
+    assert tc == 2048 + 8 * 4 * (212992 + 2 * 65536)
+    simt = size(batch=2, seq_len=200, num_seqs=2, flags=gdn.GDN_FLAG_FORCE_SIMT)
+    assert simt != tc
+    assert size(batch=2, seq_len=200, num_seqs=2, dtype=gdn.GDN_DTYPE_F32) == simt
+    assert size(batch=2, seq_len=200, num_seqs=2, head_dim_k=64, head_dim_v=64) not in (tc, simt)
+    # the tensor-core size grows with the chunks, one slot per (chunk, value head)
+    assert size(batch=2, seq_len=264, num_seqs=2) - tc == 2 * 4 * (212992 + 2 * 65536)
+    vp = ctypes.c_void_p
+    for flag in (gdn.GDN_FLAG_ONE_KERNEL, gdn.GDN_FLAG_SPLIT):
+        s = _shape(gdn, flags=flag)
+        st = gdn.LIB.gdn_chunk_backward(ctypes.byref(s), *(vp(FAKE) for _ in range(5)), None, None, vp(FAKE), None,
+                                        *(vp(FAKE) for _ in range(5)), None, vp(FAKE), ctypes.c_size_t(1 << 40), None)
+        assert st == gdn.GDN_ERR_UNSUPPORTED
+
+
 def test_backward_and_kda_argument_checks(gdn):
     """Refused before any device work: input-side flags on the backward,
     NULL gradient outputs, a short workspace, misalignment; KDA with d_k > 128."""
