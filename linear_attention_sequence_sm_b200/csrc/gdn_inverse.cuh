@@ -1,7 +1,8 @@
 // gdn_inverse.cuh -- T = (I + A)^-1 for the 64 x 64 unit-lower-triangular
 // factor of a chunk's WY representation ("Gated Attention Architectures",
 // section 2: the UT transform), shared by the kernels that invert chunk
-// factors outside the state loop (gdn_chunk_inv.cu, gdn_kda_tc.cu).
+// factors outside the state loop (gdn_chunk_inv.cu, gdn_kda_tc.cu,
+// gdn_backward_tc.cu).
 //
 // Divide and conquer on the block structure
 //   [[X, 0], [C, Z]]^-1 = [[X^-1, 0], [-Z^-1 C X^-1, Z^-1]]:
