@@ -10,7 +10,8 @@
 //       M'_c = gamma_L I - W^T diag(lambda) K                      (d_k x d_k)
 //   dS_c = gamma_L dS_{c+1} + dO^T diag(gamma) Q - dU^T W = dS_{c+1} M'_c^T + dO^T X_c,
 //       X_c = diag(gamma) Q - P W,  dU = diag(lambda) K dS_{c+1}^T + P^T dO
-// (dS_{c+1} is the gradient of the chunk's end state).  Four kernels:
+// (dS_{c+1} is the gradient of the chunk's end state).  Three kernels after
+// the schedule kernel (which fills chunk_base):
 //   1. factors, every (chunk, value head) item at once: T, W, U~, P from the
 //      chunk alone; writes M'_c, U~ diag(lambda), X_c, W, T, T diag(beta)
 //      and T diag(beta gamma) to the item;
@@ -769,10 +770,11 @@ bwd_chain_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tk, co
 }
 
 // ===========================================================================
-// 3. Gradients.  256 threads, one CTA per SM, over all (item, half of d_v)
-//    units.  Products are M = 64 (rows: tokens or the half's d_v rows);
-//    warp w reads rows 16 (w % 4) .. + 15 of an accumulator (lanes 0-15) and
-//    the column half w / 4 of it.
+// 3. Gradients.  256 threads, one CTA per SM, over groups of units: a
+//    (chunk, q/k head) with its value heads' two halves of d_v in turn.
+//    Products are M = 64 (rows: tokens or the half's d_v rows), read with
+//    every lane busy: threads 0-15 and 16-31 of warp w take rows 16 (w % 4)
+//    .. + 15 at columns 32 apart, warp group w / 4 its own 16 (or 64) columns.
 // ===========================================================================
 constexpr uint32_t kDK = 0, kDQ = 16384;        // K, Q [64][128] (TMA)
 constexpr uint32_t kDV = 32768, kDO = 40960;    // V, dO: the half's 64 columns [64][64] (TMA)
