@@ -209,10 +209,13 @@ GDN_API gdn_status_t gdn_chunk_forward_noalloc(const gdn_shape_t *shape,
                                        void *o, float *final_state,
                                        void *stream);
 
-/* Reads the device status word that gdn_chunk_forward left in `workspace`
- * (GDN_OK or GDN_ERR_DEVICE_CHECK) into *device_status.  Synchronises
- * `stream`.  This and gdn_noalloc_read_device_status are the only entry
- * points that wait for the GPU. */
+/* Reads the device status word that gdn_chunk_forward, gdn_kda_forward or
+ * gdn_chunk_backward left in `workspace` into *device_status: GDN_OK, or
+ * GDN_ERR_DEVICE_CHECK when the schedule rejected cu_seqlens or a
+ * tensor-core kernel's bounded wait timed out (the outputs are then not, or
+ * not all, written).  Synchronises `stream`.  This and
+ * gdn_noalloc_read_device_status are the only entry points that wait for
+ * the GPU. */
 GDN_API gdn_status_t gdn_read_device_status(const void *workspace, int32_t *device_status, void *stream);
 
 /* The same for gdn_chunk_forward_noalloc: reads the device status word that
