@@ -207,3 +207,15 @@ def test_backward_tc_full_size(case):
     worst["dS0"] = ((x - y).norm(dim=(2, 3)) / y.norm(dim=(2, 3)).clamp_min(1e-30)).max().item()
     print(case, worst)
     assert max(worst.values()) <= 2 * GRAD_BAR["bf16"], worst
+
+
+@pytest.mark.parametrize("hk,hv", [(2, 2), (1, 3), (2, 6)])
+def test_backward_tc_head_groups(hk, hv):
+    """One, three and three value heads per q/k head: the gradient kernel
+    takes 2 x (Hv / Hk) units per (chunk, q/k head) and sums their dq and dk
+    in registers; the T tiles are loaded once per value head."""
+    inp = bwd_inputs(335 + hv, B=2, T=130, hk=hk, hv=hv, d=128, dtype="bf16")
+    gg, ref = run_both(inp)
+    errs = worst_errors(inp, gg, ref)
+    print(hk, hv, errs)
+    assert max(errs.values()) <= GRAD_BAR["bf16"], errs
