@@ -219,3 +219,20 @@ def test_backward_tc_head_groups(hk, hv):
     errs = worst_errors(inp, gg, ref)
     print(hk, hv, errs)
     assert max(errs.values()) <= GRAD_BAR["bf16"], errs
+
+
+def test_backward_tc_optional_arguments():
+    """The tensor-core form without a final-state gradient (zeros) and with
+    and without the initial-state gradient output."""
+    from linear_attention_sequence_sm_b200 import gdn
+    inp = bwd_inputs(340, B=2, T=150, hk=1, hv=2, d=128, dtype="bf16")
+    gg, ref = run_both(inp, with_dsf=False)
+    errs = worst_errors(inp, gg, ref)
+    print(errs)
+    assert max(errs.values()) <= GRAD_BAR["bf16"], errs
+    d = {k: (v.to(DEV) if v is not None else None) for k, v in inp.items()}
+    nd = gdn.chunk_backward(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dO"], initial_state=d["initial_state"],
+                            want_d_initial_state=False)
+    assert nd["d_initial_state"] is None
+    for name in ("dq", "dk", "dv", "dg", "dbeta"):
+        assert torch.allclose(nd[name], gg[name], rtol=1e-5, atol=1e-6), name
