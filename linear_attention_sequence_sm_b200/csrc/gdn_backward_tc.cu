@@ -154,22 +154,6 @@ __device__ __forceinline__ uint32_t tlane(uint32_t tmem, int warp, int col) {
     return tmem + (uint32_t((warp & 3) * 32) << 16) + uint32_t(col);
 }
 
-// Column sums of an M = 64 accumulator slice: lanes 0-15 each hold a row's 32
-// values (lanes 16-31 pass zeros); adds the 32 column sums into dst[0..31].
-__device__ __forceinline__ void colsum_add(float (&v)[32], bool valid, float *dst, int lane) {
-    float a[16], b[16];
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-        a[u] = valid ? v[u] : 0.f;
-        b[u] = valid ? v[u + 16] : 0.f;
-    }
-    const float sa = warp_colsum16(a, lane), sb = warp_colsum16(b, lane);
-    if ((lane & 1) == 0) {
-        atomicAdd(dst + (lane >> 1), sa);
-        atomicAdd(dst + 16 + (lane >> 1), sb);
-    }
-}
-
 // Shared -> global bulk copy (one thread; completion through the bulk group).
 __device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
